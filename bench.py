@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of libpagedattn on the Llama-2-7B-shaped workload.
+
+Workload: 64 sequences, context lengths uniform in [128, 2048] before the step
+(one token appended, then decode), 32 query heads = 32 kv heads, head_dim 128,
+block_size 16, bf16 cache, pool = 1.1 x blocks needed with ids in a seeded
+shuffle, Q/K/V ~ N(0, 1). One step = the whole hot path for one batch: KV
+append (pa_reshape_and_cache) + decode attention (pa_decode, split into
+partitions with its log-sum-exp merge when the library chooses to).
+
+Metric: KV bytes read by decode per second (GB/s, fraction of HBM peak), and
+decode tokens per second. The 1.07 GB of K/V read per step is far larger than
+the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun as independent replicas (the path has no exchange
+step), one per GPU; value = all ranks' bytes / max over ranks of the time.
+`--impl reference` times the CPU oracle (the only reference this method has)
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode attention tokens/sec"
+WORKLOAD = "llama2_7b_mha_decode: 64 seqs, ctx U[128,2048]+1, 32/32 heads, D128, bs16, bf16"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# --- clocks sampling -------------------------------------------------------------
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        except Exception:
+            bus = None
+        self.sel = bus
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+            if self.sel:
+                cmd += ["-i", self.sel]
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --- workload --------------------------------------------------------------------
+
+def build_workload(seed: int, device):
+    """The pool filled with N(0,1) values on the device (it stands in for the
+    prompts' K/V), every sequence's blocks reserved through the C++ block
+    manager, then one append per sequence: the step's slots, tables, lengths."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    from paged_kv_cache_361_b200 import workloads as W
+    w = W.llama2_7b_mha(seed=seed)
+    sh = w.shape
+    dt = W.TORCH_DTYPE[sh.dtype]
+    cache = PagedKVCache(w.num_blocks, sh.num_kv_heads, sh.block_size, sh.head_dim, dt, device, w.free_order)
+    g = torch.Generator(device=device)
+    g.manual_seed(1000 + seed)
+    for t in (cache.k_cache, cache.v_cache):
+        for i in range(0, w.num_blocks, 1024):   # chunked to bound the fp32 temporary
+            t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(dt)
+    ids = list(range(w.num_seqs))
+    for s in ids:
+        cache.reserve(s, int(w.context_lens_old[s]))
+    slots, pairs = cache.bm.append_slots(ids)
+    assert len(pairs) == 0
+    for s in ids:
+        cache.lens[s] += 1
+    tables, lens32, max_len = cache.decode_inputs(ids)
+    lens = w.context_lens
+    assert lens32.tolist() == lens.tolist()
+    B_, hq, hkv, D = w.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.head_dim
+    return dict(
+        w=w, cache=cache, bm=cache.bm, kc=cache.k_cache, vc=cache.v_cache,
+        q=torch.randn((B_, hq, D), generator=g, device=device).to(dt),
+        k=torch.randn((B_, hkv, D), generator=g, device=device).to(dt),
+        v=torch.randn((B_, hkv, D), generator=g, device=device).to(dt),
+        slots=torch.from_numpy(slots).to(device),
+        tables=torch.from_numpy(tables).to(device),
+        lens=torch.from_numpy(lens32).to(device),
+        out=torch.empty((B_, hq, D), dtype=torch.float32, device=device),
+        max_len=max_len,
+        kv_bytes=int(lens.sum()) * hkv * D * 2 * 2,
+    )
+
+
+def sample_rows(d, seqs):
+    """Host copies (before any kernel runs) of the sampled sequences' K/V rows,
+    read from the device pool through their block tables: input to the CPU
+    baseline only."""
+    w, bm = d["w"], d["bm"]
+    bs = w.shape.block_size
+    rows = []
+    for s in seqs:
+        table, L = bm.block_table(s)
+        L_old = L - 1
+        t = torch.arange(L_old)
+        blk = torch.as_tensor(table, dtype=torch.int64)[t // bs].to(d["kc"].device)
+        off = (t % bs).to(d["kc"].device)
+        K = torch.cat([d["kc"][blk, :, off, :], d["k"][s:s + 1]]).cpu()
+        V = torch.cat([d["vc"][blk, :, off, :], d["v"][s:s + 1]]).cpu()
+        rows.append((s, K, V, d["q"][s].cpu()))
+    return rows
+
+
+def time_oracle(rows, scale, budget_s):
+    """Runs the CPU oracle over the sampled sequences (repeating the sample)
+    until budget_s has passed; returns (GB/s, seconds, sequences done)."""
+    from oracle.attention import decode_attention
+    done_bytes, n, t0 = 0, 0, time.perf_counter()
+    while True:
+        for s, K, V, q in rows:
+            decode_attention(q, K, V, scale)
+            done_bytes += K.numel() * 2 * 2
+            n += 1
+            if time.perf_counter() - t0 >= budget_s:
+                el = time.perf_counter() - t0
+                return done_bytes / el / 1e9, el, n
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return int(max(blas))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# --- arms --------------------------------------------------------------------------
+
+def run_ours(args, rank, world, device):
+    from paged_kv_cache_361_b200 import binding as B
+    d = build_workload(seed=rank, device=device)
+    w = d["w"]
+    sh = w.shape
+    P = args.partition
+    ws_bytes = B.pa_decode_workspace_bytes(w.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, d["max_len"],
+                                           sh.block_size, P)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device) if ws_bytes else None
+    P_eff = P if P >= 0 else B.pa_decode_partition_tokens(w.num_seqs, sh.num_q_heads, sh.num_kv_heads,
+                                                          d["max_len"], sh.block_size)
+    split = P_eff > 0 and math.ceil(d["max_len"] / P_eff) > 1
+    stream = torch.cuda.current_stream(device)
+
+    baseline_rows = sample_rows(d, list(range(4))) if rank == 0 and world == 1 and not args.no_cpu_baseline else None
+
+    def step():
+        B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
+        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], w.scale, d["out"], d["max_len"], P, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    st, info = B.pa_get_device_error()
+    if st != B.PA_OK:
+        raise RuntimeError(f"device error {st} ({info}) during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
+        ev[i][0].record(stream)
+        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], w.scale, d["out"], d["max_len"], P, ws)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    st, info = B.pa_get_device_error()
+    if st != B.PA_OK:
+        raise RuntimeError(f"device error {st} ({info}) in the timed region")
+
+    kv_bytes = d["kv_bytes"]
+    # max over ranks of the time, sum of the bytes
+    t = torch.tensor([total_ms, float(kv_bytes)], dtype=torch.float64, device=device)
+    if world > 1:
+        tm = t[:1].clone()
+        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
+        tb = t[1:].clone()
+        torch.distributed.all_reduce(tb, op=torch.distributed.ReduceOp.SUM)
+        total_ms, all_bytes = float(tm.item()), float(tb.item())
+    else:
+        all_bytes = float(kv_bytes)
+    ms_per_step = total_ms / args.steps
+    value = all_bytes / (ms_per_step * 1e-3) / 1e9
+    tokens_per_s = world * w.num_seqs / (ms_per_step * 1e-3)
+
+    # end to end through the public API: inputs from pinned host memory, output back to host
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, d, device, rank, world)
+
+    cpu = None
+    if baseline_rows is not None:
+        gbs, el, n = time_oracle(baseline_rows, w.scale, args.cpu_seconds)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"fp64 NumPy oracle over sequences 0-3 of the workload (all 32 heads), repeated for "
+                         f"{el:.1f} s ({n} sequence passes); host has {os.cpu_count()} cores"}
+
+    peak, peak_kind = peaks()
+    dec_avg_ms = statistics.mean(decode_ms)
+    achieved = kv_bytes / (dec_avg_ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "num_seqs": w.num_seqs, "num_q_heads": sh.num_q_heads,
+                       "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "block_size": sh.block_size,
+                       "num_blocks": w.num_blocks, "context_tokens": int(w.context_lens.sum()),
+                       "kv_bytes_per_step": kv_bytes, "partition_tokens": P_eff,
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                       "l2": "no flush: 1.07 GB of K/V per step >> 126 MB L2"},
+            "tokens_per_s": round(tokens_per_s, 1),
+            "pct_of_hbm_peak": {"of_measured_6540": round(value / peak, 4), "of_nominal_8000": round(value / 8000.0, 4)},
+            "e2e": e2e,
+            "gpu_launches": args.steps * (3 if split else 2),
+            "roofline": {"kernel": "pa_decode (decode + partition merge)", "bound": "hbm",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                         else "fallback", "decode_ms_avg": round(dec_avg_ms, 5)},
+            "cpu_baseline": cpu,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, d, device, rank, world):
+    """K steps through PagedKVCache.step: per step, H2D of q/k/v from pinned host
+    memory (plus the slots, tables and lengths the API uploads), append + decode,
+    D2H of the fp32 output. Context lengths grow by one per step."""
+    w = d["w"]
+    sh = w.shape
+    cache = d["cache"]
+    ids = list(range(w.num_seqs))
+    hq = torch.empty(d["q"].shape, dtype=d["q"].dtype, pin_memory=True)
+    hk = torch.empty(d["k"].shape, dtype=d["k"].dtype, pin_memory=True)
+    hv = torch.empty(d["v"].shape, dtype=d["v"].dtype, pin_memory=True)
+    hq.copy_(d["q"].cpu()); hk.copy_(d["k"].cpu()); hv.copy_(d["v"].cpu())
+    hout = torch.empty(d["out"].shape, dtype=torch.float32, pin_memory=True)
+    kv_total = 0
+    h2d = d2h = 0
+    for it in range(args.warmup + args.steps):
+        if it == args.warmup:
+            torch.cuda.synchronize(device)
+            if world > 1:
+                torch.distributed.barrier()
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record()
+            kv_total = 0
+            h2d = d2h = 0
+        q = hq.to(device, non_blocking=True)
+        k = hk.to(device, non_blocking=True)
+        v = hv.to(device, non_blocking=True)
+        out = cache.step(ids, q, k, v, w.scale, partition_tokens=args.partition)
+        hout.copy_(out, non_blocking=True)
+        torch.cuda.current_stream(device).synchronize()
+        L = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64)
+        kv_total += int(L.sum()) * sh.num_kv_heads * sh.head_dim * 2 * 2
+        nblk = int(-(-L.max() // sh.block_size))
+        h2d += 3 * q.numel() * 2 + len(ids) * 8 + len(ids) * nblk * 4 + len(ids) * 4
+        d2h += hout.numel() * 4
+    t1.record()
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1)
+    t = torch.tensor([ms, float(kv_total)], dtype=torch.float64, device=device)
+    if world > 1:
+        tm = t[:1].clone()
+        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
+        tb = t[1:].clone()
+        torch.distributed.all_reduce(tb, op=torch.distributed.ReduceOp.SUM)
+        ms, kv_total = float(tm.item()), float(tb.item())
+    return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_step": round(ms / args.steps, 4),
+            "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
+            "api": "PagedKVCache.step (pa_bm_append_slots, pa_copy_blocks, pa_reshape_and_cache, "
+                   "pa_bm_block_tables, pa_decode)"}
+
+
+def run_reference(args, rank, world):
+    """CPU oracle on this workload's shapes; each step is a bounded sample."""
+    if rank != 0:
+        return
+    from paged_kv_cache_361_b200 import workloads as W
+    w = W.llama2_7b_mha(seed=0)
+    seqs = [0, 1]
+    rows = [(s, w.history(s, "k"), w.history(s, "v"), w.query()[s]) for s in seqs]
+    from oracle.attention import decode_attention
+    bytes_per = sum(K.numel() * 2 * 2 for _, K, _, _ in rows)
+
+    def step():
+        for s, K, V, q in rows:
+            decode_attention(q, K, V, w.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    ms = el * 1e3 / args.steps
+    gbs = bytes_per / (ms * 1e-3) / 1e9
+    sample = (f"fp64 NumPy oracle, sequences {seqs} of the workload (all 32 heads, "
+              f"{bytes_per / 1e6:.1f} MB of bf16 K/V per step); host has {os.cpu_count()} cores")
+    line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample_seqs": seqs},
+            "tokens_per_s": round(len(seqs) / (ms * 1e-3), 3),
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--partition", type=int, default=-1, help="partition_tokens for pa_decode (-1: library choice)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    from paged_kv_cache_361_b200 import build as _build
+    _build.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,244 @@
+/*
+ * libpagedattn: paged KV cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * The KV cache is split into fixed-size physical blocks; each sequence reaches
+ * its blocks through a block table. This library provides the three device
+ * operations of a decode step and the host-side block manager that feeds them.
+ *
+ * Page tags used in citations:
+ *   P1 = "Paged Attention：大模型推理显存优化的核心方案" (learnblockchain.cn)
+ *   P2 = "PagedAttention：操作系统级 KV 缓存虚拟内存管理" (freeguideonline.com)
+ *   P3 = "PagedAttention 和 vLLM" (aiunderstanding.org)
+ *
+ * Conventions for every entry point:
+ *   - Every call returns a pa_status; nothing is thrown across the ABI.
+ *   - Device operations are asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream). Arguments are checked on the
+ *     host before launch (PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED, nothing is
+ *     launched). A failed launch returns PA_ERR_CUDA. Problems that only the
+ *     device can see (a block id or slot outside the pool, a context length
+ *     above its stated bound) make the kernel skip the access and record the
+ *     first such event in a per-device error word that pa_get_device_error
+ *     reads; the kernels never trap.
+ *   - All device pointers are owned by the caller, must be 16-byte aligned and
+ *     must stay valid until the stream has executed the call. The library
+ *     allocates no device memory.
+ *   - KV cache layout: K and V are each [num_blocks][num_kv_heads][block_size]
+ *     [head_dim], row-major, in the cache dtype. Token t of a sequence is at
+ *     block block_table[t / block_size], offset t % block_size (P2 §2.3, §五).
+ *     A "slot" is block * block_size + offset.
+ *   - Query head h reads kv head h / (num_q_heads / num_kv_heads).
+ *   - Supported shapes: head_dim 64 or 128; block_size 1, 2, 4, 8, 16 or 32;
+ *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; dtype fp32 or bf16.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,     /* null / misaligned pointer, negative size, bad layout */
+  PA_ERR_UNSUPPORTED = 2,     /* shape or dtype outside the supported set */
+  PA_ERR_NO_FREE_BLOCKS = 3,  /* block manager: the pool cannot satisfy the call */
+  PA_ERR_UNKNOWN_SEQ = 4,     /* block manager: no such sequence id */
+  PA_ERR_SEQ_EXISTS = 5,      /* block manager: the sequence id is already live */
+  PA_ERR_CUDA = 6,            /* a CUDA runtime call or a launch failed */
+  PA_ERR_DEVICE_BOUNDS = 7,   /* a kernel met an index outside its bounds and skipped it */
+  PA_ERR_DEVICE_TIMEOUT = 8   /* a kernel gave up a bounded wait on its own copies */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+typedef void* pa_stream; /* cudaStream_t */
+
+/* A paged KV cache in device memory (see the layout above). */
+typedef struct {
+  void* k;               /* device, [num_blocks][num_kv_heads][block_size][head_dim] */
+  void* v;               /* device, same shape as k */
+  int64_t num_blocks;    /* physical blocks in the pool, >= 1, < 2^31 */
+  int32_t num_kv_heads;  /* >= 1 */
+  int32_t block_size;    /* tokens per block */
+  int32_t head_dim;      /* elements per head row */
+  int32_t dtype;         /* pa_dtype of k, v, and of the q/k/v inputs */
+} pa_cache;
+
+/* Human-readable name of a status code (static storage). */
+const char* pa_status_string(pa_status status);
+
+/* Library ABI version, currently 1. */
+int32_t pa_version(void);
+
+/* ------------------------------------------------------------------------- */
+/* Device operations                                                          */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * KV append: write each new token's K and V rows into its slot.
+ * P2 §3.2.2 step 3 (write the new K, V at the block position) and §3.2.1
+ * (a prompt's K, V written into its blocks).
+ *
+ *   k, v          device, [num_tokens][num_kv_heads][head_dim], cache dtype,
+ *                 contiguous.
+ *   slot_mapping  device int64 [num_tokens]; slot of token i, or -1 to skip it.
+ *                 A slot outside [-1, num_blocks * block_size) is skipped and
+ *                 recorded as PA_ERR_DEVICE_BOUNDS.
+ *   num_tokens    >= 0; 0 launches nothing.
+ * Two tokens must not name the same slot in one call (the result would be
+ * either row). A bit copy: no rounding.
+ */
+pa_status pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                               const pa_cache* cache, pa_stream stream);
+
+/*
+ * Copy whole physical blocks, K and V: cache[dst] = cache[src] for each pair.
+ * P2 §3.4: before a write into a block shared by several sequences, the block
+ * is copied and the writer's table is pointed at the copy (copy-on-write).
+ *
+ *   src_dst_pairs  device int32 [n_pairs][2] = {src, dst}.
+ *   n_pairs        >= 0; 0 launches nothing.
+ * All dst must differ, and no dst may be the src of another pair in the same
+ * call (the pairs that pa_bm_append_slot(s) emits satisfy this). An id outside
+ * [0, num_blocks) skips that pair and is recorded as PA_ERR_DEVICE_BOUNDS.
+ * Apply the pairs of a decode step before the pa_reshape_and_cache that writes
+ * the step's tokens, on the same stream.
+ */
+pa_status pa_copy_blocks(const pa_cache* cache, const int32_t* src_dst_pairs, int32_t n_pairs, pa_stream stream);
+
+/*
+ * Single-query decode attention over the paged cache.
+ * P2 §1.1: out = softmax(scale * q K^T) V, one query row per head; P2 §3.2.2
+ * step 4 and §4.1: every logical block of the sequence is visited through its
+ * block table, with the softmax accumulated block by block (online softmax).
+ *
+ *   q                  device, [num_seqs][num_q_heads][head_dim], cache dtype.
+ *   block_tables       device int32 [num_seqs][max_blocks_per_seq]; entries
+ *                      past ceil(context_len / block_size) are never read.
+ *   context_lens       device int32 [num_seqs]; tokens to attend over,
+ *                      including the token appended this step. Must not
+ *                      exceed max_context_len (larger values are clamped and
+ *                      recorded as PA_ERR_DEVICE_BOUNDS). 0 gives a zero row.
+ *   max_context_len    host bound on context_lens, <= max_blocks_per_seq *
+ *                      block_size; it sizes the launch.
+ *   scale              score scale, usually 1/sqrt(head_dim).
+ *   out                device fp32 [num_seqs][num_q_heads][head_dim].
+ *   partition_tokens   0: one CTA walks the whole sequence.
+ *                      > 0 (a multiple of block_size): split each sequence
+ *                      into partitions of that many tokens, each computed
+ *                      separately; a second kernel merges them with a
+ *                      log-sum-exp reduction.
+ *                      -1: chosen by the library (pa_decode_partition_tokens).
+ *   workspace          device, >= pa_decode_workspace_bytes(...) bytes when
+ *                      the sequences are split, else may be NULL. Scratch for
+ *                      the partial results; its contents need no initial value.
+ * Accumulation is fp32. Calls sharing a workspace must not overlap on the GPU.
+ */
+pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, float scale, float* out, int32_t partition_tokens, void* workspace,
+                    size_t workspace_bytes, pa_stream stream);
+
+/* The partition size pa_decode uses for partition_tokens = -1 with these
+ * sizes (0 = no split). */
+int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t max_context_len, int32_t block_size);
+
+/* Workspace bytes pa_decode needs for these sizes (0 when nothing is split).
+ * partition_tokens may be -1 (resolved as pa_decode would). */
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t max_context_len, int32_t block_size, int32_t partition_tokens);
+
+/*
+ * Waits for `stream`, then reads and clears this device's error word.
+ * Returns PA_OK, PA_ERR_DEVICE_BOUNDS or PA_ERR_DEVICE_TIMEOUT (the first event
+ * recorded since the last read), or PA_ERR_CUDA. `info_out` (may be NULL)
+ * receives the offending value (block id, slot or length) when there is one.
+ */
+pa_status pa_get_device_error(pa_stream stream, int64_t* info_out);
+
+/*
+ * Self-test of the device wait limit. Every pipelined kernel waits for its own
+ * copies with a bounded wait; this launches one thread that waits on a barrier
+ * nothing completes. After timeout_ns (1 .. 10^10) it records
+ * PA_ERR_DEVICE_TIMEOUT in the error word and exits, leaving the context
+ * usable. Read the result with pa_get_device_error.
+ */
+pa_status pa_selftest_wait_timeout(int64_t timeout_ns, pa_stream stream);
+
+/* ------------------------------------------------------------------------- */
+/* Host block manager                                                         */
+/* ------------------------------------------------------------------------- */
+/*
+ * The pool's free list, reference counts and per-sequence block tables
+ * (P1 "Paged Attention 的工作原理", "块表（Block Table）"; P2 §2.3, §3.2, §3.3,
+ * §3.4). Not thread-safe: one thread per handle. Every call either succeeds or
+ * leaves the state unchanged.
+ * Free-list order: allocation takes the front; a block whose count drops to
+ * zero is appended at the back, in the order of the freed sequence's table.
+ * Sequences are identified by caller-chosen int64 ids.
+ */
+typedef struct pa_bm pa_bm;
+
+/* free_order: host int32 [num_blocks], a permutation of 0..num_blocks-1 giving
+ * the initial free-list order, or NULL for 0, 1, 2, ... */
+pa_status pa_bm_create(int64_t num_blocks, int32_t block_size, const int32_t* free_order, pa_bm** out);
+void pa_bm_destroy(pa_bm* bm);
+
+/* Prefill (P2 §3.2.1): new sequence of num_tokens >= 0 tokens, given
+ * ceil(num_tokens / block_size) blocks. slots_out (host int64 [num_tokens],
+ * may be NULL) receives the slot of each token. */
+pa_status pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int32_t num_tokens, int64_t* slots_out);
+
+/* Share (P1 "跨请求的内存共享"; P2 §3.4): `child` gets a copy of `parent`'s
+ * table and every block in it gains one reference. */
+pa_status pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child);
+
+/* One decode-step position (P2 §3.2.2 steps 2-3, §3.4). If the last block is
+ * full, a new block is appended to the table. If the target block is shared
+ * (count > 1) it is replaced by a fresh block and *cow_pair_out = {old, new},
+ * which must be applied with pa_copy_blocks before the token is written;
+ * otherwise *cow_pair_out = {-1, -1}. cow_pair_out may be NULL only when the
+ * caller knows no block is shared. */
+pa_status pa_bm_append_slot(pa_bm* bm, int64_t seq_id, int64_t* slot_out, int32_t* cow_pair_out);
+
+/* pa_bm_append_slot for n sequences in the given order, all or nothing.
+ * slots_out: host int64 [n]; cow_pairs_out: host int32 [n][2], of which the
+ * first *n_pairs_out are filled in order. */
+pa_status pa_bm_append_slots(pa_bm* bm, int32_t n, const int64_t* seq_ids, int64_t* slots_out,
+                             int32_t* cow_pairs_out, int32_t* n_pairs_out);
+
+/* Release a finished sequence (P2 §3.3). */
+pa_status pa_bm_free_seq(pa_bm* bm, int64_t seq_id);
+
+/* The table of one sequence: up to `cap` entries into out (host int32), the
+ * full table length into *n_out and the token count into *len_out (either may
+ * be NULL). */
+pa_status pa_bm_block_table(const pa_bm* bm, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out,
+                            int64_t* len_out);
+
+/* Decode inputs for n sequences: out (host int32 [n][cap]) gets each table,
+ * padded with `pad`; lens_out (host int32 [n]) the token counts. Fails with
+ * PA_ERR_INVALID_ARG if a table is longer than cap. */
+pa_status pa_bm_block_tables(const pa_bm* bm, int32_t n, const int64_t* seq_ids, int32_t* out, int32_t cap,
+                             int32_t pad, int32_t* lens_out);
+
+pa_status pa_bm_refcount(const pa_bm* bm, int32_t block, int32_t* out);
+
+/* free_blocks: blocks on the free list; allocated_slots: block_size times the
+ * blocks in use; used_slots: slots holding a token (a shared block counts
+ * once). allocated - used is the internal waste (P1 "内存浪费的两种形式"). */
+pa_status pa_bm_stats(const pa_bm* bm, int64_t* free_blocks, int64_t* used_slots, int64_t* allocated_slots);
+
+/* The free list in order: up to cap ids into out, the length into *n_out. */
+pa_status pa_bm_free_list(const pa_bm* bm, int32_t* out, int64_t cap, int64_t* n_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

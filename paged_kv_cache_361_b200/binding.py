@@ -1,0 +1,280 @@
+"""ctypes binding of libpagedattn (include/pagedattn.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity and passed as raw pointers with the current CUDA stream; every step
+of the computation runs in the library's kernels. There is no fallback: if the
+shared library is missing, importing a device entry point raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_NO_FREE_BLOCKS, PA_ERR_UNKNOWN_SEQ, PA_ERR_SEQ_EXISTS, \
+    PA_ERR_CUDA, PA_ERR_DEVICE_BOUNDS, PA_ERR_DEVICE_TIMEOUT = range(9)
+PA_F32, PA_BF16 = 0, 1
+_DTYPE = {torch.float32: PA_F32, torch.bfloat16: PA_BF16}
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib().pa_status_string(status).decode()} (status {status})")
+
+
+class pa_cache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("num_blocks", ctypes.c_int64),
+                ("num_kv_heads", ctypes.c_int32), ("block_size", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
+
+
+_L = None
+_VP, _I32, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_P32, _P64 = ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)
+_PCACHE = ctypes.POINTER(pa_cache)
+
+_SIGS = {
+    "pa_status_string": (ctypes.c_char_p, [_I32]),
+    "pa_version": (_I32, []),
+    "pa_reshape_and_cache": (_I32, [_VP, _VP, _VP, _I32, _PCACHE, _VP]),
+    "pa_copy_blocks": (_I32, [_PCACHE, _VP, _I32, _VP]),
+    "pa_decode": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP, _SZ, _VP]),
+    "pa_decode_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
+    "pa_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "pa_get_device_error": (_I32, [_VP, _P64]),
+    "pa_selftest_wait_timeout": (_I32, [_I64, _VP]),
+    "pa_bm_create": (_I32, [_I64, _I32, _VP, ctypes.POINTER(_VP)]),
+    "pa_bm_destroy": (None, [_VP]),
+    "pa_bm_add_seq": (_I32, [_VP, _I64, _I32, _VP]),
+    "pa_bm_fork": (_I32, [_VP, _I64, _I64]),
+    "pa_bm_append_slot": (_I32, [_VP, _I64, _P64, _P32]),
+    "pa_bm_append_slots": (_I32, [_VP, _I32, _VP, _VP, _VP, _P32]),
+    "pa_bm_free_seq": (_I32, [_VP, _I64]),
+    "pa_bm_block_table": (_I32, [_VP, _I64, _VP, _I32, _P32, _P64]),
+    "pa_bm_block_tables": (_I32, [_VP, _I32, _VP, _VP, _I32, _I32, _VP]),
+    "pa_bm_refcount": (_I32, [_VP, _I32, _P32]),
+    "pa_bm_stats": (_I32, [_VP, _P64, _P64, _P64]),
+    "pa_bm_free_list": (_I32, [_VP, _VP, _I64, _P64]),
+}
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libpagedattn.so is not built ({LIB_PATH}); run python -m paged_kv_cache_361_b200.build")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _L = lib
+    return _L
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGS)
+
+
+def _check(status: int, what: str):
+    if status != PA_OK:
+        raise PagedAttnError(status, what)
+
+
+def _stream(t: torch.Tensor, stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(t.device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> pa_cache:
+    """pa_cache view of two [num_blocks][num_kv_heads][block_size][head_dim] tensors."""
+    if k_cache.shape != v_cache.shape or k_cache.dtype != v_cache.dtype:
+        raise ValueError("k_cache and v_cache must match")
+    if k_cache.dtype not in _DTYPE:
+        raise TypeError(f"unsupported cache dtype {k_cache.dtype}")
+    nb, hkv, bs, d = k_cache.shape
+    return pa_cache(_dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4), nb, hkv, bs, d,
+                    _DTYPE[k_cache.dtype])
+
+
+# --- device operations ---------------------------------------------------------
+
+def pa_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, stream=None):
+    c = make_cache(k_cache, v_cache)
+    n = int(k.shape[0])
+    _dev(k, "k", k_cache.dtype, 3), _dev(v, "v", k_cache.dtype, 3)
+    if tuple(k.shape) != (n, c.num_kv_heads, c.head_dim) or k.shape != v.shape:
+        raise ValueError("k, v must be [num_tokens][num_kv_heads][head_dim]")
+    if slot_mapping.shape != (n,):
+        raise ValueError("slot_mapping must be [num_tokens]")
+    _check(_lib().pa_reshape_and_cache(k.data_ptr(), v.data_ptr(), _dev(slot_mapping, "slot_mapping", torch.int64),
+                                       n, ctypes.byref(c), _stream(k_cache, stream)), "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None):
+    c = make_cache(k_cache, v_cache)
+    n = int(src_dst_pairs.shape[0])
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [n][2]")
+    _check(_lib().pa_copy_blocks(ctypes.byref(c), _dev(src_dst_pairs, "src_dst_pairs", torch.int32), n,
+                                 _stream(k_cache, stream)), "pa_copy_blocks")
+
+
+def pa_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, max_context_len, block_size) -> int:
+    return int(_lib().pa_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, max_context_len, block_size))
+
+
+def pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size,
+                              partition_tokens=-1) -> int:
+    return int(_lib().pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                                block_size, partition_tokens))
+
+
+def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_context_len,
+              partition_tokens=-1, workspace=None, stream=None):
+    c = make_cache(k_cache, v_cache)
+    B, hq, d = q.shape
+    _dev(q, "q", k_cache.dtype, 3)
+    _dev(out, "out", torch.float32, 3)
+    if d != c.head_dim or tuple(out.shape) != (B, hq, d):
+        raise ValueError("q/out shape mismatch")
+    _dev(block_tables, "block_tables", torch.int32, 2)
+    _dev(context_lens, "context_lens", torch.int32, 1)
+    if block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("block_tables / context_lens must have num_seqs rows")
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_dev(workspace, "workspace"),
+                                                            workspace.numel() * workspace.element_size())
+    _check(_lib().pa_decode(q.data_ptr(), B, hq, ctypes.byref(c), block_tables.data_ptr(),
+                            int(block_tables.shape[1]), context_lens.data_ptr(), int(max_context_len), float(scale),
+                            out.data_ptr(), int(partition_tokens), ws_ptr, ws_bytes, _stream(q, stream)), "pa_decode")
+
+
+def pa_get_device_error(stream=None):
+    """(status, info) of the current device's error word; waits for the stream."""
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    info = ctypes.c_int64(0)
+    st = _lib().pa_get_device_error(handle, ctypes.byref(info))
+    return int(st), int(info.value)
+
+
+def pa_selftest_wait_timeout(timeout_ns: int, stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    _check(_lib().pa_selftest_wait_timeout(int(timeout_ns), stream.cuda_stream), "pa_selftest_wait_timeout")
+
+
+# --- host block manager --------------------------------------------------------
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class BlockManager:
+    """The C++ block manager behind pa_bm_* (one handle)."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        h = ctypes.c_void_p()
+        order = None
+        if free_order is not None:
+            self._order = np.ascontiguousarray(free_order, dtype=np.int32)
+            if self._order.shape != (num_blocks,):
+                raise ValueError("free_order must have num_blocks entries")
+            order = _i64p(self._order)
+        _check(_lib().pa_bm_create(num_blocks, block_size, order, ctypes.byref(h)), "pa_bm_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib().pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, seq_id: int, num_tokens: int) -> np.ndarray:
+        slots = np.empty(max(num_tokens, 0), dtype=np.int64)
+        _check(_lib().pa_bm_add_seq(self._h, seq_id, num_tokens, _i64p(slots)), "pa_bm_add_seq")
+        return slots
+
+    def fork(self, parent: int, child: int):
+        _check(_lib().pa_bm_fork(self._h, parent, child), "pa_bm_fork")
+
+    def append_slot(self, seq_id: int):
+        slot = ctypes.c_int64()
+        pair = (ctypes.c_int32 * 2)()
+        _check(_lib().pa_bm_append_slot(self._h, seq_id, ctypes.byref(slot), pair), "pa_bm_append_slot")
+        return int(slot.value), (None if pair[0] < 0 else (int(pair[0]), int(pair[1])))
+
+    def append_slots(self, seq_ids):
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        slots = np.empty(len(ids), dtype=np.int64)
+        pairs = np.empty((len(ids), 2), dtype=np.int32)
+        n = ctypes.c_int32(0)
+        _check(_lib().pa_bm_append_slots(self._h, len(ids), _i64p(ids), _i64p(slots), _i64p(pairs), ctypes.byref(n)),
+               "pa_bm_append_slots")
+        return slots, pairs[:n.value].copy()
+
+    def free_seq(self, seq_id: int):
+        _check(_lib().pa_bm_free_seq(self._h, seq_id), "pa_bm_free_seq")
+
+    def block_table(self, seq_id: int):
+        n = ctypes.c_int32()
+        L = ctypes.c_int64()
+        _check(_lib().pa_bm_block_table(self._h, seq_id, None, 0, ctypes.byref(n), ctypes.byref(L)), "pa_bm_block_table")
+        out = np.empty(n.value, dtype=np.int32)
+        _check(_lib().pa_bm_block_table(self._h, seq_id, _i64p(out), n.value, ctypes.byref(n), ctypes.byref(L)),
+               "pa_bm_block_table")
+        return out, int(L.value)
+
+    def block_tables(self, seq_ids, cap: int, pad: int = -1, out=None, lens_out=None):
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        if out is None:
+            out = np.empty((len(ids), cap), dtype=np.int32)
+        if lens_out is None:
+            lens_out = np.empty(len(ids), dtype=np.int32)
+        _check(_lib().pa_bm_block_tables(self._h, len(ids), _i64p(ids), _i64p(out), cap, pad, _i64p(lens_out)),
+               "pa_bm_block_tables")
+        return out, lens_out
+
+    def refcount(self, block: int) -> int:
+        r = ctypes.c_int32()
+        _check(_lib().pa_bm_refcount(self._h, block, ctypes.byref(r)), "pa_bm_refcount")
+        return int(r.value)
+
+    def stats(self) -> dict:
+        f, u, a = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(_lib().pa_bm_stats(self._h, ctypes.byref(f), ctypes.byref(u), ctypes.byref(a)), "pa_bm_stats")
+        return dict(free_blocks=f.value, used_slots=u.value, allocated_slots=a.value,
+                    internal_waste=a.value - u.value)
+
+    def free_list(self) -> np.ndarray:
+        n = ctypes.c_int64()
+        _check(_lib().pa_bm_free_list(self._h, None, 0, ctypes.byref(n)), "pa_bm_free_list")
+        out = np.empty(n.value, dtype=np.int32)
+        _check(_lib().pa_bm_free_list(self._h, _i64p(out), n.value, ctypes.byref(n)), "pa_bm_free_list")
+        return out

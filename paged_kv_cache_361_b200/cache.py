@@ -1,0 +1,128 @@
+"""PagedKVCache: a paged KV cache on one GPU, driven by the C++ block manager.
+
+This is the public API a serving loop calls. It owns the two cache tensors
+[num_blocks][num_kv_heads][block_size][head_dim], a pa_bm handle, and small
+pinned staging buffers for the per-step host -> device copies of slots, tables
+and lengths. All arithmetic runs in libpagedattn's kernels.
+
+P1 = "Paged Attention：大模型推理显存优化的核心方案", P2 = "PagedAttention：操作系统级 KV
+缓存虚拟内存管理".
+  add_sequence  prefill write (P2 §3.2.1)
+  fork          prefix sharing (P1 "跨请求的内存共享", P2 §3.4)
+  append        decode-step write with copy-on-write (P2 §3.2.2 steps 1-3, §3.4)
+  decode        attention over the block tables (P2 §3.2.2 step 4, §4.1)
+  free          return blocks to the pool (P2 §3.3)
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+class _Staging:
+    """Host -> device upload through pinned memory. Pinned blocks come from
+    torch's caching host allocator, which does not hand a block out again until
+    the copies that read it have finished, so uploads never wait for the GPU."""
+
+    def __init__(self, dtype_np, dtype_t, device):
+        self.np_dtype, self.t_dtype, self.device = dtype_np, dtype_t, device
+
+    def upload(self, arr: np.ndarray) -> torch.Tensor:
+        h = torch.empty(arr.shape, dtype=self.t_dtype, pin_memory=True)
+        h.numpy()[...] = arr
+        return h.to(self.device, non_blocking=True)
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
+                 dtype=torch.bfloat16, device="cuda", free_order=None, fill: float | None = None):
+        self.device = torch.device(device)
+        shape = (num_blocks, num_kv_heads, block_size, head_dim)
+        self.k_cache = torch.empty(shape, dtype=dtype, device=self.device)
+        self.v_cache = torch.empty(shape, dtype=dtype, device=self.device)
+        if fill is not None:
+            self.k_cache.fill_(fill)
+            self.v_cache.fill_(fill)
+        self.block_size = block_size
+        self.bm = B.BlockManager(num_blocks, block_size, free_order)
+        self.lens: dict[int, int] = {}
+        self._slots = _Staging(np.int64, torch.int64, self.device)
+        self._pairs = _Staging(np.int32, torch.int32, self.device)
+        self._tables = _Staging(np.int32, torch.int32, self.device)
+        self._lens = _Staging(np.int32, torch.int32, self.device)
+        self._ws = None
+
+    # -- host bookkeeping + writes -------------------------------------------
+    def add_sequence(self, seq_id: int, k: torch.Tensor, v: torch.Tensor) -> np.ndarray:
+        n = int(k.shape[0])
+        slots = self.bm.add_seq(seq_id, n)
+        self.lens[seq_id] = n
+        if n:
+            B.pa_reshape_and_cache(k, v, self._slots.upload(slots), self.k_cache, self.v_cache)
+        return slots
+
+    def reserve(self, seq_id: int, num_tokens: int) -> np.ndarray:
+        """Allocate blocks for a sequence whose K/V rows the caller writes itself
+        (or that are already in the pool); returns the rows' slots."""
+        slots = self.bm.add_seq(seq_id, num_tokens)
+        self.lens[seq_id] = num_tokens
+        return slots
+
+    def fork(self, parent: int, child: int):
+        self.bm.fork(parent, child)
+        self.lens[child] = self.lens[parent]
+
+    def append(self, seq_ids, k: torch.Tensor, v: torch.Tensor):
+        """One new token per listed sequence (rows of k, v in the same order).
+        Returns (slots, cow_pairs) as numpy arrays."""
+        slots, pairs = self.bm.append_slots(seq_ids)
+        for s in seq_ids:
+            self.lens[s] += 1
+        if len(pairs):
+            B.pa_copy_blocks(self.k_cache, self.v_cache, self._pairs.upload(pairs))
+        B.pa_reshape_and_cache(k, v, self._slots.upload(slots), self.k_cache, self.v_cache)
+        return slots, pairs
+
+    def free(self, seq_id: int):
+        self.bm.free_seq(seq_id)
+        del self.lens[seq_id]
+
+    # -- attention -------------------------------------------------------------
+    def decode_inputs(self, seq_ids):
+        """Host block tables [n][cap] (padded with -1) and lengths [n]."""
+        max_len = max((self.lens[s] for s in seq_ids), default=0)
+        cap = max(1, -(-max_len // self.block_size))
+        tables, lens = self.bm.block_tables(seq_ids, cap)
+        return tables, lens, max_len
+
+    def workspace(self, nbytes: int):
+        if nbytes == 0:
+            return None
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def decode(self, seq_ids, q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
+               partition_tokens: int = -1) -> torch.Tensor:
+        """Decode attention for the listed sequences with queries q [n][Hq][D];
+        returns fp32 [n][Hq][D]."""
+        n, hq, d = q.shape
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        tables, lens, max_len = self.decode_inputs(seq_ids)
+        if out is None:
+            out = torch.empty((n, hq, d), dtype=torch.float32, device=self.device)
+        hkv = self.k_cache.shape[1]
+        nbytes = B.pa_decode_workspace_bytes(n, hq, hkv, d, max_len, self.block_size, partition_tokens)
+        B.pa_decode(q, self.k_cache, self.v_cache, self._tables.upload(tables), self._lens.upload(lens), scale, out,
+                    max_len, partition_tokens, self.workspace(nbytes))
+        return out
+
+    def step(self, seq_ids, q, k, v, scale=None, out=None, partition_tokens=-1):
+        """One decode step: append each sequence's new K/V, then attend."""
+        self.append(seq_ids, k, v)
+        return self.decode(seq_ids, q, scale, out, partition_tokens)

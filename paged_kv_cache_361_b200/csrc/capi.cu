@@ -1,0 +1,244 @@
+// C-ABI entry points of libpagedattn: argument checks, kernel selection and
+// launches. The declarations and their contracts are in include/pagedattn.h.
+#include <cmath>
+#include <cstdint>
+
+#include "cache_ops.cuh"
+#include "decode_simt.cuh"
+
+namespace {
+
+using namespace pa;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2_block(int32_t bs) { return bs == 1 || bs == 2 || bs == 4 || bs == 8 || bs == 16 || bs == 32; }
+int elem_bytes(int32_t dtype) { return dtype == PA_BF16 ? 2 : 4; }
+
+pa_status check_cache(const pa_cache* c) {
+  if (!c || !c->k || !c->v || !aligned16(c->k) || !aligned16(c->v)) return PA_ERR_INVALID_ARG;
+  if (c->num_blocks <= 0 || c->num_blocks > INT32_MAX || c->num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (!pow2_block(c->block_size)) return PA_ERR_UNSUPPORTED;
+  if (c->dtype != PA_F32 && c->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  // slots must fit in int64 and block ids in int32 (checked above)
+  return PA_OK;
+}
+
+pa_status launched() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+int32_t resolve_partition(int32_t num_seqs, int32_t hkv, int32_t max_ctx, int32_t bs, int32_t requested) {
+  if (requested >= 0) return requested;
+  (void)num_seqs;
+  (void)hkv;
+  // Split long sequences into 512-token partitions: equal-sized work items
+  // balance the SMs when lengths differ, and long contexts get parallelism.
+  if (max_ctx <= 1024) return 0;
+  int32_t p = 512;
+  if (p % bs) p = bs;  // unreachable for bs <= 32; kept for clarity of the rule
+  return p;
+}
+
+int32_t num_parts(int32_t max_ctx, int32_t P) {
+  if (P <= 0 || max_ctx <= 0) return 1;
+  return (max_ctx + P - 1) / P;
+}
+
+size_t ws_bytes(int32_t num_seqs, int32_t hq, int32_t D, int32_t max_parts) {
+  if (max_parts <= 1) return 0;
+  const size_t rows = static_cast<size_t>(num_seqs) * hq * max_parts;
+  const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+  return ml + rows * D * sizeof(float);
+}
+
+template <typename T, int D, int G>
+pa_status launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
+  using Cfg = SimtCfg<T, D>;
+  auto kern = decode_simt_kernel<T, D, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(a);
+  return launched();
+}
+
+template <typename T, int D>
+pa_status dispatch_g(const DecodeArgs& a, int G, dim3 grid, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_simt<T, D, 1>(a, grid, st);
+    case 2: return launch_simt<T, D, 2>(a, grid, st);
+    case 4: return launch_simt<T, D, 4>(a, grid, st);
+    case 8: return launch_simt<T, D, 8>(a, grid, st);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+// One thread waits on an mbarrier that nothing will complete: exercises the
+// bounded-wait path that every pipelined kernel uses.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, timeout_ns);
+}
+
+template <int D>
+pa_status launch_reduce(const DecodeArgs& a, cudaStream_t st) {
+  dim3 grid(a.hq, a.num_seqs);
+  decode_reduce_kernel<D><<<grid, D, 0, st>>>(a);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_NO_FREE_BLOCKS: return "no free blocks";
+    case PA_ERR_UNKNOWN_SEQ: return "unknown sequence";
+    case PA_ERR_SEQ_EXISTS: return "sequence already exists";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_DEVICE_BOUNDS: return "device index out of bounds";
+    case PA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t pa_version(void) { return 1; }
+
+pa_status pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                               const pa_cache* cache, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
+    return PA_ERR_INVALID_ARG;
+  const int32_t row_chunks = cache->head_dim * elem_bytes(cache->dtype) / 16;
+  const int64_t total = static_cast<int64_t>(num_tokens) * cache->num_kv_heads * row_chunks;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 64) blocks = 148 * 64;  // grid-stride beyond this
+  reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const int4*>(k), static_cast<const int4*>(v), slot_mapping, static_cast<int4*>(cache->k),
+      static_cast<int4*>(cache->v), num_tokens, cache->num_kv_heads, cache->block_size, row_chunks,
+      cache->num_blocks * cache->block_size);
+  return launched();
+}
+
+pa_status pa_copy_blocks(const pa_cache* cache, const int32_t* src_dst_pairs, int32_t n_pairs, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (n_pairs < 0) return PA_ERR_INVALID_ARG;
+  if (n_pairs == 0) return PA_OK;
+  if (!src_dst_pairs || (reinterpret_cast<uintptr_t>(src_dst_pairs) & 7)) return PA_ERR_INVALID_ARG;
+  const int64_t chunks = static_cast<int64_t>(cache->num_kv_heads) * cache->block_size * cache->head_dim *
+                         elem_bytes(cache->dtype) / 16;
+  const int threads = 256;
+  int64_t bpp = (chunks + threads * 4 - 1) / (threads * 4);  // ~4 vectors per thread per tensor
+  if (bpp < 1) bpp = 1;
+  const int64_t grid = bpp * n_pairs;
+  if (grid > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  copy_blocks_kernel<<<static_cast<unsigned>(grid), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<int4*>(cache->k), static_cast<int4*>(cache->v), src_dst_pairs, n_pairs, chunks,
+      static_cast<int32_t>(bpp), cache->num_blocks);
+  return launched();
+}
+
+int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t max_context_len, int32_t block_size) {
+  (void)num_q_heads;
+  return resolve_partition(num_seqs, num_kv_heads, max_context_len, block_size, -1);
+}
+
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t max_context_len, int32_t block_size, int32_t partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0) return 0;
+  const int32_t P = resolve_partition(num_seqs, num_kv_heads, max_context_len, block_size, partition_tokens);
+  return ws_bytes(num_seqs, num_q_heads, head_dim, num_parts(max_context_len, P));
+}
+
+pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, float scale, float* out, int32_t partition_tokens, void* workspace,
+                    size_t workspace_bytes, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0) return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int G = num_q_heads / cache->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * cache->block_size)
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (partition_tokens < -1 || (partition_tokens > 0 && partition_tokens % cache->block_size))
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !block_tables || !context_lens || !out || !aligned16(q) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs > 65535) return PA_ERR_UNSUPPORTED;
+
+  const int32_t P = resolve_partition(num_seqs, cache->num_kv_heads, max_context_len, cache->block_size,
+                                      partition_tokens);
+  const int32_t parts = num_parts(max_context_len, P);
+  if (parts > 65535) return PA_ERR_UNSUPPORTED;
+  const size_t need = ws_bytes(num_seqs, num_q_heads, cache->head_dim, parts);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_INVALID_ARG;
+
+  DecodeArgs a;
+  a.q = q;
+  a.kc = cache->k;
+  a.vc = cache->v;
+  a.tables = block_tables;
+  a.lens = context_lens;
+  a.out = out;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * parts;
+  a.ws_ml = need ? static_cast<float*>(workspace) : nullptr;
+  a.ws_o = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + (rows * 2 * sizeof(float) + 255) / 256 * 256)
+                : nullptr;
+  a.num_blocks = cache->num_blocks;
+  a.num_seqs = num_seqs;
+  a.hq = num_q_heads;
+  a.hkv = cache->num_kv_heads;
+  a.bs = cache->block_size;
+  a.max_blocks = max_blocks_per_seq;
+  a.max_ctx = max_context_len;
+  a.part_tokens = parts > 1 ? P : 0;
+  a.max_parts = parts;
+  a.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(cache->num_kv_heads, num_seqs, parts);
+  const int D = cache->head_dim;
+  if (cache->dtype == PA_BF16) {
+    st = D == 128 ? dispatch_g<__nv_bfloat16, 128>(a, G, grid, s) : dispatch_g<__nv_bfloat16, 64>(a, G, grid, s);
+  } else {
+    st = D == 128 ? dispatch_g<float, 128>(a, G, grid, s) : dispatch_g<float, 64>(a, G, grid, s);
+  }
+  if (st != PA_OK || parts <= 1) return st;
+  return D == 128 ? launch_reduce<128>(a, s) : launch_reduce<64>(a, s);
+}
+
+pa_status pa_selftest_wait_timeout(int64_t timeout_ns, pa_stream stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return PA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(timeout_ns));
+  return launched();
+}
+
+pa_status pa_get_device_error(pa_stream stream, int64_t* info_out) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  unsigned long long w = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&w, pa::g_error_word, sizeof(w)) != cudaSuccess) return PA_ERR_CUDA;
+  if (w == 0) {
+    if (info_out) *info_out = 0;
+    return PA_OK;
+  }
+  if (cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PA_ERR_CUDA;
+  if (info_out) *info_out = static_cast<int64_t>(static_cast<int32_t>(w & 0xffffffffull));
+  return static_cast<pa_status>(w >> 32);
+}
+
+}  // extern "C"

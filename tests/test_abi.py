@@ -1,0 +1,90 @@
+"""The C-ABI library loads without a GPU and exports every declared entry point;
+host-side argument checks answer before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_361_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(pa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(B.LIB_PATH)
+    declared = _declared()
+    assert len(declared) >= 20
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) <= set(B.exported_symbols())
+
+
+def test_status_strings_and_version():
+    lib = B._lib()
+    assert lib.pa_version() == 1
+    for code in range(9):
+        assert lib.pa_status_string(code)
+    assert lib.pa_status_string(99) == b"unknown status"
+
+
+def _cache(**kw):
+    c = dict(k=16, v=32, num_blocks=8, num_kv_heads=2, block_size=16, head_dim=128, dtype=B.PA_BF16)
+    c.update(kw)
+    return B.pa_cache(**c)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0), B.PA_ERR_INVALID_ARG),
+    (dict(k=17), B.PA_ERR_INVALID_ARG),
+    (dict(num_blocks=0), B.PA_ERR_INVALID_ARG),
+    (dict(head_dim=96), B.PA_ERR_UNSUPPORTED),
+    (dict(block_size=3), B.PA_ERR_UNSUPPORTED),
+    (dict(block_size=64), B.PA_ERR_UNSUPPORTED),
+    (dict(dtype=7), B.PA_ERR_UNSUPPORTED),
+])
+def test_host_checks_before_launch(kw, status):
+    lib = B._lib()
+    c = _cache(**kw)
+    assert lib.pa_reshape_and_cache(16, 16, 16, 1, ctypes.byref(c), None) == status
+    assert lib.pa_copy_blocks(ctypes.byref(c), 16, 1, None) == status
+
+
+def test_decode_argument_checks():
+    lib = B._lib()
+    c = _cache()
+    args = dict(q=16, B=2, hq=4, tables=16, maxb=4, lens=16, maxctx=64, scale=0.1, out=16, P=-1, ws=0, wsb=0)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.pa_decode(a["q"], a["B"], a["hq"], ctypes.byref(c), a["tables"], a["maxb"], a["lens"], a["maxctx"],
+                             a["scale"], a["out"], a["P"], a["ws"] or None, a["wsb"], None)
+    assert call(hq=3) == B.PA_ERR_INVALID_ARG                  # not a multiple of kv heads
+    assert call(hq=32) == B.PA_ERR_UNSUPPORTED                 # group of 16
+    assert call(maxctx=65) == B.PA_ERR_INVALID_ARG             # above max_blocks * block_size
+    assert call(P=8) == B.PA_ERR_INVALID_ARG                   # not a multiple of block_size
+    assert call(scale=float("nan")) == B.PA_ERR_INVALID_ARG
+    assert call(q=0) == B.PA_ERR_INVALID_ARG
+    assert call(out=8) == B.PA_ERR_INVALID_ARG                 # misaligned
+    assert call(B=0) == B.PA_OK                                # nothing to do, nothing launched
+    assert call(P=16, maxctx=64) == B.PA_ERR_INVALID_ARG        # split needs a workspace
+
+
+def test_workspace_sizes():
+    # no split -> no workspace; split -> (m, l) rows rounded to 256 B + D floats per row
+    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 600, 16, 0) == 0
+    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 512, 16, 512) == 0
+    rows = 4 * 8 * 2
+    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 600, 16, 512) == (rows * 8 + 255) // 256 * 256 + rows * 128 * 4
+    assert B.pa_decode_partition_tokens(64, 32, 32, 2049, 16) in (0, 512) or B.pa_decode_partition_tokens(
+        64, 32, 32, 2049, 16) % 16 == 0

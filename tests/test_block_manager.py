@@ -1,0 +1,147 @@
+"""The C++ block manager (through the C ABI) against the oracle model, bit-exact:
+slots, copy-on-write pairs, tables, reference counts, free lists and waste
+statistics after the operation scripts of every workload. No GPU needed."""
+import numpy as np
+import pytest
+
+from oracle.block_manager import BlockManagerModel
+from paged_kv_cache_361_b200 import binding as B
+from paged_kv_cache_361_b200 import workloads as W
+
+
+def _replay_both(num_blocks, block_size, free_order, ops, check_every=1, check_free_every=50):
+    cpp = B.BlockManager(num_blocks, block_size, free_order)
+    ref = BlockManagerModel(num_blocks, block_size, free_order)
+    live = set()
+    n_pairs = 0
+    for i, op in enumerate(ops):
+        kind = op[0]
+        if kind == "add":
+            a = cpp.add_seq(op[1], op[2])
+            b = ref.add_seq(op[1], op[2])
+            assert a.tolist() == b
+            live.add(op[1])
+        elif kind == "fork":
+            cpp.fork(op[1], op[2])
+            ref.fork(op[1], op[2])
+            live.add(op[2])
+        elif kind == "append":
+            slots, pairs = cpp.append_slots(op[1])
+            rs, rp = [], []
+            for s in op[1]:
+                sl, cow = ref.append_slot(s)
+                rs.append(sl)
+                if cow:
+                    rp.append(list(cow))
+            assert slots.tolist() == rs
+            assert pairs.tolist() == rp
+            n_pairs += len(rp)
+        elif kind == "free":
+            cpp.free_seq(op[1])
+            ref.free_seq(op[1])
+            live.discard(op[1])
+        if i % check_every == 0 or i == len(ops) - 1:
+            for s in live:
+                t, L = cpp.block_table(s)
+                assert t.tolist() == ref.block_table(s) and L == ref.lens[s]
+        if i % check_free_every == 0 or i == len(ops) - 1:
+            assert cpp.free_list().tolist() == list(ref.free)
+            st = ref.stats()
+            got = cpp.stats()
+            for k in ("free_blocks", "used_slots", "allocated_slots", "internal_waste"):
+                assert got[k] == st[k], k
+    for b in range(num_blocks):
+        assert cpp.refcount(b) == ref.ref[b]
+    return cpp, ref, n_pairs
+
+
+def test_tiny_fp32_script():
+    w = W.tiny_fp32()
+    cpp, ref, _ = _replay_both(w.num_blocks, w.shape.block_size, w.free_order, W.simple_ops(w))
+    # sequence 0 is the page's 10-token example plus the appended token
+    assert len(ref.block_table(0)) == 3 and ref.lens[0] == 11
+
+
+def test_llama2_7b_mha_script():
+    w = W.llama2_7b_mha()
+    _replay_both(w.num_blocks, w.shape.block_size, w.free_order, W.simple_ops(w), check_free_every=1)
+
+
+def test_long_context_script():
+    w = W.long_context_split()
+    _replay_both(w.num_blocks, w.shape.block_size, w.free_order, W.simple_ops(w))
+
+
+def test_parallel_sampling_script():
+    w = W.parallel_sampling()
+    _, _, n_pairs = _replay_both(w.num_blocks, w.shape.block_size, w.free_order, W.sampling_ops(w),
+                                 check_every=64, check_free_every=200)
+    assert n_pairs == 8 * 7
+
+
+def test_continuous_batching_script():
+    tr = W.continuous_batching()
+    _replay_both(tr.num_blocks, tr.shape.block_size, tr.free_order, W.batching_ops(tr), check_every=25,
+                 check_free_every=300)
+
+
+def test_batched_append_equals_sequential_with_duplicates_and_cow():
+    rng = np.random.default_rng(0)
+    for trial in range(30):
+        bs = int(rng.choice([1, 2, 4, 8]))
+        nb = 200
+        order = rng.permutation(nb)
+        a = B.BlockManager(nb, bs, order)
+        b = BlockManagerModel(nb, bs, order)
+        a.add_seq(0, int(rng.integers(0, 3 * bs)))
+        b.add_seq(0, a.block_table(0)[1])
+        for c in range(1, 4):
+            a.fork(0, c)
+            b.fork(0, c)
+        ids = rng.integers(0, 4, size=12).tolist()
+        slots, pairs = a.append_slots(ids)
+        rs, rp = [], []
+        for s in ids:
+            sl, cow = b.append_slot(s)
+            rs.append(sl)
+            if cow:
+                rp.append(list(cow))
+        assert slots.tolist() == rs and pairs.tolist() == rp
+        assert a.free_list().tolist() == list(b.free)
+
+
+def test_errors_leave_state_unchanged():
+    bm = B.BlockManager(4, 4, [3, 2, 1, 0])
+    bm.add_seq(1, 8)
+    bm.fork(1, 2)
+    before = (bm.free_list().tolist(), bm.block_table(1)[0].tolist(), bm.block_table(2)[0].tolist())
+    with pytest.raises(B.PagedAttnError) as e:
+        bm.add_seq(3, 9)
+    assert e.value.status == B.PA_ERR_NO_FREE_BLOCKS
+    with pytest.raises(B.PagedAttnError) as e:
+        bm.add_seq(1, 1)
+    assert e.value.status == B.PA_ERR_SEQ_EXISTS
+    with pytest.raises(B.PagedAttnError) as e:
+        bm.free_seq(9)
+    assert e.value.status == B.PA_ERR_UNKNOWN_SEQ
+    with pytest.raises(B.PagedAttnError) as e:
+        bm.fork(9, 10)
+    assert e.value.status == B.PA_ERR_UNKNOWN_SEQ
+    # a batch needing 3 fresh blocks with 2 free fails whole
+    with pytest.raises(B.PagedAttnError) as e:
+        bm.append_slots([1, 2, 1, 2, 1, 2, 1, 2, 1])
+    assert e.value.status == B.PA_ERR_NO_FREE_BLOCKS
+    assert before == (bm.free_list().tolist(), bm.block_table(1)[0].tolist(), bm.block_table(2)[0].tolist())
+    with pytest.raises(B.PagedAttnError):
+        B.BlockManager(4, 4, [0, 1, 1, 2])      # not a permutation
+    with pytest.raises(B.PagedAttnError) as e:
+        bm.block_tables([1, 2], cap=1)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+def test_block_tables_padding():
+    bm = B.BlockManager(10, 4)
+    bm.add_seq(5, 9)
+    bm.add_seq(6, 1)
+    t, lens = bm.block_tables([6, 5], cap=4, pad=-1)
+    assert t.tolist() == [[3, -1, -1, -1], [0, 1, 2, -1]] and lens.tolist() == [1, 9]

@@ -1,0 +1,148 @@
+"""GPU parity of pa_decode / pa_reshape_and_cache / pa_copy_blocks against the
+oracle on small seeded cases: every block size, head size, group size and
+dtype, split and unsplit, plus the degenerate and error cases."""
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_361_b200 import PagedKVCache, binding as B
+from paged_kv_cache_361_b200 import workloads as W
+from tests.parity import Replay, TOL, bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_error_word():
+    if torch.cuda.is_available():
+        B.pa_get_device_error()
+    yield
+
+
+def test_tiny_fp32_config():
+    """2 sequences of 10 and 7 tokens (the first is the pages' 10-token example),
+    4 heads, head_dim 64, block_size 4, pool 16: full pool and outputs."""
+    w = W.tiny_fp32()
+    r = Replay(w.shape, w.num_blocks, w.free_order, w.scale).run(W.simple_ops(w))
+    r.check_pool_bitwise()
+    err = r.check_outputs(tol=1e-5)
+    assert err <= 1e-5
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("bs", [1, 2, 4, 8, 16, 32])
+def test_fuzz_shapes(dtype, D, G, bs):
+    hkv = 2
+    sh = W.Shape(hkv * G, hkv, D, bs, dtype)
+    seed = zlib.crc32(f"{dtype}-{D}-{G}-{bs}".encode()) % 100000
+    w = W.random_small(seed, num_seqs=6, shape=sh, max_len=int(np.random.default_rng(seed).integers(40, 300)))
+    for P in (0, -1, max(bs, 32), 2 * bs):
+        r = Replay(sh, w.num_blocks, w.free_order, w.scale, partition_tokens=P).run(W.simple_ops(w))
+        r.check_outputs()
+    r.check_pool_bitwise()
+
+
+@pytest.mark.parametrize("P", [0, 16, 48, 64, 512, -1])
+def test_partitions_agree(P):
+    """Splitting a sequence into partitions and merging equals the oracle."""
+    sh = W.Shape(8, 2, 128, 16, "bf16")
+    w = W.random_small(11, num_seqs=5, shape=sh, max_len=1500)
+    r = Replay(sh, w.num_blocks, w.free_order, w.scale, partition_tokens=P).run(W.simple_ops(w))
+    r.check_outputs()
+
+
+def test_empty_context_gives_zero_rows():
+    sh = W.Shape(4, 2, 64, 8, "bf16")
+    cache = PagedKVCache(8, 2, 8, 64, torch.bfloat16, "cuda", fill=float("nan"))
+    cache.add_sequence(0, torch.zeros(0, 2, 64, dtype=torch.bfloat16, device="cuda"),
+                       torch.zeros(0, 2, 64, dtype=torch.bfloat16, device="cuda"))
+    k = torch.randn(5, 2, 64, device="cuda").bfloat16()
+    cache.add_sequence(1, k, k)
+    q = torch.randn(2, 4, 64, device="cuda").bfloat16()
+    for P in (0, 8, -1):
+        out = cache.decode([0, 1], q, 0.125, partition_tokens=P)
+        assert torch.equal(out[0], torch.zeros_like(out[0]))
+        assert torch.isfinite(out[1]).all()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+
+
+def test_single_token_context_returns_v():
+    sh = W.Shape(8, 1, 128, 16, "bf16")
+    cache = PagedKVCache(4, 1, 16, 128, torch.bfloat16, "cuda", fill=float("nan"))
+    k = torch.randn(1, 1, 128, device="cuda").bfloat16()
+    v = torch.randn(1, 1, 128, device="cuda").bfloat16()
+    cache.add_sequence(7, k, v)
+    out = cache.decode([7], torch.randn(1, 8, 128, device="cuda").bfloat16(), 0.1)
+    assert torch.equal(out[0], v[0, 0].float().expand(8, 128))
+
+
+def test_physical_permutation_is_bitwise_invisible():
+    """Same sequences, different physical placement: identical output bits."""
+    sh = W.Shape(16, 4, 128, 16, "bf16")
+    w = W.random_small(5, num_seqs=4, shape=sh, max_len=700)
+    outs = []
+    for perm in range(3):
+        order = np.random.default_rng(perm).permutation(w.num_blocks)
+        r = Replay(sh, w.num_blocks, order, w.scale).run(W.simple_ops(w))
+        outs.append(r.decodes[-1][2])
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+def test_copy_blocks_bitwise_and_bounds():
+    kc = torch.randn(10, 4, 16, 128, device="cuda").bfloat16()
+    vc = torch.randn(10, 4, 16, 128, device="cuda").bfloat16()
+    k0, v0 = kc.clone(), vc.clone()
+    pairs = torch.tensor([[1, 7], [2, 8], [3, 9]], dtype=torch.int32, device="cuda")
+    B.pa_copy_blocks(kc, vc, pairs)
+    for s_, d_ in [(1, 7), (2, 8), (3, 9)]:
+        assert torch.equal(bits(kc[d_]), bits(k0[s_])) and torch.equal(bits(vc[d_]), bits(v0[s_]))
+    for b in range(7):
+        assert torch.equal(bits(kc[b]), bits(k0[b]))
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    bad = torch.tensor([[0, 10]], dtype=torch.int32, device="cuda")
+    B.pa_copy_blocks(kc, vc, bad)
+    st, info = B.pa_get_device_error()
+    assert st == B.PA_ERR_DEVICE_BOUNDS and info == 10
+
+
+def test_reshape_and_cache_skip_and_bounds():
+    kc = torch.zeros(4, 2, 4, 64, device="cuda")
+    vc = torch.zeros(4, 2, 4, 64, device="cuda")
+    k = torch.randn(3, 2, 64, device="cuda")
+    v = torch.randn(3, 2, 64, device="cuda")
+    B.pa_reshape_and_cache(k, v, torch.tensor([5, -1, 15], device="cuda"), kc, vc)
+    assert torch.equal(kc[1, :, 1], k[0]) and torch.equal(vc[3, :, 3], v[2])
+    assert int((kc != 0).sum()) == 2 * 2 * 64
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    B.pa_reshape_and_cache(k, v, torch.tensor([0, 16, -2], device="cuda"), kc, vc)
+    st, info = B.pa_get_device_error()
+    assert st == B.PA_ERR_DEVICE_BOUNDS and info in (16, -2)
+
+
+def test_decode_bad_block_id_and_length_are_reported():
+    cache = PagedKVCache(4, 1, 16, 64, torch.bfloat16, "cuda", fill=0.0)
+    q = torch.randn(1, 1, 64, device="cuda").bfloat16()
+    out = torch.empty(1, 1, 64, device="cuda")
+    tables = torch.tensor([[0, 9]], dtype=torch.int32, device="cuda")
+    B.pa_decode(q, cache.k_cache, cache.v_cache, tables, torch.tensor([20], dtype=torch.int32, device="cuda"),
+                0.1, out, 32, 0)
+    st, info = B.pa_get_device_error()
+    assert st == B.PA_ERR_DEVICE_BOUNDS and info == 9
+    B.pa_decode(q, cache.k_cache, cache.v_cache, tables, torch.tensor([40], dtype=torch.int32, device="cuda"),
+                0.1, out, 32, 0)
+    st, info = B.pa_get_device_error()
+    assert st == B.PA_ERR_DEVICE_BOUNDS and info == 40
+
+
+def test_wait_limit_returns_status():
+    """A wait that nothing completes ends with PA_ERR_DEVICE_TIMEOUT; the context stays usable."""
+    B.pa_selftest_wait_timeout(50_000_000)
+    st, _ = B.pa_get_device_error()
+    assert st == B.PA_ERR_DEVICE_TIMEOUT
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum()) == 8.0
