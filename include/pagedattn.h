@@ -161,6 +161,34 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
  */
 pa_status pa_get_device_error(pa_stream stream, int64_t* info_out);
 
+/* Bytes of the fixed device array behind pa_decode_static_workspace. */
+#define PA_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/*
+ * pa_decode without a caller-provided workspace, for callers that cannot
+ * allocate device memory. The pages have no counterpart: this is a deployment
+ * variant of pa_decode. Some hosts hand an attention kernel only its inputs
+ * and outputs: an inference runtime that reserves the whole device up front
+ * and gives plug-ins no workspace, or a latency-bound serving loop where a
+ * cudaMalloc (which may synchronise the device) is not allowed between steps.
+ * Arguments, results and errors are those of pa_decode; the partial results of
+ * a split sequence go to an array of PA_STATIC_WORKSPACE_BYTES compiled into
+ * the library, which every device that loads the library holds until the
+ * process exits. A call whose split would need more than that returns
+ * PA_ERR_INVALID_ARG and launches nothing (pa_decode_workspace_bytes gives the
+ * need; partition_tokens = 0 needs none).
+ * The first call on each device looks up that device's address of the array
+ * (make it before any stream capture). The array is shared by every call on
+ * the device and keeps the last call's contents; nothing in it needs an
+ * initial value. Calls that overlap on the GPU (other streams, other threads)
+ * race on the array and must be serialised by the caller.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t max_context_len, float scale, float* out,
+                                     int32_t partition_tokens, pa_stream stream);
+
 /*
  * Self-test of the device wait limit. Every pipelined kernel waits for its own
  * copies with a bounded wait; this launches one thread that waits on a barrier

@@ -49,6 +49,7 @@ _SIGS = {
     "pa_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_get_device_error": (_I32, [_VP, _P64]),
     "pa_selftest_wait_timeout": (_I32, [_I64, _VP]),
+    "pa_decode_static_workspace": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP]),
     "pa_bm_create": (_I32, [_I64, _I32, _VP, ctypes.POINTER(_VP)]),
     "pa_bm_destroy": (None, [_VP]),
     "pa_bm_add_seq": (_I32, [_VP, _I64, _I32, _VP]),
@@ -176,6 +177,26 @@ def pa_get_device_error(stream=None):
     info = ctypes.c_int64(0)
     st = _lib().pa_get_device_error(handle, ctypes.byref(info))
     return int(st), int(info.value)
+
+
+def pa_decode_static_workspace(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_context_len,
+                               partition_tokens=-1, stream=None):
+    """pa_decode with the library's fixed device workspace (no allocation)."""
+    c = make_cache(k_cache, v_cache)
+    B, hq, d = q.shape
+    _dev(q, "q", k_cache.dtype, 3)
+    _dev(out, "out", torch.float32, 3)
+    if d != c.head_dim or tuple(out.shape) != (B, hq, d):
+        raise ValueError("q/out shape mismatch")
+    _dev(block_tables, "block_tables", torch.int32, 2)
+    _dev(context_lens, "context_lens", torch.int32, 1)
+    if block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("block_tables / context_lens must have num_seqs rows")
+    _check(_lib().pa_decode_static_workspace(q.data_ptr(), B, hq, ctypes.byref(c), block_tables.data_ptr(),
+                                             int(block_tables.shape[1]), context_lens.data_ptr(),
+                                             int(max_context_len), float(scale), out.data_ptr(),
+                                             int(partition_tokens), _stream(q, stream)),
+           "pa_decode_static_workspace")
 
 
 def pa_selftest_wait_timeout(timeout_ns: int, stream=None):

@@ -2,6 +2,7 @@
 // launches. The declarations and their contracts are in include/pagedattn.h.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "cache_ops.cuh"
 #include "decode_simt.cuh"
@@ -242,3 +243,63 @@ pa_status pa_get_device_error(pa_stream stream, int64_t* info_out) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode (pa_decode_static_workspace).
+//
+// For callers that are handed only inputs and outputs and may not allocate
+// device memory (a runtime that owns the whole device, or a serving loop where
+// cudaMalloc's possible device synchronisation is not allowed), the split
+// partials live in this fixed array instead of a caller workspace. Every
+// device that loads the library holds it until the process exits.
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_ws[PA_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// In host code g_static_ws names a host-side stand-in, not device memory, so
+// the device address is looked up once per device (with that device current)
+// and cached. The first call on a device therefore makes a runtime query.
+void* static_ws_address(pa_status* st) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = PA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) {
+      *st = PA_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  *st = PA_OK;
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t num_q_heads,
+                                                const pa_cache* cache, const int32_t* block_tables,
+                                                int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                                int32_t max_context_len, float scale, float* out,
+                                                int32_t partition_tokens, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || partition_tokens < -1) return PA_ERR_INVALID_ARG;
+  const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, cache->num_kv_heads, cache->head_dim,
+                                                max_context_len, cache->block_size, partition_tokens);
+  if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  if (need > 0) {
+    ws = static_ws_address(&st);
+    if (st != PA_OK) return st;
+  }
+  return pa_decode(q, num_seqs, num_q_heads, cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                   scale, out, partition_tokens, ws, need > 0 ? PA_STATIC_WORKSPACE_BYTES : 0, stream);
+}
