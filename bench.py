@@ -37,7 +37,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode attention tokens/sec"
-WORKLOAD = "llama2_7b_mha_decode: 64 seqs, ctx U[128,2048]+1, 32/32 heads, D128, bs16, bf16"
 
 
 def peaks():
@@ -110,43 +109,84 @@ class Clocks:
 
 # --- workload --------------------------------------------------------------------
 
-def build_workload(seed: int, device):
-    """The pool filled with N(0,1) values on the device (it stands in for the
-    prompts' K/V), every sequence's blocks reserved through the C++ block
-    manager, then one append per sequence: the step's slots, tables, lengths."""
+WORKLOADS = {
+    "llama2_7b_mha": "llama2_7b_mha_decode: 64 seqs, ctx U[128,2048]+1, 32/32 heads, D128, bs16, bf16",
+    "long_context_split": "long_context_split_decode: 4 seqs, ctx 32768/65536/98304/131072+1, 64/8 heads, D128, bs32, "
+                          "512-token partitions, bf16",
+    "parallel_sampling": "parallel_sampling_decode: 8 prompts x 8 samples, 1000-token shared prefix + tails U[1,512], "
+                         "32/8 heads, D128, bs16, bf16",
+    "continuous_batching": "continuous_batching_decode: 256 live seqs, ctx lognormal(500,1) capped 4096, first step "
+                           "of the trace, 200k-block pool, 32/8 heads, D128, bs16, bf16",
+}
+
+
+def workload_ops(name, seed):
+    """(shape, num_blocks, free_order, scale, partition_tokens, ops) of a workload;
+    the last two ops are the measured step's append and decode."""
+    from paged_kv_cache_361_b200 import workloads as W
+    if name in ("llama2_7b_mha", "long_context_split"):
+        w = W.llama2_7b_mha(seed=seed) if name == "llama2_7b_mha" else W.long_context_split(seed=seed)
+        return w.shape, w.num_blocks, w.free_order, w.scale, w.partition_tokens, W.simple_ops(w)
+    if name == "parallel_sampling":
+        w = W.parallel_sampling(seed=seed)
+        return w.shape, w.num_blocks, w.free_order, w.scale, 0, W.sampling_ops(w, batch_tail_steps=True)
+    tr = W.continuous_batching(seed=seed)
+    return tr.shape, tr.num_blocks, tr.free_order, 1.0 / math.sqrt(tr.shape.head_dim), 0, W.batching_ops(tr, steps=1)
+
+
+def build_workload(seed: int, device, name: str = "llama2_7b_mha"):
+    """Replays the workload's operation script up to the measured step through
+    PagedKVCache: the pool is filled with N(0,1) values on the device (they
+    stand in for the prompts' K/V, so prefills only reserve blocks), forks
+    share blocks, earlier appends write random rows (with their copy-on-write
+    block copies). The measured step's slots and pairs come from the C++ block
+    manager; its tables and lengths are uploaded once."""
     from paged_kv_cache_361_b200 import PagedKVCache
     from paged_kv_cache_361_b200 import workloads as W
-    w = W.llama2_7b_mha(seed=seed)
-    sh = w.shape
+    sh, nb, order, scale, part, ops = workload_ops(name, seed)
     dt = W.TORCH_DTYPE[sh.dtype]
-    cache = PagedKVCache(w.num_blocks, sh.num_kv_heads, sh.block_size, sh.head_dim, dt, device, w.free_order)
+    cache = PagedKVCache(nb, sh.num_kv_heads, sh.block_size, sh.head_dim, dt, device, order)
     g = torch.Generator(device=device)
     g.manual_seed(1000 + seed)
     for t in (cache.k_cache, cache.v_cache):
-        for i in range(0, w.num_blocks, 1024):   # chunked to bound the fp32 temporary
+        for i in range(0, nb, 1024):   # chunked to bound the fp32 temporary
             t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(dt)
-    ids = list(range(w.num_seqs))
-    for s in ids:
-        cache.reserve(s, int(w.context_lens_old[s]))
+    hkv, D = sh.num_kv_heads, sh.head_dim
+    assert ops[-2][0] == "append" and ops[-1][0] == "decode"
+    for op in ops[:-2]:
+        if op[0] == "add":
+            cache.reserve(op[1], op[2])
+        elif op[0] == "fork":
+            cache.fork(op[1], op[2])
+        elif op[0] == "free":
+            cache.free(op[1])
+        elif op[0] == "append":
+            n = len(op[1])
+            cache.append(op[1], torch.randn((n, hkv, D), generator=g, device=device).to(dt),
+                         torch.randn((n, hkv, D), generator=g, device=device).to(dt))
+    ids = list(ops[-1][1])
     slots, pairs = cache.bm.append_slots(ids)
-    assert len(pairs) == 0
     for s in ids:
         cache.lens[s] += 1
     tables, lens32, max_len = cache.decode_inputs(ids)
-    lens = w.context_lens
-    assert lens32.tolist() == lens.tolist()
-    B_, hq, hkv, D = w.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.head_dim
+    B_, hq = len(ids), sh.num_q_heads
+    eb = 2 if sh.dtype == "bf16" else 4
+    st = cache.bm.stats()
     return dict(
-        w=w, cache=cache, bm=cache.bm, kc=cache.k_cache, vc=cache.v_cache,
+        name=name, shape=sh, scale=scale, part=part, ids=ids, cache=cache, bm=cache.bm, kc=cache.k_cache,
+        vc=cache.v_cache,
         q=torch.randn((B_, hq, D), generator=g, device=device).to(dt),
         k=torch.randn((B_, hkv, D), generator=g, device=device).to(dt),
         v=torch.randn((B_, hkv, D), generator=g, device=device).to(dt),
         slots=torch.from_numpy(slots).to(device),
+        pairs=torch.from_numpy(pairs).to(device) if len(pairs) else None,
         tables=torch.from_numpy(tables).to(device),
         lens=torch.from_numpy(lens32).to(device),
+        lens_host=lens32.astype(np.int64),
         out=torch.empty((B_, hq, D), dtype=torch.float32, device=device),
         max_len=max_len,
-        kv_bytes=int(lens.sum()) * hkv * D * 2 * 2,
+        kv_bytes=int(lens32.astype(np.int64).sum()) * hkv * D * 2 * eb,
+        unique_kv_bytes=int(st["used_slots"]) * hkv * D * 2 * eb,
     )
 
 
@@ -154,11 +194,11 @@ def sample_rows(d, seqs):
     """Host copies (before any kernel runs) of the sampled sequences' K/V rows,
     read from the device pool through their block tables: input to the CPU
     baseline only."""
-    w, bm = d["w"], d["bm"]
-    bs = w.shape.block_size
+    bm = d["bm"]
+    bs = d["shape"].block_size
     rows = []
     for s in seqs:
-        table, L = bm.block_table(s)
+        table, L = bm.block_table(d["ids"][s])
         L_old = L - 1
         t = torch.arange(L_old)
         blk = torch.as_tensor(table, dtype=torch.int64)[t // bs].to(d["kc"].device)
@@ -200,26 +240,32 @@ def cpu_threads():
 
 def run_ours(args, rank, world, device):
     from paged_kv_cache_361_b200 import binding as B
-    d = build_workload(seed=rank, device=device)
-    w = d["w"]
-    sh = w.shape
-    P = args.partition
-    ws_bytes = B.pa_decode_workspace_bytes(w.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, d["max_len"],
+    d = build_workload(seed=rank, device=device, name=args.workload)
+    sh = d["shape"]
+    nseq = len(d["ids"])
+    P = args.partition if args.partition != -2 else d["part"]
+    ws_bytes = B.pa_decode_workspace_bytes(nseq, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, d["max_len"],
                                            sh.block_size, P)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device) if ws_bytes else None
-    P_eff = P if P >= 0 else B.pa_decode_partition_tokens(w.num_seqs, sh.num_q_heads, sh.num_kv_heads,
-                                                          d["max_len"], sh.block_size)
+    P_eff = P if P >= 0 else B.pa_decode_partition_tokens(nseq, sh.num_q_heads, sh.num_kv_heads, d["max_len"],
+                                                          sh.block_size)
     split = P_eff > 0 and math.ceil(d["max_len"] / P_eff) > 1
     stream = torch.cuda.current_stream(device)
 
-    baseline_rows = sample_rows(d, list(range(4))) if rank == 0 and world == 1 and not args.no_cpu_baseline else None
+    sample_seqs = [0, 1, 2, 3] if args.workload == "llama2_7b_mha" else [0]
+    baseline_rows = sample_rows(d, sample_seqs) if rank == 0 and world == 1 and not args.no_cpu_baseline else None
 
-    def step():
+    def write_step():
+        if d["pairs"] is not None:
+            B.pa_copy_blocks(d["kc"], d["vc"], d["pairs"])
         B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
-        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], w.scale, d["out"], d["max_len"], P, ws)
+
+    def decode():
+        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"], P, ws)
 
     for _ in range(args.warmup):
-        step()
+        write_step()
+        decode()
     torch.cuda.synchronize(device)
     st, info = B.pa_get_device_error()
     if st != B.PA_OK:
@@ -234,9 +280,9 @@ def run_ours(args, rank, world, device):
     clocks.start()
     t_start.record(stream)
     for i in range(args.steps):
-        B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
+        write_step()
         ev[i][0].record(stream)
-        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], w.scale, d["out"], d["max_len"], P, ws)
+        decode()
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(device)
@@ -250,7 +296,6 @@ def run_ours(args, rank, world, device):
         raise RuntimeError(f"device error {st} ({info}) in the timed region")
 
     kv_bytes = d["kv_bytes"]
-    # max over ranks of the time, sum of the bytes
     t = torch.tensor([total_ms, float(kv_bytes)], dtype=torch.float64, device=device)
     if world > 1:
         tm = t[:1].clone()
@@ -262,39 +307,39 @@ def run_ours(args, rank, world, device):
         all_bytes = float(kv_bytes)
     ms_per_step = total_ms / args.steps
     value = all_bytes / (ms_per_step * 1e-3) / 1e9
-    tokens_per_s = world * w.num_seqs / (ms_per_step * 1e-3)
+    tokens_per_s = world * nseq / (ms_per_step * 1e-3)
 
-    # end to end through the public API: inputs from pinned host memory, output back to host
-    e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(args, d, device, rank, world)
+    e2e = None if args.no_e2e else run_e2e(args, d, device, world, P)
 
     cpu = None
     if baseline_rows is not None:
-        gbs, el, n = time_oracle(baseline_rows, w.scale, args.cpu_seconds)
+        gbs, el, n = time_oracle(baseline_rows, d["scale"], args.cpu_seconds)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"fp64 NumPy oracle over sequences 0-3 of the workload (all 32 heads), repeated for "
-                         f"{el:.1f} s ({n} sequence passes); host has {os.cpu_count()} cores"}
+               "sample": f"fp64 NumPy oracle over sequences {sample_seqs} of the workload (all heads), repeated "
+                         f"for {el:.1f} s ({n} sequence passes); host has {os.cpu_count()} cores"}
 
     peak, peak_kind = peaks()
     dec_avg_ms = statistics.mean(decode_ms)
     achieved = kv_bytes / (dec_avg_ms * 1e-3) / 1e9
+    launches = args.steps * (2 + (1 if split else 0) + (1 if d["pairs"] is not None else 0))
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "num_seqs": w.num_seqs, "num_q_heads": sh.num_q_heads,
+            "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype, "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "num_seqs": nseq, "num_q_heads": sh.num_q_heads,
                        "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "block_size": sh.block_size,
-                       "num_blocks": w.num_blocks, "context_tokens": int(w.context_lens.sum()),
-                       "kv_bytes_per_step": kv_bytes, "partition_tokens": P_eff,
+                       "num_blocks": int(d["kc"].shape[0]), "context_tokens": int(d["lens_host"].sum()),
+                       "kv_bytes_per_step": kv_bytes, "unique_kv_bytes_per_step": d["unique_kv_bytes"],
+                       "partition_tokens": P_eff,
                        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                       "l2": "no flush: 1.07 GB of K/V per step >> 126 MB L2"},
+                       "l2": "no flush: the K/V read per step is larger than the 126 MB L2"
+                       if d["unique_kv_bytes"] > 3 * 126e6 else "no flush: K/V partly L2-resident (see unique bytes)"},
             "tokens_per_s": round(tokens_per_s, 1),
             "pct_of_hbm_peak": {"of_measured_6540": round(value / peak, 4), "of_nominal_8000": round(value / 8000.0, 4)},
             "e2e": e2e,
-            "gpu_launches": args.steps * (3 if split else 2),
-            "roofline": {"kernel": "pa_decode (decode + partition merge)", "bound": "hbm",
+            "gpu_launches": launches,
+            "roofline": {"kernel": "pa_decode" + (" (decode + partition merge)" if split else ""), "bound": "hbm",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": None,
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
@@ -305,41 +350,41 @@ def run_ours(args, rank, world, device):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, d, device, rank, world):
+def run_e2e(args, d, device, world, P):
     """K steps through PagedKVCache.step: per step, H2D of q/k/v from pinned host
-    memory (plus the slots, tables and lengths the API uploads), append + decode,
-    D2H of the fp32 output. Context lengths grow by one per step."""
-    w = d["w"]
-    sh = w.shape
+    memory (plus the slots, CoW pairs, tables and lengths the API uploads),
+    append + decode, D2H of the fp32 output. Context lengths grow by one per step."""
+    sh = d["shape"]
     cache = d["cache"]
-    ids = list(range(w.num_seqs))
+    ids = d["ids"]
     hq = torch.empty(d["q"].shape, dtype=d["q"].dtype, pin_memory=True)
     hk = torch.empty(d["k"].shape, dtype=d["k"].dtype, pin_memory=True)
     hv = torch.empty(d["v"].shape, dtype=d["v"].dtype, pin_memory=True)
-    hq.copy_(d["q"].cpu()); hk.copy_(d["k"].cpu()); hv.copy_(d["v"].cpu())
+    hq.copy_(d["q"].cpu())
+    hk.copy_(d["k"].cpu())
+    hv.copy_(d["v"].cpu())
     hout = torch.empty(d["out"].shape, dtype=torch.float32, pin_memory=True)
-    kv_total = 0
-    h2d = d2h = 0
+    eb = hq.element_size()
+    kv_total = h2d = d2h = 0
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
     for it in range(args.warmup + args.steps):
         if it == args.warmup:
             torch.cuda.synchronize(device)
             if world > 1:
                 torch.distributed.barrier()
-            t0 = torch.cuda.Event(enable_timing=True)
-            t1 = torch.cuda.Event(enable_timing=True)
             t0.record()
-            kv_total = 0
-            h2d = d2h = 0
+            kv_total = h2d = d2h = 0
         q = hq.to(device, non_blocking=True)
         k = hk.to(device, non_blocking=True)
         v = hv.to(device, non_blocking=True)
-        out = cache.step(ids, q, k, v, w.scale, partition_tokens=args.partition)
+        out = cache.step(ids, q, k, v, d["scale"], partition_tokens=P)
         hout.copy_(out, non_blocking=True)
         torch.cuda.current_stream(device).synchronize()
-        L = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64)
-        kv_total += int(L.sum()) * sh.num_kv_heads * sh.head_dim * 2 * 2
+        L = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64, count=len(ids))
+        kv_total += int(L.sum()) * sh.num_kv_heads * sh.head_dim * 2 * eb
         nblk = int(-(-L.max() // sh.block_size))
-        h2d += 3 * q.numel() * 2 + len(ids) * 8 + len(ids) * nblk * 4 + len(ids) * 4
+        h2d += (hq.numel() + hk.numel() + hv.numel()) * eb + len(ids) * (8 + 4 + nblk * 4)
         d2h += hout.numel() * 4
     t1.record()
     torch.cuda.synchronize(device)
@@ -386,7 +431,7 @@ def run_reference(args, rank, world):
     line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "sample_seqs": seqs},
+            "config": {"workload": WORKLOADS["llama2_7b_mha"], "sample_seqs": seqs},
             "tokens_per_s": round(len(seqs) / (ms * 1e-3), 3),
             "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
@@ -400,7 +445,9 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--partition", type=int, default=-1, help="partition_tokens for pa_decode (-1: library choice)")
+    ap.add_argument("--partition", type=int, default=-1,
+                    help="partition_tokens for pa_decode (-1: library choice, -2: the workload's own)")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama2_7b_mha")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -4,7 +4,10 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "cache_ops.cuh"
+#include "decode_mma.cuh"
 #include "decode_simt.cuh"
 
 namespace {
@@ -70,6 +73,67 @@ pa_status dispatch_g(const DecodeArgs& a, int G, dim3 grid, cudaStream_t st) {
     case 8: return launch_simt<T, D, 8>(a, grid, st);
     default: return PA_ERR_UNSUPPORTED;
   }
+}
+
+// cuTensorMapEncodeTiled, reached through the runtime so that the library
+// needs no link-time dependency on the driver library.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// The pool viewed as rows of head_dim bf16 (row = (block * Hkv + head) * bs +
+// offset), read in [bs x 64] boxes with the 128-byte swizzle.
+bool encode_rows(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(bs)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int G>
+pa_status launch_mma(const DecodeArgs& a, const pa_cache* c, dim3 grid, cudaStream_t st) {
+  using Cfg = MmaCfg<D>;
+  CUtensorMap tk, tv;
+  const uint64_t rows = static_cast<uint64_t>(c->num_blocks) * c->num_kv_heads * c->block_size;
+  if (!encode_rows(&tk, c->k, rows, D, c->block_size) || !encode_rows(&tv, c->v, rows, D, c->block_size))
+    return PA_ERR_CUDA;
+  auto kern = decode_mma_kernel<D, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
+  return launched();
+}
+
+// Tensor-core path: bf16 cache, a group of 4 or 8 query heads, blocks of at
+// least 8 tokens (a [bs x 64] box is then a whole number of 1 KB swizzle
+// atoms), and pool rows addressable by a 32-bit TMA coordinate.
+bool mma_eligible(const pa_cache* c, int G) {
+  return c->dtype == PA_BF16 && (G == 4 || G == 8) && c->block_size >= 8 &&
+         static_cast<int64_t>(c->num_blocks) * c->num_kv_heads * c->block_size <= INT32_MAX;
+}
+
+pa_status dispatch_mma(const DecodeArgs& a, const pa_cache* c, int G, dim3 grid, cudaStream_t st) {
+  if (c->head_dim == 128) return G == 8 ? launch_mma<128, 8>(a, c, grid, st) : launch_mma<128, 4>(a, c, grid, st);
+  return G == 8 ? launch_mma<64, 8>(a, c, grid, st) : launch_mma<64, 4>(a, c, grid, st);
 }
 
 // One thread waits on an mbarrier that nothing will complete: exercises the
@@ -214,7 +278,9 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(cache->num_kv_heads, num_seqs, parts);
   const int D = cache->head_dim;
-  if (cache->dtype == PA_BF16) {
+  if (mma_eligible(cache, G)) {
+    st = dispatch_mma(a, cache, G, grid, s);
+  } else if (cache->dtype == PA_BF16) {
     st = D == 128 ? dispatch_g<__nv_bfloat16, 128>(a, G, grid, s) : dispatch_g<__nv_bfloat16, 64>(a, G, grid, s);
   } else {
     st = D == 128 ? dispatch_g<float, 128>(a, G, grid, s) : dispatch_g<float, 64>(a, G, grid, s);

@@ -1,0 +1,203 @@
+// Pieces shared by the decode kernels: arguments, the chunk pipeline (TMA
+// producer warp + consumer warps over full/empty mbarriers), the final merge
+// of the consumer warps, and the partition merge kernel.
+//
+// P2 = "PagedAttention：操作系统级 KV 缓存虚拟内存管理", §4.1: the softmax is
+// accumulated block by block with a running maximum and sum; the same algebra
+// merges the warps of a CTA and the partitions of a sequence:
+//   M = max_i m_i,  l = sum_i l_i 2^(m_i - M),  o = sum_i o_i 2^(m_i - M)
+// (scores are kept in base 2: q is pre-scaled by scale * log2 e).
+#pragma once
+
+#include "common.cuh"
+
+namespace pa {
+
+struct DecodeArgs {
+  const void* q;
+  const void* kc;
+  const void* vc;
+  const int32_t* tables;
+  const int32_t* lens;
+  float* out;
+  float* ws_ml;   // [num_seqs][hq][max_parts][2]  (m in log2 units, l)
+  float* ws_o;    // [num_seqs][hq][max_parts][D]
+  int64_t num_blocks;
+  int32_t num_seqs, hq, hkv, bs, max_blocks, max_ctx;
+  int32_t part_tokens;  // > 0: partition size; 0: one partition per sequence
+  int32_t max_parts;    // grid.z
+  float scale_log2;     // scale * log2(e)
+};
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+  static constexpr int bytes = 4;
+};
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int bytes = 2;
+};
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Context length of sequence s, clamped to [0, max_ctx]; an out-of-range value
+// is recorded (by the one thread that `report`s).
+__device__ __forceinline__ int32_t load_len(const DecodeArgs& a, int32_t s, bool report) {
+  int32_t L = __ldg(a.lens + s);
+  if (L < 0 || L > a.max_ctx) {
+    if (report) record_error(PA_ERR_DEVICE_BOUNDS, L);
+    L = L < 0 ? 0 : a.max_ctx;
+  }
+  return L;
+}
+
+// The token range a CTA owns. Returns false if the CTA has nothing to do
+// (after writing the zero row of an empty context).
+struct Part {
+  int32_t t0, t1, ntok, nparts;
+};
+
+template <int G, int D>
+__device__ __forceinline__ bool cta_part(const DecodeArgs& a, int g, int s, int p, int tid, int nthreads, Part& pt) {
+  const int32_t L = load_len(a, s, g == 0 && p == 0 && tid == 0);
+  const int32_t P = a.part_tokens > 0 ? a.part_tokens : (L > 0 ? L : 1);
+  pt.t0 = p * P;
+  if (L == 0) {
+    if (p == 0)
+      for (int idx = tid; idx < G * D; idx += nthreads)
+        a.out[(static_cast<int64_t>(s) * a.hq + g * G) * D + idx] = 0.f;
+    return false;
+  }
+  if (pt.t0 >= L) return false;
+  pt.t1 = min(pt.t0 + P, L);
+  pt.ntok = pt.t1 - pt.t0;
+  pt.nparts = a.part_tokens > 0 ? (L + P - 1) / P : 1;
+  return true;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Wait for a phase, giving up when the CTA's abort flag is raised by another
+// warp or the wall-clock limit passes (then raising the flag itself).
+__device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t start = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - start > kWaitTimeoutNs) {
+        record_error(PA_ERR_DEVICE_TIMEOUT, 0);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Per-CTA pipeline state in shared memory: S stages, each with a "full"
+// barrier (one producer arrival + the TMA byte count) and an "empty" barrier
+// (one arrival per consumer warp).
+template <int S>
+struct PipeSmem {
+  uint64_t full[S];
+  uint64_t empty[S];
+  int abort_flag;
+};
+
+template <int S>
+__device__ __forceinline__ void pipe_init(PipeSmem<S>& ps, int consumer_warps) {
+#pragma unroll
+  for (int i = 0; i < S; ++i) {
+    mbar_init(&ps.full[i], 1);
+    mbar_init(&ps.empty[i], consumer_warps);
+  }
+  ps.abort_flag = 0;
+  fence_mbar_init();
+}
+
+// Producer warp: for each chunk, wait until its stage is free, then let
+// issue(i, stage) start the chunk's copies (issue arrives on full[stage] with
+// the byte count). On abort, wait (bounded) for the copies already started.
+template <int S, class Issue>
+__device__ __forceinline__ void pipe_produce(PipeSmem<S>& ps, int nchunks, Issue issue) {
+  int i = 0;
+  for (; i < nchunks; ++i) {
+    const int st = i % S;
+    if (i >= S && !pipe_wait(&ps.empty[st], ((i / S) - 1) & 1, &ps.abort_flag)) break;
+    issue(i, st);
+  }
+  if (ps.abort_flag) {
+    // the latest phase of every stage that was filled must land before exit
+    for (int j = (i > S ? i - S : 0); j < i; ++j) mbar_wait(&ps.full[j % S], (j / S) & 1);
+  }
+}
+
+// Merge the consumer warps' (m, l, o) for the G heads of this CTA and store
+// either the final row (one partition) or the partition's partials.
+//   wm, wl: [NW][G];  wacc: [NW][G][D]
+template <int G, int D, int NW>
+__device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const float* wm, const float* wl,
+                                                      const float* wacc, int s, int p, int hq0, int nparts, int tid,
+                                                      int nthreads) {
+  for (int idx = tid; idx < G * D; idx += nthreads) {
+    const int h = idx / D, d = idx - h * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w * G + h]);
+    float l = 0.f, o = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float f = exp2f(wm[w * G + h] - M);
+      l = fmaf(wl[w * G + h], f, l);
+      o = fmaf(wacc[(w * G + h) * D + d], f, o);
+    }
+    const int64_t row = static_cast<int64_t>(s) * a.hq + hq0 + h;
+    if (nparts == 1) {
+      a.out[row * D + d] = o / l;
+    } else {
+      const int64_t prow = row * a.max_parts + p;
+      a.ws_o[prow * D + d] = o;
+      if (d == 0) {
+        a.ws_ml[prow * 2] = M;
+        a.ws_ml[prow * 2 + 1] = l;
+      }
+    }
+  }
+}
+
+// Merge the partitions of one (sequence, query head):
+//   M = max_p m_p,  out = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).
+// Grid (hq, num_seqs), D threads. Sequences with one partition were written
+// by the decode kernel and are skipped.
+template <int D>
+__global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
+  const int hq = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+  const int32_t L = load_len(a, s, false);
+  const int32_t P = a.part_tokens;
+  const int32_t nparts = (L + P - 1) / P;
+  if (nparts <= 1) return;
+  const int64_t row = static_cast<int64_t>(s) * a.hq + hq;
+  const float* ml = a.ws_ml + row * a.max_parts * 2;
+  const float* o = a.ws_o + row * a.max_parts * D;
+  float M = -INFINITY;
+  for (int q = 0; q < nparts; ++q) M = fmaxf(M, ml[2 * q]);
+  float l = 0.f, acc = 0.f;
+  for (int q = 0; q < nparts; ++q) {
+    const float f = exp2f(ml[2 * q] - M);
+    l = fmaf(ml[2 * q + 1], f, l);
+    acc = fmaf(o[static_cast<int64_t>(q) * D + d], f, acc);
+  }
+  a.out[row * D + d] = acc / l;
+}
+
+}  // namespace pa

@@ -1,0 +1,274 @@
+// Paged decode attention on the tensor cores, for grouped-query heads.
+//
+// P2 = "PagedAttention：操作系统级 KV 缓存虚拟内存管理".
+//   §1.1  out = softmax(scale * q K^T) V.
+//   §3.2.2 step 4, §4.1  every logical block is visited through the block
+//         table, the query group stays in registers, and the softmax is
+//         accumulated tile by tile.
+//   §4.2  blocks are contiguous; they are moved as whole tiles.
+//
+// When G = Hq / Hkv query heads share a kv head, each K/V byte feeds 2G
+// multiply-adds; on the CUDA cores that (plus the bf16 unpacking and the
+// cross-lane reductions) outruns the instruction issue rate before HBM is
+// saturated. Here the two contractions run as m16n8k16 bf16 MMAs with the G
+// heads as the M rows (rows G..15 are zero):
+//   S = Q K^T : A = Q (registers, loaded once), B = K tile via ldmatrix;
+//   O += P V  : A = P (the S accumulator re-packed in registers, split into a
+//               bf16 high part and a bf16 remainder so that P keeps ~16
+//               mantissa bits), B = V tile via ldmatrix.trans.
+// K/V tiles arrive by TMA tensor copies (cp.async.bulk.tensor.2d) of
+// [block_size rows x 64 dims] boxes with the 128-byte swizzle, so the 8-row
+// ldmatrix reads hit 8 different bank groups. Tokens past the context length
+// get -inf scores and their V rows are zeroed in registers, so padding (even
+// NaN) never reaches the result.
+// CTA = (kv head, sequence, partition): warp 4 is the TMA producer, warps 0-3
+// consume (warp w owns tokens [16w, 16w+16) of each 64-token chunk) over the
+// same full/empty mbarrier ring as the CUDA-core kernel.
+#pragma once
+
+#include <cuda.h>
+
+#include "decode_common.cuh"
+
+namespace pa {
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// d += A(16x16, rows 8..15 zero) * B(16x8), bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma_rows8(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// p -> (bf16(p), bf16(p - bf16(p))) for a pair.
+__device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
+template <int D>
+struct MmaCfg {
+  static constexpr int kConsumerWarps = 4;
+  static constexpr int kThreads = 32 * (kConsumerWarps + 1);
+  static constexpr int kChunk = 64;                        // tokens per stage
+  static constexpr int kHalves = D / 64;                   // 128-byte column boxes per row
+  static constexpr int kHalfBytes = kChunk * 128;          // one box column of a stage
+  static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = kStageBytes <= 16384 ? 4 : 3;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack for the swizzle
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
+                                                                        const __grid_constant__ CUtensorMap tmv,
+                                                                        const DecodeArgs a) {
+  using Cfg = MmaCfg<D>;
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = D / 8;
+  static_assert(G <= 8, "query heads of one group must fit in MMA rows 0..7");
+  static_assert(NW * G * (D + 2) * 4 <= S * Cfg::kStageBytes, "merge buffer must fit in the stage ring");
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ PipeSmem<S> ps;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;  // 1024-aligned: swizzle atoms
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+
+  const int g = blockIdx.x, s = blockIdx.y, p = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, c = lane & 3;
+  Part pt;
+  if (!cta_part<G, D>(a, g, s, p, tid, Cfg::kThreads, pt)) return;
+  const int nchunks = (pt.ntok + C - 1) / C;
+  const int hq0 = g * G;
+
+  if (tid == 0) pipe_init<S>(ps, NW);
+  __syncthreads();
+
+  float o[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+
+  if (warp == NW) {
+    // ---- producer: one 2D TMA box [bs rows x 64 dims] per (block, half) of K and V ----
+    const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
+    const uint64_t pol = l2_evict_first_policy();
+    pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+      const int32_t c0 = pt.t0 + i * C;
+      const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+      int32_t blk = -1;
+      bool ok = false;
+      if (lane < nb) {
+        blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
+        ok = blk >= 0 && blk < a.num_blocks;
+        if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * Cfg::kHalves * __popc(okmask) * box_bytes);
+      __syncwarp();
+      if (ok) {
+        const int32_t y = (blk * a.hkv + g) * a.bs;
+        const uint32_t kdst = sbase + st * Cfg::kStageBytes + lane * box_bytes;
+#pragma unroll
+        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+          tma_load_2d(kdst + hf * Cfg::kHalfBytes, &tmk, hf * 64, y, &ps.full[st], pol);
+          tma_load_2d(kdst + Cfg::kTileBytes + hf * Cfg::kHalfBytes, &tmv, hf * 64, y, &ps.full[st], pol);
+        }
+      }
+    });
+  } else {
+    // ---- consumers ----
+    // Q as MMA A fragments: a0 = row r, dims (kk*16 + 2c, +1); a2 = dims +8.
+    uint32_t qa[D / 16][2];
+    {
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                               (static_cast<int64_t>(s) * a.hq + hq0 + r) * D);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        qa[kk][0] = r < G ? __ldg(qrow + kk * 8 + c) : 0u;
+        qa[kk][1] = r < G ? __ldg(qrow + kk * 8 + 4 + c) : 0u;
+      }
+    }
+    // per-lane ldmatrix rows: K matrices (tok0, d0), (tok0, d0+8), (tok0+8, d0), (tok0+8, d0+8);
+    // V matrices (tok0, d0), (tok0+8, d0), (tok0, d0+8), (tok0+8, d0+8)
+    const int mk = lane >> 3, ik = lane & 7;
+    const int tokK = warp * 16 + (mk >> 1) * 8 + ik;
+    const int dK = (mk & 1) * 8;
+    const int tokV = warp * 16 + (mk & 1) * 8 + ik;
+    const int dV = (mk >> 1) * 8;
+
+    for (int i = 0; i < nchunks; ++i) {
+      const int st = i % S;
+      if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
+      const int nv = min(16, min(C, pt.ntok - i * C) - warp * 16);  // warp-uniform
+      if (nv > 0) {
+        const uint32_t kst = sbase + st * Cfg::kStageBytes;
+        const uint32_t vst = kst + Cfg::kTileBytes;
+        float sacc[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int d0 = kk * 16 + dK;
+          const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tokK * 128 + ((((d0 & 63) >> 3) ^ (tokK & 7)) << 4);
+          uint32_t b00, b01, b10, b11;
+          ldsm_x4(addr, b00, b01, b10, b11);
+          mma_rows8(sacc[0], qa[kk][0], qa[kk][1], b00, b01);
+          mma_rows8(sacc[1], qa[kk][0], qa[kk][1], b10, b11);
+        }
+        // scores of row r, tokens nt*8 + 2c + j
+        float sc[2][2];
+        float mloc = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int t = nt * 8 + 2 * c + j;
+            sc[nt][j] = t < nv ? sacc[nt][j] * a.scale_log2 : -INFINITY;
+            mloc = fmaxf(mloc, sc[nt][j]);
+          }
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+        const float mn = fmaxf(m_run, mloc);
+        const float alpha = exp2f(m_run - mn);
+        m_run = mn;
+        float pr[2][2];
+        float psum = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            pr[nt][j] = exp2f(sc[nt][j] - mn);
+            psum += pr[nt][j];
+          }
+        l_run = l_run * alpha + psum;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          o[j][0] *= alpha;
+          o[j][1] *= alpha;
+        }
+        uint32_t ph0, pl0, ph2, pl2;
+        split_pair(pr[0][0], pr[0][1], ph0, pl0);
+        split_pair(pr[1][0], pr[1][1], ph2, pl2);
+        // V rows of tokens >= nv are zeroed (they may be padding)
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+        if (nv < 16) {
+          mlo = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
+          mhi = (2 * c + 8 < nv ? 0x0000ffffu : 0u) | (2 * c + 9 < nv ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int dg = 0; dg < D / 16; ++dg) {
+          const int d0 = dg * 16 + dV;
+          const uint32_t addr = vst + (d0 >> 6) * Cfg::kHalfBytes + tokV * 128 + ((((d0 & 63) >> 3) ^ (tokV & 7)) << 4);
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_t(addr, v0, v1, v2, v3);
+          v0 &= mlo;
+          v1 &= mhi;
+          v2 &= mlo;
+          v3 &= mhi;
+          mma_rows8(o[2 * dg], ph0, ph2, v0, v1);
+          mma_rows8(o[2 * dg], pl0, pl2, v0, v1);
+          mma_rows8(o[2 * dg + 1], ph0, ph2, v2, v3);
+          mma_rows8(o[2 * dg + 1], pl0, pl2, v2, v3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ps.empty[st]);
+    }
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  }
+
+  __syncthreads();  // every copy consumed; the stage ring is free
+  if (ps.abort_flag) return;
+
+  float* wm = reinterpret_cast<float*>(sgen);
+  float* wl = wm + NW * G;
+  float* wacc = wl + NW * G;
+  if (warp < NW && r < G) {
+    if (c == 0) {
+      wm[warp * G + r] = m_run;
+      wl[warp * G + r] = l_run;
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      wacc[(warp * G + r) * D + j * 8 + 2 * c] = o[j][0];
+      wacc[(warp * G + r) * D + j * 8 + 2 * c + 1] = o[j][1];
+    }
+  }
+  __syncthreads();
+  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, tid, Cfg::kThreads);
+}
+
+}  // namespace pa
