@@ -351,18 +351,16 @@ def run_ours(args, rank, world, device):
 
 
 def run_e2e(args, d, device, world, P):
-    """K steps through PagedKVCache.step: per step, H2D of q/k/v from pinned host
-    memory (plus the slots, CoW pairs, tables and lengths the API uploads),
-    append + decode, D2H of the fp32 output. Context lengths grow by one per step."""
+    """K steps through PagedKVCache.step_host (the native pa_step_host): per
+    step the block manager appends, the step metadata and q/k/v go host ->
+    device from pinned memory, copy-on-write + append + decode run, and the fp32
+    output comes back to pinned host memory. Context lengths grow by one per step."""
     sh = d["shape"]
     cache = d["cache"]
     ids = d["ids"]
-    hq = torch.empty(d["q"].shape, dtype=d["q"].dtype, pin_memory=True)
-    hk = torch.empty(d["k"].shape, dtype=d["k"].dtype, pin_memory=True)
-    hv = torch.empty(d["v"].shape, dtype=d["v"].dtype, pin_memory=True)
-    hq.copy_(d["q"].cpu())
-    hk.copy_(d["k"].cpu())
-    hv.copy_(d["v"].cpu())
+    hq = d["q"].cpu().pin_memory()
+    hk = d["k"].cpu().pin_memory()
+    hv = d["v"].cpu().pin_memory()
     hout = torch.empty(d["out"].shape, dtype=torch.float32, pin_memory=True)
     eb = hq.element_size()
     kv_total = h2d = d2h = 0
@@ -375,16 +373,11 @@ def run_e2e(args, d, device, world, P):
                 torch.distributed.barrier()
             t0.record()
             kv_total = h2d = d2h = 0
-        q = hq.to(device, non_blocking=True)
-        k = hk.to(device, non_blocking=True)
-        v = hv.to(device, non_blocking=True)
-        out = cache.step(ids, q, k, v, d["scale"], partition_tokens=P)
-        hout.copy_(out, non_blocking=True)
-        torch.cuda.current_stream(device).synchronize()
+        cache.step_host(ids, hq, hk, hv, hout, d["scale"], partition_tokens=P)
         L = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64, count=len(ids))
         kv_total += int(L.sum()) * sh.num_kv_heads * sh.head_dim * 2 * eb
         nblk = int(-(-L.max() // sh.block_size))
-        h2d += (hq.numel() + hk.numel() + hv.numel()) * eb + len(ids) * (8 + 4 + nblk * 4)
+        h2d += (hq.numel() + hk.numel() + hv.numel()) * eb + len(ids) * (8 + 8 + nblk * 4 + 4)
         d2h += hout.numel() * 4
     t1.record()
     torch.cuda.synchronize(device)
@@ -399,8 +392,8 @@ def run_e2e(args, d, device, world, P):
     return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "ms_per_step": round(ms / args.steps, 4),
             "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
-            "api": "PagedKVCache.step (pa_bm_append_slots, pa_copy_blocks, pa_reshape_and_cache, "
-                   "pa_bm_block_tables, pa_decode)"}
+            "api": "pa_step_host via PagedKVCache.step_host (block manager, one metadata H2D, q/k/v H2D, "
+                   "pa_copy_blocks, pa_reshape_and_cache, pa_decode, output D2H, stream sync)"}
 
 
 def run_reference(args, rank, world):

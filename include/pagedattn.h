@@ -57,6 +57,8 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
 
 typedef void* pa_stream; /* cudaStream_t */
 
+typedef struct pa_bm pa_bm; /* host block manager handle (see below) */
+
 /* A paged KV cache in device memory (see the layout above). */
 typedef struct {
   void* k;               /* device, [num_blocks][num_kv_heads][block_size][head_dim] */
@@ -190,6 +192,42 @@ pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t nu
                                      int32_t partition_tokens, pa_stream stream);
 
 /*
+ * One whole decode step from host memory: the call a serving loop makes per
+ * generated token. P2 §3.2.2 steps 1-4 in order: for each listed sequence the
+ * block manager assigns the new token's slot (new block or copy-on-write as
+ * in pa_bm_append_slots); the CoW pairs, slots, block tables and lengths are
+ * staged in pinned host memory and sent in one copy; q, k, v are copied from
+ * the caller's host buffers; pa_copy_blocks, pa_reshape_and_cache and
+ * pa_decode run on `stream`; the fp32 output is copied back to out_host; the
+ * call returns after the stream has finished (so out_host is ready).
+ *
+ *   bm, cache       the sequences' manager and cache (same block_size).
+ *   seq_ids         host int64 [n]: sequences appending one token each.
+ *   q_host          host [n][num_q_heads][head_dim], cache dtype.
+ *   k_host, v_host  host [n][num_kv_heads][head_dim], cache dtype.
+ *   out_host        host fp32 [n][num_q_heads][head_dim].
+ *   partition_tokens as for pa_decode.
+ *   dev_staging     device, >= *dev_bytes of pa_step_staging_bytes, 256-byte aligned.
+ *   host_staging    pinned host, >= *host_bytes of pa_step_staging_bytes.
+ * Host buffers should be pinned for asynchronous copies (pageable memory works
+ * but is copied synchronously by the driver). seq_ids must be distinct. The
+ * staging sizes are checked against the lengths the step produces before
+ * anything changes: too-small staging (PA_ERR_INVALID_ARG) or a block-manager
+ * failure (PA_ERR_NO_FREE_BLOCKS, PA_ERR_UNKNOWN_SEQ) leaves the manager
+ * unchanged and launches nothing. The staging buffers are reused by the next
+ * call; the call returns only after the stream has drained.
+ */
+pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, const int64_t* seq_ids, int32_t num_q_heads,
+                       const void* q_host, const void* k_host, const void* v_host, float scale, float* out_host,
+                       int32_t partition_tokens, void* dev_staging, size_t dev_staging_bytes, void* host_staging,
+                       size_t host_staging_bytes, pa_stream stream);
+
+/* Staging sizes pa_step_host needs for up to n sequences whose lengths stay
+ * at most max_context_len after the step. */
+pa_status pa_step_staging_bytes(int32_t n, int32_t num_q_heads, const pa_cache* cache, int32_t max_context_len,
+                                int32_t partition_tokens, size_t* dev_bytes, size_t* host_bytes);
+
+/*
  * Self-test of the device wait limit. Every pipelined kernel waits for its own
  * copies with a bounded wait; this launches one thread that waits on a barrier
  * nothing completes. After timeout_ns (1 .. 10^10) it records
@@ -210,8 +248,6 @@ pa_status pa_selftest_wait_timeout(int64_t timeout_ns, pa_stream stream);
  * zero is appended at the back, in the order of the freed sequence's table.
  * Sequences are identified by caller-chosen int64 ids.
  */
-typedef struct pa_bm pa_bm;
-
 /* free_order: host int32 [num_blocks], a permutation of 0..num_blocks-1 giving
  * the initial free-list order, or NULL for 0, 1, 2, ... */
 pa_status pa_bm_create(int64_t num_blocks, int32_t block_size, const int32_t* free_order, pa_bm** out);

@@ -49,6 +49,8 @@ _SIGS = {
     "pa_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_get_device_error": (_I32, [_VP, _P64]),
     "pa_selftest_wait_timeout": (_I32, [_I64, _VP]),
+    "pa_step_host": (_I32, [_VP, _PCACHE, _I32, _VP, _I32, _VP, _VP, _VP, _F, _VP, _I32, _VP, _SZ, _VP, _SZ, _VP]),
+    "pa_step_staging_bytes": (_I32, [_I32, _I32, _PCACHE, _I32, _I32, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
     "pa_decode_static_workspace": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP]),
     "pa_bm_create": (_I32, [_I64, _I32, _VP, ctypes.POINTER(_VP)]),
     "pa_bm_destroy": (None, [_VP]),
@@ -197,6 +199,42 @@ def pa_decode_static_workspace(q, k_cache, v_cache, block_tables, context_lens, 
                                              int(max_context_len), float(scale), out.data_ptr(),
                                              int(partition_tokens), _stream(q, stream)),
            "pa_decode_static_workspace")
+
+
+def pa_step_staging_bytes(num_seqs, num_q_heads, k_cache, v_cache, max_context_len, partition_tokens=-1):
+    """(device bytes, pinned host bytes) that pa_step_host needs."""
+    c = make_cache(k_cache, v_cache)
+    db, hb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib().pa_step_staging_bytes(num_seqs, num_q_heads, ctypes.byref(c), max_context_len, partition_tokens,
+                                        ctypes.byref(db), ctypes.byref(hb)), "pa_step_staging_bytes")
+    return int(db.value), int(hb.value)
+
+
+def _host(t, name, dtype, shape):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != dtype or tuple(t.shape) != tuple(shape) \
+            or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host {dtype} tensor of shape {tuple(shape)}")
+    return t.data_ptr()
+
+
+def pa_step_host(bm: "BlockManager", k_cache, v_cache, seq_ids, q_host, k_host, v_host, scale, out_host,
+                 dev_staging, host_staging, partition_tokens=-1, stream=None):
+    """One decode step from host buffers (see pagedattn.h); returns after the stream drained."""
+    c = make_cache(k_cache, v_cache)
+    ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+    n, hq, d = q_host.shape
+    _host(q_host, "q_host", k_cache.dtype, (len(ids), hq, c.head_dim))
+    _host(k_host, "k_host", k_cache.dtype, (len(ids), c.num_kv_heads, c.head_dim))
+    _host(v_host, "v_host", k_cache.dtype, (len(ids), c.num_kv_heads, c.head_dim))
+    _host(out_host, "out_host", torch.float32, (len(ids), hq, c.head_dim))
+    _dev(dev_staging, "dev_staging")
+    if host_staging.is_cuda or not host_staging.is_contiguous():
+        raise ValueError("host_staging must be contiguous host memory")
+    _check(_lib().pa_step_host(bm._h, ctypes.byref(c), len(ids), _i64p(ids), hq, q_host.data_ptr(), k_host.data_ptr(),
+                               v_host.data_ptr(), float(scale), out_host.data_ptr(), int(partition_tokens),
+                               dev_staging.data_ptr(), dev_staging.numel() * dev_staging.element_size(),
+                               host_staging.data_ptr(), host_staging.numel() * host_staging.element_size(),
+                               _stream(k_cache, stream)), "pa_step_host")
 
 
 def pa_selftest_wait_timeout(timeout_ns: int, stream=None):

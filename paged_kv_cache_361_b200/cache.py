@@ -55,6 +55,8 @@ class PagedKVCache:
         self._tables = _Staging(np.int32, torch.int32, self.device)
         self._lens = _Staging(np.int32, torch.int32, self.device)
         self._ws = None
+        self._dev_staging = None
+        self._host_staging = None
 
     # -- host bookkeeping + writes -------------------------------------------
     def add_sequence(self, seq_id: int, k: torch.Tensor, v: torch.Tensor) -> np.ndarray:
@@ -121,6 +123,25 @@ class PagedKVCache:
         B.pa_decode(q, self.k_cache, self.v_cache, self._tables.upload(tables), self._lens.upload(lens), scale, out,
                     max_len, partition_tokens, self.workspace(nbytes))
         return out
+
+    def step_host(self, seq_ids, q_host, k_host, v_host, out_host, scale=None, partition_tokens=-1):
+        """One decode step from host tensors (pinned for asynchronous copies):
+        block-manager work, copies and kernels in one native call
+        (pa_step_host); returns when out_host holds the fp32 result."""
+        n, hq, d = q_host.shape
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        max_len = max(self.lens[s] for s in seq_ids) + 1
+        dev_b, host_b = B.pa_step_staging_bytes(n, hq, self.k_cache, self.v_cache, max_len, partition_tokens)
+        if self._dev_staging is None or self._dev_staging.numel() < dev_b:
+            self._dev_staging = torch.empty(dev_b * 5 // 4 + 4096, dtype=torch.uint8, device=self.device)
+        if self._host_staging is None or self._host_staging.numel() < host_b:
+            self._host_staging = torch.empty(host_b * 5 // 4 + 4096, dtype=torch.uint8, pin_memory=True)
+        B.pa_step_host(self.bm, self.k_cache, self.v_cache, seq_ids, q_host, k_host, v_host, scale, out_host,
+                       self._dev_staging, self._host_staging, partition_tokens)
+        for s in seq_ids:
+            self.lens[s] += 1
+        return out_host
 
     def step(self, seq_ids, q, k, v, scale=None, out=None, partition_tokens=-1):
         """One decode step: append each sequence's new K/V, then attend."""

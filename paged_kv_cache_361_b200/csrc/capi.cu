@@ -30,16 +30,27 @@ pa_status check_cache(const pa_cache* c) {
 
 pa_status launched() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
 
+// Partition size for partition_tokens = -1. Measured on a B200 with the
+// decode kernels here: unsplit CTAs win while there are enough (sequence, kv
+// head) units to fill the GPU and no unit is long; long units are cut into
+// 1024 tokens (many units) or 2048 tokens (fewer units) to balance the SMs;
+// with very few units the sequences are cut so that about 600 CTAs exist.
 int32_t resolve_partition(int32_t num_seqs, int32_t hkv, int32_t max_ctx, int32_t bs, int32_t requested) {
   if (requested >= 0) return requested;
-  (void)num_seqs;
-  (void)hkv;
-  // Split long sequences into 512-token partitions: equal-sized work items
-  // balance the SMs when lengths differ, and long contexts get parallelism.
-  if (max_ctx <= 1024) return 0;
-  int32_t p = 512;
-  if (p % bs) p = bs;  // unreachable for bs <= 32; kept for clarity of the rule
-  return p;
+  const int64_t units = static_cast<int64_t>(num_seqs) * hkv;
+  int64_t P;
+  if (units >= 256 && max_ctx <= 2560) return 0;
+  if (units >= 1024) {
+    P = 1024;
+  } else if (units >= 256) {
+    P = 2048;
+  } else {
+    const int64_t parts = (600 + units - 1) / (units > 0 ? units : 1);
+    P = (max_ctx + parts - 1) / parts;
+    P = P < 512 ? 512 : (P > 2048 ? 2048 : P);
+  }
+  P = (P + bs - 1) / bs * bs;
+  return P >= max_ctx ? 0 : static_cast<int32_t>(P);
 }
 
 int32_t num_parts(int32_t max_ctx, int32_t P) {
@@ -148,7 +159,7 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
 template <int D>
 pa_status launch_reduce(const DecodeArgs& a, cudaStream_t st) {
   dim3 grid(a.hq, a.num_seqs);
-  decode_reduce_kernel<D><<<grid, D, 0, st>>>(a);
+  decode_reduce_kernel<D><<<grid, 32 * kReduceWarps, 0, st>>>(a);
   return launched();
 }
 

@@ -177,11 +177,17 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const
 
 // Merge the partitions of one (sequence, query head):
 //   M = max_p m_p,  out = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).
-// Grid (hq, num_seqs), D threads. Sequences with one partition were written
+// Grid (hq, num_seqs), 8 warps: warp w folds partitions w, w+8, ... with each
+// lane owning D/32 dims (one coalesced row read per partition), then the warps
+// are folded through shared memory. Sequences with one partition were written
 // by the decode kernel and are skipped.
+constexpr int kReduceWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
-  const int hq = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(32 * kReduceWarps) decode_reduce_kernel(const DecodeArgs a) {
+  constexpr int VEC = D / 32;
+  const int hq = blockIdx.x, s = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int32_t L = load_len(a, s, false);
   const int32_t P = a.part_tokens;
   const int32_t nparts = (L + P - 1) / P;
@@ -189,15 +195,50 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
   const int64_t row = static_cast<int64_t>(s) * a.hq + hq;
   const float* ml = a.ws_ml + row * a.max_parts * 2;
   const float* o = a.ws_o + row * a.max_parts * D;
+  __shared__ float red[kReduceWarps];
+  __shared__ float wl[kReduceWarps];
+  __shared__ float wo[kReduceWarps][D];
+
   float M = -INFINITY;
-  for (int q = 0; q < nparts; ++q) M = fmaxf(M, ml[2 * q]);
-  float l = 0.f, acc = 0.f;
-  for (int q = 0; q < nparts; ++q) {
+  for (int q = tid; q < nparts; q += 32 * kReduceWarps) M = fmaxf(M, ml[2 * q]);
+  M = warp_max(M);
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, red[w]);
+
+  float l = 0.f, acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  for (int q = warp; q < nparts; q += kReduceWarps) {
     const float f = exp2f(ml[2 * q] - M);
     l = fmaf(ml[2 * q + 1], f, l);
-    acc = fmaf(o[static_cast<int64_t>(q) * D + d], f, acc);
+    const float* src = o + static_cast<int64_t>(q) * D + lane * VEC;
+    if (VEC == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(src);
+      acc[0] = fmaf(x.x, f, acc[0]);
+      acc[1] = fmaf(x.y, f, acc[1]);
+      acc[2] = fmaf(x.z, f, acc[2]);
+      acc[3] = fmaf(x.w, f, acc[3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] = fmaf(src[e], f, acc[e]);
+    }
   }
-  a.out[row * D + d] = acc / l;
+  if (lane == 0) wl[warp] = l;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) wo[warp][lane * VEC + e] = acc[e];
+  __syncthreads();
+  for (int d = tid; d < D; d += 32 * kReduceWarps) {
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w) {
+      num += wo[w][d];
+      den += wl[w];
+    }
+    a.out[row * D + d] = num / den;
+  }
 }
 
 }  // namespace pa

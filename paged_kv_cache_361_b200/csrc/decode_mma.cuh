@@ -53,13 +53,16 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
-// d += A(16x16, rows 8..15 zero) * B(16x8), bf16 in, fp32 accumulate.
-__device__ __forceinline__ void mma_rows8(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+// d += A(16x16, rows 8..15 zero) * B(16x8), bf16 in, fp32 accumulate. Only
+// rows 0..7 of the accumulator are kept: rows 8..15 are fed zeros and their
+// results are discarded, so they hold no registers across the loop.
+__device__ __forceinline__ void mma_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  float j2, j3;
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+      "{%10, %11, %12, %12};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(j2), "=f"(j3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -114,9 +117,9 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const _
   if (tid == 0) pipe_init<S>(ps, NW);
   __syncthreads();
 
-  float o[NT][4];
+  float o[NT][2];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
 
   if (warp == NW) {
@@ -175,9 +178,9 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const _
       if (nv > 0) {
         const uint32_t kst = sbase + st * Cfg::kStageBytes;
         const uint32_t vst = kst + Cfg::kTileBytes;
-        float sacc[2][4];
+        float sacc[2][2];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+        for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int d0 = kk * 16 + dK;

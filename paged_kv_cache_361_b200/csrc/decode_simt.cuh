@@ -102,7 +102,7 @@ struct SimtCfg {
   static constexpr int kRPW = 32 / kLPR;                       // rows per warp load
   static constexpr int kNV = kTokPerWarp / kRPW;               // token partials per lane
   static constexpr int kStageBytes = 2 * kChunk * D * Elem<T>::bytes;
-  static constexpr int kStages = kStageBytes <= 16384 ? 4 : (kStageBytes <= 32768 ? 3 : 2);
+  static constexpr int kStages = kStageBytes <= 16384 ? 4 : 2;  // 2 x 32 KB at D 128 bf16: 3 CTAs per SM
   static constexpr int kSmemBytes = kStages * kStageBytes;
   static_assert(kNV <= kLPR, "butterfly needs at least as many lanes as values");
 };

@@ -146,3 +146,52 @@ def test_wait_limit_returns_status():
     assert st == B.PA_ERR_DEVICE_TIMEOUT
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum()) == 8.0
+
+
+def test_step_host_matches_oracle_with_cow():
+    """pa_step_host (host buffers in, host buffer out) on a prefix-sharing batch:
+    the first step copies the shared partial block; slots, pairs and outputs match
+    the oracle."""
+    from oracle.replay import OracleRun
+    sh = W.Shape(16, 4, 128, 16, "bf16")
+    g = torch.Generator().manual_seed(3)
+    ref = OracleRun(sh, 64, list(range(64)), keep_pool=True)
+    cache = PagedKVCache(64, 4, 16, 128, torch.bfloat16, "cuda", list(range(64)), fill=float("nan"))
+    pk, pv = torch.randn(37, 4, 128, generator=g).bfloat16(), torch.randn(37, 4, 128, generator=g).bfloat16()
+    add = ("add", 0, 37, lambda which, device="cpu": pk if which == "k" else pv)
+    ref.apply(add)
+    cache.add_sequence(0, pk.cuda(), pv.cuda())
+    for child in (1, 2):
+        ref.apply(("fork", 0, child))
+        cache.fork(0, child)
+    ids = [2, 0, 1]
+    for step in range(3):
+        q = torch.randn(3, 16, 128, generator=g).bfloat16().pin_memory()
+        k = torch.randn(3, 4, 128, generator=g).bfloat16().pin_memory()
+        v = torch.randn(3, 4, 128, generator=g).bfloat16().pin_memory()
+        out = torch.empty(3, 16, 128, dtype=torch.float32).pin_memory()
+        rec = ref.apply(("append", ids, lambda which, device="cpu", k=k, v=v: k if which == "k" else v))
+        cache.step_host(ids, q, k, v, out, 128 ** -0.5, partition_tokens=16 if step == 1 else -1)
+        if step == 0:
+            assert len(rec["pairs"]) == 2
+        for i, s in enumerate(ids):
+            exp = ref.attend(s, q[i], 128 ** -0.5, use_pool=True)
+            assert float(np.abs(out[i].double().numpy() - exp).max()) <= TOL["bf16"]
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    for s in ids:
+        assert cache.bm.block_table(s)[0].tolist() == ref.bm.block_table(s)
+
+
+def test_step_host_rejects_small_staging_without_change():
+    cache = PagedKVCache(8, 1, 16, 64, torch.bfloat16, "cuda")
+    cache.add_sequence(0, torch.zeros(3, 1, 64, dtype=torch.bfloat16, device="cuda"),
+                       torch.zeros(3, 1, 64, dtype=torch.bfloat16, device="cuda"))
+    q = torch.zeros(1, 1, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 1, 64, dtype=torch.bfloat16)
+    out = torch.empty(1, 1, 64)
+    tiny_dev = torch.empty(256, dtype=torch.uint8, device="cuda")
+    tiny_host = torch.empty(256, dtype=torch.uint8)
+    with pytest.raises(B.PagedAttnError) as e:
+        B.pa_step_host(cache.bm, cache.k_cache, cache.v_cache, [0], q, k, k, 0.1, out, tiny_dev, tiny_host)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
+    assert cache.bm.block_table(0)[1] == 3
