@@ -113,6 +113,27 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot
 pa_status pa_copy_blocks(const pa_cache* cache, const int32_t* src_dst_pairs, int32_t n_pairs, pa_stream stream);
 
 /*
+ * Swap whole blocks between the device pool and a host pool (P2 §五 page
+ * replacement: inactive blocks move to CPU memory when the GPU runs short;
+ * P2 §八 GPU/CPU tiers).
+ *
+ *   host_k, host_v   host pools [host_num_blocks][num_kv_heads][block_size]
+ *                    [head_dim] in the cache dtype, in pinned memory mapped
+ *                    into the device's address space (cudaHostAlloc, or
+ *                    cudaHostRegister with mapping); anything else returns
+ *                    PA_ERR_INVALID_ARG before launch.
+ *   pairs            device int32 [n_pairs][2]: {device block, host block} when
+ *                    to_host != 0 (swap out), {host block, device block}
+ *                    otherwise (swap in), as pa_bm_swap_out / pa_bm_swap_in
+ *                    emit them. Ids out of range skip the pair and are recorded
+ *                    as PA_ERR_DEVICE_BOUNDS.
+ * One kernel moves every pair (no per-block copy calls). Run it before any
+ * later write reuses the released blocks, on the same stream.
+ */
+pa_status pa_swap_blocks(const pa_cache* cache, void* host_k, void* host_v, int64_t host_num_blocks,
+                         const int32_t* pairs, int32_t n_pairs, int32_t to_host, pa_stream stream);
+
+/*
  * Single-query decode attention over the paged cache.
  * P2 §1.1: out = softmax(scale * q K^T) V, one query row per head; P2 §3.2.2
  * step 4 and §4.1: every logical block of the sequence is visited through its
@@ -135,9 +156,11 @@ pa_status pa_copy_blocks(const pa_cache* cache, const int32_t* src_dst_pairs, in
  *                      separately; a second kernel merges them with a
  *                      log-sum-exp reduction.
  *                      -1: chosen by the library (pa_decode_partition_tokens).
- *   workspace          device, >= pa_decode_workspace_bytes(...) bytes when
- *                      the sequences are split, else may be NULL. Scratch for
- *                      the partial results; its contents need no initial value.
+ *   workspace          device, >= pa_decode_workspace_bytes(...) bytes,
+ *                      256-byte aligned. Always needed: it holds the work
+ *                      counters of the persistent kernels (cleared by the call
+ *                      itself) and, when sequences are split, the partial
+ *                      results. Its contents need no initial value.
  * Accumulation is fp32. Calls sharing a workspace must not overlap on the GPU.
  */
 pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
@@ -150,8 +173,9 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t max_context_len, int32_t block_size);
 
-/* Workspace bytes pa_decode needs for these sizes (0 when nothing is split).
- * partition_tokens may be -1 (resolved as pa_decode would). */
+/* Workspace bytes pa_decode needs for these sizes (a few hundred bytes of
+ * counters, plus the partials when sequences are split). partition_tokens may
+ * be -1 (resolved as pa_decode would). */
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                  int32_t max_context_len, int32_t block_size, int32_t partition_tokens);
 
@@ -258,6 +282,46 @@ void pa_bm_destroy(pa_bm* bm);
  * may be NULL) receives the slot of each token. */
 pa_status pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int32_t num_tokens, int64_t* slots_out);
 
+/* Prefill with prefix reuse (P2 §3.4 prefix block pool; P3: cached system
+ * prompts shared across requests). tokens: host int32 [num_tokens], the
+ * prompt's token ids. Whole prompt blocks are matched, from block 0 on, against
+ * a prefix cache keyed by the full token prefix up to each block's end; hits
+ * map onto the cached blocks (one more reference each) and the rest are new
+ * blocks, whose whole ones are added to the cache. slots_out (host int64
+ * [num_tokens], may be NULL) gets -1 for the *n_cached_out leading tokens
+ * already in the pool (pa_reshape_and_cache skips them) and the slot of every
+ * other token. The cache holds one reference per listed block; a listed block
+ * that only the cache holds is evictable, and any allocation of this manager
+ * takes the least recently released evictable block when the free list is
+ * empty. Keys are 64-bit hash chains whose block tokens and parent are checked
+ * on a hit, so a false hit needs a 64-bit collision of two different prefixes. */
+pa_status pa_bm_add_seq_cached(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int32_t num_tokens,
+                               int64_t* slots_out, int32_t* n_cached_out);
+
+/* Host blocks available for swapping (P2 §五): ids 0..num_host_blocks-1 on a
+ * FIFO free list. Fails (PA_ERR_INVALID_ARG) while a sequence is swapped out. */
+pa_status pa_bm_set_host_blocks(pa_bm* bm, int64_t num_host_blocks);
+
+/* Swap a live sequence out: each block of its table gets a host block and
+ * releases one device reference (a block shared with a live sequence stays).
+ * pairs_out (host int32 [cap][2]) gets {device, host} per logical block, in
+ * order; *n_pairs_out the count. Apply with pa_swap_blocks(to_host = 1)
+ * before the released device blocks are written again. The sequence keeps its
+ * length but cannot append or decode until swapped in. All or nothing. */
+pa_status pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int32_t* pairs_out, int32_t cap, int32_t* n_pairs_out);
+
+/* Swap a sequence back in: fresh device blocks (private, from the free list
+ * or by eviction of cached blocks), pairs {host, device} in table order, host
+ * blocks returned to their free list. Apply with pa_swap_blocks(to_host = 0)
+ * before decoding it. All or nothing. pa_bm_free_seq on a swapped-out
+ * sequence releases its host blocks. */
+pa_status pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int32_t* pairs_out, int32_t cap, int32_t* n_pairs_out);
+
+/* Prefix-cache counters: listed blocks, evictable ones among them, and the
+ * prompt tokens served from the cache so far. */
+pa_status pa_bm_prefix_stats(const pa_bm* bm, int64_t* cached_blocks, int64_t* evictable_blocks,
+                             int64_t* hit_tokens);
+
 /* Share (P1 "跨请求的内存共享"; P2 §3.4): `child` gets a copy of `parent`'s
  * table and every block in it gains one reference. */
 pa_status pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child);
@@ -293,9 +357,11 @@ pa_status pa_bm_block_tables(const pa_bm* bm, int32_t n, const int64_t* seq_ids,
 
 pa_status pa_bm_refcount(const pa_bm* bm, int32_t block, int32_t* out);
 
-/* free_blocks: blocks on the free list; allocated_slots: block_size times the
- * blocks in use; used_slots: slots holding a token (a shared block counts
- * once). allocated - used is the internal waste (P1 "内存浪费的两种形式"). */
+/* free_blocks: blocks on the free list (evictable cached blocks are not
+ * counted); allocated_slots: block_size times the blocks not on the free
+ * list; used_slots: slots holding a token of a live sequence (a shared block
+ * counts once). allocated - used is the internal waste (P1 "内存浪费的两种形式")
+ * plus the slots of evictable cached blocks. */
 pa_status pa_bm_stats(const pa_bm* bm, int64_t* free_blocks, int64_t* used_slots, int64_t* allocated_slots);
 
 /* The free list in order: up to cap ids into out, the length into *n_out. */

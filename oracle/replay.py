@@ -14,14 +14,14 @@ from __future__ import annotations
 import torch
 
 from .attention import decode_attention, split_decode_attention
-from .block_manager import BlockManagerModel
+from .prefix_cache import PrefixCachingModel
 from . import paged
 
 
 class OracleRun:
     def __init__(self, shape, num_blocks: int, free_order, keep_pool: bool = True, pool_fill=float("nan")):
         self.shape = shape
-        self.bm = BlockManagerModel(num_blocks, shape.block_size, free_order)
+        self.bm = PrefixCachingModel(num_blocks, shape.block_size, free_order)
         self.hist = {"k": {}, "v": {}}
         dt = {"f32": torch.float32, "bf16": torch.bfloat16}[shape.dtype]
         self.pool = None
@@ -53,6 +53,15 @@ class OracleRun:
                 if self.pool is not None:
                     paged.scatter(self.pool[w], rows[w], slots)
             rec.update(seq=seq, slots=slots)
+        elif kind == "add_cached":
+            _, seq, tokens, src = op
+            slots, n_cached = self.bm.add_seq_cached(seq, tokens)
+            rows = {w: src(w) for w in "kv"}
+            for w in "kv":
+                self.hist[w][seq] = [rows[w]] if len(tokens) else []
+                if self.pool is not None:
+                    paged.scatter(self.pool[w], rows[w], slots)   # -1 (cached) rows are skipped
+            rec.update(seq=seq, slots=slots, n_cached=n_cached)
         elif kind == "fork":
             _, parent, child = op
             self.bm.fork(parent, child)

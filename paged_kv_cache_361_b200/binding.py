@@ -56,6 +56,12 @@ _SIGS = {
     "pa_bm_destroy": (None, [_VP]),
     "pa_bm_add_seq": (_I32, [_VP, _I64, _I32, _VP]),
     "pa_bm_fork": (_I32, [_VP, _I64, _I64]),
+    "pa_bm_add_seq_cached": (_I32, [_VP, _I64, _VP, _I32, _VP, _P32]),
+    "pa_bm_set_host_blocks": (_I32, [_VP, _I64]),
+    "pa_bm_swap_out": (_I32, [_VP, _I64, _VP, _I32, _P32]),
+    "pa_bm_swap_in": (_I32, [_VP, _I64, _VP, _I32, _P32]),
+    "pa_swap_blocks": (_I32, [_PCACHE, _VP, _VP, _I64, _VP, _I32, _I32, _VP]),
+    "pa_bm_prefix_stats": (_I32, [_VP, _P64, _P64, _P64]),
     "pa_bm_append_slot": (_I32, [_VP, _I64, _P64, _P32]),
     "pa_bm_append_slots": (_I32, [_VP, _I32, _VP, _VP, _VP, _P32]),
     "pa_bm_free_seq": (_I32, [_VP, _I64]),
@@ -237,6 +243,19 @@ def pa_step_host(bm: "BlockManager", k_cache, v_cache, seq_ids, q_host, k_host, 
                                _stream(k_cache, stream)), "pa_step_host")
 
 
+def pa_swap_blocks(k_cache, v_cache, host_k, host_v, pairs, to_host: bool, stream=None):
+    """Move whole blocks between the device pool and a pinned host pool."""
+    c = make_cache(k_cache, v_cache)
+    if host_k.is_cuda or host_v.is_cuda or host_k.shape != host_v.shape or host_k.shape[1:] != k_cache.shape[1:] \
+            or host_k.dtype != k_cache.dtype or not host_k.is_contiguous() or not host_v.is_contiguous():
+        raise ValueError("host pools must be contiguous host tensors shaped like the cache (pinned)")
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [n][2]")
+    _check(_lib().pa_swap_blocks(ctypes.byref(c), host_k.data_ptr(), host_v.data_ptr(), int(host_k.shape[0]),
+                                 _dev(pairs, "pairs", torch.int32), int(pairs.shape[0]), 1 if to_host else 0,
+                                 _stream(k_cache, stream)), "pa_swap_blocks")
+
+
 def pa_selftest_wait_timeout(timeout_ns: int, stream=None):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -282,6 +301,39 @@ class BlockManager:
 
     def fork(self, parent: int, child: int):
         _check(_lib().pa_bm_fork(self._h, parent, child), "pa_bm_fork")
+
+    def add_seq_cached(self, seq_id: int, tokens):
+        """Prefill with prefix reuse: (slots with -1 for cached tokens, n_cached)."""
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        slots = np.empty(len(tok), dtype=np.int64)
+        nc = ctypes.c_int32(0)
+        _check(_lib().pa_bm_add_seq_cached(self._h, seq_id, _i64p(tok), len(tok), _i64p(slots), ctypes.byref(nc)),
+               "pa_bm_add_seq_cached")
+        return slots, int(nc.value)
+
+    def set_host_blocks(self, n: int):
+        _check(_lib().pa_bm_set_host_blocks(self._h, n), "pa_bm_set_host_blocks")
+
+    def _swap(self, fn, seq_id):
+        cap = max(1, self.num_blocks)
+        n = ctypes.c_int32(0)
+        out = np.empty((cap, 2), dtype=np.int32)
+        _check(fn(self._h, seq_id, _i64p(out), cap, ctypes.byref(n)), fn.__name__)
+        return out[:n.value].copy()
+
+    def swap_out(self, seq_id: int) -> np.ndarray:
+        """{device, host} pairs of the sequence's blocks."""
+        return self._swap(_lib().pa_bm_swap_out, seq_id)
+
+    def swap_in(self, seq_id: int) -> np.ndarray:
+        """{host, device} pairs of the sequence's blocks."""
+        return self._swap(_lib().pa_bm_swap_in, seq_id)
+
+    def prefix_stats(self) -> dict:
+        c, e, h = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(_lib().pa_bm_prefix_stats(self._h, ctypes.byref(c), ctypes.byref(e), ctypes.byref(h)),
+               "pa_bm_prefix_stats")
+        return dict(cached_blocks=c.value, evictable_blocks=e.value, hit_tokens=h.value)
 
     def append_slot(self, seq_id: int):
         slot = ctypes.c_int64()

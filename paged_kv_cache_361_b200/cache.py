@@ -67,6 +67,18 @@ class PagedKVCache:
             B.pa_reshape_and_cache(k, v, self._slots.upload(slots), self.k_cache, self.v_cache)
         return slots
 
+    def add_sequence_cached(self, seq_id: int, tokens, k: torch.Tensor, v: torch.Tensor):
+        """Prefill with prefix reuse: leading whole blocks whose token prefix is
+        already cached are shared (their rows are not written again); the
+        other rows of k, v [n][Hkv][D] are written. Returns (slots, n_cached)."""
+        slots, n_cached = self.bm.add_seq_cached(seq_id, tokens)
+        n = len(slots)
+        self.lens[seq_id] = n
+        if n > n_cached:
+            B.pa_reshape_and_cache(k[n_cached:], v[n_cached:], self._slots.upload(slots[n_cached:]),
+                                   self.k_cache, self.v_cache)
+        return slots, n_cached
+
     def reserve(self, seq_id: int, num_tokens: int) -> np.ndarray:
         """Allocate blocks for a sequence whose K/V rows the caller writes itself
         (or that are already in the pool); returns the rows' slots."""
@@ -88,6 +100,27 @@ class PagedKVCache:
             B.pa_copy_blocks(self.k_cache, self.v_cache, self._pairs.upload(pairs))
         B.pa_reshape_and_cache(k, v, self._slots.upload(slots), self.k_cache, self.v_cache)
         return slots, pairs
+
+    def enable_swap(self, num_host_blocks: int):
+        """Allocate a pinned host pool of num_host_blocks blocks (same layout)."""
+        shape = (num_host_blocks,) + tuple(self.k_cache.shape[1:])
+        self.host_k = torch.empty(shape, dtype=self.k_cache.dtype, pin_memory=True)
+        self.host_v = torch.empty(shape, dtype=self.k_cache.dtype, pin_memory=True)
+        self.bm.set_host_blocks(num_host_blocks)
+
+    def swap_out(self, seq_id: int) -> np.ndarray:
+        """Move a sequence's blocks to the host pool (P2 §五); returns the pairs."""
+        pairs = self.bm.swap_out(seq_id)
+        if len(pairs):
+            B.pa_swap_blocks(self.k_cache, self.v_cache, self.host_k, self.host_v, self._pairs.upload(pairs), True)
+        return pairs
+
+    def swap_in(self, seq_id: int) -> np.ndarray:
+        """Bring a swapped-out sequence back into fresh device blocks."""
+        pairs = self.bm.swap_in(seq_id)
+        if len(pairs):
+            B.pa_swap_blocks(self.k_cache, self.v_cache, self.host_k, self.host_v, self._pairs.upload(pairs), False)
+        return pairs
 
     def free(self, seq_id: int):
         self.bm.free_seq(seq_id)

@@ -9,12 +9,22 @@
 //   P2 §3.3: a finished sequence's blocks return to the free pool.
 //   P2 §3.4: shared blocks are reference counted; writing into one copies it
 //     first, remaps the writer's table and drops one reference from the original.
+//   P2 §3.4 (prefix block pool) / P3: prompts' whole blocks can be listed in a
+//     prefix cache keyed by their full token prefix; a later prompt with the
+//     same prefix maps its first blocks onto them. The cache holds one
+//     reference per listed block; a listed block held only by the cache is
+//     evictable and is reclaimed, least recently released first, when the free
+//     list runs dry.
+//   P2 §五 (page replacement) / §八: a sequence's blocks can be swapped out to
+//     host blocks (own FIFO free list) and back in, to relieve the device pool.
 // The free list is a FIFO ring over a fixed array (front = next allocation,
-// back = most recently freed), so every operation is O(blocks touched).
+// back = most recently freed); evictable blocks sit on an intrusive LRU list;
+// every operation is O(blocks touched).
 #include <cstdint>
 #include <cstring>
 #include <new>
 #include <unordered_map>
+#include <unordered_set>
 #include <vector>
 
 #include "../../include/pagedattn.h"
@@ -26,10 +36,47 @@ struct Seq {
   int64_t len = 0;
 };
 
+// Prefix-cache key of a prompt block: a 64-bit hash chained over every token
+// of the prompt up to the block's end. The entry keeps the parent's chain hash
+// and the block's own tokens, which a hit must match exactly.
+uint64_t mix64(uint64_t x) {
+  x ^= x >> 30;
+  x *= 0xbf58476d1ce4e5b9ull;
+  x ^= x >> 27;
+  x *= 0x94d049bb133111ebull;
+  x ^= x >> 31;
+  return x;
+}
+constexpr uint64_t kChainSeed = 0x6a09e667f3bcc909ull;
+uint64_t chain_hash(uint64_t parent, const int32_t* tok, int32_t n) {
+  uint64_t h = mix64(parent ^ 0x9e3779b97f4a7c15ull);
+  for (int32_t i = 0; i < n; ++i) h = mix64(h ^ (static_cast<uint64_t>(static_cast<uint32_t>(tok[i])) + 0x632be59bd9b4e019ull));
+  return h;
+}
+
+struct CacheEntry {
+  int32_t block;
+  uint64_t parent;
+  std::vector<int32_t> tokens;
+};
+
+struct Swapped {
+  std::vector<int32_t> host;  // host block of each logical block
+  int64_t len = 0;
+};
+
 class BlockManager {
  public:
   BlockManager(int64_t num_blocks, int32_t block_size)
-      : nb_(num_blocks), bs_(block_size), ring_(num_blocks), ref_(num_blocks, 0) {}
+      : nb_(num_blocks),
+        bs_(block_size),
+        ring_(num_blocks),
+        ref_(num_blocks, 0),
+        key_of_(num_blocks, 0),
+        cached_(num_blocks, 0),
+        lru_prev_(num_blocks, -1),
+        lru_next_(num_blocks, -1),
+        in_lru_(num_blocks, 0) {}
 
   bool init_order(const int32_t* order) {
     std::vector<uint8_t> seen(nb_, 0);
@@ -48,9 +95,9 @@ class BlockManager {
 
   pa_status add_seq(int64_t id, int32_t n, int64_t* slots) {
     if (n < 0) return PA_ERR_INVALID_ARG;
-    if (seqs_.count(id)) return PA_ERR_SEQ_EXISTS;
+    if (seqs_.count(id) || swapped_.count(id)) return PA_ERR_SEQ_EXISTS;
     int64_t need = (static_cast<int64_t>(n) + bs_ - 1) / bs_;
-    if (need > count_) return PA_ERR_NO_FREE_BLOCKS;
+    if (need > available()) return PA_ERR_NO_FREE_BLOCKS;
     Seq s;
     s.table.reserve(need);
     for (int64_t i = 0; i < need; ++i) {
@@ -68,7 +115,7 @@ class BlockManager {
   pa_status fork(int64_t parent, int64_t child) {
     auto it = seqs_.find(parent);
     if (it == seqs_.end()) return PA_ERR_UNKNOWN_SEQ;
-    if (seqs_.count(child)) return PA_ERR_SEQ_EXISTS;
+    if (seqs_.count(child) || swapped_.count(child)) return PA_ERR_SEQ_EXISTS;
     Seq c = it->second;  // copy of table and length
     for (int32_t b : c.table) ++ref_[b];
     seqs_.emplace(child, std::move(c));
@@ -86,7 +133,7 @@ class BlockManager {
     auto it = seqs_.find(id);
     if (it == seqs_.end()) return PA_ERR_UNKNOWN_SEQ;
     Seq& s = it->second;
-    if (blocks_needed(s) > count_) return PA_ERR_NO_FREE_BLOCKS;
+    if (blocks_needed(s) > available()) return PA_ERR_NO_FREE_BLOCKS;
     do_append(s, slot, pair);
     return PA_OK;
   }
@@ -122,7 +169,7 @@ class BlockManager {
       st.private_bi = bi;
       st.len += 1;
     }
-    if (need > count_) return PA_ERR_NO_FREE_BLOCKS;
+    if (need > available()) return PA_ERR_NO_FREE_BLOCKS;
     int32_t np = 0;
     for (int32_t i = 0; i < n; ++i) {
       int32_t pr[2];
@@ -140,12 +187,143 @@ class BlockManager {
   }
 
   pa_status free_seq(int64_t id) {
+    auto sw = swapped_.find(id);
+    if (sw != swapped_.end()) {
+      for (int32_t h : sw->second.host) hpush(h);
+      swapped_.erase(sw);
+      return PA_OK;
+    }
     auto it = seqs_.find(id);
     if (it == seqs_.end()) return PA_ERR_UNKNOWN_SEQ;
-    for (int32_t b : it->second.table)
-      if (--ref_[b] == 0) push(b);
+    for (int32_t b : it->second.table) {
+      if (--ref_[b] == 0)
+        push(b);
+      else if (ref_[b] == 1 && cached_[b])
+        lru_push_back(b);  // only the cache holds it now
+    }
     seqs_.erase(it);
     return PA_OK;
+  }
+
+  // Prefill with prefix reuse (see pa_bm_add_seq_cached).
+  pa_status add_seq_cached(int64_t id, const int32_t* tok, int32_t n, int64_t* slots, int32_t* n_cached) {
+    if (n < 0 || (n > 0 && !tok)) return PA_ERR_INVALID_ARG;
+    if (seqs_.count(id) || swapped_.count(id)) return PA_ERR_SEQ_EXISTS;
+    const int32_t nfull = n / bs_;
+    const int64_t nblocks = (static_cast<int64_t>(n) + bs_ - 1) / bs_;
+    std::vector<int32_t> hits;
+    std::vector<uint64_t> keys(nfull);
+    uint64_t parent = kChainSeed;
+    bool missed = false;
+    int64_t evictable_hits = 0;
+    for (int32_t i = 0; i < nfull; ++i) {
+      const int32_t* bt = tok + static_cast<int64_t>(i) * bs_;
+      keys[i] = chain_hash(parent, bt, bs_);
+      if (!missed) {
+        auto it = cache_.find(keys[i]);
+        if (it != cache_.end() && it->second.parent == parent &&
+            std::memcmp(it->second.tokens.data(), bt, sizeof(int32_t) * bs_) == 0) {
+          hits.push_back(it->second.block);
+          if (in_lru_[it->second.block]) ++evictable_hits;
+        } else {
+          missed = true;
+        }
+      }
+      parent = keys[i];
+    }
+    const int64_t need = nblocks - static_cast<int64_t>(hits.size());
+    if (need > available() - evictable_hits) return PA_ERR_NO_FREE_BLOCKS;
+    Seq s;
+    s.table.reserve(nblocks);
+    for (int32_t b : hits) {
+      if (in_lru_[b]) lru_remove(b);
+      ++ref_[b];
+      s.table.push_back(b);
+    }
+    for (int64_t i = static_cast<int64_t>(hits.size()); i < nblocks; ++i) {
+      int32_t b = pop();
+      ref_[b] = 1;
+      s.table.push_back(b);
+      if (i < nfull && !cache_.count(keys[i])) {
+        CacheEntry e;
+        e.block = b;
+        e.parent = i == 0 ? kChainSeed : keys[i - 1];
+        e.tokens.assign(tok + i * bs_, tok + (i + 1) * bs_);
+        cache_.emplace(keys[i], std::move(e));
+        key_of_[b] = keys[i];
+        cached_[b] = 1;
+        ++ref_[b];  // the cache's own reference
+      }
+    }
+    s.len = n;
+    const int32_t nc = static_cast<int32_t>(hits.size()) * bs_;
+    hit_tokens_ += nc;
+    if (slots)
+      for (int32_t t = 0; t < n; ++t) slots[t] = t < nc ? -1 : slot_of(s.table, t);
+    if (n_cached) *n_cached = nc;
+    seqs_.emplace(id, std::move(s));
+    return PA_OK;
+  }
+
+  pa_status set_host_blocks(int64_t n) {
+    if (n < 0 || n > INT32_MAX || !swapped_.empty()) return PA_ERR_INVALID_ARG;
+    hring_.assign(n, 0);
+    for (int64_t i = 0; i < n; ++i) hring_[i] = static_cast<int32_t>(i);
+    hhead_ = 0;
+    hcount_ = n;
+    return PA_OK;
+  }
+
+  pa_status swap_out(int64_t id, int32_t* pairs, int32_t cap, int32_t* n_out) {
+    auto it = seqs_.find(id);
+    if (it == seqs_.end()) return PA_ERR_UNKNOWN_SEQ;
+    const int64_t nb = static_cast<int64_t>(it->second.table.size());
+    if (nb > cap || (nb > 0 && !pairs)) return PA_ERR_INVALID_ARG;
+    if (nb > hcount_) return PA_ERR_NO_FREE_BLOCKS;
+    Swapped sw;
+    sw.len = it->second.len;
+    sw.host.reserve(nb);
+    for (int64_t i = 0; i < nb; ++i) {
+      const int32_t h = hpop();
+      sw.host.push_back(h);
+      pairs[2 * i] = it->second.table[i];
+      pairs[2 * i + 1] = h;
+    }
+    free_seq(id);  // one reference per device block
+    swapped_.emplace(id, std::move(sw));
+    if (n_out) *n_out = static_cast<int32_t>(nb);
+    return PA_OK;
+  }
+
+  pa_status swap_in(int64_t id, int32_t* pairs, int32_t cap, int32_t* n_out) {
+    auto sw = swapped_.find(id);
+    if (sw == swapped_.end()) return PA_ERR_UNKNOWN_SEQ;
+    const int64_t nb = static_cast<int64_t>(sw->second.host.size());
+    if (nb > cap || (nb > 0 && !pairs)) return PA_ERR_INVALID_ARG;
+    if (nb > available()) return PA_ERR_NO_FREE_BLOCKS;
+    Seq s;
+    s.len = sw->second.len;
+    s.table.reserve(nb);
+    for (int64_t i = 0; i < nb; ++i) {
+      const int32_t b = pop();
+      ref_[b] = 1;
+      s.table.push_back(b);
+      pairs[2 * i] = sw->second.host[i];
+      pairs[2 * i + 1] = b;
+    }
+    for (int32_t h : sw->second.host) hpush(h);
+    swapped_.erase(sw);
+    seqs_.emplace(id, std::move(s));
+    if (n_out) *n_out = static_cast<int32_t>(nb);
+    return PA_OK;
+  }
+
+  int64_t host_free() const { return hcount_; }
+
+  void prefix_stats(int64_t* cached, int64_t* evictable, int64_t* hit_tokens) const {
+    if (cached) *cached = static_cast<int64_t>(cache_.size());
+    if (evictable) *evictable = lru_size_;
+    if (hit_tokens) *hit_tokens = hit_tokens_;
   }
 
   const Seq* find(int64_t id) const {
@@ -185,7 +363,54 @@ class BlockManager {
   int64_t slot_of(const std::vector<int32_t>& table, int64_t t) const {
     return static_cast<int64_t>(table[t / bs_]) * bs_ + t % bs_;
   }
+  // Blocks an allocation can draw on: the free list plus evictable cached blocks.
+  int64_t available() const { return count_ + lru_size_; }
+
+  void lru_push_back(int32_t b) {
+    lru_prev_[b] = lru_tail_;
+    lru_next_[b] = -1;
+    if (lru_tail_ >= 0)
+      lru_next_[lru_tail_] = b;
+    else
+      lru_head_ = b;
+    lru_tail_ = b;
+    in_lru_[b] = 1;
+    ++lru_size_;
+  }
+  void lru_remove(int32_t b) {
+    if (lru_prev_[b] >= 0)
+      lru_next_[lru_prev_[b]] = lru_next_[b];
+    else
+      lru_head_ = lru_next_[b];
+    if (lru_next_[b] >= 0)
+      lru_prev_[lru_next_[b]] = lru_prev_[b];
+    else
+      lru_tail_ = lru_prev_[b];
+    in_lru_[b] = 0;
+    --lru_size_;
+  }
+  // Free list empty: drop the least recently released evictable block from
+  // the cache and put it on the free list.
+  void evict_one() {
+    const int32_t b = lru_head_;
+    lru_remove(b);
+    cache_.erase(key_of_[b]);
+    cached_[b] = 0;
+    ref_[b] = 0;
+    push(b);
+  }
+  int32_t hpop() {
+    const int32_t h = hring_[hhead_];
+    hhead_ = (hhead_ + 1) % static_cast<int64_t>(hring_.size());
+    --hcount_;
+    return h;
+  }
+  void hpush(int32_t h) {
+    hring_[(hhead_ + hcount_) % static_cast<int64_t>(hring_.size())] = h;
+    ++hcount_;
+  }
   int32_t pop() {
+    if (count_ == 0) evict_one();
     int32_t b = ring_[head_];
     head_ = (head_ + 1) % nb_;
     --count_;
@@ -226,6 +451,19 @@ class BlockManager {
   int64_t head_ = 0, count_ = 0;
   std::vector<int32_t> ref_;
   std::unordered_map<int64_t, Seq> seqs_;
+  // prefix cache
+  std::unordered_map<uint64_t, CacheEntry> cache_;
+  std::vector<uint64_t> key_of_;
+  std::vector<uint8_t> cached_;
+  std::vector<int32_t> lru_prev_, lru_next_;
+  std::vector<uint8_t> in_lru_;
+  int32_t lru_head_ = -1, lru_tail_ = -1;
+  int64_t lru_size_ = 0;
+  int64_t hit_tokens_ = 0;
+  // host blocks for swapped-out sequences
+  std::vector<int32_t> hring_;
+  int64_t hhead_ = 0, hcount_ = 0;
+  std::unordered_map<int64_t, Swapped> swapped_;
 };
 
 }  // namespace
@@ -255,6 +493,34 @@ void pa_bm_destroy(pa_bm* bm) { delete bm; }
 pa_status pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int32_t num_tokens, int64_t* slots_out) {
   if (!bm) return PA_ERR_INVALID_ARG;
   return bm->m.add_seq(seq_id, num_tokens, slots_out);
+}
+
+pa_status pa_bm_add_seq_cached(pa_bm* bm, int64_t seq_id, const int32_t* tokens, int32_t num_tokens,
+                               int64_t* slots_out, int32_t* n_cached_out) {
+  if (!bm) return PA_ERR_INVALID_ARG;
+  return bm->m.add_seq_cached(seq_id, tokens, num_tokens, slots_out, n_cached_out);
+}
+
+pa_status pa_bm_prefix_stats(const pa_bm* bm, int64_t* cached_blocks, int64_t* evictable_blocks,
+                             int64_t* hit_tokens) {
+  if (!bm) return PA_ERR_INVALID_ARG;
+  bm->m.prefix_stats(cached_blocks, evictable_blocks, hit_tokens);
+  return PA_OK;
+}
+
+pa_status pa_bm_set_host_blocks(pa_bm* bm, int64_t num_host_blocks) {
+  if (!bm) return PA_ERR_INVALID_ARG;
+  return bm->m.set_host_blocks(num_host_blocks);
+}
+
+pa_status pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int32_t* pairs_out, int32_t cap, int32_t* n_pairs_out) {
+  if (!bm || cap < 0) return PA_ERR_INVALID_ARG;
+  return bm->m.swap_out(seq_id, pairs_out, cap, n_pairs_out);
+}
+
+pa_status pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int32_t* pairs_out, int32_t cap, int32_t* n_pairs_out) {
+  if (!bm || cap < 0) return PA_ERR_INVALID_ARG;
+  return bm->m.swap_in(seq_id, pairs_out, cap, n_pairs_out);
 }
 
 pa_status pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child) {

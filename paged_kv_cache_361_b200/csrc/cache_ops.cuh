@@ -72,4 +72,35 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(int4* __restrict__ kc,
   }
 }
 
+// Swap whole blocks between the device pool and a host pool in pinned,
+// device-mapped memory (same layout): dst[pair.y] = src[pair.x] for K and V.
+// `src_nb` / `dst_nb` bound the ids on each side. Consecutive threads move
+// consecutive 16-byte chunks, so the host side sees full-line PCIe transfers.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const int4* __restrict__ sk, const int4* __restrict__ sv,
+                                                          int4* __restrict__ dk, int4* __restrict__ dv,
+                                                          const int32_t* __restrict__ pairs, int32_t n_pairs,
+                                                          int64_t chunks, int32_t blocks_per_pair, int64_t src_nb,
+                                                          int64_t dst_nb) {
+  const int32_t p = blockIdx.x / blocks_per_pair;
+  const int32_t part = blockIdx.x - p * blocks_per_pair;
+  if (p >= n_pairs) return;
+  const int32_t src = __ldg(pairs + 2 * p);
+  const int32_t dst = __ldg(pairs + 2 * p + 1);
+  if (src < 0 || src >= src_nb || dst < 0 || dst >= dst_nb) {
+    if (part == 0 && threadIdx.x == 0) record_error(PA_ERR_DEVICE_BOUNDS, (src < 0 || src >= src_nb) ? src : dst);
+    return;
+  }
+  const int4* ks = sk + static_cast<int64_t>(src) * chunks;
+  const int4* vs = sv + static_cast<int64_t>(src) * chunks;
+  int4* kd = dk + static_cast<int64_t>(dst) * chunks;
+  int4* vd = dv + static_cast<int64_t>(dst) * chunks;
+  const int64_t stride = static_cast<int64_t>(blocks_per_pair) * blockDim.x;
+  for (int64_t c = static_cast<int64_t>(part) * blockDim.x + threadIdx.x; c < chunks; c += stride) {
+    const int4 a = ks[c];
+    const int4 b = vs[c];
+    kd[c] = a;
+    vd[c] = b;
+  }
+}
+
 }  // namespace pa

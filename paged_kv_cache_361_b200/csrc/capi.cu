@@ -58,18 +58,40 @@ int32_t num_parts(int32_t max_ctx, int32_t P) {
   return (max_ctx + P - 1) / P;
 }
 
-size_t ws_bytes(int32_t num_seqs, int32_t hq, int32_t D, int32_t max_parts) {
-  if (max_parts <= 1) return 0;
-  const size_t rows = static_cast<size_t>(num_seqs) * hq * max_parts;
-  const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
-  return ml + rows * D * sizeof(float);
+// Workspace: [work counters (1 + num_seqs * hkv) x u32, 256-aligned]
+//            [split partials (m, l): num_seqs * hq * parts x 2 floats, 256-aligned]
+//            [split partials o: num_seqs * hq * parts x D floats]
+size_t counters_bytes(int32_t num_seqs, int32_t hkv) {
+  return (static_cast<size_t>(1 + static_cast<int64_t>(num_seqs) * hkv) * 4 + 255) / 256 * 256;
+}
+size_t ml_bytes(int32_t num_seqs, int32_t hq, int32_t max_parts) {
+  return (static_cast<size_t>(num_seqs) * hq * max_parts * 2 * sizeof(float) + 255) / 256 * 256;
+}
+size_t ws_bytes(int32_t num_seqs, int32_t hq, int32_t hkv, int32_t D, int32_t max_parts) {
+  size_t b = counters_bytes(num_seqs, hkv);
+  if (max_parts > 1) b += ml_bytes(num_seqs, hq, max_parts) + static_cast<size_t>(num_seqs) * hq * max_parts * D * 4;
+  return b;
+}
+
+int device_sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
 }
 
 template <typename T, int D, int G>
 pa_status launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   using Cfg = SimtCfg<T, D>;
   auto kern = decode_simt_kernel<T, D, G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+          cudaSuccess)
     return PA_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(a);
   return launched();
@@ -121,16 +143,43 @@ bool encode_rows(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) {
 }
 
 template <int D, int G>
-pa_status launch_mma(const DecodeArgs& a, const pa_cache* c, dim3 grid, cudaStream_t st) {
+pa_status launch_mma(const DecodeArgs& a, const pa_cache* c, bool persistent, cudaStream_t st) {
   using Cfg = MmaCfg<D>;
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(c->num_blocks) * c->num_kv_heads * c->block_size;
   if (!encode_rows(&tk, c->k, rows, D, c->block_size) || !encode_rows(&tv, c->v, rows, D, c->block_size))
     return PA_ERR_CUDA;
-  auto kern = decode_mma_kernel<D, G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
-    return PA_ERR_CUDA;
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
+  if (!persistent) {
+    auto kern = decode_mma_kernel<D, G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+            cudaSuccess)
+      return PA_ERR_CUDA;
+    kern<<<dim3(a.hkv, a.num_seqs, a.max_parts), Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
+    return launched();
+  }
+  auto kern = decode_mma_persistent_kernel<D, G>;
+  static int occ[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+  if (!occ[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kPersistSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+            cudaSuccess)
+      return PA_ERR_CUDA;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, Cfg::kThreads, Cfg::kPersistSmemBytes) !=
+            cudaSuccess ||
+        n < 1)
+      return PA_ERR_CUDA;
+    occ[dev] = n;
+  }
+  // one CTA per resident slot; work items handed out by counters[0]
+  if (cudaMemsetAsync(a.counters, 0, counters_bytes(a.num_seqs, a.hkv), st) != cudaSuccess) return PA_ERR_CUDA;
+  const int64_t slots = static_cast<int64_t>(occ[dev]) * device_sm_count();
+  const unsigned grid = static_cast<unsigned>(a.n_items < slots ? a.n_items : slots);
+  kern<<<grid, Cfg::kThreads, Cfg::kPersistSmemBytes, st>>>(tk, tv, a);
   return launched();
 }
 
@@ -142,9 +191,14 @@ bool mma_eligible(const pa_cache* c, int G) {
          static_cast<int64_t>(c->num_blocks) * c->num_kv_heads * c->block_size <= INT32_MAX;
 }
 
-pa_status dispatch_mma(const DecodeArgs& a, const pa_cache* c, int G, dim3 grid, cudaStream_t st) {
-  if (c->head_dim == 128) return G == 8 ? launch_mma<128, 8>(a, c, grid, st) : launch_mma<128, 4>(a, c, grid, st);
-  return G == 8 ? launch_mma<64, 8>(a, c, grid, st) : launch_mma<64, 4>(a, c, grid, st);
+// Persistent CTAs pay off when long sequences are cut into many short, equal
+// partitions (measured on a B200: 512-token partitions of 32k-131k contexts
+// gain ~12 %); with few or unequal work items one CTA per item balances better.
+pa_status dispatch_mma(const DecodeArgs& a, const pa_cache* c, int G, cudaStream_t st) {
+  const bool persistent = a.part_tokens > 0 && a.part_tokens <= 1024 && a.max_parts >= 8;
+  if (c->head_dim == 128)
+    return G == 8 ? launch_mma<128, 8>(a, c, persistent, st) : launch_mma<128, 4>(a, c, persistent, st);
+  return G == 8 ? launch_mma<64, 8>(a, c, persistent, st) : launch_mma<64, 4>(a, c, persistent, st);
 }
 
 // One thread waits on an mbarrier that nothing will complete: exercises the
@@ -158,8 +212,9 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
 
 template <int D>
 pa_status launch_reduce(const DecodeArgs& a, cudaStream_t st) {
-  dim3 grid(a.hq, a.num_seqs);
-  decode_reduce_kernel<D><<<grid, 32 * kReduceWarps, 0, st>>>(a);
+  const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.hq;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
+  decode_reduce_kernel<D><<<static_cast<unsigned>(rows < cap ? rows : cap), 32 * kReduceWarps, 0, st>>>(a);
   return launched();
 }
 
@@ -223,6 +278,46 @@ pa_status pa_copy_blocks(const pa_cache* cache, const int32_t* src_dst_pairs, in
   return launched();
 }
 
+pa_status pa_swap_blocks(const pa_cache* cache, void* host_k, void* host_v, int64_t host_num_blocks,
+                         const int32_t* pairs, int32_t n_pairs, int32_t to_host, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (n_pairs < 0 || host_num_blocks <= 0 || host_num_blocks > INT32_MAX) return PA_ERR_INVALID_ARG;
+  if (n_pairs == 0) return PA_OK;
+  if (!host_k || !host_v || !pairs || !aligned16(host_k) || !aligned16(host_v) ||
+      (reinterpret_cast<uintptr_t>(pairs) & 7))
+    return PA_ERR_INVALID_ARG;
+  // The host pools must be pinned and mapped into the device's address space:
+  // a kernel touching pageable memory would fault.
+  void* dk_host = nullptr;
+  void* dv_host = nullptr;
+  for (int i = 0; i < 2; ++i) {
+    void* hp = i == 0 ? host_k : host_v;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, hp) != cudaSuccess) {
+      cudaGetLastError();
+      return PA_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeHost || !attr.devicePointer) return PA_ERR_INVALID_ARG;
+    (i == 0 ? dk_host : dv_host) = attr.devicePointer;
+  }
+  const int64_t chunks = static_cast<int64_t>(cache->num_kv_heads) * cache->block_size * cache->head_dim *
+                         elem_bytes(cache->dtype) / 16;
+  const int threads = 256;
+  int64_t bpp = (chunks + threads * 2 - 1) / (threads * 2);
+  if (bpp < 1) bpp = 1;
+  const int64_t grid = bpp * n_pairs;
+  if (grid > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  const int4* sk = static_cast<const int4*>(to_host ? cache->k : dk_host);
+  const int4* sv = static_cast<const int4*>(to_host ? cache->v : dv_host);
+  int4* dk = static_cast<int4*>(to_host ? dk_host : cache->k);
+  int4* dv = static_cast<int4*>(to_host ? dv_host : cache->v);
+  swap_blocks_kernel<<<static_cast<unsigned>(grid), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      sk, sv, dk, dv, pairs, n_pairs, chunks, static_cast<int32_t>(bpp), to_host ? cache->num_blocks : host_num_blocks,
+      to_host ? host_num_blocks : cache->num_blocks);
+  return launched();
+}
+
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t max_context_len, int32_t block_size) {
   (void)num_q_heads;
@@ -233,7 +328,7 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
                                  int32_t max_context_len, int32_t block_size, int32_t partition_tokens) {
   if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0) return 0;
   const int32_t P = resolve_partition(num_seqs, num_kv_heads, max_context_len, block_size, partition_tokens);
-  return ws_bytes(num_seqs, num_q_heads, head_dim, num_parts(max_context_len, P));
+  return ws_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, num_parts(max_context_len, P));
 }
 
 pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
@@ -260,9 +355,10 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   const int32_t P = resolve_partition(num_seqs, cache->num_kv_heads, max_context_len, cache->block_size,
                                       partition_tokens);
   const int32_t parts = num_parts(max_context_len, P);
-  if (parts > 65535) return PA_ERR_UNSUPPORTED;
-  const size_t need = ws_bytes(num_seqs, num_q_heads, cache->head_dim, parts);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_INVALID_ARG;
+  if (parts > 65535 || static_cast<int64_t>(cache->num_kv_heads) * num_seqs * parts > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
+  const size_t need = ws_bytes(num_seqs, num_q_heads, cache->num_kv_heads, cache->head_dim, parts);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)) return PA_ERR_INVALID_ARG;
 
   DecodeArgs a;
   a.q = q;
@@ -271,10 +367,11 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   a.tables = block_tables;
   a.lens = context_lens;
   a.out = out;
-  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * parts;
-  a.ws_ml = need ? static_cast<float*>(workspace) : nullptr;
-  a.ws_o = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + (rows * 2 * sizeof(float) + 255) / 256 * 256)
-                : nullptr;
+  char* ws = static_cast<char*>(workspace);
+  a.counters = reinterpret_cast<unsigned int*>(ws);
+  const size_t cb = counters_bytes(num_seqs, cache->num_kv_heads);
+  a.ws_ml = parts > 1 ? reinterpret_cast<float*>(ws + cb) : nullptr;
+  a.ws_o = parts > 1 ? reinterpret_cast<float*>(ws + cb + ml_bytes(num_seqs, num_q_heads, parts)) : nullptr;
   a.num_blocks = cache->num_blocks;
   a.num_seqs = num_seqs;
   a.hq = num_q_heads;
@@ -285,12 +382,13 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   a.part_tokens = parts > 1 ? P : 0;
   a.max_parts = parts;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.n_items = static_cast<int32_t>(static_cast<int64_t>(cache->num_kv_heads) * num_seqs * parts);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(cache->num_kv_heads, num_seqs, parts);
   const int D = cache->head_dim;
   if (mma_eligible(cache, G)) {
-    st = dispatch_mma(a, cache, G, grid, s);
+    st = dispatch_mma(a, cache, G, s);
   } else if (cache->dtype == PA_BF16) {
     st = D == 128 ? dispatch_g<__nv_bfloat16, 128>(a, G, grid, s) : dispatch_g<__nv_bfloat16, 64>(a, G, grid, s);
   } else {

@@ -25,8 +25,12 @@ struct DecodeArgs {
   int64_t num_blocks;
   int32_t num_seqs, hq, hkv, bs, max_blocks, max_ctx;
   int32_t part_tokens;  // > 0: partition size; 0: one partition per sequence
-  int32_t max_parts;    // grid.z
+  int32_t max_parts;    // partitions of the longest sequence
   float scale_log2;     // scale * log2(e)
+  // Persistent kernels: counters[0] hands out work items. Zeroed before every
+  // launch.
+  unsigned int* counters;
+  int32_t n_items;      // hkv * num_seqs * max_parts
 };
 
 template <typename T>
@@ -81,6 +85,20 @@ __device__ __forceinline__ bool cta_part(const DecodeArgs& a, int g, int s, int 
   pt.nparts = a.part_tokens > 0 ? (L + P - 1) / P : 1;
   return true;
 }
+
+// Work item -> (kv head g, sequence s, partition p), partition-major so that
+// partition 0 of every sequence comes first.
+__device__ __forceinline__ void item_coords(const DecodeArgs& a, int item, int& g, int& s, int& p) {
+  const int per = a.hkv * a.num_seqs;
+  p = item / per;
+  const int r = item - p * per;
+  s = r / a.hkv;
+  g = r - s * a.hkv;
+}
+
+// Named barrier over the four consumer warps (threads 0..127); the producer
+// warp never joins it.
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -177,67 +195,72 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const
 
 // Merge the partitions of one (sequence, query head):
 //   M = max_p m_p,  out = sum_p o_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).
-// Grid (hq, num_seqs), 8 warps: warp w folds partitions w, w+8, ... with each
-// lane owning D/32 dims (one coalesced row read per partition), then the warps
-// are folded through shared memory. Sequences with one partition were written
-// by the decode kernel and are skipped.
+// A grid of a few CTAs per SM strides over the (sequence, query head) rows;
+// 8 warps: warp w folds partitions w, w+8, ... with each lane owning D/32 dims
+// (one coalesced row read per partition), then the warps are folded through
+// shared memory. Sequences with one partition were written by the decode
+// kernel and are skipped.
 constexpr int kReduceWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(32 * kReduceWarps) decode_reduce_kernel(const DecodeArgs a) {
   constexpr int VEC = D / 32;
-  const int hq = blockIdx.x, s = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int32_t L = load_len(a, s, false);
-  const int32_t P = a.part_tokens;
-  const int32_t nparts = (L + P - 1) / P;
-  if (nparts <= 1) return;
-  const int64_t row = static_cast<int64_t>(s) * a.hq + hq;
-  const float* ml = a.ws_ml + row * a.max_parts * 2;
-  const float* o = a.ws_o + row * a.max_parts * D;
   __shared__ float red[kReduceWarps];
   __shared__ float wl[kReduceWarps];
   __shared__ float wo[kReduceWarps][D];
+  const int64_t nrows = static_cast<int64_t>(a.num_seqs) * a.hq;
+  // grid-stride over (sequence, query head) rows; rows of unsplit sequences are skipped
+  for (int64_t row = blockIdx.x; row < nrows; row += gridDim.x) {
+    const int s = static_cast<int>(row / a.hq);
+    const int32_t L = load_len(a, s, false);
+    const int32_t P = a.part_tokens;
+    const int32_t nparts = (L + P - 1) / P;
+    if (nparts <= 1) continue;  // uniform across the CTA
+    const float* ml = a.ws_ml + row * a.max_parts * 2;
+    const float* o = a.ws_o + row * a.max_parts * D;
 
-  float M = -INFINITY;
-  for (int q = tid; q < nparts; q += 32 * kReduceWarps) M = fmaxf(M, ml[2 * q]);
-  M = warp_max(M);
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = red[0];
+    float M = -INFINITY;
+    for (int q = tid; q < nparts; q += 32 * kReduceWarps) M = fmaxf(M, ml[2 * q]);
+    M = warp_max(M);
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = red[0];
 #pragma unroll
-  for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, red[w]);
+    for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, red[w]);
 
-  float l = 0.f, acc[VEC];
+    float l = 0.f, acc[VEC];
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-  for (int q = warp; q < nparts; q += kReduceWarps) {
-    const float f = exp2f(ml[2 * q] - M);
-    l = fmaf(ml[2 * q + 1], f, l);
-    const float* src = o + static_cast<int64_t>(q) * D + lane * VEC;
-    if (VEC == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(src);
-      acc[0] = fmaf(x.x, f, acc[0]);
-      acc[1] = fmaf(x.y, f, acc[1]);
-      acc[2] = fmaf(x.z, f, acc[2]);
-      acc[3] = fmaf(x.w, f, acc[3]);
-    } else {
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+    for (int q = warp; q < nparts; q += kReduceWarps) {
+      const float f = exp2f(ml[2 * q] - M);
+      l = fmaf(ml[2 * q + 1], f, l);
+      const float* src = o + static_cast<int64_t>(q) * D + lane * VEC;
+      if (VEC == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] = fmaf(x.x, f, acc[0]);
+        acc[1] = fmaf(x.y, f, acc[1]);
+        acc[2] = fmaf(x.z, f, acc[2]);
+        acc[3] = fmaf(x.w, f, acc[3]);
+      } else {
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[e] = fmaf(src[e], f, acc[e]);
+        for (int e = 0; e < VEC; ++e) acc[e] = fmaf(src[e], f, acc[e]);
+      }
     }
-  }
-  if (lane == 0) wl[warp] = l;
+    if (lane == 0) wl[warp] = l;
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) wo[warp][lane * VEC + e] = acc[e];
-  __syncthreads();
-  for (int d = tid; d < D; d += 32 * kReduceWarps) {
-    float num = 0.f, den = 0.f;
+    for (int e = 0; e < VEC; ++e) wo[warp][lane * VEC + e] = acc[e];
+    __syncthreads();
+    for (int d = tid; d < D; d += 32 * kReduceWarps) {
+      float num = 0.f, den = 0.f;
 #pragma unroll
-    for (int w = 0; w < kReduceWarps; ++w) {
-      num += wo[w][d];
-      den += wl[w];
+      for (int w = 0; w < kReduceWarps; ++w) {
+        num += wo[w][d];
+        den += wl[w];
+      }
+      a.out[row * D + d] = num / den;
     }
-    a.out[row * D + d] = num / den;
+    __syncthreads();  // red / wl / wo are reused by the next row
   }
 }
 

@@ -21,9 +21,16 @@
 // ldmatrix reads hit 8 different bank groups. Tokens past the context length
 // get -inf scores and their V rows are zeroed in registers, so padding (even
 // NaN) never reaches the result.
-// CTA = (kv head, sequence, partition): warp 4 is the TMA producer, warps 0-3
-// consume (warp w owns tokens [16w, 16w+16) of each 64-token chunk) over the
-// same full/empty mbarrier ring as the CUDA-core kernel.
+// Persistent CTAs (as many as fit on the GPU) take work items (kv head,
+// sequence, partition) from an atomic counter. Warp 4 is the TMA producer: it
+// walks item after item without draining the stage ring, writing a small
+// descriptor per stage (which item, how many tokens, first/last chunk) and, on
+// an item's first chunk, copying the item's G query rows next to the stage.
+// Warps 0-3 consume (warp w owns tokens [16w, 16w+16) of each 64-token chunk);
+// at an item's last chunk they fold their states into warp 0 in two rounds
+// through shared memory (named barrier, producer not involved) while the
+// producer keeps prefetching the next item. A split sequence's partitions are
+// merged afterwards by decode_reduce_kernel.
 #pragma once
 
 #include <cuda.h>
@@ -63,6 +70,7 @@ __device__ __forceinline__ void mma_rows8(float (&d)[2], uint32_t a0, uint32_t a
       "{%10, %11, %12, %12};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(j2), "=f"(j3)
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f));
+  asm volatile("" ::"f"(j2), "f"(j3));  // rows 8..15: discarded
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -89,21 +97,374 @@ struct MmaCfg {
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = kStageBytes <= 16384 ? 4 : 3;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack for the swizzle
+  static constexpr int kQBytes = 8 * D * 2;                // query rows of one item (G <= 8)
+  static constexpr int kNT = D / 8;
+  static constexpr int kFoldFloats = 32 * (2 * kNT + 2);   // one warp's fragments + (m, l) per lane
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;  // one CTA per item
+  static constexpr int kPersistSmemBytes = kSmemBytes + kStages * kQBytes + 2 * kFoldFloats * 4;
 };
 
+
+// One consumer warp's share of a stage: its 16 tokens (nv of them valid) of
+// the K tile at kst and the V tile at vst. S = Q K^T (16 MMAs at D 128), online
+// softmax in base 2 on the S fragments, then O += P V with P split into a bf16
+// high part and remainder (32 MMAs). V rows of invalid tokens are zeroed in
+// registers so padding never reaches O.
+template <int D>
+__device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, const uint32_t (&qa)[D / 16][2],
+                                          float scale_log2, int lane, int warp, float& m_run, float& l_run,
+                                          float (&o)[D / 8][2]) {
+  using Cfg = MmaCfg<D>;
+  constexpr int NT = D / 8;
+  const int c = lane & 3;
+  const int mk = lane >> 3, ik = lane & 7;
+  const int tokK = warp * 16 + (mk >> 1) * 8 + ik;  // K matrices (tok0, d0), (tok0, d0+8), (tok0+8, d0), (tok0+8, d0+8)
+  const int dK = (mk & 1) * 8;
+  const int tokV = warp * 16 + (mk & 1) * 8 + ik;   // V matrices (tok0, d0), (tok0+8, d0), (tok0, d0+8), (tok0+8, d0+8)
+  const int dV = (mk >> 1) * 8;
+  float sacc[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const int d0 = kk * 16 + dK;
+    const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tokK * 128 + ((((d0 & 63) >> 3) ^ (tokK & 7)) << 4);
+    uint32_t b00, b01, b10, b11;
+    ldsm_x4(addr, b00, b01, b10, b11);
+    mma_rows8(sacc[0], qa[kk][0], qa[kk][1], b00, b01);
+    mma_rows8(sacc[1], qa[kk][0], qa[kk][1], b10, b11);
+  }
+  float sc[2][2];
+  float mloc = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int t = nt * 8 + 2 * c + j;
+      sc[nt][j] = t < nv ? sacc[nt][j] * scale_log2 : -INFINITY;
+      mloc = fmaxf(mloc, sc[nt][j]);
+    }
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+  const float mn = fmaxf(m_run, mloc);
+  const float alpha = exp2f(m_run - mn);
+  m_run = mn;
+  float pr[2][2];
+  float psum = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      pr[nt][j] = exp2f(sc[nt][j] - mn);
+      psum += pr[nt][j];
+    }
+  l_run = l_run * alpha + psum;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    o[j][0] *= alpha;
+    o[j][1] *= alpha;
+  }
+  uint32_t ph0, pl0, ph2, pl2;
+  split_pair(pr[0][0], pr[0][1], ph0, pl0);
+  split_pair(pr[1][0], pr[1][1], ph2, pl2);
+  uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+  if (nv < 16) {
+    mlo = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
+    mhi = (2 * c + 8 < nv ? 0x0000ffffu : 0u) | (2 * c + 9 < nv ? 0xffff0000u : 0u);
+  }
+#pragma unroll
+  for (int dgi = 0; dgi < D / 16; ++dgi) {
+    const int d0 = dgi * 16 + dV;
+    const uint32_t addr = vst + (d0 >> 6) * Cfg::kHalfBytes + tokV * 128 + ((((d0 & 63) >> 3) ^ (tokV & 7)) << 4);
+    uint32_t v0, v1, v2, v3;
+    ldsm_x4_t(addr, v0, v1, v2, v3);
+    v0 &= mlo;
+    v1 &= mhi;
+    v2 &= mlo;
+    v3 &= mhi;
+    mma_rows8(o[2 * dgi], ph0, ph2, v0, v1);
+    mma_rows8(o[2 * dgi], pl0, pl2, v0, v1);
+    mma_rows8(o[2 * dgi + 1], ph0, ph2, v2, v3);
+    mma_rows8(o[2 * dgi + 1], pl0, pl2, v2, v3);
+  }
+}
+
+// Q rows (bf16, row stride D) as MMA A fragments: a0 = row r, dims (kk*16 + 2c,
+// +1); a2 = dims +8; rows >= G are zero.
+template <int D, int G>
+__device__ __forceinline__ void load_q_frags(const uint32_t* qrow_words, int r, int c, uint32_t (&qa)[D / 16][2],
+                                             bool from_global) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    if (r < G) {
+      qa[kk][0] = from_global ? __ldg(qrow_words + kk * 8 + c) : qrow_words[kk * 8 + c];
+      qa[kk][1] = from_global ? __ldg(qrow_words + kk * 8 + 4 + c) : qrow_words[kk * 8 + 4 + c];
+    } else {
+      qa[kk][0] = qa[kk][1] = 0u;
+    }
+  }
+}
+
+constexpr int kDescFirst = 1, kDescLast = 2, kDescTerm = 4;
+
+struct StageDesc {
+  int32_t s, g, p, ntok, nparts, flags;
+};
+
+template <int S>
+struct PersistSmem {
+  uint64_t full[S];
+  uint64_t empty[S];
+  uint64_t cbar;  // consumer-warp barrier (one arrival per consumer warp)
+  StageDesc desc[S];
+  int abort_flag;
+};
+
+// Barrier over the consumer warps built on an mbarrier, so that its wait is
+// bounded like every other wait: it gives up (false) once the CTA aborts.
+__device__ __forceinline__ bool consumer_sync(uint64_t* bar, uint32_t& phase, volatile int* abort_flag, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = pipe_wait(bar, phase, abort_flag);
+  phase ^= 1u;
+  return ok;
+}
+
+// Fold another warp's (m, l, o) (same fragment layout) into this lane's.
+template <int NT>
+__device__ __forceinline__ void fold_state(float& m, float& l, float (&o)[NT][2], const float* src) {
+  const float m2 = src[2 * NT], l2 = src[2 * NT + 1];
+  const float M = fmaxf(m, m2);
+  if (M == -INFINITY) return;  // both empty
+  const float f1 = exp2f(m - M), f2 = exp2f(m2 - M);
+  l = l * f1 + l2 * f2;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    o[j][0] = o[j][0] * f1 + src[2 * j] * f2;
+    o[j][1] = o[j][1] * f1 + src[2 * j + 1] * f2;
+  }
+  m = M;
+}
+
+template <int NT>
+__device__ __forceinline__ void store_state(float* dst, float m, float l, const float (&o)[NT][2]) {
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    dst[2 * j] = o[j][0];
+    dst[2 * j + 1] = o[j][1];
+  }
+  dst[2 * NT] = m;
+  dst[2 * NT + 1] = l;
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_kernel(const __grid_constant__ CUtensorMap tmk,
+                                                                        const __grid_constant__ CUtensorMap tmv,
+                                                                        const DecodeArgs a) {
+  using Cfg = MmaCfg<D>;
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = Cfg::kNT;
+  static_assert(G <= 8, "query heads of one group must fit in MMA rows 0..7");
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ PersistSmem<S> ps;
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;  // 1024-aligned: swizzle atoms
+  uint8_t* sgen = smem_raw + (sbase - sraw);
+  const uint32_t qslot0 = sbase + S * Cfg::kStageBytes;
+  const uint8_t* qslot_gen = sgen + S * Cfg::kStageBytes;
+  float* fold = reinterpret_cast<float*>(sgen + S * Cfg::kStageBytes + S * Cfg::kQBytes);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, c = lane & 3;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&ps.full[i], 1);
+      mbar_init(&ps.empty[i], NW);
+    }
+    mbar_init(&ps.cbar, NW);
+    ps.abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == NW) {
+    // ------------------------------ producer ------------------------------
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
+    const uint64_t pol = l2_evict_first_policy();
+    const __nv_bfloat16* qbase = static_cast<const __nv_bfloat16*>(a.q);
+    int item = blockIdx.x;
+    int cs = 0;
+    bool aborted = false;
+    while (!aborted && item < a.n_items) {
+      unsigned nxt = 0;
+      if (lane == 0) nxt = atomicAdd(a.counters, 1u);  // next item, used at the end of this one
+      int g, s, p;
+      item_coords(a, item, g, s, p);
+      const int32_t L = load_len(a, s, g == 0 && p == 0 && lane == 0);
+      const int32_t P = a.part_tokens > 0 ? a.part_tokens : (L > 0 ? L : 1);
+      const int32_t t0 = p * P;
+      if (L == 0) {
+        if (p == 0)
+          for (int idx = lane; idx < G * D; idx += 32)
+            a.out[(static_cast<int64_t>(s) * a.hq + g * G) * D + idx] = 0.f;
+      } else if (t0 < L) {
+        const int32_t t1 = min(t0 + P, L);
+        const int nch = (t1 - t0 + C - 1) / C;
+        const int nparts = a.part_tokens > 0 ? (L + P - 1) / P : 1;
+        const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
+        for (int ch = 0; ch < nch; ++ch, ++cs) {
+          const int st = cs % S;
+          if (cs >= S && !pipe_wait(&ps.empty[st], ((cs / S) - 1) & 1, &ps.abort_flag)) {
+            aborted = true;
+            break;
+          }
+          const int32_t c0 = t0 + ch * C;
+          const int32_t n = min(C, t1 - c0);
+          const int32_t nb = (n + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+          int32_t blk = -1;
+          bool ok = false;
+          if (lane < nb) {
+            blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
+            ok = blk >= 0 && blk < a.num_blocks;
+            if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
+          }
+          const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+          if (lane == 0) {
+            StageDesc& d = ps.desc[st];
+            d.s = s;
+            d.g = g;
+            d.p = p;
+            d.ntok = n;
+            d.nparts = nparts;
+            d.flags = (ch == 0 ? kDescFirst : 0) | (ch == nch - 1 ? kDescLast : 0);
+            const uint32_t qbytes = ch == 0 ? static_cast<uint32_t>(G * D * 2) : 0u;
+            mbar_arrive_expect_tx(&ps.full[st], 2u * Cfg::kHalves * __popc(okmask) * box_bytes + qbytes);
+            if (ch == 0)
+              bulk_g2s(sgen + S * Cfg::kStageBytes + st * Cfg::kQBytes,
+                       qbase + (static_cast<int64_t>(s) * a.hq + g * G) * D, qbytes, &ps.full[st], pol);
+          }
+          __syncwarp();
+          if (ok) {
+            const int32_t y = (blk * a.hkv + g) * a.bs;
+            const uint32_t kdst = sbase + st * Cfg::kStageBytes + lane * box_bytes;
+#pragma unroll
+            for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+              tma_load_2d(kdst + hf * Cfg::kHalfBytes, &tmk, hf * 64, y, &ps.full[st], pol);
+              tma_load_2d(kdst + Cfg::kTileBytes + hf * Cfg::kHalfBytes, &tmv, hf * 64, y, &ps.full[st], pol);
+            }
+          }
+        }
+      }
+      item = static_cast<int>(gridDim.x + __shfl_sync(0xffffffffu, nxt, 0));
+    }
+    if (!aborted) {
+      const int st = cs % S;
+      if (cs >= S && !pipe_wait(&ps.empty[st], ((cs / S) - 1) & 1, &ps.abort_flag)) {
+        aborted = true;
+      } else if (lane == 0) {
+        ps.desc[st].flags = kDescTerm;
+        mbar_arrive(&ps.full[st]);
+      }
+      ++cs;
+    }
+    if (aborted && lane == 0)
+      for (int j = (cs > S ? cs - S : 0); j < cs; ++j) mbar_wait(&ps.full[j % S], (j / S) & 1);
+    return;
+  }
+
+  // -------------------------------- consumers --------------------------------
+  uint32_t qa[D / 16][2];
+  float o[NT][2];
+  float m_run = -INFINITY, l_run = 0.f;
+  uint32_t cphase = 0;
+#define PA_CSYNC()                                                    \
+  do {                                                                \
+    if (!consumer_sync(&ps.cbar, cphase, &ps.abort_flag, lane)) return; \
+  } while (0)
+#pragma unroll
+  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
+
+  for (int cs = 0;; ++cs) {
+    const int st = cs % S;
+    if (!pipe_wait(&ps.full[st], (cs / S) & 1, &ps.abort_flag)) return;
+    const volatile StageDesc& vd = ps.desc[st];
+    const int flags = vd.flags;
+    if (flags & kDescTerm) return;
+    const int ds = vd.s, dg = vd.g, dp = vd.p, dn = vd.ntok, dnp = vd.nparts;
+
+    if (flags & kDescFirst) {
+      load_q_frags<D, G>(reinterpret_cast<const uint32_t*>(qslot_gen + st * Cfg::kQBytes) + r * (D / 2), r, c, qa,
+                         false);
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
+    }
+
+    const int nv = min(16, dn - warp * 16);  // warp-uniform
+    if (nv > 0) {
+      const uint32_t kst = sbase + st * Cfg::kStageBytes;
+      mma_chunk<D>(kst, kst + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ps.empty[st]);
+
+    if (!(flags & kDescLast)) continue;
+
+    // ---- item finished: fold warps 3,2 -> 1,0 -> 0 (two rounds), then store ----
+    float lrow = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+    lrow += __shfl_xor_sync(0xffffffffu, lrow, 2);
+    float* slot0 = fold + lane * (2 * NT + 2);
+    float* slot1 = fold + Cfg::kFoldFloats + lane * (2 * NT + 2);
+    if (warp >= 2) store_state<NT>(warp == 2 ? slot0 : slot1, m_run, lrow, o);
+    PA_CSYNC();
+    if (warp < 2) fold_state<NT>(m_run, lrow, o, warp == 0 ? slot0 : slot1);
+    PA_CSYNC();
+    if (warp == 1) store_state<NT>(slot0, m_run, lrow, o);
+    PA_CSYNC();
+    if (warp == 0) fold_state<NT>(m_run, lrow, o, slot0);
+
+    const int64_t row0 = static_cast<int64_t>(ds) * a.hq + dg * G;
+    if (dnp == 1) {
+      if (warp == 0 && r < G) {
+        const float inv = 1.f / lrow;
+        float* dst = a.out + (row0 + r) * D + 2 * c;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0] * inv, o[j][1] * inv);
+      }
+      PA_CSYNC();  // the fold slots are free again
+      continue;
+    }
+    // split sequence: publish this partition's (m, l, o); decode_reduce_kernel merges
+    if (warp == 0 && r < G) {
+      const int64_t prow = (row0 + r) * a.max_parts + dp;
+      float* dst = a.ws_o + prow * D + 2 * c;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
+      if (c == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(m_run, lrow);
+    }
+    PA_CSYNC();  // the fold slots are free again
+  }
+#undef PA_CSYNC
+}
+
+// One CTA per work item (kv head, sequence, partition); grid (Hkv, B, parts),
+// partition-major dispatch. The producer warp streams the item's chunks; at the
+// end every warp's (m, l, o) goes through shared memory (the stage ring is free
+// by then) and the CTA stores the row or the partition's partials.
 template <int D, int G>
 __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const DecodeArgs a) {
   using Cfg = MmaCfg<D>;
-  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = D / 8;
-  static_assert(G <= 8, "query heads of one group must fit in MMA rows 0..7");
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = Cfg::kNT;
   static_assert(NW * G * (D + 2) * 4 <= S * Cfg::kStageBytes, "merge buffer must fit in the stage ring");
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ PipeSmem<S> ps;
-  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;  // 1024-aligned: swizzle atoms
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
 
   const int g = blockIdx.x, s = blockIdx.y, p = blockIdx.z;
@@ -123,7 +484,6 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const _
   float m_run = -INFINITY, l_run = 0.f;
 
   if (warp == NW) {
-    // ---- producer: one 2D TMA box [bs rows x 64 dims] per (block, half) of K and V ----
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_first_policy();
@@ -151,100 +511,17 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const _
       }
     });
   } else {
-    // ---- consumers ----
-    // Q as MMA A fragments: a0 = row r, dims (kk*16 + 2c, +1); a2 = dims +8.
     uint32_t qa[D / 16][2];
-    {
-      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                                               (static_cast<int64_t>(s) * a.hq + hq0 + r) * D);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        qa[kk][0] = r < G ? __ldg(qrow + kk * 8 + c) : 0u;
-        qa[kk][1] = r < G ? __ldg(qrow + kk * 8 + 4 + c) : 0u;
-      }
-    }
-    // per-lane ldmatrix rows: K matrices (tok0, d0), (tok0, d0+8), (tok0+8, d0), (tok0+8, d0+8);
-    // V matrices (tok0, d0), (tok0+8, d0), (tok0, d0+8), (tok0+8, d0+8)
-    const int mk = lane >> 3, ik = lane & 7;
-    const int tokK = warp * 16 + (mk >> 1) * 8 + ik;
-    const int dK = (mk & 1) * 8;
-    const int tokV = warp * 16 + (mk & 1) * 8 + ik;
-    const int dV = (mk >> 1) * 8;
-
+    load_q_frags<D, G>(reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                         (static_cast<int64_t>(s) * a.hq + hq0 + (r < G ? r : 0)) * D),
+                       r, c, qa, true);
     for (int i = 0; i < nchunks; ++i) {
       const int st = i % S;
       if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
       const int nv = min(16, min(C, pt.ntok - i * C) - warp * 16);  // warp-uniform
       if (nv > 0) {
         const uint32_t kst = sbase + st * Cfg::kStageBytes;
-        const uint32_t vst = kst + Cfg::kTileBytes;
-        float sacc[2][2];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int d0 = kk * 16 + dK;
-          const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tokK * 128 + ((((d0 & 63) >> 3) ^ (tokK & 7)) << 4);
-          uint32_t b00, b01, b10, b11;
-          ldsm_x4(addr, b00, b01, b10, b11);
-          mma_rows8(sacc[0], qa[kk][0], qa[kk][1], b00, b01);
-          mma_rows8(sacc[1], qa[kk][0], qa[kk][1], b10, b11);
-        }
-        // scores of row r, tokens nt*8 + 2c + j
-        float sc[2][2];
-        float mloc = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int t = nt * 8 + 2 * c + j;
-            sc[nt][j] = t < nv ? sacc[nt][j] * a.scale_log2 : -INFINITY;
-            mloc = fmaxf(mloc, sc[nt][j]);
-          }
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-        const float mn = fmaxf(m_run, mloc);
-        const float alpha = exp2f(m_run - mn);
-        m_run = mn;
-        float pr[2][2];
-        float psum = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            pr[nt][j] = exp2f(sc[nt][j] - mn);
-            psum += pr[nt][j];
-          }
-        l_run = l_run * alpha + psum;
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          o[j][0] *= alpha;
-          o[j][1] *= alpha;
-        }
-        uint32_t ph0, pl0, ph2, pl2;
-        split_pair(pr[0][0], pr[0][1], ph0, pl0);
-        split_pair(pr[1][0], pr[1][1], ph2, pl2);
-        // V rows of tokens >= nv are zeroed (they may be padding)
-        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-        if (nv < 16) {
-          mlo = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
-          mhi = (2 * c + 8 < nv ? 0x0000ffffu : 0u) | (2 * c + 9 < nv ? 0xffff0000u : 0u);
-        }
-#pragma unroll
-        for (int dg = 0; dg < D / 16; ++dg) {
-          const int d0 = dg * 16 + dV;
-          const uint32_t addr = vst + (d0 >> 6) * Cfg::kHalfBytes + tokV * 128 + ((((d0 & 63) >> 3) ^ (tokV & 7)) << 4);
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_t(addr, v0, v1, v2, v3);
-          v0 &= mlo;
-          v1 &= mhi;
-          v2 &= mlo;
-          v3 &= mhi;
-          mma_rows8(o[2 * dg], ph0, ph2, v0, v1);
-          mma_rows8(o[2 * dg], pl0, pl2, v0, v1);
-          mma_rows8(o[2 * dg + 1], ph0, ph2, v2, v3);
-          mma_rows8(o[2 * dg + 1], pl0, pl2, v2, v3);
-        }
+        mma_chunk<D>(kst, kst + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ps.empty[st]);

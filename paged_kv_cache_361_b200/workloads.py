@@ -44,7 +44,8 @@ import torch
 _LENGTHS, _FREE_ORDER, _TAILS, _FINISH, _ARRIVALS, _VALUES = 1, 2, 3, 4, 5, 6
 
 # value kinds (keys of the value streams)
-HIST_K, HIST_V, Q, NEW_K, NEW_V, PREFIX_K, PREFIX_V, TAIL_K, TAIL_V, PROMPT_K, PROMPT_V = range(1, 12)
+HIST_K, HIST_V, Q, NEW_K, NEW_V, PREFIX_K, PREFIX_V, TAIL_K, TAIL_V, PROMPT_K, PROMPT_V, TOKENS = range(1, 13)
+_REQUESTS = 7
 
 
 def _rng(seed: int, purpose: int, *keys: int) -> np.random.Generator:
@@ -341,4 +342,74 @@ def batching_ops(tr: BatchingTrace, steps: int | None = None) -> list:
         ids = list(live)
         ops.append(("append", ids, (lambda which, device="cpu", step=step, n=len(ids): tr.new_kv(step, which, n, device))))
         ops.append(("decode", ids, (lambda device="cpu", step=step, n=len(ids): tr.query(step, n, device))))
+    return ops
+
+
+@dataclass
+class PrefixTrace:
+    """Requests that start with one of a few shared system prompts.
+
+    Request r uses system prompt sys_of[r] (its tokens sys_tokens[k], K/V rows
+    drawn per (system prompt, position), so every request that shares it sees
+    the same rows) followed by its own tail of tail_lens[r] tokens. Requests
+    arrive in order; at most `live` run at once; when the batch is full the
+    oldest request finishes first (FIFO), before each decode step every live
+    request appends one token."""
+    shape: Shape
+    num_blocks: int
+    free_order: np.ndarray
+    sys_tokens: list
+    sys_of: np.ndarray
+    tail_lens: np.ndarray
+    live: int
+    seed: int
+
+    def request_tokens(self, r: int) -> np.ndarray:
+        tail = _rng(self.seed, _REQUESTS, r).integers(1000, 32000, size=int(self.tail_lens[r]))
+        return np.concatenate([self.sys_tokens[int(self.sys_of[r])], tail]).astype(np.int32)
+
+    def rows(self, r: int, which: str, device="cpu") -> torch.Tensor:
+        """K or V rows of request r's prompt: system part then tail."""
+        k = int(self.sys_of[r])
+        sys_n = len(self.sys_tokens[k])
+        a = normal(self.seed, (PREFIX_K if which == "k" else PREFIX_V, k),
+                   (sys_n, self.shape.num_kv_heads, self.shape.head_dim), self.shape.dtype, device)
+        b = normal(self.seed, (TAIL_K if which == "k" else TAIL_V, r),
+                   (int(self.tail_lens[r]), self.shape.num_kv_heads, self.shape.head_dim), self.shape.dtype, device)
+        return torch.cat([a, b])
+
+
+def prefix_caching(seed: int = 0, num_sys: int = 4, sys_len: int = 700, num_requests: int = 48, live: int = 16,
+                   num_blocks: int = 500, block_size: int = 16, head_dim: int = 128) -> PrefixTrace:
+    """A small pool (num_blocks) so that cached blocks get evicted."""
+    sh = Shape(32, 8, head_dim, block_size, "bf16")
+    rng = _rng(seed, _TOKENS_PURPOSE)
+    sys_tokens = [rng.integers(1000, 32000, size=sys_len - 37 * k).astype(np.int32) for k in range(num_sys)]
+    sys_of = _rng(seed, _LENGTHS, 11).integers(0, num_sys, size=num_requests)
+    tails = _rng(seed, _TAILS, 11).integers(1, 257, size=num_requests)
+    order = _rng(seed, _FREE_ORDER).permutation(num_blocks).astype(np.int64)
+    return PrefixTrace(sh, num_blocks, order, sys_tokens, sys_of, tails, live, seed)
+
+
+_TOKENS_PURPOSE = 8
+
+
+def prefix_ops(tr: PrefixTrace, decode_every: int = 4) -> list:
+    """Requests arrive one by one ("add_cached"); when `live` are running the
+    oldest finishes first; every request appends one token per step and the
+    batch decodes every `decode_every` arrivals and at the end."""
+    ops, live = [], []
+    for r in range(len(tr.sys_of)):
+        if len(live) == tr.live:
+            ops.append(("free", live.pop(0)))
+        toks = tr.request_tokens(r)
+        ops.append(("add_cached", r, toks, (lambda which, device="cpu", r=r: tr.rows(r, which, device))))
+        live.append(r)
+        if r % decode_every == decode_every - 1 or r == len(tr.sys_of) - 1:
+            ids = list(live)
+            ops.append(("append", ids, (lambda which, device="cpu", r=r, n=len(ids): normal(
+                tr.seed, (NEW_K if which == "k" else NEW_V, r), (n, tr.shape.num_kv_heads, tr.shape.head_dim),
+                tr.shape.dtype, device))))
+            ops.append(("decode", ids, (lambda device="cpu", r=r, n=len(ids): normal(
+                tr.seed, (Q, r), (n, tr.shape.num_q_heads, tr.shape.head_dim), tr.shape.dtype, device))))
     return ops

@@ -53,6 +53,12 @@ class Replay:
             _, seq, n, src = op
             slots = self.cache.add_sequence(seq, src("k").to(self.device), src("v").to(self.device))
             assert slots.tolist() == rec["slots"]
+        elif kind == "add_cached":
+            _, seq, tokens, src = op
+            slots, n_cached = self.cache.add_sequence_cached(seq, tokens, src("k").to(self.device),
+                                                             src("v").to(self.device))
+            assert slots.tolist() == rec["slots"] and n_cached == rec["n_cached"]
+            self.n_cached = getattr(self, "n_cached", 0) + n_cached
         elif kind == "fork":
             self.cache.fork(op[1], op[2])
         elif kind == "append":

@@ -81,10 +81,12 @@ def test_decode_argument_checks():
 
 
 def test_workspace_sizes():
-    # no split -> no workspace; split -> (m, l) rows rounded to 256 B + D floats per row
-    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 600, 16, 0) == 0
-    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 512, 16, 512) == 0
+    # counters (1 + num_seqs * hkv) x 4 B rounded to 256; split adds (m, l) rows rounded to 256 + D floats per row
+    cnt = lambda b, hkv: ((1 + b * hkv) * 4 + 255) // 256 * 256
+    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 600, 16, 0) == cnt(4, 8)
+    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 512, 16, 512) == cnt(4, 8)
     rows = 4 * 8 * 2
-    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 600, 16, 512) == (rows * 8 + 255) // 256 * 256 + rows * 128 * 4
-    assert B.pa_decode_partition_tokens(64, 32, 32, 2049, 16) in (0, 512) or B.pa_decode_partition_tokens(
-        64, 32, 32, 2049, 16) % 16 == 0
+    assert B.pa_decode_workspace_bytes(4, 8, 8, 128, 600, 16, 512) == \
+        cnt(4, 8) + (rows * 8 + 255) // 256 * 256 + rows * 128 * 4
+    P = B.pa_decode_partition_tokens(64, 32, 32, 2049, 16)
+    assert P == 0 or P % 16 == 0

@@ -145,3 +145,95 @@ def test_block_tables_padding():
     bm.add_seq(6, 1)
     t, lens = bm.block_tables([6, 5], cap=4, pad=-1)
     assert t.tolist() == [[3, -1, -1, -1], [0, 1, 2, -1]] and lens.tolist() == [1, 9]
+
+
+def _replay_prefix(tr_or_ops, num_blocks, bs, order, ops):
+    from oracle.prefix_cache import PrefixCachingModel
+    cpp = B.BlockManager(num_blocks, bs, order)
+    ref = PrefixCachingModel(num_blocks, bs, order)
+    live = set()
+    for op in ops:
+        if op[0] == "add_cached":
+            a, na = cpp.add_seq_cached(op[1], op[2])
+            b, nb = ref.add_seq_cached(op[1], op[2])
+            assert a.tolist() == b and na == nb
+            live.add(op[1])
+        elif op[0] == "append":
+            slots, pairs = cpp.append_slots(op[1])
+            rs = [ref.append_slot(s)[0] for s in op[1]]
+            assert slots.tolist() == rs
+        elif op[0] == "free":
+            cpp.free_seq(op[1])
+            ref.free_seq(op[1])
+            live.discard(op[1])
+        for s in live:
+            assert cpp.block_table(s)[0].tolist() == ref.block_table(s)
+        assert cpp.free_list().tolist() == list(ref.free)
+        st = cpp.prefix_stats()
+        assert st == ref.prefix_stats()
+    for b in range(num_blocks):
+        assert cpp.refcount(b) == ref.ref[b]
+    return cpp, ref
+
+
+def test_prefix_cache_trace_bit_exact():
+    tr = W.prefix_caching()
+    cpp, ref = _replay_prefix(tr, tr.num_blocks, tr.shape.block_size, tr.free_order, W.prefix_ops(tr))
+    st = ref.prefix_stats()
+    assert st["hit_tokens"] > 0 and st["cached_blocks"] > 0
+
+
+def test_prefix_cache_random_stress_with_eviction():
+    rng = np.random.default_rng(7)
+    for trial in range(20):
+        bs = int(rng.choice([1, 2, 4]))
+        nb = int(rng.integers(8, 40))
+        order = rng.permutation(nb)
+        prefixes = [rng.integers(0, 5, size=int(rng.integers(0, 3 * bs + 2))).tolist() for _ in range(3)]
+        ops, live, nid = [], [], 0
+        for step in range(60):
+            u = rng.random()
+            if u < 0.4 or not live:
+                toks = prefixes[int(rng.integers(0, 3))] + rng.integers(0, 5, size=int(rng.integers(0, 2 * bs))).tolist()
+                ops.append(("add_cached", nid, toks))
+                live.append(nid)
+                nid += 1
+            elif u < 0.7:
+                ops.append(("append", [live[int(rng.integers(0, len(live)))]]))
+            else:
+                ops.append(("free", live.pop(int(rng.integers(0, len(live))))))
+        # run until the first failure on the oracle side, which must fail identically in C++
+        from oracle.prefix_cache import PrefixCachingModel
+        from oracle.block_manager import NoFreeBlocks
+        cpp = B.BlockManager(nb, bs, order)
+        ref = PrefixCachingModel(nb, bs, order)
+        for op in ops:
+            try:
+                if op[0] == "add_cached":
+                    exp = ref.add_seq_cached(op[1], op[2])
+                elif op[0] == "append":
+                    exp = ref.append_slot(op[1][0])[0]
+                else:
+                    exp = ref.free_seq(op[1])
+                ok = True
+            except NoFreeBlocks:
+                ok = False
+            if op[0] == "add_cached":
+                if ok:
+                    got = cpp.add_seq_cached(op[1], op[2])
+                    assert got[0].tolist() == exp[0] and got[1] == exp[1]
+                else:
+                    with pytest.raises(B.PagedAttnError):
+                        cpp.add_seq_cached(op[1], op[2])
+                    break
+            elif op[0] == "append":
+                if ok:
+                    assert cpp.append_slot(op[1][0])[0] == exp
+                else:
+                    with pytest.raises(B.PagedAttnError):
+                        cpp.append_slot(op[1][0])
+                    break
+            else:
+                cpp.free_seq(op[1])
+            assert cpp.free_list().tolist() == list(ref.free)
+            assert cpp.prefix_stats() == ref.prefix_stats()

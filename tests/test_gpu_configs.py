@@ -73,3 +73,21 @@ def test_long_context_split(P):
     r.check_outputs()
     if P == 512:
         r.check_pool_rows()
+
+
+def test_prefix_caching_trace():
+    """Requests sharing system prompts: cached whole blocks are reused (their rows
+    are not written again) and evicted under a small pool; slots, tables and every
+    decode output match the oracle."""
+    tr = W.prefix_caching()
+    r = Replay(tr.shape, tr.num_blocks, tr.free_order, 1.0 / np.sqrt(128), keep_pool=True)
+    for op in W.prefix_ops(tr):
+        r.apply(op)
+        if op[0] == "decode":
+            r.check_outputs()
+            r.decodes.clear()
+    assert r.n_cached > 0
+    st, info = B.pa_get_device_error()
+    assert st == B.PA_OK, (st, info)
+    r.check_pool_rows()
+    assert r.cache.bm.prefix_stats() == r.oracle.bm.prefix_stats()

@@ -129,12 +129,13 @@ def test_decode_bad_block_id_and_length_are_reported():
     q = torch.randn(1, 1, 64, device="cuda").bfloat16()
     out = torch.empty(1, 1, 64, device="cuda")
     tables = torch.tensor([[0, 9]], dtype=torch.int32, device="cuda")
+    ws = torch.empty(B.pa_decode_workspace_bytes(1, 1, 1, 64, 32, 16, 0), dtype=torch.uint8, device="cuda")
     B.pa_decode(q, cache.k_cache, cache.v_cache, tables, torch.tensor([20], dtype=torch.int32, device="cuda"),
-                0.1, out, 32, 0)
+                0.1, out, 32, 0, ws)
     st, info = B.pa_get_device_error()
     assert st == B.PA_ERR_DEVICE_BOUNDS and info == 9
     B.pa_decode(q, cache.k_cache, cache.v_cache, tables, torch.tensor([40], dtype=torch.int32, device="cuda"),
-                0.1, out, 32, 0)
+                0.1, out, 32, 0, ws)
     st, info = B.pa_get_device_error()
     assert st == B.PA_ERR_DEVICE_BOUNDS and info == 40
 
@@ -195,3 +196,46 @@ def test_step_host_rejects_small_staging_without_change():
         B.pa_step_host(cache.bm, cache.k_cache, cache.v_cache, [0], q, k, k, 0.1, out, tiny_dev, tiny_host)
     assert e.value.status == B.PA_ERR_INVALID_ARG
     assert cache.bm.block_table(0)[1] == 3
+
+
+def test_swap_out_reuse_swap_in_decode():
+    """P2 §五: a sequence's blocks move to a pinned host pool, other sequences
+    reuse the released device blocks, the sequence comes back into fresh blocks
+    and decodes exactly as before."""
+    from oracle.replay import OracleRun
+    g = torch.Generator().manual_seed(5)
+    sh = W.Shape(8, 2, 128, 16, "bf16")
+    cache = PagedKVCache(12, 2, 16, 128, torch.bfloat16, "cuda", list(range(12)), fill=float("nan"))
+    cache.enable_swap(16)
+    rows = {s: (torch.randn(70, 2, 128, generator=g).bfloat16(), torch.randn(70, 2, 128, generator=g).bfloat16())
+            for s in (1, 2)}
+    for s in (1, 2):
+        cache.add_sequence(s, rows[s][0][:40].cuda(), rows[s][1][:40].cuda())
+    dev_blocks = cache.bm.block_table(1)[0].tolist()
+    before = cache.k_cache[dev_blocks].cpu()
+    pairs = cache.swap_out(1)
+    assert pairs[:, 0].tolist() == dev_blocks
+    torch.cuda.synchronize()
+    assert torch.equal(bits(cache.host_k[pairs[:, 1].tolist()]), bits(before))
+    # sequence 3 takes every free block, the released ones included, and overwrites them
+    junk = torch.randn(144, 2, 128, generator=g).bfloat16()
+    cache.add_sequence(3, junk.cuda(), junk.cuda())
+    assert set(cache.bm.block_table(3)[0].tolist()) & set(dev_blocks)
+    cache.free(2)
+    back = cache.swap_in(1)
+    assert back[:, 0].tolist() == pairs[:, 1].tolist()
+    q = torch.randn(1, 8, 128, generator=g).bfloat16()
+    out = cache.decode([1], q.cuda(), 128 ** -0.5).cpu()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    from oracle.attention import decode_attention
+    ref = decode_attention(q[0], rows[1][0][:40], rows[1][1][:40], 128 ** -0.5)
+    assert float(np.abs(out[0].double().numpy() - ref).max()) <= TOL["bf16"]
+
+
+def test_swap_blocks_rejects_pageable_host_memory():
+    kc = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
+    hk = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16)      # pageable
+    pairs = torch.tensor([[0, 1]], dtype=torch.int32, device="cuda")
+    with pytest.raises(B.PagedAttnError) as e:
+        B.pa_swap_blocks(kc, kc, hk, hk, pairs, True)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
