@@ -168,6 +168,31 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
                     int32_t max_context_len, float scale, float* out, int32_t partition_tokens, void* workspace,
                     size_t workspace_bytes, pa_stream stream);
 
+/*
+ * Causal attention of newly written prompt tokens (prefill, possibly in
+ * chunks) over the paged cache. P2 §3.2.1: the prompt's K, V are computed and
+ * written into the sequence's blocks (pa_reshape_and_cache first); each new
+ * token attends, through the block table, to every position of its sequence up
+ * to and including its own (P2 §1.1 formula, §2.3 table walk).
+ *
+ *   q              device bf16 [T][num_q_heads][head_dim], the new tokens of
+ *                  all sequences back to back (T = cu_q_lens[num_seqs]).
+ *   cu_q_lens      device int32 [num_seqs + 1]: sequence s owns rows
+ *                  cu_q_lens[s] .. cu_q_lens[s+1]-1; n_s = their count.
+ *   max_q_len      host bound on every n_s; it sizes the launch.
+ *   context_lens   device int32 [num_seqs]: length L_s including the new
+ *                  tokens; new token i of s sits at position L_s - n_s + i and
+ *                  sees positions 0 .. L_s - n_s + i. n_s > L_s or L_s above
+ *                  max_context_len is clamped and recorded (PA_ERR_DEVICE_BOUNDS).
+ *   out            device fp32 [T][num_q_heads][head_dim].
+ * Supported: bf16 cache, block_size >= 8 (16, 32 as for decode), head_dim 64
+ * or 128, num_q_heads / num_kv_heads in {1, 2, 4, 8}; fp32 caches return
+ * PA_ERR_UNSUPPORTED. Accumulation is fp32 on the tensor cores.
+ */
+pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, int32_t max_q_len, int32_t num_q_heads,
+                     const pa_cache* cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* context_lens, int32_t max_context_len, float scale, float* out, pa_stream stream);
+
 /* The partition size pa_decode uses for partition_tokens = -1 with these
  * sizes (0 = no split). */
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,

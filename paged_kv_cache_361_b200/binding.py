@@ -46,6 +46,7 @@ _SIGS = {
     "pa_copy_blocks": (_I32, [_PCACHE, _VP, _I32, _VP]),
     "pa_decode": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP, _SZ, _VP]),
     "pa_decode_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
+    "pa_prefill": (_I32, [_VP, _I32, _VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _VP]),
     "pa_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_get_device_error": (_I32, [_VP, _P64]),
     "pa_selftest_wait_timeout": (_I32, [_I64, _VP]),
@@ -175,6 +176,27 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_c
     _check(_lib().pa_decode(q.data_ptr(), B, hq, ctypes.byref(c), block_tables.data_ptr(),
                             int(block_tables.shape[1]), context_lens.data_ptr(), int(max_context_len), float(scale),
                             out.data_ptr(), int(partition_tokens), ws_ptr, ws_bytes, _stream(q, stream)), "pa_decode")
+
+
+def pa_prefill(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale, out, max_q_len, max_context_len,
+               stream=None):
+    """Causal attention of the new tokens q [T][Hq][D] (sequence s owns rows
+    cu_q_lens[s]..cu_q_lens[s+1]-1) over the paged cache; out fp32 [T][Hq][D]."""
+    c = make_cache(k_cache, v_cache)
+    T, hq, d = q.shape
+    _dev(q, "q", k_cache.dtype, 3)
+    _dev(out, "out", torch.float32, 3)
+    if d != c.head_dim or tuple(out.shape) != (T, hq, d):
+        raise ValueError("q/out shape mismatch")
+    _dev(cu_q_lens, "cu_q_lens", torch.int32, 1)
+    _dev(block_tables, "block_tables", torch.int32, 2)
+    _dev(context_lens, "context_lens", torch.int32, 1)
+    B = int(context_lens.shape[0])
+    if cu_q_lens.shape[0] != B + 1 or block_tables.shape[0] != B:
+        raise ValueError("cu_q_lens must have num_seqs + 1 entries, block_tables num_seqs rows")
+    _check(_lib().pa_prefill(q.data_ptr(), B, cu_q_lens.data_ptr(), int(max_q_len), hq, ctypes.byref(c),
+                             block_tables.data_ptr(), int(block_tables.shape[1]), context_lens.data_ptr(),
+                             int(max_context_len), float(scale), out.data_ptr(), _stream(q, stream)), "pa_prefill")
 
 
 def pa_get_device_error(stream=None):

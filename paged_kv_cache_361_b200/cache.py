@@ -157,6 +157,42 @@ class PagedKVCache:
                     max_len, partition_tokens, self.workspace(nbytes))
         return out
 
+    def prefill(self, seq_ids, counts, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+        """Chunked prefill: sequence seq_ids[i] takes counts[i] new tokens (a new
+        sequence is created; a live one grows, with copy-on-write if it shares
+        its last block). Rows of q, k, v are the new tokens of all sequences
+        back to back. Writes K/V (pa_reshape_and_cache), then runs causal
+        attention of the new tokens (pa_prefill); returns fp32 [T][Hq][D]."""
+        counts = [int(c) for c in counts]
+        T, hq, d = q.shape
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        slots_all, pairs_all = [], []
+        for s, n in zip(seq_ids, counts):
+            if s in self.lens:
+                sl, pr = self.bm.append_slots([s] * n)
+                self.lens[s] += n
+                if len(pr):
+                    pairs_all.append(pr)
+            else:
+                sl = self.bm.add_seq(s, n)
+                self.lens[s] = n
+            slots_all.append(sl)
+        if pairs_all:
+            B.pa_copy_blocks(self.k_cache, self.v_cache, self._pairs.upload(np.concatenate(pairs_all)))
+        slots = np.concatenate(slots_all) if slots_all else np.empty(0, np.int64)
+        if len(slots):
+            B.pa_reshape_and_cache(k, v, self._slots.upload(slots), self.k_cache, self.v_cache)
+        tables, lens, max_len = self.decode_inputs(seq_ids)
+        cu = np.zeros(len(counts) + 1, dtype=np.int32)
+        cu[1:] = np.cumsum(counts)
+        if out is None:
+            out = torch.empty((T, hq, d), dtype=torch.float32, device=self.device)
+        B.pa_prefill(q, self._lens.upload(cu), self.k_cache, self.v_cache, self._tables.upload(tables),
+                     self._lens.upload(lens), scale, out, max(counts, default=0), max_len)
+        return out
+
     def step_host(self, seq_ids, q_host, k_host, v_host, out_host, scale=None, partition_tokens=-1):
         """One decode step from host tensors (pinned for asynchronous copies):
         block-manager work, copies and kernels in one native call

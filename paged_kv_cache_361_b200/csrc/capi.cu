@@ -9,6 +9,7 @@
 #include "cache_ops.cuh"
 #include "decode_mma.cuh"
 #include "decode_simt.cuh"
+#include "prefill_mma.cuh"
 
 namespace {
 
@@ -316,6 +317,75 @@ pa_status pa_swap_blocks(const pa_cache* cache, void* host_k, void* host_v, int6
       sk, sv, dk, dv, pairs, n_pairs, chunks, static_cast<int32_t>(bpp), to_host ? cache->num_blocks : host_num_blocks,
       to_host ? host_num_blocks : cache->num_blocks);
   return launched();
+}
+
+pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, int32_t max_q_len, int32_t num_q_heads,
+                     const pa_cache* cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* context_lens, int32_t max_context_len, float scale, float* out, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || max_q_len < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int G = num_q_heads / cache->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (cache->dtype != PA_BF16 || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * cache->block_size ||
+      max_q_len > max_context_len)
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || max_q_len == 0) return PA_OK;
+  if (!q || !cu_q_lens || !block_tables || !context_lens || !out || !aligned16(q) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(cu_q_lens) & 3) || (reinterpret_cast<uintptr_t>(block_tables) & 3) ||
+      (reinterpret_cast<uintptr_t>(context_lens) & 3))
+    return PA_ERR_INVALID_ARG;
+  const int tt = 64 / G;
+  const int64_t ntiles = (static_cast<int64_t>(max_q_len) + tt - 1) / tt;
+  if (num_seqs > 65535 || ntiles > 65535) return PA_ERR_UNSUPPORTED;
+  PrefillArgs a;
+  a.q = q;
+  a.cu_q = cu_q_lens;
+  a.tables = block_tables;
+  a.lens = context_lens;
+  a.out = out;
+  a.num_blocks = cache->num_blocks;
+  a.num_seqs = num_seqs;
+  a.hq = num_q_heads;
+  a.hkv = cache->num_kv_heads;
+  a.bs = cache->block_size;
+  a.max_blocks = max_blocks_per_seq;
+  a.max_ctx = max_context_len;
+  a.ntiles = static_cast<int32_t>(ntiles);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  CUtensorMap tk, tv;
+  const uint64_t rows = static_cast<uint64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
+  if (!encode_rows(&tk, cache->k, rows, cache->head_dim, cache->block_size) ||
+      !encode_rows(&tv, cache->v, rows, cache->head_dim, cache->block_size))
+    return PA_ERR_CUDA;
+  const dim3 grid(cache->num_kv_heads, static_cast<unsigned>(ntiles), num_seqs);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto launch = [&](auto kern, int smem) -> pa_status {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return PA_ERR_CUDA;
+    kern<<<grid, MmaCfg<128>::kThreads, smem, s>>>(tk, tv, a);
+    return launched();
+  };
+  if (cache->head_dim == 128) {
+    switch (G) {
+      case 1: return launch(prefill_mma_kernel<128, 1>, MmaCfg<128>::kSmemBytes);
+      case 2: return launch(prefill_mma_kernel<128, 2>, MmaCfg<128>::kSmemBytes);
+      case 4: return launch(prefill_mma_kernel<128, 4>, MmaCfg<128>::kSmemBytes);
+      default: return launch(prefill_mma_kernel<128, 8>, MmaCfg<128>::kSmemBytes);
+    }
+  }
+  switch (G) {
+    case 1: return launch(prefill_mma_kernel<64, 1>, MmaCfg<64>::kSmemBytes);
+    case 2: return launch(prefill_mma_kernel<64, 2>, MmaCfg<64>::kSmemBytes);
+    case 4: return launch(prefill_mma_kernel<64, 4>, MmaCfg<64>::kSmemBytes);
+    default: return launch(prefill_mma_kernel<64, 8>, MmaCfg<64>::kSmemBytes);
+  }
 }
 
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,

@@ -1,0 +1,257 @@
+// Paged prefill attention (causal) on the tensor cores.
+//
+// P2 = "PagedAttention：操作系统级 KV 缓存虚拟内存管理".
+//   §3.2.1  prefill: the prompt's tokens are processed together and their K, V
+//           written into the sequence's blocks (pa_reshape_and_cache); here
+//           each new token attends, causally, to every earlier position of its
+//           sequence through the block table (§2.3) with out =
+//           softmax(scale * q K^T) V (§1.1). A chunk of n new tokens of a
+//           sequence of length L sits at positions L-n .. L-1 (chunked prefill).
+//
+// B200 design: CTA = (kv head g, query tile, sequence). A tile is 64 MMA rows,
+// row r = (token tok0 + r / G, query head g*G + r % G), so all G heads sharing
+// a kv head ride in one M dimension and every K/V tile read serves 64 rows.
+// Warp 4 is the TMA producer (the decode pipeline: swizzled [bs x 64] boxes of
+// K and V, 64 keys per stage, keys 0 .. the tile's last position); warps 0-3
+// each own 16 rows and run S = Q K^T and O += P V as full m16n8k16 bf16 MMAs,
+// with P split into a bf16 high part and remainder. The causal mask is applied
+// per row; a warp skips chunks that lie entirely past its rows' positions.
+// Tiles are dispatched last-first (the longest key ranges start first).
+#pragma once
+
+#include "decode_mma.cuh"
+
+namespace pa {
+
+struct PrefillArgs {
+  const void* q;          // [T][hq][D] bf16
+  const int32_t* cu_q;    // [num_seqs + 1] prefix sums of new-token counts
+  const int32_t* tables;  // [num_seqs][max_blocks]
+  const int32_t* lens;    // [num_seqs] context length including the new tokens
+  float* out;             // [T][hq][D]
+  int64_t num_blocks;
+  int32_t num_seqs, hq, hkv, bs, max_blocks, max_ctx, ntiles;
+  float scale_log2;
+};
+
+// d += A(16x16) * B(16x8), all 16 rows live.
+__device__ __forceinline__ void mma16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                      uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const __grid_constant__ CUtensorMap tmk,
+                                                                         const __grid_constant__ CUtensorMap tmv,
+                                                                         const PrefillArgs a) {
+  using Cfg = MmaCfg<D>;
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = D / 8;
+  constexpr int TT = 64 / G;  // tokens per tile
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ PipeSmem<S> ps;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+
+  const int g = blockIdx.x, s = blockIdx.z;
+  const int tile = a.ntiles - 1 - static_cast<int>(blockIdx.y);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int32_t q0 = __ldg(a.cu_q + s);
+  int32_t n = __ldg(a.cu_q + s + 1) - q0;
+  int32_t L = __ldg(a.lens + s);
+  if (L < 0 || L > a.max_ctx || n < 0 || n > L) {
+    if (tid == 0 && g == 0 && tile == 0) record_error(PA_ERR_DEVICE_BOUNDS, L);
+    L = L < 0 ? 0 : (L > a.max_ctx ? a.max_ctx : L);
+    n = n < 0 ? 0 : (n > L ? L : n);
+  }
+  const int32_t tok0 = tile * TT;
+  if (tok0 >= n) return;
+  const int32_t tok_end = min(tok0 + TT, n);
+  const int32_t base = L - n;              // position of new token 0
+  const int32_t kend = base + tok_end;     // keys 0 .. kend-1 are needed
+  const int nchunks = (kend + C - 1) / C;
+
+  if (tid == 0) pipe_init<S>(ps, NW);
+  __syncthreads();
+
+  if (warp == NW) {
+    const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
+    const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
+    pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+      const int32_t c0 = i * C;
+      const int32_t nb = (min(C, kend - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+      int32_t blk = -1;
+      bool ok = false;
+      if (lane < nb) {
+        blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
+        ok = blk >= 0 && blk < a.num_blocks;
+        if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * Cfg::kHalves * __popc(okmask) * box_bytes);
+      __syncwarp();
+      if (ok) {
+        const int32_t y = (blk * a.hkv + g) * a.bs;
+        const uint32_t kdst = sbase + st * Cfg::kStageBytes + lane * box_bytes;
+#pragma unroll
+        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+          tma_load_2d(kdst + hf * Cfg::kHalfBytes, &tmk, hf * 64, y, &ps.full[st], pol);
+          tma_load_2d(kdst + Cfg::kTileBytes + hf * Cfg::kHalfBytes, &tmv, hf * 64, y, &ps.full[st], pol);
+        }
+      }
+    });
+    return;
+  }
+
+  // ---- consumers: warp w owns tile rows [16w, 16w+16); this lane rows ra, rb = ra + 8 ----
+  const int c = lane & 3;
+  const int ra = warp * 16 + (lane >> 2), rb = ra + 8;
+  const int ta = tok0 + ra / G, tb = tok0 + rb / G;
+  const bool va = ta < n, vb = tb < n;
+  const int pa_ = va ? base + ta : -1, pb_ = vb ? base + tb : -1;  // last key each row may see
+  const int wmax = base + min(tok0 + (warp * 16 + 15) / G, n - 1);  // last key any row of this warp sees
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q);
+  const uint32_t* qra = reinterpret_cast<const uint32_t*>(
+      qb + ((static_cast<int64_t>(q0) + (va ? ta : 0)) * a.hq + g * G + ra % G) * D);
+  const uint32_t* qrb = reinterpret_cast<const uint32_t*>(
+      qb + ((static_cast<int64_t>(q0) + (vb ? tb : 0)) * a.hq + g * G + rb % G) * D);
+  uint32_t qa[D / 16][4];
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    qa[kk][0] = va ? __ldg(qra + kk * 8 + c) : 0u;
+    qa[kk][1] = vb ? __ldg(qrb + kk * 8 + c) : 0u;
+    qa[kk][2] = va ? __ldg(qra + kk * 8 + 4 + c) : 0u;
+    qa[kk][3] = vb ? __ldg(qrb + kk * 8 + 4 + c) : 0u;
+  }
+  float o[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+
+  const int mk = lane >> 3, ik = lane & 7;
+  for (int i = 0; i < nchunks; ++i) {
+    const int st = i % S;
+    if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
+    const int k0 = i * C;
+    if (k0 <= wmax) {
+      const uint32_t kst = sbase + st * Cfg::kStageBytes;
+      const uint32_t vst = kst + Cfg::kTileBytes;
+      float sacc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int d0 = kk * 16 + (mk & 1) * 8;
+#pragma unroll
+        for (int kg = 0; kg < 4; ++kg) {
+          const int tk = kg * 16 + (mk >> 1) * 8 + ik;
+          const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tk * 128 + ((((d0 & 63) >> 3) ^ (tk & 7)) << 4);
+          uint32_t b00, b01, b10, b11;
+          ldsm_x4(addr, b00, b01, b10, b11);
+          mma16(sacc[2 * kg], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b00, b01);
+          mma16(sacc[2 * kg + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b10, b11);
+        }
+      }
+      // causal mask and online softmax for rows ra (c0, c1) and rb (c2, c3)
+      float mla = -INFINITY, mlb = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int key = k0 + nt * 8 + 2 * c + j;
+          sacc[nt][j] = key <= pa_ ? sacc[nt][j] * a.scale_log2 : -INFINITY;
+          sacc[nt][2 + j] = key <= pb_ ? sacc[nt][2 + j] * a.scale_log2 : -INFINITY;
+          mla = fmaxf(mla, sacc[nt][j]);
+          mlb = fmaxf(mlb, sacc[nt][2 + j]);
+        }
+      mla = fmaxf(mla, __shfl_xor_sync(0xffffffffu, mla, 1));
+      mla = fmaxf(mla, __shfl_xor_sync(0xffffffffu, mla, 2));
+      mlb = fmaxf(mlb, __shfl_xor_sync(0xffffffffu, mlb, 1));
+      mlb = fmaxf(mlb, __shfl_xor_sync(0xffffffffu, mlb, 2));
+      const float na = fmaxf(ma, mla), nb = fmaxf(mb, mlb);
+      // a row with nothing visible yet keeps m = -inf; its weights are 0
+      const float alpha_a = na == -INFINITY ? 1.f : exp2f(ma - na);
+      const float alpha_b = nb == -INFINITY ? 1.f : exp2f(mb - nb);
+      float suma = 0.f, sumb = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          sacc[nt][j] = na == -INFINITY ? 0.f : exp2f(sacc[nt][j] - na);
+          sacc[nt][2 + j] = nb == -INFINITY ? 0.f : exp2f(sacc[nt][2 + j] - nb);
+          suma += sacc[nt][j];
+          sumb += sacc[nt][2 + j];
+        }
+      ma = na;
+      mb = nb;
+      la = la * alpha_a + suma;
+      lb = lb * alpha_b + sumb;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        o[j][0] *= alpha_a;
+        o[j][1] *= alpha_a;
+        o[j][2] *= alpha_b;
+        o[j][3] *= alpha_b;
+      }
+      // O += P V, 16 keys (n-tiles 2kg, 2kg+1) per k-step; V rows past kend are zeroed
+      const int nvk = min(C, kend - k0);
+#pragma unroll
+      for (int kg = 0; kg < 4; ++kg) {
+        uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
+        split_pair(sacc[2 * kg][0], sacc[2 * kg][1], h0, l0);          // row ra, keys 2c, 2c+1
+        split_pair(sacc[2 * kg][2], sacc[2 * kg][3], h1, l1);          // row rb
+        split_pair(sacc[2 * kg + 1][0], sacc[2 * kg + 1][1], h2, l2);  // row ra, keys +8
+        split_pair(sacc[2 * kg + 1][2], sacc[2 * kg + 1][3], h3, l3);  // row rb, keys +8
+        const int kb = kg * 16;
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+        if (kb + 16 > nvk) {
+          mlo = (kb + 2 * c < nvk ? 0x0000ffffu : 0u) | (kb + 2 * c + 1 < nvk ? 0xffff0000u : 0u);
+          mhi = (kb + 2 * c + 8 < nvk ? 0x0000ffffu : 0u) | (kb + 2 * c + 9 < nvk ? 0xffff0000u : 0u);
+        }
+        const int tv = kb + (mk & 1) * 8 + ik;
+#pragma unroll
+        for (int dg = 0; dg < D / 16; ++dg) {
+          const int d0 = dg * 16 + (mk >> 1) * 8;
+          const uint32_t addr = vst + (d0 >> 6) * Cfg::kHalfBytes + tv * 128 + ((((d0 & 63) >> 3) ^ (tv & 7)) << 4);
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_t(addr, v0, v1, v2, v3);
+          v0 &= mlo;
+          v1 &= mhi;
+          v2 &= mlo;
+          v3 &= mhi;
+          mma16(o[2 * dg], h0, h1, h2, h3, v0, v1);
+          mma16(o[2 * dg], l0, l1, l2, l3, v0, v1);
+          mma16(o[2 * dg + 1], h0, h1, h2, h3, v2, v3);
+          mma16(o[2 * dg + 1], l0, l1, l2, l3, v2, v3);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ps.empty[st]);
+  }
+  if (ps.abort_flag) return;
+
+  la += __shfl_xor_sync(0xffffffffu, la, 1);
+  la += __shfl_xor_sync(0xffffffffu, la, 2);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+  if (va) {
+    const float inv = 1.f / la;
+    float* dst = a.out + ((static_cast<int64_t>(q0) + ta) * a.hq + g * G + ra % G) * D + 2 * c;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0] * inv, o[j][1] * inv);
+  }
+  if (vb) {
+    const float inv = 1.f / lb;
+    float* dst = a.out + ((static_cast<int64_t>(q0) + tb) * a.hq + g * G + rb % G) * D + 2 * c;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][2] * inv, o[j][3] * inv);
+  }
+}
+
+}  // namespace pa

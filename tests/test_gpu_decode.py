@@ -239,3 +239,52 @@ def test_swap_blocks_rejects_pageable_host_memory():
     with pytest.raises(B.PagedAttnError) as e:
         B.pa_swap_blocks(kc, kc, hk, hk, pairs, True)
     assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_prefill_chunked_matches_oracle(G, D, bs):
+    """Chunked prefill: existing sequences grow by a chunk, new ones start; every
+    new token's causal attention over the paged cache matches the oracle."""
+    from oracle.prefill import prefill_attention
+    rng = np.random.default_rng(G * 1000 + D + bs)
+    hkv = 2
+    nseq = 5
+    pre = rng.integers(0, 300, size=nseq)
+    pre[0] = 0
+    chunk = rng.integers(1, 200, size=nseq)
+    chunk[1] = 64 // G            # exactly one query tile
+    nb = int(sum(-(-int(p + c) // bs) for p, c in zip(pre, chunk))) + 4
+    cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, "cuda", rng.permutation(nb), fill=float("nan"))
+    g = torch.Generator().manual_seed(int(rng.integers(1 << 30)))
+    K = {s: torch.randn(int(pre[s] + chunk[s]), hkv, D, generator=g).bfloat16() for s in range(nseq)}
+    V = {s: torch.randn(int(pre[s] + chunk[s]), hkv, D, generator=g).bfloat16() for s in range(nseq)}
+    for s in range(nseq):
+        if pre[s]:
+            cache.add_sequence(s, K[s][:pre[s]].cuda(), V[s][:pre[s]].cuda())
+    q = torch.randn(int(chunk.sum()), hkv * G, D, generator=g).bfloat16()
+    k_new = torch.cat([K[s][pre[s]:] for s in range(nseq)])
+    v_new = torch.cat([V[s][pre[s]:] for s in range(nseq)])
+    out = cache.prefill(list(range(nseq)), chunk, q.cuda(), k_new.cuda(), v_new.cuda(), D ** -0.5).cpu()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    row = 0
+    for s in range(nseq):
+        n = int(chunk[s])
+        ref = prefill_attention(q[row:row + n], K[s], V[s], D ** -0.5)
+        err = float(np.abs(out[row:row + n].double().numpy() - ref).max())
+        assert err <= TOL["bf16"], f"seq {s}: {err}"
+        row += n
+
+
+def test_prefill_then_decode_consistent():
+    """The last token of a whole-prompt prefill equals a decode over the same cache."""
+    sh = (4, 128, 16)
+    cache = PagedKVCache(64, 4, 16, 128, torch.bfloat16, "cuda", fill=float("nan"))
+    g = torch.Generator().manual_seed(9)
+    k = torch.randn(300, 4, 128, generator=g).bfloat16().cuda()
+    v = torch.randn(300, 4, 128, generator=g).bfloat16().cuda()
+    q = torch.randn(300, 16, 128, generator=g).bfloat16().cuda()
+    out = cache.prefill([7], [300], q, k, v, 128 ** -0.5)
+    dec = cache.decode([7], q[-1:], 128 ** -0.5)
+    assert float((out[-1] - dec[0]).abs().max()) <= 2e-3
