@@ -134,23 +134,27 @@ def workload_ops(name, seed):
     return tr.shape, tr.num_blocks, tr.free_order, 1.0 / math.sqrt(tr.shape.head_dim), 0, W.batching_ops(tr, steps=1)
 
 
-def build_workload(seed: int, device, name: str = "llama2_7b_mha"):
+def build_workload(seed: int, device, name: str = "llama2_7b_mha", kv_dtype: str = "auto"):
     """Replays the workload's operation script up to the measured step through
     PagedKVCache: the pool is filled with N(0,1) values on the device (they
     stand in for the prompts' K/V, so prefills only reserve blocks), forks
     share blocks, earlier appends write random rows (with their copy-on-write
     block copies). The measured step's slots and pairs come from the C++ block
-    manager; its tables and lengths are uploaded once."""
+    manager; its tables and lengths are uploaded once.
+
+    kv_dtype "fp8" stores the cache as e4m3 codes (per-tensor scales 1.0: the
+    N(0,1) values are inside the e4m3 range); q and the new K/V rows stay bf16."""
     from paged_kv_cache_361_b200 import PagedKVCache
     from paged_kv_cache_361_b200 import workloads as W
     sh, nb, order, scale, part, ops = workload_ops(name, seed)
     dt = W.TORCH_DTYPE[sh.dtype]
-    cache = PagedKVCache(nb, sh.num_kv_heads, sh.block_size, sh.head_dim, dt, device, order)
+    cache_dt = torch.float8_e4m3fn if kv_dtype == "fp8" else dt
+    cache = PagedKVCache(nb, sh.num_kv_heads, sh.block_size, sh.head_dim, cache_dt, device, order)
     g = torch.Generator(device=device)
     g.manual_seed(1000 + seed)
     for t in (cache.k_cache, cache.v_cache):
         for i in range(0, nb, 1024):   # chunked to bound the fp32 temporary
-            t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(dt)
+            t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(cache_dt)
     hkv, D = sh.num_kv_heads, sh.head_dim
     assert ops[-2][0] == "append" and ops[-1][0] == "decode"
     for op in ops[:-2]:
@@ -170,7 +174,7 @@ def build_workload(seed: int, device, name: str = "llama2_7b_mha"):
         cache.lens[s] += 1
     tables, lens32, max_len = cache.decode_inputs(ids)
     B_, hq = len(ids), sh.num_q_heads
-    eb = 2 if sh.dtype == "bf16" else 4
+    eb = cache.k_cache.element_size()
     st = cache.bm.stats()
     return dict(
         name=name, shape=sh, scale=scale, part=part, ids=ids, cache=cache, bm=cache.bm, kc=cache.k_cache,
@@ -190,6 +194,24 @@ def build_workload(seed: int, device, name: str = "llama2_7b_mha"):
     )
 
 
+def cascade_inputs(d, device):
+    """Group arguments of pa_decode_cascade for the measured step (host work
+    done once, before timing): sequences whose tables start with the same
+    blocks share their common prefix."""
+    from paged_kv_cache_361_b200 import binding as B
+    cache, sh = d["cache"], d["shape"]
+    tables = d["tables"].cpu().numpy()
+    lens = d["lens"].cpu().numpy()
+    offs, members, prefix, seq_prefix = cache.shared_prefix_groups(d["ids"], tables, lens,
+                                                                   64 // sh.group)
+    max_pre = int(prefix.max()) if len(prefix) else 0
+    nbytes = B.pa_decode_cascade_workspace_bytes(len(d["ids"]), sh.num_q_heads, sh.num_kv_heads, sh.head_dim,
+                                                 d["max_len"], sh.block_size, max_pre)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+    return (t(offs), t(members), t(prefix), t(seq_prefix), int(max(np.diff(offs), default=0)), max_pre, ws)
+
+
 def sample_rows(d, seqs):
     """Host copies (before any kernel runs) of the sampled sequences' K/V rows,
     read from the device pool through their block tables: input to the CPU
@@ -203,21 +225,22 @@ def sample_rows(d, seqs):
         t = torch.arange(L_old)
         blk = torch.as_tensor(table, dtype=torch.int64)[t // bs].to(d["kc"].device)
         off = (t % bs).to(d["kc"].device)
-        K = torch.cat([d["kc"][blk, :, off, :], d["k"][s:s + 1]]).cpu()
-        V = torch.cat([d["vc"][blk, :, off, :], d["v"][s:s + 1]]).cpu()
+        K = torch.cat([d["kc"][blk, :, off, :].float(), d["k"][s:s + 1].float()]).cpu()
+        V = torch.cat([d["vc"][blk, :, off, :].float(), d["v"][s:s + 1].float()]).cpu()
         rows.append((s, K, V, d["q"][s].cpu()))
     return rows
 
 
-def time_oracle(rows, scale, budget_s):
+def time_oracle(rows, scale, budget_s, elem_bytes=2):
     """Runs the CPU oracle over the sampled sequences (repeating the sample)
-    until budget_s has passed; returns (GB/s, seconds, sequences done)."""
+    until budget_s has passed; returns (GB/s, seconds, sequences done); bytes
+    are counted at the cache's element size."""
     from oracle.attention import decode_attention
     done_bytes, n, t0 = 0, 0, time.perf_counter()
     while True:
         for s, K, V, q in rows:
             decode_attention(q, K, V, scale)
-            done_bytes += K.numel() * 2 * 2
+            done_bytes += K.numel() * elem_bytes * 2
             n += 1
             if time.perf_counter() - t0 >= budget_s:
                 el = time.perf_counter() - t0
@@ -240,9 +263,12 @@ def cpu_threads():
 
 def run_ours(args, rank, world, device):
     from paged_kv_cache_361_b200 import binding as B
-    d = build_workload(seed=rank, device=device, name=args.workload)
+    d = build_workload(seed=rank, device=device, name=args.workload, kv_dtype=args.kv_dtype)
     sh = d["shape"]
     nseq = len(d["ids"])
+    cascade = None
+    if args.cascade:
+        cascade = cascade_inputs(d, device)
     P = args.partition if args.partition != -2 else d["part"]
     ws_bytes = B.pa_decode_workspace_bytes(nseq, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, d["max_len"],
                                            sh.block_size, P)
@@ -261,6 +287,10 @@ def run_ours(args, rank, world, device):
         B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
 
     def decode():
+        if cascade is not None:
+            B.pa_decode_cascade(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"],
+                                *cascade)
+            return
         B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"], P, ws)
 
     for _ in range(args.warmup):
@@ -313,7 +343,7 @@ def run_ours(args, rank, world, device):
 
     cpu = None
     if baseline_rows is not None:
-        gbs, el, n = time_oracle(baseline_rows, d["scale"], args.cpu_seconds)
+        gbs, el, n = time_oracle(baseline_rows, d["scale"], args.cpu_seconds, d["kc"].element_size())
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"fp64 NumPy oracle over sequences {sample_seqs} of the workload (all heads), repeated "
                          f"for {el:.1f} s ({n} sequence passes); host has {os.cpu_count()} cores"}
@@ -321,17 +351,26 @@ def run_ours(args, rank, world, device):
     peak, peak_kind = peaks()
     dec_avg_ms = statistics.mean(decode_ms)
     achieved = kv_bytes / (dec_avg_ms * 1e-3) / 1e9
-    launches = args.steps * (2 + (1 if split else 0) + (1 if d["pairs"] is not None else 0))
+    if cascade is not None:
+        split = True
+        n_groups = int(cascade[0].shape[0]) - 1
+        launches = args.steps * (1 + (1 if n_groups else 0) + 2 + (1 if d["pairs"] is not None else 0))
+    else:
+        launches = args.steps * (2 + (1 if split else 0) + (1 if d["pairs"] is not None else 0))
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype, "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3 cache, bf16 q" if args.kv_dtype == "fp8" else sh.dtype, "data": "synthetic",
             "config": {"workload": WORKLOADS[args.workload], "num_seqs": nseq, "num_q_heads": sh.num_q_heads,
                        "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "block_size": sh.block_size,
                        "num_blocks": int(d["kc"].shape[0]), "context_tokens": int(d["lens_host"].sum()),
                        "kv_bytes_per_step": kv_bytes, "unique_kv_bytes_per_step": d["unique_kv_bytes"],
                        "partition_tokens": P_eff,
+                       "kv_dtype": str(d["kc"].dtype).replace("torch.", ""),
+                       "decode": "pa_decode_cascade (shared prefixes read once per group)" if cascade is not None
+                       else "pa_decode",
                        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                        "l2": "no flush: the K/V read per step is larger than the 126 MB L2"
                        if d["unique_kv_bytes"] > 3 * 126e6 else "no flush: K/V partly L2-resident (see unique bytes)"},
@@ -339,7 +378,9 @@ def run_ours(args, rank, world, device):
             "pct_of_hbm_peak": {"of_measured_6540": round(value / peak, 4), "of_nominal_8000": round(value / 8000.0, 4)},
             "e2e": e2e,
             "gpu_launches": launches,
-            "roofline": {"kernel": "pa_decode" + (" (decode + partition merge)" if split else ""), "bound": "hbm",
+            "roofline": {"kernel": ("pa_decode_cascade (prefix + suffix + merge); achieved counts logical K/V bytes"
+                                    if cascade is not None else
+                                    "pa_decode" + (" (decode + partition merge)" if split else "")), "bound": "hbm",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": None,
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
@@ -351,10 +392,11 @@ def run_ours(args, rank, world, device):
 
 
 def run_e2e(args, d, device, world, P):
-    """K steps through PagedKVCache.step_host (the native pa_step_host): per
-    step the block manager appends, the step metadata and q/k/v go host ->
-    device from pinned memory, copy-on-write + append + decode run, and the fp32
-    output comes back to pinned host memory. Context lengths grow by one per step."""
+    """K steps through a prepared pa_step_host call (PagedKVCache.step_plan):
+    per step the C++ block manager appends, the step metadata and q/k/v go host
+    -> device from pinned memory, copy-on-write + append + decode run, and the
+    fp32 output comes back to pinned host memory before the call returns.
+    Context lengths grow by one per step."""
     sh = d["shape"]
     cache = d["cache"]
     ids = d["ids"]
@@ -363,25 +405,29 @@ def run_e2e(args, d, device, world, P):
     hv = d["v"].cpu().pin_memory()
     hout = torch.empty(d["out"].shape, dtype=torch.float32, pin_memory=True)
     eb = hq.element_size()
-    kv_total = h2d = d2h = 0
+    plan = cache.step_plan(ids, hq, hk, hv, hout, d["scale"], partition_tokens=P,
+                           max_context_len=int(max(cache.lens[s] for s in ids)) + args.warmup + args.steps + 1)
+    for _ in range(args.warmup):
+        plan.run()
+    L0 = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64, count=len(ids))
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    for it in range(args.warmup + args.steps):
-        if it == args.warmup:
-            torch.cuda.synchronize(device)
-            if world > 1:
-                torch.distributed.barrier()
-            t0.record()
-            kv_total = h2d = d2h = 0
-        cache.step_host(ids, hq, hk, hv, hout, d["scale"], partition_tokens=P)
-        L = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64, count=len(ids))
-        kv_total += int(L.sum()) * sh.num_kv_heads * sh.head_dim * 2 * eb
-        nblk = int(-(-L.max() // sh.block_size))
-        h2d += (hq.numel() + hk.numel() + hv.numel()) * eb + len(ids) * (8 + 8 + nblk * 4 + 4)
-        d2h += hout.numel() * 4
+    t0.record()
+    for _ in range(args.steps):
+        plan.run()
     t1.record()
     torch.cuda.synchronize(device)
     ms = t0.elapsed_time(t1)
+    # step k attends over L0 + k + 1 tokens per sequence
+    n, K = len(ids), args.steps
+    tokens = int(L0.sum()) * K + n * K * (K + 1) // 2
+    kv_total = tokens * sh.num_kv_heads * sh.head_dim * 2 * cache.k_cache.element_size()
+    nblk = int(-(-(int(L0.max()) + K) // sh.block_size))
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * eb + n * (8 + 8 + nblk * 4 + 4)
+    d2h = hout.numel() * 4
     t = torch.tensor([ms, float(kv_total)], dtype=torch.float64, device=device)
     if world > 1:
         tm = t[:1].clone()
@@ -391,9 +437,95 @@ def run_e2e(args, d, device, world, P):
         ms, kv_total = float(tm.item()), float(tb.item())
     return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "ms_per_step": round(ms / args.steps, 4),
-            "h2d_bytes_per_step": int(h2d // args.steps), "d2h_bytes_per_step": int(d2h // args.steps),
-            "api": "pa_step_host via PagedKVCache.step_host (block manager, one metadata H2D, q/k/v H2D, "
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "api": "pa_step_host via PagedKVCache.step_plan (block manager, one metadata H2D, q/k/v H2D, "
                    "pa_copy_blocks, pa_reshape_and_cache, pa_decode, output D2H, stream sync)"}
+
+
+PREFILL = {
+    "prefill_llama2_7b_mha": (32, 32, 8, 2048),   # Hq, Hkv, sequences, prompt tokens
+    "prefill_gqa8": (64, 8, 2, 8192),
+}
+
+
+def run_prefill(args, rank, world, device):
+    """Whole-prompt prefill (pa_reshape_and_cache of every prompt token +
+    pa_prefill) over a fresh paged cache; metric: causal attention TFLOP/s with
+    4 * head_dim * Hq flops per (query, visible key) pair."""
+    from paged_kv_cache_361_b200 import PagedKVCache, binding as B
+    hq, hkv, nseq, plen = PREFILL[args.workload]
+    D, bs = 128, 16
+    nb = nseq * plen // bs + 16
+    order = np.random.default_rng(rank).permutation(nb)
+    cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, device, order)
+    g = torch.Generator(device=device)
+    g.manual_seed(2000 + rank)
+    T = nseq * plen
+    q = torch.randn(T, hq, D, generator=g, device=device).bfloat16()
+    k = torch.randn(T, hkv, D, generator=g, device=device).bfloat16()
+    v = torch.randn(T, hkv, D, generator=g, device=device).bfloat16()
+    out = cache.prefill(list(range(nseq)), [plen] * nseq, q, k, v)
+    tables, lens, max_len = cache.decode_inputs(list(range(nseq)))
+    slots = torch.from_numpy(np.concatenate([cache.bm.block_table(s)[0].repeat(bs)[:plen].astype(np.int64) * bs
+                                             + np.arange(plen) % bs for s in range(nseq)])).to(device)
+    t = torch.from_numpy(tables).to(device)
+    L = torch.from_numpy(lens).to(device)
+    cu = torch.arange(0, T + 1, plen, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        B.pa_reshape_and_cache(k, v, slots, cache.k_cache, cache.v_cache)
+        B.pa_prefill(q, cu, cache.k_cache, cache.v_cache, t, L, D ** -0.5, out, plen, max_len)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks.start()
+    e0.record(stream)
+    for i in range(args.steps):
+        B.pa_reshape_and_cache(k, v, slots, cache.k_cache, cache.v_cache)
+        ev[i][0].record(stream)
+        B.pa_prefill(q, cu, cache.k_cache, cache.v_cache, t, L, D ** -0.5, out, plen, max_len)
+        ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    st, info = B.pa_get_device_error()
+    if st != B.PA_OK:
+        raise RuntimeError(f"device error {st} ({info})")
+    ms = e0.elapsed_time(e1) / args.steps
+    pf_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = 4.0 * D * hq * nseq * plen * (plen + 1) / 2
+    tm = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
+    ms = float(tm.item())
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+        src = "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    if rank == 0:
+        print(json.dumps({
+            "metric": "paged prefill attention TFLOP/s (causal; 4*head_dim*Hq flops per visible query-key pair)",
+            "value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {nseq} prompts x {plen} tokens, {hq}/{hkv} heads, D128, bs16",
+                       "l2": "no flush: K/V of one launch " + f"{2 * T * hkv * D * 2 / 1e6:.0f} MB"},
+            "gpu_launches": 2 * args.steps,
+            "roofline": {"kernel": "pa_prefill", "bound": "tensor", "achieved": round(flops / (pf_ms * 1e-3) / 1e12, 2),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(flops / (pf_ms * 1e-3) / 1e12 / peak, 4),
+                         "traffic": None, "peak_source": src,
+                         "note": "mma.sync m16n8k16 with P split into two bf16 MMAs (1.5x the algorithmic MMA work)"},
+            "clocks": clk}), flush=True)
 
 
 def run_reference(args, rank, world):
@@ -440,9 +572,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--partition", type=int, default=-1,
                     help="partition_tokens for pa_decode (-1: library choice, -2: the workload's own)")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama2_7b_mha")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL), default="llama2_7b_mha")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--kv-dtype", choices=["auto", "fp8"], default="auto",
+                    help="fp8: e4m3 cache with bf16 queries (decode workloads)")
+    ap.add_argument("--cascade", action="store_true",
+                    help="decode through pa_decode_cascade (shared prefixes read once per group)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -464,7 +600,10 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     try:
-        run_ours(args, rank, world, device)
+        if args.workload in PREFILL:
+            run_prefill(args, rank, world, device)
+        else:
+            run_ours(args, rank, world, device)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

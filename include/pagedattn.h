@@ -29,7 +29,9 @@
  *     A "slot" is block * block_size + offset.
  *   - Query head h reads kv head h / (num_q_heads / num_kv_heads).
  *   - Supported shapes: head_dim 64 or 128; block_size 1, 2, 4, 8, 16 or 32;
- *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; dtype fp32 or bf16.
+ *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; dtype fp32, bf16 or fp8
+ *     e4m3 (decode, append, copies and swaps; prefill and the shared-prefix
+ *     decode take bf16 only).
  */
 #ifndef PAGEDATTN_H
 #define PAGEDATTN_H
@@ -53,7 +55,10 @@ typedef enum {
   PA_ERR_DEVICE_TIMEOUT = 8   /* a kernel gave up a bounded wait on its own copies */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+/* Cache element types. PA_FP8_E4M3 stores K and V as 8-bit floats (e4m3,
+ * no infinities, largest 448) with one scale per tensor (pa_cache.k_scale,
+ * v_scale): element = code * scale. The q/k/v inputs of an FP8 cache are bf16. */
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 typedef void* pa_stream; /* cudaStream_t */
 
@@ -67,7 +72,9 @@ typedef struct {
   int32_t num_kv_heads;  /* >= 1 */
   int32_t block_size;    /* tokens per block */
   int32_t head_dim;      /* elements per head row */
-  int32_t dtype;         /* pa_dtype of k, v, and of the q/k/v inputs */
+  int32_t dtype;         /* pa_dtype of k, v (and of the q/k/v inputs, bf16 for FP8) */
+  float k_scale;         /* PA_FP8_E4M3 only: K element = code * k_scale (> 0) */
+  float v_scale;         /* PA_FP8_E4M3 only: V element = code * v_scale (> 0) */
 } pa_cache;
 
 /* Human-readable name of a status code (static storage). */
@@ -92,7 +99,10 @@ int32_t pa_version(void);
  *                 recorded as PA_ERR_DEVICE_BOUNDS.
  *   num_tokens    >= 0; 0 launches nothing.
  * Two tokens must not name the same slot in one call (the result would be
- * either row). A bit copy: no rounding.
+ * either row). A bit copy for fp32 / bf16 caches. For an FP8 cache the rows
+ * are bf16 and each element is stored as the e4m3 code of x / scale computed
+ * in fp32, rounded to nearest even, clamped to +-448 (the "quantised code"
+ * step of an 8-bit KV cache).
  */
 pa_status pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
                                const pa_cache* cache, pa_stream stream);
@@ -192,6 +202,42 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
 pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, int32_t max_q_len, int32_t num_q_heads,
                      const pa_cache* cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
                      const int32_t* context_lens, int32_t max_context_len, float scale, float* out, pa_stream stream);
+
+/*
+ * Decode with shared prefixes read once per group (P2 §3.4: sequences sharing
+ * a prefix point at the same physical blocks; P1 "跨请求的内存共享": parallel
+ * samples of one prompt). Same result as pa_decode, computed in three parts:
+ * for each group, one pass over the shared prefix blocks attends all members'
+ * queries at once (rows = members x query heads on the tensor cores); each
+ * sequence's own suffix [seq_prefix_tokens[s], L_s) goes through the decode
+ * kernels; a log-sum-exp merge combines them. Prefix K/V bytes are read once
+ * per group instead of once per member.
+ *
+ *   group_offsets        device int32 [num_groups + 1]; group j's members are
+ *                        group_members[group_offsets[j] .. group_offsets[j+1]).
+ *   group_members        device int32: sequence indices (0 .. num_seqs-1), each
+ *                        in at most one group; at most 64 / (num_q_heads /
+ *                        num_kv_heads) members per group (max_group_size).
+ *   group_prefix_tokens  device int32 [num_groups]: tokens shared by every
+ *                        member (identical physical blocks, read through the
+ *                        first member's table), a multiple of 64.
+ *   seq_prefix_tokens    device int32 [num_seqs]: its group's prefix length,
+ *                        0 for a sequence in no group.
+ *   max_prefix_tokens    host bound on group_prefix_tokens.
+ *   workspace            >= pa_decode_cascade_workspace_bytes(...).
+ * Other arguments as pa_decode (partition size chosen by the library).
+ * Supported: bf16 cache, block_size 8..32; other shapes return
+ * PA_ERR_UNSUPPORTED.
+ */
+pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                            int32_t max_context_len, int32_t num_groups, const int32_t* group_offsets,
+                            const int32_t* group_members, const int32_t* group_prefix_tokens,
+                            const int32_t* seq_prefix_tokens, int32_t max_group_size, int32_t max_prefix_tokens,
+                            float scale, float* out, void* workspace, size_t workspace_bytes, pa_stream stream);
+
+size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t max_context_len, int32_t block_size, int32_t max_prefix_tokens);
 
 /* The partition size pa_decode uses for partition_tokens = -1 with these
  * sizes (0 = no split). */

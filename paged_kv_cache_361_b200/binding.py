@@ -18,8 +18,13 @@ LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_NO_FREE_BLOCKS, PA_ERR_UNKNOWN_SEQ, PA_ERR_SEQ_EXISTS, \
     PA_ERR_CUDA, PA_ERR_DEVICE_BOUNDS, PA_ERR_DEVICE_TIMEOUT = range(9)
-PA_F32, PA_BF16 = 0, 1
-_DTYPE = {torch.float32: PA_F32, torch.bfloat16: PA_BF16}
+PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
+_DTYPE = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float8_e4m3fn: PA_FP8_E4M3}
+
+
+def input_dtype(cache_dtype):
+    """dtype of q and of the new K/V rows for a cache of cache_dtype."""
+    return torch.bfloat16 if cache_dtype == torch.float8_e4m3fn else cache_dtype
 
 
 class PagedAttnError(RuntimeError):
@@ -31,7 +36,7 @@ class PagedAttnError(RuntimeError):
 class pa_cache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("num_blocks", ctypes.c_int64),
                 ("num_kv_heads", ctypes.c_int32), ("block_size", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 _L = None
@@ -46,6 +51,9 @@ _SIGS = {
     "pa_copy_blocks": (_I32, [_PCACHE, _VP, _I32, _VP]),
     "pa_decode": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP, _SZ, _VP]),
     "pa_decode_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
+    "pa_decode_cascade": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32,
+                                 _F, _VP, _VP, _SZ, _VP]),
+    "pa_decode_cascade_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_prefill": (_I32, [_VP, _I32, _VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _VP]),
     "pa_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_get_device_error": (_I32, [_VP, _P64]),
@@ -115,6 +123,15 @@ def _dev(t: torch.Tensor, name: str, dtype=None, ndim=None):
     return t.data_ptr()
 
 
+# An fp8 cache carries its per-tensor scales on the two cache tensor objects
+# (set with set_fp8_scales); make_cache refuses an fp8 cache without them.
+def set_fp8_scales(k_cache, v_cache, k_scale: float, v_scale: float):
+    if k_cache.dtype != torch.float8_e4m3fn or v_cache.dtype != torch.float8_e4m3fn:
+        raise TypeError("scales belong to a float8_e4m3fn cache")
+    k_cache._pa_fp8_scale = float(k_scale)
+    v_cache._pa_fp8_scale = float(v_scale)
+
+
 def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> pa_cache:
     """pa_cache view of two [num_blocks][num_kv_heads][block_size][head_dim] tensors."""
     if k_cache.shape != v_cache.shape or k_cache.dtype != v_cache.dtype:
@@ -122,8 +139,13 @@ def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> pa_cache:
     if k_cache.dtype not in _DTYPE:
         raise TypeError(f"unsupported cache dtype {k_cache.dtype}")
     nb, hkv, bs, d = k_cache.shape
+    ks = vs = 1.0
+    if k_cache.dtype == torch.float8_e4m3fn:
+        ks, vs = getattr(k_cache, "_pa_fp8_scale", None), getattr(v_cache, "_pa_fp8_scale", None)
+        if ks is None or vs is None:
+            raise ValueError("fp8 cache without scales: call set_fp8_scales(k_cache, v_cache, k_scale, v_scale)")
     return pa_cache(_dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4), nb, hkv, bs, d,
-                    _DTYPE[k_cache.dtype])
+                    _DTYPE[k_cache.dtype], ks, vs)
 
 
 # --- device operations ---------------------------------------------------------
@@ -131,7 +153,7 @@ def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> pa_cache:
 def pa_reshape_and_cache(k, v, slot_mapping, k_cache, v_cache, stream=None):
     c = make_cache(k_cache, v_cache)
     n = int(k.shape[0])
-    _dev(k, "k", k_cache.dtype, 3), _dev(v, "v", k_cache.dtype, 3)
+    _dev(k, "k", input_dtype(k_cache.dtype), 3), _dev(v, "v", input_dtype(k_cache.dtype), 3)
     if tuple(k.shape) != (n, c.num_kv_heads, c.head_dim) or k.shape != v.shape:
         raise ValueError("k, v must be [num_tokens][num_kv_heads][head_dim]")
     if slot_mapping.shape != (n,):
@@ -163,7 +185,7 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_c
               partition_tokens=-1, workspace=None, stream=None):
     c = make_cache(k_cache, v_cache)
     B, hq, d = q.shape
-    _dev(q, "q", k_cache.dtype, 3)
+    _dev(q, "q", input_dtype(k_cache.dtype), 3)
     _dev(out, "out", torch.float32, 3)
     if d != c.head_dim or tuple(out.shape) != (B, hq, d):
         raise ValueError("q/out shape mismatch")
@@ -184,7 +206,7 @@ def pa_prefill(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale
     cu_q_lens[s]..cu_q_lens[s+1]-1) over the paged cache; out fp32 [T][Hq][D]."""
     c = make_cache(k_cache, v_cache)
     T, hq, d = q.shape
-    _dev(q, "q", k_cache.dtype, 3)
+    _dev(q, "q", input_dtype(k_cache.dtype), 3)
     _dev(out, "out", torch.float32, 3)
     if d != c.head_dim or tuple(out.shape) != (T, hq, d):
         raise ValueError("q/out shape mismatch")
@@ -197,6 +219,40 @@ def pa_prefill(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale
     _check(_lib().pa_prefill(q.data_ptr(), B, cu_q_lens.data_ptr(), int(max_q_len), hq, ctypes.byref(c),
                              block_tables.data_ptr(), int(block_tables.shape[1]), context_lens.data_ptr(),
                              int(max_context_len), float(scale), out.data_ptr(), _stream(q, stream)), "pa_prefill")
+
+
+def pa_decode_cascade_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size,
+                                      max_prefix_tokens) -> int:
+    return int(_lib().pa_decode_cascade_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                        max_context_len, block_size, max_prefix_tokens))
+
+
+def pa_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_context_len, group_offsets,
+                      group_members, group_prefix_tokens, seq_prefix_tokens, max_group_size, max_prefix_tokens,
+                      workspace, stream=None):
+    """pa_decode with shared prefixes read once per group (see pagedattn.h)."""
+    c = make_cache(k_cache, v_cache)
+    B, hq, d = q.shape
+    _dev(q, "q", input_dtype(k_cache.dtype), 3)
+    _dev(out, "out", torch.float32, 3)
+    if d != c.head_dim or tuple(out.shape) != (B, hq, d):
+        raise ValueError("q/out shape mismatch")
+    _dev(block_tables, "block_tables", torch.int32, 2)
+    _dev(context_lens, "context_lens", torch.int32, 1)
+    _dev(seq_prefix_tokens, "seq_prefix_tokens", torch.int32, 1)
+    ng = int(group_offsets.shape[0]) - 1
+    if ng > 0:
+        _dev(group_offsets, "group_offsets", torch.int32, 1)
+        _dev(group_members, "group_members", torch.int32, 1)
+        _dev(group_prefix_tokens, "group_prefix_tokens", torch.int32, 1)
+    _check(_lib().pa_decode_cascade(q.data_ptr(), B, hq, ctypes.byref(c), block_tables.data_ptr(),
+                                    int(block_tables.shape[1]), context_lens.data_ptr(), int(max_context_len), ng,
+                                    group_offsets.data_ptr() if ng else None,
+                                    group_members.data_ptr() if ng else None,
+                                    group_prefix_tokens.data_ptr() if ng else None, seq_prefix_tokens.data_ptr(),
+                                    int(max_group_size), int(max_prefix_tokens), float(scale), out.data_ptr(),
+                                    _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                    _stream(q, stream)), "pa_decode_cascade")
 
 
 def pa_get_device_error(stream=None):
@@ -214,7 +270,7 @@ def pa_decode_static_workspace(q, k_cache, v_cache, block_tables, context_lens, 
     """pa_decode with the library's fixed device workspace (no allocation)."""
     c = make_cache(k_cache, v_cache)
     B, hq, d = q.shape
-    _dev(q, "q", k_cache.dtype, 3)
+    _dev(q, "q", input_dtype(k_cache.dtype), 3)
     _dev(out, "out", torch.float32, 3)
     if d != c.head_dim or tuple(out.shape) != (B, hq, d):
         raise ValueError("q/out shape mismatch")
@@ -251,9 +307,9 @@ def pa_step_host(bm: "BlockManager", k_cache, v_cache, seq_ids, q_host, k_host, 
     c = make_cache(k_cache, v_cache)
     ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
     n, hq, d = q_host.shape
-    _host(q_host, "q_host", k_cache.dtype, (len(ids), hq, c.head_dim))
-    _host(k_host, "k_host", k_cache.dtype, (len(ids), c.num_kv_heads, c.head_dim))
-    _host(v_host, "v_host", k_cache.dtype, (len(ids), c.num_kv_heads, c.head_dim))
+    _host(q_host, "q_host", input_dtype(k_cache.dtype), (len(ids), hq, c.head_dim))
+    _host(k_host, "k_host", input_dtype(k_cache.dtype), (len(ids), c.num_kv_heads, c.head_dim))
+    _host(v_host, "v_host", input_dtype(k_cache.dtype), (len(ids), c.num_kv_heads, c.head_dim))
     _host(out_host, "out_host", torch.float32, (len(ids), hq, c.head_dim))
     _dev(dev_staging, "dev_staging")
     if host_staging.is_cuda or not host_staging.is_contiguous():

@@ -39,14 +39,23 @@ class _Staging:
 
 class PagedKVCache:
     def __init__(self, num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
-                 dtype=torch.bfloat16, device="cuda", free_order=None, fill: float | None = None):
+                 dtype=torch.bfloat16, device="cuda", free_order=None, fill: float | None = None,
+                 k_scale: float = 1.0, v_scale: float = 1.0):
+        """dtype torch.float8_e4m3fn makes an 8-bit cache with per-tensor scales
+        (element = code * scale); its q/k/v inputs are bf16."""
         self.device = torch.device(device)
         shape = (num_blocks, num_kv_heads, block_size, head_dim)
         self.k_cache = torch.empty(shape, dtype=dtype, device=self.device)
         self.v_cache = torch.empty(shape, dtype=dtype, device=self.device)
         if fill is not None:
-            self.k_cache.fill_(fill)
-            self.v_cache.fill_(fill)
+            if dtype == torch.float8_e4m3fn:
+                code = int(torch.tensor(fill, dtype=torch.float32).to(dtype).view(torch.uint8).item())
+                self.k_cache.view(torch.uint8).fill_(code)
+            else:
+                self.k_cache.fill_(fill)
+            self.v_cache.copy_(self.k_cache)
+        if dtype == torch.float8_e4m3fn:
+            B.set_fp8_scales(self.k_cache, self.v_cache, k_scale, v_scale)
         self.block_size = block_size
         self.bm = B.BlockManager(num_blocks, block_size, free_order)
         self.lens: dict[int, int] = {}
@@ -193,6 +202,60 @@ class PagedKVCache:
                      self._lens.upload(lens), scale, out, max(counts, default=0), max_len)
         return out
 
+    def shared_prefix_groups(self, seq_ids, tables: np.ndarray, lens: np.ndarray, group_rows: int):
+        """Host side of the shared-prefix decode: sequences of the batch whose
+        tables start with the same physical blocks form a group (at most
+        group_rows members each); its prefix is the longest run of whole blocks
+        common to all members, cut to a multiple of 64 tokens. Returns
+        (offsets, members, prefix_tokens, seq_prefix_tokens) as numpy arrays."""
+        bs = self.block_size
+        by_first = {}
+        for i in range(len(seq_ids)):
+            if lens[i] >= bs:
+                by_first.setdefault(int(tables[i, 0]), []).append(i)
+        offsets, members, prefix = [0], [], []
+        seq_prefix = np.zeros(len(seq_ids), dtype=np.int32)
+        for rows in by_first.values():
+            for c0 in range(0, len(rows), group_rows):
+                grp = rows[c0:c0 + group_rows]
+                if len(grp) < 2:
+                    continue
+                full = int(min(lens[i] for i in grp)) // bs
+                t = tables[grp, :full]
+                same = np.all(t == t[0], axis=0)
+                k = full if same.all() else int(np.argmin(same))
+                ptok = (k * bs) // 64 * 64
+                if ptok == 0:
+                    continue
+                members += grp
+                offsets.append(len(members))
+                prefix.append(ptok)
+                seq_prefix[grp] = ptok
+        return (np.asarray(offsets, np.int32), np.asarray(members, np.int32), np.asarray(prefix, np.int32),
+                seq_prefix)
+
+    def decode_cascade(self, seq_ids, q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None):
+        """decode() with shared prefixes (forks, prefix-cache hits) read once per
+        group of sequences (pa_decode_cascade)."""
+        n, hq, d = q.shape
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        tables, lens, max_len = self.decode_inputs(seq_ids)
+        hkv = self.k_cache.shape[1]
+        offs, members, prefix, seq_prefix = self.shared_prefix_groups(seq_ids, tables, lens, 64 // (hq // hkv))
+        if out is None:
+            out = torch.empty((n, hq, d), dtype=torch.float32, device=self.device)
+        max_pre = int(prefix.max()) if len(prefix) else 0
+        nbytes = B.pa_decode_cascade_workspace_bytes(n, hq, hkv, d, max_len, self.block_size, max_pre)
+        ws = self.workspace(nbytes)
+        empty = torch.empty(0, dtype=torch.int32, device=self.device)
+        B.pa_decode_cascade(q, self.k_cache, self.v_cache, self._tables.upload(tables), self._lens.upload(lens), scale,
+                            out, max_len, self._lens.upload(offs),
+                            self._lens.upload(members) if len(members) else empty,
+                            self._lens.upload(prefix) if len(prefix) else empty, self._lens.upload(seq_prefix),
+                            int(max(np.diff(offs), default=0)), max_pre, ws)
+        return out
+
     def step_host(self, seq_ids, q_host, k_host, v_host, out_host, scale=None, partition_tokens=-1):
         """One decode step from host tensors (pinned for asynchronous copies):
         block-manager work, copies and kernels in one native call
@@ -212,7 +275,60 @@ class PagedKVCache:
             self.lens[s] += 1
         return out_host
 
+    def step_plan(self, seq_ids, q_host, k_host, v_host, out_host, scale=None, partition_tokens=-1,
+                  max_context_len=None) -> "StepPlan":
+        """A prepared pa_step_host call for a fixed batch and fixed host buffers:
+        argument checks, staging and the C argument list are done once; each
+        StepPlan.run() is one native call. Staging is sized for contexts up to
+        max_context_len (default: the current maximum + 4096)."""
+        return StepPlan(self, seq_ids, q_host, k_host, v_host, out_host, scale, partition_tokens, max_context_len)
+
     def step(self, seq_ids, q, k, v, scale=None, out=None, partition_tokens=-1):
         """One decode step: append each sequence's new K/V, then attend."""
         self.append(seq_ids, k, v)
         return self.decode(seq_ids, q, scale, out, partition_tokens)
+
+
+class StepPlan:
+    """See PagedKVCache.step_plan."""
+
+    def __init__(self, cache: PagedKVCache, seq_ids, q_host, k_host, v_host, out_host, scale, partition_tokens,
+                 max_context_len):
+        import ctypes
+        n, hq, d = q_host.shape
+        self.cache = cache
+        self.ids = [int(s) for s in seq_ids]
+        if max_context_len is None:
+            max_context_len = max(cache.lens[s] for s in self.ids) + 4096
+        self.max_context_len = int(max_context_len)
+        dev_b, host_b = B.pa_step_staging_bytes(n, hq, cache.k_cache, cache.v_cache, self.max_context_len,
+                                                partition_tokens)
+        self.dev_staging = torch.empty(dev_b, dtype=torch.uint8, device=cache.device)
+        self.host_staging = torch.empty(host_b, dtype=torch.uint8, pin_memory=True)
+        # validate once through the checked binding path (argument shapes, dtypes, placement)
+        in_dt = B.input_dtype(cache.k_cache.dtype)
+        for name, t, shape, dt in (("q_host", q_host, (n, hq, d), in_dt),
+                                   ("k_host", k_host, (n, cache.k_cache.shape[1], d), in_dt),
+                                   ("v_host", v_host, (n, cache.k_cache.shape[1], d), in_dt),
+                                   ("out_host", out_host, (n, hq, d), torch.float32)):
+            B._host(t, name, dt, shape)
+        self._keep = (q_host, k_host, v_host, out_host)
+        self._ids = np.ascontiguousarray(self.ids, dtype=np.int64)
+        self._cache_struct = B.make_cache(cache.k_cache, cache.v_cache)
+        self._args = (cache.bm._h, ctypes.byref(self._cache_struct), n, self._ids.ctypes.data_as(ctypes.c_void_p), hq,
+                      q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                      float(scale if scale is not None else 1.0 / math.sqrt(d)), out_host.data_ptr(),
+                      int(partition_tokens), self.dev_staging.data_ptr(), dev_b, self.host_staging.data_ptr(), host_b,
+                      torch.cuda.current_stream(cache.device).cuda_stream)
+        self._fn = B._lib().pa_step_host
+        self.steps = 0
+
+    def run(self):
+        """One decode step; on return the output buffer holds the result."""
+        if max(self.cache.lens[s] for s in self.ids) + 1 > self.max_context_len:
+            raise ValueError("a sequence outgrew the plan's max_context_len")
+        B._check(self._fn(*self._args), "pa_step_host")
+        lens = self.cache.lens
+        for s in self.ids:
+            lens[s] += 1
+        self.steps += 1

@@ -45,6 +45,52 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const int4* __re
   }
 }
 
+// FP8 cache: k, v rows are bf16 [num_tokens][hkv][D]; each thread turns 16
+// bf16 inputs (two 16-byte loads) into one 16-byte store of e4m3 codes.
+//   row_chunks = D / 16 per (token, head) row
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4* __restrict__ k,
+                                                                    const uint4* __restrict__ v,
+                                                                    const int64_t* __restrict__ slots,
+                                                                    int4* __restrict__ kc, int4* __restrict__ vc,
+                                                                    int32_t num_tokens, int32_t hkv, int32_t bs,
+                                                                    int32_t row_chunks, int64_t num_slots,
+                                                                    float k_scale, float v_scale) {
+  const int64_t total = static_cast<int64_t>(num_tokens) * hkv * row_chunks;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int64_t row = i / row_chunks;
+    const int32_t c = static_cast<int32_t>(i - row * row_chunks);
+    const int64_t t = row / hkv;
+    const int32_t h = static_cast<int32_t>(row - t * hkv);
+    const int64_t slot = __ldg(slots + t);
+    if (slot == -1) continue;
+    if (slot < -1 || slot >= num_slots) {
+      if (h == 0 && c == 0) record_error(PA_ERR_DEVICE_BOUNDS, slot);
+      continue;
+    }
+    const int64_t blk = slot / bs;
+    const int64_t off = slot - blk * bs;
+    const int64_t dst = ((blk * hkv + h) * bs + off) * row_chunks + c;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint4* src = (which == 0 ? k : v) + 2 * i;
+      const float sc = which == 0 ? k_scale : v_scale;
+      const uint4 a = __ldcs(src), b = __ldcs(src + 1);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint32_t q[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t lo = w[2 * u], hi = w[2 * u + 1];
+        q[u] = static_cast<uint32_t>(quantize_e4m3(bf16lo(lo), sc)) |
+               (static_cast<uint32_t>(quantize_e4m3(bf16hi(lo), sc)) << 8) |
+               (static_cast<uint32_t>(quantize_e4m3(bf16lo(hi), sc)) << 16) |
+               (static_cast<uint32_t>(quantize_e4m3(bf16hi(hi), sc)) << 24);
+      }
+      (which == 0 ? kc : vc)[dst] = make_int4(q[0], q[1], q[2], q[3]);
+    }
+  }
+}
+
 // Grid: blocks_per_pair CTAs per pair, flattened. chunks = 16-byte chunks in
 // one physical block of one tensor (hkv * bs * head_dim * elem / 16).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(int4* __restrict__ kc, int4* __restrict__ vc,

@@ -17,14 +17,17 @@ using namespace pa;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool pow2_block(int32_t bs) { return bs == 1 || bs == 2 || bs == 4 || bs == 8 || bs == 16 || bs == 32; }
-int elem_bytes(int32_t dtype) { return dtype == PA_BF16 ? 2 : 4; }
+int elem_bytes(int32_t dtype) { return dtype == PA_FP8_E4M3 ? 1 : (dtype == PA_BF16 ? 2 : 4); }
 
 pa_status check_cache(const pa_cache* c) {
   if (!c || !c->k || !c->v || !aligned16(c->k) || !aligned16(c->v)) return PA_ERR_INVALID_ARG;
   if (c->num_blocks <= 0 || c->num_blocks > INT32_MAX || c->num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
   if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (!pow2_block(c->block_size)) return PA_ERR_UNSUPPORTED;
-  if (c->dtype != PA_F32 && c->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (c->dtype != PA_F32 && c->dtype != PA_BF16 && c->dtype != PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  if (c->dtype == PA_FP8_E4M3 && !(std::isfinite(c->k_scale) && c->k_scale > 0.f && std::isfinite(c->v_scale) &&
+                                   c->v_scale > 0.f))
+    return PA_ERR_INVALID_ARG;
   // slots must fit in int64 and block ids in int32 (checked above)
   return PA_OK;
 }
@@ -253,6 +256,13 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;  // grid-stride beyond this
+  if (cache->dtype == PA_FP8_E4M3) {
+    reshape_and_cache_fp8_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, static_cast<int4*>(cache->k),
+        static_cast<int4*>(cache->v), num_tokens, cache->num_kv_heads, cache->block_size, row_chunks,
+        cache->num_blocks * cache->block_size, cache->k_scale, cache->v_scale);
+    return launched();
+  }
   reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const int4*>(k), static_cast<const int4*>(v), slot_mapping, static_cast<int4*>(cache->k),
       static_cast<int4*>(cache->v), num_tokens, cache->num_kv_heads, cache->block_size, row_chunks,
@@ -359,6 +369,9 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   a.max_ctx = max_context_len;
   a.ntiles = static_cast<int32_t>(ntiles);
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.group_offs = a.group_members = a.group_prefix = nullptr;
+  a.prefix_part_tokens = a.max_parts = a.parts_stride = 0;
+  a.ws_ml = a.ws_o = nullptr;
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
   if (!encode_rows(&tk, cache->k, rows, cache->head_dim, cache->block_size) ||
@@ -374,18 +387,166 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   };
   if (cache->head_dim == 128) {
     switch (G) {
-      case 1: return launch(prefill_mma_kernel<128, 1>, MmaCfg<128>::kSmemBytes);
-      case 2: return launch(prefill_mma_kernel<128, 2>, MmaCfg<128>::kSmemBytes);
-      case 4: return launch(prefill_mma_kernel<128, 4>, MmaCfg<128>::kSmemBytes);
-      default: return launch(prefill_mma_kernel<128, 8>, MmaCfg<128>::kSmemBytes);
+      case 1: return launch(prefill_mma_kernel<128, 1, false>, MmaCfg<128>::kSmemBytes);
+      case 2: return launch(prefill_mma_kernel<128, 2, false>, MmaCfg<128>::kSmemBytes);
+      case 4: return launch(prefill_mma_kernel<128, 4, false>, MmaCfg<128>::kSmemBytes);
+      default: return launch(prefill_mma_kernel<128, 8, false>, MmaCfg<128>::kSmemBytes);
     }
   }
   switch (G) {
-    case 1: return launch(prefill_mma_kernel<64, 1>, MmaCfg<64>::kSmemBytes);
-    case 2: return launch(prefill_mma_kernel<64, 2>, MmaCfg<64>::kSmemBytes);
-    case 4: return launch(prefill_mma_kernel<64, 4>, MmaCfg<64>::kSmemBytes);
-    default: return launch(prefill_mma_kernel<64, 8>, MmaCfg<64>::kSmemBytes);
+    case 1: return launch(prefill_mma_kernel<64, 1, false>, MmaCfg<64>::kSmemBytes);
+    case 2: return launch(prefill_mma_kernel<64, 2, false>, MmaCfg<64>::kSmemBytes);
+    case 4: return launch(prefill_mma_kernel<64, 4, false>, MmaCfg<64>::kSmemBytes);
+    default: return launch(prefill_mma_kernel<64, 8, false>, MmaCfg<64>::kSmemBytes);
   }
+}
+
+// Shared-prefix decode: prefix partitions of this many tokens (a multiple of
+// the 64-token chunk).
+constexpr int32_t kCascadePrefixPart = 256;
+
+size_t cascade_ws_bytes(int32_t num_seqs, int32_t hq, int32_t hkv, int32_t D, int32_t suffix_parts,
+                        int32_t prefix_parts) {
+  const int32_t stride = suffix_parts + prefix_parts;
+  return counters_bytes(num_seqs, hkv) + ml_bytes(num_seqs, hq, stride) +
+         static_cast<size_t>(num_seqs) * hq * stride * D * 4;
+}
+
+size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t max_context_len, int32_t block_size, int32_t max_prefix_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_prefix_tokens < 0)
+    return 0;
+  const int32_t P = resolve_partition(num_seqs, num_kv_heads, max_context_len, block_size, -1);
+  return cascade_ws_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, num_parts(max_context_len, P),
+                          (max_prefix_tokens + kCascadePrefixPart - 1) / kCascadePrefixPart);
+}
+
+pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                            int32_t max_context_len, int32_t num_groups, const int32_t* group_offsets,
+                            const int32_t* group_members, const int32_t* group_prefix_tokens,
+                            const int32_t* seq_prefix_tokens, int32_t max_group_size, int32_t max_prefix_tokens,
+                            float scale, float* out, void* workspace, size_t workspace_bytes, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || num_groups < 0 ||
+      max_group_size < 0 || max_prefix_tokens < 0 || max_prefix_tokens > max_context_len)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int G = num_q_heads / cache->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (cache->dtype != PA_BF16 || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
+  if (max_group_size > 64 / G) return PA_ERR_INVALID_ARG;  // one 64-row tile per group
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * cache->block_size)
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !block_tables || !context_lens || !out || !seq_prefix_tokens || !aligned16(q) || !aligned16(out) ||
+      (num_groups > 0 && (!group_offsets || !group_members || !group_prefix_tokens)))
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs > 65535 || num_groups > 65535) return PA_ERR_UNSUPPORTED;
+
+  const int32_t P = resolve_partition(num_seqs, cache->num_kv_heads, max_context_len, cache->block_size, -1);
+  const int32_t parts = num_parts(max_context_len, P);
+  const int32_t pparts = (max_prefix_tokens + kCascadePrefixPart - 1) / kCascadePrefixPart;
+  const size_t need = cascade_ws_bytes(num_seqs, num_q_heads, cache->num_kv_heads, cache->head_dim, parts, pparts);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)) return PA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  const int32_t stride = parts + pparts;
+  const size_t cb = counters_bytes(num_seqs, cache->num_kv_heads);
+  float* ws_ml = reinterpret_cast<float*>(ws + cb);
+  float* ws_o = reinterpret_cast<float*>(ws + cb + ml_bytes(num_seqs, num_q_heads, stride));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = cache->head_dim;
+
+  // 1. prefix partials: one CTA per (kv head, prefix partition, group), rows = members x heads
+  if (num_groups > 0 && pparts > 0) {
+    PrefillArgs pa;
+    pa.q = q;
+    pa.cu_q = nullptr;
+    pa.tables = block_tables;
+    pa.lens = context_lens;
+    pa.out = nullptr;
+    pa.num_blocks = cache->num_blocks;
+    pa.num_seqs = num_seqs;
+    pa.hq = num_q_heads;
+    pa.hkv = cache->num_kv_heads;
+    pa.bs = cache->block_size;
+    pa.max_blocks = max_blocks_per_seq;
+    pa.max_ctx = max_context_len;
+    pa.ntiles = 0;
+    pa.scale_log2 = scale * 1.4426950408889634f;
+    pa.group_offs = group_offsets;
+    pa.group_members = group_members;
+    pa.group_prefix = group_prefix_tokens;
+    pa.prefix_part_tokens = kCascadePrefixPart;
+    pa.max_parts = parts;
+    pa.parts_stride = stride;
+    pa.ws_ml = ws_ml;
+    pa.ws_o = ws_o;
+    CUtensorMap tk, tv;
+    const uint64_t rows = static_cast<uint64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
+    if (!encode_rows(&tk, cache->k, rows, D, cache->block_size) || !encode_rows(&tv, cache->v, rows, D, cache->block_size))
+      return PA_ERR_CUDA;
+    const dim3 grid(cache->num_kv_heads, pparts, num_groups);
+    auto launch = [&](auto kern, int smem) -> pa_status {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return PA_ERR_CUDA;
+      kern<<<grid, MmaCfg<128>::kThreads, smem, s>>>(tk, tv, pa);
+      return launched();
+    };
+    if (D == 128) {
+      st = G == 1 ? launch(prefill_mma_kernel<128, 1, true>, MmaCfg<128>::kSmemBytes)
+         : G == 2 ? launch(prefill_mma_kernel<128, 2, true>, MmaCfg<128>::kSmemBytes)
+         : G == 4 ? launch(prefill_mma_kernel<128, 4, true>, MmaCfg<128>::kSmemBytes)
+                  : launch(prefill_mma_kernel<128, 8, true>, MmaCfg<128>::kSmemBytes);
+    } else {
+      st = G == 1 ? launch(prefill_mma_kernel<64, 1, true>, MmaCfg<64>::kSmemBytes)
+         : G == 2 ? launch(prefill_mma_kernel<64, 2, true>, MmaCfg<64>::kSmemBytes)
+         : G == 4 ? launch(prefill_mma_kernel<64, 4, true>, MmaCfg<64>::kSmemBytes)
+                  : launch(prefill_mma_kernel<64, 8, true>, MmaCfg<64>::kSmemBytes);
+    }
+    if (st != PA_OK) return st;
+  }
+
+  // 2. suffix partials: the decode kernels over [seq_prefix_tokens[s], L_s)
+  DecodeArgs a;
+  a.q = q;
+  a.kc = cache->k;
+  a.vc = cache->v;
+  a.tables = block_tables;
+  a.lens = context_lens;
+  a.out = out;
+  a.counters = reinterpret_cast<unsigned int*>(ws);
+  a.ws_ml = ws_ml;
+  a.ws_o = ws_o;
+  a.num_blocks = cache->num_blocks;
+  a.num_seqs = num_seqs;
+  a.hq = num_q_heads;
+  a.hkv = cache->num_kv_heads;
+  a.bs = cache->block_size;
+  a.max_blocks = max_blocks_per_seq;
+  a.max_ctx = max_context_len;
+  a.part_tokens = parts > 1 ? P : 0;
+  a.max_parts = parts;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.n_items = static_cast<int32_t>(static_cast<int64_t>(cache->num_kv_heads) * num_seqs * parts);
+  a.starts = seq_prefix_tokens;
+  a.force_partials = 1;
+  a.parts_stride = stride;
+  a.prefix_part_tokens = kCascadePrefixPart;
+  const dim3 grid(cache->num_kv_heads, num_seqs, parts);
+  if (mma_eligible(cache, G)) {
+    st = dispatch_mma(a, cache, G, s);
+  } else {
+    st = D == 128 ? dispatch_g<__nv_bfloat16, 128>(a, G, grid, s) : dispatch_g<__nv_bfloat16, 64>(a, G, grid, s);
+  }
+  if (st != PA_OK) return st;
+  // 3. merge prefix and suffix partials
+  return D == 128 ? launch_reduce<128>(a, s) : launch_reduce<64>(a, s);
 }
 
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
@@ -453,12 +614,24 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   a.max_parts = parts;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.n_items = static_cast<int32_t>(static_cast<int64_t>(cache->num_kv_heads) * num_seqs * parts);
+  a.starts = nullptr;
+  a.force_partials = 0;
+  a.parts_stride = parts;
+  a.prefix_part_tokens = 0;
+  if (cache->dtype == PA_FP8_E4M3) {
+    // q . (k_scale * code) = (k_scale * q) . code; the V scale multiplies o.
+    a.scale_log2 *= cache->k_scale;
+    a.v_scale = cache->v_scale;
+    if (!std::isfinite(a.scale_log2)) return PA_ERR_INVALID_ARG;
+  }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(cache->num_kv_heads, num_seqs, parts);
   const int D = cache->head_dim;
   if (mma_eligible(cache, G)) {
     st = dispatch_mma(a, cache, G, s);
+  } else if (cache->dtype == PA_FP8_E4M3) {
+    st = D == 128 ? dispatch_g<__nv_fp8_e4m3, 128>(a, G, grid, s) : dispatch_g<__nv_fp8_e4m3, 64>(a, G, grid, s);
   } else if (cache->dtype == PA_BF16) {
     st = D == 128 ? dispatch_g<__nv_bfloat16, 128>(a, G, grid, s) : dispatch_g<__nv_bfloat16, 64>(a, G, grid, s);
   } else {

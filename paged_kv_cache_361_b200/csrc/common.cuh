@@ -3,6 +3,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -98,6 +100,21 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// Two e4m3 codes (low byte first) -> two floats (exact: every e4m3 value is
+// representable in fp16 and fp32).
+__device__ __forceinline__ float2 fp8x2_to_float2(uint16_t w) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// x / scale in fp32 (IEEE division), rounded to the nearest e4m3 code (ties
+// to even); finite values beyond +-448 and infinities saturate to +-448, NaN
+// stays NaN.
+__device__ __forceinline__ uint8_t quantize_e4m3(float x, float scale) {
+  const float y = __fdiv_rn(x, scale);
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
 }
 
 // bf16 pair packed in a 32-bit word -> two floats (exact).

@@ -20,18 +20,33 @@ struct DecodeArgs {
   const int32_t* tables;
   const int32_t* lens;
   float* out;
-  float* ws_ml;   // [num_seqs][hq][max_parts][2]  (m in log2 units, l)
-  float* ws_o;    // [num_seqs][hq][max_parts][D]
+  float* ws_ml;   // [num_seqs][hq][parts_stride][2]  (m in log2 units, l)
+  float* ws_o;    // [num_seqs][hq][parts_stride][D]
   int64_t num_blocks;
   int32_t num_seqs, hq, hkv, bs, max_blocks, max_ctx;
   int32_t part_tokens;  // > 0: partition size; 0: one partition per sequence
   int32_t max_parts;    // partitions of the longest sequence
-  float scale_log2;     // scale * log2(e)
+  float scale_log2;     // scale * log2(e) (times the K scale of an fp8 cache)
+  float v_scale = 1.f;  // V scale of an fp8 cache, applied to o before the merge
   // Persistent kernels: counters[0] hands out work items. Zeroed before every
   // launch.
   unsigned int* counters;
   int32_t n_items;      // hkv * num_seqs * max_parts
+  // Shared-prefix (cascade) decode: this call covers tokens [starts[s], L_s)
+  // only and always writes partials; prefix partials written by the cascade
+  // prefix kernel sit after the suffix ones. Null / 0 / max_parts otherwise.
+  const int32_t* starts;
+  int32_t force_partials;
+  int32_t parts_stride;  // partial slots per (sequence, query head) row
+  int32_t prefix_part_tokens;  // tokens per prefix partial (cascade only)
 };
+
+// First token a decode CTA covers for sequence s (the cascade suffix start).
+__device__ __forceinline__ int32_t seq_start(const DecodeArgs& a, int32_t s, int32_t L) {
+  if (!a.starts) return 0;
+  int32_t st = __ldg(a.starts + s);
+  return st < 0 ? 0 : (st > L ? L : st);
+}
 
 template <typename T>
 struct Elem;
@@ -42,6 +57,21 @@ struct Elem<float> {
 template <>
 struct Elem<__nv_bfloat16> {
   static constexpr int bytes = 2;
+};
+template <>
+struct Elem<__nv_fp8_e4m3> {
+  static constexpr int bytes = 1;
+};
+
+// Element type of q for a cache of element type T: an fp8 cache is read with
+// bf16 queries.
+template <typename T>
+struct QueryOf {
+  using type = T;
+};
+template <>
+struct QueryOf<__nv_fp8_e4m3> {
+  using type = __nv_bfloat16;
 };
 
 template <typename T>
@@ -71,9 +101,11 @@ struct Part {
 template <int G, int D>
 __device__ __forceinline__ bool cta_part(const DecodeArgs& a, int g, int s, int p, int tid, int nthreads, Part& pt) {
   const int32_t L = load_len(a, s, g == 0 && p == 0 && tid == 0);
-  const int32_t P = a.part_tokens > 0 ? a.part_tokens : (L > 0 ? L : 1);
-  pt.t0 = p * P;
-  if (L == 0) {
+  const int32_t st = seq_start(a, s, L);
+  const int32_t span = L - st;
+  const int32_t P = a.part_tokens > 0 ? a.part_tokens : (span > 0 ? span : 1);
+  pt.t0 = st + p * P;
+  if (L == 0 && !a.starts) {
     if (p == 0)
       for (int idx = tid; idx < G * D; idx += nthreads)
         a.out[(static_cast<int64_t>(s) * a.hq + g * G) * D + idx] = 0.f;
@@ -82,7 +114,7 @@ __device__ __forceinline__ bool cta_part(const DecodeArgs& a, int g, int s, int 
   if (pt.t0 >= L) return false;
   pt.t1 = min(pt.t0 + P, L);
   pt.ntok = pt.t1 - pt.t0;
-  pt.nparts = a.part_tokens > 0 ? (L + P - 1) / P : 1;
+  pt.nparts = a.part_tokens > 0 ? (span + P - 1) / P : 1;
   return true;
 }
 
@@ -180,10 +212,10 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const
       o = fmaf(wacc[(w * G + h) * D + d], f, o);
     }
     const int64_t row = static_cast<int64_t>(s) * a.hq + hq0 + h;
-    if (nparts == 1) {
+    if (nparts == 1 && !a.force_partials) {
       a.out[row * D + d] = o / l;
     } else {
-      const int64_t prow = row * a.max_parts + p;
+      const int64_t prow = row * a.parts_stride + p;
       a.ws_o[prow * D + d] = o;
       if (d == 0) {
         a.ws_ml[prow * 2] = M;
@@ -214,14 +246,24 @@ __global__ void __launch_bounds__(32 * kReduceWarps) decode_reduce_kernel(const 
   for (int64_t row = blockIdx.x; row < nrows; row += gridDim.x) {
     const int s = static_cast<int>(row / a.hq);
     const int32_t L = load_len(a, s, false);
-    const int32_t P = a.part_tokens;
-    const int32_t nparts = (L + P - 1) / P;
-    if (nparts <= 1) continue;  // uniform across the CTA
-    const float* ml = a.ws_ml + row * a.max_parts * 2;
-    const float* o = a.ws_o + row * a.max_parts * D;
+    const int32_t st = seq_start(a, s, L);
+    const int32_t span = L - st;
+    const int32_t P = a.part_tokens > 0 ? a.part_tokens : (span > 0 ? span : 1);
+    const int32_t nsuf = span > 0 ? (span + P - 1) / P : 0;
+    const int32_t npre = st > 0 ? (st + a.prefix_part_tokens - 1) / a.prefix_part_tokens : 0;
+    if (!a.force_partials && nsuf <= 1) continue;  // written by the decode kernel; uniform across the CTA
+    if (nsuf + npre == 0) {                        // empty context: zero row
+      for (int d = tid; d < D; d += 32 * kReduceWarps) a.out[row * D + d] = 0.f;
+      continue;
+    }
+    const int32_t nparts = nsuf + npre;
+    const float* ml = a.ws_ml + row * a.parts_stride * 2;
+    const float* o = a.ws_o + row * a.parts_stride * D;
 
+    // slot of the i-th partial: suffix partials 0..nsuf-1, then prefix partials from max_parts on
+    auto slot = [&](int i) { return i < nsuf ? i : a.max_parts + (i - nsuf); };
     float M = -INFINITY;
-    for (int q = tid; q < nparts; q += 32 * kReduceWarps) M = fmaxf(M, ml[2 * q]);
+    for (int q = tid; q < nparts; q += 32 * kReduceWarps) M = fmaxf(M, ml[2 * slot(q)]);
     M = warp_max(M);
     if (lane == 0) red[warp] = M;
     __syncthreads();
@@ -233,9 +275,10 @@ __global__ void __launch_bounds__(32 * kReduceWarps) decode_reduce_kernel(const 
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
     for (int q = warp; q < nparts; q += kReduceWarps) {
-      const float f = exp2f(ml[2 * q] - M);
-      l = fmaf(ml[2 * q + 1], f, l);
-      const float* src = o + static_cast<int64_t>(q) * D + lane * VEC;
+      const int sq = slot(q);
+      const float f = exp2f(ml[2 * sq] - M);
+      l = fmaf(ml[2 * sq + 1], f, l);
+      const float* src = o + static_cast<int64_t>(sq) * D + lane * VEC;
       if (VEC == 4) {
         const float4 x = *reinterpret_cast<const float4*>(src);
         acc[0] = fmaf(x.x, f, acc[0]);

@@ -303,16 +303,18 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
       int g, s, p;
       item_coords(a, item, g, s, p);
       const int32_t L = load_len(a, s, g == 0 && p == 0 && lane == 0);
-      const int32_t P = a.part_tokens > 0 ? a.part_tokens : (L > 0 ? L : 1);
-      const int32_t t0 = p * P;
-      if (L == 0) {
+      const int32_t sst = seq_start(a, s, L);
+      const int32_t span = L - sst;
+      const int32_t P = a.part_tokens > 0 ? a.part_tokens : (span > 0 ? span : 1);
+      const int32_t t0 = sst + p * P;
+      if (L == 0 && !a.starts) {
         if (p == 0)
           for (int idx = lane; idx < G * D; idx += 32)
             a.out[(static_cast<int64_t>(s) * a.hq + g * G) * D + idx] = 0.f;
       } else if (t0 < L) {
         const int32_t t1 = min(t0 + P, L);
         const int nch = (t1 - t0 + C - 1) / C;
-        const int nparts = a.part_tokens > 0 ? (L + P - 1) / P : 1;
+        const int nparts = a.part_tokens > 0 ? (span + P - 1) / P : 1;
         const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
         for (int ch = 0; ch < nch; ++ch, ++cs) {
           const int st = cs % S;
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
     if (warp == 0) fold_state<NT>(m_run, lrow, o, slot0);
 
     const int64_t row0 = static_cast<int64_t>(ds) * a.hq + dg * G;
-    if (dnp == 1) {
+    if (dnp == 1 && !a.force_partials) {
       if (warp == 0 && r < G) {
         const float inv = 1.f / lrow;
         float* dst = a.out + (row0 + r) * D + 2 * c;
@@ -439,7 +441,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
     }
     // split sequence: publish this partition's (m, l, o); decode_reduce_kernel merges
     if (warp == 0 && r < G) {
-      const int64_t prow = (row0 + r) * a.max_parts + dp;
+      const int64_t prow = (row0 + r) * a.parts_stride + dp;
       float* dst = a.ws_o + prow * D + 2 * c;
 #pragma unroll
       for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);

@@ -19,8 +19,8 @@
 //     TMA byte counts, "empty" mbarriers collect one arrival per consumer
 //     warp, so no warp ever waits on a CTA-wide barrier inside the loop.
 //   * Consumer warp w owns tokens [16w, 16w+16) of a chunk. Each lane reads 16
-//     bytes (8 bf16 or 4 fp32) of a row per load, so LPR = D*elem/16 lanes
-//     cover a row and one warp load covers RPW = 32/LPR rows. Per-lane partial
+//     bytes (8 bf16 or 4 fp32; 8 bytes = 8 e4m3 codes for fp8) of a row per load, so LPR = D / (elements per
+//     load) lanes cover a row and one warp load covers RPW = 32/LPR rows. Per-lane partial
 //     dot products of the NV = 16/RPW tokens a lane touched are summed across
 //     the LPR lanes of its row group with a transposing butterfly (each step
 //     halves the values a lane carries), after which lane (h, sub) holds the
@@ -39,9 +39,16 @@ namespace pa {
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
 
-// 16 bytes of a row -> floats.
+// Bytes of a row one lane loads: 16, except 8 for fp8 so that a lane holds
+// the same 8 elements (and registers) as with bf16.
 template <typename T>
-__device__ __forceinline__ void load16(const T* p, float (&f)[16 / Elem<T>::bytes]);
+struct LaneBytes {
+  static constexpr int value = Elem<T>::bytes == 1 ? 8 : 16;
+};
+
+// One lane's bytes of a row -> floats.
+template <typename T>
+__device__ __forceinline__ void load16(const T* p, float (&f)[LaneBytes<T>::value / Elem<T>::bytes]);
 
 template <>
 __device__ __forceinline__ void load16<float>(const float* p, float (&f)[4]) {
@@ -62,6 +69,20 @@ __device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, fl
   f[5] = bf16hi(x.z);
   f[6] = bf16lo(x.w);
   f[7] = bf16hi(x.w);
+}
+template <>
+__device__ __forceinline__ void load16<__nv_fp8_e4m3>(const __nv_fp8_e4m3* p, float (&f)[8]) {
+  const uint2 x = *reinterpret_cast<const uint2*>(p);
+  const uint32_t w[2] = {x.x, x.y};
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const float2 a = fp8x2_to_float2(static_cast<uint16_t>(w[u] & 0xffffu));
+    const float2 b = fp8x2_to_float2(static_cast<uint16_t>(w[u] >> 16));
+    f[4 * u + 0] = a.x;
+    f[4 * u + 1] = a.y;
+    f[4 * u + 2] = b.x;
+    f[4 * u + 3] = b.y;
+  }
 }
 
 // Sum NV values over the LPR lanes of a row group; lanes halve the values they
@@ -97,7 +118,7 @@ struct SimtCfg {
   static constexpr int kThreads = 32 * (kConsumerWarps + 1);
   static constexpr int kTokPerWarp = 16;
   static constexpr int kChunk = kTokPerWarp * kConsumerWarps;  // tokens per stage
-  static constexpr int kEPL = 16 / Elem<T>::bytes;             // elements per lane load
+  static constexpr int kEPL = LaneBytes<T>::value / Elem<T>::bytes;  // elements per lane load
   static constexpr int kLPR = D / kEPL;                        // lanes per row
   static constexpr int kRPW = 32 / kLPR;                       // rows per warp load
   static constexpr int kNV = kTokPerWarp / kRPW;               // token partials per lane
@@ -179,9 +200,10 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
     float qv[G][EPL];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const T* qp = static_cast<const T*>(a.q) + (static_cast<int64_t>(s) * a.hq + hq0 + h) * D + sub * EPL;
+      using QT = typename QueryOf<T>::type;
+      const QT* qp = static_cast<const QT*>(a.q) + (static_cast<int64_t>(s) * a.hq + hq0 + h) * D + sub * EPL;
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) qv[h][e] = to_f<T>(qp[e]) * a.scale_log2;
+      for (int e = 0; e < EPL; ++e) qv[h][e] = to_f<QT>(qp[e]) * a.scale_log2;
     }
     const int my_j = (sub >> REP) & (NV - 1);
     const int my_tok = my_j * RPW + hrow;        // token (within the warp's 16) whose score this lane holds
@@ -247,7 +269,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
       __syncwarp();
       if (lane == 0) mbar_arrive(&ps.empty[st]);
     }
-    // fold the row groups of the warp together
+    // fold the row groups of the warp together (and apply an fp8 V scale)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       lsum[h] = warp_sum(lsum[h]);
@@ -255,6 +277,10 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
       for (int o = LPR; o < 32; o <<= 1)
 #pragma unroll
         for (int e = 0; e < EPL; ++e) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], o);
+      if (Elem<T>::bytes == 1) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[h][e] *= a.v_scale;
+      }
     }
   }
 

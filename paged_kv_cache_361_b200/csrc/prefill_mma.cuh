@@ -24,14 +24,23 @@
 namespace pa {
 
 struct PrefillArgs {
-  const void* q;          // [T][hq][D] bf16
-  const int32_t* cu_q;    // [num_seqs + 1] prefix sums of new-token counts
+  const void* q;          // prefill: [T][hq][D] new tokens; cascade: [num_seqs][hq][D] decode queries (bf16)
+  const int32_t* cu_q;    // [num_seqs + 1] prefix sums of new-token counts (prefill)
   const int32_t* tables;  // [num_seqs][max_blocks]
-  const int32_t* lens;    // [num_seqs] context length including the new tokens
-  float* out;             // [T][hq][D]
+  const int32_t* lens;    // [num_seqs] context length including the new tokens (prefill)
+  float* out;             // [T][hq][D] (prefill)
   int64_t num_blocks;
   int32_t num_seqs, hq, hkv, bs, max_blocks, max_ctx, ntiles;
   float scale_log2;
+  // cascade (shared-prefix) mode: group j = members[offs[j] .. offs[j+1]) shares
+  // its first prefix_tokens[j] tokens; CTA (g, p, j) writes the partial of
+  // prefix partition p for every member row into slot max_parts + p.
+  const int32_t* group_offs;
+  const int32_t* group_members;
+  const int32_t* group_prefix;
+  int32_t prefix_part_tokens, max_parts, parts_stride;
+  float* ws_ml;
+  float* ws_o;
 };
 
 // d += A(16x16) * B(16x8), all 16 rows live.
@@ -44,7 +53,10 @@ __device__ __forceinline__ void mma16(float (&d)[4], uint32_t a0, uint32_t a1, u
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int D, int G>
+// CASCADE = false: prefill (rows = new tokens x heads, causal).
+// CASCADE = true: shared-prefix decode (rows = group members x heads, every
+// row sees the whole prefix partition; partial results, not rows, are stored).
+template <int D, int G, bool CASCADE>
 __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                          const __grid_constant__ CUtensorMap tmv,
                                                                          const PrefillArgs a) {
@@ -56,34 +68,49 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
   __shared__ PipeSmem<S> ps;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
 
-  const int g = blockIdx.x, s = blockIdx.z;
-  const int tile = a.ntiles - 1 - static_cast<int>(blockIdx.y);
+  const int g = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  const int32_t q0 = __ldg(a.cu_q + s);
-  int32_t n = __ldg(a.cu_q + s + 1) - q0;
-  int32_t L = __ldg(a.lens + s);
-  if (L < 0 || L > a.max_ctx || n < 0 || n > L) {
-    if (tid == 0 && g == 0 && tile == 0) record_error(PA_ERR_DEVICE_BOUNDS, L);
-    L = L < 0 ? 0 : (L > a.max_ctx ? a.max_ctx : L);
-    n = n < 0 ? 0 : (n > L ? L : n);
+  // key range [k_begin, kend) of this CTA and the mapping of its 64 rows
+  int32_t k_begin = 0, kend = 0, base = 0, tok0 = 0, n = 0, q0 = 0, moff = 0, msz = 0;
+  int64_t table_row;
+  if (CASCADE) {
+    const int j = blockIdx.z, p = blockIdx.y;
+    moff = __ldg(a.group_offs + j);
+    msz = __ldg(a.group_offs + j + 1) - moff;
+    const int32_t lp = __ldg(a.group_prefix + j);
+    k_begin = p * a.prefix_part_tokens;
+    if (msz <= 0 || msz > TT || k_begin >= lp) return;
+    kend = min(k_begin + a.prefix_part_tokens, lp);
+    table_row = static_cast<int64_t>(__ldg(a.group_members + moff)) * a.max_blocks;
+  } else {
+    const int s = blockIdx.z;
+    const int tile = a.ntiles - 1 - static_cast<int>(blockIdx.y);
+    q0 = __ldg(a.cu_q + s);
+    n = __ldg(a.cu_q + s + 1) - q0;
+    int32_t L = __ldg(a.lens + s);
+    if (L < 0 || L > a.max_ctx || n < 0 || n > L) {
+      if (tid == 0 && g == 0 && tile == 0) record_error(PA_ERR_DEVICE_BOUNDS, L);
+      L = L < 0 ? 0 : (L > a.max_ctx ? a.max_ctx : L);
+      n = n < 0 ? 0 : (n > L ? L : n);
+    }
+    tok0 = tile * TT;
+    if (tok0 >= n) return;
+    const int32_t tok_end = min(tok0 + TT, n);
+    base = L - n;             // position of new token 0
+    kend = base + tok_end;    // keys 0 .. kend-1 are needed
+    table_row = static_cast<int64_t>(s) * a.max_blocks;
   }
-  const int32_t tok0 = tile * TT;
-  if (tok0 >= n) return;
-  const int32_t tok_end = min(tok0 + TT, n);
-  const int32_t base = L - n;              // position of new token 0
-  const int32_t kend = base + tok_end;     // keys 0 .. kend-1 are needed
-  const int nchunks = (kend + C - 1) / C;
+  const int nchunks = (kend - k_begin + C - 1) / C;
 
   if (tid == 0) pipe_init<S>(ps, NW);
   __syncthreads();
 
   if (warp == NW) {
-    const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
-      const int32_t c0 = i * C;
+      const int32_t c0 = k_begin + i * C;
       const int32_t nb = (min(C, kend - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
       int32_t blk = -1;
       bool ok = false;
@@ -111,15 +138,32 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
   // ---- consumers: warp w owns tile rows [16w, 16w+16); this lane rows ra, rb = ra + 8 ----
   const int c = lane & 3;
   const int ra = warp * 16 + (lane >> 2), rb = ra + 8;
-  const int ta = tok0 + ra / G, tb = tok0 + rb / G;
-  const bool va = ta < n, vb = tb < n;
-  const int pa_ = va ? base + ta : -1, pb_ = vb ? base + tb : -1;  // last key each row may see
-  const int wmax = base + min(tok0 + (warp * 16 + 15) / G, n - 1);  // last key any row of this warp sees
+  bool va, vb;
+  int pa_, pb_, wmax;
+  int64_t qrow_a, qrow_b;  // q row (and output row) of each
+  if (CASCADE) {
+    va = ra / G < msz;
+    vb = rb / G < msz;
+    pa_ = va ? kend - 1 : -1;
+    pb_ = vb ? kend - 1 : -1;
+    wmax = kend - 1;
+    const int sa = va ? __ldg(a.group_members + moff + ra / G) : 0;
+    const int sb = vb ? __ldg(a.group_members + moff + rb / G) : 0;
+    qrow_a = static_cast<int64_t>(sa) * a.hq + g * G + ra % G;
+    qrow_b = static_cast<int64_t>(sb) * a.hq + g * G + rb % G;
+  } else {
+    const int ta = tok0 + ra / G, tb = tok0 + rb / G;
+    va = ta < n;
+    vb = tb < n;
+    pa_ = va ? base + ta : -1;  // last key each row may see
+    pb_ = vb ? base + tb : -1;
+    wmax = base + min(tok0 + (warp * 16 + 15) / G, n - 1);  // last key any row of this warp sees
+    qrow_a = (static_cast<int64_t>(q0) + (va ? ta : 0)) * a.hq + g * G + ra % G;
+    qrow_b = (static_cast<int64_t>(q0) + (vb ? tb : 0)) * a.hq + g * G + rb % G;
+  }
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q);
-  const uint32_t* qra = reinterpret_cast<const uint32_t*>(
-      qb + ((static_cast<int64_t>(q0) + (va ? ta : 0)) * a.hq + g * G + ra % G) * D);
-  const uint32_t* qrb = reinterpret_cast<const uint32_t*>(
-      qb + ((static_cast<int64_t>(q0) + (vb ? tb : 0)) * a.hq + g * G + rb % G) * D);
+  const uint32_t* qra = reinterpret_cast<const uint32_t*>(qb + qrow_a * D);
+  const uint32_t* qrb = reinterpret_cast<const uint32_t*>(qb + qrow_b * D);
   uint32_t qa[D / 16][4];
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
@@ -137,7 +181,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
   for (int i = 0; i < nchunks; ++i) {
     const int st = i % S;
     if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
-    const int k0 = i * C;
+    const int k0 = k_begin + i * C;
     if (k0 <= wmax) {
       const uint32_t kst = sbase + st * Cfg::kStageBytes;
       const uint32_t vst = kst + Cfg::kTileBytes;
@@ -240,15 +284,34 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
   la += __shfl_xor_sync(0xffffffffu, la, 2);
   lb += __shfl_xor_sync(0xffffffffu, lb, 1);
   lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+  if (CASCADE) {
+    // partials of prefix partition blockIdx.y: unnormalised o, (m, l)
+    const int slot = a.max_parts + static_cast<int>(blockIdx.y);
+    if (va) {
+      const int64_t prow = qrow_a * a.parts_stride + slot;
+      float* dst = a.ws_o + prow * D + 2 * c;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
+      if (c == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(ma, la);
+    }
+    if (vb) {
+      const int64_t prow = qrow_b * a.parts_stride + slot;
+      float* dst = a.ws_o + prow * D + 2 * c;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][2], o[j][3]);
+      if (c == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(mb, lb);
+    }
+    return;
+  }
   if (va) {
     const float inv = 1.f / la;
-    float* dst = a.out + ((static_cast<int64_t>(q0) + ta) * a.hq + g * G + ra % G) * D + 2 * c;
+    float* dst = a.out + qrow_a * D + 2 * c;
 #pragma unroll
     for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0] * inv, o[j][1] * inv);
   }
   if (vb) {
     const float inv = 1.f / lb;
-    float* dst = a.out + ((static_cast<int64_t>(q0) + tb) * a.hq + g * G + rb % G) * D + 2 * c;
+    float* dst = a.out + qrow_b * D + 2 * c;
 #pragma unroll
     for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][2] * inv, o[j][3] * inv);
   }

@@ -31,7 +31,7 @@ struct StepLayout {
 bool make_layout(int32_t n, int32_t hq, const pa_cache* c, int32_t max_ctx, int32_t P, StepLayout& L) {
   if (!c || n < 0 || hq <= 0 || max_ctx < 0 || c->block_size <= 0 || c->head_dim <= 0 || c->num_kv_heads <= 0)
     return false;
-  const size_t eb = c->dtype == PA_BF16 ? 2 : 4;
+  const size_t eb = c->dtype == PA_F32 ? 4 : 2;  // q, k, v inputs: bf16 for a bf16 or fp8 cache
   const size_t N = static_cast<size_t>(n);
   L.cap = std::max<int32_t>(1, (max_ctx + c->block_size - 1) / c->block_size);
   L.m_slots = 0;
@@ -105,7 +105,7 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* d = static_cast<char*>(dev_staging);
-  const size_t eb = cache->dtype == PA_BF16 ? 2 : 4;
+  const size_t eb = cache->dtype == PA_F32 ? 4 : 2;
   const size_t qb = static_cast<size_t>(n) * num_q_heads * cache->head_dim * eb;
   const size_t kb = static_cast<size_t>(n) * cache->num_kv_heads * cache->head_dim * eb;
   if (cudaMemcpyAsync(d + L.meta, h, L.meta_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||

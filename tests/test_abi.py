@@ -52,12 +52,28 @@ def _cache(**kw):
     (dict(block_size=3), B.PA_ERR_UNSUPPORTED),
     (dict(block_size=64), B.PA_ERR_UNSUPPORTED),
     (dict(dtype=7), B.PA_ERR_UNSUPPORTED),
+    (dict(dtype=B.PA_FP8_E4M3), B.PA_ERR_INVALID_ARG),                                  # scales 0
+    (dict(dtype=B.PA_FP8_E4M3, k_scale=1.0, v_scale=float("nan")), B.PA_ERR_INVALID_ARG),
+    (dict(dtype=B.PA_FP8_E4M3, k_scale=-1.0, v_scale=1.0), B.PA_ERR_INVALID_ARG),
+    (dict(dtype=B.PA_FP8_E4M3, k_scale=float("inf"), v_scale=1.0), B.PA_ERR_INVALID_ARG),
 ])
 def test_host_checks_before_launch(kw, status):
     lib = B._lib()
     c = _cache(**kw)
     assert lib.pa_reshape_and_cache(16, 16, 16, 1, ctypes.byref(c), None) == status
     assert lib.pa_copy_blocks(ctypes.byref(c), 16, 1, None) == status
+
+
+def test_fp8_cache_needs_its_scales():
+    import torch
+    kc = torch.zeros(4, 1, 16, 64, dtype=torch.float8_e4m3fn)
+    vc = torch.zeros_like(kc)
+    with pytest.raises(ValueError, match="scales"):
+        B.make_cache(kc, vc)
+    with pytest.raises(TypeError):
+        B.set_fp8_scales(kc.float(), vc.float(), 1.0, 1.0)
+    assert B.input_dtype(torch.float8_e4m3fn) == torch.bfloat16
+    assert B.input_dtype(torch.float32) == torch.float32
 
 
 def test_decode_argument_checks():

@@ -91,3 +91,52 @@ def test_prefix_caching_trace():
     assert st == B.PA_OK, (st, info)
     r.check_pool_rows()
     assert r.cache.bm.prefix_stats() == r.oracle.bm.prefix_stats()
+
+
+def test_parallel_sampling_cascade():
+    """Shared-prefix decode on the parallel-sampling workload: each prompt's
+    prefix blocks are read once for its 8 samples; outputs match the oracle."""
+    w = W.parallel_sampling()
+    r = Replay(w.shape, w.num_blocks, w.free_order, w.scale, keep_pool=False)
+    ops = W.sampling_ops(w, batch_tail_steps=True)
+    for op in ops[:-1]:
+        r.apply(op)
+    ids, qsrc = ops[-1][1], ops[-1][2]
+    q = qsrc()
+    r.oracle.apply(ops[-1])
+    out = r.cache.decode_cascade(ids, q.cuda(), w.scale).cpu()
+    st, info = B.pa_get_device_error()
+    assert st == B.PA_OK, (st, info)
+    tables, lens, _ = r.cache.decode_inputs(ids)
+    offs, members, prefix, seq_prefix = r.cache.shared_prefix_groups(ids, tables, lens, 16)
+    assert len(prefix) == 8 and (prefix == 960).all()      # 62 shared blocks of 16 -> 960 tokens
+    r.decodes.append((list(ids), q, out))
+    r.check_outputs()
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_cascade_random_groups(G):
+    """Forked families with random suffixes (and lone sequences) against pa_decode."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    rng = np.random.default_rng(G)
+    hkv, D, bs = 2, 128, 16
+    cache = PagedKVCache(4000, hkv, bs, D, torch.bfloat16, "cuda", rng.permutation(4000), fill=float("nan"))
+    g = torch.Generator().manual_seed(G)
+    ids = []
+    for fam in range(5):
+        root = fam * 100
+        n0 = int(rng.integers(64, 700))
+        cache.add_sequence(root, torch.randn(n0, hkv, D, generator=g).bfloat16().cuda(),
+                           torch.randn(n0, hkv, D, generator=g).bfloat16().cuda())
+        ids.append(root)
+        for j in range(1, int(rng.integers(1, 64 // G + 3))):
+            cache.fork(root, root + j)
+            ids.append(root + j)
+    for _ in range(int(rng.integers(1, 40))):       # private suffixes
+        k = torch.randn(len(ids), hkv, D, generator=g).bfloat16().cuda()
+        cache.append(ids, k, k)
+    q = torch.randn(len(ids), hkv * G, D, generator=g).bfloat16().cuda()
+    a = cache.decode(ids, q, D ** -0.5)
+    b = cache.decode_cascade(ids, q, D ** -0.5)
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    assert float((a - b).abs().max()) <= 2e-3

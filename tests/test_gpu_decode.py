@@ -288,3 +288,32 @@ def test_prefill_then_decode_consistent():
     out = cache.prefill([7], [300], q, k, v, 128 ** -0.5)
     dec = cache.decode([7], q[-1:], 128 ** -0.5)
     assert float((out[-1] - dec[0]).abs().max()) <= 2e-3
+
+
+def test_step_plan_matches_oracle():
+    """The prepared pa_step_host call (one native call per step) over three steps."""
+    from oracle.replay import OracleRun
+    g = torch.Generator().manual_seed(8)
+    sh = W.Shape(4, 4, 64, 8, "bf16")
+    ref = OracleRun(sh, 40, list(range(40)), keep_pool=True)
+    cache = PagedKVCache(40, 4, 8, 64, torch.bfloat16, "cuda", list(range(40)), fill=float("nan"))
+    for s, n in ((0, 13), (1, 30), (2, 1)):
+        k, v = torch.randn(n, 4, 64, generator=g).bfloat16(), torch.randn(n, 4, 64, generator=g).bfloat16()
+        ref.apply(("add", s, n, lambda which, device="cpu", k=k, v=v: k if which == "k" else v))
+        cache.add_sequence(s, k.cuda(), v.cuda())
+    ids = [1, 0, 2]
+    q = torch.empty(3, 4, 64, dtype=torch.bfloat16).pin_memory()
+    k = torch.empty(3, 4, 64, dtype=torch.bfloat16).pin_memory()
+    v = torch.empty(3, 4, 64, dtype=torch.bfloat16).pin_memory()
+    out = torch.empty(3, 4, 64).pin_memory()
+    plan = cache.step_plan(ids, q, k, v, out, 0.125, max_context_len=64)
+    for step in range(3):
+        q.copy_(torch.randn(3, 4, 64, generator=g).bfloat16())
+        k.copy_(torch.randn(3, 4, 64, generator=g).bfloat16())
+        v.copy_(torch.randn(3, 4, 64, generator=g).bfloat16())
+        kk, vv = k.clone(), v.clone()
+        ref.apply(("append", ids, lambda which, device="cpu": kk if which == "k" else vv))
+        plan.run()
+        for i, s in enumerate(ids):
+            exp = ref.attend(s, q[i], 0.125, use_pool=True)
+            assert float(np.abs(out[i].double().numpy() - exp).max()) <= TOL["bf16"]
