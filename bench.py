@@ -524,7 +524,8 @@ def run_prefill(args, rank, world, device):
             "roofline": {"kernel": "pa_prefill", "bound": "tensor", "achieved": round(flops / (pf_ms * 1e-3) / 1e12, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(flops / (pf_ms * 1e-3) / 1e12 / peak, 4),
                          "traffic": None, "peak_source": src,
-                         "note": "mma.sync m16n8k16 with P split into two bf16 MMAs (1.5x the algorithmic MMA work)"},
+                         "note": "tcgen05.mma (M 128) with TMEM accumulators; P split into two bf16 MMAs "
+                                 "(1.5x the algorithmic MMA work)"},
             "clocks": clk}), flush=True)
 
 

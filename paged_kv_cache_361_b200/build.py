@@ -19,7 +19,8 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libpagedattn.so")
 
 SOURCES = ["capi.cu", "block_manager.cpp", "step.cpp"]
-DEPS = ["common.cuh", "cache_ops.cuh", "decode_common.cuh", "decode_simt.cuh", "decode_mma.cuh", "prefill_mma.cuh"]
+DEPS = ["common.cuh", "cache_ops.cuh", "decode_common.cuh", "decode_simt.cuh", "decode_mma.cuh", "prefill_mma.cuh",
+        "tcgen05.cuh", "prefill_tc.cuh"]
 
 
 def nvcc() -> str:

@@ -10,6 +10,7 @@
 #include "decode_mma.cuh"
 #include "decode_simt.cuh"
 #include "prefill_mma.cuh"
+#include "prefill_tc.cuh"
 
 namespace {
 
@@ -351,7 +352,7 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
       (reinterpret_cast<uintptr_t>(cu_q_lens) & 3) || (reinterpret_cast<uintptr_t>(block_tables) & 3) ||
       (reinterpret_cast<uintptr_t>(context_lens) & 3))
     return PA_ERR_INVALID_ARG;
-  const int tt = 64 / G;
+  const int tt = TcCfg<128>::kRows / G;  // tokens per 128-row tile
   const int64_t ntiles = (static_cast<int64_t>(max_q_len) + tt - 1) / tt;
   if (num_seqs > 65535 || ntiles > 65535) return PA_ERR_UNSUPPORTED;
   PrefillArgs a;
@@ -382,22 +383,22 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   auto launch = [&](auto kern, int smem) -> pa_status {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return PA_ERR_CUDA;
-    kern<<<grid, MmaCfg<128>::kThreads, smem, s>>>(tk, tv, a);
+    kern<<<grid, TcCfg<128>::kThreads, smem, s>>>(tk, tv, a);
     return launched();
   };
   if (cache->head_dim == 128) {
     switch (G) {
-      case 1: return launch(prefill_mma_kernel<128, 1, false>, MmaCfg<128>::kSmemBytes);
-      case 2: return launch(prefill_mma_kernel<128, 2, false>, MmaCfg<128>::kSmemBytes);
-      case 4: return launch(prefill_mma_kernel<128, 4, false>, MmaCfg<128>::kSmemBytes);
-      default: return launch(prefill_mma_kernel<128, 8, false>, MmaCfg<128>::kSmemBytes);
+      case 1: return launch(prefill_tc_kernel<128, 1>, TcCfg<128>::kSmemBytes);
+      case 2: return launch(prefill_tc_kernel<128, 2>, TcCfg<128>::kSmemBytes);
+      case 4: return launch(prefill_tc_kernel<128, 4>, TcCfg<128>::kSmemBytes);
+      default: return launch(prefill_tc_kernel<128, 8>, TcCfg<128>::kSmemBytes);
     }
   }
   switch (G) {
-    case 1: return launch(prefill_mma_kernel<64, 1, false>, MmaCfg<64>::kSmemBytes);
-    case 2: return launch(prefill_mma_kernel<64, 2, false>, MmaCfg<64>::kSmemBytes);
-    case 4: return launch(prefill_mma_kernel<64, 4, false>, MmaCfg<64>::kSmemBytes);
-    default: return launch(prefill_mma_kernel<64, 8, false>, MmaCfg<64>::kSmemBytes);
+    case 1: return launch(prefill_tc_kernel<64, 1>, TcCfg<64>::kSmemBytes);
+    case 2: return launch(prefill_tc_kernel<64, 2>, TcCfg<64>::kSmemBytes);
+    case 4: return launch(prefill_tc_kernel<64, 4>, TcCfg<64>::kSmemBytes);
+    default: return launch(prefill_tc_kernel<64, 8>, TcCfg<64>::kSmemBytes);
   }
 }
 

@@ -254,7 +254,8 @@ def test_prefill_chunked_matches_oracle(G, D, bs):
     pre = rng.integers(0, 300, size=nseq)
     pre[0] = 0
     chunk = rng.integers(1, 200, size=nseq)
-    chunk[1] = 64 // G            # exactly one query tile
+    chunk[1] = 128 // G           # exactly one 128-row query tile
+    chunk[2] = 64 // G            # half a tile
     nb = int(sum(-(-int(p + c) // bs) for p, c in zip(pre, chunk))) + 4
     cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, "cuda", rng.permutation(nb), fill=float("nan"))
     g = torch.Generator().manual_seed(int(rng.integers(1 << 30)))
@@ -275,6 +276,29 @@ def test_prefill_chunked_matches_oracle(G, D, bs):
         err = float(np.abs(out[row:row + n].double().numpy() - ref).max())
         assert err <= TOL["bf16"], f"seq {s}: {err}"
         row += n
+
+
+@pytest.mark.parametrize("G,D", [(1, 128), (8, 128), (4, 64)])
+def test_prefill_long_chunk_many_tiles(G, D):
+    """A 700-token chunk after 900 cached tokens: many query tiles and 25 key
+    chunks, a ragged last tile and last key chunk, NaN padding in the pool."""
+    from oracle.prefill import prefill_attention
+    hkv, bs = 2, 16
+    g = torch.Generator().manual_seed(40 + G + D)
+    pre, n = 900, 700
+    nb = -(-(pre + n) // bs) + 3
+    cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, "cuda", np.random.default_rng(G).permutation(nb),
+                         fill=float("nan"))
+    K = torch.randn(pre + n, hkv, D, generator=g).bfloat16()
+    V = torch.randn(pre + n, hkv, D, generator=g).bfloat16()
+    cache.add_sequence(0, K[:pre].cuda(), V[:pre].cuda())
+    q = torch.randn(n, hkv * G, D, generator=g).bfloat16()
+    out = cache.prefill([0], [n], q.cuda(), K[pre:].cuda(), V[pre:].cuda(), D ** -0.5).cpu()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    rows = np.r_[0:40, 300:340, n - 40:n]
+    ref = prefill_attention(q, K, V, D ** -0.5)
+    err = float(np.abs(out.double().numpy()[rows] - ref[rows]).max())
+    assert err <= TOL["bf16"], err
 
 
 def test_prefill_then_decode_consistent():
