@@ -20,7 +20,7 @@ LIB = os.path.join(HERE, "libpagedattn.so")
 
 SOURCES = ["capi.cu", "block_manager.cpp", "step.cpp"]
 DEPS = ["common.cuh", "cache_ops.cuh", "decode_common.cuh", "decode_simt.cuh", "decode_mma.cuh", "prefill_mma.cuh",
-        "tcgen05.cuh", "prefill_tc.cuh"]
+        "tcgen05.cuh", "prefill_tc.cuh", "decode_f8.cuh"]
 
 
 def nvcc() -> str:

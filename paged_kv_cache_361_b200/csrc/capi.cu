@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include "cache_ops.cuh"
+#include "decode_f8.cuh"
 #include "decode_mma.cuh"
 #include "decode_simt.cuh"
 #include "prefill_mma.cuh"
@@ -145,6 +146,53 @@ bool encode_rows(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) {
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// An e4m3 pool viewed as rows of head_dim bytes, read in [bs x head_dim] boxes
+// with the 128-byte (head_dim 128) or 64-byte (head_dim 64) swizzle.
+bool encode_rows_u8(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(bs)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core decode over an e4m3 cache (block_size >= 8, pool rows addressable by the TMA).
+bool f8_mma_eligible(const pa_cache* c) {
+  return c->dtype == PA_FP8_E4M3 && c->block_size >= 8 &&
+         static_cast<int64_t>(c->num_blocks) * c->num_kv_heads * c->block_size <= INT32_MAX;
+}
+
+template <int D, int G>
+pa_status launch_f8(const DecodeArgs& a, const pa_cache* c, dim3 grid, cudaStream_t st) {
+  using Cfg = F8Cfg<D>;
+  CUtensorMap tk, tv;
+  const uint64_t rows = static_cast<uint64_t>(c->num_blocks) * c->num_kv_heads * c->block_size;
+  if (!encode_rows_u8(&tk, c->k, rows, D, c->block_size) || !encode_rows_u8(&tv, c->v, rows, D, c->block_size))
+    return PA_ERR_CUDA;
+  auto kern = decode_f8_kernel<D, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+          cudaSuccess)
+    return PA_ERR_CUDA;
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
+  return launched();
+}
+
+template <int D>
+pa_status dispatch_f8(const DecodeArgs& a, const pa_cache* c, int G, dim3 grid, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_f8<D, 1>(a, c, grid, st);
+    case 2: return launch_f8<D, 2>(a, c, grid, st);
+    case 4: return launch_f8<D, 4>(a, c, grid, st);
+    case 8: return launch_f8<D, 8>(a, c, grid, st);
+    default: return PA_ERR_UNSUPPORTED;
+  }
 }
 
 template <int D, int G>
@@ -631,6 +679,8 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   const int D = cache->head_dim;
   if (mma_eligible(cache, G)) {
     st = dispatch_mma(a, cache, G, s);
+  } else if (f8_mma_eligible(cache)) {
+    st = D == 128 ? dispatch_f8<128>(a, cache, G, grid, s) : dispatch_f8<64>(a, cache, G, grid, s);
   } else if (cache->dtype == PA_FP8_E4M3) {
     st = D == 128 ? dispatch_g<__nv_fp8_e4m3, 128>(a, G, grid, s) : dispatch_g<__nv_fp8_e4m3, 64>(a, G, grid, s);
   } else if (cache->dtype == PA_BF16) {

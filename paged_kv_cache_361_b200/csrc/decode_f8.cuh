@@ -1,0 +1,291 @@
+// Paged decode attention over an 8-bit (e4m3) KV cache, on the tensor cores.
+//
+// P2 = "PagedAttention：操作系统级 KV 缓存虚拟内存管理".
+//   §1.1  out = softmax(scale * q K^T) V.
+//   §3.2.2 step 4, §4.1  every logical block is visited through the block
+//         table; the softmax is accumulated chunk by chunk.
+// P3 = "PagedAttention 和 vLLM", the section on its future: paged KV storage
+//   combined with quantisation. A code c stands for value(c) * scale, one
+//   scale per tensor.
+//
+// Half the bytes of a bf16 cache per token, so the conversion work per byte
+// doubles; widening every element to fp32 on the CUDA cores runs out of
+// conversion throughput long before HBM does. Here each element is widened
+// once, two at a time (cvt e4m3x2 -> f16x2, exact), straight into the operand
+// registers of m16n8k16 f16 MMAs with fp32 accumulation:
+//   S = Q K^T : A = q (bf16 -> f16, exact for |q| < 65504) in registers,
+//               B = K from shared memory with one 32-bit load per thread per
+//               16 dims. The 16 dims a k-step contracts are taken in the
+//               order that makes a thread's two B registers four adjacent
+//               bytes (dims 4c..4c+3 of the step); Q uses the same order.
+//   O += P V  : A = P as f16 (11 mantissa bits: one MMA, no split), B = V.
+//               Thread (g, c) feeds output columns 16g + j (D 128; 8g + j at
+//               D 64) of n-tile j, so it reads one 16-byte (8-byte) piece of
+//               each of its four tokens' V rows and pairs tokens with byte
+//               permutes before widening.
+// K/V tiles arrive as TMA tensor copies of [block_size rows x D bytes] with
+// the 128-byte (D 128) or 64-byte (D 64) swizzle, so the row-strided loads
+// above are free of bank conflicts (D 128). The K scale is folded into the
+// score scale, the V scale multiplies O before the merge. Tokens past the
+// context length get -inf scores and zeroed V operands (their bytes may be
+// NaN codes), as in the other decode kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "decode_common.cuh"
+#include "decode_mma.cuh"
+
+namespace pa {
+
+template <int D>
+struct F8Cfg {
+  static constexpr int kConsumerWarps = 4;
+  static constexpr int kThreads = 32 * (kConsumerWarps + 1);
+  static constexpr int kChunk = 64;                 // tokens per stage
+  static constexpr int kTileBytes = kChunk * D;     // K (or V) of one stage
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = 4;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;
+  static constexpr int kNT = D / 8;                 // output n-tiles
+};
+
+// Byte offset of (row, byte column) in a swizzled tile of D-byte rows, as the
+// TMA writes it: 16-byte chunk index XOR the row's position in the swizzle
+// atom (128-byte swizzle: row & 7; 64-byte swizzle: (row >> 1) & 3).
+template <int D>
+__device__ __forceinline__ uint32_t f8_off(int row, int col) {
+  if (D == 128) return row * 128 + ((((col >> 4) ^ (row & 7)) << 4) | (col & 15));
+  return row * 64 + ((((col >> 4) ^ ((row >> 1) & 3)) << 4) | (col & 15));
+}
+
+// Two e4m3 codes (low byte first) -> f16x2 (low half first), exact.
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// m16n8k16 f16 MMA with rows 8..15 of A zero and their results discarded.
+__device__ __forceinline__ void mma_f16_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  float j2, j3;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %12};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(j2), "=f"(j3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f));
+  asm volatile("" ::"f"(j2), "f"(j3));
+}
+
+// Output dim of n-tile j, column n.
+template <int D>
+__device__ __forceinline__ int f8_dim(int j, int n) {
+  return (D == 128 ? 16 : 8) * n + j;
+}
+
+// One consumer warp's 16 tokens (nv valid) of a stage.
+template <int D>
+__device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, int nv,
+                                         const uint32_t (&qa)[D / 16][2], float scale_log2, int lane, int warp,
+                                         float& m_run, float& l_run, float (&o)[D / 8][2]) {
+  constexpr int NT = D / 8;
+  const int gq = lane >> 2, c = lane & 3;
+  const int tw = warp * 16;
+  float sacc[2][2];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    sacc[nt][0] = sacc[nt][1] = 0.f;
+    const int row = tw + nt * 8 + gq;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(kt + f8_off<D>(row, kk * 16 + 4 * c));
+      mma_f16_rows8(sacc[nt], qa[kk][0], qa[kk][1], e4m3x2_f16x2(w), e4m3x2_f16x2(w >> 16));
+    }
+  }
+  float sc[2][2];
+  float mloc = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int t = nt * 8 + 2 * c + j;
+      sc[nt][j] = t < nv ? sacc[nt][j] * scale_log2 : -INFINITY;
+      mloc = fmaxf(mloc, sc[nt][j]);
+    }
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+  const float mn = fmaxf(m_run, mloc);
+  const float alpha = exp2f(m_run - mn);
+  m_run = mn;
+  float pr[2][2];
+  float psum = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      pr[nt][j] = exp2f(sc[nt][j] - mn);
+      psum += pr[nt][j];
+    }
+  l_run = l_run * alpha + psum;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    o[j][0] *= alpha;
+    o[j][1] *= alpha;
+  }
+  const uint32_t pa0 = pack_f16(pr[0][0], pr[0][1]);  // tokens 2c, 2c+1
+  const uint32_t pa2 = pack_f16(pr[1][0], pr[1][1]);  // tokens 8+2c, 9+2c
+  // masks for tokens past the valid ones (their V bytes may be NaN codes)
+  const uint32_t m0 = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
+  const uint32_t m1 = (2 * c + 8 < nv ? 0x0000ffffu : 0u) | (2 * c + 9 < nv ? 0xffff0000u : 0u);
+  constexpr int W = D == 128 ? 4 : 2;  // 32-bit words of V per token this thread reads
+  uint32_t va[W], vb[W], vc[W], vd[W];
+  const int col = (D == 128 ? 16 : 8) * gq;
+  const int t00 = tw + 2 * c, t10 = tw + 8 + 2 * c;
+  if constexpr (D == 128) {
+    const uint4 x0 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t00, col));
+    const uint4 x1 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t00 + 1, col));
+    const uint4 x2 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t10, col));
+    const uint4 x3 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t10 + 1, col));
+    va[0] = x0.x, va[1] = x0.y, va[2] = x0.z, va[3] = x0.w;
+    vb[0] = x1.x, vb[1] = x1.y, vb[2] = x1.z, vb[3] = x1.w;
+    vc[0] = x2.x, vc[1] = x2.y, vc[2] = x2.z, vc[3] = x2.w;
+    vd[0] = x3.x, vd[1] = x3.y, vd[2] = x3.z, vd[3] = x3.w;
+  } else {
+    const uint2 x0 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t00, col));
+    const uint2 x1 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t00 + 1, col));
+    const uint2 x2 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t10, col));
+    const uint2 x3 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t10 + 1, col));
+    va[0] = x0.x, va[1] = x0.y;
+    vb[0] = x1.x, vb[1] = x1.y;
+    vc[0] = x2.x, vc[1] = x2.y;
+    vd[0] = x3.x, vd[1] = x3.y;
+  }
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    // (token a byte k, token b byte k) pairs: bytes 0,1 then 2,3 of each word
+    const uint32_t p01 = __byte_perm(va[w], vb[w], 0x5140), p23 = __byte_perm(va[w], vb[w], 0x7362);
+    const uint32_t q01 = __byte_perm(vc[w], vd[w], 0x5140), q23 = __byte_perm(vc[w], vd[w], 0x7362);
+    mma_f16_rows8(o[4 * w + 0], pa0, pa2, e4m3x2_f16x2(p01) & m0, e4m3x2_f16x2(q01) & m1);
+    mma_f16_rows8(o[4 * w + 1], pa0, pa2, e4m3x2_f16x2(p01 >> 16) & m0, e4m3x2_f16x2(q01 >> 16) & m1);
+    mma_f16_rows8(o[4 * w + 2], pa0, pa2, e4m3x2_f16x2(p23) & m0, e4m3x2_f16x2(q23) & m1);
+    mma_f16_rows8(o[4 * w + 3], pa0, pa2, e4m3x2_f16x2(p23 >> 16) & m0, e4m3x2_f16x2(q23 >> 16) & m1);
+  }
+}
+
+// One CTA per work item (kv head, sequence, partition); grid (Hkv, B, parts),
+// partition-major. Warp 4 streams the item's K/V tiles; warps 0-3 each take
+// 16 tokens of every 64-token stage; the warps' states are merged through
+// shared memory at the end.
+template <int D, int G>
+__global__ void __launch_bounds__(F8Cfg<D>::kThreads) decode_f8_kernel(const __grid_constant__ CUtensorMap tmk,
+                                                                       const __grid_constant__ CUtensorMap tmv,
+                                                                       const DecodeArgs a) {
+  using Cfg = F8Cfg<D>;
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = Cfg::kNT;
+  static_assert(G <= 8, "query heads of one group must fit in MMA rows 0..7");
+  static_assert(NW * G * (D + 2) * 4 <= S * Cfg::kStageBytes, "merge buffer must fit in the stage ring");
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ PipeSmem<S> ps;
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - sraw);
+
+  const int g = blockIdx.x, s = blockIdx.y, p = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, c = lane & 3;
+  Part pt;
+  if (!cta_part<G, D>(a, g, s, p, tid, Cfg::kThreads, pt)) return;
+  const int nchunks = (pt.ntok + C - 1) / C;
+  const int hq0 = g * G;
+
+  if (tid == 0) pipe_init<S>(ps, NW);
+  __syncthreads();
+
+  float o[NT][2];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+
+  if (warp == NW) {
+    const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
+    const uint64_t pol = l2_evict_first_policy();
+    pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+      const int32_t c0 = pt.t0 + i * C;
+      const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+      int32_t blk = -1;
+      bool ok = false;
+      if (lane < nb) {
+        blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
+        ok = blk >= 0 && blk < a.num_blocks;
+        if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * __popc(okmask) * box_bytes);
+      __syncwarp();
+      if (ok) {
+        const int32_t y = (blk * a.hkv + g) * a.bs;
+        const uint32_t kdst = sbase + st * Cfg::kStageBytes + lane * box_bytes;
+        tma_load_2d(kdst, &tmk, 0, y, &ps.full[st], pol);
+        tma_load_2d(kdst + Cfg::kTileBytes, &tmv, 0, y, &ps.full[st], pol);
+      }
+    });
+  } else {
+    // q rows as f16 A fragments in the dim order of f8_chunk's k-steps:
+    // a0 = dims (16kk + 4c, +1), a2 = dims (16kk + 4c + 2, +3); rows >= G zero
+    uint32_t qa[D / 16][2];
+    const __nv_bfloat16* qrow =
+        static_cast<const __nv_bfloat16*>(a.q) + (static_cast<int64_t>(s) * a.hq + hq0 + (r < G ? r : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      if (r < G) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(qrow + kk * 16 + 4 * c));
+        qa[kk][0] = pack_f16(bf16lo(w.x), bf16hi(w.x));
+        qa[kk][1] = pack_f16(bf16lo(w.y), bf16hi(w.y));
+      } else {
+        qa[kk][0] = qa[kk][1] = 0u;
+      }
+    }
+    for (int i = 0; i < nchunks; ++i) {
+      const int st = i % S;
+      if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
+      const int nv = min(16, min(C, pt.ntok - i * C) - warp * 16);  // warp-uniform
+      if (nv > 0) {
+        const uint8_t* kt = sgen + st * Cfg::kStageBytes;
+        f8_chunk<D>(kt, kt + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ps.empty[st]);
+    }
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  }
+
+  __syncthreads();  // every copy consumed; the stage ring is free
+  if (ps.abort_flag) return;
+
+  float* wm = reinterpret_cast<float*>(sgen);
+  float* wl = wm + NW * G;
+  float* wacc = wl + NW * G;
+  if (warp < NW && r < G) {
+    if (c == 0) {
+      wm[warp * G + r] = m_run;
+      wl[warp * G + r] = l_run;
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      wacc[(warp * G + r) * D + f8_dim<D>(j, 2 * c)] = o[j][0] * a.v_scale;
+      wacc[(warp * G + r) * D + f8_dim<D>(j, 2 * c + 1)] = o[j][1] * a.v_scale;
+    }
+  }
+  __syncthreads();
+  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, tid, Cfg::kThreads);
+}
+
+}  // namespace pa
