@@ -400,8 +400,10 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
       (reinterpret_cast<uintptr_t>(cu_q_lens) & 3) || (reinterpret_cast<uintptr_t>(block_tables) & 3) ||
       (reinterpret_cast<uintptr_t>(context_lens) & 3))
     return PA_ERR_INVALID_ARG;
-  const int tt = TcCfg<128>::kRows / G;  // tokens per 128-row tile
-  const int64_t ntiles = (static_cast<int64_t>(max_q_len) + tt - 1) / tt;
+  // 128-row query tiles; at head_dim 128 two tiles of a sequence share one CTA
+  const int tiles_per_cta = cache->head_dim == 128 ? 2 : 1;
+  const int tt = 128 / G;
+  const int64_t ntiles = ((static_cast<int64_t>(max_q_len) + tt - 1) / tt + tiles_per_cta - 1) / tiles_per_cta;
   if (num_seqs > 65535 || ntiles > 65535) return PA_ERR_UNSUPPORTED;
   PrefillArgs a;
   a.q = q;
@@ -428,25 +430,27 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
     return PA_ERR_CUDA;
   const dim3 grid(cache->num_kv_heads, static_cast<unsigned>(ntiles), num_seqs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  auto launch = [&](auto kern, int smem) -> pa_status {
+  auto launch = [&](auto kern, int threads, int smem) -> pa_status {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return PA_ERR_CUDA;
-    kern<<<grid, TcCfg<128>::kThreads, smem, s>>>(tk, tv, a);
+    kern<<<grid, threads, smem, s>>>(tk, tv, a);
     return launched();
   };
+  using C128 = TcCfg<128, 2>;
+  using C64 = TcCfg<64, 1>;
   if (cache->head_dim == 128) {
     switch (G) {
-      case 1: return launch(prefill_tc_kernel<128, 1>, TcCfg<128>::kSmemBytes);
-      case 2: return launch(prefill_tc_kernel<128, 2>, TcCfg<128>::kSmemBytes);
-      case 4: return launch(prefill_tc_kernel<128, 4>, TcCfg<128>::kSmemBytes);
-      default: return launch(prefill_tc_kernel<128, 8>, TcCfg<128>::kSmemBytes);
+      case 1: return launch(prefill_tc_kernel<128, 1, 2>, C128::kThreads, C128::kSmemBytes);
+      case 2: return launch(prefill_tc_kernel<128, 2, 2>, C128::kThreads, C128::kSmemBytes);
+      case 4: return launch(prefill_tc_kernel<128, 4, 2>, C128::kThreads, C128::kSmemBytes);
+      default: return launch(prefill_tc_kernel<128, 8, 2>, C128::kThreads, C128::kSmemBytes);
     }
   }
   switch (G) {
-    case 1: return launch(prefill_tc_kernel<64, 1>, TcCfg<64>::kSmemBytes);
-    case 2: return launch(prefill_tc_kernel<64, 2>, TcCfg<64>::kSmemBytes);
-    case 4: return launch(prefill_tc_kernel<64, 4>, TcCfg<64>::kSmemBytes);
-    default: return launch(prefill_tc_kernel<64, 8>, TcCfg<64>::kSmemBytes);
+    case 1: return launch(prefill_tc_kernel<64, 1, 1>, C64::kThreads, C64::kSmemBytes);
+    case 2: return launch(prefill_tc_kernel<64, 2, 1>, C64::kThreads, C64::kSmemBytes);
+    case 4: return launch(prefill_tc_kernel<64, 4, 1>, C64::kThreads, C64::kSmemBytes);
+    default: return launch(prefill_tc_kernel<64, 8, 1>, C64::kThreads, C64::kSmemBytes);
   }
 }
 

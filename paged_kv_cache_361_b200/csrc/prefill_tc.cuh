@@ -38,7 +38,7 @@
 
 namespace pa {
 
-template <int D>
+template <int D, int TILES>
 struct TcCfg {
   static constexpr int kRows = 128;                        // query rows per tile (MMA M)
   static constexpr int kChunk = 64;                        // keys per stage
@@ -48,13 +48,17 @@ struct TcCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = 4;
   static constexpr int kQHalfBytes = kRows * 128;
-  static constexpr int kQBytes = kHalves * kQHalfBytes;
+  static constexpr int kQTileBytes = kHalves * kQHalfBytes;
+  static constexpr int kQBytes = TILES * kQTileBytes;
   static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes;
-  static constexpr int kThreads = 192;
-  static constexpr uint32_t kTmemCols = 256;  // O: D columns; S/P: two buffers of 64 after it
-  static constexpr uint32_t kColO = 0;
-  static constexpr uint32_t kColS = D;
-  static_assert(kColS + 2 * kChunk <= kTmemCols, "TMEM columns");
+  static constexpr int kSoftmaxWarps = 4 * TILES;          // one warpgroup per tile
+  static constexpr int kProducerWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  // per tile: O (D columns), then two S/P buffers of kChunk columns
+  static constexpr uint32_t kTileCols = D + 2 * kChunk;
+  static constexpr uint32_t kTmemCols = TILES * kTileCols <= 256 ? 256 : 512;
+  static_assert(TILES * kTileCols <= kTmemCols, "TMEM columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -64,54 +68,78 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(192, 1) prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk,
-                                                            const __grid_constant__ CUtensorMap tmv,
-                                                            const PrefillArgs a) {
-  using Cfg = TcCfg<D>;
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// TILES query tiles of one (kv head, sequence) per CTA share the K/V stream;
+// tile t is processed by softmax warpgroup t.
+template <int D, int G, int TILES>
+__global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                      const PrefillArgs a) {
+  using Cfg = TcCfg<D, TILES>;
   constexpr int S = Cfg::kStages, C = Cfg::kChunk, TT = Cfg::kRows / G;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ PipeSmem<S> ps;
-  __shared__ uint64_t q_full, s_full[2], p_full[2], o_bar, drain;
+  __shared__ uint64_t q_full, drain;
+  __shared__ uint64_t s_full[TILES][2], p_full[TILES][2], o_bar[TILES];
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint8_t* sgen = smem_raw + (sbase - raw);  // generic pointer to sbase
-  const uint32_t qs = sbase;                 // Q: kHalves x [128 rows x 128 B], swizzled
+  uint8_t* sgen = smem_raw + (sbase - raw);   // generic pointer to sbase
+  const uint32_t qs = sbase;                  // Q of tile t: kHalves x [128 rows x 128 B], swizzled
   const uint32_t kv0 = sbase + Cfg::kQBytes;  // stage st: K halves, then V halves
 
   const int g = blockIdx.x, s = blockIdx.z;
-  const int tile = a.ntiles - 1 - static_cast<int>(blockIdx.y);
+  const int pair = a.ntiles - 1 - static_cast<int>(blockIdx.y);  // longest key ranges first
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int32_t q0 = __ldg(a.cu_q + s);
   int32_t n = __ldg(a.cu_q + s + 1) - q0;
   int32_t L = __ldg(a.lens + s);
   if (L < 0 || L > a.max_ctx || n < 0 || n > L) {
-    if (tid == 0 && g == 0 && tile == 0) record_error(PA_ERR_DEVICE_BOUNDS, L);
+    if (tid == 0 && g == 0 && pair == 0) record_error(PA_ERR_DEVICE_BOUNDS, L);
     L = L < 0 ? 0 : (L > a.max_ctx ? a.max_ctx : L);
     n = n < 0 ? 0 : (n > L ? L : n);
   }
-  const int32_t tok0 = tile * TT;
-  if (tok0 >= n) return;
-  const int32_t tok_end = min(tok0 + TT, n);
-  const int32_t base = L - n;           // position of new token 0
-  const int32_t kend = base + tok_end;  // keys 0 .. kend-1 are needed (kend >= 1)
-  const int nchunks = (kend + C - 1) / C;
+  const int32_t base = L - n;  // position of new token 0
+  const int32_t tok00 = pair * TILES * TT;
+  if (tok00 >= n) return;
+  // per tile: first token, key end, chunks; the stream follows the last active tile
+  int ntiles_act = 0, nch[TILES];
+  int32_t kend_all = 0;
+#pragma unroll
+  for (int t = 0; t < TILES; ++t) {
+    const int32_t t0 = tok00 + t * TT;
+    nch[t] = 0;
+    if (t0 < n) {
+      const int32_t ke = base + min(t0 + TT, n);
+      nch[t] = (ke + C - 1) / C;
+      kend_all = ke;
+      ntiles_act = t + 1;
+    }
+  }
+  const int nchunks = nch[ntiles_act - 1];
   const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
 
   if (tid == 0) {
-    mbar_init(&q_full, 4);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(&p_full[0], 4);
-    mbar_init(&p_full[1], 4);
-    mbar_init(&o_bar, 1);
+    mbar_init(&q_full, 4 * ntiles_act);
     mbar_init(&drain, 1);
+#pragma unroll
+    for (int t = 0; t < TILES; ++t) {
+      mbar_init(&s_full[t][0], 1);
+      mbar_init(&s_full[t][1], 1);
+      mbar_init(&p_full[t][0], 4);
+      mbar_init(&p_full[t][1], 4);
+      mbar_init(&o_bar[t], 1);
+    }
     pipe_init<S>(ps, 1);  // empty stages are released by one tcgen05.commit
   }
-  if (warp == 5) {
+  if (warp == Cfg::kMmaWarp) {
     tc::alloc(smem_u32(&tmem_base_sh), Cfg::kTmemCols);
     tc::relinquish();
     tc::fence_before();
@@ -120,13 +148,13 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(const __grid_constan
   tc::fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 4) {
+  if (warp == Cfg::kProducerWarp) {
     // ---- producer ----
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       const int32_t c0 = i * C;
-      const int32_t nb = (min(C, kend - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+      const int32_t nb = (min(C, kend_all - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
       int32_t blk = -1;
       bool ok = false;
       if (lane < nb) {
@@ -147,179 +175,232 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(const __grid_constan
         }
       }
     });
-  } else if (warp == 5) {
-    // ---- MMA issuer ----
+  } else if (warp == Cfg::kMmaWarp) {
+    // ---- MMA issuer: S_t(j+1) for every tile, then O_t += P_t(j) V(j) ----
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_bf16(Cfg::kRows, C, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(Cfg::kRows, D, true);
-      auto issue_pv = [&](int i) -> bool {
-        const int sb = i & 1, st = i % S;
-        if (!pipe_wait(&p_full[sb], (i >> 1) & 1, &ps.abort_flag)) return false;
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kbase = kv0 + (j % S) * Cfg::kStageBytes;
+        const uint32_t qb = qs + t * Cfg::kQTileBytes;
+        const uint32_t dst = tmem + t * Cfg::kTileCols + D + (j & 1) * C;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32u;  // 16 dims = 32 B along the swizzled 128-byte row
+          const uint64_t qd = tc::smem_desc(qb + (kk >> 2) * Cfg::kQHalfBytes + off, 16, 1024);
+          const uint64_t kd = tc::smem_desc(kbase + (kk >> 2) * Cfg::kHalfBytes + off, 16, 1024);
+          tc::mma_ss(dst, qd, kd, kIdS, kk > 0);
+        }
+        tc::commit(smem_u32(&s_full[t][j & 1]));
+      };
+      auto issue_pv = [&](int t, int j) -> bool {
+        const int sb = j & 1;
+        if (!pipe_wait(&p_full[t][sb], (j >> 1) & 1, &ps.abort_flag)) return false;
         tc::fence_after();
-        const uint32_t vbase = kv0 + st * Cfg::kStageBytes + Cfg::kTileBytes;
-        const uint32_t tp = tmem + Cfg::kColS + sb * C;  // P high part: 32 columns, remainder: the next 32
+        const uint32_t vbase = kv0 + (j % S) * Cfg::kStageBytes + Cfg::kTileBytes;
+        const uint32_t to = tmem + t * Cfg::kTileCols;
+        const uint32_t tp = to + D + sb * C;  // P high part: 32 columns, remainder: the next 32
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks) {
           // V is N-major: 8-key groups 1024 B apart, the two 64-column halves
           // kHalfBytes apart (one half when D = 64: the offset is then unused)
           const uint64_t bd = tc::smem_desc(vbase + ks * 16 * 128, Cfg::kHalves > 1 ? Cfg::kHalfBytes : 1024, 1024);
-          tc::mma_ts(tmem + Cfg::kColO, tp + ks * 8, bd, kIdPV, i > 0 || ks > 0);
-          tc::mma_ts(tmem + Cfg::kColO, tp + C / 2 + ks * 8, bd, kIdPV, true);
+          tc::mma_ts(to, tp + ks * 8, bd, kIdPV, j > 0 || ks > 0);
+          tc::mma_ts(to, tp + C / 2 + ks * 8, bd, kIdPV, true);
         }
-        tc::commit(smem_u32(&ps.empty[st]));
-        tc::commit(smem_u32(&o_bar));
+        tc::commit(smem_u32(&o_bar[t]));
         return true;
       };
-      bool ok = pipe_wait(&q_full, 0, &ps.abort_flag);
+      bool ok = pipe_wait(&q_full, 0, &ps.abort_flag) && pipe_wait(&ps.full[0], 0, &ps.abort_flag);
       tc::fence_after();
-      for (int j = 0; ok && j < nchunks; ++j) {
-        const int st = j % S, sb = j & 1;
-        if (!pipe_wait(&ps.full[st], (j / S) & 1, &ps.abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after();
-        const uint32_t kbase = kv0 + st * Cfg::kStageBytes;
+      if (ok) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32u;  // 16 dims = 32 B along the swizzled 128-byte row
-          const uint64_t qd = tc::smem_desc(qs + (kk >> 2) * Cfg::kQHalfBytes + off, 16, 1024);
-          const uint64_t kd = tc::smem_desc(kbase + (kk >> 2) * Cfg::kHalfBytes + off, 16, 1024);
-          tc::mma_ss(tmem + Cfg::kColS + sb * C, qd, kd, kIdS, kk > 0);
-        }
-        tc::commit(smem_u32(&s_full[sb]));
-        if (j > 0) ok = issue_pv(j - 1);
+        for (int t = 0; t < TILES; ++t)
+          if (nch[t] > 0) issue_s(t, 0);
       }
-      if (ok) issue_pv(nchunks - 1);
+      for (int j = 0; ok && j < nchunks; ++j) {
+        if (j + 1 < nchunks) {
+          if (!pipe_wait(&ps.full[(j + 1) % S], ((j + 1) / S) & 1, &ps.abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+#pragma unroll
+          for (int t = 0; t < TILES; ++t)
+            if (j + 1 < nch[t]) issue_s(t, j + 1);
+        }
+#pragma unroll
+        for (int t = 0; t < TILES; ++t)
+          if (ok && j < nch[t]) ok = issue_pv(t, j);
+        if (ok) tc::commit(smem_u32(&ps.empty[j % S]));  // every tile is done with stage j
+      }
       // every MMA this thread issued has finished before TMEM is released
       tc::commit(smem_u32(&drain));
       mbar_wait(&drain, 0);
     }
     __syncwarp();
   } else {
-    // ---- softmax warps: thread = row = TMEM lane ----
-    const int r = tid;
-    const int tok = tok0 + r / G;
-    const bool valid = tok < n;
-    const int32_t pos = base + (valid ? tok : tok_end - 1);  // last key the row sees
-    const int h = r % G;
-    const int64_t orow = (static_cast<int64_t>(q0) + (valid ? tok : 0)) * a.hq + g * G + h;
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + orow * D);
+    // ---- softmax warpgroup t: thread = row = TMEM lane ----
+    const int t = warp >> 2;
+    const int r = tid & 127;
+    const int32_t tok0 = tok00 + t * TT;
+    const int mych = nch[t];
+    if (mych > 0) {
+      const int32_t tok_end = min(tok0 + TT, n);
+      const int tok = tok0 + r / G;
+      const bool valid = tok < n;
+      const int32_t pos = base + (valid ? tok : tok_end - 1);  // last key the row sees
+      const int h = r % G;
+      const int64_t orow = (static_cast<int64_t>(q0) + (valid ? tok : 0)) * a.hq + g * G + h;
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + orow * D);
+        uint8_t* qdst = sgen + t * Cfg::kQTileBytes;
 #pragma unroll
-      for (int c16 = 0; c16 < D / 8; ++c16) {
-        const uint4 v = valid ? __ldg(src + c16) : make_uint4(0u, 0u, 0u, 0u);
-        const int hf = c16 >> 3, cc = c16 & 7;
-        *reinterpret_cast<uint4*>(sgen + hf * Cfg::kQHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+        for (int c16 = 0; c16 < D / 8; ++c16) {
+          const uint4 v = valid ? __ldg(src + c16) : make_uint4(0u, 0u, 0u, 0u);
+          const int hf = c16 >> 3, cc = c16 & 7;
+          *reinterpret_cast<uint4*>(qdst + hf * Cfg::kQHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+        }
+        tc::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_full);
       }
-      tc::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&q_full);
-    }
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nchunks; ++j) {
-      const int sb = j & 1;
-      if (!warp_wait(&s_full[sb], (j >> 1) & 1, &ps.abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after();
-      uint32_t sr[C];
-      tc::ld32(trow + Cfg::kColS + sb * C, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tc::ld32(trow + Cfg::kColS + sb * C + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tc::wait_ld();
-      const int32_t k0 = j * C;
-      float x[C];
-      float mx = -INFINITY;
+      // the stream's last chunk holds rows past its last key; the lowest tile
+      // that reads that chunk zeroes their V before any P V reads them
+      bool zero_tail = false;
 #pragma unroll
-      for (int c = 0; c < C; ++c) {
-        x[c] = k0 + c <= pos ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
-      }
-      float alpha = 1.f;
-      bool resc = false;
-      if (mx > m_ref + 8.f) {
-        alpha = exp2f(m_ref - mx);  // 0 while m_ref is -inf
-        l *= alpha;
-        m_ref = mx;
-        resc = j > 0;
-      }
-      uint32_t ph[C / 2], pl[C / 2];
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < C / 2; ++c) {
-        const float p0 = exp2f(x[2 * c] - m_ref), p1 = exp2f(x[2 * c + 1] - m_ref);
-        sum += p0 + p1;
-        split_pair(p0, p1, ph[c], pl[c]);
-      }
-      l += sum;
-      tc::st32(trow + Cfg::kColS + sb * C, ph);
-      tc::st32(trow + Cfg::kColS + sb * C + C / 2, pl);
-      if (__any_sync(0xffffffffu, resc)) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled
-        if (!warp_wait(&o_bar, (j - 1) & 1, &ps.abort_flag)) {
-          tc::wait_st();
+      for (int u = 0; u < TILES; ++u)
+        if (nch[u] == nchunks) {
+          zero_tail = u == t;
+          break;
+        }
+      const uint32_t trow = tmem + t * Cfg::kTileCols + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      const float sl2 = a.scale_log2;
+      float m_ref = -INFINITY, l = 0.f;  // m_ref in scaled (log2) units
+      bool ok = true;
+      for (int j = 0; j < mych; ++j) {
+        const int sb = j & 1;
+        if (!warp_wait(&s_full[t][sb], (j >> 1) & 1, &ps.abort_flag)) {
           ok = false;
           break;
         }
         tc::fence_after();
+        uint32_t sr[C];
+        tc::ld32(trow + D + sb * C, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tc::ld32(trow + D + sb * C + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tc::wait_ld();
+        const int32_t k0 = j * C;
+        float x[C];
+        float mx = -INFINITY;
+        // warp-uniform choice: tcgen05.ld/st below need the whole warp converged
+        if (__all_sync(0xffffffffu, k0 + C - 1 <= pos)) {
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            x[c] = __uint_as_float(sr[c]);
+            mx = fmaxf(mx, x[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            x[c] = k0 + c <= pos ? __uint_as_float(sr[c]) : -INFINITY;
+            mx = fmaxf(mx, x[c]);
+          }
+        }
+        mx *= sl2;  // scale > 0 keeps the order
+        float alpha = 1.f;
+        bool resc = false;
+        if (mx > m_ref + 8.f) {
+          alpha = fast_exp2(m_ref - mx);  // 0 while m_ref is -inf
+          l *= alpha;
+          m_ref = mx;
+          resc = j > 0;
+        }
+        uint32_t ph[C / 2], pl[C / 2];
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < C / 2; ++c) {
+          const float p0 = fast_exp2(fmaf(x[2 * c], sl2, -m_ref));
+          const float p1 = fast_exp2(fmaf(x[2 * c + 1], sl2, -m_ref));
+          sum += p0 + p1;
+          split_pair(p0, p1, ph[c], pl[c]);
+        }
+        l += sum;
+        __syncwarp();
+        tc::st32(trow + D + sb * C, ph);
+        tc::st32(trow + D + sb * C + C / 2, pl);
+        if (__any_sync(0xffffffffu, resc)) {
+          // O must hold P(j-1) V(j-1) before it is rescaled (P(j-2) V(j-2) is
+          // complete: it was issued before S(j), which this chunk waited for)
+          if (!warp_wait(&o_bar[t], (j - 1) & 1, &ps.abort_flag)) {
+            tc::wait_st();
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            __syncwarp();
+            tc::ld32(trow + q * 32, o);
+            tc::wait_ld();
+            if (resc) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            }
+            __syncwarp();
+            tc::st32(trow + q * 32, o);
+          }
+        }
+        if (zero_tail && j == nchunks - 1 && kend_all - k0 < C) {
+          // V rows past the last key may hold anything (unloaded or padding);
+          // 0 * NaN would reach O, so they are zeroed before P V reads them.
+          const int nvk = kend_all - k0;
+          const int chunks16 = (C - nvk) * Cfg::kHalves * 8;
+          uint8_t* vst = sgen + Cfg::kQBytes + (j % S) * Cfg::kStageBytes + Cfg::kTileBytes;
+          tc::fence_proxy_async();
+          for (int i = r; i < chunks16; i += 128) {
+            const int row = nvk + i / (Cfg::kHalves * 8);
+            const int rem = i % (Cfg::kHalves * 8);
+            *reinterpret_cast<uint4*>(vst + (rem >> 3) * Cfg::kHalfBytes + row * 128 + (rem & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          tc::fence_proxy_async();
+        }
+        __syncwarp();
+        tc::wait_st();
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[t][sb]);
+      }
+      // S(j+1) is issued before P(j) V(j), so this warpgroup can finish its
+      // last chunk while the previous P V is still pending: wait for the two
+      // last phases in turn (a parity wait cannot tell phases two apart).
+      if (ok && mych >= 2) ok = warp_wait(&o_bar[t], (mych - 2) & 1, &ps.abort_flag);
+      if (ok) ok = warp_wait(&o_bar[t], (mych - 1) & 1, &ps.abort_flag);
+      if (ok) {
+        tc::fence_after();
+        const float inv = 1.f / l;
+        float* dst = a.out + orow * D;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
           uint32_t o[32];
-          tc::ld32(trow + Cfg::kColO + q * 32, o);
+          __syncwarp();
+          tc::ld32(trow + q * 32, o);
           tc::wait_ld();
-          if (resc) {
+          if (valid) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + q * 32 + e) =
+                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
           }
-          tc::st32(trow + Cfg::kColO + q * 32, o);
         }
       }
-      if (j == nchunks - 1 && kend - k0 < C) {
-        // V rows past the last key may hold anything (unloaded or padding);
-        // 0 * NaN would reach O, so they are zeroed before P V reads them.
-        const int nvk = kend - k0;
-        const int chunks16 = (C - nvk) * Cfg::kHalves * 8;
-        uint8_t* vst = sgen + Cfg::kQBytes + (j % S) * Cfg::kStageBytes + Cfg::kTileBytes;
-        tc::fence_proxy_async();
-        for (int i = r; i < chunks16; i += 128) {
-          const int row = nvk + i / (Cfg::kHalves * 8);
-          const int rem = i % (Cfg::kHalves * 8);
-          *reinterpret_cast<uint4*>(vst + (rem >> 3) * Cfg::kHalfBytes + row * 128 + (rem & 7) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-        tc::fence_proxy_async();
-      }
-      tc::wait_st();
       tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    if (ok) ok = warp_wait(&o_bar, (nchunks - 1) & 1, &ps.abort_flag);
-    if (ok) {
-      tc::fence_after();
-      const float inv = 1.f / l;
-      float* dst = a.out + orow * D;
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t o[32];
-        tc::ld32(trow + Cfg::kColO + q * 32, o);
-        tc::wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + q * 32 + e) =
-                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-        }
-      }
-    }
-    tc::fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == Cfg::kMmaWarp) {
     tc::fence_after();
     tc::dealloc(tmem, Cfg::kTmemCols);
   }
