@@ -57,7 +57,9 @@ typedef enum {
 
 /* Cache element types. PA_FP8_E4M3 stores K and V as 8-bit floats (e4m3,
  * no infinities, largest 448) with one scale per tensor (pa_cache.k_scale,
- * v_scale): element = code * scale. The q/k/v inputs of an FP8 cache are bf16. */
+ * v_scale): element = code * scale. The q/k/v inputs of an FP8 cache are bf16;
+ * the decode rounds q to f16 for its tensor-core products, so |q| must stay
+ * below 65504 (every bf16 value below that converts exactly). */
 typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 typedef void* pa_stream; /* cudaStream_t */

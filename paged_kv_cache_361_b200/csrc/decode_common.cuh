@@ -154,6 +154,45 @@ __device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Block ids of one table row, read ahead by the producer warp in windows of
+// 32 entries (one per lane): the current window and the next are held in
+// registers, so each chunk's ids (at most 8, block_size >= 8) come from
+// shuffles, and the next window's load is in flight while the current one is
+// used. Entries at or past `lim` are never read (they read as -1).
+struct TableAhead {
+  const int32_t* row;
+  int32_t lim, w, cur, nxt;
+
+  __device__ __forceinline__ int32_t fetch(int32_t win, int lane) const {
+    const int32_t e = win * 32 + lane;
+    return e < lim ? __ldg(row + e) : -1;
+  }
+  __device__ __forceinline__ void init(const int32_t* r, int32_t first_entry, int32_t lim_, int lane) {
+    row = r;
+    lim = lim_;
+    w = first_entry >> 5;
+    cur = fetch(w, lane);
+    nxt = fetch(w + 1, lane);
+  }
+  // Entries e0 .. e0 + n - 1 (n <= 8, e0 never decreasing between calls):
+  // lane u < n returns entry e0 + u, the other lanes -1. Whole warp.
+  __device__ __forceinline__ int32_t get(int32_t e0, int n, int lane) {
+    while ((e0 >> 5) > w) {
+      cur = nxt;
+      ++w;
+      nxt = fetch(w + 1, lane);
+    }
+    int32_t mine = -1;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int32_t e = e0 + u;
+      const int32_t v = __shfl_sync(0xffffffffu, (e >> 5) == w ? cur : nxt, e & 31);
+      if (lane == u) mine = v;
+    }
+    return lane < n ? mine : -1;
+  }
+};
+
 // Per-CTA pipeline state in shared memory: S stages, each with a "full"
 // barrier (one producer arrival + the TMA byte count) and an "empty" barrier
 // (one arrival per consumer warp).

@@ -60,10 +60,13 @@ __device__ __forceinline__ uint32_t f8_off(int row, int col) {
   return row * 64 + ((((col >> 4) ^ ((row >> 1) & 3)) << 4) | (col & 15));
 }
 
-// Two e4m3 codes (low byte first) -> f16x2 (low half first), exact.
-__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Four e4m3 codes (low byte first) -> two f16x2 words: bytes 0,1 -> lo,
+// bytes 2,3 -> hi (low byte in the low half), exact.
+__device__ __forceinline__ void e4m3x4_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
@@ -104,7 +107,9 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t w = *reinterpret_cast<const uint32_t*>(kt + f8_off<D>(row, kk * 16 + 4 * c));
-      mma_f16_rows8(sacc[nt], qa[kk][0], qa[kk][1], e4m3x2_f16x2(w), e4m3x2_f16x2(w >> 16));
+      uint32_t b0, b1;
+      e4m3x4_f16x2(w, b0, b1);
+      mma_f16_rows8(sacc[nt], qa[kk][0], qa[kk][1], b0, b1);
     }
   }
   float sc[2][2];
@@ -119,9 +124,10 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
     }
   mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
   mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-  const float mn = fmaxf(m_run, mloc);
-  const float alpha = exp2f(m_run - mn);
-  m_run = mn;
+  // the reference maximum moves only when a score exceeds it by 8 (log2
+  // units): weights stay <= 2^8 (f16 holds them) and O is rarely rescaled
+  const bool move = mloc > m_run + 8.f;
+  const float mn = move ? mloc : m_run;
   float pr[2][2];
   float psum = 0.f;
 #pragma unroll
@@ -131,12 +137,17 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
       pr[nt][j] = exp2f(sc[nt][j] - mn);
       psum += pr[nt][j];
     }
-  l_run = l_run * alpha + psum;
+  if (__any_sync(0xffffffffu, move)) {
+    const float alpha = exp2f(m_run - mn);  // 1 for rows that did not move, 0 from -inf
+    l_run *= alpha;
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    o[j][0] *= alpha;
-    o[j][1] *= alpha;
+    for (int j = 0; j < NT; ++j) {
+      o[j][0] *= alpha;
+      o[j][1] *= alpha;
+    }
   }
+  m_run = mn;
+  l_run += psum;
   const uint32_t pa0 = pack_f16(pr[0][0], pr[0][1]);  // tokens 2c, 2c+1
   const uint32_t pa2 = pack_f16(pr[1][0], pr[1][1]);  // tokens 8+2c, 9+2c
   // masks for tokens past the valid ones (their V bytes may be NaN codes)
@@ -165,15 +176,24 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
     vc[0] = x2.x, vc[1] = x2.y;
     vd[0] = x3.x, vd[1] = x3.y;
   }
+  const bool ragged = nv < 16;  // warp-uniform
 #pragma unroll
   for (int w = 0; w < W; ++w) {
     // (token a byte k, token b byte k) pairs: bytes 0,1 then 2,3 of each word
-    const uint32_t p01 = __byte_perm(va[w], vb[w], 0x5140), p23 = __byte_perm(va[w], vb[w], 0x7362);
-    const uint32_t q01 = __byte_perm(vc[w], vd[w], 0x5140), q23 = __byte_perm(vc[w], vd[w], 0x7362);
-    mma_f16_rows8(o[4 * w + 0], pa0, pa2, e4m3x2_f16x2(p01) & m0, e4m3x2_f16x2(q01) & m1);
-    mma_f16_rows8(o[4 * w + 1], pa0, pa2, e4m3x2_f16x2(p01 >> 16) & m0, e4m3x2_f16x2(q01 >> 16) & m1);
-    mma_f16_rows8(o[4 * w + 2], pa0, pa2, e4m3x2_f16x2(p23) & m0, e4m3x2_f16x2(q23) & m1);
-    mma_f16_rows8(o[4 * w + 3], pa0, pa2, e4m3x2_f16x2(p23 >> 16) & m0, e4m3x2_f16x2(q23 >> 16) & m1);
+    uint32_t b[8];
+    e4m3x4_f16x2(__byte_perm(va[w], vb[w], 0x5140), b[0], b[1]);
+    e4m3x4_f16x2(__byte_perm(va[w], vb[w], 0x7362), b[2], b[3]);
+    e4m3x4_f16x2(__byte_perm(vc[w], vd[w], 0x5140), b[4], b[5]);
+    e4m3x4_f16x2(__byte_perm(vc[w], vd[w], 0x7362), b[6], b[7]);
+    if (ragged) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        b[k] &= m0;
+        b[4 + k] &= m1;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mma_f16_rows8(o[4 * w + k], pa0, pa2, b[k], b[4 + k]);
   }
 }
 
@@ -216,13 +236,14 @@ __global__ void __launch_bounds__(F8Cfg<D>::kThreads) decode_f8_kernel(const __g
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
     const uint64_t pol = l2_evict_first_policy();
+    TableAhead ta;
+    ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       const int32_t c0 = pt.t0 + i * C;
       const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
-      int32_t blk = -1;
+      const int32_t blk = ta.get(c0 / a.bs, nb, lane);
       bool ok = false;
       if (lane < nb) {
-        blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
         ok = blk >= 0 && blk < a.num_blocks;
         if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
       }

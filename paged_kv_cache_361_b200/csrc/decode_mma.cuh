@@ -146,9 +146,10 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
     }
   mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
   mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-  const float mn = fmaxf(m_run, mloc);
-  const float alpha = exp2f(m_run - mn);
-  m_run = mn;
+  // the reference maximum moves only when a score exceeds it by 8 (log2
+  // units): weights stay <= 2^8 and O is rarely rescaled
+  const bool move = mloc > m_run + 8.f;
+  const float mn = move ? mloc : m_run;
   float pr[2][2];
   float psum = 0.f;
 #pragma unroll
@@ -158,12 +159,17 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
       pr[nt][j] = exp2f(sc[nt][j] - mn);
       psum += pr[nt][j];
     }
-  l_run = l_run * alpha + psum;
+  if (__any_sync(0xffffffffu, move)) {
+    const float alpha = exp2f(m_run - mn);  // 1 for rows that did not move, 0 from -inf
+    l_run *= alpha;
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    o[j][0] *= alpha;
-    o[j][1] *= alpha;
+    for (int j = 0; j < NT; ++j) {
+      o[j][0] *= alpha;
+      o[j][1] *= alpha;
+    }
   }
+  m_run = mn;
+  l_run += psum;
   uint32_t ph0, pl0, ph2, pl2;
   split_pair(pr[0][0], pr[0][1], ph0, pl0);
   split_pair(pr[1][0], pr[1][1], ph2, pl2);
@@ -489,13 +495,14 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const _
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_first_policy();
+    TableAhead ta;
+    ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       const int32_t c0 = pt.t0 + i * C;
       const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
-      int32_t blk = -1;
+      const int32_t blk = ta.get(c0 / a.bs, nb, lane);
       bool ok = false;
       if (lane < nb) {
-        blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
         ok = blk >= 0 && blk < a.num_blocks;
         if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
       }

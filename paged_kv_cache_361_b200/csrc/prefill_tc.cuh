@@ -152,13 +152,14 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
     // ---- producer ----
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
+    TableAhead ta;
+    ta.init(a.tables + table_row, 0, min(a.max_blocks, (kend_all + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       const int32_t c0 = i * C;
       const int32_t nb = (min(C, kend_all - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
-      int32_t blk = -1;
+      const int32_t blk = ta.get(c0 / a.bs, nb, lane);
       bool ok = false;
       if (lane < nb) {
-        blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
         ok = blk >= 0 && blk < a.num_blocks;
         if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
       }
