@@ -48,6 +48,20 @@ def peaks():
         return 6650.0, "fallback"
 
 
+# --- ranks -------------------------------------------------------------------------
+
+def combine_ranks(ms: float, nbytes: float, world: int, device) -> tuple[float, float]:
+    """Whole-job figures of a replicated run: the slowest rank's time and the
+    bytes of all ranks (one float64 all-reduce each; no-op for one rank)."""
+    if world <= 1:
+        return float(ms), float(nbytes)
+    tm = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    tb = torch.tensor([float(nbytes)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.all_reduce(tb, op=torch.distributed.ReduceOp.SUM)
+    return float(tm.item()), float(tb.item())
+
+
 # --- clocks sampling -------------------------------------------------------------
 
 class Clocks:
@@ -326,15 +340,7 @@ def run_ours(args, rank, world, device):
         raise RuntimeError(f"device error {st} ({info}) in the timed region")
 
     kv_bytes = d["kv_bytes"]
-    t = torch.tensor([total_ms, float(kv_bytes)], dtype=torch.float64, device=device)
-    if world > 1:
-        tm = t[:1].clone()
-        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
-        tb = t[1:].clone()
-        torch.distributed.all_reduce(tb, op=torch.distributed.ReduceOp.SUM)
-        total_ms, all_bytes = float(tm.item()), float(tb.item())
-    else:
-        all_bytes = float(kv_bytes)
+    total_ms, all_bytes = combine_ranks(total_ms, kv_bytes, world, device)
     ms_per_step = total_ms / args.steps
     value = all_bytes / (ms_per_step * 1e-3) / 1e9
     tokens_per_s = world * nseq / (ms_per_step * 1e-3)
@@ -428,13 +434,7 @@ def run_e2e(args, d, device, world, P):
     nblk = int(-(-(int(L0.max()) + K) // sh.block_size))
     h2d = (hq.numel() + hk.numel() + hv.numel()) * eb + n * (8 + 8 + nblk * 4 + 4)
     d2h = hout.numel() * 4
-    t = torch.tensor([ms, float(kv_total)], dtype=torch.float64, device=device)
-    if world > 1:
-        tm = t[:1].clone()
-        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
-        tb = t[1:].clone()
-        torch.distributed.all_reduce(tb, op=torch.distributed.ReduceOp.SUM)
-        ms, kv_total = float(tm.item()), float(tb.item())
+    ms, kv_total = combine_ranks(ms, kv_total, world, device)
     return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "ms_per_step": round(ms / args.steps, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -502,10 +502,7 @@ def run_prefill(args, rank, world, device):
     ms = e0.elapsed_time(e1) / args.steps
     pf_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     flops = 4.0 * D * hq * nseq * plen * (plen + 1) / 2
-    tm = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(tm, op=torch.distributed.ReduceOp.MAX)
-    ms = float(tm.item())
+    ms, all_flops = combine_ranks(ms, flops, world, device)
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             peak = float(json.load(f)["bf16_tflops"])
@@ -515,7 +512,7 @@ def run_prefill(args, rank, world, device):
     if rank == 0:
         print(json.dumps({
             "metric": "paged prefill attention TFLOP/s (causal; 4*head_dim*Hq flops per visible query-key pair)",
-            "value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "value": round(all_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{args.workload}: {nseq} prompts x {plen} tokens, {hq}/{hkv} heads, D128, bs16",
