@@ -38,6 +38,14 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode attention tokens/sec"
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# dominant kernel, from an ncu capture of
+#   python bench.py --steps 3 --warmup 3 --no-e2e --no-cpu-baseline
+# (profiles/decode_simt_llama2_7b_mha.md), keyed by (workload, cache dtype,
+# partition tokens). Configurations without a capture of the current kernel
+# report null.
+NCU_TRAFFIC = {("llama2_7b_mha", "bfloat16", 0): 1_082_858_240}
+
 
 def peaks():
     try:
@@ -388,7 +396,9 @@ def run_ours(args, rank, world, device):
                                     if cascade is not None else
                                     "pa_decode" + (" (decode + partition merge)" if split else "")), "bound": "hbm",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "frac": round(achieved / peak, 4),
+                         "traffic": None if cascade is not None else NCU_TRAFFIC.get(
+                             (args.workload, str(d["kc"].dtype).replace("torch.", ""), P_eff)),
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                          else "fallback", "decode_ms_avg": round(dec_avg_ms, 5)},
             "cpu_baseline": cpu,

@@ -3,6 +3,8 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include <cudaTypedefs.h>
 
@@ -91,14 +93,31 @@ int device_sm_count() {
   return cache[dev];
 }
 
+// Sets a kernel's dynamic shared-memory limit (and the max-shared carveout)
+// once per (kernel, device): the attributes persist for the process, and the
+// per-token host path should not pay for the calls on every launch.
+bool smem_attrs(const void* kern, int bytes, bool max_carveout) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<const void*, int>, int>> done;  // ((kernel, device), bytes)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& e : done)
+    if (e.first.first == kern && e.first.second == dev && e.second >= bytes) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (max_carveout &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+          cudaSuccess)
+    return false;
+  done.push_back({{kern, dev}, bytes});
+  return true;
+}
+
 template <typename T, int D, int G>
 pa_status launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   using Cfg = SimtCfg<T, D>;
   auto kern = decode_simt_kernel<T, D, G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
-          cudaSuccess)
-    return PA_ERR_CUDA;
+  if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(a);
   return launched();
 }
@@ -176,10 +195,7 @@ pa_status launch_f8(const DecodeArgs& a, const pa_cache* c, dim3 grid, cudaStrea
   if (!encode_rows_u8(&tk, c->k, rows, D, c->block_size) || !encode_rows_u8(&tv, c->v, rows, D, c->block_size))
     return PA_ERR_CUDA;
   auto kern = decode_f8_kernel<D, G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
-          cudaSuccess)
-    return PA_ERR_CUDA;
+  if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
   return launched();
 }
@@ -204,10 +220,7 @@ pa_status launch_mma(const DecodeArgs& a, const pa_cache* c, bool persistent, cu
     return PA_ERR_CUDA;
   if (!persistent) {
     auto kern = decode_mma_kernel<D, G>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
-            cudaSuccess)
-      return PA_ERR_CUDA;
+    if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;
     kern<<<dim3(a.hkv, a.num_seqs, a.max_parts), Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
     return launched();
   }
@@ -431,8 +444,7 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   const dim3 grid(cache->num_kv_heads, static_cast<unsigned>(ntiles), num_seqs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto launch = [&](auto kern, int threads, int smem) -> pa_status {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return PA_ERR_CUDA;
+    if (!smem_attrs(reinterpret_cast<const void*>(kern), smem, false)) return PA_ERR_CUDA;
     kern<<<grid, threads, smem, s>>>(tk, tv, a);
     return launched();
   };
@@ -546,8 +558,7 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
       return PA_ERR_CUDA;
     const dim3 grid(cache->num_kv_heads, pparts, num_groups);
     auto launch = [&](auto kern, int smem) -> pa_status {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return PA_ERR_CUDA;
+      if (!smem_attrs(reinterpret_cast<const void*>(kern), smem, false)) return PA_ERR_CUDA;
       kern<<<grid, MmaCfg<128>::kThreads, smem, s>>>(tk, tv, pa);
       return launched();
     };

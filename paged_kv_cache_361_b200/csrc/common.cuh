@@ -117,6 +117,14 @@ __device__ __forceinline__ uint8_t quantize_e4m3(float x, float scale) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
 }
 
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error ~2^-22,
+// results below 2^-126 flush to 0, 2^-inf = 0). Used for softmax weights.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // bf16 pair packed in a 32-bit word -> two floats (exact).
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

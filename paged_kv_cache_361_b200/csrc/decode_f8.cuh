@@ -74,7 +74,8 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// m16n8k16 f16 MMA with rows 8..15 of A zero and their results discarded.
+// m16n8k16 f16 MMA with rows 8..15 of A zero and their results discarded
+// (as mma_rows8).
 __device__ __forceinline__ void mma_f16_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   float j2, j3;
   asm volatile(
@@ -134,11 +135,11 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      pr[nt][j] = exp2f(sc[nt][j] - mn);
+      pr[nt][j] = fast_exp2(sc[nt][j] - mn);
       psum += pr[nt][j];
     }
   if (__any_sync(0xffffffffu, move)) {
-    const float alpha = exp2f(m_run - mn);  // 1 for rows that did not move, 0 from -inf
+    const float alpha = fast_exp2(m_run - mn);  // 1 for rows that did not move, 0 from -inf
     l_run *= alpha;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
@@ -150,9 +151,7 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
   l_run += psum;
   const uint32_t pa0 = pack_f16(pr[0][0], pr[0][1]);  // tokens 2c, 2c+1
   const uint32_t pa2 = pack_f16(pr[1][0], pr[1][1]);  // tokens 8+2c, 9+2c
-  // masks for tokens past the valid ones (their V bytes may be NaN codes)
-  const uint32_t m0 = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
-  const uint32_t m1 = (2 * c + 8 < nv ? 0x0000ffffu : 0u) | (2 * c + 9 < nv ? 0xffff0000u : 0u);
+
   constexpr int W = D == 128 ? 4 : 2;  // 32-bit words of V per token this thread reads
   uint32_t va[W], vb[W], vc[W], vd[W];
   const int col = (D == 128 ? 16 : 8) * gq;
@@ -186,6 +185,9 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
     e4m3x4_f16x2(__byte_perm(vc[w], vd[w], 0x5140), b[4], b[5]);
     e4m3x4_f16x2(__byte_perm(vc[w], vd[w], 0x7362), b[6], b[7]);
     if (ragged) {
+      // tokens past the valid ones: their V bytes may be NaN codes
+      const uint32_t m0 = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
+      const uint32_t m1 = (2 * c + 8 < nv ? 0x0000ffffu : 0u) | (2 * c + 9 < nv ? 0xffff0000u : 0u);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         b[k] &= m0;

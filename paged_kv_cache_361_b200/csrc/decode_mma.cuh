@@ -63,6 +63,9 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
 // d += A(16x16, rows 8..15 zero) * B(16x8), bf16 in, fp32 accumulate. Only
 // rows 0..7 of the accumulator are kept: rows 8..15 are fed zeros and their
 // results are discarded, so they hold no registers across the loop.
+// m16n8k16 bf16 MMA with rows 8..15 of A zero: their accumulator lanes get
+// fresh zero inputs and are discarded, so no registers are held for them and
+// the MMAs on different accumulators stay independent.
 __device__ __forceinline__ void mma_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   float j2, j3;
   asm volatile(
@@ -156,11 +159,11 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      pr[nt][j] = exp2f(sc[nt][j] - mn);
+      pr[nt][j] = fast_exp2(sc[nt][j] - mn);
       psum += pr[nt][j];
     }
   if (__any_sync(0xffffffffu, move)) {
-    const float alpha = exp2f(m_run - mn);  // 1 for rows that did not move, 0 from -inf
+    const float alpha = fast_exp2(m_run - mn);  // 1 for rows that did not move, 0 from -inf
     l_run *= alpha;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {

@@ -68,12 +68,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // TILES query tiles of one (kv head, sequence) per CTA share the K/V stream;
 // tile t is processed by softmax warpgroup t.
 template <int D, int G, int TILES>

@@ -140,3 +140,47 @@ def test_cascade_random_groups(G):
     b = cache.decode_cascade(ids, q, D ** -0.5)
     assert B.pa_get_device_error()[0] == B.PA_OK
     assert float((a - b).abs().max()) <= 2e-3
+
+
+def test_llama2_7b_mha_fp8_cache():
+    """The metric workload over an e4m3 cache: every sequence's codes equal the
+    oracle's quantisation of its rows bitwise; every output row within the bf16
+    bound of the fp64 attention over the dequantised rows."""
+    from tests.test_gpu_fp8 import Fp8Replay
+    w = W.llama2_7b_mha()
+    r = Fp8Replay(w.shape, w.num_blocks, w.free_order, w.scale).run(W.simple_ops(w))
+    r.check_pool_codes()
+    r.check_outputs()
+
+
+def test_prefill_benchmark_size_sampled_rows():
+    """The prefill benchmark's launch (8 prompts x 2048 tokens, 32/32 heads, D 128,
+    bs 16, whole prompts in one pa_prefill): 24 sampled token rows of every
+    prompt (first, last and across the 128-row tiles), all heads."""
+    import torch
+    from oracle.attention import decode_attention
+    from paged_kv_cache_361_b200 import PagedKVCache
+    nseq, plen, H, D, bs = 8, 2048, 32, 128, 16
+    nb = nseq * plen // bs + 16
+    cache = PagedKVCache(nb, H, bs, D, torch.bfloat16, "cuda", np.random.default_rng(3).permutation(nb),
+                         fill=float("nan"))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    T = nseq * plen
+    q = torch.randn(T, H, D, generator=g, device="cuda").bfloat16()
+    k = torch.randn(T, H, D, generator=g, device="cuda").bfloat16()
+    v = torch.randn(T, H, D, generator=g, device="cuda").bfloat16()
+    out = cache.prefill(list(range(nseq)), [plen] * nseq, q, k, v, D ** -0.5)
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    rows = np.unique(np.r_[0, 1, 127, 128, 255, 256, 1000, 1023, 1024, 2047,
+                           np.random.default_rng(5).integers(0, plen, 14)])
+    worst = 0.0
+    for s in range(nseq):
+        base = s * plen
+        K = k[base:base + plen].cpu()
+        V = v[base:base + plen].cpu()
+        for t in rows:
+            ref = decode_attention(q[base + t].cpu(), K[:t + 1], V[:t + 1], D ** -0.5)
+            err = float(np.abs(out[base + t].double().cpu().numpy() - ref).max())
+            worst = max(worst, err)
+    assert worst <= 4e-3, worst
