@@ -86,6 +86,18 @@ __device__ __forceinline__ void mma_f16_rows8(float (&d)[2], uint32_t a0, uint32
   asm volatile("" ::"f"(j2), "f"(j3));
 }
 
+// The same MMA for a dependent chain (one accumulator over the k-steps): rows
+// 8..15 accumulate into the chain's own `dead` pair (never read), which
+// saves materialising zero inputs per MMA without adding dependences.
+__device__ __forceinline__ void mma_f16_rows8_chain(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0,
+                                                    uint32_t b1, float (&dead)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(dead[0]), "+f"(dead[1])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
 // Output dim of n-tile j, column n.
 template <int D>
 __device__ __forceinline__ int f8_dim(int j, int n) {
@@ -101,16 +113,24 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
   const int gq = lane >> 2, c = lane & 3;
   const int tw = warp * 16;
   float sacc[2][2];
+  // A row's start (the 1024-byte aligned tile base plus row * D) has bits
+  // 0..6 (128-byte rows) or 0..5 (64-byte rows) clear, so the swizzled address
+  // of 16-byte chunk kk is (row start | swizzle key << 4 | byte) ^ (kk << 4).
+  const uint32_t kts = smem_u32(kt);
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     sacc[nt][0] = sacc[nt][1] = 0.f;
+    float dead[2] = {0.f, 0.f};
     const int row = tw + nt * 8 + gq;
+    const uint32_t key = D == 128 ? static_cast<uint32_t>(row & 7) : static_cast<uint32_t>((row >> 1) & 3);
+    const uint32_t rbase = (kts + static_cast<uint32_t>(row * D)) | (key << 4) | static_cast<uint32_t>(4 * c);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(kt + f8_off<D>(row, kk * 16 + 4 * c));
+      uint32_t w;
+      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w) : "r"(rbase ^ static_cast<uint32_t>(kk << 4)));
       uint32_t b0, b1;
       e4m3x4_f16x2(w, b0, b1);
-      mma_f16_rows8(sacc[nt], qa[kk][0], qa[kk][1], b0, b1);
+      mma_f16_rows8_chain(sacc[nt], qa[kk][0], qa[kk][1], b0, b1, dead);
     }
   }
   float sc[2][2];

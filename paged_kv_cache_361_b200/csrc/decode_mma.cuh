@@ -76,6 +76,18 @@ __device__ __forceinline__ void mma_rows8(float (&d)[2], uint32_t a0, uint32_t a
   asm volatile("" ::"f"(j2), "f"(j3));  // rows 8..15: discarded
 }
 
+// The same MMA for a dependent chain (one accumulator over the k-steps): rows
+// 8..15 accumulate into the chain's own `dead` pair (never read), which
+// saves materialising zero inputs per MMA without adding dependences.
+__device__ __forceinline__ void mma_rows8_chain(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1,
+                                                float (&dead)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(dead[0]), "+f"(dead[1])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -126,6 +138,7 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
   const int tokV = warp * 16 + (mk & 1) * 8 + ik;   // V matrices (tok0, d0), (tok0+8, d0), (tok0, d0+8), (tok0+8, d0+8)
   const int dV = (mk >> 1) * 8;
   float sacc[2][2];
+  float dead0[2] = {0.f, 0.f}, dead1[2] = {0.f, 0.f};
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = 0.f;
 #pragma unroll
@@ -134,8 +147,8 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
     const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tokK * 128 + ((((d0 & 63) >> 3) ^ (tokK & 7)) << 4);
     uint32_t b00, b01, b10, b11;
     ldsm_x4(addr, b00, b01, b10, b11);
-    mma_rows8(sacc[0], qa[kk][0], qa[kk][1], b00, b01);
-    mma_rows8(sacc[1], qa[kk][0], qa[kk][1], b10, b11);
+    mma_rows8_chain(sacc[0], qa[kk][0], qa[kk][1], b00, b01, dead0);
+    mma_rows8_chain(sacc[1], qa[kk][0], qa[kk][1], b10, b11, dead1);
   }
   float sc[2][2];
   float mloc = -INFINITY;
