@@ -286,21 +286,25 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
         tc::wait_ld();
         const int32_t k0 = j * C;
         float x[C];
-        float mx = -INFINITY;
+        // the row maximum over 8 independent partial maxima (short dependence chains)
+        float pm[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
         // warp-uniform choice: tcgen05.ld/st below need the whole warp converged
         if (__all_sync(0xffffffffu, k0 + C - 1 <= pos)) {
 #pragma unroll
           for (int c = 0; c < C; ++c) {
             x[c] = __uint_as_float(sr[c]);
-            mx = fmaxf(mx, x[c]);
+            pm[c & 7] = fmaxf(pm[c & 7], x[c]);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < C; ++c) {
             x[c] = k0 + c <= pos ? __uint_as_float(sr[c]) : -INFINITY;
-            mx = fmaxf(mx, x[c]);
+            pm[c & 7] = fmaxf(pm[c & 7], x[c]);
           }
         }
+        float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         mx *= sl2;  // scale > 0 keeps the order
         float alpha = 1.f;
         bool resc = false;
@@ -311,15 +315,15 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
           resc = j > 0;
         }
         uint32_t ph[C / 2], pl[C / 2];
-        float sum = 0.f;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums (short dependence chains)
 #pragma unroll
         for (int c = 0; c < C / 2; ++c) {
           const float p0 = fast_exp2(fmaf(x[2 * c], sl2, -m_ref));
           const float p1 = fast_exp2(fmaf(x[2 * c + 1], sl2, -m_ref));
-          sum += p0 + p1;
+          part[c & 3] += p0 + p1;
           split_pair(p0, p1, ph[c], pl[c]);
         }
-        l += sum;
+        l += (part[0] + part[1]) + (part[2] + part[3]);
         __syncwarp();
         tc::st32(trow + D + sb * C, ph);
         tc::st32(trow + D + sb * C + C / 2, pl);
