@@ -175,16 +175,23 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_bf16(Cfg::kRows, C, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(Cfg::kRows, D, true);
+      // Descriptors are built once; an operand at a byte offset from a base
+      // is the base descriptor plus offset / 16 (the start-address field,
+      // addresses stay below 256 KB so the field never carries over).
+      const uint64_t qdesc0 = tc::smem_desc(qs, 16, 1024);
+      const uint64_t kdesc0 = tc::smem_desc(kv0, 16, 1024);
+      const uint64_t vdesc0 =
+          tc::smem_desc(kv0 + Cfg::kTileBytes, Cfg::kHalves > 1 ? Cfg::kHalfBytes : 1024, 1024);
       auto issue_s = [&](int t, int j) {
-        const uint32_t kbase = kv0 + (j % S) * Cfg::kStageBytes;
-        const uint32_t qb = qs + t * Cfg::kQTileBytes;
+        const uint64_t qb = qdesc0 + static_cast<uint64_t>((t * Cfg::kQTileBytes) >> 4);
+        const uint64_t kb = kdesc0 + static_cast<uint64_t>(((j % S) * Cfg::kStageBytes) >> 4);
         const uint32_t dst = tmem + t * Cfg::kTileCols + D + (j & 1) * C;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32u;  // 16 dims = 32 B along the swizzled 128-byte row
-          const uint64_t qd = tc::smem_desc(qb + (kk >> 2) * Cfg::kQHalfBytes + off, 16, 1024);
-          const uint64_t kd = tc::smem_desc(kbase + (kk >> 2) * Cfg::kHalfBytes + off, 16, 1024);
-          tc::mma_ss(dst, qd, kd, kIdS, kk > 0);
+          // 16 dims = 32 B along the swizzled 128-byte row; 64 dims per box column
+          const uint32_t offq = static_cast<uint32_t>((kk >> 2) * Cfg::kQHalfBytes + (kk & 3) * 32) >> 4;
+          const uint32_t offk = static_cast<uint32_t>((kk >> 2) * Cfg::kHalfBytes + (kk & 3) * 32) >> 4;
+          tc::mma_ss(dst, qb + offq, kb + offk, kIdS, kk > 0);
         }
         tc::commit(smem_u32(&s_full[t][j & 1]));
       };
@@ -192,14 +199,14 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
         const int sb = j & 1;
         if (!pipe_wait(&p_full[t][sb], (j >> 1) & 1, &ps.abort_flag)) return false;
         tc::fence_after();
-        const uint32_t vbase = kv0 + (j % S) * Cfg::kStageBytes + Cfg::kTileBytes;
+        // V is N-major: 8-key groups 1024 B apart, the two 64-column halves
+        // kHalfBytes apart (one half when D = 64: the offset is then unused)
+        const uint64_t vb = vdesc0 + static_cast<uint64_t>(((j % S) * Cfg::kStageBytes) >> 4);
         const uint32_t to = tmem + t * Cfg::kTileCols;
         const uint32_t tp = to + D + sb * C;  // P high part: 32 columns, remainder: the next 32
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks) {
-          // V is N-major: 8-key groups 1024 B apart, the two 64-column halves
-          // kHalfBytes apart (one half when D = 64: the offset is then unused)
-          const uint64_t bd = tc::smem_desc(vbase + ks * 16 * 128, Cfg::kHalves > 1 ? Cfg::kHalfBytes : 1024, 1024);
+          const uint64_t bd = vb + static_cast<uint64_t>((ks * 16 * 128) >> 4);
           tc::mma_ts(to, tp + ks * 8, bd, kIdPV, j > 0 || ks > 0);
           tc::mma_ts(to, tp + C / 2 + ks * 8, bd, kIdPV, true);
         }
