@@ -89,8 +89,8 @@ class Clocks:
 
     def start(self):
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            import tempfile
+            self.path = os.path.join(tempfile.gettempdir(), f"pa_bench_clocks_{os.getpid()}.csv")
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
             if self.sel:
                 cmd += ["-i", self.sel]
