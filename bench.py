@@ -461,13 +461,20 @@ PREFILL = {
 def run_prefill(args, rank, world, device):
     """Whole-prompt prefill (pa_reshape_and_cache of every prompt token +
     pa_prefill) over a fresh paged cache; metric: causal attention TFLOP/s with
-    4 * head_dim * Hq flops per (query, visible key) pair."""
+    4 * head_dim * Hq flops per (query, visible key) pair. --kv-dtype fp8 keeps
+    the cache as e4m3 codes (per-tensor scales 4/448: N(0, 1) rows use the
+    code range)."""
     from paged_kv_cache_361_b200 import PagedKVCache, binding as B
     hq, hkv, nseq, plen = PREFILL[args.workload]
     D, bs = 128, 16
     nb = nseq * plen // bs + 16
     order = np.random.default_rng(rank).permutation(nb)
-    cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, device, order)
+    f8 = args.kv_dtype == "fp8"
+    if f8:
+        cache = PagedKVCache(nb, hkv, bs, D, torch.float8_e4m3fn, device, order, k_scale=4.0 / 448,
+                             v_scale=4.0 / 448)
+    else:
+        cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, device, order)
     g = torch.Generator(device=device)
     g.manual_seed(2000 + rank)
     T = nseq * plen
@@ -524,15 +531,20 @@ def run_prefill(args, rank, world, device):
             "metric": "paged prefill attention TFLOP/s (causal; 4*head_dim*Hq flops per visible query-key pair)",
             "value": round(all_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3 cache, bf16 q (f16 MMA)" if f8 else "bf16", "data": "synthetic",
             "config": {"workload": f"{args.workload}: {nseq} prompts x {plen} tokens, {hq}/{hkv} heads, D128, bs16",
-                       "l2": "no flush: K/V of one launch " + f"{2 * T * hkv * D * 2 / 1e6:.0f} MB"},
+                       "kv_dtype": "float8_e4m3fn" if f8 else "bfloat16",
+                       "l2": "no flush: K/V of one launch "
+                             + f"{2 * T * hkv * D * (1 if f8 else 2) / 1e6:.0f} MB"},
             "gpu_launches": 2 * args.steps,
             "roofline": {"kernel": "pa_prefill", "bound": "tensor", "achieved": round(flops / (pf_ms * 1e-3) / 1e12, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(flops / (pf_ms * 1e-3) / 1e12 / peak, 4),
                          "traffic": None, "peak_source": src,
-                         "note": "tcgen05.mma (M 128) with TMEM accumulators; P split into two bf16 MMAs "
-                                 "(1.5x the algorithmic MMA work)"},
+                         "note": ("tcgen05.mma (M 128) with TMEM accumulators; K/V codes widened to f16 in "
+                                  "shared memory, one f16 P V MMA per k-step") if f8 else
+                                 ("tcgen05.mma (M 128) with TMEM accumulators; P split into two bf16 MMAs "
+                                  "(1.5x the algorithmic MMA work)")},
             "clocks": clk}), flush=True)
 
 
@@ -584,7 +596,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--kv-dtype", choices=["auto", "fp8"], default="auto",
-                    help="fp8: e4m3 cache with bf16 queries (decode workloads)")
+                    help="fp8: e4m3 cache with bf16 queries")
     ap.add_argument("--cascade", action="store_true",
                     help="decode through pa_decode_cascade (shared prefixes read once per group)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

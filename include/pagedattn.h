@@ -30,8 +30,8 @@
  *   - Query head h reads kv head h / (num_q_heads / num_kv_heads).
  *   - Supported shapes: head_dim 64 or 128; block_size 1, 2, 4, 8, 16 or 32;
  *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; dtype fp32, bf16 or fp8
- *     e4m3 (decode, append, copies and swaps; prefill and the shared-prefix
- *     decode take bf16 only).
+ *     e4m3 (decode, prefill, append, copies and swaps; the shared-prefix
+ *     decode takes bf16 only).
  */
 #ifndef PAGEDATTN_H
 #define PAGEDATTN_H
@@ -58,8 +58,9 @@ typedef enum {
 /* Cache element types. PA_FP8_E4M3 stores K and V as 8-bit floats (e4m3,
  * no infinities, largest 448) with one scale per tensor (pa_cache.k_scale,
  * v_scale): element = code * scale. The q/k/v inputs of an FP8 cache are bf16;
- * the decode rounds q to f16 for its tensor-core products, so |q| must stay
- * below 65504 (every bf16 value below that converts exactly). */
+ * the decode and the prefill round q to f16 for their tensor-core products, so
+ * |q| must stay below 65504 (bf16 values from 2^-17 up to that convert exactly;
+ * smaller ones move by at most 2^-25). */
 typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 typedef void* pa_stream; /* cudaStream_t */
@@ -197,9 +198,12 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
  *                  sees positions 0 .. L_s - n_s + i. n_s > L_s or L_s above
  *                  max_context_len is clamped and recorded (PA_ERR_DEVICE_BOUNDS).
  *   out            device fp32 [T][num_q_heads][head_dim].
- * Supported: bf16 cache, block_size >= 8 (16, 32 as for decode), head_dim 64
- * or 128, num_q_heads / num_kv_heads in {1, 2, 4, 8}; fp32 caches return
- * PA_ERR_UNSUPPORTED. Accumulation is fp32 on the tensor cores.
+ * Supported: bf16 or e4m3 cache, block_size >= 8 (16, 32 as for decode),
+ * head_dim 64 or 128, num_q_heads / num_kv_heads in {1, 2, 4, 8}; fp32 caches
+ * return PA_ERR_UNSUPPORTED. Accumulation is fp32 on the tensor cores. Over an
+ * e4m3 cache the codes are widened to f16 (exactly), q is rounded to f16 and
+ * the softmax weights enter the P V product as f16 (11 significant bits; the
+ * bf16 path keeps about 16 through a two-part split).
  */
 pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, int32_t max_q_len, int32_t num_q_heads,
                      const pa_cache* cache, const int32_t* block_tables, int32_t max_blocks_per_seq,

@@ -401,9 +401,10 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
   const int G = num_q_heads / cache->num_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
-  if (cache->dtype != PA_BF16 || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
+  if ((cache->dtype != PA_BF16 && cache->dtype != PA_FP8_E4M3) || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size > INT32_MAX)
     return PA_ERR_UNSUPPORTED;
+  const bool f8 = cache->dtype == PA_FP8_E4M3;
   if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * cache->block_size ||
       max_q_len > max_context_len)
     return PA_ERR_INVALID_ARG;
@@ -433,13 +434,20 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   a.max_ctx = max_context_len;
   a.ntiles = static_cast<int32_t>(ntiles);
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.v_scale = 1.f;
+  if (f8) {
+    // q . (k_scale * code) = (k_scale * q) . code; the V scale multiplies O.
+    a.scale_log2 *= cache->k_scale;
+    a.v_scale = cache->v_scale;
+  }
   a.group_offs = a.group_members = a.group_prefix = nullptr;
   a.prefix_part_tokens = a.max_parts = a.parts_stride = 0;
   a.ws_ml = a.ws_o = nullptr;
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
-  if (!encode_rows(&tk, cache->k, rows, cache->head_dim, cache->block_size) ||
-      !encode_rows(&tv, cache->v, rows, cache->head_dim, cache->block_size))
+  auto enc = f8 ? encode_rows_u8 : encode_rows;
+  if (!enc(&tk, cache->k, rows, cache->head_dim, cache->block_size) ||
+      !enc(&tv, cache->v, rows, cache->head_dim, cache->block_size))
     return PA_ERR_CUDA;
   const dim3 grid(cache->num_kv_heads, static_cast<unsigned>(ntiles), num_seqs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -448,6 +456,24 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
     kern<<<grid, threads, smem, s>>>(tk, tv, a);
     return launched();
   };
+  if (f8) {
+    using F128 = TcCfg<128, 2, true>;
+    using F64 = TcCfg<64, 1, true>;
+    if (cache->head_dim == 128) {
+      switch (G) {
+        case 1: return launch(prefill_tc_kernel<128, 1, 2, true>, F128::kThreads, F128::kSmemBytes);
+        case 2: return launch(prefill_tc_kernel<128, 2, 2, true>, F128::kThreads, F128::kSmemBytes);
+        case 4: return launch(prefill_tc_kernel<128, 4, 2, true>, F128::kThreads, F128::kSmemBytes);
+        default: return launch(prefill_tc_kernel<128, 8, 2, true>, F128::kThreads, F128::kSmemBytes);
+      }
+    }
+    switch (G) {
+      case 1: return launch(prefill_tc_kernel<64, 1, 1, true>, F64::kThreads, F64::kSmemBytes);
+      case 2: return launch(prefill_tc_kernel<64, 2, 1, true>, F64::kThreads, F64::kSmemBytes);
+      case 4: return launch(prefill_tc_kernel<64, 4, 1, true>, F64::kThreads, F64::kSmemBytes);
+      default: return launch(prefill_tc_kernel<64, 8, 1, true>, F64::kThreads, F64::kSmemBytes);
+    }
+  }
   using C128 = TcCfg<128, 2>;
   using C64 = TcCfg<64, 1>;
   if (cache->head_dim == 128) {
@@ -544,6 +570,7 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
     pa.max_ctx = max_context_len;
     pa.ntiles = 0;
     pa.scale_log2 = scale * 1.4426950408889634f;
+    pa.v_scale = 1.f;
     pa.group_offs = group_offsets;
     pa.group_members = group_members;
     pa.group_prefix = group_prefix_tokens;

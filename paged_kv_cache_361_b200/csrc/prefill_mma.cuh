@@ -32,6 +32,7 @@ struct PrefillArgs {
   int64_t num_blocks;
   int32_t num_seqs, hq, hkv, bs, max_blocks, max_ctx, ntiles;
   float scale_log2;
+  float v_scale;  // e4m3 cache: multiplies O (1 for bf16)
   // cascade (shared-prefix) mode: group j = members[offs[j] .. offs[j+1]) shares
   // its first prefix_tokens[j] tokens; CTA (g, p, j) writes the partial of
   // prefix partition p for every member row into slot max_parts + p.

@@ -31,30 +31,52 @@
 // The running maximum is moved (and O rescaled in TMEM) only when a row's
 // maximum grows by more than 8 in log2 units, so weights stay below 2^8 and
 // most chunks never touch O; the result is the same softmax.
+//
+// 8-bit (e4m3) cache (F8). P3 = "PagedAttention 和 vLLM", the section on its
+// future: paged KV storage combined with quantisation, a code c standing for
+// value(c) * scale with one scale per tensor. A kind::f16 MMA takes A and B of
+// one type, so the keys and values are widened to f16 (cvt e4m3x2 -> f16x2,
+// exact) by a fourth role:
+//   warps +2..+5  converter: the producer copies [bs x D] byte boxes of codes
+//              (128-byte swizzle at D 128, 64-byte at D 64) into a small
+//              staging ring; the converter writes each chunk as f16 K and V
+//              tiles in the swizzled layout the bf16 path gets from the TMA,
+//              with rows past the stream's last key written as zeros (their
+//              bytes may be anything, a NaN code included).
+// Q is rounded to f16 by the softmax warps as they stage it (exact for
+// 2^-17 <= |q| <= 65504); P is written as f16 (11 mantissa bits, one P V MMA
+// per k-step instead of the bf16 high/low pair). The K scale is folded into
+// the score scale; the V scale multiplies O in the final division.
 #pragma once
 
+#include "decode_f8.cuh"
 #include "prefill_mma.cuh"
 #include "tcgen05.cuh"
 
 namespace pa {
 
-template <int D, int TILES>
+template <int D, int TILES, bool F8 = false>
 struct TcCfg {
   static constexpr int kRows = 128;                        // query rows per tile (MMA M)
   static constexpr int kChunk = 64;                        // keys per stage
   static constexpr int kHalves = D / 64;                   // 128-byte column boxes per row
   static constexpr int kHalfBytes = kChunk * 128;          // one box column of K or V in a stage
-  static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage
+  static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage (16-bit elements)
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = 4;
+  static constexpr int kStages = F8 && TILES > 1 ? 3 : 4;
+  static constexpr int kCodeTileBytes = kChunk * D;        // e4m3 K (or V) of one staging slot
+  static constexpr int kCodeStageBytes = 2 * kCodeTileBytes;
+  static constexpr int kCodeStages = F8 ? (TILES > 1 ? 2 : 3) : 0;
   static constexpr int kQHalfBytes = kRows * 128;
   static constexpr int kQTileBytes = kHalves * kQHalfBytes;
   static constexpr int kQBytes = TILES * kQTileBytes;
-  static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kCodeStages * kCodeStageBytes;
   static constexpr int kSoftmaxWarps = 4 * TILES;          // one warpgroup per tile
   static constexpr int kProducerWarp = kSoftmaxWarps;
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  static constexpr int kConvWarp0 = kSoftmaxWarps + 2;
+  static constexpr int kConvWarps = F8 ? 4 : 0;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kConvWarps);
   // per tile: O (D columns), then two S/P buffers of kChunk columns
   static constexpr uint32_t kTileCols = D + 2 * kChunk;
   static constexpr uint32_t kTmemCols = TILES * kTileCols <= 256 ? 256 : 512;
@@ -70,15 +92,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 // TILES query tiles of one (kv head, sequence) per CTA share the K/V stream;
 // tile t is processed by softmax warpgroup t.
-template <int D, int G, int TILES>
-__global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
+template <int D, int G, int TILES, bool F8 = false>
+__global__ void __launch_bounds__(TcCfg<D, TILES, F8>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                       const PrefillArgs a) {
-  using Cfg = TcCfg<D, TILES>;
+  using Cfg = TcCfg<D, TILES, F8>;
   constexpr int S = Cfg::kStages, C = Cfg::kChunk, TT = Cfg::kRows / G;
+  constexpr int CS = F8 ? Cfg::kCodeStages : 1;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ PipeSmem<S> ps;
+  __shared__ PipeSmem<S> ps;  // 16-bit K/V stages: filled by the TMA (bf16) or the converter (F8)
+  __shared__ uint64_t cfull[CS], cempty[CS];  // F8: code staging ring, producer <-> converter
   __shared__ uint64_t q_full, drain;
   __shared__ uint64_t s_full[TILES][2], p_full[TILES][2], o_bar[TILES];
   __shared__ uint32_t tmem_base_sh;
@@ -87,6 +111,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
   uint8_t* sgen = smem_raw + (sbase - raw);   // generic pointer to sbase
   const uint32_t qs = sbase;                  // Q of tile t: kHalves x [128 rows x 128 B], swizzled
   const uint32_t kv0 = sbase + Cfg::kQBytes;  // stage st: K halves, then V halves
+  const uint32_t cs0 = kv0 + S * Cfg::kStageBytes;  // F8 staging slot: K codes, then V codes
 
   const int g = blockIdx.x, s = blockIdx.z;
   const int pair = a.ntiles - 1 - static_cast<int>(blockIdx.y);  // longest key ranges first
@@ -131,7 +156,22 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
       mbar_init(&p_full[t][1], 4);
       mbar_init(&o_bar[t], 1);
     }
-    pipe_init<S>(ps, 1);  // empty stages are released by one tcgen05.commit
+    if constexpr (F8) {
+#pragma unroll
+      for (int i = 0; i < S; ++i) {
+        mbar_init(&ps.full[i], Cfg::kConvWarps);
+        mbar_init(&ps.empty[i], 1);
+      }
+#pragma unroll
+      for (int i = 0; i < CS; ++i) {
+        mbar_init(&cfull[i], 1);
+        mbar_init(&cempty[i], Cfg::kConvWarps);
+      }
+      ps.abort_flag = 0;
+      fence_mbar_init();
+    } else {
+      pipe_init<S>(ps, 1);  // empty stages are released by one tcgen05.commit
+    }
   }
   if (warp == Cfg::kMmaWarp) {
     tc::alloc(smem_u32(&tmem_base_sh), Cfg::kTmemCols);
@@ -142,7 +182,78 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
   tc::fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == Cfg::kProducerWarp) {
+  if (F8 && warp == Cfg::kProducerWarp) {
+    // ---- producer (F8): codes of chunk i into staging slot i % CS ----
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
+    const uint64_t pol = l2_evict_last_policy();
+    TableAhead ta;
+    ta.init(a.tables + table_row, 0, min(a.max_blocks, (kend_all + a.bs - 1) / a.bs), lane);
+    int i = 0;
+    for (; i < nchunks; ++i) {
+      const int cst = i % CS;
+      if (i >= CS && !warp_wait(&cempty[cst], ((i / CS) - 1) & 1, &ps.abort_flag)) break;
+      const int32_t c0 = i * C;
+      const int32_t nb = (min(C, kend_all - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+      const int32_t blk = ta.get(c0 / a.bs, nb, lane);
+      bool ok = false;
+      if (lane < nb) {
+        ok = blk >= 0 && blk < a.num_blocks;
+        if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) mbar_arrive_expect_tx(&cfull[cst], 2u * __popc(okmask) * box_bytes);
+      __syncwarp();
+      if (ok) {
+        const int32_t y = (blk * a.hkv + g) * a.bs;
+        const uint32_t dst = cs0 + cst * Cfg::kCodeStageBytes + lane * box_bytes;
+        tma_load_2d(dst, &tmk, 0, y, &cfull[cst], pol);
+        tma_load_2d(dst + Cfg::kCodeTileBytes, &tmv, 0, y, &cfull[cst], pol);
+      }
+    }
+    if (ps.abort_flag && lane == 0)  // copies already started land before exit
+      for (int j = (i > CS ? i - CS : 0); j < i; ++j) mbar_wait(&cfull[j % CS], (j / CS) & 1);
+  } else if (F8 && warp >= Cfg::kConvWarp0) {
+    // ---- converter (F8): thread = (row of the chunk, half of its dims) ----
+    const int ct = tid - 32 * Cfg::kConvWarp0;
+    const int row = ct >> 1, half = ct & 1;
+    const int key = D == 128 ? (row & 7) : ((row >> 1) & 3);  // swizzle of the staged code row
+    constexpr int DH = D / 2;
+    const uint8_t* cs0g = sgen + (cs0 - sbase);
+    uint8_t* kv0g = sgen + Cfg::kQBytes;
+    for (int i = 0; i < nchunks; ++i) {
+      const int cst = i % CS, st = i % S;
+      if (!warp_wait(&cfull[cst], (i / CS) & 1, &ps.abort_flag)) break;
+      if (i >= S && !warp_wait(&ps.empty[st], ((i / S) - 1) & 1, &ps.abort_flag)) break;
+      const bool live = i * C + row < kend_all;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint8_t* src = cs0g + cst * Cfg::kCodeStageBytes + which * Cfg::kCodeTileBytes + row * D;
+        uint8_t* dst = kv0g + st * Cfg::kStageBytes + which * Cfg::kTileBytes + row * 128;
+#pragma unroll
+        for (int u = 0; u < DH / 16; ++u) {
+          const int d0 = half * DH + 16 * u;  // 16 codes -> dims d0 .. d0 + 15
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (live) w = *reinterpret_cast<const uint4*>(src + (((d0 >> 4) ^ key) << 4));
+          uint32_t h[8];
+          e4m3x4_f16x2(w.x, h[0], h[1]);
+          e4m3x4_f16x2(w.y, h[2], h[3]);
+          e4m3x4_f16x2(w.z, h[4], h[5]);
+          e4m3x4_f16x2(w.w, h[6], h[7]);
+          // two 16-byte pieces of the 128-byte row of box column d0 / 64
+          uint8_t* rp = dst + (d0 >> 6) * Cfg::kHalfBytes;
+          const int cc = (d0 & 63) >> 3;
+          *reinterpret_cast<uint4*>(rp + ((cc ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(rp + (((cc + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+      }
+      tc::fence_proxy_async();  // generic-proxy writes -> tensor-core reads
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&ps.full[st]);
+        mbar_arrive(&cempty[cst]);
+      }
+    }
+  } else if (warp == Cfg::kProducerWarp) {
     // ---- producer ----
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
@@ -173,8 +284,8 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
   } else if (warp == Cfg::kMmaWarp) {
     // ---- MMA issuer: S_t(j+1) for every tile, then O_t += P_t(j) V(j) ----
     if (lane == 0) {
-      constexpr uint32_t kIdS = tc::idesc_bf16(Cfg::kRows, C, false);
-      constexpr uint32_t kIdPV = tc::idesc_bf16(Cfg::kRows, D, true);
+      constexpr uint32_t kIdS = F8 ? tc::idesc_f16(Cfg::kRows, C, false) : tc::idesc_bf16(Cfg::kRows, C, false);
+      constexpr uint32_t kIdPV = F8 ? tc::idesc_f16(Cfg::kRows, D, true) : tc::idesc_bf16(Cfg::kRows, D, true);
       // Descriptors are built once; an operand at a byte offset from a base
       // is the base descriptor plus offset / 16 (the start-address field,
       // addresses stay below 256 KB so the field never carries over).
@@ -203,12 +314,12 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
         // kHalfBytes apart (one half when D = 64: the offset is then unused)
         const uint64_t vb = vdesc0 + static_cast<uint64_t>(((j % S) * Cfg::kStageBytes) >> 4);
         const uint32_t to = tmem + t * Cfg::kTileCols;
-        const uint32_t tp = to + D + sb * C;  // P high part: 32 columns, remainder: the next 32
+        const uint32_t tp = to + D + sb * C;  // P (bf16 high part, or f16): 32 columns; bf16 remainder: the next 32
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks) {
           const uint64_t bd = vb + static_cast<uint64_t>((ks * 16 * 128) >> 4);
           tc::mma_ts(to, tp + ks * 8, bd, kIdPV, j > 0 || ks > 0);
-          tc::mma_ts(to, tp + C / 2 + ks * 8, bd, kIdPV, true);
+          if constexpr (!F8) tc::mma_ts(to, tp + C / 2 + ks * 8, bd, kIdPV, true);
         }
         tc::commit(smem_u32(&o_bar[t]));
         return true;
@@ -259,7 +370,10 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
         uint8_t* qdst = sgen + t * Cfg::kQTileBytes;
 #pragma unroll
         for (int c16 = 0; c16 < D / 8; ++c16) {
-          const uint4 v = valid ? __ldg(src + c16) : make_uint4(0u, 0u, 0u, 0u);
+          uint4 v = valid ? __ldg(src + c16) : make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (F8)
+            v = make_uint4(pack_f16(bf16lo(v.x), bf16hi(v.x)), pack_f16(bf16lo(v.y), bf16hi(v.y)),
+                           pack_f16(bf16lo(v.z), bf16hi(v.z)), pack_f16(bf16lo(v.w), bf16hi(v.w)));
           const int hf = c16 >> 3, cc = c16 & 7;
           *reinterpret_cast<uint4*>(qdst + hf * Cfg::kQHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
         }
@@ -268,10 +382,11 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
         if (lane == 0) mbar_arrive(&q_full);
       }
       // the stream's last chunk holds rows past its last key; the lowest tile
-      // that reads that chunk zeroes their V before any P V reads them
+      // that reads that chunk zeroes their V before any P V reads them (the
+      // converter writes them as zeros on the F8 path)
       bool zero_tail = false;
 #pragma unroll
-      for (int u = 0; u < TILES; ++u)
+      for (int u = 0; u < (F8 ? 0 : TILES); ++u)
         if (nch[u] == nchunks) {
           zero_tail = u == t;
           break;
@@ -328,12 +443,15 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
           const float p0 = fast_exp2(fmaf(x[2 * c], sl2, -m_ref));
           const float p1 = fast_exp2(fmaf(x[2 * c + 1], sl2, -m_ref));
           part[c & 3] += p0 + p1;
-          split_pair(p0, p1, ph[c], pl[c]);
+          if constexpr (F8)
+            ph[c] = pack_f16(p0, p1);  // weights <= 2^8
+          else
+            split_pair(p0, p1, ph[c], pl[c]);
         }
         l += (part[0] + part[1]) + (part[2] + part[3]);
         __syncwarp();
         tc::st32(trow + D + sb * C, ph);
-        tc::st32(trow + D + sb * C + C / 2, pl);
+        if constexpr (!F8) tc::st32(trow + D + sb * C + C / 2, pl);
         if (__any_sync(0xffffffffu, resc)) {
           // O must hold P(j-1) V(j-1) before it is rescaled (P(j-2) V(j-2) is
           // complete: it was issued before S(j), which this chunk waited for)
@@ -385,7 +503,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES>::kThreads, 1)
       if (ok) ok = warp_wait(&o_bar[t], (mych - 1) & 1, &ps.abort_flag);
       if (ok) {
         tc::fence_after();
-        const float inv = 1.f / l;
+        const float inv = (F8 ? a.v_scale : 1.f) / l;
         float* dst = a.out + orow * D;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {

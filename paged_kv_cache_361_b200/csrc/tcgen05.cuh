@@ -10,7 +10,8 @@
 //     [32, 46), version 1 in [46, 48), base offset 0 in [49, 52), layout in
 //     [61, 64) (2 = 128-byte swizzle).
 //   instruction descriptor for kind::f16 (32 bit): D format in [4, 6)
-//     (1 = f32), A format in [7, 10) and B format in [10, 13) (1 = bf16), A
+//     (1 = f32), A format in [7, 10) and B format in [10, 13) (0 = f16,
+//     1 = bf16; A and B of one MMA have the same format), A
 //     major bit 15 and B major bit 16 (0 = K-major, 1 = M/N-major), N / 8 in
 //     [17, 23), M / 16 in [24, 29).
 //   TMEM address: lane in bits [16, 32), column in [0, 16). A warp may touch
@@ -31,6 +32,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
 // bf16 x bf16 -> f32, M x N, A K-major, B K-major (b_mn = false) or N-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// f16 x f16 -> f32, M x N, A K-major, B K-major (b_mn = false) or N-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn) {
+  return (1u << 4) | (b_mn ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

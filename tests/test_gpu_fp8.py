@@ -203,14 +203,84 @@ def test_fp8_step_host_matches_oracle():
 
 
 def test_fp8_unsupported_paths_say_so():
+    """The shared-prefix decode has no e4m3 path: it says so instead of reading codes as bf16."""
     cache = PagedKVCache(8, 2, 16, 128, torch.float8_e4m3fn, "cuda", fill=0.0, k_scale=1.0, v_scale=1.0)
-    k = torch.randn(20, 2, 128, device="cuda").bfloat16()
+    k = torch.randn(80, 2, 128, device="cuda").bfloat16()
     cache.add_sequence(0, k, k)
-    q = torch.randn(4, 8, 128, device="cuda").bfloat16()
-    kn = torch.randn(4, 2, 128, device="cuda").bfloat16()
+    cache.fork(0, 1)
+    q = torch.randn(2, 8, 128, device="cuda").bfloat16()
     with pytest.raises(B.PagedAttnError) as e:
-        cache.prefill([0], [4], q, kn, kn, 0.1)
+        cache.decode_cascade([0, 1], q, 0.1)
     assert e.value.status == B.PA_ERR_UNSUPPORTED
+
+
+def _dq(x, scale):
+    """The oracle's view of bf16 rows stored in an e4m3 cache: dequantised codes (fp64)."""
+    return fp8.dequantize(fp8.quantize(x.float().numpy(), scale), scale)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_fp8_prefill_chunked_matches_oracle(G, D, bs):
+    """Chunked prefill over an e4m3 cache: sequences grow by a chunk or start;
+    every new token's causal attention matches the oracle's fp64 attention over
+    the dequantised rows. Pool padding is NaN codes."""
+    from oracle.prefill import prefill_attention
+    rng = np.random.default_rng(7000 + G * 1000 + D + bs)
+    hkv, nseq = 2, 5
+    pre = rng.integers(0, 300, size=nseq)
+    pre[0] = 0
+    chunk = rng.integers(1, 200, size=nseq)
+    chunk[1] = 128 // G           # exactly one 128-row query tile
+    chunk[2] = 64 // G            # half a tile
+    chunk[3] = 256 // G + 3       # two tiles (one CTA at head_dim 128) and a ragged third
+    nb = int(sum(-(-int(p + c) // bs) for p, c in zip(pre, chunk))) + 4
+    cache = PagedKVCache(nb, hkv, bs, D, torch.float8_e4m3fn, "cuda", rng.permutation(nb), fill=float("nan"),
+                         k_scale=K_SCALE, v_scale=V_SCALE)
+    g = torch.Generator().manual_seed(int(rng.integers(1 << 30)))
+    K = {s: torch.randn(int(pre[s] + chunk[s]), hkv, D, generator=g).bfloat16() for s in range(nseq)}
+    V = {s: torch.randn(int(pre[s] + chunk[s]), hkv, D, generator=g).bfloat16() for s in range(nseq)}
+    for s in range(nseq):
+        if pre[s]:
+            cache.add_sequence(s, K[s][:pre[s]].cuda(), V[s][:pre[s]].cuda())
+    q = torch.randn(int(chunk.sum()), hkv * G, D, generator=g).bfloat16()
+    k_new = torch.cat([K[s][pre[s]:] for s in range(nseq)])
+    v_new = torch.cat([V[s][pre[s]:] for s in range(nseq)])
+    out = cache.prefill(list(range(nseq)), chunk, q.cuda(), k_new.cuda(), v_new.cuda(), D ** -0.5).cpu()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    row = 0
+    for s in range(nseq):
+        n = int(chunk[s])
+        ref = prefill_attention(q[row:row + n], _dq(K[s], K_SCALE), _dq(V[s], V_SCALE), D ** -0.5)
+        o = out[row:row + n].double().numpy()
+        assert np.isfinite(o).all()
+        err = float(np.abs(o - ref).max())
+        assert err <= TOL_FP8, f"seq {s}: {err}"
+        row += n
+
+
+@pytest.mark.parametrize("G,D", [(1, 128), (8, 128), (4, 64)])
+def test_fp8_prefill_long_chunk_many_tiles(G, D):
+    """A 700-token chunk after 900 cached tokens over an e4m3 cache: many query
+    tiles, 25 key chunks, a ragged last tile and key chunk (sampled rows)."""
+    from oracle.prefill import prefill_attention
+    hkv, bs = 2, 16
+    g = torch.Generator().manual_seed(90 + G + D)
+    pre, n = 900, 700
+    nb = -(-(pre + n) // bs) + 3
+    cache = PagedKVCache(nb, hkv, bs, D, torch.float8_e4m3fn, "cuda", np.random.default_rng(G).permutation(nb),
+                         fill=float("nan"), k_scale=K_SCALE, v_scale=V_SCALE)
+    K = torch.randn(pre + n, hkv, D, generator=g).bfloat16()
+    V = torch.randn(pre + n, hkv, D, generator=g).bfloat16()
+    cache.add_sequence(0, K[:pre].cuda(), V[:pre].cuda())
+    q = torch.randn(n, hkv * G, D, generator=g).bfloat16()
+    out = cache.prefill([0], [n], q.cuda(), K[pre:].cuda(), V[pre:].cuda(), D ** -0.5).cpu()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    rows = np.r_[0:30, 300:330, n - 30:n]
+    ref = prefill_attention(q, _dq(K, K_SCALE), _dq(V, V_SCALE), D ** -0.5)
+    err = float(np.abs(out.double().numpy()[rows] - ref[rows]).max())
+    assert err <= TOL_FP8, err
 
 
 def test_fp8_bad_scale_rejected():
