@@ -165,18 +165,25 @@ def build_workload(seed: int, device, name: str = "llama2_7b_mha", kv_dtype: str
     manager; its tables and lengths are uploaded once.
 
     kv_dtype "fp8" stores the cache as e4m3 codes (per-tensor scales 1.0: the
-    N(0,1) values are inside the e4m3 range); q and the new K/V rows stay bf16."""
+    N(0,1) values are inside the e4m3 range), "int8" as uniform random int8
+    codes in [-127, 127] (scales 4/127); q and the new K/V rows stay bf16."""
     from paged_kv_cache_361_b200 import PagedKVCache
     from paged_kv_cache_361_b200 import workloads as W
     sh, nb, order, scale, part, ops = workload_ops(name, seed)
     dt = W.TORCH_DTYPE[sh.dtype]
-    cache_dt = torch.float8_e4m3fn if kv_dtype == "fp8" else dt
-    cache = PagedKVCache(nb, sh.num_kv_heads, sh.block_size, sh.head_dim, cache_dt, device, order)
+    cache_dt = {"fp8": torch.float8_e4m3fn, "int8": torch.int8}.get(kv_dtype, dt)
+    sc = 4.0 / 127 if kv_dtype == "int8" else 1.0
+    cache = PagedKVCache(nb, sh.num_kv_heads, sh.block_size, sh.head_dim, cache_dt, device, order, k_scale=sc,
+                         v_scale=sc)
     g = torch.Generator(device=device)
     g.manual_seed(1000 + seed)
     for t in (cache.k_cache, cache.v_cache):
         for i in range(0, nb, 1024):   # chunked to bound the fp32 temporary
-            t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(cache_dt)
+            if kv_dtype == "int8":
+                t[i:i + 1024] = torch.randint(-127, 128, t[i:i + 1024].shape, generator=g, device=device,
+                                              dtype=torch.int8)
+            else:
+                t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(cache_dt)
     hkv, D = sh.num_kv_heads, sh.head_dim
     assert ops[-2][0] == "append" and ops[-1][0] == "decode"
     for op in ops[:-2]:
@@ -376,7 +383,8 @@ def run_ours(args, rank, world, device):
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8_e4m3 cache, bf16 q" if args.kv_dtype == "fp8" else sh.dtype, "data": "synthetic",
+            "dtype": {"fp8": "fp8_e4m3 cache, bf16 q", "int8": "int8 cache, bf16 q"}.get(args.kv_dtype, sh.dtype),
+            "data": "synthetic",
             "config": {"workload": WORKLOADS[args.workload], "num_seqs": nseq, "num_q_heads": sh.num_q_heads,
                        "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "block_size": sh.block_size,
                        "num_blocks": int(d["kc"].shape[0]), "context_tokens": int(d["lens_host"].sum()),
@@ -469,10 +477,12 @@ def run_prefill(args, rank, world, device):
     D, bs = 128, 16
     nb = nseq * plen // bs + 16
     order = np.random.default_rng(rank).permutation(nb)
-    f8 = args.kv_dtype == "fp8"
-    if f8:
+    f8 = args.kv_dtype in ("fp8", "int8")
+    if args.kv_dtype == "fp8":
         cache = PagedKVCache(nb, hkv, bs, D, torch.float8_e4m3fn, device, order, k_scale=4.0 / 448,
                              v_scale=4.0 / 448)
+    elif args.kv_dtype == "int8":
+        cache = PagedKVCache(nb, hkv, bs, D, torch.int8, device, order, k_scale=4.0 / 127, v_scale=4.0 / 127)
     else:
         cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, device, order)
     g = torch.Generator(device=device)
@@ -532,9 +542,10 @@ def run_prefill(args, rank, world, device):
             "value": round(all_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8_e4m3 cache, bf16 q (f16 MMA)" if f8 else "bf16", "data": "synthetic",
+            "dtype": f"{'fp8_e4m3' if args.kv_dtype == 'fp8' else 'int8'} cache, bf16 q (f16 MMA)" if f8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": f"{args.workload}: {nseq} prompts x {plen} tokens, {hq}/{hkv} heads, D128, bs16",
-                       "kv_dtype": "float8_e4m3fn" if f8 else "bfloat16",
+                       "kv_dtype": str(cache.k_cache.dtype).replace("torch.", ""),
                        "l2": "no flush: K/V of one launch "
                              + f"{2 * T * hkv * D * (1 if f8 else 2) / 1e6:.0f} MB"},
             "gpu_launches": 2 * args.steps,
@@ -595,8 +606,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL), default="llama2_7b_mha")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--kv-dtype", choices=["auto", "fp8"], default="auto",
-                    help="fp8: e4m3 cache with bf16 queries")
+    ap.add_argument("--kv-dtype", choices=["auto", "fp8", "int8"], default="auto",
+                    help="fp8 / int8: an 8-bit cache (e4m3 or int8 codes) with bf16 queries")
     ap.add_argument("--cascade", action="store_true",
                     help="decode through pa_decode_cascade (shared prefixes read once per group)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -29,8 +29,8 @@
  *     A "slot" is block * block_size + offset.
  *   - Query head h reads kv head h / (num_q_heads / num_kv_heads).
  *   - Supported shapes: head_dim 64 or 128; block_size 1, 2, 4, 8, 16 or 32;
- *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; dtype fp32, bf16 or fp8
- *     e4m3 (decode, prefill, append, copies and swaps; the shared-prefix
+ *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; dtype fp32, bf16, or 8-bit
+ *     e4m3 / int8 (decode, prefill, append, copies and swaps; the shared-prefix
  *     decode takes bf16 only).
  */
 #ifndef PAGEDATTN_H
@@ -56,12 +56,13 @@ typedef enum {
 } pa_status;
 
 /* Cache element types. PA_FP8_E4M3 stores K and V as 8-bit floats (e4m3,
- * no infinities, largest 448) with one scale per tensor (pa_cache.k_scale,
- * v_scale): element = code * scale. The q/k/v inputs of an FP8 cache are bf16;
+ * no infinities, largest 448), PA_INT8 as integers in [-127, 127], each with
+ * one scale per tensor (pa_cache.k_scale, v_scale): element = code * scale.
+ * The q/k/v inputs of an 8-bit cache are bf16;
  * the decode and the prefill round q to f16 for their tensor-core products, so
  * |q| must stay below 65504 (bf16 values from 2^-17 up to that convert exactly;
  * smaller ones move by at most 2^-25). */
-typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2, PA_INT8 = 3 } pa_dtype;
 
 typedef void* pa_stream; /* cudaStream_t */
 
@@ -75,9 +76,9 @@ typedef struct {
   int32_t num_kv_heads;  /* >= 1 */
   int32_t block_size;    /* tokens per block */
   int32_t head_dim;      /* elements per head row */
-  int32_t dtype;         /* pa_dtype of k, v (and of the q/k/v inputs, bf16 for FP8) */
-  float k_scale;         /* PA_FP8_E4M3 only: K element = code * k_scale (> 0) */
-  float v_scale;         /* PA_FP8_E4M3 only: V element = code * v_scale (> 0) */
+  int32_t dtype;         /* pa_dtype of k, v (and of the q/k/v inputs, bf16 for 8-bit) */
+  float k_scale;         /* 8-bit dtypes only: K element = code * k_scale (> 0) */
+  float v_scale;         /* 8-bit dtypes only: V element = code * v_scale (> 0) */
 } pa_cache;
 
 /* Human-readable name of a status code (static storage). */
@@ -102,10 +103,11 @@ int32_t pa_version(void);
  *                 recorded as PA_ERR_DEVICE_BOUNDS.
  *   num_tokens    >= 0; 0 launches nothing.
  * Two tokens must not name the same slot in one call (the result would be
- * either row). A bit copy for fp32 / bf16 caches. For an FP8 cache the rows
- * are bf16 and each element is stored as the e4m3 code of x / scale computed
- * in fp32, rounded to nearest even, clamped to +-448 (the "quantised code"
- * step of an 8-bit KV cache).
+ * either row). A bit copy for fp32 / bf16 caches. For an 8-bit cache the
+ * rows are bf16 and each element is stored as the code of x / scale computed
+ * in fp32 and rounded to nearest even: e4m3 clamped to +-448 (NaN stays NaN),
+ * int8 clamped to [-127, 127] (NaN becomes 0) (the "quantised code" step of
+ * an 8-bit KV cache).
  */
 pa_status pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
                                const pa_cache* cache, pa_stream stream);
@@ -198,10 +200,10 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
  *                  sees positions 0 .. L_s - n_s + i. n_s > L_s or L_s above
  *                  max_context_len is clamped and recorded (PA_ERR_DEVICE_BOUNDS).
  *   out            device fp32 [T][num_q_heads][head_dim].
- * Supported: bf16 or e4m3 cache, block_size >= 8 (16, 32 as for decode),
+ * Supported: bf16, e4m3 or int8 cache, block_size >= 8 (16, 32 as for decode),
  * head_dim 64 or 128, num_q_heads / num_kv_heads in {1, 2, 4, 8}; fp32 caches
  * return PA_ERR_UNSUPPORTED. Accumulation is fp32 on the tensor cores. Over an
- * e4m3 cache the codes are widened to f16 (exactly), q is rounded to f16 and
+ * 8-bit cache the codes are widened to f16 (exactly), q is rounded to f16 and
  * the softmax weights enter the P V product as f16 (11 significant bits; the
  * bf16 path keeps about 16 through a two-part split).
  */

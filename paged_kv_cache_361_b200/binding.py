@@ -18,13 +18,14 @@ LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_NO_FREE_BLOCKS, PA_ERR_UNKNOWN_SEQ, PA_ERR_SEQ_EXISTS, \
     PA_ERR_CUDA, PA_ERR_DEVICE_BOUNDS, PA_ERR_DEVICE_TIMEOUT = range(9)
-PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
-_DTYPE = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float8_e4m3fn: PA_FP8_E4M3}
+PA_F32, PA_BF16, PA_FP8_E4M3, PA_INT8 = 0, 1, 2, 3
+_DTYPE = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float8_e4m3fn: PA_FP8_E4M3, torch.int8: PA_INT8}
+CODED_DTYPES = (torch.float8_e4m3fn, torch.int8)   # 8-bit caches: codes times a per-tensor scale
 
 
 def input_dtype(cache_dtype):
     """dtype of q and of the new K/V rows for a cache of cache_dtype."""
-    return torch.bfloat16 if cache_dtype == torch.float8_e4m3fn else cache_dtype
+    return torch.bfloat16 if cache_dtype in CODED_DTYPES else cache_dtype
 
 
 class PagedAttnError(RuntimeError):
@@ -123,13 +124,13 @@ def _dev(t: torch.Tensor, name: str, dtype=None, ndim=None):
     return t.data_ptr()
 
 
-# An fp8 cache carries its per-tensor scales on the two cache tensor objects
-# (set with set_fp8_scales); make_cache refuses an fp8 cache without them.
-def set_fp8_scales(k_cache, v_cache, k_scale: float, v_scale: float):
-    if k_cache.dtype != torch.float8_e4m3fn or v_cache.dtype != torch.float8_e4m3fn:
-        raise TypeError("scales belong to a float8_e4m3fn cache")
-    k_cache._pa_fp8_scale = float(k_scale)
-    v_cache._pa_fp8_scale = float(v_scale)
+# An 8-bit cache (e4m3 or int8) carries its per-tensor scales on the two cache
+# tensor objects (set with set_kv_scales); make_cache refuses one without them.
+def set_kv_scales(k_cache, v_cache, k_scale: float, v_scale: float):
+    if k_cache.dtype not in CODED_DTYPES or v_cache.dtype != k_cache.dtype:
+        raise TypeError("scales belong to a float8_e4m3fn or int8 cache")
+    k_cache._pa_kv_scale = float(k_scale)
+    v_cache._pa_kv_scale = float(v_scale)
 
 
 def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> pa_cache:
@@ -140,10 +141,10 @@ def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> pa_cache:
         raise TypeError(f"unsupported cache dtype {k_cache.dtype}")
     nb, hkv, bs, d = k_cache.shape
     ks = vs = 1.0
-    if k_cache.dtype == torch.float8_e4m3fn:
-        ks, vs = getattr(k_cache, "_pa_fp8_scale", None), getattr(v_cache, "_pa_fp8_scale", None)
+    if k_cache.dtype in CODED_DTYPES:
+        ks, vs = getattr(k_cache, "_pa_kv_scale", None), getattr(v_cache, "_pa_kv_scale", None)
         if ks is None or vs is None:
-            raise ValueError("fp8 cache without scales: call set_fp8_scales(k_cache, v_cache, k_scale, v_scale)")
+            raise ValueError("8-bit cache without scales: call set_kv_scales(k_cache, v_cache, k_scale, v_scale)")
     return pa_cache(_dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4), nb, hkv, bs, d,
                     _DTYPE[k_cache.dtype], ks, vs)
 

@@ -41,8 +41,11 @@ class PagedKVCache:
     def __init__(self, num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
                  dtype=torch.bfloat16, device="cuda", free_order=None, fill: float | None = None,
                  k_scale: float = 1.0, v_scale: float = 1.0):
-        """dtype torch.float8_e4m3fn makes an 8-bit cache with per-tensor scales
-        (element = code * scale); its q/k/v inputs are bf16."""
+        """dtype torch.float8_e4m3fn or torch.int8 makes an 8-bit cache with
+        per-tensor scales (element = code * scale); its q/k/v inputs are bf16.
+        fill sets every pool byte before use: an e4m3 cache stores the code of
+        fill; an int8 cache has no NaN, so a NaN fill stores -128, the code
+        quantisation never writes."""
         self.device = torch.device(device)
         shape = (num_blocks, num_kv_heads, block_size, head_dim)
         self.k_cache = torch.empty(shape, dtype=dtype, device=self.device)
@@ -51,11 +54,13 @@ class PagedKVCache:
             if dtype == torch.float8_e4m3fn:
                 code = int(torch.tensor(fill, dtype=torch.float32).to(dtype).view(torch.uint8).item())
                 self.k_cache.view(torch.uint8).fill_(code)
+            elif dtype == torch.int8:
+                self.k_cache.fill_(-128 if math.isnan(fill) else int(fill))
             else:
                 self.k_cache.fill_(fill)
             self.v_cache.copy_(self.k_cache)
-        if dtype == torch.float8_e4m3fn:
-            B.set_fp8_scales(self.k_cache, self.v_cache, k_scale, v_scale)
+        if dtype in B.CODED_DTYPES:
+            B.set_kv_scales(self.k_cache, self.v_cache, k_scale, v_scale)
         self.block_size = block_size
         self.bm = B.BlockManager(num_blocks, block_size, free_order)
         self.lens: dict[int, int] = {}

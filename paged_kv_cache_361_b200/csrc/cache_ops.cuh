@@ -45,10 +45,20 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const int4* __re
   }
 }
 
-// FP8 cache: k, v rows are bf16 [num_tokens][hkv][D]; each thread turns 16
-// bf16 inputs (two 16-byte loads) into one 16-byte store of e4m3 codes.
+// 8-bit cache (CF: e4m3 or int8 codes): k, v rows are bf16 [num_tokens][hkv][D];
+// each thread turns 16 bf16 inputs (two 16-byte loads) into one 16-byte store
+// of codes.
 //   row_chunks = D / 16 per (token, head) row
-__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4* __restrict__ k,
+template <int CF>
+__device__ __forceinline__ uint32_t quantize_code(float x, float scale) {
+  if constexpr (CF == kCodeS8)
+    return static_cast<uint8_t>(quantize_s8(x, scale));
+  else
+    return quantize_e4m3(x, scale);
+}
+
+template <int CF>
+__global__ void __launch_bounds__(256) reshape_and_cache_q8_kernel(const uint4* __restrict__ k,
                                                                     const uint4* __restrict__ v,
                                                                     const int64_t* __restrict__ slots,
                                                                     int4* __restrict__ kc, int4* __restrict__ vc,
@@ -81,10 +91,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4*
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const uint32_t lo = w[2 * u], hi = w[2 * u + 1];
-        q[u] = static_cast<uint32_t>(quantize_e4m3(bf16lo(lo), sc)) |
-               (static_cast<uint32_t>(quantize_e4m3(bf16hi(lo), sc)) << 8) |
-               (static_cast<uint32_t>(quantize_e4m3(bf16lo(hi), sc)) << 16) |
-               (static_cast<uint32_t>(quantize_e4m3(bf16hi(hi), sc)) << 24);
+        q[u] = quantize_code<CF>(bf16lo(lo), sc) | (quantize_code<CF>(bf16hi(lo), sc) << 8) |
+               (quantize_code<CF>(bf16lo(hi), sc) << 16) | (quantize_code<CF>(bf16hi(hi), sc) << 24);
       }
       (which == 0 ? kc : vc)[dst] = make_int4(q[0], q[1], q[2], q[3]);
     }

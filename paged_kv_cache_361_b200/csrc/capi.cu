@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -21,16 +22,17 @@ using namespace pa;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool pow2_block(int32_t bs) { return bs == 1 || bs == 2 || bs == 4 || bs == 8 || bs == 16 || bs == 32; }
-int elem_bytes(int32_t dtype) { return dtype == PA_FP8_E4M3 ? 1 : (dtype == PA_BF16 ? 2 : 4); }
+bool is_8bit(int32_t dtype) { return dtype == PA_FP8_E4M3 || dtype == PA_INT8; }
+int elem_bytes(int32_t dtype) { return is_8bit(dtype) ? 1 : (dtype == PA_BF16 ? 2 : 4); }
 
 pa_status check_cache(const pa_cache* c) {
   if (!c || !c->k || !c->v || !aligned16(c->k) || !aligned16(c->v)) return PA_ERR_INVALID_ARG;
   if (c->num_blocks <= 0 || c->num_blocks > INT32_MAX || c->num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
   if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (!pow2_block(c->block_size)) return PA_ERR_UNSUPPORTED;
-  if (c->dtype != PA_F32 && c->dtype != PA_BF16 && c->dtype != PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
-  if (c->dtype == PA_FP8_E4M3 && !(std::isfinite(c->k_scale) && c->k_scale > 0.f && std::isfinite(c->v_scale) &&
-                                   c->v_scale > 0.f))
+  if (c->dtype != PA_F32 && c->dtype != PA_BF16 && !is_8bit(c->dtype)) return PA_ERR_UNSUPPORTED;
+  if (is_8bit(c->dtype) && !(std::isfinite(c->k_scale) && c->k_scale > 0.f && std::isfinite(c->v_scale) &&
+                             c->v_scale > 0.f))
     return PA_ERR_INVALID_ARG;
   // slots must fit in int64 and block ids in int32 (checked above)
   return PA_OK;
@@ -181,34 +183,40 @@ bool encode_rows_u8(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tensor-core decode over an e4m3 cache (block_size >= 8, pool rows addressable by the TMA).
+// Tensor-core decode over an 8-bit cache (block_size >= 8, pool rows addressable by the TMA).
 bool f8_mma_eligible(const pa_cache* c) {
-  return c->dtype == PA_FP8_E4M3 && c->block_size >= 8 &&
+  return is_8bit(c->dtype) && c->block_size >= 8 &&
          static_cast<int64_t>(c->num_blocks) * c->num_kv_heads * c->block_size <= INT32_MAX;
 }
 
-template <int D, int G>
+template <int D, int G, int CF>
 pa_status launch_f8(const DecodeArgs& a, const pa_cache* c, dim3 grid, cudaStream_t st) {
   using Cfg = F8Cfg<D>;
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(c->num_blocks) * c->num_kv_heads * c->block_size;
   if (!encode_rows_u8(&tk, c->k, rows, D, c->block_size) || !encode_rows_u8(&tv, c->v, rows, D, c->block_size))
     return PA_ERR_CUDA;
-  auto kern = decode_f8_kernel<D, G>;
+  auto kern = decode_f8_kernel<D, G, CF>;
   if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;
   kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
   return launched();
 }
 
-template <int D>
-pa_status dispatch_f8(const DecodeArgs& a, const pa_cache* c, int G, dim3 grid, cudaStream_t st) {
+template <int D, int CF>
+pa_status dispatch_f8_cf(const DecodeArgs& a, const pa_cache* c, int G, dim3 grid, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_f8<D, 1>(a, c, grid, st);
-    case 2: return launch_f8<D, 2>(a, c, grid, st);
-    case 4: return launch_f8<D, 4>(a, c, grid, st);
-    case 8: return launch_f8<D, 8>(a, c, grid, st);
+    case 1: return launch_f8<D, 1, CF>(a, c, grid, st);
+    case 2: return launch_f8<D, 2, CF>(a, c, grid, st);
+    case 4: return launch_f8<D, 4, CF>(a, c, grid, st);
+    case 8: return launch_f8<D, 8, CF>(a, c, grid, st);
     default: return PA_ERR_UNSUPPORTED;
   }
+}
+
+template <int D>
+pa_status dispatch_f8(const DecodeArgs& a, const pa_cache* c, int G, dim3 grid, cudaStream_t st) {
+  return c->dtype == PA_INT8 ? dispatch_f8_cf<D, kCodeS8>(a, c, G, grid, st)
+                             : dispatch_f8_cf<D, kCodeE4M3>(a, c, G, grid, st);
 }
 
 template <int D, int G>
@@ -318,8 +326,9 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, const int64_t* slot
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;  // grid-stride beyond this
-  if (cache->dtype == PA_FP8_E4M3) {
-    reshape_and_cache_fp8_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+  if (is_8bit(cache->dtype)) {
+    auto kern = cache->dtype == PA_INT8 ? reshape_and_cache_q8_kernel<kCodeS8> : reshape_and_cache_q8_kernel<kCodeE4M3>;
+    kern<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, static_cast<int4*>(cache->k),
         static_cast<int4*>(cache->v), num_tokens, cache->num_kv_heads, cache->block_size, row_chunks,
         cache->num_blocks * cache->block_size, cache->k_scale, cache->v_scale);
@@ -401,10 +410,10 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
   const int G = num_q_heads / cache->num_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
-  if ((cache->dtype != PA_BF16 && cache->dtype != PA_FP8_E4M3) || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
+  if ((cache->dtype != PA_BF16 && !is_8bit(cache->dtype)) || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size > INT32_MAX)
     return PA_ERR_UNSUPPORTED;
-  const bool f8 = cache->dtype == PA_FP8_E4M3;
+  const bool f8 = is_8bit(cache->dtype);
   if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * cache->block_size ||
       max_q_len > max_context_len)
     return PA_ERR_INVALID_ARG;
@@ -456,24 +465,28 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
     kern<<<grid, threads, smem, s>>>(tk, tv, a);
     return launched();
   };
-  if (f8) {
+  auto launch8 = [&](auto cf) -> pa_status {
+    constexpr int CF = decltype(cf)::value;
     using F128 = TcCfg<128, 2, true>;
     using F64 = TcCfg<64, 1, true>;
     if (cache->head_dim == 128) {
       switch (G) {
-        case 1: return launch(prefill_tc_kernel<128, 1, 2, true>, F128::kThreads, F128::kSmemBytes);
-        case 2: return launch(prefill_tc_kernel<128, 2, 2, true>, F128::kThreads, F128::kSmemBytes);
-        case 4: return launch(prefill_tc_kernel<128, 4, 2, true>, F128::kThreads, F128::kSmemBytes);
-        default: return launch(prefill_tc_kernel<128, 8, 2, true>, F128::kThreads, F128::kSmemBytes);
+        case 1: return launch(prefill_tc_kernel<128, 1, 2, CF>, F128::kThreads, F128::kSmemBytes);
+        case 2: return launch(prefill_tc_kernel<128, 2, 2, CF>, F128::kThreads, F128::kSmemBytes);
+        case 4: return launch(prefill_tc_kernel<128, 4, 2, CF>, F128::kThreads, F128::kSmemBytes);
+        default: return launch(prefill_tc_kernel<128, 8, 2, CF>, F128::kThreads, F128::kSmemBytes);
       }
     }
     switch (G) {
-      case 1: return launch(prefill_tc_kernel<64, 1, 1, true>, F64::kThreads, F64::kSmemBytes);
-      case 2: return launch(prefill_tc_kernel<64, 2, 1, true>, F64::kThreads, F64::kSmemBytes);
-      case 4: return launch(prefill_tc_kernel<64, 4, 1, true>, F64::kThreads, F64::kSmemBytes);
-      default: return launch(prefill_tc_kernel<64, 8, 1, true>, F64::kThreads, F64::kSmemBytes);
+      case 1: return launch(prefill_tc_kernel<64, 1, 1, CF>, F64::kThreads, F64::kSmemBytes);
+      case 2: return launch(prefill_tc_kernel<64, 2, 1, CF>, F64::kThreads, F64::kSmemBytes);
+      case 4: return launch(prefill_tc_kernel<64, 4, 1, CF>, F64::kThreads, F64::kSmemBytes);
+      default: return launch(prefill_tc_kernel<64, 8, 1, CF>, F64::kThreads, F64::kSmemBytes);
     }
-  }
+  };
+  if (f8)
+    return cache->dtype == PA_INT8 ? launch8(std::integral_constant<int, kCodeS8>{})
+                                   : launch8(std::integral_constant<int, kCodeE4M3>{});
   using C128 = TcCfg<128, 2>;
   using C64 = TcCfg<64, 1>;
   if (cache->head_dim == 128) {
@@ -709,7 +722,7 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   a.force_partials = 0;
   a.parts_stride = parts;
   a.prefix_part_tokens = 0;
-  if (cache->dtype == PA_FP8_E4M3) {
+  if (is_8bit(cache->dtype)) {
     // q . (k_scale * code) = (k_scale * q) . code; the V scale multiplies o.
     a.scale_log2 *= cache->k_scale;
     a.v_scale = cache->v_scale;
@@ -725,6 +738,8 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
     st = D == 128 ? dispatch_f8<128>(a, cache, G, grid, s) : dispatch_f8<64>(a, cache, G, grid, s);
   } else if (cache->dtype == PA_FP8_E4M3) {
     st = D == 128 ? dispatch_g<__nv_fp8_e4m3, 128>(a, G, grid, s) : dispatch_g<__nv_fp8_e4m3, 64>(a, G, grid, s);
+  } else if (cache->dtype == PA_INT8) {
+    st = D == 128 ? dispatch_g<int8_t, 128>(a, G, grid, s) : dispatch_g<int8_t, 64>(a, G, grid, s);
   } else if (cache->dtype == PA_BF16) {
     st = D == 128 ? dispatch_g<__nv_bfloat16, 128>(a, G, grid, s) : dispatch_g<__nv_bfloat16, 64>(a, G, grid, s);
   } else {

@@ -117,6 +117,28 @@ __device__ __forceinline__ uint8_t quantize_e4m3(float x, float scale) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
 }
 
+// x / scale in fp32 (IEEE division), rounded to the nearest integer (ties to
+// even) and clamped to [-127, 127] (infinities too); NaN becomes 0.
+__device__ __forceinline__ int8_t quantize_s8(float x, float scale) {
+  float y = __fdiv_rn(x, scale);
+  y = y != y ? 0.f : fminf(fmaxf(y, -127.f), 127.f);
+  return static_cast<int8_t>(__float2int_rn(y));
+}
+
+// Element formats of an 8-bit cache: e4m3 floats, or symmetric int8.
+enum CodeFmt : int { kCodeE4M3 = 1, kCodeS8 = 2 };
+
+// Four int8 codes (low byte first) -> four floats, exact: each byte, biased
+// by 128, becomes the low byte of the fp32 2^23, whose unit is 1, and
+// 2^23 + 128 is subtracted.
+__device__ __forceinline__ void s8x4_to_float(uint32_t w, float (&f)[4]) {
+  const uint32_t u = w ^ 0x80808080u;
+  f[0] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)) - 8388736.f;
+  f[1] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541)) - 8388736.f;
+  f[2] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)) - 8388736.f;
+  f[3] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543)) - 8388736.f;
+}
+
 // 2^x by the hardware approximation (ex2.approx.ftz: relative error ~2^-22,
 // results below 2^-126 flush to 0, 2^-inf = 0). Used for softmax weights.
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -62,15 +62,23 @@ template <>
 struct Elem<__nv_fp8_e4m3> {
   static constexpr int bytes = 1;
 };
+template <>
+struct Elem<int8_t> {
+  static constexpr int bytes = 1;
+};
 
-// Element type of q for a cache of element type T: an fp8 cache is read with
-// bf16 queries.
+// Element type of q for a cache of element type T: an 8-bit cache is read
+// with bf16 queries.
 template <typename T>
 struct QueryOf {
   using type = T;
 };
 template <>
 struct QueryOf<__nv_fp8_e4m3> {
+  using type = __nv_bfloat16;
+};
+template <>
+struct QueryOf<int8_t> {
   using type = __nv_bfloat16;
 };
 

@@ -69,6 +69,25 @@ __device__ __forceinline__ void e4m3x4_f16x2(uint32_t w, uint32_t& lo, uint32_t&
       : "r"(w));
 }
 
+// Four int8 codes (low byte first) -> two f16x2 words, paired as
+// e4m3x4_f16x2 does, exact: each byte, biased by 128, becomes the low byte of
+// the f16 1024 (whose unit is 1), and 1152 is subtracted.
+__device__ __forceinline__ void s8x4_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint32_t l = __byte_perm(u, 0x64646464u, 0x5140), h = __byte_perm(u, 0x64646464u, 0x7362);
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(l), "r"(0x64806480u));
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(h), "r"(0x64806480u));
+}
+
+// Four codes of format CF -> two f16x2 words (bytes 0,1 -> lo; 2,3 -> hi).
+template <int CF>
+__device__ __forceinline__ void widen4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  if constexpr (CF == kCodeS8)
+    s8x4_f16x2(w, lo, hi);
+  else
+    e4m3x4_f16x2(w, lo, hi);
+}
+
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -105,7 +124,7 @@ __device__ __forceinline__ int f8_dim(int j, int n) {
 }
 
 // One consumer warp's 16 tokens (nv valid) of a stage.
-template <int D>
+template <int D, int CF>
 __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, int nv,
                                          const uint32_t (&qa)[D / 16][2], float scale_log2, int lane, int warp,
                                          float& m_run, float& l_run, float (&o)[D / 8][2]) {
@@ -129,7 +148,7 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
       uint32_t w;
       asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w) : "r"(rbase ^ static_cast<uint32_t>(kk << 4)));
       uint32_t b0, b1;
-      e4m3x4_f16x2(w, b0, b1);
+      widen4<CF>(w, b0, b1);
       mma_f16_rows8_chain(sacc[nt], qa[kk][0], qa[kk][1], b0, b1, dead);
     }
   }
@@ -200,10 +219,10 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
   for (int w = 0; w < W; ++w) {
     // (token a byte k, token b byte k) pairs: bytes 0,1 then 2,3 of each word
     uint32_t b[8];
-    e4m3x4_f16x2(__byte_perm(va[w], vb[w], 0x5140), b[0], b[1]);
-    e4m3x4_f16x2(__byte_perm(va[w], vb[w], 0x7362), b[2], b[3]);
-    e4m3x4_f16x2(__byte_perm(vc[w], vd[w], 0x5140), b[4], b[5]);
-    e4m3x4_f16x2(__byte_perm(vc[w], vd[w], 0x7362), b[6], b[7]);
+    widen4<CF>(__byte_perm(va[w], vb[w], 0x5140), b[0], b[1]);
+    widen4<CF>(__byte_perm(va[w], vb[w], 0x7362), b[2], b[3]);
+    widen4<CF>(__byte_perm(vc[w], vd[w], 0x5140), b[4], b[5]);
+    widen4<CF>(__byte_perm(vc[w], vd[w], 0x7362), b[6], b[7]);
     if (ragged) {
       // tokens past the valid ones: their V bytes may be NaN codes
       const uint32_t m0 = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
@@ -223,7 +242,7 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
 // partition-major. Warp 4 streams the item's K/V tiles; warps 0-3 each take
 // 16 tokens of every 64-token stage; the warps' states are merged through
 // shared memory at the end.
-template <int D, int G>
+template <int D, int G, int CF>
 __global__ void __launch_bounds__(F8Cfg<D>::kThreads) decode_f8_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                        const __grid_constant__ CUtensorMap tmv,
                                                                        const DecodeArgs a) {
@@ -301,7 +320,7 @@ __global__ void __launch_bounds__(F8Cfg<D>::kThreads) decode_f8_kernel(const __g
       const int nv = min(16, min(C, pt.ntok - i * C) - warp * 16);  // warp-uniform
       if (nv > 0) {
         const uint8_t* kt = sgen + st * Cfg::kStageBytes;
-        f8_chunk<D>(kt, kt + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
+        f8_chunk<D, CF>(kt, kt + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ps.empty[st]);

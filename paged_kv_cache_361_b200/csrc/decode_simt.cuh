@@ -85,6 +85,19 @@ __device__ __forceinline__ void load16<__nv_fp8_e4m3>(const __nv_fp8_e4m3* p, fl
   }
 }
 
+template <>
+__device__ __forceinline__ void load16<int8_t>(const int8_t* p, float (&f)[8]) {
+  const uint2 x = *reinterpret_cast<const uint2*>(p);
+  float a[4], b[4];
+  s8x4_to_float(x.x, a);
+  s8x4_to_float(x.y, b);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[e] = a[e];
+    f[4 + e] = b[e];
+  }
+}
+
 // Sum NV values over the LPR lanes of a row group; lanes halve the values they
 // carry at each of the first log2(NV) steps. Returns the full sum of value
 // j = (sub >> (log LPR - log NV)) & (NV - 1).

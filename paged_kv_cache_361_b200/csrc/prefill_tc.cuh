@@ -32,11 +32,12 @@
 // maximum grows by more than 8 in log2 units, so weights stay below 2^8 and
 // most chunks never touch O; the result is the same softmax.
 //
-// 8-bit (e4m3) cache (F8). P3 = "PagedAttention 和 vLLM", the section on its
-// future: paged KV storage combined with quantisation, a code c standing for
-// value(c) * scale with one scale per tensor. A kind::f16 MMA takes A and B of
-// one type, so the keys and values are widened to f16 (cvt e4m3x2 -> f16x2,
-// exact) by a fourth role:
+// 8-bit cache (CF: e4m3 or int8 codes). P3 = "PagedAttention 和 vLLM", the
+// section on its future: paged KV storage combined with quantisation, a code c
+// standing for value(c) * scale with one scale per tensor. A kind::f16 MMA
+// takes A and B of one type, so the keys and values are widened to f16 (cvt
+// e4m3x2 -> f16x2, or the int8 byte-permute widening; both exact) by a fourth
+// role:
 //   warps +2..+5  converter: the producer copies [bs x D] byte boxes of codes
 //              (128-byte swizzle at D 128, 64-byte at D 64) into a small
 //              staging ring; the converter writes each chunk as f16 K and V
@@ -92,10 +93,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 // TILES query tiles of one (kv head, sequence) per CTA share the K/V stream;
 // tile t is processed by softmax warpgroup t.
-template <int D, int G, int TILES, bool F8 = false>
-__global__ void __launch_bounds__(TcCfg<D, TILES, F8>::kThreads, 1)
+// CF = 0: bf16 cache; kCodeE4M3 / kCodeS8: an 8-bit cache of that format.
+template <int D, int G, int TILES, int CF = 0>
+__global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                       const PrefillArgs a) {
+  constexpr bool F8 = CF != 0;
   using Cfg = TcCfg<D, TILES, F8>;
   constexpr int S = Cfg::kStages, C = Cfg::kChunk, TT = Cfg::kRows / G;
   constexpr int CS = F8 ? Cfg::kCodeStages : 1;
@@ -235,10 +238,10 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, F8>::kThreads, 1)
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
           if (live) w = *reinterpret_cast<const uint4*>(src + (((d0 >> 4) ^ key) << 4));
           uint32_t h[8];
-          e4m3x4_f16x2(w.x, h[0], h[1]);
-          e4m3x4_f16x2(w.y, h[2], h[3]);
-          e4m3x4_f16x2(w.z, h[4], h[5]);
-          e4m3x4_f16x2(w.w, h[6], h[7]);
+          widen4<CF>(w.x, h[0], h[1]);
+          widen4<CF>(w.y, h[2], h[3]);
+          widen4<CF>(w.z, h[4], h[5]);
+          widen4<CF>(w.w, h[6], h[7]);
           // two 16-byte pieces of the 128-byte row of box column d0 / 64
           uint8_t* rp = dst + (d0 >> 6) * Cfg::kHalfBytes;
           const int cc = (d0 & 63) >> 3;

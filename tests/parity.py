@@ -122,3 +122,65 @@ class Replay:
         """Whole device pool equals the oracle's paged pool (small cases)."""
         for w, pool in (("k", self.cache.k_cache), ("v", self.cache.v_cache)):
             assert torch.equal(bits(pool.cpu()), bits(self.oracle.pool[w]))
+
+
+# 8-bit caches: torch dtype, oracle codec module, integer view of the pool bytes
+def _codecs():
+    from oracle import fp8, int8
+    return {"e4m3": (torch.float8_e4m3fn, fp8, torch.uint8), "int8": (torch.int8, int8, torch.int8)}
+
+
+class CodedReplay(Replay):
+    """Replay with an 8-bit device cache (e4m3 or int8 codes, per-tensor
+    scales); the oracle keeps the bf16 history and quantises it itself."""
+
+    def __init__(self, shape, num_blocks, free_order, scale, partition_tokens=-1, k_scale=4.0 / 448.0,
+                 v_scale=3.0 / 448.0, fmt="e4m3"):
+        assert shape.dtype == "bf16"
+        self.shape, self.scale, self.P = shape, scale, partition_tokens
+        self.ks, self.vs = k_scale, v_scale
+        self.dt, self.codec, self.view = _codecs()[fmt]
+        self.cache = PagedKVCache(num_blocks, shape.num_kv_heads, shape.block_size, shape.head_dim,
+                                  self.dt, "cuda", free_order, fill=float("nan"),
+                                  k_scale=k_scale, v_scale=v_scale)
+        self.oracle = OracleRun(shape, num_blocks, free_order, keep_pool=False)
+        self.device = "cuda"
+        self.decodes = []
+        self.n_pairs = 0
+
+    def codes(self, seq, which):
+        return self.codec.quantize(self.oracle.history(seq, which).float().numpy(),
+                                   self.ks if which == "k" else self.vs)
+
+    def rows(self, seq, which):
+        return self.codec.dequantize(self.codes(seq, which), self.ks if which == "k" else self.vs)
+
+    def check_pool_codes(self):
+        bs = self.shape.block_size
+        for s in self.cache.lens:
+            table, L = self.cache.bm.block_table(s)
+            t = torch.arange(L)
+            blk = torch.as_tensor(table, dtype=torch.int64)[t // bs].cuda()
+            off = (t % bs).cuda()
+            for w, pool in (("k", self.cache.k_cache), ("v", self.cache.v_cache)):
+                got = pool.view(self.view)[blk, :, off, :].cpu().numpy()
+                assert np.array_equal(got, self.codes(s, w)), f"seq {s} {w} codes differ"
+
+    def check_outputs(self, which=-1, tol=TOL["bf16"]):
+        """Outputs are fp32 sums over exactly representable inputs (codes times
+        a scale, bf16 queries), as for a bf16 cache: the bf16 bound applies."""
+        ids, q, out = self.decodes[which]
+        G = self.shape.group
+        worst = 0.0
+        for i, s in enumerate(ids):
+            K, V = self.rows(s, "k"), self.rows(s, "v")
+            ref = np.zeros((self.shape.num_q_heads, self.shape.head_dim))
+            for g in range(self.shape.num_kv_heads):
+                ref[g * G:(g + 1) * G] = decode_attention(q[i][g * G:(g + 1) * G], K[:, g:g + 1], V[:, g:g + 1],
+                                                          self.scale)
+            o = out[i].double().numpy()
+            assert np.isfinite(o).all()
+            err = float(np.abs(o - ref).max())
+            worst = max(worst, err)
+            assert err <= tol, f"seq {s}: max-abs {err:.3e} > {tol}"
+        return worst

@@ -56,6 +56,8 @@ def _cache(**kw):
     (dict(dtype=B.PA_FP8_E4M3, k_scale=1.0, v_scale=float("nan")), B.PA_ERR_INVALID_ARG),
     (dict(dtype=B.PA_FP8_E4M3, k_scale=-1.0, v_scale=1.0), B.PA_ERR_INVALID_ARG),
     (dict(dtype=B.PA_FP8_E4M3, k_scale=float("inf"), v_scale=1.0), B.PA_ERR_INVALID_ARG),
+    (dict(dtype=B.PA_INT8), B.PA_ERR_INVALID_ARG),                                      # scales 0
+    (dict(dtype=B.PA_INT8, k_scale=1.0, v_scale=-2.0), B.PA_ERR_INVALID_ARG),
 ])
 def test_host_checks_before_launch(kw, status):
     lib = B._lib()
@@ -64,15 +66,16 @@ def test_host_checks_before_launch(kw, status):
     assert lib.pa_copy_blocks(ctypes.byref(c), 16, 1, None) == status
 
 
-def test_fp8_cache_needs_its_scales():
+@pytest.mark.parametrize("dt", ["float8_e4m3fn", "int8"])
+def test_8bit_cache_needs_its_scales(dt):
     import torch
-    kc = torch.zeros(4, 1, 16, 64, dtype=torch.float8_e4m3fn)
+    kc = torch.zeros(4, 1, 16, 64, dtype=getattr(torch, dt))
     vc = torch.zeros_like(kc)
     with pytest.raises(ValueError, match="scales"):
         B.make_cache(kc, vc)
     with pytest.raises(TypeError):
-        B.set_fp8_scales(kc.float(), vc.float(), 1.0, 1.0)
-    assert B.input_dtype(torch.float8_e4m3fn) == torch.bfloat16
+        B.set_kv_scales(kc.float(), vc.float(), 1.0, 1.0)
+    assert B.input_dtype(kc.dtype) == torch.bfloat16
     assert B.input_dtype(torch.float32) == torch.float32
 
 

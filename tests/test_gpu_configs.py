@@ -146,9 +146,21 @@ def test_llama2_7b_mha_fp8_cache():
     """The metric workload over an e4m3 cache: every sequence's codes equal the
     oracle's quantisation of its rows bitwise; every output row within the bf16
     bound of the fp64 attention over the dequantised rows."""
-    from tests.test_gpu_fp8 import Fp8Replay
+    from tests.parity import CodedReplay
     w = W.llama2_7b_mha()
-    r = Fp8Replay(w.shape, w.num_blocks, w.free_order, w.scale).run(W.simple_ops(w))
+    r = CodedReplay(w.shape, w.num_blocks, w.free_order, w.scale).run(W.simple_ops(w))
+    r.check_pool_codes()
+    r.check_outputs()
+
+
+def test_llama2_7b_mha_int8_cache():
+    """The metric workload over an int8 cache (scales 4/127, 3/127): codes equal
+    the oracle's quantisation bitwise; every output row within the bf16 bound
+    of the fp64 attention over the dequantised rows."""
+    from tests.parity import CodedReplay
+    w = W.llama2_7b_mha()
+    r = CodedReplay(w.shape, w.num_blocks, w.free_order, w.scale, k_scale=4.0 / 127, v_scale=3.0 / 127,
+                    fmt="int8").run(W.simple_ops(w))
     r.check_pool_codes()
     r.check_outputs()
 

@@ -13,7 +13,7 @@ from oracle.attention import decode_attention
 from oracle.replay import OracleRun
 from paged_kv_cache_361_b200 import PagedKVCache, binding as B
 from paged_kv_cache_361_b200 import workloads as W
-from tests.parity import Replay
+from tests.parity import CodedReplay
 
 pytestmark = pytest.mark.gpu
 
@@ -31,58 +31,6 @@ def _clean_error_word():
     yield
 
 
-class Fp8Replay(Replay):
-    """Replay with an fp8 device cache; the oracle keeps the bf16 history and
-    quantises it itself."""
-
-    def __init__(self, shape, num_blocks, free_order, scale, partition_tokens=-1, k_scale=K_SCALE,
-                 v_scale=V_SCALE):
-        assert shape.dtype == "bf16"
-        self.shape, self.scale, self.P = shape, scale, partition_tokens
-        self.ks, self.vs = k_scale, v_scale
-        self.cache = PagedKVCache(num_blocks, shape.num_kv_heads, shape.block_size, shape.head_dim,
-                                  torch.float8_e4m3fn, "cuda", free_order, fill=float("nan"),
-                                  k_scale=k_scale, v_scale=v_scale)
-        self.oracle = OracleRun(shape, num_blocks, free_order, keep_pool=False)
-        self.device = "cuda"
-        self.decodes = []
-        self.n_pairs = 0
-
-    def codes(self, seq, which):
-        return fp8.quantize(self.oracle.history(seq, which).float().numpy(), self.ks if which == "k" else self.vs)
-
-    def rows(self, seq, which):
-        return fp8.dequantize(self.codes(seq, which), self.ks if which == "k" else self.vs)
-
-    def check_pool_codes(self):
-        bs = self.shape.block_size
-        for s in self.cache.lens:
-            table, L = self.cache.bm.block_table(s)
-            t = torch.arange(L)
-            blk = torch.as_tensor(table, dtype=torch.int64)[t // bs].cuda()
-            off = (t % bs).cuda()
-            for w, pool in (("k", self.cache.k_cache), ("v", self.cache.v_cache)):
-                got = pool.view(torch.uint8)[blk, :, off, :].cpu().numpy()
-                assert np.array_equal(got, self.codes(s, w)), f"seq {s} {w} codes differ"
-
-    def check_outputs(self, which=-1, tol=TOL_FP8):
-        ids, q, out = self.decodes[which]
-        G = self.shape.group
-        worst = 0.0
-        for i, s in enumerate(ids):
-            K, V = self.rows(s, "k"), self.rows(s, "v")
-            ref = np.zeros((self.shape.num_q_heads, self.shape.head_dim))
-            for g in range(self.shape.num_kv_heads):
-                ref[g * G:(g + 1) * G] = decode_attention(q[i][g * G:(g + 1) * G], K[:, g:g + 1], V[:, g:g + 1],
-                                                          self.scale)
-            o = out[i].double().numpy()
-            assert np.isfinite(o).all()
-            err = float(np.abs(o - ref).max())
-            worst = max(worst, err)
-            assert err <= tol, f"seq {s}: max-abs {err:.3e} > {tol}"
-        return worst
-
-
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("bs", [1, 8, 16, 32])
@@ -92,7 +40,7 @@ def test_fp8_fuzz_shapes(D, G, bs):
     seed = zlib.crc32(f"fp8-{D}-{G}-{bs}".encode()) % 100000
     w = W.random_small(seed, num_seqs=6, shape=sh, max_len=int(np.random.default_rng(seed).integers(40, 400)))
     for P in (0, -1, 2 * max(bs, 16)):
-        r = Fp8Replay(sh, w.num_blocks, w.free_order, w.scale, partition_tokens=P).run(W.simple_ops(w))
+        r = CodedReplay(sh, w.num_blocks, w.free_order, w.scale, partition_tokens=P).run(W.simple_ops(w))
         r.check_outputs()
     r.check_pool_codes()
 
@@ -103,7 +51,7 @@ def test_fp8_long_split_and_mha():
     sh = W.Shape(32, 32, 128, 16, "bf16")
     w = W.random_small(21, num_seqs=3, shape=sh, max_len=4096)
     for P in (0, 512, -1):
-        r = Fp8Replay(sh, w.num_blocks, w.free_order, w.scale, partition_tokens=P).run(W.simple_ops(w))
+        r = CodedReplay(sh, w.num_blocks, w.free_order, w.scale, partition_tokens=P).run(W.simple_ops(w))
         r.check_outputs()
     r.check_pool_codes()
 
@@ -121,7 +69,7 @@ def test_fp8_fork_copy_on_write():
         ops.append(("append", [2, 0, 1], lambda which, device="cpu", k=k, v=v: k if which == "k" else v))
     q = torch.randn(3, 8, 128, generator=g).bfloat16()
     ops.append(("decode", [0, 1, 2], lambda device="cpu": q))
-    r = Fp8Replay(sh, 20, list(range(20)), 128 ** -0.5).run(ops)
+    r = CodedReplay(sh, 20, list(range(20)), 128 ** -0.5).run(ops)
     assert r.n_pairs == 2
     r.check_pool_codes()
     r.check_outputs()
@@ -286,7 +234,7 @@ def test_fp8_prefill_long_chunk_many_tiles(G, D):
 def test_fp8_bad_scale_rejected():
     kc = torch.zeros(4, 1, 16, 64, dtype=torch.float8_e4m3fn, device="cuda")
     vc = torch.zeros_like(kc)
-    B.set_fp8_scales(kc, vc, 0.0, 1.0)
+    B.set_kv_scales(kc, vc, 0.0, 1.0)
     rows = torch.zeros(1, 1, 64, dtype=torch.bfloat16, device="cuda")
     slots = torch.zeros(1, dtype=torch.int64, device="cuda")
     with pytest.raises(B.PagedAttnError) as e:
