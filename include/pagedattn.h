@@ -30,8 +30,8 @@
  *   - Query head h reads kv head h / (num_q_heads / num_kv_heads).
  *   - Supported shapes: head_dim 64 or 128; block_size 1, 2, 4, 8, 16 or 32;
  *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; dtype fp32, bf16, or 8-bit
- *     e4m3 / int8 (decode, prefill, append, copies and swaps; the shared-prefix
- *     decode takes bf16 only).
+ *     e4m3 / int8 (every operation; fp32 has no prefill and no shared-prefix
+ *     decode).
  */
 #ifndef PAGEDATTN_H
 #define PAGEDATTN_H
@@ -234,8 +234,9 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
  *   max_prefix_tokens    host bound on group_prefix_tokens.
  *   workspace            >= pa_decode_cascade_workspace_bytes(...).
  * Other arguments as pa_decode (partition size chosen by the library).
- * Supported: bf16 cache, block_size 8..32; other shapes return
- * PA_ERR_UNSUPPORTED.
+ * Supported: bf16, e4m3 or int8 cache, block_size 8..32; other shapes return
+ * PA_ERR_UNSUPPORTED. Over an 8-bit cache the prefix pass widens the codes to
+ * f16 in shared memory and multiplies by f16 weights (as pa_prefill does).
  */
 pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
                             const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,

@@ -540,7 +540,7 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
   if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
   const int G = num_q_heads / cache->num_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
-  if (cache->dtype != PA_BF16 || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
+  if ((cache->dtype != PA_BF16 && !is_8bit(cache->dtype)) || cache->block_size < 8) return PA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size > INT32_MAX)
     return PA_ERR_UNSUPPORTED;
   if (max_group_size > 64 / G) return PA_ERR_INVALID_ARG;  // one 64-row tile per group
@@ -584,6 +584,11 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
     pa.ntiles = 0;
     pa.scale_log2 = scale * 1.4426950408889634f;
     pa.v_scale = 1.f;
+    if (is_8bit(cache->dtype)) {
+      // q . (k_scale * code) = (k_scale * q) . code; the V scale multiplies the partial o.
+      pa.scale_log2 *= cache->k_scale;
+      pa.v_scale = cache->v_scale;
+    }
     pa.group_offs = group_offsets;
     pa.group_members = group_members;
     pa.group_prefix = group_prefix_tokens;
@@ -594,7 +599,8 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
     pa.ws_o = ws_o;
     CUtensorMap tk, tv;
     const uint64_t rows = static_cast<uint64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
-    if (!encode_rows(&tk, cache->k, rows, D, cache->block_size) || !encode_rows(&tv, cache->v, rows, D, cache->block_size))
+    auto enc = is_8bit(cache->dtype) ? encode_rows_u8 : encode_rows;
+    if (!enc(&tk, cache->k, rows, D, cache->block_size) || !enc(&tv, cache->v, rows, D, cache->block_size))
       return PA_ERR_CUDA;
     const dim3 grid(cache->num_kv_heads, pparts, num_groups);
     auto launch = [&](auto kern, int smem) -> pa_status {
@@ -602,17 +608,22 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
       kern<<<grid, MmaCfg<128>::kThreads, smem, s>>>(tk, tv, pa);
       return launched();
     };
-    if (D == 128) {
-      st = G == 1 ? launch(prefill_mma_kernel<128, 1, true>, MmaCfg<128>::kSmemBytes)
-         : G == 2 ? launch(prefill_mma_kernel<128, 2, true>, MmaCfg<128>::kSmemBytes)
-         : G == 4 ? launch(prefill_mma_kernel<128, 4, true>, MmaCfg<128>::kSmemBytes)
-                  : launch(prefill_mma_kernel<128, 8, true>, MmaCfg<128>::kSmemBytes);
-    } else {
-      st = G == 1 ? launch(prefill_mma_kernel<64, 1, true>, MmaCfg<64>::kSmemBytes)
-         : G == 2 ? launch(prefill_mma_kernel<64, 2, true>, MmaCfg<64>::kSmemBytes)
-         : G == 4 ? launch(prefill_mma_kernel<64, 4, true>, MmaCfg<64>::kSmemBytes)
-                  : launch(prefill_mma_kernel<64, 8, true>, MmaCfg<64>::kSmemBytes);
-    }
+    auto launch_cf = [&](auto cf) -> pa_status {
+      constexpr int CF = decltype(cf)::value;
+      constexpr int S128 = prefill_mma_smem_bytes<128, CF>(), S64 = prefill_mma_smem_bytes<64, CF>();
+      if (D == 128)
+        return G == 1 ? launch(prefill_mma_kernel<128, 1, true, CF>, S128)
+             : G == 2 ? launch(prefill_mma_kernel<128, 2, true, CF>, S128)
+             : G == 4 ? launch(prefill_mma_kernel<128, 4, true, CF>, S128)
+                      : launch(prefill_mma_kernel<128, 8, true, CF>, S128);
+      return G == 1 ? launch(prefill_mma_kernel<64, 1, true, CF>, S64)
+           : G == 2 ? launch(prefill_mma_kernel<64, 2, true, CF>, S64)
+           : G == 4 ? launch(prefill_mma_kernel<64, 4, true, CF>, S64)
+                    : launch(prefill_mma_kernel<64, 8, true, CF>, S64);
+    };
+    st = cache->dtype == PA_INT8       ? launch_cf(std::integral_constant<int, kCodeS8>{})
+         : cache->dtype == PA_FP8_E4M3 ? launch_cf(std::integral_constant<int, kCodeE4M3>{})
+                                       : launch_cf(std::integral_constant<int, 0>{});
     if (st != PA_OK) return st;
   }
 
@@ -642,11 +653,19 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
   a.force_partials = 1;
   a.parts_stride = stride;
   a.prefix_part_tokens = kCascadePrefixPart;
+  if (is_8bit(cache->dtype)) {
+    a.scale_log2 *= cache->k_scale;
+    a.v_scale = cache->v_scale;
+  }
   const dim3 grid(cache->num_kv_heads, num_seqs, parts);
   if (mma_eligible(cache, G)) {
     st = dispatch_mma(a, cache, G, s);
-  } else {
+  } else if (f8_mma_eligible(cache)) {
+    st = D == 128 ? dispatch_f8<128>(a, cache, G, grid, s) : dispatch_f8<64>(a, cache, G, grid, s);
+  } else if (cache->dtype == PA_BF16) {
     st = D == 128 ? dispatch_g<__nv_bfloat16, 128>(a, G, grid, s) : dispatch_g<__nv_bfloat16, 64>(a, G, grid, s);
+  } else {
+    return PA_ERR_UNSUPPORTED;  // unreachable: an 8-bit cache here has block_size >= 8
   }
   if (st != PA_OK) return st;
   // 3. merge prefix and suffix partials

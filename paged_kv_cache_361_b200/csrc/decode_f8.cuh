@@ -93,6 +93,39 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// One row of a 64-key chunk of codes, half of its dims, widened to f16. src:
+// the chunk's codes as the TMA stages them ([rows x D] bytes, 128-byte swizzle
+// at D 128, 64-byte at D 64); dst: the 128-byte-swizzled [rows x 64] f16 box
+// columns, kHalfBytes apart, that a bf16 tile has after its TMA copy. live =
+// false writes zeros (rows past the last key: their bytes may be anything).
+template <int D, int CF, int kHalfBytes>
+__device__ __forceinline__ void widen_row_half(const uint8_t* src, uint8_t* dst, int row, int half, bool live) {
+  constexpr int DH = D / 2;  // dims per thread
+  const int key = D == 128 ? (row & 7) : ((row >> 1) & 3);  // swizzle of the staged code row
+  src += row * D;
+  dst += row * 128;
+#pragma unroll
+  for (int u0 = 0; u0 < DH / 16; ++u0) {
+    // at D 128 the two halves of a row would store to the same 16-byte columns
+    // at once (lanes 2r and 2r+1 share a store phase); half 1 takes its
+    // pieces in rotated order, so a phase hits 8 columns
+    const int u = D == 128 && half ? (u0 ^ 2) : u0;
+    const int d0 = half * DH + 16 * u;  // 16 codes -> dims d0 .. d0 + 15
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (live) w = *reinterpret_cast<const uint4*>(src + (((d0 >> 4) ^ key) << 4));
+    uint32_t h[8];
+    widen4<CF>(w.x, h[0], h[1]);
+    widen4<CF>(w.y, h[2], h[3]);
+    widen4<CF>(w.z, h[4], h[5]);
+    widen4<CF>(w.w, h[6], h[7]);
+    // two 16-byte pieces of the 128-byte row of box column d0 / 64
+    uint8_t* rp = dst + (d0 >> 6) * kHalfBytes;
+    const int cc = (d0 & 63) >> 3;
+    *reinterpret_cast<uint4*>(rp + ((cc ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(rp + (((cc + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+  }
+}
+
 // m16n8k16 f16 MMA with rows 8..15 of A zero and their results discarded
 // (as mma_rows8).
 __device__ __forceinline__ void mma_f16_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {

@@ -17,8 +17,17 @@
 // with P split into a bf16 high part and remainder. The causal mask is applied
 // per row; a warp skips chunks that lie entirely past its rows' positions.
 // Tiles are dispatched last-first (the longest key ranges start first).
+//
+// 8-bit cache (CF = kCodeE4M3 or kCodeS8; cascade mode only): the producer
+// copies [bs x D] byte boxes of codes into a staging slot of the stage; the
+// four consumer warps widen the chunk to f16 tiles in the stage (thread = row,
+// half of its dims; rows past the last key as zeros), meet on an mbarrier, and
+// run the same MMAs in f16 (q rounded to f16, P as one f16 operand; P3 "PagedAttention
+// 和 vLLM", the section on its future: a code c stands for value(c) * scale).
+// The K scale is folded into the score scale, the V scale into the partials.
 #pragma once
 
+#include "decode_f8.cuh"
 #include "decode_mma.cuh"
 
 namespace pa {
@@ -54,20 +63,43 @@ __device__ __forceinline__ void mma16(float (&d)[4], uint32_t a0, uint32_t a1, u
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// d += A(16x16) * B(16x8), f16 operands, all 16 rows live.
+__device__ __forceinline__ void mma16_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Shared memory of prefill_mma_kernel: the stage ring, plus per stage a
+// staging slot of K and V codes for an 8-bit cache.
+template <int D, int CF>
+constexpr int prefill_mma_smem_bytes() {
+  return MmaCfg<D>::kSmemBytes + (CF != 0 ? MmaCfg<D>::kStages * 2 * MmaCfg<D>::kChunk * D : 0);
+}
+
 // CASCADE = false: prefill (rows = new tokens x heads, causal).
 // CASCADE = true: shared-prefix decode (rows = group members x heads, every
 // row sees the whole prefix partition; partial results, not rows, are stored).
-template <int D, int G, bool CASCADE>
+template <int D, int G, bool CASCADE, int CF = 0>
 __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                          const __grid_constant__ CUtensorMap tmv,
                                                                          const PrefillArgs a) {
   using Cfg = MmaCfg<D>;
   constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = D / 8;
   constexpr int TT = 64 / G;  // tokens per tile
+  static_assert(CF == 0 || CASCADE, "8-bit codes in cascade mode only (every warp visits every chunk)");
+  static_assert(NW * 32 == 2 * C, "one (row, half) of the chunk per consumer thread");
+  constexpr int kCodeTileBytes = C * D, kCodeStageBytes = 2 * kCodeTileBytes;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ PipeSmem<S> ps;
+  __shared__ uint64_t conv_bar[CF != 0 ? S : 1];  // 8-bit: the consumer warps have widened stage st
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t cs0 = sbase + S * Cfg::kStageBytes;  // 8-bit: code staging slots
 
   const int g = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -104,9 +136,38 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
   }
   const int nchunks = (kend - k_begin + C - 1) / C;
 
-  if (tid == 0) pipe_init<S>(ps, NW);
+  if (tid == 0) {
+    if constexpr (CF != 0)
+      for (int i = 0; i < S; ++i) mbar_init(&conv_bar[i], NW);
+    pipe_init<S>(ps, NW);
+  }
   __syncthreads();
 
+  if (CF != 0 && warp == NW) {
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
+    const uint64_t pol = l2_evict_last_policy();
+    pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+      const int32_t c0 = k_begin + i * C;
+      const int32_t nb = (min(C, kend - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+      int32_t blk = -1;
+      bool ok = false;
+      if (lane < nb) {
+        blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
+        ok = blk >= 0 && blk < a.num_blocks;
+        if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * __popc(okmask) * box_bytes);
+      __syncwarp();
+      if (ok) {
+        const int32_t y = (blk * a.hkv + g) * a.bs;
+        const uint32_t dst = cs0 + st * kCodeStageBytes + lane * box_bytes;
+        tma_load_2d(dst, &tmk, 0, y, &ps.full[st], pol);
+        tma_load_2d(dst + kCodeTileBytes, &tmv, 0, y, &ps.full[st], pol);
+      }
+    });
+    return;
+  }
   if (warp == NW) {
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
@@ -172,6 +233,9 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
     qa[kk][1] = vb ? __ldg(qrb + kk * 8 + c) : 0u;
     qa[kk][2] = va ? __ldg(qra + kk * 8 + 4 + c) : 0u;
     qa[kk][3] = vb ? __ldg(qrb + kk * 8 + 4 + c) : 0u;
+    if constexpr (CF != 0)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qa[kk][e] = pack_f16(bf16lo(qa[kk][e]), bf16hi(qa[kk][e]));
   }
   float o[NT][4];
 #pragma unroll
@@ -183,6 +247,18 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
     const int st = i % S;
     if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
     const int k0 = k_begin + i * C;
+    if constexpr (CF != 0) {
+      // widen the chunk into the stage's f16 tiles; every warp reads all of it
+      const int row = tid >> 1, half = tid & 1;
+      const uint8_t* src = sgen + (cs0 - sbase) + st * kCodeStageBytes;
+      uint8_t* dst = sgen + st * Cfg::kStageBytes;
+      widen_row_half<D, CF, Cfg::kHalfBytes>(src, dst, row, half, k0 + row < kend);
+      widen_row_half<D, CF, Cfg::kHalfBytes>(src + kCodeTileBytes, dst + Cfg::kTileBytes, row, half,
+                                             k0 + row < kend);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&conv_bar[st]);
+      if (!pipe_wait(&conv_bar[st], (i / S) & 1, &ps.abort_flag)) break;
+    }
     if (k0 <= wmax) {
       const uint32_t kst = sbase + st * Cfg::kStageBytes;
       const uint32_t vst = kst + Cfg::kTileBytes;
@@ -198,8 +274,13 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
           const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tk * 128 + ((((d0 & 63) >> 3) ^ (tk & 7)) << 4);
           uint32_t b00, b01, b10, b11;
           ldsm_x4(addr, b00, b01, b10, b11);
-          mma16(sacc[2 * kg], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b00, b01);
-          mma16(sacc[2 * kg + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b10, b11);
+          if constexpr (CF != 0) {
+            mma16_f16(sacc[2 * kg], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b00, b01);
+            mma16_f16(sacc[2 * kg + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b10, b11);
+          } else {
+            mma16(sacc[2 * kg], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b00, b01);
+            mma16(sacc[2 * kg + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b10, b11);
+          }
         }
       }
       // causal mask and online softmax for rows ra (c0, c1) and rb (c2, c3)
@@ -248,10 +329,18 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg) {
         uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
-        split_pair(sacc[2 * kg][0], sacc[2 * kg][1], h0, l0);          // row ra, keys 2c, 2c+1
-        split_pair(sacc[2 * kg][2], sacc[2 * kg][3], h1, l1);          // row rb
-        split_pair(sacc[2 * kg + 1][0], sacc[2 * kg + 1][1], h2, l2);  // row ra, keys +8
-        split_pair(sacc[2 * kg + 1][2], sacc[2 * kg + 1][3], h3, l3);  // row rb, keys +8
+        if constexpr (CF != 0) {  // weights <= 1 as f16, one MMA
+          h0 = pack_f16(sacc[2 * kg][0], sacc[2 * kg][1]);
+          h1 = pack_f16(sacc[2 * kg][2], sacc[2 * kg][3]);
+          h2 = pack_f16(sacc[2 * kg + 1][0], sacc[2 * kg + 1][1]);
+          h3 = pack_f16(sacc[2 * kg + 1][2], sacc[2 * kg + 1][3]);
+          l0 = l1 = l2 = l3 = 0u;
+        } else {
+          split_pair(sacc[2 * kg][0], sacc[2 * kg][1], h0, l0);          // row ra, keys 2c, 2c+1
+          split_pair(sacc[2 * kg][2], sacc[2 * kg][3], h1, l1);          // row rb
+          split_pair(sacc[2 * kg + 1][0], sacc[2 * kg + 1][1], h2, l2);  // row ra, keys +8
+          split_pair(sacc[2 * kg + 1][2], sacc[2 * kg + 1][3], h3, l3);  // row rb, keys +8
+        }
         const int kb = kg * 16;
         uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
         if (kb + 16 > nvk) {
@@ -269,10 +358,15 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
           v1 &= mhi;
           v2 &= mlo;
           v3 &= mhi;
-          mma16(o[2 * dg], h0, h1, h2, h3, v0, v1);
-          mma16(o[2 * dg], l0, l1, l2, l3, v0, v1);
-          mma16(o[2 * dg + 1], h0, h1, h2, h3, v2, v3);
-          mma16(o[2 * dg + 1], l0, l1, l2, l3, v2, v3);
+          if constexpr (CF != 0) {
+            mma16_f16(o[2 * dg], h0, h1, h2, h3, v0, v1);
+            mma16_f16(o[2 * dg + 1], h0, h1, h2, h3, v2, v3);
+          } else {
+            mma16(o[2 * dg], h0, h1, h2, h3, v0, v1);
+            mma16(o[2 * dg], l0, l1, l2, l3, v0, v1);
+            mma16(o[2 * dg + 1], h0, h1, h2, h3, v2, v3);
+            mma16(o[2 * dg + 1], l0, l1, l2, l3, v2, v3);
+          }
         }
       }
     }
@@ -286,20 +380,24 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
   lb += __shfl_xor_sync(0xffffffffu, lb, 1);
   lb += __shfl_xor_sync(0xffffffffu, lb, 2);
   if (CASCADE) {
-    // partials of prefix partition blockIdx.y: unnormalised o, (m, l)
+    // partials of prefix partition blockIdx.y: unnormalised o (times the V
+    // scale of an 8-bit cache, 1 otherwise), (m, l)
     const int slot = a.max_parts + static_cast<int>(blockIdx.y);
+    const float vs = a.v_scale;
     if (va) {
       const int64_t prow = qrow_a * a.parts_stride + slot;
       float* dst = a.ws_o + prow * D + 2 * c;
 #pragma unroll
-      for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
+      for (int j = 0; j < NT; ++j)
+        *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0] * vs, o[j][1] * vs);
       if (c == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(ma, la);
     }
     if (vb) {
       const int64_t prow = qrow_b * a.parts_stride + slot;
       float* dst = a.ws_o + prow * D + 2 * c;
 #pragma unroll
-      for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][2], o[j][3]);
+      for (int j = 0; j < NT; ++j)
+        *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][2] * vs, o[j][3] * vs);
       if (c == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(mb, lb);
     }
     return;

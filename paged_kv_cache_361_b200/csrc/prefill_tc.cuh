@@ -219,36 +219,17 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
     // ---- converter (F8): thread = (row of the chunk, half of its dims) ----
     const int ct = tid - 32 * Cfg::kConvWarp0;
     const int row = ct >> 1, half = ct & 1;
-    const int key = D == 128 ? (row & 7) : ((row >> 1) & 3);  // swizzle of the staged code row
-    constexpr int DH = D / 2;
     const uint8_t* cs0g = sgen + (cs0 - sbase);
     uint8_t* kv0g = sgen + Cfg::kQBytes;
     for (int i = 0; i < nchunks; ++i) {
       const int cst = i % CS, st = i % S;
       if (!warp_wait(&cfull[cst], (i / CS) & 1, &ps.abort_flag)) break;
       if (i >= S && !warp_wait(&ps.empty[st], ((i / S) - 1) & 1, &ps.abort_flag)) break;
-      const bool live = i * C + row < kend_all;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint8_t* src = cs0g + cst * Cfg::kCodeStageBytes + which * Cfg::kCodeTileBytes + row * D;
-        uint8_t* dst = kv0g + st * Cfg::kStageBytes + which * Cfg::kTileBytes + row * 128;
-#pragma unroll
-        for (int u = 0; u < DH / 16; ++u) {
-          const int d0 = half * DH + 16 * u;  // 16 codes -> dims d0 .. d0 + 15
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (live) w = *reinterpret_cast<const uint4*>(src + (((d0 >> 4) ^ key) << 4));
-          uint32_t h[8];
-          widen4<CF>(w.x, h[0], h[1]);
-          widen4<CF>(w.y, h[2], h[3]);
-          widen4<CF>(w.z, h[4], h[5]);
-          widen4<CF>(w.w, h[6], h[7]);
-          // two 16-byte pieces of the 128-byte row of box column d0 / 64
-          uint8_t* rp = dst + (d0 >> 6) * Cfg::kHalfBytes;
-          const int cc = (d0 & 63) >> 3;
-          *reinterpret_cast<uint4*>(rp + ((cc ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(rp + (((cc + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
-        }
-      }
+      const bool live = i * C + row < kend_all;  // rows past the last key become zeros
+      const uint8_t* src = cs0g + cst * Cfg::kCodeStageBytes;
+      uint8_t* dst = kv0g + st * Cfg::kStageBytes;
+      widen_row_half<D, CF, Cfg::kHalfBytes>(src, dst, row, half, live);
+      widen_row_half<D, CF, Cfg::kHalfBytes>(src + Cfg::kCodeTileBytes, dst + Cfg::kTileBytes, row, half, live);
       tc::fence_proxy_async();  // generic-proxy writes -> tensor-core reads
       __syncwarp();
       if (lane == 0) {

@@ -142,6 +142,55 @@ def test_cascade_random_groups(G):
     assert float((a - b).abs().max()) <= 2e-3
 
 
+@pytest.mark.parametrize("fmt,G,D", [("e4m3", 1, 128), ("e4m3", 8, 128), ("int8", 4, 128), ("int8", 2, 64),
+                                       ("e4m3", 4, 64), ("int8", 8, 128)])
+def test_cascade_8bit_cache(fmt, G, D):
+    """Shared-prefix decode over an 8-bit cache: forked families with private
+    suffixes and lone sequences; equal to pa_decode on the same cache, and to
+    the oracle's attention over the dequantised rows on sampled sequences."""
+    from oracle import fp8, int8
+    from oracle.attention import decode_attention
+    from paged_kv_cache_361_b200 import PagedKVCache
+    codec, dt, ks, vs = ((fp8, torch.float8_e4m3fn, 4.0 / 448, 3.0 / 448) if fmt == "e4m3"
+                         else (int8, torch.int8, 4.0 / 127, 3.0 / 127))
+    rng = np.random.default_rng(100 + G + D)
+    hkv, bs = 2, 16
+    cache = PagedKVCache(3000, hkv, bs, D, dt, "cuda", rng.permutation(3000), fill=float("nan"), k_scale=ks,
+                         v_scale=vs)
+    g = torch.Generator().manual_seed(G + D)
+    ids, hist = [], {}
+    for fam in range(4):
+        root = fam * 100
+        n0 = int(rng.integers(64, 700))
+        k0, v0 = torch.randn(n0, hkv, D, generator=g).bfloat16(), torch.randn(n0, hkv, D, generator=g).bfloat16()
+        cache.add_sequence(root, k0.cuda(), v0.cuda())
+        ids.append(root)
+        hist[root] = ([k0], [v0])
+        for j in range(1, int(rng.integers(1, 64 // G + 2))):
+            cache.fork(root, root + j)
+            ids.append(root + j)
+            hist[root + j] = ([k0], [v0])
+    for _ in range(int(rng.integers(1, 30))):       # private suffixes
+        k = torch.randn(len(ids), hkv, D, generator=g).bfloat16()
+        v = torch.randn(len(ids), hkv, D, generator=g).bfloat16()
+        cache.append(ids, k.cuda(), v.cuda())
+        for i, s in enumerate(ids):
+            hist[s] = (hist[s][0] + [k[i:i + 1]], hist[s][1] + [v[i:i + 1]])
+    q = torch.randn(len(ids), hkv * G, D, generator=g).bfloat16()
+    a = cache.decode(ids, q.cuda(), D ** -0.5).cpu()
+    b = cache.decode_cascade(ids, q.cuda(), D ** -0.5).cpu()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    tables, lens, _ = cache.decode_inputs(ids)
+    assert len(cache.shared_prefix_groups(ids, tables, lens, 64 // G)[2]) > 0   # some prefix is shared
+    assert float((a - b).abs().max()) <= 2e-3
+    for i in (0, len(ids) // 2, len(ids) - 1):
+        s = ids[i]
+        K = codec.dequantize(codec.quantize(torch.cat(hist[s][0]).float().numpy(), ks), ks)
+        V = codec.dequantize(codec.quantize(torch.cat(hist[s][1]).float().numpy(), vs), vs)
+        ref = decode_attention(q[i], K, V, D ** -0.5)
+        assert float(np.abs(b[i].double().numpy() - ref).max()) <= 4e-3
+
+
 def test_llama2_7b_mha_fp8_cache():
     """The metric workload over an e4m3 cache: every sequence's codes equal the
     oracle's quantisation of its rows bitwise; every output row within the bf16

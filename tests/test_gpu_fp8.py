@@ -150,18 +150,6 @@ def test_fp8_step_host_matches_oracle():
     assert B.pa_get_device_error()[0] == B.PA_OK
 
 
-def test_fp8_unsupported_paths_say_so():
-    """The shared-prefix decode has no e4m3 path: it says so instead of reading codes as bf16."""
-    cache = PagedKVCache(8, 2, 16, 128, torch.float8_e4m3fn, "cuda", fill=0.0, k_scale=1.0, v_scale=1.0)
-    k = torch.randn(80, 2, 128, device="cuda").bfloat16()
-    cache.add_sequence(0, k, k)
-    cache.fork(0, 1)
-    q = torch.randn(2, 8, 128, device="cuda").bfloat16()
-    with pytest.raises(B.PagedAttnError) as e:
-        cache.decode_cascade([0, 1], q, 0.1)
-    assert e.value.status == B.PA_ERR_UNSUPPORTED
-
-
 def _dq(x, scale):
     """The oracle's view of bf16 rows stored in an e4m3 cache: dequantised codes (fp64)."""
     return fp8.dequantize(fp8.quantize(x.float().numpy(), scale), scale)
