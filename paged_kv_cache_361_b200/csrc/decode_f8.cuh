@@ -1,4 +1,7 @@
-// Paged decode attention over an 8-bit (e4m3) KV cache, on the tensor cores.
+// Paged decode attention over an 8-bit (e4m3 or int8) KV cache, on the tensor
+// cores. The two formats differ only in the widening of four codes to two
+// f16x2 words (widen4<CF>): conversion instructions for e4m3, byte permutes
+// and one f16x2 subtraction for int8; the text below says e4m3 for both.
 //
 // P2 = "PagedAttention：操作系统级 KV 缓存虚拟内存管理".
 //   §1.1  out = softmax(scale * q K^T) V.
