@@ -14,7 +14,8 @@
 // a kv head read every K/V tile once. Six warps:
 //   warp 4     TMA producer: swizzled [bs x 64] boxes of K and V, 64 keys per
 //              stage (the ring and its full/empty barriers of the decode path).
-//   warp 5     allocates TMEM; one lane issues every MMA:
+//   warp 5     allocates TMEM and walks the MMA schedule; one lane chosen
+//              by elect.sync issues every MMA:
 //                S_j = Q K_j^T        (M 128, N 64, K = D; A and B in shared
 //                                      memory, K-major) into TMEM buffer j % 2
 //                O  += P_j V_j        (M 128, N = D, K 64; A = P from TMEM,
@@ -266,8 +267,9 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       }
     });
   } else if (warp == Cfg::kMmaWarp) {
-    // ---- MMA issuer: S_t(j+1) for every tile, then O_t += P_t(j) V(j) ----
-    if (lane == 0) {
+    // ---- MMA issuer: S_t(j+1) for every tile, then O_t += P_t(j) V(j); the
+    // whole warp walks the schedule and waits, one elected lane issues ----
+    {
       constexpr uint32_t kIdS = F8 ? tc::idesc_f16(Cfg::kRows, C, false) : tc::idesc_bf16(Cfg::kRows, C, false);
       constexpr uint32_t kIdPV = F8 ? tc::idesc_f16(Cfg::kRows, D, true) : tc::idesc_bf16(Cfg::kRows, D, true);
       // Descriptors are built once; an operand at a byte offset from a base
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       };
       auto issue_pv = [&](int t, int j) -> bool {
         const int sb = j & 1;
-        if (!pipe_wait(&p_full[t][sb], (j >> 1) & 1, &ps.abort_flag)) return false;
+        if (!warp_wait(&p_full[t][sb], (j >> 1) & 1, &ps.abort_flag)) return false;
         tc::fence_after();
         // V is N-major: 8-key groups 1024 B apart, the two 64-column halves
         // kHalfBytes apart (one half when D = 64: the offset is then unused)
@@ -308,7 +310,8 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         tc::commit(smem_u32(&o_bar[t]));
         return true;
       };
-      bool ok = pipe_wait(&q_full, 0, &ps.abort_flag) && pipe_wait(&ps.full[0], 0, &ps.abort_flag);
+      bool ok = warp_wait(&q_full, 0, &ps.abort_flag);
+      ok = ok && warp_wait(&ps.full[0], 0, &ps.abort_flag);
       tc::fence_after();
       if (ok) {
 #pragma unroll
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       }
       for (int j = 0; ok && j < nchunks; ++j) {
         if (j + 1 < nchunks) {
-          if (!pipe_wait(&ps.full[(j + 1) % S], ((j + 1) / S) & 1, &ps.abort_flag)) {
+          if (!warp_wait(&ps.full[(j + 1) % S], ((j + 1) / S) & 1, &ps.abort_flag)) {
             ok = false;
             break;
           }
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
           if (ok && j < nch[t]) ok = issue_pv(t, j);
         if (ok) tc::commit(smem_u32(&ps.empty[j % S]));  // every tile is done with stage j
       }
-      // every MMA this thread issued has finished before TMEM is released
+      // every MMA the warp issued has finished before TMEM is released
       tc::commit(smem_u32(&drain));
       mbar_wait(&drain, 0);
     }
