@@ -79,6 +79,20 @@ def test_8bit_cache_needs_its_scales(dt):
     assert B.input_dtype(torch.float32) == torch.float32
 
 
+def test_8bit_scales_need_matching_caches():
+    """K and V of one 8-bit cache share a format: mixed e4m3 / int8 pools or a
+    16-bit pool are refused before anything reaches the library."""
+    import torch
+    k8 = torch.zeros(4, 1, 16, 64, dtype=torch.int8)
+    kf = torch.zeros(4, 1, 16, 64, dtype=torch.float8_e4m3fn)
+    with pytest.raises(TypeError):
+        B.set_kv_scales(k8, kf, 1.0, 1.0)
+    with pytest.raises(TypeError):
+        B.set_kv_scales(k8.bfloat16(), k8.bfloat16(), 1.0, 1.0)
+    with pytest.raises(ValueError, match="match"):
+        B.make_cache(k8, kf)
+
+
 def test_decode_argument_checks():
     lib = B._lib()
     c = _cache()
