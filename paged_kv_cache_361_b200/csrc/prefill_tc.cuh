@@ -66,7 +66,7 @@ struct TcCfg {
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage (16-bit elements)
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = F8 && TILES > 1 ? 3 : 4;
-  static constexpr int kCodeTileBytes = kChunk * D;        // e4m3 K (or V) of one staging slot
+  static constexpr int kCodeTileBytes = kChunk * D;        // 8-bit K (or V) codes of one staging slot
   static constexpr int kCodeStageBytes = 2 * kCodeTileBytes;
   static constexpr int kCodeStages = F8 ? (TILES > 1 ? 2 : 3) : 0;
   static constexpr int kQHalfBytes = kRows * 128;
