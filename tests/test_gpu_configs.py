@@ -142,9 +142,11 @@ def test_cascade_random_groups(G):
     assert float((a - b).abs().max()) <= 2e-3
 
 
-@pytest.mark.parametrize("fmt,G,D", [("e4m3", 1, 128), ("e4m3", 8, 128), ("int8", 4, 128), ("int8", 2, 64),
-                                       ("e4m3", 4, 64), ("int8", 8, 128)])
-def test_cascade_8bit_cache(fmt, G, D):
+@pytest.mark.parametrize("fmt,G,D,bs", [("e4m3", 1, 128, 16), ("e4m3", 8, 128, 16), ("int8", 4, 128, 16),
+                                          ("int8", 2, 64, 16), ("e4m3", 4, 64, 16), ("int8", 8, 128, 16),
+                                          ("e4m3", 2, 128, 8), ("int8", 1, 64, 8), ("int8", 4, 128, 32),
+                                          ("e4m3", 8, 64, 32)])
+def test_cascade_8bit_cache(fmt, G, D, bs):
     """Shared-prefix decode over an 8-bit cache: forked families with private
     suffixes and lone sequences; equal to pa_decode on the same cache, and to
     the oracle's attention over the dequantised rows on sampled sequences."""
@@ -153,8 +155,8 @@ def test_cascade_8bit_cache(fmt, G, D):
     from paged_kv_cache_361_b200 import PagedKVCache
     codec, dt, ks, vs = ((fp8, torch.float8_e4m3fn, 4.0 / 448, 3.0 / 448) if fmt == "e4m3"
                          else (int8, torch.int8, 4.0 / 127, 3.0 / 127))
-    rng = np.random.default_rng(100 + G + D)
-    hkv, bs = 2, 16
+    rng = np.random.default_rng(100 + G + D + bs)
+    hkv = 2
     cache = PagedKVCache(3000, hkv, bs, D, dt, "cuda", rng.permutation(3000), fill=float("nan"), k_scale=ks,
                          v_scale=vs)
     g = torch.Generator().manual_seed(G + D)
