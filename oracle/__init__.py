@@ -28,6 +28,12 @@ Modules and what pins each one (tests/test_oracle_*.py):
                  function; a key built to score ln 3 higher weights 3:1), the
                  head-to-group map, shift invariance, and a 50-digit mpmath
                  brute force on tiny inputs.
+  prefix_groups  which batch sequences share leading physical blocks and how
+                 many tokens of them (the host side of the shared-prefix
+                 decode). Pinned by hand-worked cases (forks of one prompt,
+                 a copy-on-write split inside the prefix, lone sequences,
+                 group-size cuts, the alignment cut) in
+                 tests/test_oracle_prefix_groups.py.
   replay         replays an operation script (paged_kv_cache_361_b200.workloads)
                  on the oracle's block manager and a contiguous per-sequence
                  history (the "traditional" layout of P1 and P2 §1.2).

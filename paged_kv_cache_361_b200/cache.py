@@ -207,37 +207,14 @@ class PagedKVCache:
                      self._lens.upload(lens), scale, out, max(counts, default=0), max_len)
         return out
 
-    def shared_prefix_groups(self, seq_ids, tables: np.ndarray, lens: np.ndarray, group_rows: int):
-        """Host side of the shared-prefix decode: sequences of the batch whose
-        tables start with the same physical blocks form a group (at most
-        group_rows members each); its prefix is the longest run of whole blocks
-        common to all members, cut to a multiple of 64 tokens. Returns
-        (offsets, members, prefix_tokens, seq_prefix_tokens) as numpy arrays."""
-        bs = self.block_size
-        by_first = {}
-        for i in range(len(seq_ids)):
-            if lens[i] >= bs:
-                by_first.setdefault(int(tables[i, 0]), []).append(i)
-        offsets, members, prefix = [0], [], []
-        seq_prefix = np.zeros(len(seq_ids), dtype=np.int32)
-        for rows in by_first.values():
-            for c0 in range(0, len(rows), group_rows):
-                grp = rows[c0:c0 + group_rows]
-                if len(grp) < 2:
-                    continue
-                full = int(min(lens[i] for i in grp)) // bs
-                t = tables[grp, :full]
-                same = np.all(t == t[0], axis=0)
-                k = full if same.all() else int(np.argmin(same))
-                ptok = (k * bs) // 64 * 64
-                if ptok == 0:
-                    continue
-                members += grp
-                offsets.append(len(members))
-                prefix.append(ptok)
-                seq_prefix[grp] = ptok
-        return (np.asarray(offsets, np.int32), np.asarray(members, np.int32), np.asarray(prefix, np.int32),
-                seq_prefix)
+    def shared_prefix_groups(self, seq_ids, group_rows: int):
+        """Host side of the shared-prefix decode, from the C++ block manager
+        (pa_bm_prefix_groups): sequences of the batch whose tables start with
+        the same physical blocks form a group (at most group_rows members
+        each); its prefix is the longest run of whole blocks common to all
+        members, cut to a multiple of 64 tokens. Returns (offsets, members,
+        prefix_tokens, seq_prefix_tokens, max_prefix)."""
+        return self.bm.prefix_groups(seq_ids, group_rows, 64)
 
     def decode_cascade(self, seq_ids, q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None):
         """decode() with shared prefixes (forks, prefix-cache hits) read once per
@@ -247,10 +224,9 @@ class PagedKVCache:
             scale = 1.0 / math.sqrt(d)
         tables, lens, max_len = self.decode_inputs(seq_ids)
         hkv = self.k_cache.shape[1]
-        offs, members, prefix, seq_prefix = self.shared_prefix_groups(seq_ids, tables, lens, 64 // (hq // hkv))
+        offs, members, prefix, seq_prefix, max_pre = self.shared_prefix_groups(seq_ids, 64 // (hq // hkv))
         if out is None:
             out = torch.empty((n, hq, d), dtype=torch.float32, device=self.device)
-        max_pre = int(prefix.max()) if len(prefix) else 0
         nbytes = B.pa_decode_cascade_workspace_bytes(n, hq, hkv, d, max_len, self.block_size, max_pre)
         ws = self.workspace(nbytes)
         empty = torch.empty(0, dtype=torch.int32, device=self.device)

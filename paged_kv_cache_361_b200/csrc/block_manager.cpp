@@ -20,6 +20,7 @@
 // The free list is a FIFO ring over a fixed array (front = next allocation,
 // back = most recently freed); evictable blocks sit on an intrusive LRU list;
 // every operation is O(blocks touched).
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -572,6 +573,75 @@ pa_status pa_bm_block_tables(const pa_bm* bm, int32_t n, const int64_t* seq_ids,
     for (int32_t j = m; j < cap; ++j) row[j] = pad;
     lens_out[i] = static_cast<int32_t>(s->len);
   }
+  return PA_OK;
+}
+
+// Shared-prefix groups of a decode batch (P2 §3.4: sequences that share a
+// prefix hold the same physical blocks; P1 "跨请求的内存共享": the samples of
+// one prompt). Sequences are keyed by the physical id of their first block
+// (only those with at least one whole block take part), keys in order of first
+// appearance in the batch; each key's sequences, in batch order, are cut into
+// groups of at most max_group_size. A group's prefix is the longest run of
+// leading table entries that every member holds identically, counted over the
+// whole blocks of its shortest member and cut down to a multiple of
+// align_tokens; a group of one member, or with a prefix of zero tokens, is
+// dropped and its sequences get no prefix.
+pa_status pa_bm_prefix_groups(const pa_bm* bm, int32_t n, const int64_t* seq_ids, int32_t max_group_size,
+                              int32_t align_tokens, int32_t* group_offsets, int32_t* group_members,
+                              int32_t* group_prefix_tokens, int32_t* seq_prefix_tokens, int32_t* n_groups_out,
+                              int32_t* max_prefix_out) {
+  if (!bm || n < 0 || max_group_size < 1 || align_tokens < 1 || !group_offsets || !n_groups_out ||
+      (n > 0 && (!seq_ids || !group_members || !group_prefix_tokens || !seq_prefix_tokens)))
+    return PA_ERR_INVALID_ARG;
+  const int32_t bs = bm->m.block_size();
+  std::vector<const Seq*> seqs(n);
+  for (int32_t i = 0; i < n; ++i) {
+    seqs[i] = bm->m.find(seq_ids[i]);
+    if (!seqs[i]) return PA_ERR_UNKNOWN_SEQ;
+  }
+  std::unordered_map<int32_t, std::vector<int32_t>> by_first;
+  std::vector<int32_t> keys;
+  for (int32_t i = 0; i < n; ++i) {
+    if (seqs[i]->len < bs) continue;
+    auto it = by_first.find(seqs[i]->table[0]);
+    if (it == by_first.end()) {
+      keys.push_back(seqs[i]->table[0]);
+      by_first.emplace(seqs[i]->table[0], std::vector<int32_t>{i});
+    } else {
+      it->second.push_back(i);
+    }
+  }
+  int32_t ng = 0, nm = 0, maxp = 0;
+  group_offsets[0] = 0;
+  for (int32_t i = 0; i < n; ++i) seq_prefix_tokens[i] = 0;
+  for (int32_t key : keys) {
+    const std::vector<int32_t>& rows = by_first[key];
+    for (size_t c0 = 0; c0 < rows.size(); c0 += max_group_size) {
+      const size_t c1 = std::min(rows.size(), c0 + static_cast<size_t>(max_group_size));
+      if (c1 - c0 < 2) continue;
+      int64_t full = INT64_MAX;
+      for (size_t u = c0; u < c1; ++u) full = std::min(full, seqs[rows[u]]->len / bs);
+      const std::vector<int32_t>& t0 = seqs[rows[c0]]->table;
+      int64_t k = 0;
+      for (; k < full; ++k) {
+        bool same = true;
+        for (size_t u = c0 + 1; u < c1 && same; ++u) same = seqs[rows[u]]->table[k] == t0[k];
+        if (!same) break;
+      }
+      const int64_t ptok = k * bs / align_tokens * align_tokens;
+      if (ptok == 0) continue;
+      if (ptok > INT32_MAX) return PA_ERR_UNSUPPORTED;
+      for (size_t u = c0; u < c1; ++u) {
+        group_members[nm++] = rows[u];
+        seq_prefix_tokens[rows[u]] = static_cast<int32_t>(ptok);
+      }
+      group_prefix_tokens[ng] = static_cast<int32_t>(ptok);
+      group_offsets[++ng] = nm;
+      maxp = std::max(maxp, static_cast<int32_t>(ptok));
+    }
+  }
+  *n_groups_out = ng;
+  if (max_prefix_out) *max_prefix_out = maxp;
   return PA_OK;
 }
 

@@ -107,8 +107,7 @@ def test_parallel_sampling_cascade():
     out = r.cache.decode_cascade(ids, q.cuda(), w.scale).cpu()
     st, info = B.pa_get_device_error()
     assert st == B.PA_OK, (st, info)
-    tables, lens, _ = r.cache.decode_inputs(ids)
-    offs, members, prefix, seq_prefix = r.cache.shared_prefix_groups(ids, tables, lens, 16)
+    offs, members, prefix, seq_prefix, _ = r.cache.shared_prefix_groups(ids, 16)
     assert len(prefix) == 8 and (prefix == 960).all()      # 62 shared blocks of 16 -> 960 tokens
     r.decodes.append((list(ids), q, out))
     r.check_outputs()
@@ -182,8 +181,7 @@ def test_cascade_8bit_cache(fmt, G, D, bs):
     a = cache.decode(ids, q.cuda(), D ** -0.5).cpu()
     b = cache.decode_cascade(ids, q.cuda(), D ** -0.5).cpu()
     assert B.pa_get_device_error()[0] == B.PA_OK
-    tables, lens, _ = cache.decode_inputs(ids)
-    assert len(cache.shared_prefix_groups(ids, tables, lens, 64 // G)[2]) > 0   # some prefix is shared
+    assert len(cache.shared_prefix_groups(ids, 64 // G)[2]) > 0   # some prefix is shared
     assert float((a - b).abs().max()) <= 2e-3
     for i in (0, len(ids) // 2, len(ids) - 1):
         s = ids[i]
