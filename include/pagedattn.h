@@ -149,6 +149,18 @@ pa_status pa_swap_blocks(const pa_cache* cache, void* host_k, void* host_v, int6
                          const int32_t* pairs, int32_t n_pairs, int32_t to_host, pa_stream stream);
 
 /*
+ * pa_swap_blocks on the copy engines: the same move, with the pairs in host
+ * memory and one cudaMemcpyAsync per tensor for every run of pairs whose
+ * source and destination ids both advance by one (a single block when the ids
+ * are scattered). host_k, host_v: pinned host pools (cudaHostAlloc or
+ * cudaHostRegister; no device mapping needed). Ids are checked on the host
+ * before any copy (PA_ERR_INVALID_ARG). Leaves the SMs free; costs one host
+ * call per run.
+ */
+pa_status pa_swap_blocks_copy(const pa_cache* cache, void* host_k, void* host_v, int64_t host_num_blocks,
+                              const int32_t* host_pairs, int32_t n_pairs, int32_t to_host, pa_stream stream);
+
+/*
  * Single-query decode attention over the paged cache.
  * P2 §1.1: out = softmax(scale * q K^T) V, one query row per head; P2 §3.2.2
  * step 4 and §4.1: every logical block of the sequence is visited through its
@@ -277,17 +289,20 @@ pa_status pa_get_device_error(pa_stream stream, int64_t* info_out);
  * and outputs: an inference runtime that reserves the whole device up front
  * and gives plug-ins no workspace, or a latency-bound serving loop where a
  * cudaMalloc (which may synchronise the device) is not allowed between steps.
- * Arguments, results and errors are those of pa_decode; the partial results of
- * a split sequence go to an array of PA_STATIC_WORKSPACE_BYTES compiled into
- * the library, which every device that loads the library holds until the
- * process exits. A call whose split would need more than that returns
- * PA_ERR_INVALID_ARG and launches nothing (pa_decode_workspace_bytes gives the
- * need; partition_tokens = 0 needs none).
- * The first call on each device looks up that device's address of the array
- * (make it before any stream capture). The array is shared by every call on
- * the device and keeps the last call's contents; nothing in it needs an
- * initial value. Calls that overlap on the GPU (other streams, other threads)
- * race on the array and must be serialised by the caller.
+ * Arguments, results and errors are those of pa_decode; the workspace pa_decode
+ * would take (its work counters and the partial results of split sequences)
+ * is an array of PA_STATIC_WORKSPACE_BYTES compiled into the library, which
+ * every device that loads the library holds until the process exits. Every
+ * call with num_seqs > 0 uses the array (the counters at least, whatever
+ * partition_tokens is). A call whose need (pa_decode_workspace_bytes) is
+ * larger than the array returns PA_ERR_INVALID_ARG and launches nothing.
+ * The first such call on each device looks up that device's address of the
+ * array and keeps it; make that first call before any stream capture. The
+ * kept address is not refreshed, so the library must not outlive a reset of
+ * the device (cudaDeviceReset) in the same process. The array is shared by
+ * every call on the device and keeps the last call's contents; nothing in it
+ * needs an initial value. Calls that overlap on the GPU (other streams, other
+ * threads) race on the array and must be serialised by the caller.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
@@ -325,6 +340,24 @@ pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, const int64_
                        const void* q_host, const void* k_host, const void* v_host, float scale, float* out_host,
                        int32_t partition_tokens, void* dev_staging, size_t dev_staging_bytes, void* host_staging,
                        size_t host_staging_bytes, pa_stream stream);
+
+/* Host wall-clock phases of the calling thread's last successful
+ * pa_step_host call, in microseconds (all zero after a failed call): the
+ * block-manager work (argument checks, slots, copy-on-write pairs, tables),
+ * enqueueing the host -> device copies, the three device-operation calls,
+ * enqueueing the device -> host copy of the output, and the wait for the
+ * stream; total_us spans the whole call. The device runs the copies and
+ * kernels between the first enqueue and the end of the wait. */
+typedef struct {
+  double block_manager_us;
+  double h2d_enqueue_us;
+  double launch_us;
+  double d2h_enqueue_us;
+  double wait_us;
+  double total_us;
+} pa_step_timing;
+
+pa_status pa_step_host_last_timing(pa_step_timing* out);
 
 /* Staging sizes pa_step_host needs for up to n sequences whose lengths stay
  * at most max_context_len after the step. */
@@ -436,6 +469,36 @@ pa_status pa_bm_block_tables(const pa_bm* bm, int32_t n, const int64_t* seq_ids,
                              int32_t pad, int32_t* lens_out);
 
 pa_status pa_bm_refcount(const pa_bm* bm, int32_t block, int32_t* out);
+
+/*
+ * Shared-prefix groups of a decode batch, the host side of pa_decode_cascade
+ * (P2 §3.4: sequences sharing a prefix point at the same physical blocks;
+ * P1 "跨请求的内存共享": parallel samples of one prompt).
+ *
+ *   seq_ids              host int64 [n]: the batch, in the order of its rows.
+ *   max_group_size       >= 1; pass 64 / (num_q_heads / num_kv_heads) for
+ *                        pa_decode_cascade.
+ *   align_tokens         >= 1; prefixes are cut down to a multiple of it
+ *                        (64 for pa_decode_cascade).
+ *   group_offsets        host int32, at least n / 2 + 1 entries: group j owns
+ *                        group_members[group_offsets[j] .. group_offsets[j+1]).
+ *   group_members        host int32 [n]: batch row indices.
+ *   group_prefix_tokens  host int32, at least n / 2 entries.
+ *   seq_prefix_tokens    host int32 [n]: the row's group prefix, 0 if none.
+ *   *n_groups_out        number of groups; *max_prefix_out (may be NULL) the
+ *                        largest prefix.
+ * Rule: sequences with at least one whole block are keyed by the physical id
+ * of their first block (keys in order of first appearance); each key's rows,
+ * in batch order, are cut into groups of at most max_group_size; a group's
+ * prefix is the longest run of leading table entries identical in every
+ * member, counted over the whole blocks of its shortest member, cut down to a
+ * multiple of align_tokens. Groups of one member or with no prefix left are
+ * dropped. Reads the manager only; PA_ERR_UNKNOWN_SEQ if an id is not live.
+ */
+pa_status pa_bm_prefix_groups(const pa_bm* bm, int32_t n, const int64_t* seq_ids, int32_t max_group_size,
+                              int32_t align_tokens, int32_t* group_offsets, int32_t* group_members,
+                              int32_t* group_prefix_tokens, int32_t* seq_prefix_tokens, int32_t* n_groups_out,
+                              int32_t* max_prefix_out);
 
 /* free_blocks: blocks on the free list (evictable cached blocks are not
  * counted); allocated_slots: block_size times the blocks not on the free

@@ -71,6 +71,9 @@ _SIGS = {
     "pa_bm_swap_out": (_I32, [_VP, _I64, _VP, _I32, _P32]),
     "pa_bm_swap_in": (_I32, [_VP, _I64, _VP, _I32, _P32]),
     "pa_swap_blocks": (_I32, [_PCACHE, _VP, _VP, _I64, _VP, _I32, _I32, _VP]),
+    "pa_swap_blocks_copy": (_I32, [_PCACHE, _VP, _VP, _I64, _VP, _I32, _I32, _VP]),
+    "pa_step_host_last_timing": (_I32, [_VP]),
+    "pa_bm_prefix_groups": (_I32, [_VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _P32, _P32]),
     "pa_bm_prefix_stats": (_I32, [_VP, _P64, _P64, _P64]),
     "pa_bm_append_slot": (_I32, [_VP, _I64, _P64, _P32]),
     "pa_bm_append_slots": (_I32, [_VP, _I32, _VP, _VP, _VP, _P32]),
@@ -335,6 +338,32 @@ def pa_swap_blocks(k_cache, v_cache, host_k, host_v, pairs, to_host: bool, strea
                                  _stream(k_cache, stream)), "pa_swap_blocks")
 
 
+def pa_swap_blocks_copy(k_cache, v_cache, host_k, host_v, pairs: np.ndarray, to_host: bool, stream=None):
+    """pa_swap_blocks on the copy engines: pairs in host memory, one
+    cudaMemcpyAsync per tensor per run of consecutive ids."""
+    c = make_cache(k_cache, v_cache)
+    if host_k.is_cuda or host_v.is_cuda or host_k.shape != host_v.shape or host_k.shape[1:] != k_cache.shape[1:] \
+            or host_k.dtype != k_cache.dtype or not host_k.is_contiguous() or not host_v.is_contiguous():
+        raise ValueError("host pools must be contiguous host tensors shaped like the cache (pinned)")
+    pr = np.ascontiguousarray(pairs, dtype=np.int32).reshape(-1, 2)
+    _check(_lib().pa_swap_blocks_copy(ctypes.byref(c), host_k.data_ptr(), host_v.data_ptr(), int(host_k.shape[0]),
+                                      _i64p(pr), int(pr.shape[0]), 1 if to_host else 0, _stream(k_cache, stream)),
+           "pa_swap_blocks_copy")
+
+
+class pa_step_timing(ctypes.Structure):
+    _fields_ = [("block_manager_us", ctypes.c_double), ("h2d_enqueue_us", ctypes.c_double),
+                ("launch_us", ctypes.c_double), ("d2h_enqueue_us", ctypes.c_double), ("wait_us", ctypes.c_double),
+                ("total_us", ctypes.c_double)]
+
+
+def pa_step_host_last_timing() -> dict:
+    """Host phases (microseconds) of this thread's last pa_step_host call."""
+    t = pa_step_timing()
+    _check(_lib().pa_step_host_last_timing(ctypes.byref(t)), "pa_step_host_last_timing")
+    return {name: float(getattr(t, name)) for name, _ in pa_step_timing._fields_}
+
+
 def pa_selftest_wait_timeout(timeout_ns: int, stream=None):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -450,6 +479,23 @@ class BlockManager:
         _check(_lib().pa_bm_block_tables(self._h, len(ids), _i64p(ids), _i64p(out), cap, pad, _i64p(lens_out)),
                "pa_bm_block_tables")
         return out, lens_out
+
+    def prefix_groups(self, seq_ids, max_group_size: int, align_tokens: int = 64):
+        """Shared-prefix groups of a batch (pa_bm_prefix_groups): (offsets,
+        members, prefix_tokens, seq_prefix_tokens, max_prefix) as numpy arrays
+        and an int."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = len(ids)
+        offs = np.zeros(n // 2 + 1, dtype=np.int32)
+        members = np.zeros(max(n, 1), dtype=np.int32)
+        prefix = np.zeros(max(n // 2, 1), dtype=np.int32)
+        seq_prefix = np.zeros(max(n, 1), dtype=np.int32)
+        ng, mp = ctypes.c_int32(0), ctypes.c_int32(0)
+        _check(_lib().pa_bm_prefix_groups(self._h, n, _i64p(ids), int(max_group_size), int(align_tokens), _i64p(offs),
+                                          _i64p(members), _i64p(prefix), _i64p(seq_prefix), ctypes.byref(ng),
+                                          ctypes.byref(mp)), "pa_bm_prefix_groups")
+        g = ng.value
+        return offs[:g + 1].copy(), members[:offs[g]].copy(), prefix[:g].copy(), seq_prefix[:n].copy(), int(mp.value)
 
     def refcount(self, block: int) -> int:
         r = ctypes.c_int32()

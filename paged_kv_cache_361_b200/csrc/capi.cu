@@ -400,6 +400,51 @@ pa_status pa_swap_blocks(const pa_cache* cache, void* host_k, void* host_v, int6
   return launched();
 }
 
+pa_status pa_swap_blocks_copy(const pa_cache* cache, void* host_k, void* host_v, int64_t host_num_blocks,
+                              const int32_t* host_pairs, int32_t n_pairs, int32_t to_host, pa_stream stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (n_pairs < 0 || host_num_blocks <= 0 || host_num_blocks > INT32_MAX) return PA_ERR_INVALID_ARG;
+  if (n_pairs == 0) return PA_OK;
+  if (!host_k || !host_v || !host_pairs) return PA_ERR_INVALID_ARG;
+  for (int i = 0; i < 2; ++i) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, i == 0 ? host_k : host_v) != cudaSuccess) {
+      cudaGetLastError();
+      return PA_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeHost) return PA_ERR_INVALID_ARG;  // pinned only: async copies
+  }
+  const int64_t src_nb = to_host ? cache->num_blocks : host_num_blocks;
+  const int64_t dst_nb = to_host ? host_num_blocks : cache->num_blocks;
+  for (int32_t p = 0; p < n_pairs; ++p) {
+    const int32_t a = host_pairs[2 * p], b = host_pairs[2 * p + 1];
+    if (a < 0 || a >= src_nb || b < 0 || b >= dst_nb) return PA_ERR_INVALID_ARG;
+  }
+  const size_t blk = static_cast<size_t>(cache->num_kv_heads) * cache->block_size * cache->head_dim *
+                     elem_bytes(cache->dtype);
+  char* sk = static_cast<char*>(to_host ? cache->k : host_k);
+  char* sv = static_cast<char*>(to_host ? cache->v : host_v);
+  char* dk = static_cast<char*>(to_host ? host_k : cache->k);
+  char* dv = static_cast<char*>(to_host ? host_v : cache->v);
+  const cudaMemcpyKind kind = to_host ? cudaMemcpyDeviceToHost : cudaMemcpyHostToDevice;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int32_t p = 0; p < n_pairs;) {
+    int32_t q = p + 1;  // extend the run while both ids advance by one
+    while (q < n_pairs && host_pairs[2 * q] == host_pairs[2 * q - 2] + 1 &&
+           host_pairs[2 * q + 1] == host_pairs[2 * q - 1] + 1)
+      ++q;
+    const size_t off_s = static_cast<size_t>(host_pairs[2 * p]) * blk;
+    const size_t off_d = static_cast<size_t>(host_pairs[2 * p + 1]) * blk;
+    const size_t bytes = static_cast<size_t>(q - p) * blk;
+    if (cudaMemcpyAsync(dk + off_d, sk + off_s, bytes, kind, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv + off_d, sv + off_s, bytes, kind, s) != cudaSuccess)
+      return PA_ERR_CUDA;
+    p = q;
+  }
+  return PA_OK;
+}
+
 pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, int32_t max_q_len, int32_t num_q_heads,
                      const pa_cache* cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
                      const int32_t* context_lens, int32_t max_context_len, float scale, float* out, pa_stream stream) {

@@ -11,12 +11,20 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <chrono>
 #include <cstdint>
 #include <vector>
 
 #include "../../include/pagedattn.h"
 
 namespace {
+
+// Host-side phase times of the calling thread's last pa_step_host call.
+thread_local pa_step_timing g_last_timing = {};
+
+double us_since(std::chrono::steady_clock::time_point t0, std::chrono::steady_clock::time_point t1) {
+  return std::chrono::duration<double, std::micro>(t1 - t0).count();
+}
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -69,6 +77,9 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
                                   float scale, float* out_host, int32_t partition_tokens, void* dev_staging,
                                   size_t dev_staging_bytes, void* host_staging, size_t host_staging_bytes,
                                   pa_stream stream) {
+  using clock = std::chrono::steady_clock;
+  const clock::time_point t_begin = clock::now();
+  g_last_timing = pa_step_timing{};
   if (!bm || !cache || n < 0 || num_q_heads <= 0 || partition_tokens < -1) return PA_ERR_INVALID_ARG;
   if (n == 0) return PA_OK;
   if (!seq_ids || !q_host || !k_host || !v_host || !out_host || !dev_staging || !host_staging ||
@@ -102,6 +113,7 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
   st = pa_bm_block_tables(bm, n, seq_ids, reinterpret_cast<int32_t*>(h + L.m_tables), L.cap, -1,
                           reinterpret_cast<int32_t*>(h + L.m_lens));
   if (st != PA_OK) return st;
+  const clock::time_point t_bm = clock::now();
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* d = static_cast<char*>(dev_staging);
@@ -113,6 +125,7 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
       cudaMemcpyAsync(d + L.k, k_host, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(d + L.v, v_host, kb, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return PA_ERR_CUDA;
+  const clock::time_point t_h2d = clock::now();
   char* meta = d + L.meta;
   if (n_pairs > 0) {
     st = pa_copy_blocks(cache, reinterpret_cast<const int32_t*>(meta + L.m_pairs), n_pairs, stream);
@@ -125,8 +138,23 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
                  reinterpret_cast<const int32_t*>(meta + L.m_lens), static_cast<int32_t>(max_len), scale, out_dev,
                  partition_tokens, L.ws_bytes ? d + L.ws : nullptr, L.ws_bytes, stream);
   if (st != PA_OK) return st;
+  const clock::time_point t_launch = clock::now();
   const size_t ob = static_cast<size_t>(n) * num_q_heads * cache->head_dim * 4;
   if (cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s) != cudaSuccess) return PA_ERR_CUDA;
+  const clock::time_point t_d2h = clock::now();
   if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  const clock::time_point t_end = clock::now();
+  g_last_timing.block_manager_us = us_since(t_begin, t_bm);
+  g_last_timing.h2d_enqueue_us = us_since(t_bm, t_h2d);
+  g_last_timing.launch_us = us_since(t_h2d, t_launch);
+  g_last_timing.d2h_enqueue_us = us_since(t_launch, t_d2h);
+  g_last_timing.wait_us = us_since(t_d2h, t_end);
+  g_last_timing.total_us = us_since(t_begin, t_end);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_step_host_last_timing(pa_step_timing* out) {
+  if (!out) return PA_ERR_INVALID_ARG;
+  *out = g_last_timing;
   return PA_OK;
 }
