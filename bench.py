@@ -39,12 +39,32 @@ sys.path.insert(0, ROOT)
 METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode attention tokens/sec"
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# dominant kernel, from an ncu capture of
-#   python bench.py --steps 3 --warmup 3 --no-e2e --no-cpu-baseline
-# (profiles/decode_simt_llama2_7b_mha.md), keyed by (workload, cache dtype,
-# partition tokens). Configurations without a capture of the current kernel
-# report null.
-NCU_TRAFFIC = {("llama2_7b_mha", "bfloat16", 0): 1_082_858_240}
+# dominant kernel, from one-pass ncu captures of this script, keyed by
+# (workload, cache dtype, partition tokens) -> (bytes, source files of that
+# kernel, their hash at capture). A capture whose files have changed since is
+# stale and reported as null, as is any configuration without a capture.
+NCU_TRAFFIC: dict = {}
+CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
+
+
+def src_hash(files) -> str:
+    """sha256 (16 hex digits) over the named CUDA sources of the library."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in sorted(files):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(key):
+    e = NCU_TRAFFIC.get(key)
+    if e is None:
+        return None, "no capture of this configuration"
+    nbytes, files, sha = e
+    if src_hash(files) != sha:
+        return None, "stale: the kernel's sources changed since the capture"
+    return nbytes, f"one-pass ncu capture of the current kernel (sources {sha})"
 
 
 def peaks():
@@ -137,8 +157,9 @@ WORKLOADS = {
                           "512-token partitions, bf16",
     "parallel_sampling": "parallel_sampling_decode: 8 prompts x 8 samples, 1000-token shared prefix + tails U[1,512], "
                          "32/8 heads, D128, bs16, bf16",
-    "continuous_batching": "continuous_batching_decode: 256 live seqs, ctx lognormal(500,1) capped 4096, first step "
-                           "of the trace, 200k-block pool, 32/8 heads, D128, bs16, bf16",
+    "continuous_batching": "continuous_batching_decode: 256 live seqs, ctx lognormal(500,1) capped 4096, all 200 steps "
+                           "of the trace (finish p 0.005, arrivals lognormal(300,1)), 200k-block pool, 32/8 heads, D128, "
+                           "bs16, bf16",
 }
 
 
@@ -156,6 +177,28 @@ def workload_ops(name, seed):
     return tr.shape, tr.num_blocks, tr.free_order, 1.0 / math.sqrt(tr.shape.head_dim), 0, W.batching_ops(tr, steps=1)
 
 
+def fill_pool(cache, nb, kv_dtype, g, device):
+    """Device-generated pool contents standing in for the prompts' K/V: N(0,1)
+    values (bf16, or e4m3 codes at scale 1), or uniform int8 codes."""
+    for t in (cache.k_cache, cache.v_cache):
+        for i in range(0, nb, 1024):   # chunked to bound the fp32 temporary
+            if kv_dtype == "int8":
+                t[i:i + 1024] = torch.randint(-127, 128, t[i:i + 1024].shape, generator=g, device=device,
+                                              dtype=torch.int8)
+            else:
+                t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(t.dtype)
+
+
+def make_cache(sh, nb, order, kv_dtype, device):
+    from paged_kv_cache_361_b200 import PagedKVCache
+    from paged_kv_cache_361_b200 import workloads as W
+    dt = W.TORCH_DTYPE[sh.dtype]
+    cache_dt = {"fp8": torch.float8_e4m3fn, "int8": torch.int8}.get(kv_dtype, dt)
+    sc = 4.0 / 127 if kv_dtype == "int8" else 1.0
+    return PagedKVCache(nb, sh.num_kv_heads, sh.block_size, sh.head_dim, cache_dt, device, order, k_scale=sc,
+                        v_scale=sc), dt
+
+
 def build_workload(seed: int, device, name: str = "llama2_7b_mha", kv_dtype: str = "auto"):
     """Replays the workload's operation script up to the measured step through
     PagedKVCache: the pool is filled with N(0,1) values on the device (they
@@ -167,23 +210,11 @@ def build_workload(seed: int, device, name: str = "llama2_7b_mha", kv_dtype: str
     kv_dtype "fp8" stores the cache as e4m3 codes (per-tensor scales 1.0: the
     N(0,1) values are inside the e4m3 range), "int8" as uniform random int8
     codes in [-127, 127] (scales 4/127); q and the new K/V rows stay bf16."""
-    from paged_kv_cache_361_b200 import PagedKVCache
-    from paged_kv_cache_361_b200 import workloads as W
     sh, nb, order, scale, part, ops = workload_ops(name, seed)
-    dt = W.TORCH_DTYPE[sh.dtype]
-    cache_dt = {"fp8": torch.float8_e4m3fn, "int8": torch.int8}.get(kv_dtype, dt)
-    sc = 4.0 / 127 if kv_dtype == "int8" else 1.0
-    cache = PagedKVCache(nb, sh.num_kv_heads, sh.block_size, sh.head_dim, cache_dt, device, order, k_scale=sc,
-                         v_scale=sc)
+    cache, dt = make_cache(sh, nb, order, kv_dtype, device)
     g = torch.Generator(device=device)
     g.manual_seed(1000 + seed)
-    for t in (cache.k_cache, cache.v_cache):
-        for i in range(0, nb, 1024):   # chunked to bound the fp32 temporary
-            if kv_dtype == "int8":
-                t[i:i + 1024] = torch.randint(-127, 128, t[i:i + 1024].shape, generator=g, device=device,
-                                              dtype=torch.int8)
-            else:
-                t[i:i + 1024] = torch.randn(t[i:i + 1024].shape, generator=g, device=device).to(cache_dt)
+    fill_pool(cache, nb, kv_dtype, g, device)
     hkv, D = sh.num_kv_heads, sh.head_dim
     assert ops[-2][0] == "append" and ops[-1][0] == "decode"
     for op in ops[:-2]:
@@ -225,15 +256,12 @@ def build_workload(seed: int, device, name: str = "llama2_7b_mha", kv_dtype: str
 
 def cascade_inputs(d, device):
     """Group arguments of pa_decode_cascade for the measured step (host work
-    done once, before timing): sequences whose tables start with the same
-    blocks share their common prefix."""
+    done once, before timing), from the C++ block manager
+    (pa_bm_prefix_groups): sequences whose tables start with the same blocks
+    share their common prefix."""
     from paged_kv_cache_361_b200 import binding as B
     cache, sh = d["cache"], d["shape"]
-    tables = d["tables"].cpu().numpy()
-    lens = d["lens"].cpu().numpy()
-    offs, members, prefix, seq_prefix = cache.shared_prefix_groups(d["ids"], tables, lens,
-                                                                   64 // sh.group)
-    max_pre = int(prefix.max()) if len(prefix) else 0
+    offs, members, prefix, seq_prefix, max_pre = cache.shared_prefix_groups(d["ids"], 64 // sh.group)
     nbytes = B.pa_decode_cascade_workspace_bytes(len(d["ids"]), sh.num_q_heads, sh.num_kv_heads, sh.head_dim,
                                                  d["max_len"], sh.block_size, max_pre)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -288,20 +316,86 @@ def cpu_threads():
     return os.cpu_count() or 1
 
 
+def cpu_baseline_record(rows, scale, seconds, elem_bytes, sample_desc):
+    """The oracle on all of the BLAS pool's threads and on one thread (the
+    pool limited by threadpoolctl), each for about `seconds`."""
+    import threadpoolctl
+    cores = cpu_threads()
+    gbs, el, n = time_oracle(rows, scale, seconds, elem_bytes)
+    with threadpoolctl.threadpool_limits(limits=1, user_api="blas"):
+        gbs1, el1, n1 = time_oracle(rows, scale, seconds, elem_bytes)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 NumPy oracle over {sample_desc}, repeated for {el:.1f} s ({n} sequence passes) on "
+                      f"{cores} BLAS threads and {el1:.1f} s ({n1} passes) on 1 thread; host has "
+                      f"{os.cpu_count()} cores",
+            "by_threads": {str(cores): round(gbs, 4), "1": round(gbs1, 4)}}
+
+
+# --- timing helpers --------------------------------------------------------------
+
+def ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def time_calls(pre, timed, steps, warmup, stream):
+    """Runs pre(); timed() `warmup` times untimed, then `steps` times with CUDA
+    events around each timed() on `stream`. Returns (per-call ms list, whole
+    region ms)."""
+    for _ in range(warmup):
+        pre()
+        timed()
+    torch.cuda.synchronize()
+    evs = [(ev(), ev()) for _ in range(steps)]
+    t0, t1 = ev(), ev()
+    t0.record(stream)
+    for i in range(steps):
+        pre()
+        evs[i][0].record(stream)
+        timed()
+        evs[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs], t0.elapsed_time(t1)
+
+
+def check_device(B, what):
+    st, info = B.pa_get_device_error()
+    if st != B.PA_OK:
+        raise RuntimeError(f"device error {st} ({info}) in {what}")
+
+
 # --- arms --------------------------------------------------------------------------
+
+def decode_fns(B, d, P, cascade=None):
+    def write_step():
+        if d["pairs"] is not None:
+            B.pa_copy_blocks(d["kc"], d["vc"], d["pairs"])
+        B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
+
+    sh = d["shape"]
+    nseq = len(d["ids"])
+    ws_bytes = B.pa_decode_workspace_bytes(nseq, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, d["max_len"],
+                                           sh.block_size, P)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=d["kc"].device)
+
+    def decode():
+        if cascade is not None:
+            B.pa_decode_cascade(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"],
+                                *cascade)
+            return
+        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"], P, ws)
+    return write_step, decode
+
 
 def run_ours(args, rank, world, device):
     from paged_kv_cache_361_b200 import binding as B
+    if args.workload == "continuous_batching":
+        return run_batching_line(args, rank, world, device)
     d = build_workload(seed=rank, device=device, name=args.workload, kv_dtype=args.kv_dtype)
     sh = d["shape"]
     nseq = len(d["ids"])
-    cascade = None
-    if args.cascade:
-        cascade = cascade_inputs(d, device)
+    cascade = cascade_inputs(d, device) if args.cascade else None
     P = args.partition if args.partition != -2 else d["part"]
-    ws_bytes = B.pa_decode_workspace_bytes(nseq, sh.num_q_heads, sh.num_kv_heads, sh.head_dim, d["max_len"],
-                                           sh.block_size, P)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device) if ws_bytes else None
     P_eff = P if P >= 0 else B.pa_decode_partition_tokens(nseq, sh.num_q_heads, sh.num_kv_heads, d["max_len"],
                                                           sh.block_size)
     split = P_eff > 0 and math.ceil(d["max_len"] / P_eff) > 1
@@ -310,28 +404,15 @@ def run_ours(args, rank, world, device):
     sample_seqs = [0, 1, 2, 3] if args.workload == "llama2_7b_mha" else [0]
     baseline_rows = sample_rows(d, sample_seqs) if rank == 0 and world == 1 and not args.no_cpu_baseline else None
 
-    def write_step():
-        if d["pairs"] is not None:
-            B.pa_copy_blocks(d["kc"], d["vc"], d["pairs"])
-        B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
-
-    def decode():
-        if cascade is not None:
-            B.pa_decode_cascade(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"],
-                                *cascade)
-            return
-        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"], P, ws)
-
+    write_step, decode = decode_fns(B, d, P, cascade)
     for _ in range(args.warmup):
         write_step()
         decode()
     torch.cuda.synchronize(device)
-    st, info = B.pa_get_device_error()
-    if st != B.PA_OK:
-        raise RuntimeError(f"device error {st} ({info}) during warm-up")
+    check_device(B, "warm-up")
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [(ev(), ev()) for _ in range(args.steps)]
+    t_start, t_end = ev(), ev()
     clocks = Clocks(device)
     if world > 1:
         torch.distributed.barrier()
@@ -340,19 +421,17 @@ def run_ours(args, rank, world, device):
     t_start.record(stream)
     for i in range(args.steps):
         write_step()
-        ev[i][0].record(stream)
+        evs[i][0].record(stream)
         decode()
-        ev[i][1].record(stream)
+        evs[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(device)
     clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
     total_ms = t_start.elapsed_time(t_end)
-    decode_ms = [a.elapsed_time(b) for a, b in ev]
-    st, info = B.pa_get_device_error()
-    if st != B.PA_OK:
-        raise RuntimeError(f"device error {st} ({info}) in the timed region")
+    decode_ms = [a.elapsed_time(b) for a, b in evs]
+    check_device(B, "the timed region")
 
     kv_bytes = d["kv_bytes"]
     total_ms, all_bytes = combine_ranks(total_ms, kv_bytes, world, device)
@@ -364,10 +443,8 @@ def run_ours(args, rank, world, device):
 
     cpu = None
     if baseline_rows is not None:
-        gbs, el, n = time_oracle(baseline_rows, d["scale"], args.cpu_seconds, d["kc"].element_size())
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"fp64 NumPy oracle over sequences {sample_seqs} of the workload (all heads), repeated "
-                         f"for {el:.1f} s ({n} sequence passes); host has {os.cpu_count()} cores"}
+        cpu = cpu_baseline_record(baseline_rows, d["scale"], args.cpu_seconds, d["kc"].element_size(),
+                                  f"sequences {sample_seqs} of the workload (all heads)")
 
     peak, peak_kind = peaks()
     dec_avg_ms = statistics.mean(decode_ms)
@@ -378,110 +455,232 @@ def run_ours(args, rank, world, device):
         launches = args.steps * (1 + (1 if n_groups else 0) + 2 + (1 if d["pairs"] is not None else 0))
     else:
         launches = args.steps * (2 + (1 if split else 0) + (1 if d["pairs"] is not None else 0))
+    dtype_key = str(d["kc"].dtype).replace("torch.", "")
+    traffic, traffic_src = (None, "not captured for the cascade path") if cascade is not None else \
+        ncu_traffic((args.workload, dtype_key, P_eff))
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": {"fp8": "fp8_e4m3 cache, bf16 q", "int8": "int8 cache, bf16 q"}.get(args.kv_dtype, sh.dtype),
+        "data": "synthetic",
+        "config": {"workload": WORKLOADS[args.workload], "num_seqs": nseq, "num_q_heads": sh.num_q_heads,
+                   "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "block_size": sh.block_size,
+                   "num_blocks": int(d["kc"].shape[0]), "context_tokens": int(d["lens_host"].sum()),
+                   "kv_bytes_per_step": kv_bytes, "unique_kv_bytes_per_step": d["unique_kv_bytes"],
+                   "partition_tokens": P_eff,
+                   "kv_dtype": dtype_key,
+                   "decode": "pa_decode_cascade (shared prefixes read once per group)" if cascade is not None
+                   else "pa_decode",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": "no flush: the K/V read per step is larger than the 126 MB L2"
+                   if d["unique_kv_bytes"] > 3 * 126e6 else "no flush: K/V partly L2-resident (see unique bytes)"},
+        "tokens_per_s": round(tokens_per_s, 1),
+        "pct_of_hbm_peak": {"of_measured_6540": round(value / peak, 4), "of_nominal_8000": round(value / 8000.0, 4)},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "roofline": {"kernel": ("pa_decode_cascade (prefix + suffix + merge); achieved counts logical K/V bytes"
+                                if cascade is not None else
+                                "pa_decode" + (" (decode + partition merge)" if split else "")), "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_source": traffic_src,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback", "decode_ms_avg": round(dec_avg_ms, 5)},
+        "cpu_baseline": cpu,
+        "clocks": clk,
+    }
+    # free this workload's device memory before the per-workload records
+    del d, write_step, decode
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and args.workload == "llama2_7b_mha" and args.kv_dtype == "auto" \
+            and not args.cascade and not args.no_workloads:
+        clocks = Clocks(device)
+        clocks.start()
+        line["workloads"] = run_workloads(args, device)
+        line["workloads"]["clocks"] = clocks.stop()
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None,
-            "dtype": {"fp8": "fp8_e4m3 cache, bf16 q", "int8": "int8 cache, bf16 q"}.get(args.kv_dtype, sh.dtype),
-            "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.workload], "num_seqs": nseq, "num_q_heads": sh.num_q_heads,
-                       "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "block_size": sh.block_size,
-                       "num_blocks": int(d["kc"].shape[0]), "context_tokens": int(d["lens_host"].sum()),
-                       "kv_bytes_per_step": kv_bytes, "unique_kv_bytes_per_step": d["unique_kv_bytes"],
-                       "partition_tokens": P_eff,
-                       "kv_dtype": str(d["kc"].dtype).replace("torch.", ""),
-                       "decode": "pa_decode_cascade (shared prefixes read once per group)" if cascade is not None
-                       else "pa_decode",
-                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                       "l2": "no flush: the K/V read per step is larger than the 126 MB L2"
-                       if d["unique_kv_bytes"] > 3 * 126e6 else "no flush: K/V partly L2-resident (see unique bytes)"},
-            "tokens_per_s": round(tokens_per_s, 1),
-            "pct_of_hbm_peak": {"of_measured_6540": round(value / peak, 4), "of_nominal_8000": round(value / 8000.0, 4)},
-            "e2e": e2e,
-            "gpu_launches": launches,
-            "roofline": {"kernel": ("pa_decode_cascade (prefix + suffix + merge); achieved counts logical K/V bytes"
-                                    if cascade is not None else
-                                    "pa_decode" + (" (decode + partition merge)" if split else "")), "bound": "hbm",
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4),
-                         "traffic": None if cascade is not None else NCU_TRAFFIC.get(
-                             (args.workload, str(d["kc"].dtype).replace("torch.", ""), P_eff)),
-                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                         else "fallback", "decode_ms_avg": round(dec_avg_ms, 5)},
-            "cpu_baseline": cpu,
-            "clocks": clk,
-        }
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, d, device, world, P):
-    """K steps through a prepared pa_step_host call (PagedKVCache.step_plan):
-    per step the C++ block manager appends, the step metadata and q/k/v go host
-    -> device from pinned memory, copy-on-write + append + decode run, and the
-    fp32 output comes back to pinned host memory before the call returns.
-    Context lengths grow by one per step."""
+def decode_record(B, d, P, steps, warmup, device, cascade=None):
+    """pa_decode (or the cascade) of one workload: kernel time per launch and the
+    whole step (append + decode), with the fractions of the measured peak."""
+    stream = torch.cuda.current_stream(device)
+    write_step, decode = decode_fns(B, d, P, cascade)
+    dec, total = time_calls(write_step, decode, steps, warmup, stream)
+    check_device(B, d["name"])
+    peak, kind = peaks()
+    ms = statistics.mean(dec)
+    gbs = d["kv_bytes"] / (ms * 1e-3) / 1e9
+    nseq = len(d["ids"])
     sh = d["shape"]
-    cache = d["cache"]
-    ids = d["ids"]
-    hq = d["q"].cpu().pin_memory()
-    hk = d["k"].cpu().pin_memory()
-    hv = d["v"].cpu().pin_memory()
-    hout = torch.empty(d["out"].shape, dtype=torch.float32, pin_memory=True)
-    eb = hq.element_size()
-    plan = cache.step_plan(ids, hq, hk, hv, hout, d["scale"], partition_tokens=P,
-                           max_context_len=int(max(cache.lens[s] for s in ids)) + args.warmup + args.steps + 1)
-    for _ in range(args.warmup):
-        plan.run()
-    L0 = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64, count=len(ids))
-    torch.cuda.synchronize(device)
+    P_eff = P if P >= 0 else B.pa_decode_partition_tokens(nseq, sh.num_q_heads, sh.num_kv_heads, d["max_len"],
+                                                          sh.block_size)
+    dtype_key = str(d["kc"].dtype).replace("torch.", "")
+    traffic, src = ncu_traffic((d["name"], dtype_key, P_eff)) if cascade is None else (None, "not captured")
+    rec = {"decode_ms": round(ms, 5), "step_ms": round(total / steps, 5), "kv_bytes": d["kv_bytes"],
+           "gbs": round(gbs, 1), "frac_of_measured_peak": round(gbs / peak, 4),
+           "frac_of_nominal_8000": round(gbs / 8000, 4), "tokens_per_s": round(nseq / (ms * 1e-3), 1),
+           "tokens_per_s_step": round(nseq / (total / steps * 1e-3), 1), "partition_tokens": P_eff,
+           "kv_dtype": dtype_key, "traffic": traffic, "traffic_source": src}
+    if d["unique_kv_bytes"] != d["kv_bytes"]:
+        rec["unique_kv_bytes"] = d["unique_kv_bytes"]
+        rec["unique_gbs"] = round(d["unique_kv_bytes"] / (ms * 1e-3) / 1e9, 1)
+    return rec
+
+
+def batching_trace(device, seed=0, kv_dtype="auto", num_blocks=None):
+    """The continuous-batching trace, all of its steps: host block-manager work
+    per step (frees, arrivals, one slot per live sequence, block tables),
+    timed on the host, and each step's slots / tables / lengths uploaded for the
+    device loop. Arrivals only reserve blocks: the device-filled pool stands in
+    for their prompts' K/V."""
+    from paged_kv_cache_361_b200 import workloads as W
+    tr = W.continuous_batching(seed=seed) if num_blocks is None else \
+        W.continuous_batching(seed=seed, num_blocks=num_blocks)
+    sh = tr.shape
+    cache, dt = make_cache(sh, tr.num_blocks, tr.free_order, kv_dtype, device)
+    g = torch.Generator(device=device)
+    g.manual_seed(3000 + seed)
+    fill_pool(cache, tr.num_blocks, kv_dtype, g, device)
+    ops = W.batching_ops(tr)
+    steps, host_s = [], []
+    t_host = 0.0
+    pending_slots = None
+    for op in ops:
+        t0 = time.perf_counter()
+        if op[0] == "add":
+            cache.reserve(op[1], op[2])
+        elif op[0] == "free":
+            cache.free(op[1])
+        elif op[0] == "append":
+            pending_slots, pairs = cache.bm.append_slots(op[1])
+            assert len(pairs) == 0
+            for s in op[1]:
+                cache.lens[s] += 1
+        elif op[0] == "decode":
+            tables, lens32, max_len = cache.decode_inputs(op[1])
+        t_host += time.perf_counter() - t0
+        if op[0] == "decode":
+            host_s.append(t_host)
+            t_host = 0.0
+            steps.append(dict(slots=torch.from_numpy(pending_slots).to(device),
+                              tables=torch.from_numpy(tables).to(device), lens=torch.from_numpy(lens32).to(device),
+                              max_len=int(max_len), tokens=int(lens32.astype(np.int64).sum()), n=len(op[1])))
+    n = steps[0]["n"]
+    hkv, D = sh.num_kv_heads, sh.head_dim
+    io = dict(q=torch.randn((n, sh.num_q_heads, D), generator=g, device=device).to(dt),
+              k=torch.randn((n, hkv, D), generator=g, device=device).to(dt),
+              v=torch.randn((n, hkv, D), generator=g, device=device).to(dt),
+              out=torch.empty((n, sh.num_q_heads, D), dtype=torch.float32, device=device))
+    return tr, cache, steps, host_s, io
+
+
+def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None):
+    """Every step of the continuous-batching trace on the device, in order
+    (append + pa_decode with the library's partition choice), `reps` passes
+    after one untimed pass; per-step averages over the whole trace."""
+    tr, cache, steps, host_s, io = batching_trace(device, seed, kv_dtype, num_blocks)
+    sh = tr.shape
+    eb = cache.k_cache.element_size()
+    ws_bytes = max(B.pa_decode_workspace_bytes(st["n"], sh.num_q_heads, sh.num_kv_heads, sh.head_dim, st["max_len"],
+                                               sh.block_size, -1) for st in steps)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+    scale = 1.0 / math.sqrt(sh.head_dim)
+    stream = torch.cuda.current_stream(device)
+    kc, vc = cache.k_cache, cache.v_cache
+
+    def one_pass(evs=None):
+        for i, st in enumerate(steps):
+            B.pa_reshape_and_cache(io["k"], io["v"], st["slots"], kc, vc)
+            if evs is not None:
+                evs[i][0].record(stream)
+            B.pa_decode(io["q"], kc, vc, st["tables"], st["lens"], scale, io["out"], st["max_len"], -1, ws)
+            if evs is not None:
+                evs[i][1].record(stream)
+
+    one_pass()
+    torch.cuda.synchronize()
+    check_device(B, "continuous batching warm-up")
+    dec, totals = [], []
+    for _ in range(reps):
+        evs = [(ev(), ev()) for _ in steps]
+        t0, t1 = ev(), ev()
+        t0.record(stream)
+        one_pass(evs)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        dec.append([a.elapsed_time(b) for a, b in evs])
+        totals.append(t0.elapsed_time(t1))
+    check_device(B, "continuous batching")
+    peak, _ = peaks()
+    nsteps = len(steps)
+    dec_ms = [statistics.mean(x[i] for x in dec) for i in range(nsteps)]
+    kv = [st["tokens"] * sh.num_kv_heads * sh.head_dim * 2 * eb for st in steps]
+    tot_dec = sum(dec_ms)
+    gbs = sum(kv) / (tot_dec * 1e-3) / 1e9
+    step_ms = statistics.mean(totals) / nsteps
+    ntok = sum(st["n"] for st in steps)
+    rec = {"steps": nsteps, "passes": reps, "decode_ms_avg": round(tot_dec / nsteps, 5),
+           "decode_ms_min": round(min(dec_ms), 5), "decode_ms_max": round(max(dec_ms), 5),
+           "step_ms_avg": round(step_ms, 5), "kv_bytes_avg": int(sum(kv) / nsteps),
+           "gbs": round(gbs, 1), "frac_of_measured_peak": round(gbs / peak, 4),
+           "frac_of_nominal_8000": round(gbs / 8000, 4), "tokens_per_s": round(ntok / (tot_dec * 1e-3), 1),
+           "tokens_per_s_step": round(ntok / (step_ms * nsteps * 1e-3), 1),
+           "host_block_manager_ms_avg": round(1e3 * statistics.mean(host_s), 4),
+           "host_block_manager_ms_max": round(1e3 * max(host_s), 4),
+           "host_note": "C++ block manager through the ctypes binding per step: frees, arrival reservations, one "
+                        "slot per live sequence, block tables; timed on the host, outside the device time",
+           "partition_tokens": sorted({B.pa_decode_partition_tokens(st["n"], sh.num_q_heads, sh.num_kv_heads,
+                                                                    st["max_len"], sh.block_size) for st in steps}),
+           "kv_dtype": str(kc.dtype).replace("torch.", "")}
+    return rec, dec_ms, kv
+
+
+def run_batching_line(args, rank, world, device):
+    """--workload continuous_batching: the contract's line for the whole
+    200-step trace (value = all steps' K/V bytes / all steps' time)."""
+    from paged_kv_cache_361_b200 import binding as B
+    clocks = Clocks(device)
     if world > 1:
         torch.distributed.barrier()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(args.steps):
-        plan.run()
-    t1.record()
-    torch.cuda.synchronize(device)
-    ms = t0.elapsed_time(t1)
-    # step k attends over L0 + k + 1 tokens per sequence
-    n, K = len(ids), args.steps
-    tokens = int(L0.sum()) * K + n * K * (K + 1) // 2
-    kv_total = tokens * sh.num_kv_heads * sh.head_dim * 2 * cache.k_cache.element_size()
-    nblk = int(-(-(int(L0.max()) + K) // sh.block_size))
-    h2d = (hq.numel() + hk.numel() + hv.numel()) * eb + n * (8 + 8 + nblk * 4 + 4)
-    d2h = hout.numel() * 4
-    ms, kv_total = combine_ranks(ms, kv_total, world, device)
-    return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
-            "ms_per_step": round(ms / args.steps, 4),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "api": "pa_step_host via PagedKVCache.step_plan (block manager, one metadata H2D, q/k/v H2D, "
-                   "pa_copy_blocks, pa_reshape_and_cache, pa_decode, output D2H, stream sync)"}
+    clocks.start()
+    rec, dec_ms, kv = batching_record(B, device, reps=max(1, args.steps // 10), kv_dtype=args.kv_dtype, seed=rank,
+                                      num_blocks=args.pool_blocks)
+    clk = clocks.stop()
+    ms_total = rec["step_ms_avg"] * rec["steps"]
+    ms_total, all_bytes = combine_ranks(ms_total, sum(kv), world, device)
+    value = all_bytes / (ms_total * 1e-3) / 1e9
+    peak, kind = peaks()
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": rec["steps"],
+            "warmup": rec["steps"], "ms_per_step": rec["step_ms_avg"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": rec["kv_dtype"], "data": "synthetic",
+            "config": {"workload": WORKLOADS["continuous_batching"] + (
+                           f" (pool cut to {args.pool_blocks} blocks)" if args.pool_blocks else ""),
+                       "passes": rec["passes"],
+                       "l2": "no flush: ~0.8 GB of K/V per step against the 126 MB L2"},
+            "tokens_per_s": rec["tokens_per_s_step"], "gpu_launches": rec["steps"] * rec["passes"] * 3,
+            "roofline": {"kernel": "pa_decode (200-step average)", "bound": "hbm", "achieved": rec["gbs"],
+                         "peak": peak, "unit": "GB/s", "frac": rec["frac_of_measured_peak"], "traffic": None,
+                         "peak_source": kind},
+            "batching": rec, "clocks": clk}), flush=True)
 
 
-PREFILL = {
-    "prefill_llama2_7b_mha": (32, 32, 8, 2048),   # Hq, Hkv, sequences, prompt tokens
-    "prefill_gqa8": (64, 8, 2, 8192),
-}
-
-
-def run_prefill(args, rank, world, device):
+def prefill_record(B, workload, kv_dtype, steps, warmup, device, rank=0):
     """Whole-prompt prefill (pa_reshape_and_cache of every prompt token +
-    pa_prefill) over a fresh paged cache; metric: causal attention TFLOP/s with
-    4 * head_dim * Hq flops per (query, visible key) pair. --kv-dtype fp8 keeps
-    the cache as e4m3 codes (per-tensor scales 4/448: N(0, 1) rows use the
-    code range)."""
-    from paged_kv_cache_361_b200 import PagedKVCache, binding as B
-    hq, hkv, nseq, plen = PREFILL[args.workload]
+    pa_prefill) over a fresh paged cache: causal attention TFLOP/s with
+    4 * head_dim * Hq flops per (query, visible key) pair."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    hq, hkv, nseq, plen = PREFILL[workload]
     D, bs = 128, 16
     nb = nseq * plen // bs + 16
     order = np.random.default_rng(rank).permutation(nb)
-    f8 = args.kv_dtype in ("fp8", "int8")
-    if args.kv_dtype == "fp8":
+    if kv_dtype == "fp8":
         cache = PagedKVCache(nb, hkv, bs, D, torch.float8_e4m3fn, device, order, k_scale=4.0 / 448,
                              v_scale=4.0 / 448)
-    elif args.kv_dtype == "int8":
+    elif kv_dtype == "int8":
         cache = PagedKVCache(nb, hkv, bs, D, torch.int8, device, order, k_scale=4.0 / 127, v_scale=4.0 / 127)
     else:
         cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, device, order)
@@ -499,63 +698,203 @@ def run_prefill(args, rank, world, device):
     L = torch.from_numpy(lens).to(device)
     cu = torch.arange(0, T + 1, plen, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
-
-    def step():
-        B.pa_reshape_and_cache(k, v, slots, cache.k_cache, cache.v_cache)
-        B.pa_prefill(q, cu, cache.k_cache, cache.v_cache, t, L, D ** -0.5, out, plen, max_len)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(device)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = Clocks(device)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(device)
-    clocks.start()
-    e0.record(stream)
-    for i in range(args.steps):
-        B.pa_reshape_and_cache(k, v, slots, cache.k_cache, cache.v_cache)
-        ev[i][0].record(stream)
-        B.pa_prefill(q, cu, cache.k_cache, cache.v_cache, t, L, D ** -0.5, out, plen, max_len)
-        ev[i][1].record(stream)
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    clk = clocks.stop()
-    st, info = B.pa_get_device_error()
-    if st != B.PA_OK:
-        raise RuntimeError(f"device error {st} ({info})")
-    ms = e0.elapsed_time(e1) / args.steps
-    pf_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    pf, total = time_calls(lambda: B.pa_reshape_and_cache(k, v, slots, cache.k_cache, cache.v_cache),
+                           lambda: B.pa_prefill(q, cu, cache.k_cache, cache.v_cache, t, L, D ** -0.5, out, plen,
+                                                max_len), steps, warmup, stream)
+    check_device(B, workload)
     flops = 4.0 * D * hq * nseq * plen * (plen + 1) / 2
-    ms, all_flops = combine_ranks(ms, flops, world, device)
+    pf_ms = statistics.mean(pf)
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             peak = float(json.load(f)["bf16_tflops"])
         src = "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
     except Exception:
         peak, src = 1590.0, "fallback"
+    return {"workload": f"{workload}: {nseq} prompts x {plen} tokens, {hq}/{hkv} heads, D128, bs16",
+            "kv_dtype": str(cache.k_cache.dtype).replace("torch.", ""), "prefill_ms": round(pf_ms, 4),
+            "step_ms": round(total / steps, 4), "flops": flops,
+            "tflops": round(flops / (pf_ms * 1e-3) / 1e12, 2), "peak": peak, "peak_source": src,
+            "frac": round(flops / (pf_ms * 1e-3) / 1e12 / peak, 4)}
+
+
+def swap_record(B, device, n_pairs=1024, reps=3):
+    """Swap throughput: n_pairs blocks of the metric workload's shape (32 kv
+    heads x 16 tokens x 128 dims, bf16: 128 KiB per tensor) moved out to a
+    pinned host pool and back, by the pa_swap_blocks kernel (SMs reading and
+    writing device-mapped host memory) and by pa_swap_blocks_copy (one
+    cudaMemcpyAsync per run of consecutive ids on the copy engines; the ids
+    here are scattered, so one per block)."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    hkv, bs, D = 32, 16, 128
+    nb = 2 * n_pairs
+    cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, device)
+    cache.k_cache.normal_()
+    cache.v_cache.normal_()
+    hk = torch.empty((n_pairs,) + tuple(cache.k_cache.shape[1:]), dtype=torch.bfloat16, pin_memory=True)
+    hv = torch.empty(hk.shape, dtype=torch.bfloat16, pin_memory=True)
+    rng = np.random.default_rng(7)
+    dev_ids = rng.permutation(nb)[:n_pairs].astype(np.int32)
+    host_ids = rng.permutation(n_pairs).astype(np.int32)
+    out_pairs = np.stack([dev_ids, host_ids], 1)
+    in_pairs = np.stack([host_ids, dev_ids], 1)
+    dout, din = torch.from_numpy(out_pairs).to(device), torch.from_numpy(in_pairs).to(device)
+    nbytes = 2 * n_pairs * hkv * bs * D * 2
+    stream = torch.cuda.current_stream(device)
+    rec = {"pairs": n_pairs, "bytes_each_way": nbytes}
+    variants = {
+        "kernel": (lambda: B.pa_swap_blocks(cache.k_cache, cache.v_cache, hk, hv, dout, True),
+                   lambda: B.pa_swap_blocks(cache.k_cache, cache.v_cache, hk, hv, din, False)),
+        "copy_engine": (lambda: B.pa_swap_blocks_copy(cache.k_cache, cache.v_cache, hk, hv, out_pairs, True),
+                        lambda: B.pa_swap_blocks_copy(cache.k_cache, cache.v_cache, hk, hv, in_pairs, False)),
+    }
+    for name, (out_fn, in_fn) in variants.items():
+        t_out, _ = time_calls(lambda: None, out_fn, reps, 1, stream)
+        t_in, _ = time_calls(lambda: None, in_fn, reps, 1, stream)
+        # host wall time of issuing the calls (the copy-engine path makes one call per run)
+        t0 = time.perf_counter()
+        out_fn()
+        issue_ms = (time.perf_counter() - t0) * 1e3
+        torch.cuda.synchronize()
+        rec[name] = {"out_ms": round(statistics.mean(t_out), 4), "in_ms": round(statistics.mean(t_in), 4),
+                     "out_gbs": round(nbytes / (statistics.mean(t_out) * 1e-3) / 1e9, 2),
+                     "in_gbs": round(nbytes / (statistics.mean(t_in) * 1e-3) / 1e9, 2),
+                     "host_issue_ms": round(issue_ms, 3)}
+    check_device(B, "swap")
+    # round trip leaves the pool unchanged
+    return rec
+
+
+def run_workloads(args, device):
+    """One record per workload of the pages' configurations beyond the metric
+    workload (each built, timed and freed in turn)."""
+    from paged_kv_cache_361_b200 import binding as B
+    steps, warm = 20, 5
+    rec = {}
+
+    def release(*objs):
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+    d = build_workload(0, device, "long_context_split")
+    rec["long_context_split_p512"] = decode_record(B, d, 512, steps, warm, device)
+    rec["long_context_split_auto"] = decode_record(B, d, -1, steps, warm, device)
+    del d
+    release()
+    for kvd in ("fp8", "int8"):
+        d = build_workload(0, device, "llama2_7b_mha", kv_dtype=kvd)
+        rec[f"llama2_7b_mha_{kvd}"] = decode_record(B, d, -1, steps, warm, device)
+        del d
+        release()
+    d = build_workload(0, device, "parallel_sampling")
+    rec["parallel_sampling"] = decode_record(B, d, -1, steps, warm, device)
+    rec["parallel_sampling_cascade"] = decode_record(B, d, -1, steps, warm, device, cascade_inputs(d, device))
+    del d
+    release()
+    cb, _, _ = batching_record(B, device, reps=2)
+    rec["continuous_batching_200_steps"] = cb
+    release()
+    for wl in ("prefill_llama2_7b_mha", "prefill_gqa8"):
+        rec[wl] = prefill_record(B, wl, "auto", 10, 3, device)
+        release()
+    rec["swap"] = swap_record(B, device)
+    release()
+    return rec
+
+
+def run_e2e(args, d, device, world, P):
+    """K steps through a prepared pa_step_host call (PagedKVCache.step_plan):
+    per step the C++ block manager appends, the step metadata and q/k/v go host
+    -> device from pinned memory, copy-on-write + append + decode run, and the
+    fp32 output comes back to pinned host memory before the call returns.
+    Context lengths grow by one per step. The breakdown averages the call's
+    own host phase timers (pa_step_host_last_timing) and times the same bytes'
+    copies alone (pinned, one stream) for the link's share."""
+    from paged_kv_cache_361_b200 import binding as B
+    sh = d["shape"]
+    cache = d["cache"]
+    ids = d["ids"]
+    hq = d["q"].cpu().pin_memory()
+    hk = d["k"].cpu().pin_memory()
+    hv = d["v"].cpu().pin_memory()
+    hout = torch.empty(d["out"].shape, dtype=torch.float32, pin_memory=True)
+    eb = hq.element_size()
+    plan = cache.step_plan(ids, hq, hk, hv, hout, d["scale"], partition_tokens=P,
+                           max_context_len=int(max(cache.lens[s] for s in ids)) + args.warmup + args.steps + 1)
+    for _ in range(args.warmup):
+        plan.run()
+    L0 = np.fromiter((cache.lens[s] for s in ids), dtype=np.int64, count=len(ids))
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    phases = []
+    t0, t1 = ev(), ev()
+    t0.record()
+    for _ in range(args.steps):
+        plan.run()
+        phases.append(B.pa_step_host_last_timing())
+    t1.record()
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1)
+    # step k attends over L0 + k + 1 tokens per sequence
+    n, K = len(ids), args.steps
+    tokens = int(L0.sum()) * K + n * K * (K + 1) // 2
+    kv_total = tokens * sh.num_kv_heads * sh.head_dim * 2 * cache.k_cache.element_size()
+    nblk = int(-(-(int(L0.max()) + K) // sh.block_size))
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * eb + n * (8 + 8 + nblk * 4 + 4)
+    d2h = hout.numel() * 4
+    # the same bytes over the link alone
+    dq = torch.empty(h2d, dtype=torch.uint8, device=device)
+    hsrc = torch.empty(h2d, dtype=torch.uint8, pin_memory=True)
+    dout = torch.empty(d2h, dtype=torch.uint8, device=device)
+    hdst = torch.empty(d2h, dtype=torch.uint8, pin_memory=True)
+    stream = torch.cuda.current_stream(device)
+    h2d_ms, _ = time_calls(lambda: None, lambda: dq.copy_(hsrc, non_blocking=True), 10, 3, stream)
+    d2h_ms, _ = time_calls(lambda: None, lambda: hdst.copy_(dout, non_blocking=True), 10, 3, stream)
+    mean = lambda key: round(statistics.mean(p[key] for p in phases), 2)
+    breakdown = {k: mean(k) for k in ("block_manager_us", "h2d_enqueue_us", "launch_us", "d2h_enqueue_us",
+                                      "wait_us", "total_us")}
+    breakdown["h2d_copy_alone_us"] = round(1e3 * statistics.mean(h2d_ms), 2)
+    breakdown["d2h_copy_alone_us"] = round(1e3 * statistics.mean(d2h_ms), 2)
+    ms, kv_total = combine_ranks(ms, kv_total, world, device)
+    return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_step": round(ms / args.steps, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "breakdown": breakdown,
+            "api": "pa_step_host via PagedKVCache.step_plan (block manager, one metadata H2D, q/k/v H2D, "
+                   "pa_copy_blocks, pa_reshape_and_cache, pa_decode, output D2H, stream sync)"}
+
+
+PREFILL = {
+    "prefill_llama2_7b_mha": (32, 32, 8, 2048),   # Hq, Hkv, sequences, prompt tokens
+    "prefill_gqa8": (64, 8, 2, 8192),
+}
+
+
+def run_prefill(args, rank, world, device):
+    """--workload prefill_*: the contract's line for whole-prompt prefill.
+    --kv-dtype fp8 / int8 keeps the cache as 8-bit codes (scales 4/448, 4/127)."""
+    from paged_kv_cache_361_b200 import binding as B
+    clocks = Clocks(device)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.start()
+    r = prefill_record(B, args.workload, args.kv_dtype, args.steps, args.warmup, device, rank)
+    clk = clocks.stop()
+    ms, all_flops = combine_ranks(r["step_ms"], r["flops"], world, device)
+    f8 = args.kv_dtype in ("fp8", "int8")
     if rank == 0:
         print(json.dumps({
             "metric": "paged prefill attention TFLOP/s (causal; 4*head_dim*Hq flops per visible query-key pair)",
             "value": round(all_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": f"{'fp8_e4m3' if args.kv_dtype == 'fp8' else 'int8'} cache, bf16 q (f16 MMA)" if f8 else "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{args.workload}: {nseq} prompts x {plen} tokens, {hq}/{hkv} heads, D128, bs16",
-                       "kv_dtype": str(cache.k_cache.dtype).replace("torch.", ""),
-                       "l2": "no flush: K/V of one launch "
-                             + f"{2 * T * hkv * D * (1 if f8 else 2) / 1e6:.0f} MB"},
+            "config": {"workload": r["workload"], "kv_dtype": r["kv_dtype"], "l2": "no flush: K/V of one launch "
+                       "larger than the 126 MB L2"},
             "gpu_launches": 2 * args.steps,
-            "roofline": {"kernel": "pa_prefill", "bound": "tensor", "achieved": round(flops / (pf_ms * 1e-3) / 1e12, 2),
-                         "peak": peak, "unit": "TFLOP/s", "frac": round(flops / (pf_ms * 1e-3) / 1e12 / peak, 4),
-                         "traffic": None, "peak_source": src,
-                         "note": ("tcgen05.mma (M 128) with TMEM accumulators; K/V codes widened to f16 in "
-                                  "shared memory, one f16 P V MMA per k-step") if f8 else
-                                 ("tcgen05.mma (M 128) with TMEM accumulators; P split into two bf16 MMAs "
-                                  "(1.5x the algorithmic MMA work)")},
+            "roofline": {"kernel": "pa_prefill", "bound": "tensor", "achieved": r["tflops"], "peak": r["peak"],
+                         "unit": "TFLOP/s", "frac": r["frac"], "traffic": None, "peak_source": r["peak_source"]},
             "clocks": clk}), flush=True)
 
 
@@ -604,13 +943,18 @@ def main():
     ap.add_argument("--partition", type=int, default=-1,
                     help="partition_tokens for pa_decode (-1: library choice, -2: the workload's own)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL), default="llama2_7b_mha")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=6.0,
+                    help="seconds of oracle work for each of the two CPU-baseline timings")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload records of the default run")
     ap.add_argument("--kv-dtype", choices=["auto", "fp8", "int8"], default="auto",
                     help="fp8 / int8: an 8-bit cache (e4m3 or int8 codes) with bf16 queries")
     ap.add_argument("--cascade", action="store_true",
                     help="decode through pa_decode_cascade (shared prefixes read once per group)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pool-blocks", type=int, default=None,
+                    help="continuous_batching only: a smaller pool (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -42,10 +42,12 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def command(out: str = LIB, ptxas_verbose: bool = False) -> list[str]:
+def command(out: str = LIB, ptxas_verbose: bool = False, defines=()) -> list[str]:
+    """nvcc command line; `defines` are extra -D settings of the kernels'
+    build-time tuning knobs (none for the library itself)."""
     cmd = [nvcc(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
            "-Xcompiler", "-fPIC,-O2", "-shared", "-cudart", "static", f"-I{INCLUDE}",
-           "-o", out] + [os.path.join(CSRC, f) for f in SOURCES]
+           "-o", out] + [f"-D{d}" for d in defines] + [os.path.join(CSRC, f) for f in SOURCES]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     return cmd

@@ -92,6 +92,30 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return pol;
 }
 
+__device__ __forceinline__ uint64_t l2_evict_normal_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// L2 priority of the decode kernels' K/V reads. Every byte of a plain decode
+// is read once per step, so evict-first keeps the stream from displacing
+// other data; a block shared by several sequences of the batch (forked
+// samples, cached prefixes) is read once per holder, and an evict-normal
+// stream lets the later readers hit in L2.
+#ifndef PA_KV_STREAM_POLICY
+#define PA_KV_STREAM_POLICY 0
+#endif
+__device__ __forceinline__ uint64_t kv_stream_policy() {
+#if PA_KV_STREAM_POLICY == 1
+  return l2_evict_normal_policy();
+#elif PA_KV_STREAM_POLICY == 2
+  return l2_evict_last_policy();
+#else
+  return l2_evict_first_policy();
+#endif
+}
+
 // One contiguous global -> shared copy by the TMA unit, completing on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t policy) {

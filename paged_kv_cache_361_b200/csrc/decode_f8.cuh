@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(F8Cfg<D>::kThreads) decode_f8_kernel(const __g
   if (warp == NW) {
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
-    const uint64_t pol = l2_evict_first_policy();
+    const uint64_t pol = kv_stream_policy();
     TableAhead ta;
     ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {

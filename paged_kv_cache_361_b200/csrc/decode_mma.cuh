@@ -102,6 +102,16 @@ __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint3
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
+// Build-time tuning knobs of the one-CTA-per-item kernel (defaults measured
+// on B200): ring stages at head_dim 128 (0 = the default of 3), and the CTAs
+// per SM its register budget is fitted to.
+#ifndef PA_MMA_STAGES
+#define PA_MMA_STAGES 0
+#endif
+#ifndef PA_MMA_MIN_CTAS
+#define PA_MMA_MIN_CTAS 1
+#endif
+
 template <int D>
 struct MmaCfg {
   static constexpr int kConsumerWarps = 4;
@@ -111,7 +121,7 @@ struct MmaCfg {
   static constexpr int kHalfBytes = kChunk * 128;          // one box column of a stage
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = kStageBytes <= 16384 ? 4 : 3;
+  static constexpr int kStages = kStageBytes <= 16384 ? 4 : (PA_MMA_STAGES > 0 ? PA_MMA_STAGES : 3);
   static constexpr int kQBytes = 8 * D * 2;                // query rows of one item (G <= 8)
   static constexpr int kNT = D / 8;
   static constexpr int kFoldFloats = 32 * (2 * kNT + 2);   // one warp's fragments + (m, l) per lane
@@ -314,7 +324,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
   if (warp == NW) {
     // ------------------------------ producer ------------------------------
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
-    const uint64_t pol = l2_evict_first_policy();
+    const uint64_t pol = kv_stream_policy();
     const __nv_bfloat16* qbase = static_cast<const __nv_bfloat16*>(a.q);
     int item = blockIdx.x;
     int cs = 0;
@@ -479,7 +489,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
 // end every warp's (m, l, o) goes through shared memory (the stage ring is free
 // by then) and the CTA stores the row or the partition's partials.
 template <int D, int G>
-__global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void __launch_bounds__(MmaCfg<D>::kThreads, PA_MMA_MIN_CTAS) decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const DecodeArgs a) {
   using Cfg = MmaCfg<D>;
@@ -510,7 +520,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_kernel(const _
   if (warp == NW) {
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
-    const uint64_t pol = l2_evict_first_policy();
+    const uint64_t pol = kv_stream_policy();
     TableAhead ta;
     ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {

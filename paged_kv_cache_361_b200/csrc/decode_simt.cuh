@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
     const uint32_t tile_bytes = static_cast<uint32_t>(a.bs) * D * Elem<T>::bytes;
     const T* kc = static_cast<const T*>(a.kc);
     const T* vc = static_cast<const T*>(a.vc);
-    const uint64_t pol = l2_evict_first_policy();
+    const uint64_t pol = kv_stream_policy();
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       const int32_t c0 = pt.t0 + i * C;
       const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 64 (C = 64, bs >= 1)
