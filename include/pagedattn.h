@@ -214,10 +214,13 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
  *   out            device fp32 [T][num_q_heads][head_dim].
  * Supported: bf16, e4m3 or int8 cache, block_size >= 8 (16, 32 as for decode),
  * head_dim 64 or 128, num_q_heads / num_kv_heads in {1, 2, 4, 8}; fp32 caches
- * return PA_ERR_UNSUPPORTED. Accumulation is fp32 on the tensor cores. Over an
- * 8-bit cache the codes are widened to f16 (exactly), q is rounded to f16 and
- * the softmax weights enter the P V product as f16 (11 significant bits; the
- * bf16 path keeps about 16 through a two-part split).
+ * return PA_ERR_UNSUPPORTED. Accumulation is fp32 on the tensor cores. The
+ * softmax weights enter the P V product as f16 (11 significant bits, weights
+ * at most 2^8), so V is read as f16: over a bf16 cache each V element is
+ * converted on chip, exactly for |v| in [2^-14, 65504] (smaller values move by
+ * less than 2^-25; |v| above 65504 is out of range); q and K stay bf16 for the
+ * q K^T product. Over an 8-bit cache the codes are widened to f16 (exactly)
+ * and q is rounded to f16.
  */
 pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, int32_t max_q_len, int32_t num_q_heads,
                      const pa_cache* cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
@@ -335,6 +338,13 @@ pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t nu
  * failure (PA_ERR_NO_FREE_BLOCKS, PA_ERR_UNKNOWN_SEQ) leaves the manager
  * unchanged and launches nothing. The staging buffers are reused by the next
  * call; the call returns only after the stream has drained.
+ * A batch of 16 or more sequences is cut into up to four row chunks whose
+ * copies, appends and decodes run as separate chains on streams the library
+ * creates once per device (kept until the process exits): the copy engines
+ * move one chunk's inputs and another's output while a third computes. The
+ * chains start after the work already queued on `stream`, and `stream` waits
+ * for all of them, so the call's ordering against the caller's stream is that
+ * of a single chain.
  */
 pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, const int64_t* seq_ids, int32_t num_q_heads,
                        const void* q_host, const void* k_host, const void* v_host, float scale, float* out_host,
@@ -344,17 +354,18 @@ pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, const int64_
 /* Host wall-clock phases of the calling thread's last successful
  * pa_step_host call, in microseconds (all zero after a failed call): the
  * block-manager work (argument checks, slots, copy-on-write pairs, tables),
- * enqueueing the host -> device copies, the three device-operation calls,
- * enqueueing the device -> host copy of the output, and the wait for the
- * stream; total_us spans the whole call. The device runs the copies and
- * kernels between the first enqueue and the end of the wait. */
+ * enqueueing the metadata copy and the copy-on-write block copies,
+ * enqueueing the row chunks' chains (q/k/v copies, append, decode, output
+ * copy), and the wait for the stream; total_us spans the whole call; chunks is
+ * the number of row chunks the batch was cut into. The device runs the copies
+ * and kernels between the first enqueue and the end of the wait. */
 typedef struct {
   double block_manager_us;
-  double h2d_enqueue_us;
-  double launch_us;
-  double d2h_enqueue_us;
+  double metadata_enqueue_us;
+  double chains_enqueue_us;
   double wait_us;
   double total_us;
+  int32_t chunks;
 } pa_step_timing;
 
 pa_status pa_step_host_last_timing(pa_step_timing* out);

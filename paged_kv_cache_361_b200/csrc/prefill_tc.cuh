@@ -26,29 +26,32 @@
 //   warps 0-3  one thread per row (TMEM lane): load the row's Q into shared
 //              memory; per chunk read S from TMEM, mask causally, keep the
 //              running maximum m and sum l in base 2, write P back into the
-//              S buffer as a bf16 high part and a bf16 remainder (two MMAs
-//              for P V keep ~16 mantissa bits of each weight); at the end read
-//              O, divide by l, store fp32.
+//              S buffer as f16 (11 significant bits; weights are at most
+//              2^8); at the end read O, divide by l, store fp32.
+//   warps +2..+5  converter: a kind::f16 MMA takes A and B of one type, so
+//              with P in f16 the V operand must be f16 too. The converter
+//              rewrites each stage's V tile in place, bf16 -> f16 (exact for
+//              normal f16 values, |v| <= 65504; values below 2^-14 keep their
+//              f16 subnormal bits, an absolute change below 2^-25), and writes
+//              rows past the stream's last key as zeros (their bytes may be
+//              padding or NaN), then releases the stage's V to the MMA warp.
+//              S = Q K^T stays bf16 x bf16 (Q and K straight from the cache).
 // The running maximum is moved (and O rescaled in TMEM) only when a row's
 // maximum grows by more than 8 in log2 units, so weights stay below 2^8 and
 // most chunks never touch O; the result is the same softmax.
 //
 // 8-bit cache (CF: e4m3 or int8 codes). P3 = "PagedAttention 和 vLLM", the
 // section on its future: paged KV storage combined with quantisation, a code c
-// standing for value(c) * scale with one scale per tensor. A kind::f16 MMA
-// takes A and B of one type, so the keys and values are widened to f16 (cvt
-// e4m3x2 -> f16x2, or the int8 byte-permute widening; both exact) by a fourth
-// role:
-//   warps +2..+5  converter: the producer copies [bs x D] byte boxes of codes
-//              (128-byte swizzle at D 128, 64-byte at D 64) into a small
-//              staging ring; the converter writes each chunk as f16 K and V
-//              tiles in the swizzled layout the bf16 path gets from the TMA,
-//              with rows past the stream's last key written as zeros (their
-//              bytes may be anything, a NaN code included).
+// standing for value(c) * scale with one scale per tensor. The keys and values
+// are widened to f16 (cvt e4m3x2 -> f16x2, or the int8 byte-permute widening;
+// both exact) by the converter role: the producer copies [bs x D] byte boxes
+// of codes (128-byte swizzle at D 128, 64-byte at D 64) into a small staging
+// ring; the converter writes each chunk as f16 K and V tiles in the swizzled
+// layout the bf16 path gets from the TMA, with rows past the stream's last key
+// written as zeros (their bytes may be anything, a NaN code included).
 // Q is rounded to f16 by the softmax warps as they stage it (exact for
-// 2^-17 <= |q| <= 65504); P is written as f16 (11 mantissa bits, one P V MMA
-// per k-step instead of the bf16 high/low pair). The K scale is folded into
-// the score scale; the V scale multiplies O in the final division.
+// 2^-17 <= |q| <= 65504). The K scale is folded into the score scale; the V
+// scale multiplies O in the final division.
 #pragma once
 
 #include "decode_f8.cuh"
@@ -56,6 +59,12 @@
 #include "tcgen05.cuh"
 
 namespace pa {
+
+// Build-time knob: K/V stages of the bf16 path (64 keys each; 5 still fits
+// beside two Q tiles at head_dim 128).
+#ifndef PA_TC_STAGES
+#define PA_TC_STAGES 4
+#endif
 
 template <int D, int TILES, bool F8 = false>
 struct TcCfg {
@@ -65,7 +74,7 @@ struct TcCfg {
   static constexpr int kHalfBytes = kChunk * 128;          // one box column of K or V in a stage
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage (16-bit elements)
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = F8 && TILES > 1 ? 3 : 4;
+  static constexpr int kStages = F8 && TILES > 1 ? 3 : PA_TC_STAGES;
   static constexpr int kCodeTileBytes = kChunk * D;        // 8-bit K (or V) codes of one staging slot
   static constexpr int kCodeStageBytes = 2 * kCodeTileBytes;
   static constexpr int kCodeStages = F8 ? (TILES > 1 ? 2 : 3) : 0;
@@ -77,7 +86,7 @@ struct TcCfg {
   static constexpr int kProducerWarp = kSoftmaxWarps;
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
   static constexpr int kConvWarp0 = kSoftmaxWarps + 2;
-  static constexpr int kConvWarps = F8 ? 4 : 0;
+  static constexpr int kConvWarps = 4;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kConvWarps);
   // per tile: O (D columns), then two S/P buffers of kChunk columns
   static constexpr uint32_t kTileCols = D + 2 * kChunk;
@@ -85,6 +94,32 @@ struct TcCfg {
   static_assert(TILES * kTileCols <= kTmemCols, "TMEM columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
+
+// One row of a stage's V tile (64 keys x D, bf16, as the TMA wrote it:
+// [rows x 64] box columns of 128-byte rows with the 128-byte swizzle,
+// kHalfBytes apart), rewritten in place as f16: the box column `half` at
+// D 128, or the half `half` of the single 128-byte row at D 64. live = false
+// writes zeros. At D 128 the two box columns of a row are handled by
+// neighbouring lanes; half 1 walks its 16-byte chunks in rotated order so that
+// the eight lanes of a shared-memory phase touch eight different chunk
+// positions (at D 64 the two halves already do).
+template <int D, int kHalfBytes>
+__device__ __forceinline__ void v_to_f16_inplace(uint8_t* vt, int row, int half, bool live) {
+  constexpr int NCH = D == 128 ? 8 : 4;  // 16-byte chunks per thread
+  uint8_t* rp = vt + (D == 128 ? half * kHalfBytes : 0) + row * 128;
+#pragma unroll
+  for (int u0 = 0; u0 < NCH; ++u0) {
+    const int c = D == 128 ? (half ? (u0 ^ 4) : u0) : half * 4 + u0;  // logical chunk of the 128-byte row
+    uint4* ptr = reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4));
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (live) {
+      const uint4 x = *ptr;
+      w = make_uint4(pack_f16(bf16lo(x.x), bf16hi(x.x)), pack_f16(bf16lo(x.y), bf16hi(x.y)),
+                     pack_f16(bf16lo(x.z), bf16hi(x.z)), pack_f16(bf16lo(x.w), bf16hi(x.w)));
+    }
+    *ptr = w;
+  }
+}
 
 // All lanes wait; the warp proceeds only if every lane saw the phase.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -107,6 +142,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ PipeSmem<S> ps;  // 16-bit K/V stages: filled by the TMA (bf16) or the converter (F8)
   __shared__ uint64_t cfull[CS], cempty[CS];  // F8: code staging ring, producer <-> converter
+  __shared__ uint64_t vready[S];              // bf16: the stage's V rewritten as f16 (converter -> MMA)
   __shared__ uint64_t q_full, drain;
   __shared__ uint64_t s_full[TILES][2], p_full[TILES][2], o_bar[TILES];
   __shared__ uint32_t tmem_base_sh;
@@ -174,6 +210,8 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       ps.abort_flag = 0;
       fence_mbar_init();
     } else {
+#pragma unroll
+      for (int i = 0; i < S; ++i) mbar_init(&vready[i], Cfg::kConvWarps);
       pipe_init<S>(ps, 1);  // empty stages are released by one tcgen05.commit
     }
   }
@@ -238,6 +276,21 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         mbar_arrive(&cempty[cst]);
       }
     }
+  } else if (!F8 && warp >= Cfg::kConvWarp0) {
+    // ---- converter (bf16): the stage's V tile, bf16 -> f16 in place; thread =
+    // (row of the chunk, box column at D 128 / half of the row at D 64) ----
+    const int ct = tid - 32 * Cfg::kConvWarp0;
+    const int row = ct >> 1, half = ct & 1;
+    uint8_t* kv0g = sgen + Cfg::kQBytes;
+    for (int i = 0; i < nchunks; ++i) {
+      const int st = i % S;
+      if (!warp_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
+      const bool live = i * C + row < kend_all;  // rows past the last key become zeros
+      v_to_f16_inplace<D, Cfg::kHalfBytes>(kv0g + st * Cfg::kStageBytes + Cfg::kTileBytes, row, half, live);
+      tc::fence_proxy_async();  // generic-proxy writes -> tensor-core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&vready[st]);
+    }
   } else if (warp == Cfg::kProducerWarp) {
     // ---- producer ----
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
@@ -271,7 +324,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
     // whole warp walks the schedule and waits, one elected lane issues ----
     {
       constexpr uint32_t kIdS = F8 ? tc::idesc_f16(Cfg::kRows, C, false) : tc::idesc_bf16(Cfg::kRows, C, false);
-      constexpr uint32_t kIdPV = F8 ? tc::idesc_f16(Cfg::kRows, D, true) : tc::idesc_bf16(Cfg::kRows, D, true);
+      constexpr uint32_t kIdPV = tc::idesc_f16(Cfg::kRows, D, true);  // P and V as f16
       // Descriptors are built once; an operand at a byte offset from a base
       // is the base descriptor plus offset / 16 (the start-address field,
       // addresses stay below 256 KB so the field never carries over).
@@ -300,12 +353,11 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         // kHalfBytes apart (one half when D = 64: the offset is then unused)
         const uint64_t vb = vdesc0 + static_cast<uint64_t>(((j % S) * Cfg::kStageBytes) >> 4);
         const uint32_t to = tmem + t * Cfg::kTileCols;
-        const uint32_t tp = to + D + sb * C;  // P (bf16 high part, or f16): 32 columns; bf16 remainder: the next 32
+        const uint32_t tp = to + D + sb * C;  // P as f16: 32 columns
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks) {
           const uint64_t bd = vb + static_cast<uint64_t>((ks * 16 * 128) >> 4);
           tc::mma_ts(to, tp + ks * 8, bd, kIdPV, j > 0 || ks > 0);
-          if constexpr (!F8) tc::mma_ts(to, tp + C / 2 + ks * 8, bd, kIdPV, true);
         }
         tc::commit(smem_u32(&o_bar[t]));
         return true;
@@ -328,6 +380,14 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
 #pragma unroll
           for (int t = 0; t < TILES; ++t)
             if (j + 1 < nch[t]) issue_s(t, j + 1);
+        }
+        if constexpr (!F8) {
+          // the converter has rewritten this stage's V as f16
+          if (!warp_wait(&vready[j % S], (j / S) & 1, &ps.abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
         }
 #pragma unroll
         for (int t = 0; t < TILES; ++t)
@@ -368,16 +428,6 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&q_full);
       }
-      // the stream's last chunk holds rows past its last key; the lowest tile
-      // that reads that chunk zeroes their V before any P V reads them (the
-      // converter writes them as zeros on the F8 path)
-      bool zero_tail = false;
-#pragma unroll
-      for (int u = 0; u < (F8 ? 0 : TILES); ++u)
-        if (nch[u] == nchunks) {
-          zero_tail = u == t;
-          break;
-        }
       const uint32_t trow = tmem + t * Cfg::kTileCols + (static_cast<uint32_t>((warp & 3) * 32) << 16);
       const float sl2 = a.scale_log2;
       float m_ref = -INFINITY, l = 0.f;  // m_ref in scaled (log2) units
@@ -395,25 +445,22 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         tc::wait_ld();
         const int32_t k0 = j * C;
         float x[C];
-        // the row maximum over 8 independent partial maxima (short dependence chains)
-        float pm[8];
+        // the row maximum over 4 independent partial maxima (three-input max:
+        // short dependence chains, one instruction per two scores)
+        float pm[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+        for (int u = 0; u < 4; ++u) pm[u] = -INFINITY;
         // warp-uniform choice: tcgen05.ld/st below need the whole warp converged
         if (__all_sync(0xffffffffu, k0 + C - 1 <= pos)) {
 #pragma unroll
-          for (int c = 0; c < C; ++c) {
-            x[c] = __uint_as_float(sr[c]);
-            pm[c & 7] = fmaxf(pm[c & 7], x[c]);
-          }
+          for (int c = 0; c < C; ++c) x[c] = __uint_as_float(sr[c]);
         } else {
 #pragma unroll
-          for (int c = 0; c < C; ++c) {
-            x[c] = k0 + c <= pos ? __uint_as_float(sr[c]) : -INFINITY;
-            pm[c & 7] = fmaxf(pm[c & 7], x[c]);
-          }
+          for (int c = 0; c < C; ++c) x[c] = k0 + c <= pos ? __uint_as_float(sr[c]) : -INFINITY;
         }
-        float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+#pragma unroll
+        for (int c = 0; c < C / 2; ++c) pm[c & 3] = fmax3(pm[c & 3], x[2 * c], x[2 * c + 1]);
+        float mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
         mx *= sl2;  // scale > 0 keeps the order
         float alpha = 1.f;
         bool resc = false;
@@ -423,22 +470,21 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
           m_ref = mx;
           resc = j > 0;
         }
-        uint32_t ph[C / 2], pl[C / 2];
-        float part[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums (short dependence chains)
+        uint32_t ph[C / 2];
+        // weights as packed pairs: (x0, x1) * scale - m in one instruction, the
+        // sums in two packed partial sums (short dependence chains)
+        const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
+        float2 part[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < C / 2; ++c) {
-          const float p0 = fast_exp2(fmaf(x[2 * c], sl2, -m_ref));
-          const float p1 = fast_exp2(fmaf(x[2 * c + 1], sl2, -m_ref));
-          part[c & 3] += p0 + p1;
-          if constexpr (F8)
-            ph[c] = pack_f16(p0, p1);  // weights <= 2^8
-          else
-            split_pair(p0, p1, ph[c], pl[c]);
+          const float2 y = ffma2(make_float2(x[2 * c], x[2 * c + 1]), sc2, nm2);
+          const float2 pp = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          part[c & 1] = fadd2(part[c & 1], pp);
+          ph[c] = pack_f16(pp.x, pp.y);  // weights <= 2^8
         }
-        l += (part[0] + part[1]) + (part[2] + part[3]);
+        l += (part[0].x + part[0].y) + (part[1].x + part[1].y);
         __syncwarp();
         tc::st32(trow + D + sb * C, ph);
-        if constexpr (!F8) tc::st32(trow + D + sb * C + C / 2, pl);
         if (__any_sync(0xffffffffu, resc)) {
           // O must hold P(j-1) V(j-1) before it is rescaled (P(j-2) V(j-2) is
           // complete: it was issued before S(j), which this chunk waited for)
@@ -461,21 +507,6 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
             __syncwarp();
             tc::st32(trow + q * 32, o);
           }
-        }
-        if (zero_tail && j == nchunks - 1 && kend_all - k0 < C) {
-          // V rows past the last key may hold anything (unloaded or padding);
-          // 0 * NaN would reach O, so they are zeroed before P V reads them.
-          const int nvk = kend_all - k0;
-          const int chunks16 = (C - nvk) * Cfg::kHalves * 8;
-          uint8_t* vst = sgen + Cfg::kQBytes + (j % S) * Cfg::kStageBytes + Cfg::kTileBytes;
-          tc::fence_proxy_async();
-          for (int i = r; i < chunks16; i += 128) {
-            const int row = nvk + i / (Cfg::kHalves * 8);
-            const int rem = i % (Cfg::kHalves * 8);
-            *reinterpret_cast<uint4*>(vst + (rem >> 3) * Cfg::kHalfBytes + row * 128 + (rem & 7) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          tc::fence_proxy_async();
         }
         __syncwarp();
         tc::wait_st();

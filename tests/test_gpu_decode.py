@@ -301,6 +301,26 @@ def test_prefill_long_chunk_many_tiles(G, D):
     assert err <= TOL["bf16"], err
 
 
+@pytest.mark.parametrize("vscale", [2000.0, 1e-3])
+def test_prefill_value_range_through_f16(vscale):
+    """The prefill reads V as f16 (its P V product is f16 x f16): V rows scaled
+    to |v| of a few thousand, or down to about 1e-3, come out within the bf16
+    tolerance scaled by the same factor."""
+    from oracle.prefill import prefill_attention
+    hkv, bs, D, G = 2, 16, 128, 4
+    g = torch.Generator().manual_seed(77)
+    n = 300
+    cache = PagedKVCache(-(-n // bs) + 2, hkv, bs, D, torch.bfloat16, "cuda", fill=float("nan"))
+    K = torch.randn(n, hkv, D, generator=g).bfloat16()
+    V = (torch.randn(n, hkv, D, generator=g) * vscale).bfloat16()
+    q = torch.randn(n, hkv * G, D, generator=g).bfloat16()
+    out = cache.prefill([0], [n], q.cuda(), K.cuda(), V.cuda(), D ** -0.5).cpu()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    ref = prefill_attention(q, K, V, D ** -0.5)
+    err = float(np.abs(out.double().numpy() - ref).max())
+    assert err <= TOL["bf16"] * vscale, err
+
+
 def test_prefill_then_decode_consistent():
     """The last token of a whole-prompt prefill equals a decode over the same cache."""
     sh = (4, 128, 16)
@@ -341,3 +361,117 @@ def test_step_plan_matches_oracle():
         for i, s in enumerate(ids):
             exp = ref.attend(s, q[i], 0.125, use_pool=True)
             assert float(np.abs(out[i].double().numpy() - exp).max()) <= TOL["bf16"]
+
+
+def test_swap_copy_engine_equals_kernel_swap():
+    """pa_swap_blocks_copy (copy engines, host pairs; runs of consecutive ids
+    merged into one copy) moves the same bytes as the pa_swap_blocks kernel."""
+    g = torch.Generator().manual_seed(9)
+    kc = torch.randn(40, 2, 16, 64, generator=g).bfloat16().cuda()
+    vc = torch.randn(40, 2, 16, 64, generator=g).bfloat16().cuda()
+    shape = (24, 2, 16, 64)
+    hk1, hv1 = (torch.zeros(shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(2))
+    hk2, hv2 = (torch.zeros(shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(2))
+    # scattered ids plus a run of five consecutive (device, host) pairs
+    pairs = np.array([[7, 3], [30, 0], [11, 12], [12, 13], [13, 14], [14, 15], [15, 16], [2, 23], [39, 1]],
+                     dtype=np.int32)
+    B.pa_swap_blocks(kc, vc, hk1, hv1, torch.from_numpy(pairs).cuda(), True)
+    B.pa_swap_blocks_copy(kc, vc, hk2, hv2, pairs, True)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(hk1), bits(hk2)) and torch.equal(bits(hv1), bits(hv2))
+    assert torch.equal(bits(hk2[pairs[:, 1]]), bits(kc[pairs[:, 0]].cpu()))
+    # and back into other device blocks
+    back = np.stack([pairs[:, 1], np.arange(20, 29, dtype=np.int32)], 1)
+    kc2, vc2 = kc.clone(), vc.clone()
+    B.pa_swap_blocks(kc, vc, hk1, hv1, torch.from_numpy(back).cuda(), False)
+    B.pa_swap_blocks_copy(kc2, vc2, hk2, hv2, back, False)
+    torch.cuda.synchronize()
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    assert torch.equal(bits(kc), bits(kc2)) and torch.equal(bits(vc), bits(vc2))
+
+
+def test_swap_copy_engine_checks_ids_on_the_host():
+    kc = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
+    hk = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16, pin_memory=True)
+    for bad in ([[0, 4]], [[4, 0]], [[-1, 0]]):
+        with pytest.raises(B.PagedAttnError) as e:
+            B.pa_swap_blocks_copy(kc, kc, hk, hk, np.array(bad, np.int32), True)
+        assert e.value.status == B.PA_ERR_INVALID_ARG
+    pageable = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(B.PagedAttnError) as e:
+        B.pa_swap_blocks_copy(kc, kc, pageable, pageable, np.array([[0, 1]], np.int32), True)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+def test_step_host_phase_timers():
+    g = torch.Generator().manual_seed(4)
+    cache = PagedKVCache(64, 2, 16, 128, torch.bfloat16, "cuda")
+    for s in range(3):
+        cache.add_sequence(s, torch.randn(50, 2, 128, generator=g).bfloat16().cuda(),
+                           torch.randn(50, 2, 128, generator=g).bfloat16().cuda())
+    q = torch.randn(3, 8, 128, generator=g).bfloat16().pin_memory()
+    k = torch.randn(3, 2, 128, generator=g).bfloat16().pin_memory()
+    out = torch.empty(3, 8, 128, pin_memory=True)
+    cache.step_host([0, 1, 2], q, k, k, out)
+    t = B.pa_step_host_last_timing()
+    parts = ("block_manager_us", "metadata_enqueue_us", "chains_enqueue_us", "wait_us")
+    assert all(t[p] >= 0 for p in parts) and t["total_us"] > 0 and t["chunks"] == 1
+    assert sum(t[p] for p in parts) <= t["total_us"] * 1.0001 + 1e-3
+
+
+@pytest.mark.parametrize("dtype,G", [("f32", 1), ("bf16", 1), ("bf16", 4), ("bf16", 8)])
+def test_last_cta_merge_and_merge_kernel_agree_with_oracle(dtype, G):
+    """Few partitions (2..7) are merged by the last CTA of each (sequence, kv
+    head); many by the merge kernel. Both against the oracle."""
+    sh = W.Shape(2 * G, 2, 128, 16, dtype)
+    w = W.random_small(31 + G, num_seqs=5, shape=sh, max_len=700)
+    for P in (128, 16):   # <= 6 partitions of 128 tokens; up to 44 of 16
+        r = Replay(sh, w.num_blocks, w.free_order, w.scale, partition_tokens=P).run(W.simple_ops(w))
+        r.check_outputs()
+
+
+@pytest.mark.parametrize("n,G", [(16, 4), (37, 1), (64, 8)])
+def test_step_host_chunked_matches_oracle(n, G):
+    """A batch of 16 or more sequences runs as row chunks on the library's own
+    streams (copies of one chunk overlap another's kernels); families of forked
+    sequences make the first step copy shared blocks. Slots, pairs, tables and
+    every output row match the oracle over three steps, one of them split."""
+    from oracle.replay import OracleRun
+    hkv, D, bs = 2, 128, 16
+    sh = W.Shape(hkv * G, hkv, D, bs, "bf16")
+    rng = np.random.default_rng(n * 10 + G)
+    nb = 24 * n
+    order = rng.permutation(nb)
+    ref = OracleRun(sh, nb, order, keep_pool=True)
+    cache = PagedKVCache(nb, hkv, bs, D, torch.bfloat16, "cuda", order, fill=float("nan"))
+    g = torch.Generator().manual_seed(n + G)
+    ids = []
+    s = 0
+    while len(ids) < n:
+        L = int(rng.integers(1, 300))
+        k = torch.randn(L, hkv, D, generator=g).bfloat16()
+        v = torch.randn(L, hkv, D, generator=g).bfloat16()
+        ref.apply(("add", s, L, lambda which, device="cpu", k=k, v=v: k if which == "k" else v))
+        cache.add_sequence(s, k.cuda(), v.cuda())
+        ids.append(s)
+        for j in range(int(rng.integers(0, 3))):   # forks share the prompt's blocks
+            if len(ids) < n:
+                ref.apply(("fork", s, s + 1 + j))
+                cache.fork(s, s + 1 + j)
+                ids.append(s + 1 + j)
+        s += 10
+    ids = [int(x) for x in rng.permutation(ids)]
+    for step in range(3):
+        q = torch.randn(n, hkv * G, D, generator=g).bfloat16().pin_memory()
+        k = torch.randn(n, hkv, D, generator=g).bfloat16().pin_memory()
+        v = torch.randn(n, hkv, D, generator=g).bfloat16().pin_memory()
+        out = torch.full((n, hkv * G, D), float("nan"), dtype=torch.float32).pin_memory()
+        ref.apply(("append", ids, lambda which, device="cpu", k=k, v=v: k if which == "k" else v))
+        cache.step_host(ids, q, k, v, out, D ** -0.5, partition_tokens=64 if step == 1 else -1)
+        assert B.pa_step_host_last_timing()["chunks"] == min(4, n // 8)
+        for i, sid in enumerate(ids):
+            exp = ref.attend(sid, q[i], D ** -0.5, use_pool=True)
+            assert float(np.abs(out[i].double().numpy() - exp).max()) <= TOL["bf16"], (step, sid)
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    for sid in ids:
+        assert cache.bm.block_table(sid)[0].tolist() == ref.bm.block_table(sid)
