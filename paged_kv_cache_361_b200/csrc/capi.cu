@@ -63,6 +63,9 @@ int32_t resolve_partition(int32_t num_seqs, int32_t hkv, int32_t max_ctx, int32_
   return P >= max_ctx ? 0 : static_cast<int32_t>(P);
 }
 
+// Split decodes with fewer partitions than this merge in their last CTA.
+constexpr int32_t kFuseMergeMaxParts = 8;
+
 int32_t num_parts(int32_t max_ctx, int32_t P) {
   if (P <= 0 || max_ctx <= 0) return 1;
   return (max_ctx + P - 1) / P;
@@ -268,8 +271,17 @@ bool mma_eligible(const pa_cache* c, int G) {
 // Persistent CTAs pay off when long sequences are cut into many short, equal
 // partitions (measured on a B200: 512-token partitions of 32k-131k contexts
 // gain ~12 %); with few or unequal work items one CTA per item balances better.
+// (The continuous-batching trace, 1024-token partitions of 256 sequences,
+// gained 6 % over one CTA per item.)
+#ifndef PA_MMA_PERSIST_MIN_PARTS
+#define PA_MMA_PERSIST_MIN_PARTS 2
+#endif
+bool mma_persistent(const DecodeArgs& a) {
+  return a.part_tokens > 0 && a.part_tokens <= 1024 && a.max_parts >= PA_MMA_PERSIST_MIN_PARTS;
+}
+
 pa_status dispatch_mma(const DecodeArgs& a, const pa_cache* c, int G, cudaStream_t st) {
-  const bool persistent = a.part_tokens > 0 && a.part_tokens <= 1024 && a.max_parts >= 8;
+  const bool persistent = mma_persistent(a);
   if (c->head_dim == 128)
     return G == 8 ? launch_mma<128, 8>(a, c, persistent, st) : launch_mma<128, 4>(a, c, persistent, st);
   return G == 8 ? launch_mma<64, 8>(a, c, persistent, st) : launch_mma<64, 4>(a, c, persistent, st);
@@ -796,6 +808,16 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(cache->num_kv_heads, num_seqs, parts);
   const int D = cache->head_dim;
+  // With few partitions per sequence the CTA that finishes a (sequence, kv
+  // head) last merges its partials (no merge launch); many partitions keep the
+  // merge kernel, which spreads the rows over the whole GPU.
+  if (parts > 1 && parts < kFuseMergeMaxParts) {
+    a.fuse_merge = 1;
+    // (the persistent kernel's launch clears the counters itself)
+    if (!(mma_eligible(cache, G) && mma_persistent(a)) &&
+        cudaMemsetAsync(a.counters, 0, counters_bytes(num_seqs, cache->num_kv_heads), s) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
   if (mma_eligible(cache, G)) {
     st = dispatch_mma(a, cache, G, s);
   } else if (f8_mma_eligible(cache)) {
@@ -809,7 +831,7 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   } else {
     st = D == 128 ? dispatch_g<float, 128>(a, G, grid, s) : dispatch_g<float, 64>(a, G, grid, s);
   }
-  if (st != PA_OK || parts <= 1) return st;
+  if (st != PA_OK || parts <= 1 || a.fuse_merge) return st;
   return D == 128 ? launch_reduce<128>(a, s) : launch_reduce<64>(a, s);
 }
 

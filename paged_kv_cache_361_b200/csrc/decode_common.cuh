@@ -39,6 +39,9 @@ struct DecodeArgs {
   int32_t force_partials;
   int32_t parts_stride;  // partial slots per (sequence, query head) row
   int32_t prefix_part_tokens;  // tokens per prefix partial (cascade only)
+  // Split sequences merged by the CTA that finishes last: each CTA counts its
+  // arrival in counters[1 + s * hkv + g] (zeroed before the launch).
+  int32_t fuse_merge = 0;
 };
 
 // First token a decode CTA covers for sequence s (the cascade suffix start).
@@ -239,6 +242,39 @@ __device__ __forceinline__ void pipe_produce(PipeSmem<S>& ps, int nchunks, Issue
   }
 }
 
+// Arrival of one partition of (sequence s, kv head g) whose partials are
+// stored and fenced; true for the last of its nparts partitions.
+__device__ __forceinline__ bool count_arrival(const DecodeArgs& a, int s, int g, int nparts) {
+  const unsigned prev = atomicAdd(a.counters + 1 + static_cast<int64_t>(s) * a.hkv + g, 1u);
+  __threadfence();
+  return prev == static_cast<unsigned>(nparts - 1);
+}
+
+// The same log-sum-exp merge as decode_reduce_kernel, over the nparts
+// partials of the G heads of kv head hq0 / G of sequence s, by threads
+// tid = 0 .. nthreads-1, straight into out. The partials were written by other
+// CTAs: read through L2 after the arrivals.
+template <int G, int D>
+__device__ __forceinline__ void merge_partials_to_out(const DecodeArgs& a, int s, int hq0, int nparts, int tid,
+                                                      int nthreads) {
+  __threadfence();
+  for (int idx = tid; idx < G * D; idx += nthreads) {
+    const int h = idx / D, d = idx - h * D;
+    const int64_t row = static_cast<int64_t>(s) * a.hq + hq0 + h;
+    const float* ml = a.ws_ml + row * a.parts_stride * 2;
+    const float* po = a.ws_o + row * a.parts_stride * D + d;
+    float M = -INFINITY;
+    for (int q = 0; q < nparts; ++q) M = fmaxf(M, __ldcg(ml + 2 * q));
+    float l = 0.f, o = 0.f;
+    for (int q = 0; q < nparts; ++q) {
+      const float f = exp2f(__ldcg(ml + 2 * q) - M);
+      l = fmaf(__ldcg(ml + 2 * q + 1), f, l);
+      o = fmaf(__ldcg(po + static_cast<int64_t>(q) * D), f, o);
+    }
+    a.out[row * D + d] = o / l;
+  }
+}
+
 // Merge the consumer warps' (m, l, o) for the G heads of this CTA and store
 // either the final row (one partition) or the partition's partials.
 //   wm, wl: [NW][G];  wacc: [NW][G][D]
@@ -270,6 +306,14 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const
       }
     }
   }
+  if (!a.fuse_merge || nparts == 1) return;
+  // Merge in the last CTA of this (sequence, kv head).
+  __shared__ int is_last;
+  __threadfence();  // this thread's partials are visible device-wide ...
+  __syncthreads();  // ... for every thread of the CTA, before the arrival counts
+  if (tid == 0) is_last = count_arrival(a, s, hq0 / G, nparts);
+  __syncthreads();
+  if (is_last) merge_partials_to_out<G, D>(a, s, hq0, nparts, tid, nthreads);
 }
 
 // Merge the partitions of one (sequence, query head):
@@ -321,20 +365,38 @@ __global__ void __launch_bounds__(32 * kReduceWarps) decode_reduce_kernel(const 
     float l = 0.f, acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-    for (int q = warp; q < nparts; q += kReduceWarps) {
-      const int sq = slot(q);
-      const float f = exp2f(ml[2 * sq] - M);
-      l = fmaf(ml[2 * sq + 1], f, l);
-      const float* src = o + static_cast<int64_t>(sq) * D + lane * VEC;
-      if (VEC == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] = fmaf(x.x, f, acc[0]);
-        acc[1] = fmaf(x.y, f, acc[1]);
-        acc[2] = fmaf(x.z, f, acc[2]);
-        acc[3] = fmaf(x.w, f, acc[3]);
-      } else {
+    // kUnroll partitions per warp per round: their loads are all in flight
+    // before the first one is folded in (a long sequence has hundreds)
+    constexpr int kUnroll = 4;
+    for (int q0 = warp; q0 < nparts; q0 += kUnroll * kReduceWarps) {
+      float mp[kUnroll], lp[kUnroll], x[kUnroll][VEC];
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] = fmaf(src[e], f, acc[e]);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int q = q0 + u * kReduceWarps;
+        mp[u] = -INFINITY;
+        lp[u] = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) x[u][e] = 0.f;
+        if (q < nparts) {
+          const int sq = slot(q);
+          mp[u] = ml[2 * sq];
+          lp[u] = ml[2 * sq + 1];
+          const float* src = o + static_cast<int64_t>(sq) * D + lane * VEC;
+          if (VEC == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            x[u][0] = v.x, x[u][1] = v.y, x[u][2] = v.z, x[u][3] = v.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) x[u][e] = src[e];
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const float f = exp2f(mp[u] - M);  // 0 for the empty slots of the last round
+        l = fmaf(lp[u], f, l);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] = fmaf(x[u][e], f, acc[e]);
       }
     }
     if (lane == 0) wl[warp] = l;

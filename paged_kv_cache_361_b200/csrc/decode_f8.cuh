@@ -42,6 +42,32 @@
 
 namespace pa {
 
+// Build-time tuning knobs, defaults measured on B200 (e4m3 metric workload:
+// 0.1278 ms with q fragments in registers, 4 stages and 3 CTAs per SM; 0.1219 ms
+// with all four below): split each QK^T accumulation chain in two; the q
+// fragments read from shared memory at every k-step and V one 32-bit word at
+// a time (fewer registers); 3 stages; the register budget fitted to 4 CTAs per
+// SM (96 registers, a few spilled words).
+#ifndef PA_F8_SPLIT_CHAINS
+#define PA_F8_SPLIT_CHAINS 1
+#endif
+#ifndef PA_F8_MIN_CTAS
+#define PA_F8_MIN_CTAS 4
+#endif
+#ifndef PA_F8_LEAN
+#define PA_F8_LEAN 1
+#endif
+#ifndef PA_F8_STAGES
+#define PA_F8_STAGES 3
+#endif
+// A minimum-CTA bound changes ptxas's register choice even when it is 1, so
+// 0 leaves it out.
+#if PA_F8_MIN_CTAS > 0
+#define PA_F8_LAUNCH_BOUNDS(n) __launch_bounds__(n, PA_F8_MIN_CTAS)
+#else
+#define PA_F8_LAUNCH_BOUNDS(n) __launch_bounds__(n)
+#endif
+
 template <int D>
 struct F8Cfg {
   static constexpr int kConsumerWarps = 4;
@@ -49,8 +75,9 @@ struct F8Cfg {
   static constexpr int kChunk = 64;                 // tokens per stage
   static constexpr int kTileBytes = kChunk * D;     // K (or V) of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = 4;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;
+  static constexpr int kStages = PA_F8_STAGES;
+  static constexpr int kQSmemBytes = PA_F8_LEAN ? 32 * (D / 16) * 8 : 0;  // q fragments of every lane
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kQSmemBytes;
   static constexpr int kNT = D / 8;                 // output n-tiles
 };
 
@@ -153,6 +180,19 @@ __device__ __forceinline__ void mma_f16_rows8_chain(float (&d)[2], uint32_t a0, 
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
+// The q fragments of a lane for k-step kk: held in registers, or read from
+// shared memory (32 lanes' pairs per k-step).
+template <int D>
+struct QFragRegs {
+  uint32_t v[D / 16][2];
+  __device__ __forceinline__ uint2 operator()(int kk) const { return make_uint2(v[kk][0], v[kk][1]); }
+};
+struct QFragSmem {
+  const uint2* p;
+  int lane;
+  __device__ __forceinline__ uint2 operator()(int kk) const { return p[kk * 32 + lane]; }
+};
+
 // Output dim of n-tile j, column n.
 template <int D>
 __device__ __forceinline__ int f8_dim(int j, int n) {
@@ -160,10 +200,10 @@ __device__ __forceinline__ int f8_dim(int j, int n) {
 }
 
 // One consumer warp's 16 tokens (nv valid) of a stage.
-template <int D, int CF>
-__device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, int nv,
-                                         const uint32_t (&qa)[D / 16][2], float scale_log2, int lane, int warp,
-                                         float& m_run, float& l_run, float (&o)[D / 8][2]) {
+template <int D, int CF, class QFrag>
+__device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, int nv, const QFrag& qa,
+                                         float scale_log2, int lane, int warp, float& m_run, float& l_run,
+                                         float (&o)[D / 8][2]) {
   constexpr int NT = D / 8;
   const int gq = lane >> 2, c = lane & 3;
   const int tw = warp * 16;
@@ -172,6 +212,32 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
   // 0..6 (128-byte rows) or 0..5 (64-byte rows) clear, so the swizzled address
   // of 16-byte chunk kk is (row start | swizzle key << 4 | byte) ^ (kk << 4).
   const uint32_t kts = smem_u32(kt);
+#if PA_F8_LEAN
+  {
+    // both n-tiles per k-step, the k-step's q pair read from shared memory
+    float dead0[2] = {0.f, 0.f}, dead1[2] = {0.f, 0.f};
+    uint32_t rb[2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      sacc[nt][0] = sacc[nt][1] = 0.f;
+      const int row = tw + nt * 8 + gq;
+      const uint32_t key = D == 128 ? static_cast<uint32_t>(row & 7) : static_cast<uint32_t>((row >> 1) & 3);
+      rb[nt] = (kts + static_cast<uint32_t>(row * D)) | (key << 4) | static_cast<uint32_t>(4 * c);
+    }
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint2 qq = qa(kk);
+      uint32_t w0, w1;
+      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w0) : "r"(rb[0] ^ static_cast<uint32_t>(kk << 4)));
+      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w1) : "r"(rb[1] ^ static_cast<uint32_t>(kk << 4)));
+      uint32_t b00, b01, b10, b11;
+      widen4<CF>(w0, b00, b01);
+      widen4<CF>(w1, b10, b11);
+      mma_f16_rows8_chain(sacc[0], qq.x, qq.y, b00, b01, dead0);
+      mma_f16_rows8_chain(sacc[1], qq.x, qq.y, b10, b11, dead1);
+    }
+  }
+#else
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     sacc[nt][0] = sacc[nt][1] = 0.f;
@@ -179,15 +245,29 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
     const int row = tw + nt * 8 + gq;
     const uint32_t key = D == 128 ? static_cast<uint32_t>(row & 7) : static_cast<uint32_t>((row >> 1) & 3);
     const uint32_t rbase = (kts + static_cast<uint32_t>(row * D)) | (key << 4) | static_cast<uint32_t>(4 * c);
+#if PA_F8_SPLIT_CHAINS
+    // two accumulators per n-tile (even and odd k-steps): half the chain length
+    float s2[2] = {0.f, 0.f}, dead2[2] = {0.f, 0.f};
+#endif
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       uint32_t w;
       asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w) : "r"(rbase ^ static_cast<uint32_t>(kk << 4)));
       uint32_t b0, b1;
       widen4<CF>(w, b0, b1);
-      mma_f16_rows8_chain(sacc[nt], qa[kk][0], qa[kk][1], b0, b1, dead);
+#if PA_F8_SPLIT_CHAINS
+      if (kk & 1)
+        mma_f16_rows8_chain(s2, qa(kk).x, qa(kk).y, b0, b1, dead2);
+      else
+#endif
+        mma_f16_rows8_chain(sacc[nt], qa(kk).x, qa(kk).y, b0, b1, dead);
     }
+#if PA_F8_SPLIT_CHAINS
+    sacc[nt][0] += s2[0];
+    sacc[nt][1] += s2[1];
+#endif
   }
+#endif
   float sc[2][2];
   float mloc = -INFINITY;
 #pragma unroll
@@ -228,9 +308,17 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
   const uint32_t pa2 = pack_f16(pr[1][0], pr[1][1]);  // tokens 8+2c, 9+2c
 
   constexpr int W = D == 128 ? 4 : 2;  // 32-bit words of V per token this thread reads
-  uint32_t va[W], vb[W], vc[W], vd[W];
   const int col = (D == 128 ? 16 : 8) * gq;
   const int t00 = tw + 2 * c, t10 = tw + 8 + 2 * c;
+#if PA_F8_LEAN
+  // one 32-bit word of each of the four tokens' pieces at a time
+  const uint8_t* pa_ = vt + f8_off<D>(t00, col);
+  const uint8_t* pb_ = vt + f8_off<D>(t00 + 1, col);
+  const uint8_t* pc_ = vt + f8_off<D>(t10, col);
+  const uint8_t* pd_ = vt + f8_off<D>(t10 + 1, col);
+#define PA_VWORD(p, w) (*reinterpret_cast<const uint32_t*>((p) + 4 * (w)))
+#else
+  uint32_t va[W], vb[W], vc[W], vd[W];
   if constexpr (D == 128) {
     const uint4 x0 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t00, col));
     const uint4 x1 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t00 + 1, col));
@@ -250,15 +338,22 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
     vc[0] = x2.x, vc[1] = x2.y;
     vd[0] = x3.x, vd[1] = x3.y;
   }
+#endif
   const bool ragged = nv < 16;  // warp-uniform
 #pragma unroll
   for (int w = 0; w < W; ++w) {
     // (token a byte k, token b byte k) pairs: bytes 0,1 then 2,3 of each word
     uint32_t b[8];
-    widen4<CF>(__byte_perm(va[w], vb[w], 0x5140), b[0], b[1]);
-    widen4<CF>(__byte_perm(va[w], vb[w], 0x7362), b[2], b[3]);
-    widen4<CF>(__byte_perm(vc[w], vd[w], 0x5140), b[4], b[5]);
-    widen4<CF>(__byte_perm(vc[w], vd[w], 0x7362), b[6], b[7]);
+#if PA_F8_LEAN
+    const uint32_t xa = PA_VWORD(pa_, w), xb = PA_VWORD(pb_, w), xc = PA_VWORD(pc_, w), xd = PA_VWORD(pd_, w);
+#undef PA_VWORD
+#else
+    const uint32_t xa = va[w], xb = vb[w], xc = vc[w], xd = vd[w];
+#endif
+    widen4<CF>(__byte_perm(xa, xb, 0x5140), b[0], b[1]);
+    widen4<CF>(__byte_perm(xa, xb, 0x7362), b[2], b[3]);
+    widen4<CF>(__byte_perm(xc, xd, 0x5140), b[4], b[5]);
+    widen4<CF>(__byte_perm(xc, xd, 0x7362), b[6], b[7]);
     if (ragged) {
       // tokens past the valid ones: their V bytes may be NaN codes
       const uint32_t m0 = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
@@ -279,7 +374,7 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
 // 16 tokens of every 64-token stage; the warps' states are merged through
 // shared memory at the end.
 template <int D, int G, int CF>
-__global__ void __launch_bounds__(F8Cfg<D>::kThreads) decode_f8_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                        const __grid_constant__ CUtensorMap tmv,
                                                                        const DecodeArgs a) {
   using Cfg = F8Cfg<D>;
@@ -337,26 +432,38 @@ __global__ void __launch_bounds__(F8Cfg<D>::kThreads) decode_f8_kernel(const __g
   } else {
     // q rows as f16 A fragments in the dim order of f8_chunk's k-steps:
     // a0 = dims (16kk + 4c, +1), a2 = dims (16kk + 4c + 2, +3); rows >= G zero
-    uint32_t qa[D / 16][2];
+    QFragRegs<D> qa;
     const __nv_bfloat16* qrow =
         static_cast<const __nv_bfloat16*>(a.q) + (static_cast<int64_t>(s) * a.hq + hq0 + (r < G ? r : 0)) * D;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       if (r < G) {
         const uint2 w = __ldg(reinterpret_cast<const uint2*>(qrow + kk * 16 + 4 * c));
-        qa[kk][0] = pack_f16(bf16lo(w.x), bf16hi(w.x));
-        qa[kk][1] = pack_f16(bf16lo(w.y), bf16hi(w.y));
+        qa.v[kk][0] = pack_f16(bf16lo(w.x), bf16hi(w.x));
+        qa.v[kk][1] = pack_f16(bf16lo(w.y), bf16hi(w.y));
       } else {
-        qa[kk][0] = qa[kk][1] = 0u;
+        qa.v[kk][0] = qa.v[kk][1] = 0u;
       }
     }
+#if PA_F8_LEAN
+    // every consumer warp has the same fragments: warp 0 parks them in shared memory
+    uint2* qsm = reinterpret_cast<uint2*>(sgen + S * Cfg::kStageBytes);
+    if (warp == 0) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) qsm[kk * 32 + lane] = make_uint2(qa.v[kk][0], qa.v[kk][1]);
+    }
+    consumer_bar();
+    const QFragSmem qf{qsm, lane};
+#else
+    const QFragRegs<D>& qf = qa;
+#endif
     for (int i = 0; i < nchunks; ++i) {
       const int st = i % S;
       if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
       const int nv = min(16, min(C, pt.ntok - i * C) - warp * 16);  // warp-uniform
       if (nv > 0) {
         const uint8_t* kt = sgen + st * Cfg::kStageBytes;
-        f8_chunk<D, CF>(kt, kt + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
+        f8_chunk<D, CF>(kt, kt + Cfg::kTileBytes, nv, qf, a.scale_log2, lane, warp, m_run, l_run, o);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ps.empty[st]);

@@ -109,7 +109,14 @@ __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint3
 #define PA_MMA_STAGES 0
 #endif
 #ifndef PA_MMA_MIN_CTAS
-#define PA_MMA_MIN_CTAS 1
+#define PA_MMA_MIN_CTAS 0
+#endif
+// A minimum-CTA bound changes ptxas's register choice even when it is 1, so
+// the default (0) leaves it out.
+#if PA_MMA_MIN_CTAS > 0
+#define PA_MMA_LAUNCH_BOUNDS(n) __launch_bounds__(n, PA_MMA_MIN_CTAS)
+#else
+#define PA_MMA_LAUNCH_BOUNDS(n) __launch_bounds__(n)
 #endif
 
 template <int D>
@@ -250,6 +257,7 @@ struct PersistSmem {
   uint64_t cbar;  // consumer-warp barrier (one arrival per consumer warp)
   StageDesc desc[S];
   int abort_flag;
+  int merge_here;  // the item just finished completes its (sequence, kv head): merge it
 };
 
 // Barrier over the consumer warps built on an mbarrier, so that its wait is
@@ -471,13 +479,21 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
       PA_CSYNC();  // the fold slots are free again
       continue;
     }
-    // split sequence: publish this partition's (m, l, o); decode_reduce_kernel merges
+    // split sequence: publish this partition's (m, l, o); the last partition's
+    // consumers (fused merge) or decode_reduce_kernel merge them
     if (warp == 0 && r < G) {
       const int64_t prow = (row0 + r) * a.parts_stride + dp;
       float* dst = a.ws_o + prow * D + 2 * c;
 #pragma unroll
       for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
       if (c == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(m_run, lrow);
+    }
+    if (a.fuse_merge) {
+      __threadfence();
+      PA_CSYNC();
+      if (warp == 0 && lane == 0) ps.merge_here = count_arrival(a, ds, dg, dnp);
+      PA_CSYNC();
+      if (ps.merge_here) merge_partials_to_out<G, D>(a, ds, dg * G, dnp, tid, 32 * NW);
     }
     PA_CSYNC();  // the fold slots are free again
   }
@@ -489,7 +505,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
 // end every warp's (m, l, o) goes through shared memory (the stage ring is free
 // by then) and the CTA stores the row or the partition's partials.
 template <int D, int G>
-__global__ void __launch_bounds__(MmaCfg<D>::kThreads, PA_MMA_MIN_CTAS) decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const DecodeArgs a) {
   using Cfg = MmaCfg<D>;
