@@ -352,16 +352,16 @@ def pa_swap_blocks_copy(k_cache, v_cache, host_k, host_v, pairs: np.ndarray, to_
 
 
 class pa_step_timing(ctypes.Structure):
-    _fields_ = [("block_manager_us", ctypes.c_double), ("h2d_enqueue_us", ctypes.c_double),
-                ("launch_us", ctypes.c_double), ("d2h_enqueue_us", ctypes.c_double), ("wait_us", ctypes.c_double),
-                ("total_us", ctypes.c_double)]
+    _fields_ = [("block_manager_us", ctypes.c_double), ("metadata_enqueue_us", ctypes.c_double),
+                ("chains_enqueue_us", ctypes.c_double), ("wait_us", ctypes.c_double), ("total_us", ctypes.c_double),
+                ("chunks", ctypes.c_int32)]
 
 
 def pa_step_host_last_timing() -> dict:
     """Host phases (microseconds) of this thread's last pa_step_host call."""
     t = pa_step_timing()
     _check(_lib().pa_step_host_last_timing(ctypes.byref(t)), "pa_step_host_last_timing")
-    return {name: float(getattr(t, name)) for name, _ in pa_step_timing._fields_}
+    return {name: (int if name == "chunks" else float)(getattr(t, name)) for name, _ in pa_step_timing._fields_}
 
 
 def pa_selftest_wait_timeout(timeout_ns: int, stream=None):

@@ -123,3 +123,16 @@ def test_workspace_sizes():
         cnt(4, 8) + (rows * 8 + 255) // 256 * 256 + rows * 128 * 4
     P = B.pa_decode_partition_tokens(64, 32, 32, 2049, 16)
     assert P == 0 or P % 16 == 0
+
+
+def test_step_timing_and_copy_swap_host_checks():
+    lib = B._lib()
+    assert lib.pa_step_host_last_timing(None) == B.PA_ERR_INVALID_ARG
+    t = B.pa_step_host_last_timing()
+    assert t["total_us"] == 0.0            # no pa_step_host call on this thread
+    c = _cache()
+    pairs = (ctypes.c_int32 * 2)(0, 1)
+    assert lib.pa_swap_blocks_copy(ctypes.byref(c), 16, 16, 4, pairs, -1, 1, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_swap_blocks_copy(ctypes.byref(c), 16, 16, 0, pairs, 1, 1, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_swap_blocks_copy(ctypes.byref(c), 16, 16, 4, pairs, 0, 1, None) == B.PA_OK
+    assert lib.pa_swap_blocks_copy(ctypes.byref(c), None, 16, 4, pairs, 1, 1, None) == B.PA_ERR_INVALID_ARG
