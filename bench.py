@@ -454,7 +454,9 @@ def run_ours(args, rank, world, device):
         n_groups = int(cascade[0].shape[0]) - 1
         launches = args.steps * (1 + (1 if n_groups else 0) + 2 + (1 if d["pairs"] is not None else 0))
     else:
-        launches = args.steps * (2 + (1 if split else 0) + (1 if d["pairs"] is not None else 0))
+        # the merge kernel runs for 8 or more partitions; fewer are merged by the decode's last CTA
+        merge_kernel = split and math.ceil(d["max_len"] / P_eff) >= 8
+        launches = args.steps * (2 + (1 if merge_kernel else 0) + (1 if d["pairs"] is not None else 0))
     dtype_key = str(d["kc"].dtype).replace("torch.", "")
     traffic, traffic_src = (None, "not captured for the cascade path") if cascade is not None else \
         ncu_traffic((args.workload, dtype_key, P_eff))
@@ -701,7 +703,11 @@ def prefill_record(B, workload, kv_dtype, steps, warmup, device, rank=0):
     pf, total = time_calls(lambda: B.pa_reshape_and_cache(k, v, slots, cache.k_cache, cache.v_cache),
                            lambda: B.pa_prefill(q, cu, cache.k_cache, cache.v_cache, t, L, D ** -0.5, out, plen,
                                                 max_len), steps, warmup, stream)
+    # the prompt write alone (pa_reshape_and_cache of every prompt row): HBM-bound at this size
+    ap, _ = time_calls(lambda: None, lambda: B.pa_reshape_and_cache(k, v, slots, cache.k_cache, cache.v_cache),
+                       steps, warmup, stream)
     check_device(B, workload)
+    append_bytes = 2 * T * hkv * D * (2 + cache.k_cache.element_size())   # bf16 rows read, cache rows written
     flops = 4.0 * D * hq * nseq * plen * (plen + 1) / 2
     pf_ms = statistics.mean(pf)
     try:
@@ -714,7 +720,9 @@ def prefill_record(B, workload, kv_dtype, steps, warmup, device, rank=0):
             "kv_dtype": str(cache.k_cache.dtype).replace("torch.", ""), "prefill_ms": round(pf_ms, 4),
             "step_ms": round(total / steps, 4), "flops": flops,
             "tflops": round(flops / (pf_ms * 1e-3) / 1e12, 2), "peak": peak, "peak_source": src,
-            "frac": round(flops / (pf_ms * 1e-3) / 1e12 / peak, 4)}
+            "frac": round(flops / (pf_ms * 1e-3) / 1e12 / peak, 4),
+            "append_ms": round(statistics.mean(ap), 4), "append_bytes": append_bytes,
+            "append_gbs": round(append_bytes / (statistics.mean(ap) * 1e-3) / 1e9, 1)}
 
 
 def swap_record(B, device, n_pairs=1024, reps=3):
@@ -759,8 +767,14 @@ def swap_record(B, device, n_pairs=1024, reps=3):
                      "out_gbs": round(nbytes / (statistics.mean(t_out) * 1e-3) / 1e9, 2),
                      "in_gbs": round(nbytes / (statistics.mean(t_in) * 1e-3) / 1e9, 2),
                      "host_issue_ms": round(issue_ms, 3)}
+    # copy-on-write block copies at scale: n_pairs blocks copied within the pool
+    cp = torch.from_numpy(np.stack([dev_ids, np.setdiff1d(np.arange(nb), dev_ids)[:n_pairs].astype(np.int32)],
+                                   1)).to(device)
+    t_cp, _ = time_calls(lambda: None, lambda: B.pa_copy_blocks(cache.k_cache, cache.v_cache, cp), reps, 1, stream)
+    rec["copy_blocks"] = {"ms": round(statistics.mean(t_cp), 4), "bytes": 2 * nbytes,
+                          "gbs": round(2 * nbytes / (statistics.mean(t_cp) * 1e-3) / 1e9, 1),
+                          "note": "read + write bytes of the pairs' K and V blocks"}
     check_device(B, "swap")
-    # round trip leaves the pool unchanged
     return rec
 
 
@@ -851,8 +865,9 @@ def run_e2e(args, d, device, world, P):
     h2d_ms, _ = time_calls(lambda: None, lambda: dq.copy_(hsrc, non_blocking=True), 10, 3, stream)
     d2h_ms, _ = time_calls(lambda: None, lambda: hdst.copy_(dout, non_blocking=True), 10, 3, stream)
     mean = lambda key: round(statistics.mean(p[key] for p in phases), 2)
-    breakdown = {k: mean(k) for k in ("block_manager_us", "h2d_enqueue_us", "launch_us", "d2h_enqueue_us",
-                                      "wait_us", "total_us")}
+    breakdown = {k: mean(k) for k in ("block_manager_us", "metadata_enqueue_us", "chains_enqueue_us", "wait_us",
+                                      "total_us")}
+    breakdown["chunks"] = phases[-1]["chunks"]
     breakdown["h2d_copy_alone_us"] = round(1e3 * statistics.mean(h2d_ms), 2)
     breakdown["d2h_copy_alone_us"] = round(1e3 * statistics.mean(d2h_ms), 2)
     ms, kv_total = combine_ranks(ms, kv_total, world, device)
