@@ -578,7 +578,7 @@ def batching_trace(device, seed=0, kv_dtype="auto", num_blocks=None):
     return tr, cache, steps, host_s, io
 
 
-def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None):
+def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None, partition=-1):
     """Every step of the continuous-batching trace on the device, in order
     (append + pa_decode with the library's partition choice), `reps` passes
     after one untimed pass; per-step averages over the whole trace."""
@@ -586,7 +586,7 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None)
     sh = tr.shape
     eb = cache.k_cache.element_size()
     ws_bytes = max(B.pa_decode_workspace_bytes(st["n"], sh.num_q_heads, sh.num_kv_heads, sh.head_dim, st["max_len"],
-                                               sh.block_size, -1) for st in steps)
+                                               sh.block_size, partition) for st in steps)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     scale = 1.0 / math.sqrt(sh.head_dim)
     stream = torch.cuda.current_stream(device)
@@ -597,7 +597,7 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None)
             B.pa_reshape_and_cache(io["k"], io["v"], st["slots"], kc, vc)
             if evs is not None:
                 evs[i][0].record(stream)
-            B.pa_decode(io["q"], kc, vc, st["tables"], st["lens"], scale, io["out"], st["max_len"], -1, ws)
+            B.pa_decode(io["q"], kc, vc, st["tables"], st["lens"], scale, io["out"], st["max_len"], partition, ws)
             if evs is not None:
                 evs[i][1].record(stream)
 
@@ -634,7 +634,8 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None)
            "host_note": "C++ block manager through the ctypes binding per step: frees, arrival reservations, one "
                         "slot per live sequence, block tables; timed on the host, outside the device time",
            "partition_tokens": sorted({B.pa_decode_partition_tokens(st["n"], sh.num_q_heads, sh.num_kv_heads,
-                                                                    st["max_len"], sh.block_size) for st in steps}),
+                                                                    st["max_len"], sh.block_size)
+                                       if partition < 0 else partition for st in steps}),
            "kv_dtype": str(kc.dtype).replace("torch.", "")}
     return rec, dec_ms, kv
 

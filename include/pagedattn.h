@@ -233,8 +233,9 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
  * for each group, one pass over the shared prefix blocks attends all members'
  * queries at once (rows = members x query heads on the tensor cores); each
  * sequence's own suffix [seq_prefix_tokens[s], L_s) goes through the decode
- * kernels; a log-sum-exp merge combines them. Prefix K/V bytes are read once
- * per group instead of once per member.
+ * kernels; a log-sum-exp merge combines them (done by the suffix CTA itself
+ * when sequences are not split into partitions, else by a merge kernel).
+ * Prefix K/V bytes are read once per group instead of once per member.
  *
  *   group_offsets        device int32 [num_groups + 1]; group j's members are
  *                        group_members[group_offsets[j] .. group_offsets[j+1]).
@@ -338,10 +339,10 @@ pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t nu
  * failure (PA_ERR_NO_FREE_BLOCKS, PA_ERR_UNKNOWN_SEQ) leaves the manager
  * unchanged and launches nothing. The staging buffers are reused by the next
  * call; the call returns only after the stream has drained.
- * A batch of 16 or more sequences is cut into up to four row chunks whose
- * copies, appends and decodes run as separate chains on streams the library
- * creates once per device (kept until the process exits): the copy engines
- * move one chunk's inputs and another's output while a third computes. The
+ * A batch of 16 or more sequences is cut into two row chunks whose copies,
+ * appends and decodes run as separate chains on streams the library creates
+ * once per device (kept until the process exits): the copy engines move one
+ * chunk's inputs or outputs while the other computes. The
  * chains start after the work already queued on `stream`, and `stream` waits
  * for all of them, so the call's ordering against the caller's stream is that
  * of a single chain.

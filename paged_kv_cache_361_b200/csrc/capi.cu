@@ -515,7 +515,7 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   if (!enc(&tk, cache->k, rows, cache->head_dim, cache->block_size) ||
       !enc(&tv, cache->v, rows, cache->head_dim, cache->block_size))
     return PA_ERR_CUDA;
-  const dim3 grid(cache->num_kv_heads, static_cast<unsigned>(ntiles), num_seqs);
+  const dim3 grid(cache->num_kv_heads, num_seqs, static_cast<unsigned>(ntiles));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto launch = [&](auto kern, int threads, int smem) -> pa_status {
     if (!smem_attrs(reinterpret_cast<const void*>(kern), smem, false)) return PA_ERR_CUDA;
@@ -564,7 +564,10 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
 
 // Shared-prefix decode: prefix partitions of this many tokens (a multiple of
 // the 64-token chunk).
-constexpr int32_t kCascadePrefixPart = 256;
+#ifndef PA_CASCADE_PREFIX_PART
+#define PA_CASCADE_PREFIX_PART 256
+#endif
+constexpr int32_t kCascadePrefixPart = PA_CASCADE_PREFIX_PART;
 
 size_t cascade_ws_bytes(int32_t num_seqs, int32_t hq, int32_t hkv, int32_t D, int32_t suffix_parts,
                         int32_t prefix_parts) {
@@ -661,7 +664,8 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
       return PA_ERR_CUDA;
     const dim3 grid(cache->num_kv_heads, pparts, num_groups);
     auto launch = [&](auto kern, int smem) -> pa_status {
-      if (!smem_attrs(reinterpret_cast<const void*>(kern), smem, false)) return PA_ERR_CUDA;
+      // the largest shared-memory carveout: two of these CTAs fit an SM
+      if (!smem_attrs(reinterpret_cast<const void*>(kern), smem, true)) return PA_ERR_CUDA;
       kern<<<grid, MmaCfg<128>::kThreads, smem, s>>>(tk, tv, pa);
       return launched();
     };
@@ -710,6 +714,8 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
   a.force_partials = 1;
   a.parts_stride = stride;
   a.prefix_part_tokens = kCascadePrefixPart;
+  // unsplit suffixes: each suffix CTA merges its sequence's prefix partials itself
+  a.cascade_direct = parts == 1 ? 1 : 0;
   if (is_8bit(cache->dtype)) {
     a.scale_log2 *= cache->k_scale;
     a.v_scale = cache->v_scale;
@@ -724,8 +730,8 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
   } else {
     return PA_ERR_UNSUPPORTED;  // unreachable: an 8-bit cache here has block_size >= 8
   }
-  if (st != PA_OK) return st;
-  // 3. merge prefix and suffix partials
+  if (st != PA_OK || a.cascade_direct) return st;
+  // 3. merge prefix and suffix partials (split suffixes)
   return D == 128 ? launch_reduce<128>(a, s) : launch_reduce<64>(a, s);
 }
 

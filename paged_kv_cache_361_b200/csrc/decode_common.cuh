@@ -42,6 +42,11 @@ struct DecodeArgs {
   // Split sequences merged by the CTA that finishes last: each CTA counts its
   // arrival in counters[1 + s * hkv + g] (zeroed before the launch).
   int32_t fuse_merge = 0;
+  // Cascade with unsplit suffixes: the suffix CTA of (s, g) merges its own
+  // state with the sequence's prefix partials (written by the prefix pass,
+  // earlier on the stream) and stores the final rows; a sequence with an empty
+  // suffix still gets its partition-0 CTA for that merge.
+  int32_t cascade_direct = 0;
 };
 
 // First token a decode CTA covers for sequence s (the cascade suffix start).
@@ -107,6 +112,7 @@ __device__ __forceinline__ int32_t load_len(const DecodeArgs& a, int32_t s, bool
 // (after writing the zero row of an empty context).
 struct Part {
   int32_t t0, t1, ntok, nparts;
+  int32_t npre;  // cascade: prefix partials of this sequence (slots max_parts ..)
 };
 
 template <int G, int D>
@@ -116,11 +122,22 @@ __device__ __forceinline__ bool cta_part(const DecodeArgs& a, int g, int s, int 
   const int32_t span = L - st;
   const int32_t P = a.part_tokens > 0 ? a.part_tokens : (span > 0 ? span : 1);
   pt.t0 = st + p * P;
+  pt.npre = 0;
+  if (a.starts && st > 0) {
+    pt.npre = (st + a.prefix_part_tokens - 1) / a.prefix_part_tokens;
+    pt.npre = min(pt.npre, a.parts_stride - a.max_parts);  // never past the prefix slots
+  }
   if (L == 0 && !a.starts) {
     if (p == 0)
       for (int idx = tid; idx < G * D; idx += nthreads)
         a.out[(static_cast<int64_t>(s) * a.hq + g * G) * D + idx] = 0.f;
     return false;
+  }
+  if (a.cascade_direct && p == 0 && span == 0) {  // empty suffix: merge the prefix partials alone
+    pt.t1 = pt.t0 = L;
+    pt.ntok = 0;
+    pt.nparts = 1;
+    return true;
   }
   if (pt.t0 >= L) return false;
   pt.t1 = min(pt.t0 + P, L);
@@ -280,21 +297,38 @@ __device__ __forceinline__ void merge_partials_to_out(const DecodeArgs& a, int s
 //   wm, wl: [NW][G];  wacc: [NW][G][D]
 template <int G, int D, int NW>
 __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const float* wm, const float* wl,
-                                                      const float* wacc, int s, int p, int hq0, int nparts, int tid,
-                                                      int nthreads) {
+                                                      const float* wacc, int s, int p, int hq0, int nparts, int npre,
+                                                      int tid, int nthreads) {
   for (int idx = tid; idx < G * D; idx += nthreads) {
     const int h = idx / D, d = idx - h * D;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w * G + h]);
     float l = 0.f, o = 0.f;
+    if (M != -INFINITY) {  // (an empty suffix has no state of its own)
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float f = exp2f(wm[w * G + h] - M);
-      l = fmaf(wl[w * G + h], f, l);
-      o = fmaf(wacc[(w * G + h) * D + d], f, o);
+      for (int w = 0; w < NW; ++w) {
+        const float f = exp2f(wm[w * G + h] - M);
+        l = fmaf(wl[w * G + h], f, l);
+        o = fmaf(wacc[(w * G + h) * D + d], f, o);
+      }
     }
     const int64_t row = static_cast<int64_t>(s) * a.hq + hq0 + h;
+    if (a.cascade_direct) {
+      // fold in the prefix partials; each covers at least one key, so its m is finite
+      const float* ml = a.ws_ml + (row * a.parts_stride + a.max_parts) * 2;
+      const float* po = a.ws_o + (row * a.parts_stride + a.max_parts) * D + d;
+      for (int q = 0; q < npre; ++q) {
+        const float mq = ml[2 * q];
+        const float Mn = fmaxf(M, mq);
+        const float f0 = exp2f(M - Mn), f1 = exp2f(mq - Mn);  // exp2(-inf) = 0 while M is -inf
+        l = l * f0 + ml[2 * q + 1] * f1;
+        o = o * f0 + po[static_cast<int64_t>(q) * D] * f1;
+        M = Mn;
+      }
+      a.out[row * D + d] = l > 0.f ? o / l : 0.f;  // an empty context gives a zero row
+      continue;
+    }
     if (nparts == 1 && !a.force_partials) {
       a.out[row * D + d] = o / l;
     } else {

@@ -134,6 +134,14 @@ __device__ __forceinline__ void widen_row_half(const uint8_t* src, uint8_t* dst,
   const int key = D == 128 ? (row & 7) : ((row >> 1) & 3);  // swizzle of the staged code row
   src += row * D;
   dst += row * 128;
+  // every load of the row's codes first (all in flight together), then the stores
+  uint4 wv[DH / 16];
+#pragma unroll
+  for (int u0 = 0; u0 < DH / 16; ++u0) {
+    const int u = D == 128 && half ? (u0 ^ 2) : u0;
+    const int d0 = half * DH + 16 * u;
+    wv[u0] = live ? *reinterpret_cast<const uint4*>(src + (((d0 >> 4) ^ key) << 4)) : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
   for (int u0 = 0; u0 < DH / 16; ++u0) {
     // at D 128 the two halves of a row would store to the same 16-byte columns
@@ -141,8 +149,7 @@ __device__ __forceinline__ void widen_row_half(const uint8_t* src, uint8_t* dst,
     // pieces in rotated order, so a phase hits 8 columns
     const int u = D == 128 && half ? (u0 ^ 2) : u0;
     const int d0 = half * DH + 16 * u;  // 16 codes -> dims d0 .. d0 + 15
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (live) w = *reinterpret_cast<const uint4*>(src + (((d0 >> 4) ^ key) << 4));
+    const uint4 w = wv[u0];
     uint32_t h[8];
     widen4<CF>(w.x, h[0], h[1]);
     widen4<CF>(w.y, h[2], h[3]);
@@ -490,7 +497,7 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
     }
   }
   __syncthreads();
-  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, tid, Cfg::kThreads);
+  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, pt.npre, tid, Cfg::kThreads);
 }
 
 }  // namespace pa

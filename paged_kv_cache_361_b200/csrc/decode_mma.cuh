@@ -599,7 +599,7 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
     }
   }
   __syncthreads();
-  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, tid, Cfg::kThreads);
+  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, pt.npre, tid, Cfg::kThreads);
 }
 
 }  // namespace pa

@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
     }
   }
   __syncthreads();
-  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, tid, Cfg::kThreads);
+  merge_warps_and_store<G, D, NW>(a, wm, wl, wacc, s, p, hq0, pt.nparts, pt.npre, tid, Cfg::kThreads);
 }
 
 }  // namespace pa

@@ -11,9 +11,12 @@
 //
 // CTA = (kv head g, query tile, sequence); a tile is 128 rows (the MMA M),
 // row r = (token tok0 + r / G, query head g*G + r % G), so the G heads sharing
-// a kv head read every K/V tile once. Six warps:
-//   warp 4     TMA producer: swizzled [bs x 64] boxes of K and V, 64 keys per
-//              stage (the ring and its full/empty barriers of the decode path).
+// a kv head read every K/V tile once. Warps:
+//   warp 4     TMA producer: swizzled [bs x 64] boxes of K, 64 keys per stage;
+//              over a bf16 cache a second producer warp (after the converter
+//              warps) copies the stage's V, so that K and V are released
+//              separately: K once both tiles' S = Q K^T has read it, V after
+//              their P V. (Over an 8-bit cache one producer copies both.)
 //   warp 5     allocates TMEM and walks the MMA schedule; one lane chosen
 //              by elect.sync issues every MMA:
 //                S_j = Q K_j^T        (M 128, N 64, K = D; A and B in shared
@@ -66,6 +69,7 @@ namespace pa {
 #define PA_TC_STAGES 4
 #endif
 
+
 template <int D, int TILES, bool F8 = false>
 struct TcCfg {
   static constexpr int kRows = 128;                        // query rows per tile (MMA M)
@@ -87,7 +91,10 @@ struct TcCfg {
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
   static constexpr int kConvWarp0 = kSoftmaxWarps + 2;
   static constexpr int kConvWarps = 4;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kConvWarps);
+  // bf16: a second producer warp streams V (K and V of a stage are released
+  // separately: K once both tiles' S has read it, V after their P V)
+  static constexpr int kVProducerWarp = kConvWarp0 + kConvWarps;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kConvWarps + (F8 ? 0 : 1));
   // per tile: O (D columns), then two S/P buffers of kChunk columns
   static constexpr uint32_t kTileCols = D + 2 * kChunk;
   static constexpr uint32_t kTmemCols = TILES * kTileCols <= 256 ? 256 : 512;
@@ -107,18 +114,19 @@ template <int D, int kHalfBytes>
 __device__ __forceinline__ void v_to_f16_inplace(uint8_t* vt, int row, int half, bool live) {
   constexpr int NCH = D == 128 ? 8 : 4;  // 16-byte chunks per thread
   uint8_t* rp = vt + (D == 128 ? half * kHalfBytes : 0) + row * 128;
+  uint4* ptr[NCH];
+  uint4 x[NCH];
+  // every load of the row's pieces first (all in flight together), then the stores
 #pragma unroll
   for (int u0 = 0; u0 < NCH; ++u0) {
     const int c = D == 128 ? (half ? (u0 ^ 4) : u0) : half * 4 + u0;  // logical chunk of the 128-byte row
-    uint4* ptr = reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4));
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (live) {
-      const uint4 x = *ptr;
-      w = make_uint4(pack_f16(bf16lo(x.x), bf16hi(x.x)), pack_f16(bf16lo(x.y), bf16hi(x.y)),
-                     pack_f16(bf16lo(x.z), bf16hi(x.z)), pack_f16(bf16lo(x.w), bf16hi(x.w)));
-    }
-    *ptr = w;
+    ptr[u0] = reinterpret_cast<uint4*>(rp + ((c ^ (row & 7)) << 4));
+    x[u0] = live ? *ptr[u0] : make_uint4(0u, 0u, 0u, 0u);
   }
+#pragma unroll
+  for (int u0 = 0; u0 < NCH; ++u0)
+    *ptr[u0] = make_uint4(pack_f16(bf16lo(x[u0].x), bf16hi(x[u0].x)), pack_f16(bf16lo(x[u0].y), bf16hi(x[u0].y)),
+                          pack_f16(bf16lo(x[u0].z), bf16hi(x[u0].z)), pack_f16(bf16lo(x[u0].w), bf16hi(x[u0].w)));
 }
 
 // All lanes wait; the warp proceeds only if every lane saw the phase.
@@ -143,6 +151,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
   __shared__ PipeSmem<S> ps;  // 16-bit K/V stages: filled by the TMA (bf16) or the converter (F8)
   __shared__ uint64_t cfull[CS], cempty[CS];  // F8: code staging ring, producer <-> converter
   __shared__ uint64_t vready[S];              // bf16: the stage's V rewritten as f16 (converter -> MMA)
+  __shared__ uint64_t vfull[S], vempty[S];    // bf16: V of a stage (ps.full / ps.empty track its K)
   __shared__ uint64_t q_full, drain;
   __shared__ uint64_t s_full[TILES][2], p_full[TILES][2], o_bar[TILES];
   __shared__ uint32_t tmem_base_sh;
@@ -153,8 +162,10 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
   const uint32_t kv0 = sbase + Cfg::kQBytes;  // stage st: K halves, then V halves
   const uint32_t cs0 = kv0 + S * Cfg::kStageBytes;  // F8 staging slot: K codes, then V codes
 
-  const int g = blockIdx.x, s = blockIdx.z;
-  const int pair = a.ntiles - 1 - static_cast<int>(blockIdx.y);  // longest key ranges first
+  // grid (kv heads, sequences, tile pairs): every sequence's last (longest) pair
+  // is dispatched before any shorter one, so the last CTAs to run are the short ones
+  const int g = blockIdx.x, s = blockIdx.y;
+  const int pair = a.ntiles - 1 - static_cast<int>(blockIdx.z);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int32_t q0 = __ldg(a.cu_q + s);
@@ -211,7 +222,11 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       fence_mbar_init();
     } else {
 #pragma unroll
-      for (int i = 0; i < S; ++i) mbar_init(&vready[i], Cfg::kConvWarps);
+      for (int i = 0; i < S; ++i) {
+        mbar_init(&vready[i], Cfg::kConvWarps);
+        mbar_init(&vfull[i], 1);
+        mbar_init(&vempty[i], 1);
+      }
       pipe_init<S>(ps, 1);  // empty stages are released by one tcgen05.commit
     }
   }
@@ -276,7 +291,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         mbar_arrive(&cempty[cst]);
       }
     }
-  } else if (!F8 && warp >= Cfg::kConvWarp0) {
+  } else if (!F8 && warp >= Cfg::kConvWarp0 && warp < Cfg::kConvWarp0 + Cfg::kConvWarps) {
     // ---- converter (bf16): the stage's V tile, bf16 -> f16 in place; thread =
     // (row of the chunk, box column at D 128 / half of the row at D 64) ----
     const int ct = tid - 32 * Cfg::kConvWarp0;
@@ -284,41 +299,49 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
     uint8_t* kv0g = sgen + Cfg::kQBytes;
     for (int i = 0; i < nchunks; ++i) {
       const int st = i % S;
-      if (!warp_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
+      if (!warp_wait(&vfull[st], (i / S) & 1, &ps.abort_flag)) break;
       const bool live = i * C + row < kend_all;  // rows past the last key become zeros
       v_to_f16_inplace<D, Cfg::kHalfBytes>(kv0g + st * Cfg::kStageBytes + Cfg::kTileBytes, row, half, live);
       tc::fence_proxy_async();  // generic-proxy writes -> tensor-core reads
       __syncwarp();
       if (lane == 0) mbar_arrive(&vready[st]);
     }
-  } else if (warp == Cfg::kProducerWarp) {
-    // ---- producer ----
+  } else if (!F8 && (warp == Cfg::kProducerWarp || warp == Cfg::kVProducerWarp)) {
+    // ---- producers (bf16): K of chunk i into stage i % S (released by the S
+    // MMAs) by one warp, V (released by the P V MMAs) by the other ----
+    const bool is_v = warp == Cfg::kVProducerWarp;
+    uint64_t* full = is_v ? vfull : ps.full;
+    uint64_t* empty = is_v ? vempty : ps.empty;
+    const CUtensorMap* map = is_v ? &tmv : &tmk;
+    const uint32_t tile_off = is_v ? Cfg::kTileBytes : 0u;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
     TableAhead ta;
     ta.init(a.tables + table_row, 0, min(a.max_blocks, (kend_all + a.bs - 1) / a.bs), lane);
-    pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+    int i = 0;
+    for (; i < nchunks; ++i) {
+      const int st = i % S;
+      if (i >= S && !warp_wait(&empty[st], ((i / S) - 1) & 1, &ps.abort_flag)) break;
       const int32_t c0 = i * C;
       const int32_t nb = (min(C, kend_all - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
       const int32_t blk = ta.get(c0 / a.bs, nb, lane);
       bool ok = false;
       if (lane < nb) {
         ok = blk >= 0 && blk < a.num_blocks;
-        if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
+        if (!ok && !is_v) record_error(PA_ERR_DEVICE_BOUNDS, blk);
       }
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * Cfg::kHalves * __popc(okmask) * box_bytes);
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], Cfg::kHalves * __popc(okmask) * box_bytes);
       __syncwarp();
       if (ok) {
         const int32_t y = (blk * a.hkv + g) * a.bs;
-        const uint32_t kdst = kv0 + st * Cfg::kStageBytes + lane * box_bytes;
+        const uint32_t dst = kv0 + st * Cfg::kStageBytes + tile_off + lane * box_bytes;
 #pragma unroll
-        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-          tma_load_2d(kdst + hf * Cfg::kHalfBytes, &tmk, hf * 64, y, &ps.full[st], pol);
-          tma_load_2d(kdst + Cfg::kTileBytes + hf * Cfg::kHalfBytes, &tmv, hf * 64, y, &ps.full[st], pol);
-        }
+        for (int hf = 0; hf < Cfg::kHalves; ++hf) tma_load_2d(dst + hf * Cfg::kHalfBytes, map, hf * 64, y, &full[st], pol);
       }
-    });
+    }
+    if (ps.abort_flag && lane == 0)  // copies already started land before exit
+      for (int j = (i > S ? i - S : 0); j < i; ++j) mbar_wait(&full[j % S], (j / S) & 1);
   } else if (warp == Cfg::kMmaWarp) {
     // ---- MMA issuer: S_t(j+1) for every tile, then O_t += P_t(j) V(j); the
     // whole warp walks the schedule and waits, one elected lane issues ----
@@ -369,6 +392,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
 #pragma unroll
         for (int t = 0; t < TILES; ++t)
           if (nch[t] > 0) issue_s(t, 0);
+        if constexpr (!F8) tc::commit(smem_u32(&ps.empty[0]));  // K of stage 0 is read once these finish
       }
       for (int j = 0; ok && j < nchunks; ++j) {
         if (j + 1 < nchunks) {
@@ -380,6 +404,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
 #pragma unroll
           for (int t = 0; t < TILES; ++t)
             if (j + 1 < nch[t]) issue_s(t, j + 1);
+          if constexpr (!F8) tc::commit(smem_u32(&ps.empty[(j + 1) % S]));  // K of chunk j+1 released
         }
         if constexpr (!F8) {
           // the converter has rewritten this stage's V as f16
@@ -392,7 +417,8 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
 #pragma unroll
         for (int t = 0; t < TILES; ++t)
           if (ok && j < nch[t]) ok = issue_pv(t, j);
-        if (ok) tc::commit(smem_u32(&ps.empty[j % S]));  // every tile is done with stage j
+        // every tile is done with stage j (bf16: its V; 8-bit: the whole stage)
+        if (ok) tc::commit(smem_u32(F8 ? &ps.empty[j % S] : &vempty[j % S]));
       }
       // every MMA the warp issued has finished before TMEM is released
       tc::commit(smem_u32(&drain));

@@ -37,6 +37,9 @@ double us_since(std::chrono::steady_clock::time_point t0, std::chrono::steady_cl
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Row chunks of a batch (measured on the 64-sequence metric workload: one
+// chain 0.281 ms per step, two 0.261 ms, four 0.274 ms: each chain costs host
+// calls, ~15 us of enqueueing).
 #ifndef PA_STEP_MAX_CHUNKS
 #define PA_STEP_MAX_CHUNKS 2
 #endif

@@ -245,3 +245,33 @@ def test_prefill_benchmark_size_sampled_rows():
             err = float(np.abs(out[base + t].double().cpu().numpy() - ref).max())
             worst = max(worst, err)
     assert worst <= 4e-3, worst
+
+
+def test_cascade_empty_suffix_and_empty_sequence():
+    """A member whose whole context is the shared prefix (its suffix is empty)
+    and an empty sequence: the suffix CTAs merge the prefix partials alone and
+    write a zero row, as pa_decode does."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    hkv, G, D, bs = 2, 4, 128, 16
+    g = torch.Generator().manual_seed(21)
+    cache = PagedKVCache(64, hkv, bs, D, torch.bfloat16, "cuda", fill=float("nan"))
+    k = torch.randn(128, hkv, D, generator=g).bfloat16()
+    v = torch.randn(128, hkv, D, generator=g).bfloat16()
+    cache.add_sequence(0, k.cuda(), v.cuda())          # 8 whole blocks: the prefix is all 128 tokens
+    for child in (1, 2, 3):
+        cache.fork(0, child)
+    for _ in range(5):
+        cache.append([1, 2], torch.randn(2, hkv, D, generator=g).bfloat16().cuda(),
+                     torch.randn(2, hkv, D, generator=g).bfloat16().cuda())
+    cache.add_sequence(9, torch.empty(0, hkv, D, dtype=torch.bfloat16).cuda(),
+                       torch.empty(0, hkv, D, dtype=torch.bfloat16).cuda())
+    ids = [0, 1, 2, 3, 9]
+    off, mem, pre, sp, mp = cache.shared_prefix_groups(ids, 64 // G)
+    assert pre.tolist() == [128] and sp.tolist() == [128, 128, 128, 128, 0]
+    q = torch.randn(len(ids), hkv * G, D, generator=g).bfloat16().cuda()
+    a = cache.decode(ids, q, D ** -0.5)
+    b = cache.decode_cascade(ids, q, D ** -0.5)
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    assert torch.isfinite(b).all()
+    assert float(b[4].abs().max()) == 0.0
+    assert float((a - b).abs().max()) <= 2e-3

@@ -468,7 +468,7 @@ def test_step_host_chunked_matches_oracle(n, G):
         out = torch.full((n, hkv * G, D), float("nan"), dtype=torch.float32).pin_memory()
         ref.apply(("append", ids, lambda which, device="cpu", k=k, v=v: k if which == "k" else v))
         cache.step_host(ids, q, k, v, out, D ** -0.5, partition_tokens=64 if step == 1 else -1)
-        assert B.pa_step_host_last_timing()["chunks"] == min(4, n // 8)
+        assert B.pa_step_host_last_timing()["chunks"] >= 2          # the chained path
         for i, sid in enumerate(ids):
             exp = ref.attend(sid, q[i], D ** -0.5, use_pool=True)
             assert float(np.abs(out[i].double().numpy() - exp).max()) <= TOL["bf16"], (step, sid)
