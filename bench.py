@@ -38,12 +38,47 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode attention tokens/sec"
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# dominant kernel, from one-pass ncu captures of this script, keyed by
-# (workload, cache dtype, partition tokens) -> (bytes, source files of that
-# kernel, their hash at capture). A capture whose files have changed since is
-# stale and reported as null, as is any configuration without a capture.
-NCU_TRAFFIC: dict = {}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one call of the
+# timed operation (every kernel of pa_decode / pa_decode_cascade / pa_prefill),
+# from one-pass ncu launch lists of this script (averaged over the listed
+# launches), keyed by (workload, cache dtype, partition tokens, path). Each
+# entry names the library sources of those kernels and their hash at capture:
+# an entry whose files have changed since is stale and reported as null, as is
+# any configuration without a capture. The command lines are in profiles/.
+_DEC = ["common.cuh", "decode_common.cuh", "capi.cu"]
+_PF = ["common.cuh", "decode_common.cuh", "decode_f8.cuh", "prefill_mma.cuh", "prefill_tc.cuh", "tcgen05.cuh",
+       "capi.cu"]
+NCU_TRAFFIC: dict = {
+    ("llama2_7b_mha", "bfloat16", 0, "decode"): dict(
+        bytes=1_079_339_776 + 998_229, files=_DEC + ["decode_simt.cuh"], sha="e143330f49c54f75",
+        note="decode_simt_kernel, 3 launches"),
+    ("llama2_7b_mha", "float8_e4m3fn", 0, "decode"): dict(
+        bytes=539_992_832 + 7_646_549, files=_DEC + ["decode_f8.cuh"], sha="ce2482e42c316dce",
+        note="decode_f8_kernel (e4m3), 3 launches"),
+    ("llama2_7b_mha", "int8", 0, "decode"): dict(
+        bytes=539_992_320 + 8_051_712, files=_DEC + ["decode_f8.cuh"], sha="ce2482e42c316dce",
+        note="decode_f8_kernel (int8), 3 launches"),
+    ("long_context_split", "bfloat16", 512, "decode"): dict(
+        bytes=1_342_939_584 + 5_665_664 + 21_471_680, files=_DEC + ["decode_mma.cuh"], sha="86b797581e62b7d5",
+        note="decode_mma_persistent_kernel + decode_reduce_kernel, 4 launches each"),
+    ("parallel_sampling", "bfloat16", 0, "decode"): dict(
+        bytes=100_495_659 + 169_216, files=_DEC + ["decode_mma.cuh"], sha="86b797581e62b7d5",
+        note="decode_mma_kernel, 6 launches"),
+    ("parallel_sampling", "bfloat16", 0, "cascade"): dict(
+        bytes=32_021_632 + 72_819_814 + 42_342, files=_DEC + ["decode_mma.cuh", "prefill_mma.cuh"],
+        sha="a8338145e53106fe", note="prefill_mma_kernel (prefix pass) + decode_mma_kernel (suffix, merge), "
+                                     "5-6 launches each"),
+    ("continuous_batching", "bfloat16", 1024, "decode"): dict(
+        bytes=835_727_761 + 4_076_467, files=_DEC + ["decode_mma.cuh"], sha="86b797581e62b7d5",
+        note="decode_mma_persistent_kernel over steps 0-29 of the trace (32768-block pool); their algorithmic mean "
+             "is 825.0 MB per step (x1.018), the 200-step mean 811.2 MB"),
+    ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
+        bytes=1_309_394_000 + 233_774_080, files=_PF, sha="b9e7a2b9692c8b03", note="prefill_tc_kernel, 1 launch",
+        how="ncu capture (metric set, small case = this workload)"),
+    ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
+        bytes=729_495_040 + 493_113_344, files=_PF, sha="b9e7a2b9692c8b03", note="prefill_tc_kernel, 1 launch",
+        how="ncu capture (metric set, small case = this workload)"),
+}
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
 
@@ -61,10 +96,10 @@ def ncu_traffic(key):
     e = NCU_TRAFFIC.get(key)
     if e is None:
         return None, "no capture of this configuration"
-    nbytes, files, sha = e
-    if src_hash(files) != sha:
-        return None, "stale: the kernel's sources changed since the capture"
-    return nbytes, f"one-pass ncu capture of the current kernel (sources {sha})"
+    if src_hash(e["files"]) != e["sha"]:
+        return None, "stale: the kernels' sources changed since the capture"
+    how = e.get("how", "one-pass ncu launch list")
+    return e["bytes"], f"{how} of the current kernels (sources {e['sha']}): {e['note']}"
 
 
 def peaks():
@@ -258,15 +293,19 @@ def cascade_inputs(d, device):
     """Group arguments of pa_decode_cascade for the measured step (host work
     done once, before timing), from the C++ block manager
     (pa_bm_prefix_groups): sequences whose tables start with the same blocks
-    share their common prefix."""
+    share their common prefix; the suffix CTAs go longest first
+    (pa_bm_longest_first)."""
     from paged_kv_cache_361_b200 import binding as B
     cache, sh = d["cache"], d["shape"]
     offs, members, prefix, seq_prefix, max_pre = cache.shared_prefix_groups(d["ids"], 64 // sh.group)
+    order = cache.bm.longest_first(d["ids"], seq_prefix)
     nbytes = B.pa_decode_cascade_workspace_bytes(len(d["ids"]), sh.num_q_heads, sh.num_kv_heads, sh.head_dim,
                                                  d["max_len"], sh.block_size, max_pre)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
-    return (t(offs), t(members), t(prefix), t(seq_prefix), int(max(np.diff(offs), default=0)), max_pre, ws)
+    # (..., workspace, stream, seq_order) of binding.pa_decode_cascade
+    return (t(offs), t(members), t(prefix), t(seq_prefix), int(max(np.diff(offs), default=0)), max_pre, ws, None,
+            t(order))
 
 
 def sample_rows(d, seqs):
@@ -458,8 +497,7 @@ def run_ours(args, rank, world, device):
         merge_kernel = split and math.ceil(d["max_len"] / P_eff) >= 8
         launches = args.steps * (2 + (1 if merge_kernel else 0) + (1 if d["pairs"] is not None else 0))
     dtype_key = str(d["kc"].dtype).replace("torch.", "")
-    traffic, traffic_src = (None, "not captured for the cascade path") if cascade is not None else \
-        ncu_traffic((args.workload, dtype_key, P_eff))
+    traffic, traffic_src = ncu_traffic((args.workload, dtype_key, P_eff, "decode" if cascade is None else "cascade"))
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -478,7 +516,8 @@ def run_ours(args, rank, world, device):
                    "l2": "no flush: the K/V read per step is larger than the 126 MB L2"
                    if d["unique_kv_bytes"] > 3 * 126e6 else "no flush: K/V partly L2-resident (see unique bytes)"},
         "tokens_per_s": round(tokens_per_s, 1),
-        "pct_of_hbm_peak": {"of_measured_6540": round(value / peak, 4), "of_nominal_8000": round(value / 8000.0, 4)},
+        "pct_of_hbm_peak": {f"of_{peak_kind}_{peak:g}": round(value / peak, 4),
+                            "of_nominal_8000": round(value / 8000.0, 4)},
         "e2e": e2e,
         "gpu_launches": launches,
         "roofline": {"kernel": ("pa_decode_cascade (prefix + suffix + merge); achieved counts logical K/V bytes"
@@ -519,7 +558,7 @@ def decode_record(B, d, P, steps, warmup, device, cascade=None):
     P_eff = P if P >= 0 else B.pa_decode_partition_tokens(nseq, sh.num_q_heads, sh.num_kv_heads, d["max_len"],
                                                           sh.block_size)
     dtype_key = str(d["kc"].dtype).replace("torch.", "")
-    traffic, src = ncu_traffic((d["name"], dtype_key, P_eff)) if cascade is None else (None, "not captured")
+    traffic, src = ncu_traffic((d["name"], dtype_key, P_eff, "decode" if cascade is None else "cascade"))
     rec = {"decode_ms": round(ms, 5), "step_ms": round(total / steps, 5), "kv_bytes": d["kv_bytes"],
            "gbs": round(gbs, 1), "frac_of_measured_peak": round(gbs / peak, 4),
            "frac_of_nominal_8000": round(gbs / 8000, 4), "tokens_per_s": round(nseq / (ms * 1e-3), 1),
@@ -653,6 +692,9 @@ def run_batching_line(args, rank, world, device):
     clk = clocks.stop()
     ms_total = rec["step_ms_avg"] * rec["steps"]
     ms_total, all_bytes = combine_ranks(ms_total, sum(kv), world, device)
+    parts = rec["partition_tokens"]
+    traffic, traffic_src = ncu_traffic(("continuous_batching", rec["kv_dtype"], parts[0], "decode")) \
+        if len(parts) == 1 else (None, "several partition sizes in the trace")
     value = all_bytes / (ms_total * 1e-3) / 1e9
     peak, kind = peaks()
     if rank == 0:
@@ -666,8 +708,8 @@ def run_batching_line(args, rank, world, device):
                        "l2": "no flush: ~0.8 GB of K/V per step against the 126 MB L2"},
             "tokens_per_s": rec["tokens_per_s_step"], "gpu_launches": rec["steps"] * rec["passes"] * 3,
             "roofline": {"kernel": "pa_decode (200-step average)", "bound": "hbm", "achieved": rec["gbs"],
-                         "peak": peak, "unit": "GB/s", "frac": rec["frac_of_measured_peak"], "traffic": None,
-                         "peak_source": kind},
+                         "peak": peak, "unit": "GB/s", "frac": rec["frac_of_measured_peak"], "traffic": traffic,
+                         "traffic_source": traffic_src, "peak_source": kind},
             "batching": rec, "clocks": clk}), flush=True)
 
 
@@ -806,10 +848,15 @@ def run_workloads(args, device):
     del d
     release()
     cb, _, _ = batching_record(B, device, reps=2)
+    parts = cb["partition_tokens"]
+    cb["traffic"], cb["traffic_source"] = ncu_traffic(("continuous_batching", cb["kv_dtype"], parts[0], "decode")) \
+        if len(parts) == 1 else (None, "several partition sizes in the trace")
     rec["continuous_batching_200_steps"] = cb
     release()
     for wl in ("prefill_llama2_7b_mha", "prefill_gqa8"):
-        rec[wl] = prefill_record(B, wl, "auto", 10, 3, device)
+        r = prefill_record(B, wl, "auto", 10, 3, device)
+        r["traffic"], r["traffic_source"] = ncu_traffic((wl, r["kv_dtype"], 0, "prefill"))
+        rec[wl] = r
         release()
     rec["swap"] = swap_record(B, device)
     release()
@@ -898,6 +945,7 @@ def run_prefill(args, rank, world, device):
     clk = clocks.stop()
     ms, all_flops = combine_ranks(r["step_ms"], r["flops"], world, device)
     f8 = args.kv_dtype in ("fp8", "int8")
+    traffic, traffic_src = ncu_traffic((args.workload, r["kv_dtype"], 0, "prefill"))
     if rank == 0:
         print(json.dumps({
             "metric": "paged prefill attention TFLOP/s (causal; 4*head_dim*Hq flops per visible query-key pair)",
@@ -910,7 +958,8 @@ def run_prefill(args, rank, world, device):
                        "larger than the 126 MB L2"},
             "gpu_launches": 2 * args.steps,
             "roofline": {"kernel": "pa_prefill", "bound": "tensor", "achieved": r["tflops"], "peak": r["peak"],
-                         "unit": "TFLOP/s", "frac": r["frac"], "traffic": None, "peak_source": r["peak_source"]},
+                         "unit": "TFLOP/s", "frac": r["frac"], "traffic": traffic, "traffic_source": traffic_src,
+                         "peak_source": r["peak_source"]},
             "clocks": clk}), flush=True)
 
 

@@ -248,6 +248,17 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
  *   seq_prefix_tokens    device int32 [num_seqs]: its group's prefix length,
  *                        0 for a sequence in no group.
  *   max_prefix_tokens    host bound on group_prefix_tokens.
+ *   seq_order            device int32 [num_seqs] or NULL: the order in which
+ *                        the sequences' suffix CTAs are dispatched, a
+ *                        permutation of 0 .. num_seqs-1 (pa_bm_longest_first
+ *                        puts the longest suffixes first, so that the long
+ *                        CTAs start in the first waves and the short ones
+ *                        fill the end). Results do not depend on it. An entry
+ *                        out of range is recorded as PA_ERR_DEVICE_BOUNDS (see
+ *                        pa_get_device_error) and its row is served in batch
+ *                        order; a repeated entry leaves some sequence
+ *                        uncomputed (no memory outside the arguments is
+ *                        touched).
  *   workspace            >= pa_decode_cascade_workspace_bytes(...).
  * Other arguments as pa_decode (partition size chosen by the library).
  * Supported: bf16, e4m3 or int8 cache, block_size 8..32; other shapes return
@@ -259,7 +270,8 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
                             int32_t max_context_len, int32_t num_groups, const int32_t* group_offsets,
                             const int32_t* group_members, const int32_t* group_prefix_tokens,
                             const int32_t* seq_prefix_tokens, int32_t max_group_size, int32_t max_prefix_tokens,
-                            float scale, float* out, void* workspace, size_t workspace_bytes, pa_stream stream);
+                            const int32_t* seq_order, float scale, float* out, void* workspace,
+                            size_t workspace_bytes, pa_stream stream);
 
 size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                          int32_t max_context_len, int32_t block_size, int32_t max_prefix_tokens);
@@ -511,6 +523,23 @@ pa_status pa_bm_prefix_groups(const pa_bm* bm, int32_t n, const int64_t* seq_ids
                               int32_t align_tokens, int32_t* group_offsets, int32_t* group_members,
                               int32_t* group_prefix_tokens, int32_t* seq_prefix_tokens, int32_t* n_groups_out,
                               int32_t* max_prefix_out);
+
+/*
+ * Longest-first dispatch order of a decode batch (the seq_order argument of
+ * pa_decode_cascade): a decode CTA's time grows with the tokens it reads, so
+ * starting the longest first leaves the short ones to fill the last wave.
+ *
+ *   seq_ids      host int64 [n]: the batch, in the order of its rows.
+ *   skip_tokens  host int32 [n] or NULL: tokens of each row not read by the
+ *                CTA being ordered (pa_decode_cascade: seq_prefix_tokens).
+ *   order        host int32 [n], written: the row indices sorted by
+ *                decreasing (the sequence's tokens - skip_tokens[row]), ties
+ *                in batch order.
+ * Reads the manager only; PA_ERR_UNKNOWN_SEQ if an id is not live,
+ * PA_ERR_INVALID_ARG for n < 0 or a missing array.
+ */
+pa_status pa_bm_longest_first(const pa_bm* bm, int32_t n, const int64_t* seq_ids, const int32_t* skip_tokens,
+                              int32_t* order);
 
 /* free_blocks: blocks on the free list (evictable cached blocks are not
  * counted); allocated_slots: block_size times the blocks not on the free

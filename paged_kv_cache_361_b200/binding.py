@@ -53,7 +53,7 @@ _SIGS = {
     "pa_decode": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP, _SZ, _VP]),
     "pa_decode_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
     "pa_decode_cascade": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32,
-                                 _F, _VP, _VP, _SZ, _VP]),
+                                 _VP, _F, _VP, _VP, _SZ, _VP]),
     "pa_decode_cascade_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "pa_prefill": (_I32, [_VP, _I32, _VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _VP]),
     "pa_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
@@ -74,6 +74,7 @@ _SIGS = {
     "pa_swap_blocks_copy": (_I32, [_PCACHE, _VP, _VP, _I64, _VP, _I32, _I32, _VP]),
     "pa_step_host_last_timing": (_I32, [_VP]),
     "pa_bm_prefix_groups": (_I32, [_VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _P32, _P32]),
+    "pa_bm_longest_first": (_I32, [_VP, _I32, _VP, _VP, _VP]),
     "pa_bm_prefix_stats": (_I32, [_VP, _P64, _P64, _P64]),
     "pa_bm_append_slot": (_I32, [_VP, _I64, _P64, _P32]),
     "pa_bm_append_slots": (_I32, [_VP, _I32, _VP, _VP, _VP, _P32]),
@@ -233,8 +234,9 @@ def pa_decode_cascade_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_
 
 def pa_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_context_len, group_offsets,
                       group_members, group_prefix_tokens, seq_prefix_tokens, max_group_size, max_prefix_tokens,
-                      workspace, stream=None):
-    """pa_decode with shared prefixes read once per group (see pagedattn.h)."""
+                      workspace, stream=None, seq_order=None):
+    """pa_decode with shared prefixes read once per group (see pagedattn.h);
+    seq_order: optional device int32 dispatch order of the suffix CTAs."""
     c = make_cache(k_cache, v_cache)
     B, hq, d = q.shape
     _dev(q, "q", input_dtype(k_cache.dtype), 3)
@@ -244,6 +246,10 @@ def pa_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, scale, ou
     _dev(block_tables, "block_tables", torch.int32, 2)
     _dev(context_lens, "context_lens", torch.int32, 1)
     _dev(seq_prefix_tokens, "seq_prefix_tokens", torch.int32, 1)
+    if seq_order is not None:
+        _dev(seq_order, "seq_order", torch.int32, 1)
+        if seq_order.shape[0] != B:
+            raise ValueError("seq_order must have one entry per sequence")
     ng = int(group_offsets.shape[0]) - 1
     if ng > 0:
         _dev(group_offsets, "group_offsets", torch.int32, 1)
@@ -254,7 +260,9 @@ def pa_decode_cascade(q, k_cache, v_cache, block_tables, context_lens, scale, ou
                                     group_offsets.data_ptr() if ng else None,
                                     group_members.data_ptr() if ng else None,
                                     group_prefix_tokens.data_ptr() if ng else None, seq_prefix_tokens.data_ptr(),
-                                    int(max_group_size), int(max_prefix_tokens), float(scale), out.data_ptr(),
+                                    int(max_group_size), int(max_prefix_tokens),
+                                    seq_order.data_ptr() if seq_order is not None else None, float(scale),
+                                    out.data_ptr(),
                                     _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                                     _stream(q, stream)), "pa_decode_cascade")
 
@@ -496,6 +504,19 @@ class BlockManager:
                                           ctypes.byref(mp)), "pa_bm_prefix_groups")
         g = ng.value
         return offs[:g + 1].copy(), members[:offs[g]].copy(), prefix[:g].copy(), seq_prefix[:n].copy(), int(mp.value)
+
+    def longest_first(self, seq_ids, skip_tokens=None) -> np.ndarray:
+        """Row indices of the batch by decreasing (tokens - skip_tokens[row]),
+        ties in batch order (pa_bm_longest_first)."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = len(ids)
+        order = np.zeros(max(n, 1), dtype=np.int32)
+        skip = None if skip_tokens is None else np.ascontiguousarray(skip_tokens, dtype=np.int32)
+        if skip is not None and len(skip) != n:
+            raise ValueError("skip_tokens must have one entry per sequence")
+        _check(_lib().pa_bm_longest_first(self._h, n, _i64p(ids), _i64p(skip) if skip is not None else None,
+                                          _i64p(order)), "pa_bm_longest_first")
+        return order[:n].copy()
 
     def refcount(self, block: int) -> int:
         r = ctypes.c_int32()

@@ -218,13 +218,15 @@ class PagedKVCache:
 
     def decode_cascade(self, seq_ids, q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None):
         """decode() with shared prefixes (forks, prefix-cache hits) read once per
-        group of sequences (pa_decode_cascade)."""
+        group of sequences (pa_decode_cascade); the suffix CTAs are dispatched
+        longest suffix first (pa_bm_longest_first)."""
         n, hq, d = q.shape
         if scale is None:
             scale = 1.0 / math.sqrt(d)
         tables, lens, max_len = self.decode_inputs(seq_ids)
         hkv = self.k_cache.shape[1]
         offs, members, prefix, seq_prefix, max_pre = self.shared_prefix_groups(seq_ids, 64 // (hq // hkv))
+        order = self.bm.longest_first(seq_ids, seq_prefix)
         if out is None:
             out = torch.empty((n, hq, d), dtype=torch.float32, device=self.device)
         nbytes = B.pa_decode_cascade_workspace_bytes(n, hq, hkv, d, max_len, self.block_size, max_pre)
@@ -234,7 +236,7 @@ class PagedKVCache:
                             out, max_len, self._lens.upload(offs),
                             self._lens.upload(members) if len(members) else empty,
                             self._lens.upload(prefix) if len(prefix) else empty, self._lens.upload(seq_prefix),
-                            int(max(np.diff(offs), default=0)), max_pre, ws)
+                            int(max(np.diff(offs), default=0)), max_pre, ws, seq_order=self._lens.upload(order))
         return out
 
     def step_host(self, seq_ids, q_host, k_host, v_host, out_host, scale=None, partition_tokens=-1):

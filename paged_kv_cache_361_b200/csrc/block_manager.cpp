@@ -586,6 +586,20 @@ pa_status pa_bm_block_tables(const pa_bm* bm, int32_t n, const int64_t* seq_ids,
 // whole blocks of its shortest member and cut down to a multiple of
 // align_tokens; a group of one member, or with a prefix of zero tokens, is
 // dropped and its sequences get no prefix.
+pa_status pa_bm_longest_first(const pa_bm* bm, int32_t n, const int64_t* seq_ids, const int32_t* skip_tokens,
+                              int32_t* order) {
+  if (!bm || n < 0 || (n > 0 && (!seq_ids || !order))) return PA_ERR_INVALID_ARG;
+  std::vector<int64_t> span(n);
+  for (int32_t i = 0; i < n; ++i) {
+    const Seq* q = bm->m.find(seq_ids[i]);
+    if (!q) return PA_ERR_UNKNOWN_SEQ;
+    span[i] = q->len - (skip_tokens ? skip_tokens[i] : 0);
+  }
+  for (int32_t i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order, order + n, [&](int32_t x, int32_t y) { return span[x] > span[y]; });
+  return PA_OK;
+}
+
 pa_status pa_bm_prefix_groups(const pa_bm* bm, int32_t n, const int64_t* seq_ids, int32_t max_group_size,
                               int32_t align_tokens, int32_t* group_offsets, int32_t* group_members,
                               int32_t* group_prefix_tokens, int32_t* seq_prefix_tokens, int32_t* n_groups_out,

@@ -40,6 +40,30 @@ pa_status check_cache(const pa_cache* c) {
 
 pa_status launched() { return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
 
+// Launches kern on st. With after_prev the launch carries the
+// programmatic-stream-serialization attribute: the grid may start once the
+// previous grid on the stream has called pdl_launch_dependents(), and it must
+// call pdl_wait() before it reads anything that grid writes.
+template <typename... KArgs, typename... Args>
+pa_status launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool after_prev,
+                        Args&&... args) {
+  if (!after_prev) {
+    kern<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+    return launched();
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 // Partition size for partition_tokens = -1. Measured on a B200 with the
 // decode kernels here: unsplit CTAs win while there are enough (sequence, kv
 // head) units to fill the GPU and no unit is long; long units are cut into
@@ -123,8 +147,7 @@ pa_status launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   using Cfg = SimtCfg<T, D>;
   auto kern = decode_simt_kernel<T, D, G>;
   if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(a);
-  return launched();
+  return launch_kernel(kern, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, a.after_prefix_pass != 0, a);
 }
 
 template <typename T, int D>
@@ -201,8 +224,7 @@ pa_status launch_f8(const DecodeArgs& a, const pa_cache* c, dim3 grid, cudaStrea
     return PA_ERR_CUDA;
   auto kern = decode_f8_kernel<D, G, CF>;
   if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
-  return launched();
+  return launch_kernel(kern, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, a.after_prefix_pass != 0, tk, tv, a);
 }
 
 template <int D, int CF>
@@ -232,8 +254,8 @@ pa_status launch_mma(const DecodeArgs& a, const pa_cache* c, bool persistent, cu
   if (!persistent) {
     auto kern = decode_mma_kernel<D, G>;
     if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;
-    kern<<<dim3(a.hkv, a.num_seqs, a.max_parts), Cfg::kThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
-    return launched();
+    return launch_kernel(kern, dim3(a.hkv, a.num_seqs, a.max_parts), dim3(Cfg::kThreads), Cfg::kSmemBytes, st,
+                         a.after_prefix_pass != 0, tk, tv, a);
   }
   auto kern = decode_mma_persistent_kernel<D, G>;
   static int occ[64] = {};
@@ -591,7 +613,8 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
                             int32_t max_context_len, int32_t num_groups, const int32_t* group_offsets,
                             const int32_t* group_members, const int32_t* group_prefix_tokens,
                             const int32_t* seq_prefix_tokens, int32_t max_group_size, int32_t max_prefix_tokens,
-                            float scale, float* out, void* workspace, size_t workspace_bytes, pa_stream stream) {
+                            const int32_t* seq_order, float scale, float* out, void* workspace,
+                            size_t workspace_bytes, pa_stream stream) {
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || num_groups < 0 ||
@@ -609,7 +632,8 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
   if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return PA_OK;
   if (!q || !block_tables || !context_lens || !out || !seq_prefix_tokens || !aligned16(q) || !aligned16(out) ||
-      (num_groups > 0 && (!group_offsets || !group_members || !group_prefix_tokens)))
+      (num_groups > 0 && (!group_offsets || !group_members || !group_prefix_tokens)) ||
+      (reinterpret_cast<uintptr_t>(seq_order) & 3))
     return PA_ERR_INVALID_ARG;
   if (num_seqs > 65535 || num_groups > 65535) return PA_ERR_UNSUPPORTED;
 
@@ -716,6 +740,10 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
   a.prefix_part_tokens = kCascadePrefixPart;
   // unsplit suffixes: each suffix CTA merges its sequence's prefix partials itself
   a.cascade_direct = parts == 1 ? 1 : 0;
+  a.seq_order = seq_order;
+  // the suffix pass runs alongside the prefix pass (launched just before it on
+  // this stream) and waits for it only where it folds in the prefix partials
+  a.after_prefix_pass = a.cascade_direct && num_groups > 0 && pparts > 0 ? 1 : 0;
   if (is_8bit(cache->dtype)) {
     a.scale_log2 *= cache->k_scale;
     a.v_scale = cache->v_scale;

@@ -171,6 +171,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Programmatic dependent launch (a grid launched with the
+// programmatic-stream-serialization attribute may start before the previous
+// grid on its stream has finished): the previous grid lets it start with
+// launch_dependents; the dependent grid's wait returns once the previous grid
+// has completed and its memory operations are visible. Both are no-ops when
+// the grids were launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Three-input maximum (one instruction on sm_100a; NaN-ignoring like fmaxf).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

@@ -47,7 +47,27 @@ struct DecodeArgs {
   // earlier on the stream) and stores the final rows; a sequence with an empty
   // suffix still gets its partition-0 CTA for that merge.
   int32_t cascade_direct = 0;
+  // Optional dispatch order: grid row y (or work item row) serves sequence
+  // seq_order[y], a permutation of 0 .. num_seqs-1 (longest first puts the
+  // long CTAs in the first waves). An entry out of range is recorded and that
+  // row serves sequence y.
+  const int32_t* seq_order = nullptr;
+  // Host side: launch the decode kernel as the programmatic dependent of the
+  // cascade prefix pass (it runs alongside that pass and waits for it before
+  // folding in the prefix partials).
+  int32_t after_prefix_pass = 0;
 };
+
+// Sequence served by grid (or item) row y.
+__device__ __forceinline__ int grid_seq(const DecodeArgs& a, int y, bool report) {
+  if (!a.seq_order) return y;
+  const int s = __ldg(a.seq_order + y);
+  if (s < 0 || s >= a.num_seqs) {
+    if (report) record_error(PA_ERR_DEVICE_BOUNDS, s);
+    return y;
+  }
+  return s;
+}
 
 // First token a decode CTA covers for sequence s (the cascade suffix start).
 __device__ __forceinline__ int32_t seq_start(const DecodeArgs& a, int32_t s, int32_t L) {
@@ -154,6 +174,7 @@ __device__ __forceinline__ void item_coords(const DecodeArgs& a, int item, int& 
   const int r = item - p * per;
   s = r / a.hkv;
   g = r - s * a.hkv;
+  s = grid_seq(a, s, g == 0);
 }
 
 // Named barrier over the four consumer warps (threads 0..127); the producer
@@ -315,15 +336,18 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeArgs& a, const
     }
     const int64_t row = static_cast<int64_t>(s) * a.hq + hq0 + h;
     if (a.cascade_direct) {
-      // fold in the prefix partials; each covers at least one key, so its m is finite
+      // fold in the prefix partials (written by the prefix pass: wait for it
+      // when this grid was launched alongside it); each covers at least one
+      // key, so its m is finite
+      pdl_wait();
       const float* ml = a.ws_ml + (row * a.parts_stride + a.max_parts) * 2;
       const float* po = a.ws_o + (row * a.parts_stride + a.max_parts) * D + d;
-      for (int q = 0; q < npre; ++q) {
-        const float mq = ml[2 * q];
+      for (int q = 0; q < npre; ++q) {  // through L2: written by the other grid
+        const float mq = __ldcg(ml + 2 * q);
         const float Mn = fmaxf(M, mq);
         const float f0 = exp2f(M - Mn), f1 = exp2f(mq - Mn);  // exp2(-inf) = 0 while M is -inf
-        l = l * f0 + ml[2 * q + 1] * f1;
-        o = o * f0 + po[static_cast<int64_t>(q) * D] * f1;
+        l = l * f0 + __ldcg(ml + 2 * q + 1) * f1;
+        o = o * f0 + __ldcg(po + static_cast<int64_t>(q) * D) * f1;
         M = Mn;
       }
       a.out[row * D + d] = l > 0.f ? o / l : 0.f;  // an empty context gives a zero row

@@ -517,7 +517,8 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
 
-  const int g = blockIdx.x, s = blockIdx.y, p = blockIdx.z;
+  const int g = blockIdx.x, p = blockIdx.z;
+  const int s = grid_seq(a, blockIdx.y, g == 0 && p == 0 && threadIdx.x == 0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = lane >> 2, c = lane & 3;
   Part pt;

@@ -154,7 +154,8 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
   T* sK = reinterpret_cast<T*>(smem);
   T* sV = sK + S * C * D;
 
-  const int g = blockIdx.x, s = blockIdx.y, p = blockIdx.z;
+  const int g = blockIdx.x, p = blockIdx.z;
+  const int s = grid_seq(a, blockIdx.y, g == 0 && p == 0 && threadIdx.x == 0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Part pt;
   if (!cta_part<G, D>(a, g, s, p, tid, Cfg::kThreads, pt)) return;

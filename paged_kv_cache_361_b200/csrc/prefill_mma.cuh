@@ -83,8 +83,11 @@ constexpr int prefill_mma_smem_bytes() {
 // CASCADE = false: prefill (rows = new tokens x heads, causal).
 // CASCADE = true: shared-prefix decode (rows = group members x heads, every
 // row sees the whole prefix partition; partial results, not rows, are stored).
+#ifndef PA_PMMA_MAXNREG
+#define PA_PMMA_MAXNREG 168
+#endif
 template <int D, int G, bool CASCADE, int CF = 0>
-__global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void __maxnreg__(PA_PMMA_MAXNREG) prefill_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                          const __grid_constant__ CUtensorMap tmv,
                                                                          const PrefillArgs a) {
   using Cfg = MmaCfg<D>;
@@ -103,6 +106,9 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) prefill_mma_kernel(const 
 
   const int g = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // cascade: the suffix pass, launched as this grid's programmatic dependent,
+  // may start now; it waits for this whole grid before it reads the partials
+  if (CASCADE) pdl_launch_dependents();
 
   // key range [k_begin, kend) of this CTA and the mapping of its 64 rows
   int32_t k_begin = 0, kend = 0, base = 0, tok0 = 0, n = 0, q0 = 0, moff = 0, msz = 0;

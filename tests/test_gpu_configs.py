@@ -275,3 +275,53 @@ def test_cascade_empty_suffix_and_empty_sequence():
     assert torch.isfinite(b).all()
     assert float(b[4].abs().max()) == 0.0
     assert float((a - b).abs().max()) <= 2e-3
+
+
+def test_cascade_dispatch_order():
+    """The suffix CTAs' dispatch order (seq_order) changes no result: no order,
+    longest first and reversed give bitwise-equal outputs; an entry out of range
+    is recorded as a bounds error and its row served in batch order."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    rng = np.random.default_rng(7)
+    hkv, G, D, bs = 2, 4, 128, 16
+    cache = PagedKVCache(4000, hkv, bs, D, torch.bfloat16, "cuda", rng.permutation(4000), fill=float("nan"))
+    g = torch.Generator().manual_seed(7)
+    ids = []
+    for fam in range(4):
+        root = fam * 100
+        n0 = int(rng.integers(64, 600))
+        cache.add_sequence(root, torch.randn(n0, hkv, D, generator=g).bfloat16().cuda(),
+                           torch.randn(n0, hkv, D, generator=g).bfloat16().cuda())
+        ids.append(root)
+        for j in range(1, 6):
+            cache.fork(root, root + j)
+            ids.append(root + j)
+    for s in ids:                                    # suffixes of different lengths
+        for _ in range(int(rng.integers(0, 90))):
+            cache.append([s], torch.randn(1, hkv, D, generator=g).bfloat16().cuda(),
+                         torch.randn(1, hkv, D, generator=g).bfloat16().cuda())
+    n = len(ids)
+    q = torch.randn(n, hkv * G, D, generator=g).bfloat16().cuda()
+    tables, lens, max_len = cache.decode_inputs(ids)
+    offs, members, prefix, seq_prefix, max_pre = cache.shared_prefix_groups(ids, 64 // G)
+    order = cache.bm.longest_first(ids, seq_prefix)
+    span = np.array([cache.lens[s] for s in ids]) - seq_prefix
+    assert sorted(order.tolist()) == list(range(n)) and (np.diff(span[order]) <= 0).all()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+    ws = torch.empty(B.pa_decode_cascade_workspace_bytes(n, hkv * G, hkv, D, max_len, bs, max_pre),
+                     dtype=torch.uint8, device="cuda")
+    args = (t(offs), t(members), t(prefix), t(seq_prefix), int(max(np.diff(offs), default=0)), max_pre, ws)
+    outs = []
+    bad = np.arange(n, dtype=np.int32)
+    bad[3] = n + 5
+    for so in (None, order, order[::-1], bad):
+        out = torch.full((n, hkv * G, D), float("nan"), dtype=torch.float32, device="cuda")
+        B.pa_decode_cascade(q, cache.k_cache, cache.v_cache, t(tables), t(lens), D ** -0.5, out, max_len, *args,
+                            seq_order=None if so is None else t(so))
+        st, info = B.pa_get_device_error()
+        assert (st, info) == ((B.PA_ERR_DEVICE_BOUNDS, n + 5) if so is bad else (B.PA_OK, 0))
+        outs.append(out)
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    ref = cache.decode(ids, q, D ** -0.5)
+    assert float((ref - outs[0]).abs().max()) <= 2e-3

@@ -86,3 +86,20 @@ def test_cpp_prefix_groups_errors():
     assert e.value.status == B.PA_ERR_INVALID_ARG
     off, mem, pre, sp, mp = bm.prefix_groups([], 4)
     assert off.tolist() == [0] and len(mem) == 0 and mp == 0
+
+
+def test_cpp_longest_first():
+    """pa_bm_longest_first: rows by decreasing (tokens - skip), ties in batch
+    order; unknown ids and missing arrays are errors."""
+    bm = B.BlockManager(64, 4)
+    for sid, n in ((10, 5), (11, 9), (12, 9), (13, 1), (14, 12)):
+        bm.add_seq(sid, n)
+    assert bm.longest_first([10, 11, 12, 13, 14]).tolist() == [4, 1, 2, 0, 3]
+    # spans 5-0, 9-8, 9-0, 1-0, 12-12 -> 9, 5, 1, 1, 0
+    assert bm.longest_first([10, 11, 12, 13, 14], [0, 8, 0, 0, 12]).tolist() == [2, 0, 1, 3, 4]
+    assert bm.longest_first([]).tolist() == []
+    with pytest.raises(B.PagedAttnError) as e:
+        bm.longest_first([10, 99])
+    assert e.value.status == B.PA_ERR_UNKNOWN_SEQ
+    with pytest.raises(ValueError):
+        bm.longest_first([10, 11], [0])
