@@ -195,6 +195,23 @@ bool encode_rows(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A bf16 pool with head_dim 128 for the grouped-head decode: one copy per
+// (block, head) tile. Dimensions (64 elements, pool rows, 2 halves) with byte
+// strides (256 per row, 128 per half) and a box of (64, bs, 2): the copy
+// lands as [half][row][128 bytes] with the 128-byte swizzle, as the two 2-D
+// column boxes would, in one request instead of two.
+bool encode_rows_halves(CUtensorMap* map, void* base, uint64_t rows, int bs) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {64, rows, 2};
+  const cuuint64_t strides[2] = {256, 128};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(bs), 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // An e4m3 pool viewed as rows of head_dim bytes, read in [bs x head_dim] boxes
 // with the 128-byte (head_dim 128) or 64-byte (head_dim 64) swizzle.
 bool encode_rows_u8(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) {
@@ -249,8 +266,11 @@ pa_status launch_mma(const DecodeArgs& a, const pa_cache* c, bool persistent, cu
   using Cfg = MmaCfg<D>;
   CUtensorMap tk, tv;
   const uint64_t rows = static_cast<uint64_t>(c->num_blocks) * c->num_kv_heads * c->block_size;
-  if (!encode_rows(&tk, c->k, rows, D, c->block_size) || !encode_rows(&tv, c->v, rows, D, c->block_size))
-    return PA_ERR_CUDA;
+  const bool ok = D == 128 ? encode_rows_halves(&tk, c->k, rows, c->block_size) &&
+                                 encode_rows_halves(&tv, c->v, rows, c->block_size)
+                           : encode_rows(&tk, c->k, rows, D, c->block_size) &&
+                                 encode_rows(&tv, c->v, rows, D, c->block_size);
+  if (!ok) return PA_ERR_CUDA;
   if (!persistent) {
     auto kern = decode_mma_kernel<D, G>;
     if (!smem_attrs(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, true)) return PA_ERR_CUDA;

@@ -48,6 +48,29 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// The same for a 3-D map: coordinates (x, y, z).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// One (block, kv head) tile of K or V, [bs rows x D], into a stage: one copy
+// whatever D is. At D 128 the map is 3-D (x: 64 elements = one 128-byte
+// column box, y: pool row, z: which 64-element half, stride 128 bytes), so the
+// copy lands as [half][row][128 B]; at D 64 it is the 2-D [row][128 B] box.
+template <int D>
+__device__ __forceinline__ void tma_block(uint32_t dst, const CUtensorMap* map, int32_t y, uint64_t* bar,
+                                          uint64_t policy) {
+  if constexpr (D == 128)
+    tma_load_3d(dst, map, 0, y, 0, bar, policy);
+  else
+    tma_load_2d(dst, map, 0, y, bar, policy);
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -105,6 +128,12 @@ __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint3
 // Build-time tuning knobs of the one-CTA-per-item kernel (defaults measured
 // on B200): ring stages at head_dim 128 (0 = the default of 3), and the CTAs
 // per SM its register budget is fitted to.
+// Build-time knob: k-steps (and P V steps) whose shared-memory fragments are
+// loaded ahead of the MMAs in mma_chunk.
+#ifndef PA_MMA_PREFETCH
+#define PA_MMA_PREFETCH 4
+#endif
+
 #ifndef PA_MMA_STAGES
 #define PA_MMA_STAGES 0
 #endif
@@ -125,7 +154,7 @@ struct MmaCfg {
   static constexpr int kThreads = 32 * (kConsumerWarps + 1);
   static constexpr int kChunk = 64;                        // tokens per stage
   static constexpr int kHalves = D / 64;                   // 128-byte column boxes per row
-  static constexpr int kHalfBytes = kChunk * 128;          // one box column of a stage
+  static constexpr int kHalfBytes = kChunk * 128;          // one 64-element column of a stage's K (or V)
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = kStageBytes <= 16384 ? 4 : (PA_MMA_STAGES > 0 ? PA_MMA_STAGES : 3);
@@ -145,7 +174,7 @@ struct MmaCfg {
 template <int D>
 __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, const uint32_t (&qa)[D / 16][2],
                                           float scale_log2, int lane, int warp, float& m_run, float& l_run,
-                                          float (&o)[D / 8][2]) {
+                                          float (&o)[D / 8][2], int bs) {
   using Cfg = MmaCfg<D>;
   constexpr int NT = D / 8;
   const int c = lane & 3;
@@ -158,15 +187,41 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
   float dead0[2] = {0.f, 0.f}, dead1[2] = {0.f, 0.f};
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  // K fragments run kPre k-steps ahead of the MMAs that use them (a ring of
+  // kPre x 4 registers), so a load's latency is hidden behind earlier MMAs
+  // instead of stalling each k-step (the asm statements keep source order)
+  constexpr int kPre = PA_MMA_PREFETCH;
+  constexpr int KS = D / 16;
+  // stage layout: block b of the chunk at b * bs * D * 2 bytes, inside it the
+  // 64-element half h at h * bs * 128, row t at t * 128, its 16-byte pieces
+  // swizzled by (t & 7) (the 128-byte swizzle of the TMA; block and half
+  // offsets are multiples of 1024 bytes, so the phase is the token's)
+  const uint32_t hstride = static_cast<uint32_t>(bs) * 128u;
+  const uint32_t kbase = kst + (tokK + (tokK & ~(bs - 1)) * (Cfg::kHalves - 1)) * 128;
+  const uint32_t vbase = vst + (tokV + (tokV & ~(bs - 1)) * (Cfg::kHalves - 1)) * 128;
+  auto k_addr = [&](int kk) {
     const int d0 = kk * 16 + dK;
-    const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tokK * 128 + ((((d0 & 63) >> 3) ^ (tokK & 7)) << 4);
-    uint32_t b00, b01, b10, b11;
-    ldsm_x4(addr, b00, b01, b10, b11);
+    return kbase + (d0 >> 6) * hstride + ((((d0 & 63) >> 3) ^ (tokK & 7)) << 4);
+  };
+  auto v_addr = [&](int dgi) {
+    const int d0 = dgi * 16 + dV;
+    return vbase + (d0 >> 6) * hstride + ((((d0 & 63) >> 3) ^ (tokV & 7)) << 4);
+  };
+  uint32_t kf[kPre][4];
+#pragma unroll
+  for (int u = 0; u < kPre; ++u) ldsm_x4(k_addr(u), kf[u][0], kf[u][1], kf[u][2], kf[u][3]);
+#pragma unroll
+  for (int kk = 0; kk < KS; ++kk) {
+    const uint32_t b00 = kf[kk % kPre][0], b01 = kf[kk % kPre][1], b10 = kf[kk % kPre][2], b11 = kf[kk % kPre][3];
+    if (kk + kPre < KS)
+      ldsm_x4(k_addr(kk + kPre), kf[kk % kPre][0], kf[kk % kPre][1], kf[kk % kPre][2], kf[kk % kPre][3]);
     mma_rows8_chain(sacc[0], qa[kk][0], qa[kk][1], b00, b01, dead0);
     mma_rows8_chain(sacc[1], qa[kk][0], qa[kk][1], b10, b11, dead1);
   }
+  // the first V fragments are loaded before the softmax, which hides their latency
+  uint32_t vf[kPre][4];
+#pragma unroll
+  for (int u = 0; u < kPre; ++u) ldsm_x4_t(v_addr(u), vf[u][0], vf[u][1], vf[u][2], vf[u][3]);
   float sc[2][2];
   float mloc = -INFINITY;
 #pragma unroll
@@ -213,10 +268,9 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
   }
 #pragma unroll
   for (int dgi = 0; dgi < D / 16; ++dgi) {
-    const int d0 = dgi * 16 + dV;
-    const uint32_t addr = vst + (d0 >> 6) * Cfg::kHalfBytes + tokV * 128 + ((((d0 & 63) >> 3) ^ (tokV & 7)) << 4);
-    uint32_t v0, v1, v2, v3;
-    ldsm_x4_t(addr, v0, v1, v2, v3);
+    uint32_t v0 = vf[dgi % kPre][0], v1 = vf[dgi % kPre][1], v2 = vf[dgi % kPre][2], v3 = vf[dgi % kPre][3];
+    if (dgi + kPre < D / 16)
+      ldsm_x4_t(v_addr(dgi + kPre), vf[dgi % kPre][0], vf[dgi % kPre][1], vf[dgi % kPre][2], vf[dgi % kPre][3]);
     v0 &= mlo;
     v1 &= mhi;
     v2 &= mlo;
@@ -331,7 +385,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
 
   if (warp == NW) {
     // ------------------------------ producer ------------------------------
-    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D * 2u;  // one (block, head) tile of K or V
     const uint64_t pol = kv_stream_policy();
     const __nv_bfloat16* qbase = static_cast<const __nv_bfloat16*>(a.q);
     int item = blockIdx.x;
@@ -356,8 +410,18 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
         const int nch = (t1 - t0 + C - 1) / C;
         const int nparts = a.part_tokens > 0 ? (span + P - 1) / P : 1;
         const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
+        // block ids of chunk ch (lane < its block count), loaded one chunk
+        // ahead so that the table read overlaps the wait for a free stage
+        auto chunk_ids = [&](int ch) -> int32_t {
+          const int32_t c0 = t0 + ch * C;
+          const int32_t nb = (min(C, t1 - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
+          return lane < nb ? __ldg(a.tables + table_row + c0 / a.bs + lane) : -1;
+        };
+        int32_t blk_next = chunk_ids(0);
         for (int ch = 0; ch < nch; ++ch, ++cs) {
           const int st = cs % S;
+          const int32_t blk = blk_next;
+          if (ch + 1 < nch) blk_next = chunk_ids(ch + 1);
           if (cs >= S && !pipe_wait(&ps.empty[st], ((cs / S) - 1) & 1, &ps.abort_flag)) {
             aborted = true;
             break;
@@ -365,10 +429,8 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
           const int32_t c0 = t0 + ch * C;
           const int32_t n = min(C, t1 - c0);
           const int32_t nb = (n + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
-          int32_t blk = -1;
           bool ok = false;
           if (lane < nb) {
-            blk = __ldg(a.tables + table_row + c0 / a.bs + lane);
             ok = blk >= 0 && blk < a.num_blocks;
             if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
           }
@@ -382,7 +444,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
             d.nparts = nparts;
             d.flags = (ch == 0 ? kDescFirst : 0) | (ch == nch - 1 ? kDescLast : 0);
             const uint32_t qbytes = ch == 0 ? static_cast<uint32_t>(G * D * 2) : 0u;
-            mbar_arrive_expect_tx(&ps.full[st], 2u * Cfg::kHalves * __popc(okmask) * box_bytes + qbytes);
+            mbar_arrive_expect_tx(&ps.full[st], 2u * __popc(okmask) * box_bytes + qbytes);
             if (ch == 0)
               bulk_g2s(sgen + S * Cfg::kStageBytes + st * Cfg::kQBytes,
                        qbase + (static_cast<int64_t>(s) * a.hq + g * G) * D, qbytes, &ps.full[st], pol);
@@ -391,11 +453,8 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
           if (ok) {
             const int32_t y = (blk * a.hkv + g) * a.bs;
             const uint32_t kdst = sbase + st * Cfg::kStageBytes + lane * box_bytes;
-#pragma unroll
-            for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-              tma_load_2d(kdst + hf * Cfg::kHalfBytes, &tmk, hf * 64, y, &ps.full[st], pol);
-              tma_load_2d(kdst + Cfg::kTileBytes + hf * Cfg::kHalfBytes, &tmv, hf * 64, y, &ps.full[st], pol);
-            }
+            tma_block<D>(kdst, &tmk, y, &ps.full[st], pol);
+            tma_block<D>(kdst + Cfg::kTileBytes, &tmv, y, &ps.full[st], pol);
           }
         }
       }
@@ -448,7 +507,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
     const int nv = min(16, dn - warp * 16);  // warp-uniform
     if (nv > 0) {
       const uint32_t kst = sbase + st * Cfg::kStageBytes;
-      mma_chunk<D>(kst, kst + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
+      mma_chunk<D>(kst, kst + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o, a.bs);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&ps.empty[st]);
@@ -536,7 +595,7 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
 
   if (warp == NW) {
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
-    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D * 2u;  // one (block, head) tile of K or V
     const uint64_t pol = kv_stream_policy();
     TableAhead ta;
     ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
@@ -550,16 +609,13 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
         if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
       }
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * Cfg::kHalves * __popc(okmask) * box_bytes);
+      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * __popc(okmask) * box_bytes);
       __syncwarp();
       if (ok) {
         const int32_t y = (blk * a.hkv + g) * a.bs;
         const uint32_t kdst = sbase + st * Cfg::kStageBytes + lane * box_bytes;
-#pragma unroll
-        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-          tma_load_2d(kdst + hf * Cfg::kHalfBytes, &tmk, hf * 64, y, &ps.full[st], pol);
-          tma_load_2d(kdst + Cfg::kTileBytes + hf * Cfg::kHalfBytes, &tmv, hf * 64, y, &ps.full[st], pol);
-        }
+        tma_block<D>(kdst, &tmk, y, &ps.full[st], pol);
+        tma_block<D>(kdst + Cfg::kTileBytes, &tmv, y, &ps.full[st], pol);
       }
     });
   } else {
@@ -573,7 +629,7 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
       const int nv = min(16, min(C, pt.ntok - i * C) - warp * 16);  // warp-uniform
       if (nv > 0) {
         const uint32_t kst = sbase + st * Cfg::kStageBytes;
-        mma_chunk<D>(kst, kst + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o);
+        mma_chunk<D>(kst, kst + Cfg::kTileBytes, nv, qa, a.scale_log2, lane, warp, m_run, l_run, o, a.bs);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ps.empty[st]);
