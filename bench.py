@@ -279,6 +279,8 @@ def build_workload(seed: int, device, name: str = "llama2_7b_mha", kv_dtype: str
         v=torch.randn((B_, hkv, D), generator=g, device=device).to(dt),
         slots=torch.from_numpy(slots).to(device),
         pairs=torch.from_numpy(pairs).to(device) if len(pairs) else None,
+        # dispatch order of the decode CTAs: longest sequence first (C++ block manager)
+        order=torch.from_numpy(cache.bm.longest_first(ids)).to(device),
         tables=torch.from_numpy(tables).to(device),
         lens=torch.from_numpy(lens32).to(device),
         lens_host=lens32.astype(np.int64),
@@ -422,7 +424,8 @@ def decode_fns(B, d, P, cascade=None):
             B.pa_decode_cascade(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"],
                                 *cascade)
             return
-        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"], P, ws)
+        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"], P, ws,
+                    seq_order=d["order"])
     return write_step, decode
 
 
@@ -511,7 +514,7 @@ def run_ours(args, rank, world, device):
                    "partition_tokens": P_eff,
                    "kv_dtype": dtype_key,
                    "decode": "pa_decode_cascade (shared prefixes read once per group)" if cascade is not None
-                   else "pa_decode",
+                   else "pa_decode_ordered (longest sequence first)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "no flush: the K/V read per step is larger than the 126 MB L2"
                    if d["unique_kv_bytes"] > 3 * 126e6 else "no flush: K/V partly L2-resident (see unique bytes)"},
@@ -601,12 +604,14 @@ def batching_trace(device, seed=0, kv_dtype="auto", num_blocks=None):
                 cache.lens[s] += 1
         elif op[0] == "decode":
             tables, lens32, max_len = cache.decode_inputs(op[1])
+            order = cache.bm.longest_first(op[1])
         t_host += time.perf_counter() - t0
         if op[0] == "decode":
             host_s.append(t_host)
             t_host = 0.0
             steps.append(dict(slots=torch.from_numpy(pending_slots).to(device),
                               tables=torch.from_numpy(tables).to(device), lens=torch.from_numpy(lens32).to(device),
+                              order=torch.from_numpy(order).to(device),
                               max_len=int(max_len), tokens=int(lens32.astype(np.int64).sum()), n=len(op[1])))
     n = steps[0]["n"]
     hkv, D = sh.num_kv_heads, sh.head_dim
@@ -636,7 +641,8 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None,
             B.pa_reshape_and_cache(io["k"], io["v"], st["slots"], kc, vc)
             if evs is not None:
                 evs[i][0].record(stream)
-            B.pa_decode(io["q"], kc, vc, st["tables"], st["lens"], scale, io["out"], st["max_len"], partition, ws)
+            B.pa_decode(io["q"], kc, vc, st["tables"], st["lens"], scale, io["out"], st["max_len"], partition, ws,
+                        seq_order=st["order"])
             if evs is not None:
                 evs[i][1].record(stream)
 
@@ -671,7 +677,8 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None,
            "host_block_manager_ms_avg": round(1e3 * statistics.mean(host_s), 4),
            "host_block_manager_ms_max": round(1e3 * max(host_s), 4),
            "host_note": "C++ block manager through the ctypes binding per step: frees, arrival reservations, one "
-                        "slot per live sequence, block tables; timed on the host, outside the device time",
+                        "slot per live sequence, block tables, longest-first dispatch order; timed on the host, "
+                        "outside the device time",
            "partition_tokens": sorted({B.pa_decode_partition_tokens(st["n"], sh.num_q_heads, sh.num_kv_heads,
                                                                     st["max_len"], sh.block_size)
                                        if partition < 0 else partition for st in steps}),

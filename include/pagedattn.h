@@ -196,6 +196,25 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
                     size_t workspace_bytes, pa_stream stream);
 
 /*
+ * pa_decode with a dispatch order: sequence seq_order[y] is served by grid
+ * row y (and, in the persistent kernels, by the items of row y), so passing
+ * the rows longest first (pa_bm_longest_first) starts the long CTAs in the
+ * first waves and leaves the short ones for the end. Results are those of
+ * pa_decode, bit for bit.
+ *   seq_order  device int32 [num_seqs], a permutation of 0 .. num_seqs-1,
+ *              4-byte aligned (NULL: batch order). An entry out of range is
+ *              recorded as PA_ERR_DEVICE_BOUNDS (pa_get_device_error) and its
+ *              row served in batch order; a repeated entry leaves some
+ *              sequence uncomputed (no memory outside the arguments is
+ *              touched).
+ * Other arguments, supported shapes and errors as pa_decode.
+ */
+pa_status pa_decode_ordered(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                            int32_t max_context_len, const int32_t* seq_order, float scale, float* out,
+                            int32_t partition_tokens, void* workspace, size_t workspace_bytes, pa_stream stream);
+
+/*
  * Causal attention of newly written prompt tokens (prefill, possibly in
  * chunks) over the paged cache. P2 §3.2.1: the prompt's K, V are computed and
  * written into the sequence's blocks (pa_reshape_and_cache first); each new

@@ -51,6 +51,7 @@ _SIGS = {
     "pa_reshape_and_cache": (_I32, [_VP, _VP, _VP, _I32, _PCACHE, _VP]),
     "pa_copy_blocks": (_I32, [_PCACHE, _VP, _I32, _VP]),
     "pa_decode": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP, _SZ, _VP]),
+    "pa_decode_ordered": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _VP, _F, _VP, _I32, _VP, _SZ, _VP]),
     "pa_decode_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
     "pa_decode_cascade": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32,
                                  _VP, _F, _VP, _VP, _SZ, _VP]),
@@ -187,7 +188,9 @@ def pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max
 
 
 def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_context_len,
-              partition_tokens=-1, workspace=None, stream=None):
+              partition_tokens=-1, workspace=None, stream=None, seq_order=None):
+    """pa_decode, or pa_decode_ordered when seq_order (device int32, one entry
+    per sequence: the dispatch order) is given."""
     c = make_cache(k_cache, v_cache)
     B, hq, d = q.shape
     _dev(q, "q", input_dtype(k_cache.dtype), 3)
@@ -200,6 +203,15 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_c
         raise ValueError("block_tables / context_lens must have num_seqs rows")
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (_dev(workspace, "workspace"),
                                                             workspace.numel() * workspace.element_size())
+    if seq_order is not None:
+        _dev(seq_order, "seq_order", torch.int32, 1)
+        if seq_order.shape[0] != B:
+            raise ValueError("seq_order must have one entry per sequence")
+        _check(_lib().pa_decode_ordered(q.data_ptr(), B, hq, ctypes.byref(c), block_tables.data_ptr(),
+                                        int(block_tables.shape[1]), context_lens.data_ptr(), int(max_context_len),
+                                        seq_order.data_ptr(), float(scale), out.data_ptr(), int(partition_tokens),
+                                        ws_ptr, ws_bytes, _stream(q, stream)), "pa_decode_ordered")
+        return
     _check(_lib().pa_decode(q.data_ptr(), B, hq, ctypes.byref(c), block_tables.data_ptr(),
                             int(block_tables.shape[1]), context_lens.data_ptr(), int(max_context_len), float(scale),
                             out.data_ptr(), int(partition_tokens), ws_ptr, ws_bytes, _stream(q, stream)), "pa_decode")

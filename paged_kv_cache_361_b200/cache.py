@@ -156,9 +156,11 @@ class PagedKVCache:
         return self._ws
 
     def decode(self, seq_ids, q: torch.Tensor, scale: float | None = None, out: torch.Tensor | None = None,
-               partition_tokens: int = -1) -> torch.Tensor:
+               partition_tokens: int = -1, longest_first: bool = True) -> torch.Tensor:
         """Decode attention for the listed sequences with queries q [n][Hq][D];
-        returns fp32 [n][Hq][D]."""
+        returns fp32 [n][Hq][D]. longest_first dispatches the longest
+        sequences' CTAs first (pa_bm_longest_first, pa_decode_ordered); the
+        result is the same bit for bit."""
         n, hq, d = q.shape
         if scale is None:
             scale = 1.0 / math.sqrt(d)
@@ -167,8 +169,9 @@ class PagedKVCache:
             out = torch.empty((n, hq, d), dtype=torch.float32, device=self.device)
         hkv = self.k_cache.shape[1]
         nbytes = B.pa_decode_workspace_bytes(n, hq, hkv, d, max_len, self.block_size, partition_tokens)
+        order = self._lens.upload(self.bm.longest_first(seq_ids)) if longest_first and n > 1 else None
         B.pa_decode(q, self.k_cache, self.v_cache, self._tables.upload(tables), self._lens.upload(lens), scale, out,
-                    max_len, partition_tokens, self.workspace(nbytes))
+                    max_len, partition_tokens, self.workspace(nbytes), seq_order=order)
         return out
 
     def prefill(self, seq_ids, counts, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,

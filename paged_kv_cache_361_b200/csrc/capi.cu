@@ -703,9 +703,17 @@ pa_status pa_decode_cascade(const void* q, int32_t num_seqs, int32_t num_q_heads
     pa.ws_o = ws_o;
     CUtensorMap tk, tv;
     const uint64_t rows = static_cast<uint64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
-    auto enc = is_8bit(cache->dtype) ? encode_rows_u8 : encode_rows;
-    if (!enc(&tk, cache->k, rows, D, cache->block_size) || !enc(&tv, cache->v, rows, D, cache->block_size))
-      return PA_ERR_CUDA;
+    bool enc_ok;
+    if (is_8bit(cache->dtype))
+      enc_ok = encode_rows_u8(&tk, cache->k, rows, D, cache->block_size) &&
+               encode_rows_u8(&tv, cache->v, rows, D, cache->block_size);
+    else if (D == 128)  // one copy per (block, head) tile, as the grouped-head decode
+      enc_ok = encode_rows_halves(&tk, cache->k, rows, cache->block_size) &&
+               encode_rows_halves(&tv, cache->v, rows, cache->block_size);
+    else
+      enc_ok = encode_rows(&tk, cache->k, rows, D, cache->block_size) &&
+               encode_rows(&tv, cache->v, rows, D, cache->block_size);
+    if (!enc_ok) return PA_ERR_CUDA;
     const dim3 grid(cache->num_kv_heads, pparts, num_groups);
     auto launch = [&](auto kern, int smem) -> pa_status {
       // the largest shared-memory carveout: two of these CTAs fit an SM
@@ -796,10 +804,12 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
   return ws_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, num_parts(max_context_len, P));
 }
 
-pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
-                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
-                    int32_t max_context_len, float scale, float* out, int32_t partition_tokens, void* workspace,
-                    size_t workspace_bytes, pa_stream stream) {
+namespace {
+
+pa_status decode_impl(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                      const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                      int32_t max_context_len, const int32_t* seq_order, float scale, float* out,
+                      int32_t partition_tokens, void* workspace, size_t workspace_bytes, pa_stream stream) {
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0) return PA_ERR_INVALID_ARG;
@@ -813,7 +823,8 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
     return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return PA_OK;
   if (!q || !block_tables || !context_lens || !out || !aligned16(q) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
+      (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3) ||
+      (reinterpret_cast<uintptr_t>(seq_order) & 3))
     return PA_ERR_INVALID_ARG;
   if (num_seqs > 65535) return PA_ERR_UNSUPPORTED;
 
@@ -852,6 +863,7 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   a.force_partials = 0;
   a.parts_stride = parts;
   a.prefix_part_tokens = 0;
+  a.seq_order = seq_order;
   if (is_8bit(cache->dtype)) {
     // q . (k_scale * code) = (k_scale * q) . code; the V scale multiplies o.
     a.scale_log2 *= cache->k_scale;
@@ -887,6 +899,24 @@ pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const 
   }
   if (st != PA_OK || parts <= 1 || a.fuse_merge) return st;
   return D == 128 ? launch_reduce<128>(a, s) : launch_reduce<64>(a, s);
+}
+
+}  // namespace
+
+pa_status pa_decode(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, float scale, float* out, int32_t partition_tokens, void* workspace,
+                    size_t workspace_bytes, pa_stream stream) {
+  return decode_impl(q, num_seqs, num_q_heads, cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, nullptr, scale, out, partition_tokens, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_ordered(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                            int32_t max_context_len, const int32_t* seq_order, float scale, float* out,
+                            int32_t partition_tokens, void* workspace, size_t workspace_bytes, pa_stream stream) {
+  return decode_impl(q, num_seqs, num_q_heads, cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, seq_order, scale, out, partition_tokens, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_selftest_wait_timeout(int64_t timeout_ns, pa_stream stream) {

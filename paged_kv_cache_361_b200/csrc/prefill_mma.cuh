@@ -175,7 +175,7 @@ __global__ void __maxnreg__(PA_PMMA_MAXNREG) prefill_mma_kernel(const __grid_con
     return;
   }
   if (warp == NW) {
-    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
+    const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D * 2u;  // one (block, head) tile of K or V
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       const int32_t c0 = k_begin + i * C;
@@ -188,16 +188,13 @@ __global__ void __maxnreg__(PA_PMMA_MAXNREG) prefill_mma_kernel(const __grid_con
         if (!ok) record_error(PA_ERR_DEVICE_BOUNDS, blk);
       }
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * Cfg::kHalves * __popc(okmask) * box_bytes);
+      if (lane == 0) mbar_arrive_expect_tx(&ps.full[st], 2u * __popc(okmask) * box_bytes);
       __syncwarp();
       if (ok) {
         const int32_t y = (blk * a.hkv + g) * a.bs;
         const uint32_t kdst = sbase + st * Cfg::kStageBytes + lane * box_bytes;
-#pragma unroll
-        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-          tma_load_2d(kdst + hf * Cfg::kHalfBytes, &tmk, hf * 64, y, &ps.full[st], pol);
-          tma_load_2d(kdst + Cfg::kTileBytes + hf * Cfg::kHalfBytes, &tmv, hf * 64, y, &ps.full[st], pol);
-        }
+        tma_block<D>(kdst, &tmk, y, &ps.full[st], pol);
+        tma_block<D>(kdst + Cfg::kTileBytes, &tmv, y, &ps.full[st], pol);
       }
     });
     return;
@@ -249,6 +246,17 @@ __global__ void __maxnreg__(PA_PMMA_MAXNREG) prefill_mma_kernel(const __grid_con
   float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
 
   const int mk = lane >> 3, ik = lane & 7;
+  // address of row t, dims d0 .. d0+7 of a stage tile: block-major as the TMA
+  // writes it over a bf16 cache (block t / bs at t / bs * bs * D * 2 bytes,
+  // 64-element half at half * bs * 128, row at (t % bs) * 128), half-major as
+  // the converter writes it over an 8-bit cache; 128-byte swizzle phase t & 7
+  auto tile_addr = [&](uint32_t base, int t, int d0) -> uint32_t {
+    const uint32_t swz = static_cast<uint32_t>((((d0 & 63) >> 3) ^ (t & 7)) << 4);
+    if constexpr (CF != 0)
+      return base + (d0 >> 6) * Cfg::kHalfBytes + t * 128 + swz;
+    else
+      return base + (t + (t & ~(a.bs - 1)) * (Cfg::kHalves - 1)) * 128 + (d0 >> 6) * a.bs * 128 + swz;
+  };
   for (int i = 0; i < nchunks; ++i) {
     const int st = i % S;
     if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
@@ -277,7 +285,7 @@ __global__ void __maxnreg__(PA_PMMA_MAXNREG) prefill_mma_kernel(const __grid_con
 #pragma unroll
         for (int kg = 0; kg < 4; ++kg) {
           const int tk = kg * 16 + (mk >> 1) * 8 + ik;
-          const uint32_t addr = kst + (d0 >> 6) * Cfg::kHalfBytes + tk * 128 + ((((d0 & 63) >> 3) ^ (tk & 7)) << 4);
+          const uint32_t addr = tile_addr(kst, tk, d0);
           uint32_t b00, b01, b10, b11;
           ldsm_x4(addr, b00, b01, b10, b11);
           if constexpr (CF != 0) {
@@ -357,7 +365,7 @@ __global__ void __maxnreg__(PA_PMMA_MAXNREG) prefill_mma_kernel(const __grid_con
 #pragma unroll
         for (int dg = 0; dg < D / 16; ++dg) {
           const int d0 = dg * 16 + (mk >> 1) * 8;
-          const uint32_t addr = vst + (d0 >> 6) * Cfg::kHalfBytes + tv * 128 + ((((d0 & 63) >> 3) ^ (tv & 7)) << 4);
+          const uint32_t addr = tile_addr(vst, tv, d0);
           uint32_t v0, v1, v2, v3;
           ldsm_x4_t(addr, v0, v1, v2, v3);
           v0 &= mlo;

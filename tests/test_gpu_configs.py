@@ -325,3 +325,45 @@ def test_cascade_dispatch_order():
         assert torch.equal(o, outs[0])
     ref = cache.decode(ids, q, D ** -0.5)
     assert float((ref - outs[0]).abs().max()) <= 2e-3
+
+
+@pytest.mark.parametrize("dtype,G,part", [("bf16", 1, 0), ("bf16", 4, 0), ("bf16", 4, 128), ("bf16", 8, 256),
+                                           ("bf16", 2, 64), ("e4m3", 1, 0), ("e4m3", 4, 128), ("int8", 8, 0)])
+def test_decode_ordered_matches_decode(dtype, G, part):
+    """pa_decode_ordered is pa_decode bit for bit whatever the order (longest
+    first, reversed), on every kernel family: CUDA-core (G 1-2), tensor-core
+    one-CTA-per-item and persistent (split), 8-bit; an out-of-range entry is
+    recorded and its row served in batch order."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    rng = np.random.default_rng(G * 7 + part)
+    hkv, D, bs = 2, 128, 16
+    tdt = {"bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn, "int8": torch.int8}[dtype]
+    sc = 4.0 / 127 if dtype == "int8" else 1.0
+    cache = PagedKVCache(3000, hkv, bs, D, tdt, "cuda", rng.permutation(3000), k_scale=sc, v_scale=sc)
+    g = torch.Generator().manual_seed(G + part)
+    ids = list(range(23))
+    for s in ids:
+        n = int(rng.integers(1, 900))
+        cache.add_sequence(s, torch.randn(n, hkv, D, generator=g).bfloat16().cuda(),
+                           torch.randn(n, hkv, D, generator=g).bfloat16().cuda())
+    n = len(ids)
+    q = torch.randn(n, hkv * G, D, generator=g).bfloat16().cuda()
+    tables, lens, max_len = cache.decode_inputs(ids)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+    ws = torch.empty(max(256, B.pa_decode_workspace_bytes(n, hkv * G, hkv, D, max_len, bs, part)),
+                     dtype=torch.uint8, device="cuda")
+    order = cache.bm.longest_first(ids)
+    assert (np.diff(lens[order]) <= 0).all()
+    bad = np.arange(n, dtype=np.int32)
+    bad[5] = -3
+    outs = []
+    for so in (None, order, order[::-1], bad):
+        out = torch.full((n, hkv * G, D), float("nan"), dtype=torch.float32, device="cuda")
+        B.pa_decode(q, cache.k_cache, cache.v_cache, t(tables), t(lens), D ** -0.5, out, max_len, part, ws,
+                    seq_order=None if so is None else t(so))
+        st, info = B.pa_get_device_error()
+        assert (st, info) == ((B.PA_ERR_DEVICE_BOUNDS, -3) if so is bad else (B.PA_OK, 0))
+        outs.append(out)
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    assert torch.isfinite(outs[0]).all()
