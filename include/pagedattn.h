@@ -376,7 +376,8 @@ pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t nu
  * chunk's inputs or outputs while the other computes. The
  * chains start after the work already queued on `stream`, and `stream` waits
  * for all of them, so the call's ordering against the caller's stream is that
- * of a single chain.
+ * of a single chain. Each chain's decode is pa_decode_ordered with its rows
+ * longest first (the order changes no result bit).
  */
 pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, const int64_t* seq_ids, int32_t num_q_heads,
                        const void* q_host, const void* k_host, const void* v_host, float scale, float* out_host,

@@ -5,7 +5,8 @@
 // block manager grows the tables (or copies a shared block, §3.4); the new K, V
 // are written at their slots; attention runs over every block of the table.
 // This file only orchestrates: block-manager calls on the host, one H2D copy of
-// all step metadata (slots, CoW pairs, tables, lengths) packed in pinned memory,
+// all step metadata (slots, CoW pairs, tables, lengths, each chunk's
+// longest-first dispatch order) packed in pinned memory,
 // the H2D copies of q/k/v, the three device operations, and the D2H copy of the
 // output.
 //
@@ -57,7 +58,7 @@ struct StepLayout {
   // device regions (byte offsets into dev_staging)
   size_t q, k, v, out, meta, ws, dev_total, ws_bytes;  // ws_bytes: one chunk's workspace
   // metadata (same layout on host and device, starting at `meta`)
-  size_t m_slots, m_pairs, m_tables, m_lens, meta_bytes;
+  size_t m_slots, m_pairs, m_tables, m_lens, m_order, meta_bytes;
 };
 
 bool make_layout(int32_t n, int32_t hq, const pa_cache* c, int32_t max_ctx, int32_t P, StepLayout& L) {
@@ -71,7 +72,8 @@ bool make_layout(int32_t n, int32_t hq, const pa_cache* c, int32_t max_ctx, int3
   L.m_pairs = up256(N * 8);
   L.m_tables = L.m_pairs + up256(N * 8);
   L.m_lens = L.m_tables + up256(N * L.cap * 4);
-  L.meta_bytes = L.m_lens + up256(N * 4);
+  L.m_order = L.m_lens + up256(N * 4);
+  L.meta_bytes = L.m_order + up256(N * 4);
   L.q = 0;
   L.k = up256(N * hq * c->head_dim * eb);
   L.v = L.k + up256(N * c->num_kv_heads * c->head_dim * eb);
@@ -174,6 +176,17 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
   st = pa_bm_block_tables(bm, n, seq_ids, reinterpret_cast<int32_t*>(h + L.m_tables), L.cap, -1,
                           reinterpret_cast<int32_t*>(h + L.m_lens));
   if (st != PA_OK) return st;
+  {
+    // each chunk's decode dispatches its rows longest first (indices within the chunk)
+    const int32_t* hl = reinterpret_cast<const int32_t*>(h + L.m_lens);
+    int32_t* ho = reinterpret_cast<int32_t*>(h + L.m_order);
+    const int32_t rows = chunk_rows(n, L.chunks);
+    for (int32_t r0 = 0; r0 < n; r0 += rows) {
+      const int32_t m = std::min(n, r0 + rows) - r0;
+      for (int32_t i = 0; i < m; ++i) ho[r0 + i] = i;
+      std::stable_sort(ho + r0, ho + r0 + m, [&](int32_t x, int32_t y) { return hl[r0 + x] > hl[r0 + y]; });
+    }
+  }
   const clock::time_point t_bm = clock::now();
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -186,6 +199,7 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
   const auto* slots = reinterpret_cast<const int64_t*>(meta + L.m_slots);
   const auto* tables = reinterpret_cast<const int32_t*>(meta + L.m_tables);
   const auto* lens = reinterpret_cast<const int32_t*>(meta + L.m_lens);
+  const auto* order = reinterpret_cast<const int32_t*>(meta + L.m_order);
   float* out_dev = reinterpret_cast<float*>(d + L.out);
 
   // One chain: inputs of rows [r0, r1), their append and decode, their output back.
@@ -200,9 +214,9 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
       return PA_ERR_CUDA;
     pa_status r = pa_reshape_and_cache(d + L.k + r0 * kv_row, d + L.v + r0 * kv_row, slots + r0, m, cache, cs);
     if (r != PA_OK) return r;
-    r = pa_decode(d + L.q + r0 * q_row, m, num_q_heads, cache, tables + static_cast<int64_t>(r0) * L.cap, L.cap,
-                  lens + r0, static_cast<int32_t>(max_len), scale, out_dev + r0 * (o_row / 4), partition_tokens,
-                  L.ws_bytes ? ws : nullptr, L.ws_bytes, cs);
+    r = pa_decode_ordered(d + L.q + r0 * q_row, m, num_q_heads, cache, tables + static_cast<int64_t>(r0) * L.cap,
+                          L.cap, lens + r0, static_cast<int32_t>(max_len), order + r0, scale,
+                          out_dev + r0 * (o_row / 4), partition_tokens, L.ws_bytes ? ws : nullptr, L.ws_bytes, cs);
     if (r != PA_OK) return r;
     if (cudaMemcpyAsync(reinterpret_cast<char*>(out_host) + r0 * o_row, reinterpret_cast<char*>(out_dev) + r0 * o_row,
                         m * o_row, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
