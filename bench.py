@@ -408,10 +408,14 @@ def check_device(B, what):
 # --- arms --------------------------------------------------------------------------
 
 def decode_fns(B, d, P, cascade=None):
+    """(pre, timed) of one decode step: the copy-on-write copies, then either
+    pa_decode_append (the KV append done by the decode CTAs, one launch) or,
+    for the cascade, pa_reshape_and_cache followed by pa_decode_cascade."""
     def write_step():
         if d["pairs"] is not None:
             B.pa_copy_blocks(d["kc"], d["vc"], d["pairs"])
-        B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
+        if cascade is not None:
+            B.pa_reshape_and_cache(d["k"], d["v"], d["slots"], d["kc"], d["vc"])
 
     sh = d["shape"]
     nseq = len(d["ids"])
@@ -424,8 +428,8 @@ def decode_fns(B, d, P, cascade=None):
             B.pa_decode_cascade(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"],
                                 *cascade)
             return
-        B.pa_decode(d["q"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"], d["out"], d["max_len"], P, ws,
-                    seq_order=d["order"])
+        B.pa_decode_append(d["q"], d["k"], d["v"], d["slots"], d["kc"], d["vc"], d["tables"], d["lens"], d["scale"],
+                           d["out"], d["max_len"], P, ws, seq_order=d["order"])
     return write_step, decode
 
 
@@ -494,11 +498,14 @@ def run_ours(args, rank, world, device):
     if cascade is not None:
         split = True
         n_groups = int(cascade[0].shape[0]) - 1
-        launches = args.steps * (1 + (1 if n_groups else 0) + 2 + (1 if d["pairs"] is not None else 0))
+        # append, prefix pass (when there are groups), suffix pass, merge kernel (split suffixes only)
+        launches = args.steps * (2 + (1 if n_groups else 0) + (1 if P_eff > 0 else 0) +
+                                 (1 if d["pairs"] is not None else 0))
     else:
-        # the merge kernel runs for 8 or more partitions; fewer are merged by the decode's last CTA
+        # one launch (the KV append is fused); the merge kernel runs for 8 or more partitions, fewer are merged
+        # by the decode's last CTA
         merge_kernel = split and math.ceil(d["max_len"] / P_eff) >= 8
-        launches = args.steps * (2 + (1 if merge_kernel else 0) + (1 if d["pairs"] is not None else 0))
+        launches = args.steps * (1 + (1 if merge_kernel else 0) + (1 if d["pairs"] is not None else 0))
     dtype_key = str(d["kc"].dtype).replace("torch.", "")
     traffic, traffic_src = ncu_traffic((args.workload, dtype_key, P_eff, "decode" if cascade is None else "cascade"))
     line = {
@@ -513,8 +520,9 @@ def run_ours(args, rank, world, device):
                    "kv_bytes_per_step": kv_bytes, "unique_kv_bytes_per_step": d["unique_kv_bytes"],
                    "partition_tokens": P_eff,
                    "kv_dtype": dtype_key,
-                   "decode": "pa_decode_cascade (shared prefixes read once per group)" if cascade is not None
-                   else "pa_decode_ordered (longest sequence first)",
+                   "decode": "pa_reshape_and_cache + pa_decode_cascade (shared prefixes read once per group)"
+                   if cascade is not None else "pa_decode_append (KV append fused into the decode, longest sequence "
+                                               "first)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "no flush: the K/V read per step is larger than the 126 MB L2"
                    if d["unique_kv_bytes"] > 3 * 126e6 else "no flush: K/V partly L2-resident (see unique bytes)"},
@@ -638,11 +646,10 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None,
 
     def one_pass(evs=None):
         for i, st in enumerate(steps):
-            B.pa_reshape_and_cache(io["k"], io["v"], st["slots"], kc, vc)
             if evs is not None:
                 evs[i][0].record(stream)
-            B.pa_decode(io["q"], kc, vc, st["tables"], st["lens"], scale, io["out"], st["max_len"], partition, ws,
-                        seq_order=st["order"])
+            B.pa_decode_append(io["q"], io["k"], io["v"], st["slots"], kc, vc, st["tables"], st["lens"], scale,
+                               io["out"], st["max_len"], partition, ws, seq_order=st["order"])
             if evs is not None:
                 evs[i][1].record(stream)
 
@@ -682,6 +689,10 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None,
            "partition_tokens": sorted({B.pa_decode_partition_tokens(st["n"], sh.num_q_heads, sh.num_kv_heads,
                                                                     st["max_len"], sh.block_size)
                                        if partition < 0 else partition for st in steps}),
+           "max_parts": max(math.ceil(st["max_len"] / pt) if pt > 0 else 1
+                            for st in steps for pt in [B.pa_decode_partition_tokens(
+                                st["n"], sh.num_q_heads, sh.num_kv_heads, st["max_len"], sh.block_size)
+                                if partition < 0 else partition]),
            "kv_dtype": str(kc.dtype).replace("torch.", "")}
     return rec, dec_ms, kv
 
@@ -713,8 +724,10 @@ def run_batching_line(args, rank, world, device):
                            f" (pool cut to {args.pool_blocks} blocks)" if args.pool_blocks else ""),
                        "passes": rec["passes"],
                        "l2": "no flush: ~0.8 GB of K/V per step against the 126 MB L2"},
-            "tokens_per_s": rec["tokens_per_s_step"], "gpu_launches": rec["steps"] * rec["passes"] * 3,
-            "roofline": {"kernel": "pa_decode (200-step average)", "bound": "hbm", "achieved": rec["gbs"],
+            "tokens_per_s": rec["tokens_per_s_step"],
+            "gpu_launches": rec["steps"] * rec["passes"] * (1 + (1 if max(parts) > 0 and rec["max_parts"] >= 8 else 0)),
+            "roofline": {"kernel": "pa_decode_append (200-step average; the KV append is fused)", "bound": "hbm",
+                         "achieved": rec["gbs"],
                          "peak": peak, "unit": "GB/s", "frac": rec["frac_of_measured_peak"], "traffic": traffic,
                          "traffic_source": traffic_src, "peak_source": kind},
             "batching": rec, "clocks": clk}), flush=True)

@@ -215,6 +215,36 @@ pa_status pa_decode_ordered(const void* q, int32_t num_seqs, int32_t num_q_heads
                             int32_t partition_tokens, void* workspace, size_t workspace_bytes, pa_stream stream);
 
 /*
+ * One decode step in one launch: the KV append (pa_reshape_and_cache of each
+ * sequence's new token, P2 §3.2.2 step 3) fused into pa_decode_ordered (step
+ * 4). The CTA (or persistent work item) that covers sequence s's last token
+ * first writes, for its kv head, the new K and V rows at slot_mapping[s] and
+ * only then starts the copies that read that block; no other CTA of the launch
+ * reads that position. Results and cache contents are those of
+ * pa_reshape_and_cache followed by pa_decode, bit for bit.
+ *   k_new, v_new   device [num_seqs][num_kv_heads][head_dim], 16-byte aligned:
+ *                  bf16 for a bf16 or 8-bit cache (quantised with the cache's
+ *                  k_scale / v_scale as pa_reshape_and_cache does), fp32 for
+ *                  an fp32 cache.
+ *   slot_mapping   device int64 [num_seqs], 8-byte aligned: the slot of each
+ *                  sequence's new token, which must be its position
+ *                  context_lens[s] - 1 in its block table (as
+ *                  pa_bm_append_slots returns it); -1 writes nothing. The
+ *                  target block must not be shared (run pa_copy_blocks for the
+ *                  step's copy-on-write pairs first, on the same stream). A
+ *                  slot outside the pool is recorded as PA_ERR_DEVICE_BOUNDS
+ *                  and not written.
+ * Other arguments, supported shapes and errors as pa_decode_ordered
+ * (seq_order may be NULL). Not for the cascade (pa_decode_cascade): append
+ * first there.
+ */
+pa_status pa_decode_append(const void* q, const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                           int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context_len,
+                           const int32_t* seq_order, float scale, float* out, int32_t partition_tokens,
+                           void* workspace, size_t workspace_bytes, pa_stream stream);
+
+/*
  * Causal attention of newly written prompt tokens (prefill, possibly in
  * chunks) over the paged cache. P2 §3.2.1: the prompt's K, V are computed and
  * written into the sequence's blocks (pa_reshape_and_cache first); each new
@@ -351,9 +381,10 @@ pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t nu
  * block manager assigns the new token's slot (new block or copy-on-write as
  * in pa_bm_append_slots); the CoW pairs, slots, block tables and lengths are
  * staged in pinned host memory and sent in one copy; q, k, v are copied from
- * the caller's host buffers; pa_copy_blocks, pa_reshape_and_cache and
- * pa_decode run on `stream`; the fp32 output is copied back to out_host; the
- * call returns after the stream has finished (so out_host is ready).
+ * the caller's host buffers; pa_copy_blocks and pa_decode_append (the KV
+ * append done by the decode CTAs) run on `stream`; the fp32 output is copied
+ * back to out_host; the call returns after the stream has finished (so
+ * out_host is ready).
  *
  *   bm, cache       the sequences' manager and cache (same block_size).
  *   seq_ids         host int64 [n]: sequences appending one token each.
@@ -376,7 +407,7 @@ pa_status pa_decode_static_workspace(const void* q, int32_t num_seqs, int32_t nu
  * chunk's inputs or outputs while the other computes. The
  * chains start after the work already queued on `stream`, and `stream` waits
  * for all of them, so the call's ordering against the caller's stream is that
- * of a single chain. Each chain's decode is pa_decode_ordered with its rows
+ * of a single chain. Each chain's pa_decode_append dispatches its rows
  * longest first (the order changes no result bit).
  */
 pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, const int64_t* seq_ids, int32_t num_q_heads,

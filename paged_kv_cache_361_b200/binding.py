@@ -52,6 +52,8 @@ _SIGS = {
     "pa_copy_blocks": (_I32, [_PCACHE, _VP, _I32, _VP]),
     "pa_decode": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _F, _VP, _I32, _VP, _SZ, _VP]),
     "pa_decode_ordered": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _VP, _F, _VP, _I32, _VP, _SZ, _VP]),
+    "pa_decode_append": (_I32, [_VP, _VP, _VP, _VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _VP, _F, _VP, _I32, _VP,
+                                _SZ, _VP]),
     "pa_decode_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
     "pa_decode_cascade": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32,
                                  _VP, _F, _VP, _VP, _SZ, _VP]),
@@ -215,6 +217,40 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, max_c
     _check(_lib().pa_decode(q.data_ptr(), B, hq, ctypes.byref(c), block_tables.data_ptr(),
                             int(block_tables.shape[1]), context_lens.data_ptr(), int(max_context_len), float(scale),
                             out.data_ptr(), int(partition_tokens), ws_ptr, ws_bytes, _stream(q, stream)), "pa_decode")
+
+
+def pa_decode_append(q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables, context_lens, scale, out,
+                     max_context_len, partition_tokens=-1, workspace=None, stream=None, seq_order=None):
+    """One decode step in one launch: the new K/V rows written at their slots
+    (as pa_reshape_and_cache) by the decode CTAs, then the decode
+    (pa_decode_ordered)."""
+    c = make_cache(k_cache, v_cache)
+    B, hq, d = q.shape
+    _dev(q, "q", input_dtype(k_cache.dtype), 3)
+    _dev(k_new, "k_new", input_dtype(k_cache.dtype), 3)
+    _dev(v_new, "v_new", input_dtype(k_cache.dtype), 3)
+    if tuple(k_new.shape) != (B, c.num_kv_heads, d) or tuple(v_new.shape) != (B, c.num_kv_heads, d):
+        raise ValueError("k_new / v_new must be [num_seqs][num_kv_heads][head_dim]")
+    _dev(slot_mapping, "slot_mapping", torch.int64, 1)
+    _dev(out, "out", torch.float32, 3)
+    if d != c.head_dim or tuple(out.shape) != (B, hq, d):
+        raise ValueError("q/out shape mismatch")
+    _dev(block_tables, "block_tables", torch.int32, 2)
+    _dev(context_lens, "context_lens", torch.int32, 1)
+    if block_tables.shape[0] != B or context_lens.shape[0] != B or slot_mapping.shape[0] != B:
+        raise ValueError("block_tables / context_lens / slot_mapping must have num_seqs rows")
+    if seq_order is not None:
+        _dev(seq_order, "seq_order", torch.int32, 1)
+        if seq_order.shape[0] != B:
+            raise ValueError("seq_order must have one entry per sequence")
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_dev(workspace, "workspace"),
+                                                            workspace.numel() * workspace.element_size())
+    _check(_lib().pa_decode_append(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), slot_mapping.data_ptr(), B, hq,
+                                   ctypes.byref(c), block_tables.data_ptr(), int(block_tables.shape[1]),
+                                   context_lens.data_ptr(), int(max_context_len),
+                                   seq_order.data_ptr() if seq_order is not None else None, float(scale),
+                                   out.data_ptr(), int(partition_tokens), ws_ptr, ws_bytes, _stream(q, stream)),
+           "pa_decode_append")
 
 
 def pa_prefill(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale, out, max_q_len, max_context_len,

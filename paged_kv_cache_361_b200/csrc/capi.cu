@@ -806,10 +806,13 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
 
 namespace {
 
+// k_new / v_new / slot_mapping non-null: the fused KV append of pa_decode_append.
 pa_status decode_impl(const void* q, int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache,
                       const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
                       int32_t max_context_len, const int32_t* seq_order, float scale, float* out,
-                      int32_t partition_tokens, void* workspace, size_t workspace_bytes, pa_stream stream) {
+                      int32_t partition_tokens, void* workspace, size_t workspace_bytes, pa_stream stream,
+                      const void* k_new = nullptr, const void* v_new = nullptr,
+                      const int64_t* slot_mapping = nullptr) {
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0) return PA_ERR_INVALID_ARG;
@@ -825,6 +828,9 @@ pa_status decode_impl(const void* q, int32_t num_seqs, int32_t num_q_heads, cons
   if (!q || !block_tables || !context_lens || !out || !aligned16(q) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3) ||
       (reinterpret_cast<uintptr_t>(seq_order) & 3))
+    return PA_ERR_INVALID_ARG;
+  if (slot_mapping && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new) ||
+                       (reinterpret_cast<uintptr_t>(slot_mapping) & 7)))
     return PA_ERR_INVALID_ARG;
   if (num_seqs > 65535) return PA_ERR_UNSUPPORTED;
 
@@ -864,6 +870,12 @@ pa_status decode_impl(const void* q, int32_t num_seqs, int32_t num_q_heads, cons
   a.parts_stride = parts;
   a.prefix_part_tokens = 0;
   a.seq_order = seq_order;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.slot_mapping = slot_mapping;
+  a.num_slots = static_cast<int64_t>(cache->num_blocks) * cache->block_size;
+  a.k_scale_store = cache->k_scale;
+  a.v_scale_store = cache->v_scale;
   if (is_8bit(cache->dtype)) {
     // q . (k_scale * code) = (k_scale * q) . code; the V scale multiplies o.
     a.scale_log2 *= cache->k_scale;
@@ -917,6 +929,17 @@ pa_status pa_decode_ordered(const void* q, int32_t num_seqs, int32_t num_q_heads
                             int32_t partition_tokens, void* workspace, size_t workspace_bytes, pa_stream stream) {
   return decode_impl(q, num_seqs, num_q_heads, cache, block_tables, max_blocks_per_seq, context_lens,
                      max_context_len, seq_order, scale, out, partition_tokens, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_append(const void* q, const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                           int32_t num_seqs, int32_t num_q_heads, const pa_cache* cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context_len,
+                           const int32_t* seq_order, float scale, float* out, int32_t partition_tokens,
+                           void* workspace, size_t workspace_bytes, pa_stream stream) {
+  if (!slot_mapping) return PA_ERR_INVALID_ARG;
+  return decode_impl(q, num_seqs, num_q_heads, cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, seq_order, scale, out, partition_tokens, workspace, workspace_bytes, stream,
+                     k_new, v_new, slot_mapping);
 }
 
 pa_status pa_selftest_wait_timeout(int64_t timeout_ns, pa_stream stream) {

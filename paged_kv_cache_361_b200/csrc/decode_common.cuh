@@ -9,6 +9,8 @@
 // (scores are kept in base 2: q is pre-scaled by scale * log2 e).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace pa {
@@ -56,6 +58,16 @@ struct DecodeArgs {
   // cascade prefix pass (it runs alongside that pass and waits for it before
   // folding in the prefix partials).
   int32_t after_prefix_pass = 0;
+  // Fused KV append (pa_decode_append): the CTA, or persistent item, that
+  // covers sequence s's last token first writes kv head g's new K and V rows
+  // (k_new / v_new [num_seqs][hkv][D], bf16 for an 8-bit cache, else the
+  // cache type) at slot_mapping[s] (-1: none), quantised with the cache's
+  // k_scale / v_scale for an 8-bit cache. Null otherwise.
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  const int64_t* slot_mapping = nullptr;
+  int64_t num_slots = 0;  // num_blocks * bs
+  float k_scale_store = 1.f, v_scale_store = 1.f;
 };
 
 // Sequence served by grid (or item) row y.
@@ -133,6 +145,7 @@ __device__ __forceinline__ int32_t load_len(const DecodeArgs& a, int32_t s, bool
 struct Part {
   int32_t t0, t1, ntok, nparts;
   int32_t npre;  // cascade: prefix partials of this sequence (slots max_parts ..)
+  bool last;     // covers the sequence's last token
 };
 
 template <int G, int D>
@@ -143,6 +156,7 @@ __device__ __forceinline__ bool cta_part(const DecodeArgs& a, int g, int s, int 
   const int32_t P = a.part_tokens > 0 ? a.part_tokens : (span > 0 ? span : 1);
   pt.t0 = st + p * P;
   pt.npre = 0;
+  pt.last = false;
   if (a.starts && st > 0) {
     pt.npre = (st + a.prefix_part_tokens - 1) / a.prefix_part_tokens;
     pt.npre = min(pt.npre, a.parts_stride - a.max_parts);  // never past the prefix slots
@@ -162,9 +176,109 @@ __device__ __forceinline__ bool cta_part(const DecodeArgs& a, int g, int s, int 
   if (pt.t0 >= L) return false;
   pt.t1 = min(pt.t0 + P, L);
   pt.ntok = pt.t1 - pt.t0;
+  pt.last = pt.t1 == L;
   pt.nparts = a.part_tokens > 0 ? (span + P - 1) / P : 1;
   return true;
 }
+
+// Fused KV append, by one warp (see DecodeArgs::k_new): load() reads kv head
+// g's new K and V rows of sequence s into registers (at most two 16-byte
+// pieces per lane at head_dim 128), write() stores them at the sequence's
+// slot, publish() makes the stores visible to the async proxy, so that the
+// bulk / tensor copies issued next (after a __syncwarp) read the new row.
+// The producer loads at its start, writes once its first chunk's copies are
+// issued, and publishes just before it issues the chunk that holds the slot
+// (the CTA's last): the load and the store are then long complete and
+// nothing waits for them. step() does that for chunk i of n.
+template <typename T, int D>
+struct AppendRow {
+  static constexpr bool kCoded = Elem<T>::bytes == 1;
+  // 16-byte pieces of the two cache rows (K then V); an 8-bit piece takes two
+  // bf16 input pieces
+  static constexpr int kPieces = kCoded ? 2 * (D / 16) : 2 * (D * Elem<T>::bytes / 16);
+  static constexpr int kPerLane = (kPieces + 31) / 32;
+  uint4 x[kPerLane][kCoded ? 2 : 1];
+  int64_t row;  // cache row of the slot; -1: nothing to write
+
+  __device__ __forceinline__ void load(const DecodeArgs& a, int s, int g, int lane) {
+    const int64_t slot = __ldg(a.slot_mapping + s);
+    row = -1;
+    if (slot == -1) return;
+    if (slot < 0 || slot >= a.num_slots) {
+      if (lane == 0) record_error(PA_ERR_DEVICE_BOUNDS, slot);
+      return;
+    }
+    const int64_t blk = slot / a.bs;
+    row = (blk * a.hkv + g) * a.bs + (slot - blk * a.bs);
+    const int64_t src_row = static_cast<int64_t>(s) * a.hkv + g;
+    constexpr int CH = kPieces / 2;
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) {
+      const int i = lane + 32 * u;
+      if (i < kPieces) {
+        const int which = i / CH, c = i - which * CH;
+        const uint4* src = static_cast<const uint4*>(which ? a.v_new : a.k_new);
+        if constexpr (kCoded) {
+          x[u][0] = __ldg(src + (src_row * CH + c) * 2);
+          x[u][1] = __ldg(src + (src_row * CH + c) * 2 + 1);
+        } else {
+          x[u][0] = __ldg(src + src_row * CH + c);
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void write(const DecodeArgs& a, int lane) {
+    if (row < 0) return;
+    // the cache pools are the caller's writable device memory (held const here for the readers)
+    uint4* kc = static_cast<uint4*>(const_cast<void*>(a.kc));
+    uint4* vc = static_cast<uint4*>(const_cast<void*>(a.vc));
+    constexpr int CH = kPieces / 2;
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) {
+      const int i = lane + 32 * u;
+      if (i < kPieces) {
+        const int which = i / CH, c = i - which * CH;
+        uint4 v = x[u][0];
+        if constexpr (kCoded) {
+          const float sc = which ? a.v_scale_store : a.k_scale_store;
+          const uint32_t w[8] = {x[u][0].x, x[u][0].y, x[u][0].z, x[u][0].w,
+                                 x[u][1].x, x[u][1].y, x[u][1].z, x[u][1].w};
+          uint32_t q[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float f[4] = {bf16lo(w[2 * e2]), bf16hi(w[2 * e2]), bf16lo(w[2 * e2 + 1]), bf16hi(w[2 * e2 + 1])};
+            uint32_t b[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if constexpr (std::is_same<T, int8_t>::value)
+                b[e] = static_cast<uint8_t>(quantize_s8(f[e], sc));
+              else
+                b[e] = quantize_e4m3(f[e], sc);
+            }
+            q[e2] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+          }
+          v = make_uint4(q[0], q[1], q[2], q[3]);
+        }
+        (which ? vc : kc)[row * CH + c] = v;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void publish() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+  // Before chunk i's copies (of n): the row goes out before the last chunk.
+  __device__ __forceinline__ void before_chunk(const DecodeArgs& a, int i, int n, int lane) {
+    if (i != n - 1) return;
+    if (n == 1) write(a, lane);
+    publish();
+    __syncwarp();
+  }
+  // After chunk i's copies: the write, once the first chunk is on its way.
+  __device__ __forceinline__ void after_chunk(const DecodeArgs& a, int i, int n, int lane) {
+    if (i == 0 && n > 1) write(a, lane);
+  }
+};
 
 // Work item -> (kv head g, sequence s, partition p), partition-major so that
 // partition 0 of every sequence comes first.

@@ -413,12 +413,19 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
   float m_run = -INFINITY, l_run = 0.f;
 
   if (warp == NW) {
+    // fused KV append: the new row is loaded now and stored before the last
+    // chunk's copies, which read it
+    using Code = typename std::conditional<CF == kCodeS8, int8_t, __nv_fp8_e4m3>::type;
+    const bool do_append = a.slot_mapping && pt.last;
+    AppendRow<Code, D> ar;
+    if (do_append) ar.load(a, s, g, lane);
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
     const uint64_t pol = kv_stream_policy();
     TableAhead ta;
     ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+      if (do_append) ar.before_chunk(a, i, nchunks, lane);
       const int32_t c0 = pt.t0 + i * C;
       const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
       const int32_t blk = ta.get(c0 / a.bs, nb, lane);
@@ -436,6 +443,7 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
         tma_load_2d(kdst, &tmk, 0, y, &ps.full[st], pol);
         tma_load_2d(kdst + Cfg::kTileBytes, &tmv, 0, y, &ps.full[st], pol);
       }
+      if (do_append) ar.after_chunk(a, i, nchunks, lane);
     });
   } else {
     // q rows as f16 A fragments in the dim order of f8_chunk's k-steps:

@@ -408,6 +408,11 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
       } else if (t0 < L) {
         const int32_t t1 = min(t0 + P, L);
         const int nch = (t1 - t0 + C - 1) / C;
+        // fused KV append: the new row is loaded now and stored before the
+        // item's last chunk's copies, which read it
+        const bool do_append = a.slot_mapping && t1 == L;
+        AppendRow<__nv_bfloat16, D> ar;
+        if (do_append) ar.load(a, s, g, lane);
         const int nparts = a.part_tokens > 0 ? (span + P - 1) / P : 1;
         const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
         // block ids of chunk ch (lane < its block count), loaded one chunk
@@ -426,6 +431,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
             aborted = true;
             break;
           }
+          if (do_append) ar.before_chunk(a, ch, nch, lane);
           const int32_t c0 = t0 + ch * C;
           const int32_t n = min(C, t1 - c0);
           const int32_t nb = (n + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
@@ -456,6 +462,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
             tma_block<D>(kdst, &tmk, y, &ps.full[st], pol);
             tma_block<D>(kdst + Cfg::kTileBytes, &tmv, y, &ps.full[st], pol);
           }
+          if (do_append) ar.after_chunk(a, ch, nch, lane);
         }
       }
       item = static_cast<int>(gridDim.x + __shfl_sync(0xffffffffu, nxt, 0));
@@ -594,12 +601,18 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
   float m_run = -INFINITY, l_run = 0.f;
 
   if (warp == NW) {
+    // fused KV append: the new row is loaded now and stored before the last
+    // chunk's copies, which read it
+    const bool do_append = a.slot_mapping && pt.last;
+    AppendRow<__nv_bfloat16, D> ar;
+    if (do_append) ar.load(a, s, g, lane);
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D * 2u;  // one (block, head) tile of K or V
     const uint64_t pol = kv_stream_policy();
     TableAhead ta;
     ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+      if (do_append) ar.before_chunk(a, i, nchunks, lane);
       const int32_t c0 = pt.t0 + i * C;
       const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 8 (bs >= 8)
       const int32_t blk = ta.get(c0 / a.bs, nb, lane);
@@ -617,6 +630,7 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
         tma_block<D>(kdst, &tmk, y, &ps.full[st], pol);
         tma_block<D>(kdst + Cfg::kTileBytes, &tmv, y, &ps.full[st], pol);
       }
+      if (do_append) ar.after_chunk(a, i, nchunks, lane);
     });
   } else {
     uint32_t qa[D / 16][2];

@@ -177,12 +177,18 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
 
   if (warp == NW) {
     // ---- producer ----
+    // fused KV append: the new row is loaded now and stored before the last
+    // chunk's copies, which read it
+    const bool do_append = a.slot_mapping && pt.last;
+    AppendRow<T, D> ar;
+    if (do_append) ar.load(a, s, g, lane);
     const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t tile_bytes = static_cast<uint32_t>(a.bs) * D * Elem<T>::bytes;
     const T* kc = static_cast<const T*>(a.kc);
     const T* vc = static_cast<const T*>(a.vc);
     const uint64_t pol = kv_stream_policy();
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
+      if (do_append) ar.before_chunk(a, i, nchunks, lane);
       const int32_t c0 = pt.t0 + i * C;
       const int32_t nb = (min(C, pt.t1 - c0) + a.bs - 1) / a.bs;  // <= 64 (C = 64, bs >= 1)
       int32_t blk[2] = {-1, -1};
@@ -208,6 +214,7 @@ __global__ void __launch_bounds__(SimtCfg<T, D>::kThreads) decode_simt_kernel(co
           bulk_g2s(sV + (st * C + row) * D, vc + off, tile_bytes, &ps.full[st], pol);
         }
       }
+      if (do_append) ar.after_chunk(a, i, nchunks, lane);
     });
   } else {
     // ---- consumers ----

@@ -7,7 +7,8 @@
 // This file only orchestrates: block-manager calls on the host, one H2D copy of
 // all step metadata (slots, CoW pairs, tables, lengths, each chunk's
 // longest-first dispatch order) packed in pinned memory,
-// the H2D copies of q/k/v, the three device operations, and the D2H copy of the
+// the H2D copies of q/k/v, the device operations (copy-on-write copies, then the
+// decode with the KV append fused, pa_decode_append), and the D2H copy of the
 // output.
 //
 // A batch of at least kMinChunkRows sequences is cut into row chunks, each on
@@ -212,11 +213,11 @@ extern "C" pa_status pa_step_host(pa_bm* bm, const pa_cache* cache, int32_t n, c
         cudaMemcpyAsync(d + L.v + r0 * kv_row, static_cast<const char*>(v_host) + r0 * kv_row, m * kv_row,
                         cudaMemcpyHostToDevice, cs) != cudaSuccess)
       return PA_ERR_CUDA;
-    pa_status r = pa_reshape_and_cache(d + L.k + r0 * kv_row, d + L.v + r0 * kv_row, slots + r0, m, cache, cs);
-    if (r != PA_OK) return r;
-    r = pa_decode_ordered(d + L.q + r0 * q_row, m, num_q_heads, cache, tables + static_cast<int64_t>(r0) * L.cap,
-                          L.cap, lens + r0, static_cast<int32_t>(max_len), order + r0, scale,
-                          out_dev + r0 * (o_row / 4), partition_tokens, L.ws_bytes ? ws : nullptr, L.ws_bytes, cs);
+    // the KV append is done by the decode CTAs (one launch per chain)
+    pa_status r = pa_decode_append(d + L.q + r0 * q_row, d + L.k + r0 * kv_row, d + L.v + r0 * kv_row, slots + r0, m,
+                                   num_q_heads, cache, tables + static_cast<int64_t>(r0) * L.cap, L.cap, lens + r0,
+                                   static_cast<int32_t>(max_len), order + r0, scale, out_dev + r0 * (o_row / 4),
+                                   partition_tokens, L.ws_bytes ? ws : nullptr, L.ws_bytes, cs);
     if (r != PA_OK) return r;
     if (cudaMemcpyAsync(reinterpret_cast<char*>(out_host) + r0 * o_row, reinterpret_cast<char*>(out_dev) + r0 * o_row,
                         m * o_row, cudaMemcpyDeviceToHost, cs) != cudaSuccess)

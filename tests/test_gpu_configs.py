@@ -367,3 +367,78 @@ def test_decode_ordered_matches_decode(dtype, G, part):
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
     assert torch.isfinite(outs[0]).all()
+
+
+@pytest.mark.parametrize("dtype,G,part,bs", [("bf16", 1, 0, 16), ("bf16", 4, 0, 16), ("bf16", 4, 128, 16),
+                                              ("bf16", 8, 256, 32), ("bf16", 2, 64, 8), ("e4m3", 1, 0, 16),
+                                              ("e4m3", 4, 128, 16), ("int8", 8, 0, 16), ("int8", 2, 0, 4),
+                                              ("fp32", 1, 0, 16), ("fp32", 4, 96, 16)])
+def test_decode_append_matches_append_then_decode(dtype, G, part, bs):
+    """pa_decode_append (the KV append done by the decode CTAs) leaves the same
+    pool bytes and the same outputs, bit for bit, as pa_reshape_and_cache then
+    pa_decode, on every kernel family; slot -1 writes nothing; a slot outside
+    the pool is recorded and not written."""
+    from paged_kv_cache_361_b200 import PagedKVCache
+    rng = np.random.default_rng(G * 11 + part + bs)
+    hkv, D = 2, 128
+    tdt = {"bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn, "int8": torch.int8, "fp32": torch.float32}[dtype]
+    idt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    sc = 4.0 / 127 if dtype == "int8" else 1.0
+    nb = 4000 * 16 // bs
+    cache = PagedKVCache(nb, hkv, bs, D, tdt, "cuda", rng.permutation(nb), fill=0.0, k_scale=sc, v_scale=sc)
+    g = torch.Generator().manual_seed(G + part + bs)
+    ids = list(range(19))
+    for s in ids:
+        n = int(rng.integers(0, 700))
+        cache.add_sequence(s, torch.randn(n, hkv, D, generator=g).to(idt).cuda(),
+                           torch.randn(n, hkv, D, generator=g).to(idt).cuda())
+    slots, pairs = cache.bm.append_slots(ids)
+    assert len(pairs) == 0
+    for s in ids:
+        cache.lens[s] += 1
+    n = len(ids)
+    tables, lens, max_len = cache.decode_inputs(ids)
+    q = torch.randn(n, hkv * G, D, generator=g).to(idt).cuda()
+    kn = torch.randn(n, hkv, D, generator=g).to(idt).cuda()
+    vn = torch.randn(n, hkv, D, generator=g).to(idt).cuda()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+    ws = torch.empty(max(256, B.pa_decode_workspace_bytes(n, hkv * G, hkv, D, max_len, bs, part)),
+                     dtype=torch.uint8, device="cuda")
+    order = t(cache.bm.longest_first(ids))
+    pools = (cache.k_cache.clone(), cache.v_cache.clone())
+    sl = torch.from_numpy(slots).cuda()
+
+    def run(fused, slot_t):
+        kc, vc = pools[0].clone(), pools[1].clone()
+        if dtype in ("e4m3", "int8"):
+            B.set_kv_scales(kc, vc, sc, sc)
+        out = torch.full((n, hkv * G, D), float("nan"), dtype=torch.float32, device="cuda")
+        if fused:
+            B.pa_decode_append(q, kn, vn, slot_t, kc, vc, t(tables), t(lens), D ** -0.5, out, max_len, part, ws,
+                               seq_order=order)
+        else:
+            B.pa_reshape_and_cache(kn, vn, slot_t, kc, vc)
+            B.pa_decode(q, kc, vc, t(tables), t(lens), D ** -0.5, out, max_len, part, ws, seq_order=order)
+        return out, kc, vc
+
+    ref = run(False, sl)
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    got = run(True, sl)
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    assert torch.equal(got[0], ref[0])
+    for a_, b_ in zip(got[1:], ref[1:]):
+        assert torch.equal(a_.view(torch.uint8), b_.view(torch.uint8))
+    # slot -1 for sequence 3 writes nothing there (its row keeps the old bytes), others as before
+    sl2 = sl.clone()
+    sl2[3] = -1
+    ref2 = run(False, sl2)
+    got2 = run(True, sl2)
+    assert torch.equal(got2[0], ref2[0]) and torch.equal(got2[1].view(torch.uint8), ref2[1].view(torch.uint8))
+    assert B.pa_get_device_error()[0] == B.PA_OK
+    # a slot outside the pool: recorded, nothing written for it
+    sl3 = sl2.clone()
+    sl3[3] = nb * bs + 5
+    got3 = run(True, sl3)
+    st, info = B.pa_get_device_error()
+    assert st == B.PA_ERR_DEVICE_BOUNDS and info == nb * bs + 5
+    assert torch.equal(got3[1].view(torch.uint8), ref2[1].view(torch.uint8))
