@@ -442,8 +442,9 @@ def run_ours(args, rank, world, device):
     nseq = len(d["ids"])
     cascade = cascade_inputs(d, device) if args.cascade else None
     P = args.partition if args.partition != -2 else d["part"]
-    P_eff = P if P >= 0 else B.pa_decode_partition_tokens(nseq, sh.num_q_heads, sh.num_kv_heads, d["max_len"],
-                                                          sh.block_size)
+    # the cascade resolves -1 as pa_decode does; the ordered decode as pa_decode_ordered does
+    P_eff = P if P >= 0 else (B.pa_decode_partition_tokens if args.cascade else B.pa_decode_ordered_partition_tokens)(
+        nseq, sh.num_q_heads, sh.num_kv_heads, d["max_len"], sh.block_size)
     split = P_eff > 0 and math.ceil(d["max_len"] / P_eff) > 1
     stream = torch.cuda.current_stream(device)
 
@@ -566,8 +567,9 @@ def decode_record(B, d, P, steps, warmup, device, cascade=None):
     gbs = d["kv_bytes"] / (ms * 1e-3) / 1e9
     nseq = len(d["ids"])
     sh = d["shape"]
-    P_eff = P if P >= 0 else B.pa_decode_partition_tokens(nseq, sh.num_q_heads, sh.num_kv_heads, d["max_len"],
-                                                          sh.block_size)
+    P_eff = P if P >= 0 else (B.pa_decode_partition_tokens if cascade is not None
+                              else B.pa_decode_ordered_partition_tokens)(nseq, sh.num_q_heads, sh.num_kv_heads,
+                                                                         d["max_len"], sh.block_size)
     dtype_key = str(d["kc"].dtype).replace("torch.", "")
     traffic, src = ncu_traffic((d["name"], dtype_key, P_eff, "decode" if cascade is None else "cascade"))
     rec = {"decode_ms": round(ms, 5), "step_ms": round(total / steps, 5), "kv_bytes": d["kv_bytes"],
@@ -686,11 +688,11 @@ def batching_record(B, device, reps=2, kv_dtype="auto", seed=0, num_blocks=None,
            "host_note": "C++ block manager through the ctypes binding per step: frees, arrival reservations, one "
                         "slot per live sequence, block tables, longest-first dispatch order; timed on the host, "
                         "outside the device time",
-           "partition_tokens": sorted({B.pa_decode_partition_tokens(st["n"], sh.num_q_heads, sh.num_kv_heads,
+           "partition_tokens": sorted({B.pa_decode_ordered_partition_tokens(st["n"], sh.num_q_heads, sh.num_kv_heads,
                                                                     st["max_len"], sh.block_size)
                                        if partition < 0 else partition for st in steps}),
            "max_parts": max(math.ceil(st["max_len"] / pt) if pt > 0 else 1
-                            for st in steps for pt in [B.pa_decode_partition_tokens(
+                            for st in steps for pt in [B.pa_decode_ordered_partition_tokens(
                                 st["n"], sh.num_q_heads, sh.num_kv_heads, st["max_len"], sh.block_size)
                                 if partition < 0 else partition]),
            "kv_dtype": str(kc.dtype).replace("torch.", "")}

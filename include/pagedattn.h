@@ -330,6 +330,13 @@ size_t pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, 
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t max_context_len, int32_t block_size);
 
+/* The same for pa_decode_ordered / pa_decode_append with a seq_order (the
+ * CTAs dispatched longest first balance the waves, so fewer splits pay):
+ * never more partitions than pa_decode_partition_tokens gives, so
+ * pa_decode_workspace_bytes(..., -1) covers it. */
+int32_t pa_decode_ordered_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                           int32_t max_context_len, int32_t block_size);
+
 /* Workspace bytes pa_decode needs for these sizes (a few hundred bytes of
  * counters, plus the partials when sequences are split). partition_tokens may
  * be -1 (resolved as pa_decode would). */

@@ -55,6 +55,7 @@ _SIGS = {
     "pa_decode_append": (_I32, [_VP, _VP, _VP, _VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _VP, _F, _VP, _I32, _VP,
                                 _SZ, _VP]),
     "pa_decode_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
+    "pa_decode_ordered_partition_tokens": (_I32, [_I32, _I32, _I32, _I32, _I32]),
     "pa_decode_cascade": (_I32, [_VP, _I32, _I32, _PCACHE, _VP, _I32, _VP, _I32, _I32, _VP, _VP, _VP, _VP, _I32, _I32,
                                  _VP, _F, _VP, _VP, _SZ, _VP]),
     "pa_decode_cascade_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
@@ -181,6 +182,12 @@ def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None):
 
 def pa_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, max_context_len, block_size) -> int:
     return int(_lib().pa_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, max_context_len, block_size))
+
+
+def pa_decode_ordered_partition_tokens(num_seqs, num_q_heads, num_kv_heads, max_context_len, block_size) -> int:
+    """The partition size pa_decode_ordered / pa_decode_append choose for -1 when given a seq_order."""
+    return int(_lib().pa_decode_ordered_partition_tokens(num_seqs, num_q_heads, num_kv_heads, max_context_len,
+                                                         block_size))
 
 
 def pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size,

@@ -123,6 +123,15 @@ def test_workspace_sizes():
         cnt(4, 8) + (rows * 8 + 255) // 256 * 256 + rows * 128 * 4
     P = B.pa_decode_partition_tokens(64, 32, 32, 2049, 16)
     assert P == 0 or P % 16 == 0
+    # with a dispatch order: never more partitions than without, and no split for many moderate units
+    for args in ((256, 32, 8, 4097, 16), (4, 64, 8, 131073, 32), (64, 32, 8, 1513, 16), (64, 32, 32, 2049, 16),
+                 (300, 8, 8, 9000, 16), (16, 8, 8, 5000, 8)):
+        po, pu = B.pa_decode_ordered_partition_tokens(*args), B.pa_decode_partition_tokens(*args)
+        parts = lambda p: 1 if p == 0 else -(-args[3] // p)
+        assert parts(po) <= parts(pu)
+    assert B.pa_decode_ordered_partition_tokens(256, 32, 8, 4097, 16) == 0
+    assert B.pa_decode_partition_tokens(256, 32, 8, 4097, 16) == 1024
+    assert B.pa_decode_ordered_partition_tokens(4, 64, 8, 131073, 32) > 0
 
 
 def test_step_timing_and_copy_swap_host_checks():
