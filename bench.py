@@ -50,34 +50,33 @@ _PF = ["common.cuh", "decode_common.cuh", "decode_f8.cuh", "prefill_mma.cuh", "p
        "capi.cu"]
 NCU_TRAFFIC: dict = {
     ("llama2_7b_mha", "bfloat16", 0, "decode"): dict(
-        bytes=1_079_339_776 + 998_229, files=_DEC + ["decode_simt.cuh"], sha="e143330f49c54f75",
-        note="decode_simt_kernel, 3 launches"),
+        bytes=1_079_315_883 + 2_277_120, files=_DEC + ["decode_simt.cuh"], sha="9489fe02f3c535bb",
+        note="decode_simt_kernel of pa_decode_append (the step's only launch), 3 launches"),
     ("llama2_7b_mha", "float8_e4m3fn", 0, "decode"): dict(
-        bytes=539_992_832 + 7_646_549, files=_DEC + ["decode_f8.cuh"], sha="ce2482e42c316dce",
-        note="decode_f8_kernel (e4m3), 3 launches"),
+        bytes=540_494_763 + 8_050_091, files=_DEC + ["decode_f8.cuh"], sha="0821c9cb1e81d0ca",
+        note="decode_f8_kernel (e4m3) of pa_decode_append, 3 launches"),
     ("llama2_7b_mha", "int8", 0, "decode"): dict(
-        bytes=539_992_320 + 8_051_712, files=_DEC + ["decode_f8.cuh"], sha="ce2482e42c316dce",
-        note="decode_f8_kernel (int8), 3 launches"),
+        bytes=540_492_373 + 8_290_987, files=_DEC + ["decode_f8.cuh"], sha="0821c9cb1e81d0ca",
+        note="decode_f8_kernel (int8) of pa_decode_append, 3 launches"),
     ("long_context_split", "bfloat16", 512, "decode"): dict(
-        bytes=1_342_939_584 + 5_665_664 + 21_471_680, files=_DEC + ["decode_mma.cuh"], sha="86b797581e62b7d5",
-        note="decode_mma_persistent_kernel + decode_reduce_kernel, 4 launches each"),
+        bytes=1_343_023_275 + 6_138_112 + 21_472_341, files=_DEC + ["decode_mma.cuh"], sha="a8e832b3f88ba6d7",
+        note="decode_mma_persistent_kernel + decode_reduce_kernel, 3 launches each"),
     ("parallel_sampling", "bfloat16", 0, "decode"): dict(
-        bytes=100_495_659 + 169_216, files=_DEC + ["decode_mma.cuh"], sha="86b797581e62b7d5",
-        note="decode_mma_kernel, 6 launches"),
+        bytes=121_091_200 + 469_760, files=_DEC + ["decode_mma.cuh"], sha="a8e832b3f88ba6d7",
+        note="decode_mma_kernel of pa_decode_append, 6 launches (1.25x the 97.5 MB of distinct blocks: with the "
+             "longest-first order a prompt's samples no longer all run at once)"),
     ("parallel_sampling", "bfloat16", 0, "cascade"): dict(
-        bytes=32_021_632 + 72_819_814 + 42_342, files=_DEC + ["decode_mma.cuh", "prefill_mma.cuh"],
-        sha="a8338145e53106fe", note="prefill_mma_kernel (prefix pass) + decode_mma_kernel (suffix, merge), "
-                                     "5-6 launches each"),
-    ("continuous_batching", "bfloat16", 1024, "decode"): dict(
-        bytes=835_727_761 + 4_076_467, files=_DEC + ["decode_mma.cuh"], sha="86b797581e62b7d5",
-        note="decode_mma_persistent_kernel over steps 0-29 of the trace (32768-block pool); their algorithmic mean "
-             "is 825.0 MB per step (x1.018), the 200-step mean 811.2 MB"),
+        bytes=32_023_552 + 5_205 + 72_904_397 + 77_824, files=_DEC + ["decode_mma.cuh", "prefill_mma.cuh"], sha="3220a31f59111fd6",
+        note="prefill_mma_kernel (prefix pass) + decode_mma_kernel (suffixes and fold), 5-6 launches each"),
+    ("continuous_batching", "bfloat16", 0, "decode"): dict(
+        bytes=835_075_447 + 2_500_437, files=_DEC + ["decode_mma.cuh"], sha="a8e832b3f88ba6d7",
+        note="decode_mma_kernel of pa_decode_append over steps 0-29 of the trace (32768-block pool); their "
+             "algorithmic mean is 825.0 MB per step (x1.015), the 200-step mean 811.2 MB"),
     ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
-        bytes=1_309_394_000 + 233_774_080, files=_PF, sha="b9e7a2b9692c8b03", note="prefill_tc_kernel, 1 launch",
-        how="ncu capture (metric set, small case = this workload)"),
+        bytes=1_309_527_296 + 230_245_449, files=_PF, sha="d85c79484f101e28",
+        note="prefill_tc_kernel, 7 launches (Q, K/V per tile pair not served by L2, the fp32 output)"),
     ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
-        bytes=729_495_040 + 493_113_344, files=_PF, sha="b9e7a2b9692c8b03", note="prefill_tc_kernel, 1 launch",
-        how="ncu capture (metric set, small case = this workload)"),
+        bytes=760_672_549 + 489_605_010, files=_PF, sha="d85c79484f101e28", note="prefill_tc_kernel, 7 launches"),
 }
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
