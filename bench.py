@@ -945,7 +945,7 @@ def run_e2e(args, d, device, world, P):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "breakdown": breakdown,
             "api": "pa_step_host via PagedKVCache.step_plan (block manager, one metadata H2D, q/k/v H2D, "
-                   "pa_copy_blocks, pa_reshape_and_cache, pa_decode, output D2H, stream sync)"}
+                   "pa_copy_blocks, pa_decode_append (append fused, longest first), output D2H, stream sync)"}
 
 
 PREFILL = {
