@@ -164,7 +164,7 @@ __device__ __forceinline__ void widen_row_half(const uint8_t* src, uint8_t* dst,
 }
 
 // m16n8k16 f16 MMA with rows 8..15 of A zero and their results discarded
-// (as mma_rows8).
+// (their registers are never held).
 __device__ __forceinline__ void mma_f16_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   float j2, j3;
   asm volatile(

@@ -10,17 +10,19 @@
 // When G = Hq / Hkv query heads share a kv head, each K/V byte feeds 2G
 // multiply-adds; on the CUDA cores that (plus the bf16 unpacking and the
 // cross-lane reductions) outruns the instruction issue rate before HBM is
-// saturated. Here the two contractions run as m16n8k16 bf16 MMAs with the G
-// heads as the M rows (rows G..15 are zero):
-//   S = Q K^T : A = Q (registers, loaded once), B = K tile via ldmatrix;
-//   O += P V  : A = P (the S accumulator re-packed in registers, split into a
-//               bf16 high part and a bf16 remainder so that P keeps ~16
-//               mantissa bits), B = V tile via ldmatrix.trans.
-// K/V tiles arrive by TMA tensor copies (cp.async.bulk.tensor.2d) of
-// [block_size rows x 64 dims] boxes with the 128-byte swizzle, so the 8-row
-// ldmatrix reads hit 8 different bank groups. Tokens past the context length
-// get -inf scores and their V rows are zeroed in registers, so padding (even
-// NaN) never reaches the result.
+// saturated. Here the two contractions run as m16n8k16 bf16 MMAs with a
+// warp's 16 tokens (or 16 dims) as the M rows and the G heads as the N columns
+// (columns G..7 are zero), so no MMA row is padding:
+//   S^T = K Q^T  : A = K tile via ldmatrix, B = Q (registers, loaded once);
+//   O^T += V^T P^T: A = V tile via ldmatrix.trans, B = P (the S^T accumulator
+//                   transposed in registers by movmatrix, split into a bf16
+//                   high part and a bf16 remainder so that P keeps ~16
+//                   mantissa bits).
+// K/V tiles arrive by TMA tensor copies, one cp.async.bulk.tensor.3d per
+// (block, head) tile landing as [half][block_size rows][128 B] with the
+// 128-byte swizzle, so the 8-row ldmatrix reads hit 8 different bank groups.
+// Tokens past the context length get -inf scores and their V rows are zeroed
+// in registers, so padding (even NaN) never reaches the result.
 // Persistent CTAs (as many as fit on the GPU) take work items (kv head,
 // sequence, partition) from an atomic counter. Warp 4 is the TMA producer: it
 // walks item after item without draining the stage ring, writing a small
@@ -83,39 +85,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
-// d += A(16x16, rows 8..15 zero) * B(16x8), bf16 in, fp32 accumulate. Only
-// rows 0..7 of the accumulator are kept: rows 8..15 are fed zeros and their
-// results are discarded, so they hold no registers across the loop.
-// m16n8k16 bf16 MMA with rows 8..15 of A zero: their accumulator lanes get
-// fresh zero inputs and are discarded, so no registers are held for them and
-// the MMAs on different accumulators stay independent.
-__device__ __forceinline__ void mma_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  float j2, j3;
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%10, %11, %12, %12};"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(j2), "=f"(j3)
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f));
-  asm volatile("" ::"f"(j2), "f"(j3));  // rows 8..15: discarded
-}
-
-// The same MMA for a dependent chain (one accumulator over the k-steps): rows
-// 8..15 accumulate into the chain's own `dead` pair (never read), which
-// saves materialising zero inputs per MMA without adding dependences.
-__device__ __forceinline__ void mma_rows8_chain(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1,
-                                                float (&dead)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(dead[0]), "+f"(dead[1])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // p -> (bf16(p), bf16(p - bf16(p))) for a pair.
 __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint32_t& lo) {
   __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
@@ -128,12 +97,6 @@ __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint3
 // Build-time tuning knobs of the one-CTA-per-item kernel (defaults measured
 // on B200): ring stages at head_dim 128 (0 = the default of 3), and the CTAs
 // per SM its register budget is fitted to.
-// Build-time knob: k-steps (and P V steps) whose shared-memory fragments are
-// loaded ahead of the MMAs in mma_chunk.
-#ifndef PA_MMA_PREFETCH
-#define PA_MMA_PREFETCH 4
-#endif
-
 #ifndef PA_MMA_STAGES
 #define PA_MMA_STAGES 0
 #endif
@@ -159,39 +122,56 @@ struct MmaCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = kStageBytes <= 16384 ? 4 : (PA_MMA_STAGES > 0 ? PA_MMA_STAGES : 3);
   static constexpr int kQBytes = 8 * D * 2;                // query rows of one item (G <= 8)
-  static constexpr int kNT = D / 8;
-  static constexpr int kFoldFloats = 32 * (2 * kNT + 2);   // one warp's fragments + (m, l) per lane
+  static constexpr int kFoldFloats = 32 * (D / 4 + 4);     // one warp's O fragments + (m, l) of 2 heads per lane
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;  // one CTA per item
   static constexpr int kPersistSmemBytes = kSmemBytes + kStages * kQBytes + 2 * kFoldFloats * 4;
 };
 
 
+// m16n8k16 bf16 MMA, fp32 accumulate in place (all four A registers).
+__device__ __forceinline__ void mma16x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose of an 8x8 matrix of 16-bit pairs held as MMA fragments: the lane
+// holding (row i, columns 2j, 2j+1) receives (row j', ...) of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // One consumer warp's share of a stage: its 16 tokens (nv of them valid) of
-// the K tile at kst and the V tile at vst. S = Q K^T (16 MMAs at D 128), online
-// softmax in base 2 on the S fragments, then O += P V with P split into a bf16
-// high part and remainder (32 MMAs). V rows of invalid tokens are zeroed in
-// registers so padding never reaches O.
+// the K tile at kst and the V tile at vst, with the tokens as the MMA's M:
+//   S^T = K q^T   (M 16 tokens, N 8 heads, K 16 dims per step: 8 MMAs at D 128,
+//                  in two independent chains)
+//   O^T += V^T P^T (M 16 dims, N 8 heads, K 16 tokens: 2 MMAs per 16 dims,
+//                  P split into a bf16 high part and remainder)
+// so no MMA row is spent on padding heads (G <= 8 fill the N columns). A lane
+// holds heads 2c, 2c+1 (c = lane % 4) of tokens / dims r, r + 8 (r = lane / 4);
+// the running max and sum are per head; P^T's fragments come from S^T's by an
+// 8x8 transpose in registers (movmatrix). V rows of invalid tokens are zeroed
+// in registers so padding never reaches O.
+//   o[t][0..3]: dims 16t + r (heads 2c, 2c+1), 16t + r + 8 (heads 2c, 2c+1)
 template <int D>
-__device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, const uint32_t (&qa)[D / 16][2],
-                                          float scale_log2, int lane, int warp, float& m_run, float& l_run,
-                                          float (&o)[D / 8][2], int bs) {
+__device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, const uint32_t (&qb)[D / 16][2],
+                                          float scale_log2, int lane, int warp, float (&m_run)[2], float (&l_run)[2],
+                                          float (&o)[D / 16][4], int bs) {
   using Cfg = MmaCfg<D>;
-  constexpr int NT = D / 8;
-  const int c = lane & 3;
-  const int mk = lane >> 3, ik = lane & 7;
-  const int tokK = warp * 16 + (mk >> 1) * 8 + ik;  // K matrices (tok0, d0), (tok0, d0+8), (tok0+8, d0), (tok0+8, d0+8)
-  const int dK = (mk & 1) * 8;
-  const int tokV = warp * 16 + (mk & 1) * 8 + ik;   // V matrices (tok0, d0), (tok0+8, d0), (tok0, d0+8), (tok0+8, d0+8)
-  const int dV = (mk >> 1) * 8;
-  float sacc[2][2];
-  float dead0[2] = {0.f, 0.f}, dead1[2] = {0.f, 0.f};
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = 0.f;
-  // K fragments run kPre k-steps ahead of the MMAs that use them (a ring of
-  // kPre x 4 registers), so a load's latency is hidden behind earlier MMAs
-  // instead of stalling each k-step (the asm statements keep source order)
-  constexpr int kPre = PA_MMA_PREFETCH;
   constexpr int KS = D / 16;
+  const int c = lane & 3, r = lane >> 2;
+  const int mk = lane >> 3, ik = lane & 7;
+  // ldmatrix rows: K matrices (tok0, d0), (tok0, d0+8), (tok0+8, d0), (tok0+8, d0+8);
+  // V matrices (tok0, d0), (tok0+8, d0), (tok0, d0+8), (tok0+8, d0+8)
+  const int tokK = warp * 16 + (mk >> 1) * 8 + ik;
+  const int dK = (mk & 1) * 8;
+  const int tokV = warp * 16 + (mk & 1) * 8 + ik;
+  const int dV = (mk >> 1) * 8;
   // stage layout: block b of the chunk at b * bs * D * 2 bytes, inside it the
   // 64-element half h at h * bs * 128, row t at t * 128, its 16-byte pieces
   // swizzled by (t & 7) (the 128-byte swizzle of the TMA; block and half
@@ -207,60 +187,62 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
     const int d0 = dgi * 16 + dV;
     return vbase + (d0 >> 6) * hstride + ((((d0 & 63) >> 3) ^ (tokV & 7)) << 4);
   };
-  uint32_t kf[kPre][4];
-#pragma unroll
-  for (int u = 0; u < kPre; ++u) ldsm_x4(k_addr(u), kf[u][0], kf[u][1], kf[u][2], kf[u][3]);
+  float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int kk = 0; kk < KS; ++kk) {
-    const uint32_t b00 = kf[kk % kPre][0], b01 = kf[kk % kPre][1], b10 = kf[kk % kPre][2], b11 = kf[kk % kPre][3];
-    if (kk + kPre < KS)
-      ldsm_x4(k_addr(kk + kPre), kf[kk % kPre][0], kf[kk % kPre][1], kf[kk % kPre][2], kf[kk % kPre][3]);
-    mma_rows8_chain(sacc[0], qa[kk][0], qa[kk][1], b00, b01, dead0);
-    mma_rows8_chain(sacc[1], qa[kk][0], qa[kk][1], b10, b11, dead1);
+    uint32_t m0, m1, m2, m3;
+    ldsm_x4(k_addr(kk), m0, m1, m2, m3);
+    // A = K rows (tokens) x 16 dims: a0 (tok0, d0), a1 (tok0+8, d0), a2 (tok0, d0+8), a3 (tok0+8, d0+8)
+    mma16x8(kk & 1 ? s1 : s0, m0, m2, m1, m3, qb[kk][0], qb[kk][1]);
   }
-  // the first V fragments are loaded before the softmax, which hides their latency
-  uint32_t vf[kPre][4];
+  float x[4];
+  const bool va = r < nv, vb = r + 8 < nv;
 #pragma unroll
-  for (int u = 0; u < kPre; ++u) ldsm_x4_t(v_addr(u), vf[u][0], vf[u][1], vf[u][2], vf[u][3]);
-  float sc[2][2];
-  float mloc = -INFINITY;
+  for (int e = 0; e < 4; ++e) x[e] = (e < 2 ? va : vb) ? (s0[e] + s1[e]) * scale_log2 : -INFINITY;
+  float mloc[2];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int t = nt * 8 + 2 * c + j;
-      sc[nt][j] = t < nv ? sacc[nt][j] * scale_log2 : -INFINITY;
-      mloc = fmaxf(mloc, sc[nt][j]);
-    }
-  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+  for (int j = 0; j < 2; ++j) {
+    float v = fmaxf(x[j], x[2 + j]);
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+    mloc[j] = v;
+  }
   // the reference maximum moves only when a score exceeds it by 8 (log2
   // units): weights stay <= 2^8 and O is rarely rescaled
-  const bool move = mloc > m_run + 8.f;
-  const float mn = move ? mloc : m_run;
-  float pr[2][2];
-  float psum = 0.f;
+  bool move[2];
+  float mn[2];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int j = 0; j < 2; ++j) {
+    move[j] = mloc[j] > m_run[j] + 8.f;
+    mn[j] = move[j] ? mloc[j] : m_run[j];
+  }
+  float pr[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - mn[e & 1]);
+  if (__any_sync(0xffffffffu, move[0] || move[1])) {
+    float alpha[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      pr[nt][j] = fast_exp2(sc[nt][j] - mn);
-      psum += pr[nt][j];
+      alpha[j] = fast_exp2(m_run[j] - mn[j]);  // 1 for heads that did not move, 0 from -inf
+      l_run[j] *= alpha[j];
     }
-  if (__any_sync(0xffffffffu, move)) {
-    const float alpha = fast_exp2(m_run - mn);  // 1 for rows that did not move, 0 from -inf
-    l_run *= alpha;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      o[j][0] *= alpha;
-      o[j][1] *= alpha;
-    }
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[t][e] *= alpha[e & 1];
   }
-  m_run = mn;
-  l_run += psum;
-  uint32_t ph0, pl0, ph2, pl2;
-  split_pair(pr[0][0], pr[0][1], ph0, pl0);
-  split_pair(pr[1][0], pr[1][1], ph2, pl2);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    m_run[j] = mn[j];
+    l_run[j] += pr[j] + pr[2 + j];
+  }
+  // P^T as B fragments (K 16 tokens x N 8 heads): transpose the S^T-layout pairs
+  uint32_t h01, l01, h23, l23;
+  split_pair(pr[0], pr[1], h01, l01);
+  split_pair(pr[2], pr[3], h23, l23);
+  const uint32_t bh0 = movmatrix_t(h01), bh1 = movmatrix_t(h23);
+  const uint32_t bl0 = movmatrix_t(l01), bl1 = movmatrix_t(l23);
   uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
   if (nv < 16) {
     mlo = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
@@ -268,22 +250,30 @@ __device__ __forceinline__ void mma_chunk(uint32_t kst, uint32_t vst, int nv, co
   }
 #pragma unroll
   for (int dgi = 0; dgi < D / 16; ++dgi) {
-    uint32_t v0 = vf[dgi % kPre][0], v1 = vf[dgi % kPre][1], v2 = vf[dgi % kPre][2], v3 = vf[dgi % kPre][3];
-    if (dgi + kPre < D / 16)
-      ldsm_x4_t(v_addr(dgi + kPre), vf[dgi % kPre][0], vf[dgi % kPre][1], vf[dgi % kPre][2], vf[dgi % kPre][3]);
+    uint32_t v0, v1, v2, v3;
+    ldsm_x4_t(v_addr(dgi), v0, v1, v2, v3);
+    // A = V^T (16 dims x 16 tokens): a0 (d0, tok0), a1 (d0+8, tok0), a2 (d0, tok0+8), a3 (d0+8, tok0+8)
     v0 &= mlo;
     v1 &= mhi;
     v2 &= mlo;
     v3 &= mhi;
-    mma_rows8(o[2 * dgi], ph0, ph2, v0, v1);
-    mma_rows8(o[2 * dgi], pl0, pl2, v0, v1);
-    mma_rows8(o[2 * dgi + 1], ph0, ph2, v2, v3);
-    mma_rows8(o[2 * dgi + 1], pl0, pl2, v2, v3);
+    mma16x8(o[dgi], v0, v2, v1, v3, bh0, bh1);
+    mma16x8(o[dgi], v0, v2, v1, v3, bl0, bl1);
   }
 }
 
-// Q rows (bf16, row stride D) as MMA A fragments: a0 = row r, dims (kk*16 + 2c,
-// +1); a2 = dims +8; rows >= G are zero.
+// A warp's l, summed over its lanes' tokens (lanes of one c hold the same heads).
+__device__ __forceinline__ void sum_l(float (&l)[2]) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    l[j] += __shfl_xor_sync(0xffffffffu, l[j], 4);
+    l[j] += __shfl_xor_sync(0xffffffffu, l[j], 8);
+    l[j] += __shfl_xor_sync(0xffffffffu, l[j], 16);
+  }
+}
+
+// Q rows (bf16, row stride D) as the B fragments of S^T = K q^T (column r =
+// head r): b0 = dims (kk*16 + 2c, +1), b1 = dims +8; heads >= G are zero.
 template <int D, int G>
 __device__ __forceinline__ void load_q_frags(const uint32_t* qrow_words, int r, int c, uint32_t (&qa)[D / 16][2],
                                              bool from_global) {
@@ -324,31 +314,37 @@ __device__ __forceinline__ bool consumer_sync(uint64_t* bar, uint32_t& phase, vo
   return ok;
 }
 
-// Fold another warp's (m, l, o) (same fragment layout) into this lane's.
-template <int NT>
-__device__ __forceinline__ void fold_state(float& m, float& l, float (&o)[NT][2], const float* src) {
-  const float m2 = src[2 * NT], l2 = src[2 * NT + 1];
-  const float M = fmaxf(m, m2);
-  if (M == -INFINITY) return;  // both empty
-  const float f1 = exp2f(m - M), f2 = exp2f(m2 - M);
-  l = l * f1 + l2 * f2;
+// Fold another warp's (m, l, o) (same fragment layout) into this lane's:
+// per head j of the lane (o[t][j], o[t][2 + j]).
+template <int D>
+__device__ __forceinline__ void fold_state(float (&m)[2], float (&l)[2], float (&o)[D / 16][4], const float* src) {
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    o[j][0] = o[j][0] * f1 + src[2 * j] * f2;
-    o[j][1] = o[j][1] * f1 + src[2 * j + 1] * f2;
+  for (int j = 0; j < 2; ++j) {
+    const float m2 = src[D / 4 + j], l2 = src[D / 4 + 2 + j];
+    const float M = fmaxf(m[j], m2);
+    if (M == -INFINITY) continue;  // both empty
+    const float f1 = exp2f(m[j] - M), f2 = exp2f(m2 - M);
+    l[j] = l[j] * f1 + l2 * f2;
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t) {
+      o[t][j] = o[t][j] * f1 + src[4 * t + j] * f2;
+      o[t][2 + j] = o[t][2 + j] * f1 + src[4 * t + 2 + j] * f2;
+    }
+    m[j] = M;
   }
-  m = M;
 }
 
-template <int NT>
-__device__ __forceinline__ void store_state(float* dst, float m, float l, const float (&o)[NT][2]) {
+template <int D>
+__device__ __forceinline__ void store_state(float* dst, const float (&m)[2], const float (&l)[2],
+                                            const float (&o)[D / 16][4]) {
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    dst[2 * j] = o[j][0];
-    dst[2 * j + 1] = o[j][1];
-  }
-  dst[2 * NT] = m;
-  dst[2 * NT + 1] = l;
+  for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[4 * t + e] = o[t][e];
+  dst[D / 4] = m[0];
+  dst[D / 4 + 1] = m[1];
+  dst[D / 4 + 2] = l[0];
+  dst[D / 4 + 3] = l[1];
 }
 
 template <int D, int G>
@@ -356,7 +352,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const DecodeArgs a) {
   using Cfg = MmaCfg<D>;
-  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = Cfg::kNT;
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages;
   static_assert(G <= 8, "query heads of one group must fit in MMA rows 0..7");
 
   extern __shared__ uint8_t smem_raw[];
@@ -484,15 +480,15 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
 
   // -------------------------------- consumers --------------------------------
   uint32_t qa[D / 16][2];
-  float o[NT][2];
-  float m_run = -INFINITY, l_run = 0.f;
+  float o[D / 16][4];
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
   uint32_t cphase = 0;
 #define PA_CSYNC()                                                    \
   do {                                                                \
     if (!consumer_sync(&ps.cbar, cphase, &ps.abort_flag, lane)) return; \
   } while (0)
 #pragma unroll
-  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
+  for (int t = 0; t < D / 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
 
   for (int cs = 0;; ++cs) {
     const int st = cs % S;
@@ -505,10 +501,13 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
     if (flags & kDescFirst) {
       load_q_frags<D, G>(reinterpret_cast<const uint32_t*>(qslot_gen + st * Cfg::kQBytes) + r * (D / 2), r, c, qa,
                          false);
-      m_run = -INFINITY;
-      l_run = 0.f;
 #pragma unroll
-      for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
+      for (int j = 0; j < 2; ++j) {
+        m_run[j] = -INFINITY;
+        l_run[j] = 0.f;
+      }
+#pragma unroll
+      for (int t = 0; t < D / 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
     }
 
     const int nv = min(16, dn - warp * 16);  // warp-uniform
@@ -522,37 +521,51 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
     if (!(flags & kDescLast)) continue;
 
     // ---- item finished: fold warps 3,2 -> 1,0 -> 0 (two rounds), then store ----
-    float lrow = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
-    lrow += __shfl_xor_sync(0xffffffffu, lrow, 2);
-    float* slot0 = fold + lane * (2 * NT + 2);
-    float* slot1 = fold + Cfg::kFoldFloats + lane * (2 * NT + 2);
-    if (warp >= 2) store_state<NT>(warp == 2 ? slot0 : slot1, m_run, lrow, o);
+    float lrow[2] = {l_run[0], l_run[1]};
+    sum_l(lrow);
+    float* slot0 = fold + lane * (D / 4 + 4);
+    float* slot1 = fold + Cfg::kFoldFloats + lane * (D / 4 + 4);
+    if (warp >= 2) store_state<D>(warp == 2 ? slot0 : slot1, m_run, lrow, o);
     PA_CSYNC();
-    if (warp < 2) fold_state<NT>(m_run, lrow, o, warp == 0 ? slot0 : slot1);
+    if (warp < 2) fold_state<D>(m_run, lrow, o, warp == 0 ? slot0 : slot1);
     PA_CSYNC();
-    if (warp == 1) store_state<NT>(slot0, m_run, lrow, o);
+    if (warp == 1) store_state<D>(slot0, m_run, lrow, o);
     PA_CSYNC();
-    if (warp == 0) fold_state<NT>(m_run, lrow, o, slot0);
+    if (warp == 0) fold_state<D>(m_run, lrow, o, slot0);
 
     const int64_t row0 = static_cast<int64_t>(ds) * a.hq + dg * G;
     if (dnp == 1 && !a.force_partials) {
-      if (warp == 0 && r < G) {
-        const float inv = 1.f / lrow;
-        float* dst = a.out + (row0 + r) * D + 2 * c;
+      if (warp == 0) {
 #pragma unroll
-        for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0] * inv, o[j][1] * inv);
+        for (int j = 0; j < 2; ++j) {
+          if (2 * c + j >= G) continue;
+          const float inv = 1.f / lrow[j];
+          float* dst = a.out + (row0 + 2 * c + j) * D + r;
+#pragma unroll
+          for (int t = 0; t < D / 16; ++t) {
+            dst[16 * t] = o[t][j] * inv;
+            dst[16 * t + 8] = o[t][2 + j] * inv;
+          }
+        }
       }
       PA_CSYNC();  // the fold slots are free again
       continue;
     }
     // split sequence: publish this partition's (m, l, o); the last partition's
     // consumers (fused merge) or decode_reduce_kernel merge them
-    if (warp == 0 && r < G) {
-      const int64_t prow = (row0 + r) * a.parts_stride + dp;
-      float* dst = a.ws_o + prow * D + 2 * c;
+    if (warp == 0) {
 #pragma unroll
-      for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
-      if (c == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(m_run, lrow);
+      for (int j = 0; j < 2; ++j) {
+        if (2 * c + j >= G) continue;
+        const int64_t prow = (row0 + 2 * c + j) * a.parts_stride + dp;
+        float* dst = a.ws_o + prow * D + r;
+#pragma unroll
+        for (int t = 0; t < D / 16; ++t) {
+          dst[16 * t] = o[t][j];
+          dst[16 * t + 8] = o[t][2 + j];
+        }
+        if (r == 0) *reinterpret_cast<float2*>(a.ws_ml + prow * 2) = make_float2(m_run[j], lrow[j]);
+      }
     }
     if (a.fuse_merge) {
       __threadfence();
@@ -575,7 +588,7 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const DecodeArgs a) {
   using Cfg = MmaCfg<D>;
-  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = Cfg::kNT;
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages;
   static_assert(NW * G * (D + 2) * 4 <= S * Cfg::kStageBytes, "merge buffer must fit in the stage ring");
 
   extern __shared__ uint8_t smem_raw[];
@@ -595,10 +608,10 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
   if (tid == 0) pipe_init<S>(ps, NW);
   __syncthreads();
 
-  float o[NT][2];
+  float o[D / 16][4];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  for (int t = 0; t < D / 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
   if (warp == NW) {
     // fused KV append: the new row is loaded now and stored before the last
@@ -648,8 +661,7 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&ps.empty[st]);
     }
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    sum_l(l_run);
   }
 
   __syncthreads();  // every copy consumed; the stage ring is free
@@ -658,15 +670,20 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
   float* wm = reinterpret_cast<float*>(sgen);
   float* wl = wm + NW * G;
   float* wacc = wl + NW * G;
-  if (warp < NW && r < G) {
-    if (c == 0) {
-      wm[warp * G + r] = m_run;
-      wl[warp * G + r] = l_run;
-    }
+  if (warp < NW) {
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      wacc[(warp * G + r) * D + j * 8 + 2 * c] = o[j][0];
-      wacc[(warp * G + r) * D + j * 8 + 2 * c + 1] = o[j][1];
+    for (int j = 0; j < 2; ++j) {
+      const int h = 2 * c + j;
+      if (h >= G) continue;
+      if (r == 0) {
+        wm[warp * G + h] = m_run[j];
+        wl[warp * G + h] = l_run[j];
+      }
+#pragma unroll
+      for (int t = 0; t < D / 16; ++t) {
+        wacc[(warp * G + h) * D + 16 * t + r] = o[t][j];
+        wacc[(warp * G + h) * D + 16 * t + r + 8] = o[t][2 + j];
+      }
     }
   }
   __syncthreads();
