@@ -95,7 +95,7 @@ __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint3
 }
 
 // Build-time tuning knobs of the one-CTA-per-item kernel (defaults measured
-// on B200): ring stages at head_dim 128 (0 = the default of 3), and the CTAs
+// on B200): ring stages at head_dim 128 (0 = the default of 2), and the CTAs
 // per SM its register budget is fitted to.
 #ifndef PA_MMA_STAGES
 #define PA_MMA_STAGES 0
@@ -120,11 +120,17 @@ struct MmaCfg {
   static constexpr int kHalfBytes = kChunk * 128;          // one 64-element column of a stage's K (or V)
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = kStageBytes <= 16384 ? 4 : (PA_MMA_STAGES > 0 ? PA_MMA_STAGES : 3);
+  // one-CTA-per-item kernels (and the cascade prefix pass): two 32 KB stages at
+  // head_dim 128, so three CTAs share an SM (measured on B200 against three
+  // stages and two CTAs: continuous batching 0.1383 -> 0.1322 ms, the cascade
+  // 0.0427 -> 0.0407 ms); the persistent kernel keeps three (its producer runs
+  // across items; two stages there: long context 0.2253 -> 0.2347 ms)
+  static constexpr int kStages = kStageBytes <= 16384 ? 4 : (PA_MMA_STAGES > 0 ? PA_MMA_STAGES : 2);
+  static constexpr int kPStages = kStageBytes <= 16384 ? 4 : 3;
   static constexpr int kQBytes = 8 * D * 2;                // query rows of one item (G <= 8)
   static constexpr int kFoldFloats = 32 * (D / 4 + 4);     // one warp's O fragments + (m, l) of 2 heads per lane
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes;  // one CTA per item
-  static constexpr int kPersistSmemBytes = kSmemBytes + kStages * kQBytes + 2 * kFoldFloats * 4;
+  static constexpr int kPersistSmemBytes = 1024 + kPStages * kStageBytes + kPStages * kQBytes + 2 * kFoldFloats * 4;
 };
 
 
@@ -352,7 +358,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads) decode_mma_persistent_ker
                                                                         const __grid_constant__ CUtensorMap tmv,
                                                                         const DecodeArgs a) {
   using Cfg = MmaCfg<D>;
-  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages;
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kPStages;
   static_assert(G <= 8, "query heads of one group must fit in MMA rows 0..7");
 
   extern __shared__ uint8_t smem_raw[];
