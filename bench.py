@@ -53,30 +53,30 @@ NCU_TRAFFIC: dict = {
         bytes=1_079_315_883 + 2_277_120, files=_DEC + ["decode_simt.cuh"], sha="9489fe02f3c535bb",
         note="decode_simt_kernel of pa_decode_append (the step's only launch), 3 launches"),
     ("llama2_7b_mha", "float8_e4m3fn", 0, "decode"): dict(
-        bytes=540_494_763 + 8_050_091, files=_DEC + ["decode_f8.cuh"], sha="0821c9cb1e81d0ca",
+        bytes=540_494_763 + 8_050_091, files=_DEC + ["decode_f8.cuh"], sha="e3c3f2af2d50fd9c",
         note="decode_f8_kernel (e4m3) of pa_decode_append, 3 launches"),
     ("llama2_7b_mha", "int8", 0, "decode"): dict(
-        bytes=540_492_373 + 8_290_987, files=_DEC + ["decode_f8.cuh"], sha="0821c9cb1e81d0ca",
+        bytes=540_492_373 + 8_290_987, files=_DEC + ["decode_f8.cuh"], sha="e3c3f2af2d50fd9c",
         note="decode_f8_kernel (int8) of pa_decode_append, 3 launches"),
     ("long_context_split", "bfloat16", 512, "decode"): dict(
-        bytes=1_343_023_275 + 6_138_112 + 21_472_341, files=_DEC + ["decode_mma.cuh"], sha="a8e832b3f88ba6d7",
+        bytes=1_342_990_080 + 6_214_229 + 21_473_621, files=_DEC + ["decode_mma.cuh"], sha="915c9bdf9030f201",
         note="decode_mma_persistent_kernel + decode_reduce_kernel, 3 launches each"),
     ("parallel_sampling", "bfloat16", 0, "decode"): dict(
-        bytes=121_091_200 + 469_760, files=_DEC + ["decode_mma.cuh"], sha="a8e832b3f88ba6d7",
-        note="decode_mma_kernel of pa_decode_append, 6 launches (1.25x the 97.5 MB of distinct blocks: with the "
+        bytes=113_246_549 + 388_437, files=_DEC + ["decode_mma.cuh"], sha="915c9bdf9030f201",
+        note="decode_mma_kernel of pa_decode_append, 6 launches (1.17x the 97.5 MB of distinct blocks: with the "
              "longest-first order a prompt's samples no longer all run at once)"),
     ("parallel_sampling", "bfloat16", 0, "cascade"): dict(
-        bytes=32_023_552 + 5_205 + 72_904_397 + 77_824, files=_DEC + ["decode_mma.cuh", "prefill_mma.cuh"], sha="3220a31f59111fd6",
+        bytes=32_022_485 + 1_323 + 72_883_917 + 106_394, files=_DEC + ["decode_mma.cuh", "prefill_mma.cuh"], sha="96f8c67c8ea950e0",
         note="prefill_mma_kernel (prefix pass) + decode_mma_kernel (suffixes and fold), 5-6 launches each"),
     ("continuous_batching", "bfloat16", 0, "decode"): dict(
-        bytes=835_075_447 + 2_500_437, files=_DEC + ["decode_mma.cuh"], sha="a8e832b3f88ba6d7",
+        bytes=835_070_020 + 2_660_804, files=_DEC + ["decode_mma.cuh"], sha="915c9bdf9030f201",
         note="decode_mma_kernel of pa_decode_append over steps 0-29 of the trace (32768-block pool); their "
              "algorithmic mean is 825.0 MB per step (x1.015), the 200-step mean 811.2 MB"),
     ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
-        bytes=1_309_527_296 + 230_245_449, files=_PF, sha="d85c79484f101e28",
+        bytes=1_309_527_296 + 230_245_449, files=_PF, sha="11b6569f1f58cdf6",
         note="prefill_tc_kernel, 7 launches (Q, K/V per tile pair not served by L2, the fp32 output)"),
     ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
-        bytes=760_672_549 + 489_605_010, files=_PF, sha="d85c79484f101e28", note="prefill_tc_kernel, 7 launches"),
+        bytes=760_672_549 + 489_605_010, files=_PF, sha="11b6569f1f58cdf6", note="prefill_tc_kernel, 7 launches"),
 }
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
