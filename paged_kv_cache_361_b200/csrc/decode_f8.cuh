@@ -42,20 +42,12 @@
 
 namespace pa {
 
-// Build-time tuning knobs, defaults measured on B200 (e4m3 metric workload:
-// 0.1278 ms with q fragments in registers, 4 stages and 3 CTAs per SM; 0.1219 ms
-// with all four below): split each QK^T accumulation chain in two; the q
-// fragments read from shared memory at every k-step and V one 32-bit word at
-// a time (fewer registers); 3 stages; the register budget fitted to 4 CTAs per
-// SM (96 registers, a few spilled words).
-#ifndef PA_F8_SPLIT_CHAINS
-#define PA_F8_SPLIT_CHAINS 1
-#endif
+// Build-time tuning knobs, defaults measured on B200 (e4m3 metric workload):
+// 3 stages and the register budget fitted to 4 CTAs per SM (q fragments read
+// from shared memory at every k-step, V one 32-bit word at a time; with q in
+// registers, 4 stages and 3 CTAs per SM the kernel was 5 % slower).
 #ifndef PA_F8_MIN_CTAS
 #define PA_F8_MIN_CTAS 4
-#endif
-#ifndef PA_F8_LEAN
-#define PA_F8_LEAN 1
 #endif
 #ifndef PA_F8_STAGES
 #define PA_F8_STAGES 3
@@ -76,9 +68,8 @@ struct F8Cfg {
   static constexpr int kTileBytes = kChunk * D;     // K (or V) of one stage
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = PA_F8_STAGES;
-  static constexpr int kQSmemBytes = PA_F8_LEAN ? 32 * (D / 16) * 8 : 0;  // q fragments of every lane
+  static constexpr int kQSmemBytes = 32 * (D / 16) * 8;  // q fragments of every lane
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kQSmemBytes;
-  static constexpr int kNT = D / 8;                 // output n-tiles
 };
 
 // Byte offset of (row, byte column) in a swizzled tile of D-byte rows, as the
@@ -163,203 +154,139 @@ __device__ __forceinline__ void widen_row_half(const uint8_t* src, uint8_t* dst,
   }
 }
 
-// m16n8k16 f16 MMA with rows 8..15 of A zero and their results discarded
-// (their registers are never held).
-__device__ __forceinline__ void mma_f16_rows8(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  float j2, j3;
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%10, %11, %12, %12};"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(j2), "=f"(j3)
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f));
-  asm volatile("" ::"f"(j2), "f"(j3));
-}
-
-// The same MMA for a dependent chain (one accumulator over the k-steps): rows
-// 8..15 accumulate into the chain's own `dead` pair (never read), which
-// saves materialising zero inputs per MMA without adding dependences.
-__device__ __forceinline__ void mma_f16_rows8_chain(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0,
-                                                    uint32_t b1, float (&dead)[2]) {
+// m16n8k16 f16 MMA, fp32 accumulate in place (all four A registers).
+__device__ __forceinline__ void mma16x8_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(dead[0]), "+f"(dead[1])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// The q fragments of a lane for k-step kk: held in registers, or read from
-// shared memory (32 lanes' pairs per k-step).
-template <int D>
-struct QFragRegs {
-  uint32_t v[D / 16][2];
-  __device__ __forceinline__ uint2 operator()(int kk) const { return make_uint2(v[kk][0], v[kk][1]); }
-};
+// The q fragments of a lane for k-step kk, read from shared memory (every
+// consumer warp uses the same ones: 32 lanes' pairs per k-step).
 struct QFragSmem {
   const uint2* p;
   int lane;
   __device__ __forceinline__ uint2 operator()(int kk) const { return p[kk * 32 + lane]; }
 };
 
-// Output dim of n-tile j, column n.
+// Output dim of row r (r < 8) of m-tile t in f8_chunk's O^T, and of row r + 8
+// one more: a lane's rows cover dims [16r, 16r + 16) at head_dim 128 ([8r,
+// 8r + 8) at 64), which are the bytes of the one V piece it reads per token.
 template <int D>
-__device__ __forceinline__ int f8_dim(int j, int n) {
-  return (D == 128 ? 16 : 8) * n + j;
+__device__ __forceinline__ int f8_dim(int t, int r) {
+  return (D == 128 ? 16 : 8) * r + 2 * t;
 }
 
-// One consumer warp's 16 tokens (nv valid) of a stage.
-template <int D, int CF, class QFrag>
-__device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, int nv, const QFrag& qa,
-                                         float scale_log2, int lane, int warp, float& m_run, float& l_run,
-                                         float (&o)[D / 8][2]) {
-  constexpr int NT = D / 8;
-  const int gq = lane >> 2, c = lane & 3;
+// One consumer warp's 16 tokens (nv valid) of a stage, with the tokens (or
+// dims) as the MMA's M and the heads as its N:
+//   S^T = K q^T : A = the warp's K rows widened to f16; per k-step a thread's
+//                 registers are four adjacent codes of one row, dims
+//                 (16kk + 4c, +1) and (16kk + 4c + 2, +3) (one 32-bit shared
+//                 load per row), q is taken in the same order; two chains
+//   O^T += V^T P^T: A = V^T widened, M row r of m-tile t being dim
+//                 f8_dim(t, r) (r + 8: one more), so that a thread's rows of
+//                 every m-tile come from one piece of each of its four tokens'
+//                 V rows, paired across tokens by byte permutes; B = P^T, the
+//                 f16 weights of S^T transposed in registers (movmatrix)
+// A lane keeps the running maximum and sum of heads 2c, 2c+1 (c = lane % 4).
+//   o[t][0..3]: dim f8_dim(t, r) (heads 2c, 2c+1), that dim + 1 (heads 2c, 2c+1)
+template <int D, int CF>
+__device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, int nv, const QFragSmem& qa,
+                                         float scale_log2, int lane, int warp, float (&m_run)[2], float (&l_run)[2],
+                                         float (&o)[D / 16][4]) {
+  const int r = lane >> 2, c = lane & 3;
   const int tw = warp * 16;
-  float sacc[2][2];
   // A row's start (the 1024-byte aligned tile base plus row * D) has bits
   // 0..6 (128-byte rows) or 0..5 (64-byte rows) clear, so the swizzled address
   // of 16-byte chunk kk is (row start | swizzle key << 4 | byte) ^ (kk << 4).
   const uint32_t kts = smem_u32(kt);
-#if PA_F8_LEAN
-  {
-    // both n-tiles per k-step, the k-step's q pair read from shared memory
-    float dead0[2] = {0.f, 0.f}, dead1[2] = {0.f, 0.f};
-    uint32_t rb[2];
+  uint32_t rb[2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      sacc[nt][0] = sacc[nt][1] = 0.f;
-      const int row = tw + nt * 8 + gq;
-      const uint32_t key = D == 128 ? static_cast<uint32_t>(row & 7) : static_cast<uint32_t>((row >> 1) & 3);
-      rb[nt] = (kts + static_cast<uint32_t>(row * D)) | (key << 4) | static_cast<uint32_t>(4 * c);
-    }
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint2 qq = qa(kk);
-      uint32_t w0, w1;
-      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w0) : "r"(rb[0] ^ static_cast<uint32_t>(kk << 4)));
-      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w1) : "r"(rb[1] ^ static_cast<uint32_t>(kk << 4)));
-      uint32_t b00, b01, b10, b11;
-      widen4<CF>(w0, b00, b01);
-      widen4<CF>(w1, b10, b11);
-      mma_f16_rows8_chain(sacc[0], qq.x, qq.y, b00, b01, dead0);
-      mma_f16_rows8_chain(sacc[1], qq.x, qq.y, b10, b11, dead1);
-    }
-  }
-#else
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    sacc[nt][0] = sacc[nt][1] = 0.f;
-    float dead[2] = {0.f, 0.f};
-    const int row = tw + nt * 8 + gq;
+  for (int h = 0; h < 2; ++h) {
+    const int row = tw + h * 8 + r;
     const uint32_t key = D == 128 ? static_cast<uint32_t>(row & 7) : static_cast<uint32_t>((row >> 1) & 3);
-    const uint32_t rbase = (kts + static_cast<uint32_t>(row * D)) | (key << 4) | static_cast<uint32_t>(4 * c);
-#if PA_F8_SPLIT_CHAINS
-    // two accumulators per n-tile (even and odd k-steps): half the chain length
-    float s2[2] = {0.f, 0.f}, dead2[2] = {0.f, 0.f};
-#endif
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t w;
-      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w) : "r"(rbase ^ static_cast<uint32_t>(kk << 4)));
-      uint32_t b0, b1;
-      widen4<CF>(w, b0, b1);
-#if PA_F8_SPLIT_CHAINS
-      if (kk & 1)
-        mma_f16_rows8_chain(s2, qa(kk).x, qa(kk).y, b0, b1, dead2);
-      else
-#endif
-        mma_f16_rows8_chain(sacc[nt], qa(kk).x, qa(kk).y, b0, b1, dead);
-    }
-#if PA_F8_SPLIT_CHAINS
-    sacc[nt][0] += s2[0];
-    sacc[nt][1] += s2[1];
-#endif
+    rb[h] = (kts + static_cast<uint32_t>(row * D)) | (key << 4) | static_cast<uint32_t>(4 * c);
   }
-#endif
-  float sc[2][2];
-  float mloc = -INFINITY;
+  float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint2 qq = qa(kk);
+    uint32_t w0, w1;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w0) : "r"(rb[0] ^ static_cast<uint32_t>(kk << 4)));
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w1) : "r"(rb[1] ^ static_cast<uint32_t>(kk << 4)));
+    uint32_t k00, k01, k10, k11;
+    widen4<CF>(w0, k00, k01);  // token r: dims (4c, 4c+1), (4c+2, 4c+3) of the k-step
+    widen4<CF>(w1, k10, k11);  // token r + 8
+    mma16x8_f16(kk & 1 ? s1 : s0, k00, k10, k01, k11, qq.x, qq.y);
+  }
+  float x[4];
+  const bool va = r < nv, vb = r + 8 < nv;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int t = nt * 8 + 2 * c + j;
-      sc[nt][j] = t < nv ? sacc[nt][j] * scale_log2 : -INFINITY;
-      mloc = fmaxf(mloc, sc[nt][j]);
-    }
-  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+  for (int e = 0; e < 4; ++e) x[e] = (e < 2 ? va : vb) ? (s0[e] + s1[e]) * scale_log2 : -INFINITY;
+  float mloc[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float v = fmaxf(x[j], x[2 + j]);
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+    mloc[j] = v;
+  }
   // the reference maximum moves only when a score exceeds it by 8 (log2
   // units): weights stay <= 2^8 (f16 holds them) and O is rarely rescaled
-  const bool move = mloc > m_run + 8.f;
-  const float mn = move ? mloc : m_run;
-  float pr[2][2];
-  float psum = 0.f;
+  bool move[2];
+  float mn[2];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int j = 0; j < 2; ++j) {
+    move[j] = mloc[j] > m_run[j] + 8.f;
+    mn[j] = move[j] ? mloc[j] : m_run[j];
+  }
+  float pr[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - mn[e & 1]);
+  if (__any_sync(0xffffffffu, move[0] || move[1])) {
+    float alpha[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      pr[nt][j] = fast_exp2(sc[nt][j] - mn);
-      psum += pr[nt][j];
+      alpha[j] = fast_exp2(m_run[j] - mn[j]);  // 1 for heads that did not move, 0 from -inf
+      l_run[j] *= alpha[j];
     }
-  if (__any_sync(0xffffffffu, move)) {
-    const float alpha = fast_exp2(m_run - mn);  // 1 for rows that did not move, 0 from -inf
-    l_run *= alpha;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      o[j][0] *= alpha;
-      o[j][1] *= alpha;
-    }
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[t][e] *= alpha[e & 1];
   }
-  m_run = mn;
-  l_run += psum;
-  const uint32_t pa0 = pack_f16(pr[0][0], pr[0][1]);  // tokens 2c, 2c+1
-  const uint32_t pa2 = pack_f16(pr[1][0], pr[1][1]);  // tokens 8+2c, 9+2c
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    m_run[j] = mn[j];
+    l_run[j] += pr[j] + pr[2 + j];
+  }
+  // P^T as B fragments (K 16 tokens x N 8 heads), f16
+  const uint32_t pb0 = movmatrix_t(pack_f16(pr[0], pr[1]));  // tokens 2c, 2c+1
+  const uint32_t pb1 = movmatrix_t(pack_f16(pr[2], pr[3]));  // tokens 8+2c, 9+2c
 
   constexpr int W = D == 128 ? 4 : 2;  // 32-bit words of V per token this thread reads
-  const int col = (D == 128 ? 16 : 8) * gq;
+  const int col = f8_dim<D>(0, r);
   const int t00 = tw + 2 * c, t10 = tw + 8 + 2 * c;
-#if PA_F8_LEAN
-  // one 32-bit word of each of the four tokens' pieces at a time
   const uint8_t* pa_ = vt + f8_off<D>(t00, col);
   const uint8_t* pb_ = vt + f8_off<D>(t00 + 1, col);
   const uint8_t* pc_ = vt + f8_off<D>(t10, col);
   const uint8_t* pd_ = vt + f8_off<D>(t10 + 1, col);
-#define PA_VWORD(p, w) (*reinterpret_cast<const uint32_t*>((p) + 4 * (w)))
-#else
-  uint32_t va[W], vb[W], vc[W], vd[W];
-  if constexpr (D == 128) {
-    const uint4 x0 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t00, col));
-    const uint4 x1 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t00 + 1, col));
-    const uint4 x2 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t10, col));
-    const uint4 x3 = *reinterpret_cast<const uint4*>(vt + f8_off<D>(t10 + 1, col));
-    va[0] = x0.x, va[1] = x0.y, va[2] = x0.z, va[3] = x0.w;
-    vb[0] = x1.x, vb[1] = x1.y, vb[2] = x1.z, vb[3] = x1.w;
-    vc[0] = x2.x, vc[1] = x2.y, vc[2] = x2.z, vc[3] = x2.w;
-    vd[0] = x3.x, vd[1] = x3.y, vd[2] = x3.z, vd[3] = x3.w;
-  } else {
-    const uint2 x0 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t00, col));
-    const uint2 x1 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t00 + 1, col));
-    const uint2 x2 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t10, col));
-    const uint2 x3 = *reinterpret_cast<const uint2*>(vt + f8_off<D>(t10 + 1, col));
-    va[0] = x0.x, va[1] = x0.y;
-    vb[0] = x1.x, vb[1] = x1.y;
-    vc[0] = x2.x, vc[1] = x2.y;
-    vd[0] = x3.x, vd[1] = x3.y;
-  }
-#endif
   const bool ragged = nv < 16;  // warp-uniform
 #pragma unroll
   for (int w = 0; w < W; ++w) {
     // (token a byte k, token b byte k) pairs: bytes 0,1 then 2,3 of each word
+    const uint32_t xa = *reinterpret_cast<const uint32_t*>(pa_ + 4 * w);
+    const uint32_t xb = *reinterpret_cast<const uint32_t*>(pb_ + 4 * w);
+    const uint32_t xc = *reinterpret_cast<const uint32_t*>(pc_ + 4 * w);
+    const uint32_t xd = *reinterpret_cast<const uint32_t*>(pd_ + 4 * w);
     uint32_t b[8];
-#if PA_F8_LEAN
-    const uint32_t xa = PA_VWORD(pa_, w), xb = PA_VWORD(pb_, w), xc = PA_VWORD(pc_, w), xd = PA_VWORD(pd_, w);
-#undef PA_VWORD
-#else
-    const uint32_t xa = va[w], xb = vb[w], xc = vc[w], xd = vd[w];
-#endif
-    widen4<CF>(__byte_perm(xa, xb, 0x5140), b[0], b[1]);
-    widen4<CF>(__byte_perm(xa, xb, 0x7362), b[2], b[3]);
-    widen4<CF>(__byte_perm(xc, xd, 0x5140), b[4], b[5]);
+    widen4<CF>(__byte_perm(xa, xb, 0x5140), b[0], b[1]);  // dims col+4w, col+4w+1 of tokens 2c, 2c+1
+    widen4<CF>(__byte_perm(xa, xb, 0x7362), b[2], b[3]);  // dims col+4w+2, col+4w+3
+    widen4<CF>(__byte_perm(xc, xd, 0x5140), b[4], b[5]);  // the same of tokens 8+2c, 9+2c
     widen4<CF>(__byte_perm(xc, xd, 0x7362), b[6], b[7]);
     if (ragged) {
       // tokens past the valid ones: their V bytes may be NaN codes
@@ -371,8 +298,9 @@ __device__ __forceinline__ void f8_chunk(const uint8_t* kt, const uint8_t* vt, i
         b[4 + k] &= m1;
       }
     }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) mma_f16_rows8(o[4 * w + k], pa0, pa2, b[k], b[4 + k]);
+    // m-tile 2w: rows r, r+8 = dims col+4w, col+4w+1; m-tile 2w+1: col+4w+2, col+4w+3
+    mma16x8_f16(o[2 * w], b[0], b[1], b[4], b[5], pb0, pb1);
+    mma16x8_f16(o[2 * w + 1], b[2], b[3], b[6], b[7], pb0, pb1);
   }
 }
 
@@ -385,8 +313,8 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
                                                                        const __grid_constant__ CUtensorMap tmv,
                                                                        const DecodeArgs a) {
   using Cfg = F8Cfg<D>;
-  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages, NT = Cfg::kNT;
-  static_assert(G <= 8, "query heads of one group must fit in MMA rows 0..7");
+  constexpr int NW = Cfg::kConsumerWarps, C = Cfg::kChunk, S = Cfg::kStages;
+  static_assert(G <= 8, "query heads of one group must fit in the MMA's 8 columns");
   static_assert(NW * G * (D + 2) * 4 <= S * Cfg::kStageBytes, "merge buffer must fit in the stage ring");
 
   extern __shared__ uint8_t smem_raw[];
@@ -407,10 +335,10 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
   if (tid == 0) pipe_init<S>(ps, NW);
   __syncthreads();
 
-  float o[NT][2];
+  float o[D / 16][4];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  for (int t = 0; t < D / 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
   if (warp == NW) {
     // fused KV append: the new row is loaded now and stored before the last
@@ -446,9 +374,11 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
       if (do_append) ar.after_chunk(a, i, nchunks, lane);
     });
   } else {
-    // q rows as f16 A fragments in the dim order of f8_chunk's k-steps:
-    // a0 = dims (16kk + 4c, +1), a2 = dims (16kk + 4c + 2, +3); rows >= G zero
-    QFragRegs<D> qa;
+    // q of head r as the f16 B fragments of f8_chunk's k-steps: dims
+    // (16kk + 4c, +1) and (16kk + 4c + 2, +3); heads >= G zero
+    struct {
+      uint32_t v[D / 16][2];
+    } qa;
     const __nv_bfloat16* qrow =
         static_cast<const __nv_bfloat16*>(a.q) + (static_cast<int64_t>(s) * a.hq + hq0 + (r < G ? r : 0)) * D;
 #pragma unroll
@@ -461,7 +391,6 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
         qa.v[kk][0] = qa.v[kk][1] = 0u;
       }
     }
-#if PA_F8_LEAN
     // every consumer warp has the same fragments: warp 0 parks them in shared memory
     uint2* qsm = reinterpret_cast<uint2*>(sgen + S * Cfg::kStageBytes);
     if (warp == 0) {
@@ -470,9 +399,6 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
     }
     consumer_bar();
     const QFragSmem qf{qsm, lane};
-#else
-    const QFragRegs<D>& qf = qa;
-#endif
     for (int i = 0; i < nchunks; ++i) {
       const int st = i % S;
       if (!pipe_wait(&ps.full[st], (i / S) & 1, &ps.abort_flag)) break;
@@ -484,8 +410,7 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
       __syncwarp();
       if (lane == 0) mbar_arrive(&ps.empty[st]);
     }
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    sum_l(l_run);
   }
 
   __syncthreads();  // every copy consumed; the stage ring is free
@@ -494,15 +419,20 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
   float* wm = reinterpret_cast<float*>(sgen);
   float* wl = wm + NW * G;
   float* wacc = wl + NW * G;
-  if (warp < NW && r < G) {
-    if (c == 0) {
-      wm[warp * G + r] = m_run;
-      wl[warp * G + r] = l_run;
-    }
+  if (warp < NW) {
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      wacc[(warp * G + r) * D + f8_dim<D>(j, 2 * c)] = o[j][0] * a.v_scale;
-      wacc[(warp * G + r) * D + f8_dim<D>(j, 2 * c + 1)] = o[j][1] * a.v_scale;
+    for (int j = 0; j < 2; ++j) {
+      const int h = 2 * c + j;
+      if (h >= G) continue;
+      if (r == 0) {
+        wm[warp * G + h] = m_run[j];
+        wl[warp * G + h] = l_run[j];
+      }
+#pragma unroll
+      for (int t = 0; t < D / 16; ++t) {
+        wacc[(warp * G + h) * D + f8_dim<D>(t, r)] = o[t][j] * a.v_scale;
+        wacc[(warp * G + h) * D + f8_dim<D>(t, r) + 1] = o[t][2 + j] * a.v_scale;
+      }
     }
   }
   __syncthreads();
