@@ -53,10 +53,10 @@ NCU_TRAFFIC: dict = {
         bytes=1_079_315_883 + 2_277_120, files=_DEC + ["decode_simt.cuh"], sha="9489fe02f3c535bb",
         note="decode_simt_kernel of pa_decode_append (the step's only launch), 3 launches"),
     ("llama2_7b_mha", "float8_e4m3fn", 0, "decode"): dict(
-        bytes=540_494_763 + 8_050_091, files=_DEC + ["decode_f8.cuh"], sha="e3c3f2af2d50fd9c",
+        bytes=540_498_517 + 1_985_109, files=_DEC + ["decode_f8.cuh"], sha="7a656a575bb54728",
         note="decode_f8_kernel (e4m3) of pa_decode_append, 3 launches"),
     ("llama2_7b_mha", "int8", 0, "decode"): dict(
-        bytes=540_492_373 + 8_290_987, files=_DEC + ["decode_f8.cuh"], sha="e3c3f2af2d50fd9c",
+        bytes=540_495_019 + 2_137_771, files=_DEC + ["decode_f8.cuh"], sha="7a656a575bb54728",
         note="decode_f8_kernel (int8) of pa_decode_append, 3 launches"),
     ("long_context_split", "bfloat16", 512, "decode"): dict(
         bytes=1_342_990_080 + 6_214_229 + 21_473_621, files=_DEC + ["decode_mma.cuh"], sha="915c9bdf9030f201",
@@ -73,10 +73,10 @@ NCU_TRAFFIC: dict = {
         note="decode_mma_kernel of pa_decode_append over steps 0-29 of the trace (32768-block pool); their "
              "algorithmic mean is 825.0 MB per step (x1.015), the 200-step mean 811.2 MB"),
     ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
-        bytes=1_309_527_296 + 230_245_449, files=_PF, sha="11b6569f1f58cdf6",
+        bytes=1_309_527_296 + 230_245_449, files=_PF, sha="48766827097f5b34",
         note="prefill_tc_kernel, 7 launches (Q, K/V per tile pair not served by L2, the fp32 output)"),
     ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
-        bytes=760_672_549 + 489_605_010, files=_PF, sha="11b6569f1f58cdf6", note="prefill_tc_kernel, 7 launches"),
+        bytes=760_672_549 + 489_605_010, files=_PF, sha="48766827097f5b34", note="prefill_tc_kernel, 7 launches"),
 }
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
