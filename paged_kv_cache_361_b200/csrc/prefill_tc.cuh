@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
   __shared__ uint64_t vfull[S], vempty[S];    // bf16: V of a stage (ps.full / ps.empty track its K)
   __shared__ uint64_t q_full, drain;
   __shared__ uint64_t s_full[TILES][2], p_full[TILES][2], o_bar[TILES];
+  __shared__ uint64_t o_last[TILES];  // one phase: tile t's last P V (and every MMA before it) complete
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       mbar_init(&p_full[t][0], 4);
       mbar_init(&p_full[t][1], 4);
       mbar_init(&o_bar[t], 1);
+      mbar_init(&o_last[t], 1);
     }
     if constexpr (F8) {
 #pragma unroll
@@ -383,6 +385,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
           tc::mma_ts(to, tp + ks * 8, bd, kIdPV, j > 0 || ks > 0);
         }
         tc::commit(smem_u32(&o_bar[t]));
+        if (j == nch[t] - 1) tc::commit(smem_u32(&o_last[t]));
         return true;
       };
       bool ok = warp_wait(&q_full, 0, &ps.abort_flag);
@@ -540,11 +543,10 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[t][sb]);
       }
-      // S(j+1) is issued before P(j) V(j), so this warpgroup can finish its
-      // last chunk while the previous P V is still pending: wait for the two
-      // last phases in turn (a parity wait cannot tell phases two apart).
-      if (ok && mych >= 2) ok = warp_wait(&o_bar[t], (mych - 2) & 1, &ps.abort_flag);
-      if (ok) ok = warp_wait(&o_bar[t], (mych - 1) & 1, &ps.abort_flag);
+      // O is final once the last P V has completed; its own single-phase
+      // barrier (o_bar may by then be two phases past the one a parity wait
+      // would name, if this warp is slow to get here after its last arrival)
+      if (ok) ok = warp_wait(&o_last[t], 0, &ps.abort_flag);
       if (ok) {
         tc::fence_after();
         const float inv = (F8 ? a.v_scale : 1.f) / l;
