@@ -73,10 +73,12 @@ NCU_TRAFFIC: dict = {
         note="decode_mma_kernel of pa_decode_append over steps 0-29 of the trace (32768-block pool); their "
              "algorithmic mean is 825.0 MB per step (x1.015), the 200-step mean 811.2 MB"),
     ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
-        bytes=1_309_527_296 + 230_245_449, files=_PF, sha="48766827097f5b34",
-        note="prefill_tc_kernel, 7 launches (Q, K/V per tile pair not served by L2, the fp32 output)"),
+        bytes=1_311_341_000 + 233_682_432, files=_PF, sha="6cd8591114f59451",
+        note="prefill_tc_kernel, 1 launch (Q, K/V per tile pair not served by L2, the fp32 output)"),
+    ("prefill_llama2_7b_mha", "float8_e4m3fn", 0, "prefill"): dict(
+        bytes=640_181_760 + 224_479_488, files=_PF, sha="6cd8591114f59451", note="prefill_tc_kernel (e4m3), 1 launch"),
     ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
-        bytes=760_672_549 + 489_605_010, files=_PF, sha="48766827097f5b34", note="prefill_tc_kernel, 7 launches"),
+        bytes=757_724_928 + 492_665_856, files=_PF, sha="6cd8591114f59451", note="prefill_tc_kernel, 1 launch"),
 }
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
