@@ -444,9 +444,13 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       {
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + orow * D);
         uint8_t* qdst = sgen + t * Cfg::kQTileBytes;
+        // every piece of the row in flight at once, then the shared-memory stores
+        uint4 qv[D / 8];
+#pragma unroll
+        for (int c16 = 0; c16 < D / 8; ++c16) qv[c16] = valid ? __ldg(src + c16) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int c16 = 0; c16 < D / 8; ++c16) {
-          uint4 v = valid ? __ldg(src + c16) : make_uint4(0u, 0u, 0u, 0u);
+          uint4 v = qv[c16];
           if constexpr (F8)
             v = make_uint4(pack_f16(bf16lo(v.x), bf16hi(v.x)), pack_f16(bf16lo(v.y), bf16hi(v.y)),
                            pack_f16(bf16lo(v.z), bf16hi(v.z)), pack_f16(bf16lo(v.w), bf16hi(v.w)));
@@ -550,19 +554,36 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       if (ok) {
         tc::fence_after();
         const float inv = (F8 ? a.v_scale : 1.f) / l;
-        float* dst = a.out + orow * D;
+        // O leaves through shared memory, 32 columns at a time, staged in the
+        // tile's Q area (free: every MMA of the tile has completed). Each
+        // thread writes its row's 128 bytes (16-byte pieces rotated by row: no
+        // bank conflicts), then the warp stores its 32 rows as whole 128-byte
+        // segments, eight lanes per row, four rows per instruction, instead of
+        // one 16-byte piece of 32 different rows per instruction.
+        uint8_t* stg = sgen + t * Cfg::kQTileBytes + (warp & 3) * 32 * 128;
+        const int pc = lane & 7;  // store phase: 16-byte piece of the row
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
           uint32_t o[32];
           __syncwarp();
           tc::ld32(trow + q * 32, o);
           tc::wait_ld();
-          if (valid) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(dst + q * 32 + e) =
-                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<float4*>(stg + lane * 128 + ((e ^ (lane & 7)) << 4)) =
+                make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                            __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rw = 4 * i + (lane >> 3);         // row within the warp's 32
+            const int rr = (warp & 3) * 32 + rw;        // row within the tile
+            const int32_t tk = tok0 + rr / G;
+            if (tk < n) {
+              const int64_t orr = (static_cast<int64_t>(q0) + tk) * a.hq + g * G + rr % G;
+              *reinterpret_cast<float4*>(a.out + orr * D + q * 32 + pc * 4) =
+                  *reinterpret_cast<const float4*>(stg + rw * 128 + ((pc ^ (rw & 7)) << 4));
+            }
           }
         }
       }
