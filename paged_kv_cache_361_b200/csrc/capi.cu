@@ -218,6 +218,38 @@ bool encode_rows_halves(CUtensorMap* map, void* base, uint64_t rows, int bs) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The prefill output [tokens][heads][head_dim] fp32 as a 3-D map for TMA
+// stores of [128 / G tokens x G heads x 32 columns] boxes (one query tile's O
+// in 32-column slices) with the 128-byte swizzle. `tokens` bounds the rows the
+// kernel stores (only tiles whose rows are all inside their sequence).
+bool encode_out_tiles(CUtensorMap* map, void* base, uint64_t tokens, int hq, int D, int G) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(hq), tokens};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(hq) * D * 4};
+  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The prefill queries [tokens][heads][head_dim] bf16 as a 3-D map for TMA
+// loads of [128 / G tokens x G heads x 64 dims] boxes (one 64-dim half of a
+// query tile) with the 128-byte swizzle. The kernel loads only tiles whose
+// rows are all inside their sequence, so every row it reads exists.
+bool encode_q_tiles(CUtensorMap* map, void* base, uint64_t tokens, int hq, int D, int G) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(hq), tokens};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(hq) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // An e4m3 pool viewed as rows of head_dim bytes, read in [bs x head_dim] boxes
 // with the 128-byte (head_dim 128) or 64-byte (head_dim 64) swizzle.
 bool encode_rows_u8(CUtensorMap* map, void* base, uint64_t rows, int D, int bs) {
@@ -557,17 +589,20 @@ pa_status pa_prefill(const void* q, int32_t num_seqs, const int32_t* cu_q_lens, 
   a.group_offs = a.group_members = a.group_prefix = nullptr;
   a.prefix_part_tokens = a.max_parts = a.parts_stride = 0;
   a.ws_ml = a.ws_o = nullptr;
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, to, tq;
   const uint64_t rows = static_cast<uint64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
   auto enc = f8 ? encode_rows_u8 : encode_rows;
   if (!enc(&tk, cache->k, rows, cache->head_dim, cache->block_size) ||
-      !enc(&tv, cache->v, rows, cache->head_dim, cache->block_size))
+      !enc(&tv, cache->v, rows, cache->head_dim, cache->block_size) ||
+      !encode_out_tiles(&to, out, static_cast<uint64_t>(num_seqs) * max_q_len, num_q_heads, cache->head_dim, G) ||
+      !encode_q_tiles(&tq, const_cast<void*>(q), static_cast<uint64_t>(num_seqs) * max_q_len, num_q_heads,
+                      cache->head_dim, G))
     return PA_ERR_CUDA;
   const dim3 grid(cache->num_kv_heads, num_seqs, static_cast<unsigned>(ntiles));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto launch = [&](auto kern, int threads, int smem) -> pa_status {
     if (!smem_attrs(reinterpret_cast<const void*>(kern), smem, false)) return PA_ERR_CUDA;
-    kern<<<grid, threads, smem, s>>>(tk, tv, a);
+    kern<<<grid, threads, smem, s>>>(tk, tv, to, tq, a);
     return launched();
   };
   auto launch8 = [&](auto cf) -> pa_status {

@@ -135,12 +135,25 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
+// TMA store of one box of a 3-D map from shared memory (coordinates x, y, z),
+// in this thread's bulk group; the group's reads of shared memory are awaited
+// with bulk_wait_read.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // TILES query tiles of one (kv head, sequence) per CTA share the K/V stream;
 // tile t is processed by softmax warpgroup t.
 // CF = 0: bf16 cache; kCodeE4M3 / kCodeS8: an 8-bit cache of that format.
 template <int D, int G, int TILES, int CF = 0>
 __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                      const __grid_constant__ CUtensorMap tmo, const __grid_constant__ CUtensorMap tmq,
                       const PrefillArgs a) {
   constexpr bool F8 = CF != 0;
   using Cfg = TcCfg<D, TILES, F8>;
@@ -155,6 +168,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
   __shared__ uint64_t q_full, drain;
   __shared__ uint64_t s_full[TILES][2], p_full[TILES][2], o_bar[TILES];
   __shared__ uint64_t o_last[TILES];  // one phase: tile t's last P V (and every MMA before it) complete
+  __shared__ uint64_t o_staged;       // the last tile's O is in shared memory (one arrival per warp)
   __shared__ uint32_t tmem_base_sh;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -196,10 +210,21 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
   }
   const int nchunks = nch[ntiles_act - 1];
   const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
+  // Q of a tile whose rows all lie inside the sequence arrives by TMA (bf16:
+  // the rows as they are); otherwise the softmax warps load it row by row
+  // (zeros past the sequence; f16 over an 8-bit cache)
+  auto q_by_tma = [&](int t) { return !F8 && t < ntiles_act && tok00 + (t + 1) * TT <= n; };
+  int q_arrivals = 0, q_tma_tiles = 0;
+#pragma unroll
+  for (int t = 0; t < TILES; ++t) {
+    if (q_by_tma(t)) ++q_tma_tiles;
+    else if (t < ntiles_act) q_arrivals += 4;
+  }
 
   if (tid == 0) {
-    mbar_init(&q_full, 4 * ntiles_act);
+    mbar_init(&q_full, q_arrivals + (q_tma_tiles > 0 ? 1 : 0));
     mbar_init(&drain, 1);
+    mbar_init(&o_staged, 4);
 #pragma unroll
     for (int t = 0; t < TILES; ++t) {
       mbar_init(&s_full[t][0], 1);
@@ -230,6 +255,19 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         mbar_init(&vempty[i], 1);
       }
       pipe_init<S>(ps, 1);  // empty stages are released by one tcgen05.commit
+    }
+    if (q_tma_tiles > 0) {
+      // [128 / G tokens x G heads x 64 dims] boxes, one per 64-dim half of a tile
+      mbar_arrive_expect_tx(&q_full, static_cast<uint32_t>(q_tma_tiles * Cfg::kQTileBytes));
+      const uint64_t pol = l2_evict_first_policy();
+#pragma unroll
+      for (int t = 0; t < TILES; ++t)
+        if (q_by_tma(t)) {
+#pragma unroll
+          for (int hf = 0; hf < Cfg::kHalves; ++hf)
+            tma_load_3d(sbase + t * Cfg::kQTileBytes + hf * Cfg::kQHalfBytes, &tmq, hf * 64, g * G,
+                        q0 + tok00 + t * TT, &q_full, pol);
+        }
     }
   }
   if (warp == Cfg::kMmaWarp) {
@@ -441,7 +479,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       const int32_t pos = base + (valid ? tok : tok_end - 1);  // last key the row sees
       const int h = r % G;
       const int64_t orow = (static_cast<int64_t>(q0) + (valid ? tok : 0)) * a.hq + g * G + h;
-      {
+      if (!q_by_tma(t)) {
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + orow * D);
         uint8_t* qdst = sgen + t * Cfg::kQTileBytes;
         // every piece of the row in flight at once, then the shared-memory stores
@@ -554,6 +592,40 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
       if (ok) {
         tc::fence_after();
         const float inv = (F8 ? a.v_scale : 1.f) / l;
+        if (t == ntiles_act - 1 && tok0 + TT <= n) {
+          // The last tile, all rows valid: its last P V was the CTA's last MMA,
+          // so the K/V stages are free. O goes there as D / 32 boxes of
+          // [128 rows x 32 columns] fp32 in the TMA's 128-byte swizzle, and one
+          // thread stores them with the TMA (rows = (token, head) of the
+          // output's [tokens][heads][D] layout); the CTA waits only for the
+          // copies' reads of shared memory.
+          uint8_t* stg = sgen + Cfg::kQBytes;
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            __syncwarp();
+            tc::ld32(trow + q * 32, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              *reinterpret_cast<float4*>(stg + q * (128 * 128) + r * 128 + ((e ^ (r & 7)) << 4)) =
+                  make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                              __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+          }
+          tc::fence_proxy_async();  // generic-proxy writes -> the TMA's reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_staged);
+          if ((warp & 3) == 0) {
+            if (warp_wait(&o_staged, 0, &ps.abort_flag) && lane == 0) {
+#pragma unroll
+              for (int q = 0; q < D / 32; ++q)
+                tma_store_3d(&tmo, smem_u32(stg) + q * (128 * 128), q * 32, g * G, q0 + tok0);
+              bulk_commit();
+              bulk_wait_read();
+            }
+            __syncwarp();
+          }
+        } else {
         // O leaves through shared memory, 32 columns at a time, staged in the
         // tile's Q area (free: every MMA of the tile has completed). Each
         // thread writes its row's 128 bytes (16-byte pieces rotated by row: no
@@ -585,6 +657,7 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
                   *reinterpret_cast<const float4*>(stg + rw * 128 + ((pc ^ (rw & 7)) << 4));
             }
           }
+        }
         }
       }
       tc::fence_before();
