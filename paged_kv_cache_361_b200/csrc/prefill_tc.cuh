@@ -144,6 +144,10 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sr
                "r"(src), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
+// Fetch a tensor map's descriptor ahead of its first copy.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
@@ -182,6 +186,12 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
   const int g = blockIdx.x, s = blockIdx.y;
   const int pair = a.ntiles - 1 - static_cast<int>(blockIdx.z);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+    prefetch_tmap(&tmq);
+    prefetch_tmap(&tmo);
+  }
 
   const int32_t q0 = __ldg(a.cu_q + s);
   int32_t n = __ldg(a.cu_q + s + 1) - q0;
@@ -270,6 +280,11 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
         }
     }
   }
+  // the producers' first block-table window is read while the CTA sets up
+  // (its ids feed the first K/V copies: one memory round trip less at the start)
+  TableAhead ta;
+  if (warp == Cfg::kProducerWarp || (!F8 && warp == Cfg::kVProducerWarp))
+    ta.init(a.tables + table_row, 0, min(a.max_blocks, (kend_all + a.bs - 1) / a.bs), lane);
   if (warp == Cfg::kMmaWarp) {
     tc::alloc(smem_u32(&tmem_base_sh), Cfg::kTmemCols);
     tc::relinquish();
@@ -283,8 +298,6 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
     // ---- producer (F8): codes of chunk i into staging slot i % CS ----
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
     const uint64_t pol = l2_evict_last_policy();
-    TableAhead ta;
-    ta.init(a.tables + table_row, 0, min(a.max_blocks, (kend_all + a.bs - 1) / a.bs), lane);
     int i = 0;
     for (; i < nchunks; ++i) {
       const int cst = i % CS;
@@ -356,8 +369,6 @@ __global__ void __launch_bounds__(TcCfg<D, TILES, CF != 0>::kThreads, 1)
     const uint32_t tile_off = is_v ? Cfg::kTileBytes : 0u;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * 128u;
     const uint64_t pol = l2_evict_last_policy();  // later tiles of this sequence read the same keys
-    TableAhead ta;
-    ta.init(a.tables + table_row, 0, min(a.max_blocks, (kend_all + a.bs - 1) / a.bs), lane);
     int i = 0;
     for (; i < nchunks; ++i) {
       const int st = i % S;
