@@ -73,12 +73,12 @@ NCU_TRAFFIC: dict = {
         note="decode_mma_kernel of pa_decode_append over steps 0-29 of the trace (32768-block pool); their "
              "algorithmic mean is 825.0 MB per step (x1.015), the 200-step mean 811.2 MB"),
     ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
-        bytes=1_311_341_000 + 233_682_432, files=_PF, sha="6cd8591114f59451",
-        note="prefill_tc_kernel, 1 launch (Q, K/V per tile pair not served by L2, the fp32 output)"),
+        bytes=1_311_638_000 + 228_689_664, files=_PF, sha="b97a7e2608d45579",
+        how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch (Q, K/V per tile pair not served by L2, the fp32 output)"),
     ("prefill_llama2_7b_mha", "float8_e4m3fn", 0, "prefill"): dict(
-        bytes=640_181_760 + 224_479_488, files=_PF, sha="6cd8591114f59451", note="prefill_tc_kernel (e4m3), 1 launch"),
+        bytes=661_085_952 + 226_466_816, files=_PF, sha="b97a7e2608d45579", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel (e4m3), 1 launch"),
     ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
-        bytes=757_724_928 + 492_665_856, files=_PF, sha="6cd8591114f59451", note="prefill_tc_kernel, 1 launch"),
+        bytes=749_158_656 + 483_207_424, files=_PF, sha="b97a7e2608d45579", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch"),
 }
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
