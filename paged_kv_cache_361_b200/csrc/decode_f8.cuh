@@ -332,7 +332,23 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
   const int nchunks = (pt.ntok + C - 1) / C;
   const int hq0 = g * G;
 
-  if (tid == 0) pipe_init<S>(ps, NW);
+  // the producer's global reads (its first block-table window; with the fused
+  // KV append the new row, stored before the last chunk's copies, which read
+  // it) go out before the CTA-wide barrier
+  using Code = typename std::conditional<CF == kCodeS8, int8_t, __nv_fp8_e4m3>::type;
+  const bool do_append = a.slot_mapping && pt.last;
+  AppendRow<Code, D> ar;
+  TableAhead ta;
+  if (warp == NW) {
+    if (do_append) ar.load(a, s, g, lane);
+    ta.init(a.tables + static_cast<int64_t>(s) * a.max_blocks, pt.t0 / a.bs,
+            min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
+  }
+  if (tid == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+    pipe_init<S>(ps, NW);
+  }
   __syncthreads();
 
   float o[D / 16][4];
@@ -341,17 +357,8 @@ __global__ void PA_F8_LAUNCH_BOUNDS(F8Cfg<D>::kThreads) decode_f8_kernel(const _
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
   if (warp == NW) {
-    // fused KV append: the new row is loaded now and stored before the last
-    // chunk's copies, which read it
-    using Code = typename std::conditional<CF == kCodeS8, int8_t, __nv_fp8_e4m3>::type;
-    const bool do_append = a.slot_mapping && pt.last;
-    AppendRow<Code, D> ar;
-    if (do_append) ar.load(a, s, g, lane);
-    const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D;
     const uint64_t pol = kv_stream_policy();
-    TableAhead ta;
-    ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       if (do_append) ar.before_chunk(a, i, nchunks, lane);
       const int32_t c0 = pt.t0 + i * C;

@@ -50,6 +50,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Fetch a tensor map's descriptor ahead of its first copy.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 // The same for a 3-D map: coordinates (x, y, z).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
                                             uint64_t* bar, uint64_t policy) {
@@ -611,7 +616,22 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
   const int nchunks = (pt.ntok + C - 1) / C;
   const int hq0 = g * G;
 
-  if (tid == 0) pipe_init<S>(ps, NW);
+  // the producer's global reads (its first block-table window; with the fused
+  // KV append the new row, stored before the last chunk's copies, which read
+  // it) go out before the CTA-wide barrier
+  const bool do_append = a.slot_mapping && pt.last;
+  AppendRow<__nv_bfloat16, D> ar;
+  TableAhead ta;
+  if (warp == NW) {
+    if (do_append) ar.load(a, s, g, lane);
+    ta.init(a.tables + static_cast<int64_t>(s) * a.max_blocks, pt.t0 / a.bs,
+            min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
+  }
+  if (tid == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+    pipe_init<S>(ps, NW);
+  }
   __syncthreads();
 
   float o[D / 16][4];
@@ -620,16 +640,8 @@ __global__ void PA_MMA_LAUNCH_BOUNDS(MmaCfg<D>::kThreads) decode_mma_kernel(cons
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
   if (warp == NW) {
-    // fused KV append: the new row is loaded now and stored before the last
-    // chunk's copies, which read it
-    const bool do_append = a.slot_mapping && pt.last;
-    AppendRow<__nv_bfloat16, D> ar;
-    if (do_append) ar.load(a, s, g, lane);
-    const int64_t table_row = static_cast<int64_t>(s) * a.max_blocks;
     const uint32_t box_bytes = static_cast<uint32_t>(a.bs) * D * 2u;  // one (block, head) tile of K or V
     const uint64_t pol = kv_stream_policy();
-    TableAhead ta;
-    ta.init(a.tables + table_row, pt.t0 / a.bs, min(a.max_blocks, (pt.t1 + a.bs - 1) / a.bs), lane);
     pipe_produce<S>(ps, nchunks, [&](int i, int st) {
       if (do_append) ar.before_chunk(a, i, nchunks, lane);
       const int32_t c0 = pt.t0 + i * C;
