@@ -50,35 +50,35 @@ _PF = ["common.cuh", "decode_common.cuh", "decode_f8.cuh", "prefill_mma.cuh", "p
        "capi.cu"]
 NCU_TRAFFIC: dict = {
     ("llama2_7b_mha", "bfloat16", 0, "decode"): dict(
-        bytes=1_079_315_883 + 2_277_120, files=_DEC + ["decode_simt.cuh"], sha="9489fe02f3c535bb",
+        bytes=1_079_387_221 + 2_192_299, files=_DEC + ["decode_simt.cuh"], sha="8e318919c2abc840",
         note="decode_simt_kernel of pa_decode_append (the step's only launch), 3 launches"),
     ("llama2_7b_mha", "float8_e4m3fn", 0, "decode"): dict(
-        bytes=540_498_517 + 1_985_109, files=_DEC + ["decode_f8.cuh"], sha="7a656a575bb54728",
+        bytes=540_502_443 + 1_836_459, files=_DEC + ["decode_f8.cuh"], sha="5ff75b7b610d5d43",
         note="decode_f8_kernel (e4m3) of pa_decode_append, 3 launches"),
     ("llama2_7b_mha", "int8", 0, "decode"): dict(
-        bytes=540_495_019 + 2_137_771, files=_DEC + ["decode_f8.cuh"], sha="7a656a575bb54728",
+        bytes=540_523_947 + 1_852_928, files=_DEC + ["decode_f8.cuh"], sha="5ff75b7b610d5d43",
         note="decode_f8_kernel (int8) of pa_decode_append, 3 launches"),
     ("long_context_split", "bfloat16", 512, "decode"): dict(
-        bytes=1_342_990_080 + 6_214_229 + 21_473_621, files=_DEC + ["decode_mma.cuh"], sha="915c9bdf9030f201",
+        bytes=1_343_030_613 + 6_136_832 + 21_471_744, files=_DEC + ["decode_mma.cuh"], sha="572fd0d77d91b599",
         note="decode_mma_persistent_kernel + decode_reduce_kernel, 3 launches each"),
     ("parallel_sampling", "bfloat16", 0, "decode"): dict(
-        bytes=113_246_549 + 388_437, files=_DEC + ["decode_mma.cuh"], sha="915c9bdf9030f201",
+        bytes=113_622_400 + 601_728, files=_DEC + ["decode_mma.cuh"], sha="572fd0d77d91b599",
         note="decode_mma_kernel of pa_decode_append, 6 launches (1.17x the 97.5 MB of distinct blocks: with the "
              "longest-first order a prompt's samples no longer all run at once)"),
     ("parallel_sampling", "bfloat16", 0, "cascade"): dict(
-        bytes=32_022_485 + 1_323 + 72_883_917 + 106_394, files=_DEC + ["decode_mma.cuh", "prefill_mma.cuh"], sha="96f8c67c8ea950e0",
+        bytes=32_022_272 + 768 + 72_888_013 + 103_168, files=_DEC + ["decode_mma.cuh", "prefill_mma.cuh"], sha="de27b89ffdac9c43",
         note="prefill_mma_kernel (prefix pass) + decode_mma_kernel (suffixes and fold), 5-6 launches each"),
     ("continuous_batching", "bfloat16", 0, "decode"): dict(
-        bytes=835_070_020 + 2_660_804, files=_DEC + ["decode_mma.cuh"], sha="915c9bdf9030f201",
+        bytes=835_087_625 + 2_439_945, files=_DEC + ["decode_mma.cuh"], sha="572fd0d77d91b599",
         note="decode_mma_kernel of pa_decode_append over steps 0-29 of the trace (32768-block pool); their "
              "algorithmic mean is 825.0 MB per step (x1.015), the 200-step mean 811.2 MB"),
     ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
-        bytes=1_311_638_000 + 228_689_664, files=_PF, sha="b97a7e2608d45579",
+        bytes=1_308_493_000 + 228_926_976, files=_PF, sha="e0aea23930d12b9d",
         how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch (Q, K/V per tile pair not served by L2, the fp32 output)"),
     ("prefill_llama2_7b_mha", "float8_e4m3fn", 0, "prefill"): dict(
-        bytes=661_085_952 + 226_466_816, files=_PF, sha="b97a7e2608d45579", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel (e4m3), 1 launch"),
+        bytes=660_428_288 + 226_866_688, files=_PF, sha="e0aea23930d12b9d", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel (e4m3), 1 launch"),
     ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
-        bytes=749_158_656 + 483_207_424, files=_PF, sha="b97a7e2608d45579", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch"),
+        bytes=742_350_848 + 484_450_816, files=_PF, sha="e0aea23930d12b9d", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch"),
 }
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
