@@ -26,11 +26,14 @@
 //              S_{j+1} is issued before O += P_j V_j so the tensor core works
 //              while the softmax warps handle chunk j. Completions reach the
 //              other warps through tcgen05.commit on mbarriers.
-//   warps 0-3  one thread per row (TMEM lane): load the row's Q into shared
-//              memory; per chunk read S from TMEM, mask causally, keep the
-//              running maximum m and sum l in base 2, write P back into the
-//              S buffer as f16 (11 significant bits; weights are at most
-//              2^8); at the end read O, divide by l, store fp32.
+//   warps 0-3  one thread per row (TMEM lane): per chunk read S from TMEM,
+//              mask causally, keep the running maximum m and sum l in base
+//              2, write P back into the S buffer as f16 (11 significant
+//              bits; weights are at most 2^8); at the end read O, divide by
+//              l and store it fp32 through shared memory (the CTA's last
+//              tile by TMA stores from the freed K/V stages). Q of a tile
+//              whose rows all lie in the sequence arrives by TMA (bf16
+//              cache); otherwise these threads load it row by row.
 //   warps +2..+5  converter: a kind::f16 MMA takes A and B of one type, so
 //              with P in f16 the V operand must be f16 too. The converter
 //              rewrites each stage's V tile in place, bf16 -> f16 (exact for
