@@ -73,12 +73,12 @@ NCU_TRAFFIC: dict = {
         note="decode_mma_kernel of pa_decode_append over steps 0-29 of the trace (32768-block pool); their "
              "algorithmic mean is 825.0 MB per step (x1.015), the 200-step mean 811.2 MB"),
     ("prefill_llama2_7b_mha", "bfloat16", 0, "prefill"): dict(
-        bytes=1_308_493_000 + 228_926_976, files=_PF, sha="e0aea23930d12b9d",
+        bytes=1_308_881_000 + 228_545_280, files=_PF, sha="de28dba00f317626",
         how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch (Q, K/V per tile pair not served by L2, the fp32 output)"),
     ("prefill_llama2_7b_mha", "float8_e4m3fn", 0, "prefill"): dict(
-        bytes=660_428_288 + 226_866_688, files=_PF, sha="e0aea23930d12b9d", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel (e4m3), 1 launch"),
+        bytes=662_598_656 + 226_810_368, files=_PF, sha="de28dba00f317626", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel (e4m3), 1 launch"),
     ("prefill_gqa8", "bfloat16", 0, "prefill"): dict(
-        bytes=742_350_848 + 484_450_816, files=_PF, sha="e0aea23930d12b9d", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch"),
+        bytes=758_603_264 + 483_280_640, files=_PF, sha="de28dba00f317626", how="ncu capture (the profile's metric set, one launch)", note="prefill_tc_kernel, 1 launch"),
 }
 CSRC = os.path.join(ROOT, "paged_kv_cache_361_b200", "csrc")
 
