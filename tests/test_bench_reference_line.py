@@ -23,3 +23,22 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert "workload" in d["config"]
+
+
+def test_traffic_table_entries_are_well_formed():
+    """Every DRAM-traffic entry names existing library sources, a hash of them,
+    a positive byte count and a note; a stale entry (sources changed since the
+    capture) is reported as null with its reason, never as a number."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for key, e in bench.NCU_TRAFFIC.items():
+        assert len(key) == 4 and key[3] in ("decode", "cascade", "prefill"), key
+        assert e["bytes"] > 0 and e["note"], key
+        for f in e["files"]:
+            assert os.path.exists(os.path.join(bench.CSRC, f)), (key, f)
+        value, why = bench.ncu_traffic(key)
+        if bench.src_hash(e["files"]) == e["sha"]:
+            assert value == e["bytes"], key
+        else:
+            assert value is None and why.startswith("stale"), key
+    assert bench.ncu_traffic(("no such workload", "bfloat16", 0, "decode")) == (None, "no capture of this configuration")
