@@ -35,6 +35,9 @@ namespace {
 struct Seq {
   std::vector<int32_t> table;
   int64_t len = 0;
+  // dry run of a batched append (valid while batch == the manager's batch number)
+  uint64_t batch = 0;
+  int64_t shadow_len = 0, shadow_bi = -1;
 };
 
 // Prefix-cache key of a prompt block: a 64-bit hash chained over every token
@@ -144,37 +147,49 @@ class BlockManager {
     // After an append at length L the block at logical index L / bs is private
     // to the sequence (fresh, copied, or already held once), and counts only
     // fall during a batch, so a later append into the same index copies nothing.
-    struct Shadow {
-      int64_t len;
-      int64_t private_bi;
-    };
-    std::unordered_map<int64_t, Shadow> sh;
-    std::unordered_map<int32_t, int32_t> dref;
+    // The shadow state lives in the sequences (tagged with this batch's
+    // number) and the count changes in a per-block array reset afterwards:
+    // no allocation per call once the scratch vectors have grown.
+    ++batch_no_;
+    batch_.resize(static_cast<size_t>(n));
+    if (static_cast<int64_t>(dref_.size()) != nb_) dref_.assign(static_cast<size_t>(nb_), 0);
+    dref_touched_.clear();
     int64_t need = 0;
+    pa_status err = PA_OK;
     for (int32_t i = 0; i < n; ++i) {
       auto it = seqs_.find(ids[i]);
-      if (it == seqs_.end()) return PA_ERR_UNKNOWN_SEQ;
-      const Seq& s = it->second;
-      auto ins = sh.emplace(ids[i], Shadow{s.len, -1});
-      Shadow& st = ins.first->second;
-      int64_t bi = st.len / bs_;
-      if (st.len % bs_ == 0) {
+      if (it == seqs_.end()) {
+        err = PA_ERR_UNKNOWN_SEQ;
+        break;
+      }
+      Seq& s = it->second;
+      batch_[i] = &s;
+      if (s.batch != batch_no_) {
+        s.batch = batch_no_;
+        s.shadow_len = s.len;
+        s.shadow_bi = -1;
+      }
+      const int64_t bi = s.shadow_len / bs_;
+      if (s.shadow_len % bs_ == 0) {
         ++need;
-      } else if (bi != st.private_bi) {
-        int32_t b = s.table[bi];
-        if (ref_[b] + dref[b] > 1) {
+      } else if (bi != s.shadow_bi) {
+        const int32_t b = s.table[bi];
+        if (ref_[b] + dref_[b] > 1) {
           ++need;
-          dref[b] -= 1;
+          if (dref_[b] == 0) dref_touched_.push_back(b);
+          dref_[b] -= 1;
         }
       }
-      st.private_bi = bi;
-      st.len += 1;
+      s.shadow_bi = bi;
+      s.shadow_len += 1;
     }
+    for (int32_t b : dref_touched_) dref_[b] = 0;
+    if (err != PA_OK) return err;
     if (need > available()) return PA_ERR_NO_FREE_BLOCKS;
     int32_t np = 0;
     for (int32_t i = 0; i < n; ++i) {
       int32_t pr[2];
-      do_append(seqs_.find(ids[i])->second, &slots[i], pr);
+      do_append(*batch_[i], &slots[i], pr);
       if (pr[0] >= 0) {
         if (pairs) {
           pairs[2 * np] = pr[0];
@@ -452,6 +467,10 @@ class BlockManager {
   int64_t head_ = 0, count_ = 0;
   std::vector<int32_t> ref_;
   std::unordered_map<int64_t, Seq> seqs_;
+  // batched-append scratch (see append_many)
+  uint64_t batch_no_ = 0;
+  std::vector<Seq*> batch_;
+  std::vector<int32_t> dref_, dref_touched_;
   // prefix cache
   std::unordered_map<uint64_t, CacheEntry> cache_;
   std::vector<uint64_t> key_of_;
@@ -560,13 +579,18 @@ pa_status pa_bm_block_table(const pa_bm* bm, int64_t seq_id, int32_t* out, int32
 pa_status pa_bm_block_tables(const pa_bm* bm, int32_t n, const int64_t* seq_ids, int32_t* out, int32_t cap,
                              int32_t pad, int32_t* lens_out) {
   if (!bm || n < 0 || cap < 0 || (n > 0 && (!seq_ids || !out || !lens_out))) return PA_ERR_INVALID_ARG;
+  // every id is checked before any row is written; the lookups of a batch of
+  // up to kKeep sequences are kept for the copy pass
+  constexpr int32_t kKeep = 512;
+  const Seq* kept[kKeep];
   for (int32_t i = 0; i < n; ++i) {
     const Seq* s = bm->m.find(seq_ids[i]);
     if (!s) return PA_ERR_UNKNOWN_SEQ;
     if (static_cast<int64_t>(s->table.size()) > cap || s->len > INT32_MAX) return PA_ERR_INVALID_ARG;
+    if (i < kKeep) kept[i] = s;
   }
   for (int32_t i = 0; i < n; ++i) {
-    const Seq* s = bm->m.find(seq_ids[i]);
+    const Seq* s = i < kKeep ? kept[i] : bm->m.find(seq_ids[i]);
     int32_t* row = out + static_cast<int64_t>(i) * cap;
     int32_t m = static_cast<int32_t>(s->table.size());
     if (m) std::memcpy(row, s->table.data(), sizeof(int32_t) * m);
