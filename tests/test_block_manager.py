@@ -237,3 +237,73 @@ def test_prefix_cache_random_stress_with_eviction():
                 cpp.free_seq(op[1])
             assert cpp.free_list().tolist() == list(ref.free)
             assert cpp.prefix_stats() == ref.prefix_stats()
+
+
+def test_batched_append_stress_one_manager():
+    """Many batched appends on one manager (its batch scratch reused across
+    calls): random batches with repeated ids over forked sequences, frees and
+    adds in between, and batches that must fail whole (too few free blocks, an
+    unknown id); after every call slots, pairs, tables and the free list equal
+    the oracle's sequential appends, and a failed batch changes nothing."""
+    import copy
+    from oracle.block_manager import NoFreeBlocks, UnknownSeq
+    rng = np.random.default_rng(11)
+    nb, bs = 48, 4
+    order = rng.permutation(nb)
+    a = B.BlockManager(nb, bs, order)
+    m = BlockManagerModel(nb, bs, order)
+    next_id = 0
+    live = []
+    for rnd in range(400):
+        op = rng.random()
+        if (op < 0.15 or not live) and len(live) < 10:
+            n = int(rng.integers(0, 3 * bs))
+            try:
+                m2 = copy.deepcopy(m)
+                m2.add_seq(next_id, n)
+            except NoFreeBlocks:
+                with pytest.raises(B.PagedAttnError):
+                    a.add_seq(next_id, n)
+                continue
+            a.add_seq(next_id, n)
+            m = m2
+            live.append(next_id)
+            next_id += 1
+        elif op < 0.25 and len(live) < 10:
+            parent = int(rng.choice(live))
+            a.fork(parent, next_id)
+            m.fork(parent, next_id)
+            live.append(next_id)
+            next_id += 1
+        elif op < 0.35 and len(live) > 1:
+            s = int(live.pop(int(rng.integers(len(live)))))
+            a.free_seq(s)
+            m.free_seq(s)
+        else:
+            ids = [int(x) for x in rng.choice(live, size=int(rng.integers(1, 9)))]
+            if rng.random() < 0.05:
+                ids.insert(int(rng.integers(len(ids) + 1)), 10 ** 6)   # unknown id: the batch fails whole
+            m2 = copy.deepcopy(m)
+            rs, rp, err = [], [], None
+            try:
+                for s in ids:
+                    sl, cow = m2.append_slot(s)
+                    rs.append(sl)
+                    if cow:
+                        rp.append(list(cow))
+            except (NoFreeBlocks, UnknownSeq) as e:
+                err = e
+            before = (a.free_list().tolist(), [a.block_table(s)[0].tolist() for s in live])
+            if err is not None:
+                with pytest.raises(B.PagedAttnError) as e:
+                    a.append_slots(ids)
+                # every id is looked up before the blocks are counted: an unknown id wins
+                assert e.value.status == (B.PA_ERR_UNKNOWN_SEQ if 10 ** 6 in ids else B.PA_ERR_NO_FREE_BLOCKS)
+                assert before == (a.free_list().tolist(), [a.block_table(s)[0].tolist() for s in live])
+                continue
+            slots, pairs = a.append_slots(ids)
+            m = m2
+            assert slots.tolist() == rs and pairs.tolist() == rp, rnd
+        assert a.free_list().tolist() == list(m.free), rnd
+        for s in live:
+            assert a.block_table(s)[0].tolist() == m.block_table(s), (rnd, s)
