@@ -4,9 +4,10 @@
 Workload: 64 sequences, context lengths uniform in [128, 2048] before the step
 (one token appended, then decode), 32 query heads = 32 kv heads, head_dim 128,
 block_size 16, bf16 cache, pool = 1.1 x blocks needed with ids in a seeded
-shuffle, Q/K/V ~ N(0, 1). One step = the whole hot path for one batch: KV
-append (pa_reshape_and_cache) + decode attention (pa_decode, split into
-partitions with its log-sum-exp merge when the library chooses to).
+shuffle, Q/K/V ~ N(0, 1). One step = the whole hot path for one batch: the
+KV append and decode attention in one launch (pa_decode_append: the decode
+CTAs write the step's new K/V rows at their slots), split into partitions with
+its log-sum-exp merge when the library chooses to.
 
 Metric: KV bytes read by decode per second (GB/s, fraction of HBM peak), and
 decode tokens per second. The 1.07 GB of K/V read per step is far larger than
