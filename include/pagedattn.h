@@ -255,12 +255,17 @@ pa_status pa_decode_append(const void* q, const void* k_new, const void* v_new, 
  *                  all sequences back to back (T = cu_q_lens[num_seqs]).
  *   cu_q_lens      device int32 [num_seqs + 1]: sequence s owns rows
  *                  cu_q_lens[s] .. cu_q_lens[s+1]-1; n_s = their count.
- *   max_q_len      host bound on every n_s; it sizes the launch.
+ *   max_q_len      host bound on every n_s; it sizes the launch, and
+ *                  num_seqs * max_q_len bounds the rows the kernel's
+ *                  tensor-memory copies of q and out may address (only rows of
+ *                  query tiles lying wholly inside their sequence are copied
+ *                  that way, so every row they touch exists).
  *   context_lens   device int32 [num_seqs]: length L_s including the new
  *                  tokens; new token i of s sits at position L_s - n_s + i and
  *                  sees positions 0 .. L_s - n_s + i. n_s > L_s or L_s above
  *                  max_context_len is clamped and recorded (PA_ERR_DEVICE_BOUNDS).
  *   out            device fp32 [T][num_q_heads][head_dim].
+ * q and out must be 16-byte aligned (PA_ERR_INVALID_ARG otherwise).
  * Supported: bf16, e4m3 or int8 cache, block_size >= 8 (16, 32 as for decode),
  * head_dim 64 or 128, num_q_heads / num_kv_heads in {1, 2, 4, 8}; fp32 caches
  * return PA_ERR_UNSUPPORTED. Accumulation is fp32 on the tensor cores. The
